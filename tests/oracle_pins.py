@@ -1,0 +1,300 @@
+"""Pins for the CPU oracle: checks that tie it to something other than itself.
+
+Each ``check_*`` takes an ``oracle.Oracle`` and raises AssertionError on a mismatch.  The test
+module runs them on the real oracle (all must pass); the mutation test runs them on copies of
+the oracle with one plausible mistake planted (each copy must fail at least one).
+
+What pins what (definitions from "MISA: Mixture of Indexer Sparse Attention for Long-Context
+LLM Inference", gist.science/paper/2605.07363, "Methodology: MISA" and "Hierarchical Variant"):
+  * hand-computed fixture (tests/golden/hand_example.json): block means, router scores, routed
+    heads, token scores, top-k with exact ties, dense scores, MISA-dagger;
+  * special cases that reduce to numpy routines: B = 1 pools to the keys themselves, B >= n
+    pools to ``numpy.mean``; top-k equals a stable ``numpy.argsort``;
+  * brute force on tiny integer inputs: the routed set by enumerating every h-subset;
+  * exact invariants: scaling q, k or w by 2 scales every score by 2 and keeps every selection;
+    relabelling heads permutes the router scores; h = H_I is the dense indexer bit for bit;
+    k' >= n makes MISA-dagger the dense indexer, k' = k makes it MISA, and the dense top-k
+    restricted to the candidates is always kept; keys past a query's prefix change nothing;
+  * a planted needle (the tiny fp32 workload) is routed and selected.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+from long_context_sparse_mean_b200 import workloads as wlmod
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "hand_example.json")
+
+
+def _load_golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+def check_hand_example(o):
+    g = _load_golden()
+    k = np.array(g["keys"], np.float32)
+    q = np.array(g["q"], np.float32)
+    w = np.array(g["w"], np.float32)
+    B = g["B"]
+    for qc in g["queries"]:
+        n = qc["n"]
+        assert np.array_equal(o.pool_keys(k, B, n), np.array(qc["kbar"], np.float64)), "block means"
+        r, heads = o.route(q, w, k, n, B, 1)
+        assert np.array_equal(r, np.array(qc["r"], np.float64)), f"router scores n={n}: {r}"
+        assert list(heads) == qc["h1"]["heads"], f"routed head n={n}: {heads}"
+        I = o.token_scores(q, w, heads, k, n)
+        assert np.array_equal(I, np.array(qc["h1"]["I"], np.float64)), f"token scores h=1 n={n}: {I}"
+        top, _ = o.topk(I, 2)
+        assert list(top) == qc["h1"]["top2"], f"top-2 h=1 n={n}: {top}"
+        if "h2" in qc:
+            _, heads2 = o.route(q, w, k, n, B, 2)
+            assert list(heads2) == qc["h2"]["heads"], heads2
+            I2 = o.token_scores(q, w, heads2, k, n)
+            assert np.array_equal(I2, np.array(qc["h2"]["I"], np.float64)), I2
+            assert list(o.topk(I2, 2)[0]) == qc["h2"]["top2"]
+            assert list(o.topk(I2, 4)[0]) == qc["h2"]["top4"]
+            F = o.token_scores(q, w, np.arange(3), k, n)
+            assert np.array_equal(F, np.array(qc["dense"]["F"], np.float64)), F
+            for kk, key in ((2, "top2"), (4, "top4")):
+                dsa = o.indexer(2, q[None], w[None], k, 0, np.array([n]), B, 3, kk)
+                assert list(dsa["idx"][0]) == qc["dense"][key], dsa["idx"]
+            dag = o.indexer(1, q[None], w[None], k, 0, np.array([n]), B, 1, 2, kp=3)
+            assert list(dag["cand"][0]) == qc["dagger_h1_kp3"]["cand"], dag["cand"]
+            assert sorted(dag["idx"][0]) == sorted(qc["dagger_h1_kp3"]["top2"]), dag["idx"]
+
+
+def check_topk_vs_stable_argsort(o):
+    rng = np.random.default_rng(7)
+    for n, k in ((1, 1), (10, 3), (257, 64), (1000, 999), (50, 80)):
+        v = rng.integers(-5, 6, size=n).astype(np.float64)  # many exact ties
+        ids, vals = o.topk(v, k)
+        ref = np.argsort(-v, kind="stable")[:k]
+        m = min(n, k)
+        assert np.array_equal(ids[:m], ref[:m]), (n, k)
+        assert np.all(ids[m:] == -1)
+        assert np.array_equal(vals[:m], v[ref[:m]])
+
+
+def check_topk_with_ids(o):
+    rng = np.random.default_rng(8)
+    v = rng.integers(0, 4, size=40).astype(np.float64)
+    ids = rng.permutation(1000)[:40].astype(np.int32)
+    ids[::7] = -1  # empty slots are skipped
+    got, _ = o.topk(v, 12, ids)
+    # brute force: rank every valid item by (value desc, id asc) by counting the items it loses to
+    valid = [a for a in range(40) if ids[a] >= 0]
+    want = [ids[a] for a in valid
+            if sum((v[b] > v[a]) or (v[b] == v[a] and ids[b] < ids[a]) for b in valid) < 12]
+    assert sorted(got.tolist()) == sorted(want)
+
+
+def check_pool_special_cases(o):
+    rng = np.random.default_rng(9)
+    k = rng.standard_normal((37, 16)).astype(np.float32)
+    assert np.array_equal(o.pool_keys(k, 1), k.astype(np.float64)), "B = 1 pools to the keys"
+    for B in (37, 64):
+        got = o.pool_keys(k, B)
+        assert got.shape == (1, 16)
+        assert np.allclose(got[0], k.astype(np.float64).mean(axis=0), rtol=1e-14, atol=1e-15)
+    kc = np.tile(np.array([0.5, -2.0, 3.0, 0.0], np.float32), (10, 1))
+    assert np.array_equal(o.pool_keys(kc, 4), np.tile(kc[0].astype(np.float64), (3, 1)))
+    full = o.pool_keys(k, 8)  # 4 full blocks and one of 5 keys
+    k64 = k.astype(np.float64)
+    assert np.allclose(full[:4], k64[:32].reshape(4, 8, 16).mean(axis=1), rtol=1e-14, atol=1e-15)
+    assert np.allclose(full[4], k64[32:].mean(axis=0), rtol=1e-14, atol=1e-15)
+
+
+def _np_router_scores(q, w, k, n, B):
+    q, w, k = (np.asarray(a, np.float64) for a in (q, w, k))
+    M = -(-n // B)
+    means = np.stack([k[b * B:min((b + 1) * B, n)].mean(axis=0) for b in range(M)])
+    return w * np.maximum(q @ means.T, 0.0).sum(axis=1)
+
+
+def _brute_top_set(vals, h):
+    """The h-subset whose every member beats every non-member (value desc, index asc)."""
+    H = len(vals)
+    for S in itertools.combinations(range(H), h):
+        if all((vals[a] > vals[b]) or (vals[a] == vals[b] and a < b)
+               for a in S for b in range(H) if b not in S):
+            return set(S)
+    raise AssertionError("no consistent subset")
+
+
+def check_router_bruteforce(o):
+    rng = np.random.default_rng(10)
+    for trial in range(30):
+        H_I, d = 4, 4
+        L = int(rng.integers(1, 11))
+        B = int(rng.integers(1, 5))
+        h = int(rng.integers(1, H_I + 1))
+        q = rng.integers(-3, 4, size=(H_I, d)).astype(np.float32)
+        w = rng.integers(-2, 3, size=H_I).astype(np.float32)
+        k = rng.integers(-3, 4, size=(L, d)).astype(np.float32)
+        n = int(rng.integers(0, L + 1))
+        r, heads = o.route(q, w, k, n, B, h)
+        if n > 0:
+            assert np.allclose(r, _np_router_scores(q, w, k, n, B), rtol=1e-12, atol=1e-12), trial
+        else:
+            assert np.all(r == 0.0)
+        assert set(heads.tolist()) == _brute_top_set(r, h), (trial, r, heads)
+        assert all(r[heads[a]] >= r[heads[a + 1]] for a in range(h - 1)), "heads by descending r"
+
+
+def check_scores_bruteforce(o):
+    rng = np.random.default_rng(11)
+    for trial in range(20):
+        H_I, d, n = 5, 3, int(rng.integers(1, 9))
+        q = rng.integers(-3, 4, size=(H_I, d)).astype(np.float32)
+        w = rng.integers(-2, 3, size=H_I).astype(np.float32)
+        k = rng.integers(-3, 4, size=(n, d)).astype(np.float32)
+        heads = rng.permutation(H_I)[: int(rng.integers(1, H_I + 1))]
+        I = o.token_scores(q, w, heads, k, n)
+        for s in range(n):
+            want = 0.0
+            for j in sorted(heads):
+                dot = sum(float(q[j, i]) * float(k[s, i]) for i in range(d))
+                want += float(w[j]) * max(dot, 0.0)
+            assert I[s] == want, (trial, s, I[s], want)
+
+
+def _small_clustered(seed=0, H_I=8, d=16, L=300):
+    rng = np.random.default_rng(100 + seed)
+    k = rng.standard_normal((L, d)).astype(np.float32)
+    q = rng.standard_normal((H_I, d)).astype(np.float32)
+    w = (rng.standard_normal(H_I) / math.sqrt(H_I)).astype(np.float32)
+    return q, w, k
+
+
+def check_scaling(o):
+    q, w, k = _small_clustered(1)
+    n, B, h = 250, 16, 3
+    r, heads = o.route(q, w, k, n, B, h)
+    I = o.token_scores(q, w, heads, k, n)
+    top = o.topk(I, 20)[0]
+    for name, (q2, w2, k2) in {"k": (q, w, 2 * k), "q": (2 * q, w, k), "w": (q, 2 * w, k)}.items():
+        r2, heads2 = o.route(q2, w2, k2, n, B, h)
+        assert np.array_equal(r2, 2 * r), f"router scores scale with {name}"
+        assert np.array_equal(heads2, heads), f"routing unchanged under scaling of {name}"
+        I2 = o.token_scores(q2, w2, heads2, k2, n)
+        assert np.array_equal(I2, 2 * I), f"token scores scale with {name}"
+        assert np.array_equal(o.topk(I2, 20)[0], top)
+
+
+def check_head_permutation(o):
+    q, w, k = _small_clustered(2)
+    n, B, h = 300, 32, 4
+    r, heads = o.route(q, w, k, n, B, h)
+    perm = np.random.default_rng(3).permutation(q.shape[0])
+    r2, heads2 = o.route(q[perm], w[perm], k, n, B, h)
+    assert np.array_equal(r2, r[perm]), "router scores follow the head labels"
+    assert set(perm[heads2].tolist()) == set(heads.tolist())
+
+
+def check_full_routing_is_dense(o):
+    q, w, k = _small_clustered(3)
+    n = np.array([300, 123, 7], np.int32)
+    Q = np.stack([q, q[::-1], q * 0.5])
+    W = np.stack([w, -w, w])
+    H_I = q.shape[0]
+    for kk in (1, 10, 64):
+        m = o.indexer(0, Q, W, k, 0, n, 16, H_I, kk)
+        dd = o.indexer(2, Q, W, k, 0, n, 16, H_I, kk)
+        assert np.array_equal(m["idx"], dd["idx"]), "h = H_I reproduces the dense indexer"
+        assert np.array_equal(m["idx_v"], dd["idx_v"]), "bit-identical scores"
+
+
+def check_dagger_invariants(o):
+    q, w, k = _small_clustered(4, H_I=8, d=16, L=400)
+    Q = np.stack([q, q[::-1]])
+    W = np.stack([w, w[::-1]])
+    n = np.array([400, 333], np.int32)
+    B, h, kk = 25, 2, 16
+    dsa = o.indexer(2, Q, W, k, 0, n, B, h, kk)
+    misa = o.indexer(0, Q, W, k, 0, n, B, h, kk)
+    full = o.indexer(1, Q, W, k, 0, n, B, h, kk, kp=400)
+    assert np.array_equal(full["idx"], dsa["idx"]), "k' >= n makes MISA-dagger the dense indexer"
+    same = o.indexer(1, Q, W, k, 0, n, B, h, kk, kp=kk)
+    for t in range(2):
+        assert set(same["idx"][t]) == set(misa["idx"][t]), "k' = k makes MISA-dagger MISA"
+    prev = -1
+    for kp in (16, 32, 64, 128, 256, 400):
+        dag = o.indexer(1, Q, W, k, 0, n, B, h, kk, kp=kp)
+        rec = 0
+        for t in range(2):
+            C = set(dag["cand"][t]) - {-1}
+            S = set(dag["idx"][t]) - {-1}
+            D = set(dsa["idx"][t]) - {-1}
+            assert (D & C) <= S, "dense top-k tokens inside the candidate set are kept"
+            rec += len(D & S)
+        assert rec >= prev, "recovery does not drop as k' grows"
+        prev = rec
+
+
+def check_prefix_only(o):
+    q, w, k = _small_clustered(5)
+    n, B, h = 201, 16, 3
+    k2 = k.copy()
+    k2[n:] = 1000.0 * np.sign(k2[n:]) + 3.0
+    a = o.indexer(1, q[None], w[None], k, 0, np.array([n]), B, h, 20, kp=60)
+    b = o.indexer(1, q[None], w[None], k2, 0, np.array([n]), B, h, 20, kp=60)
+    for key in ("r", "heads", "cand", "idx", "idx_v"):
+        assert np.array_equal(a[key], b[key]), f"keys past the prefix changed {key}"
+    assert a["idx"].max() < n and a["cand"].max() < n
+
+
+def check_empty_and_short(o):
+    q, w, k = _small_clustered(6)
+    H_I = q.shape[0]
+    e = o.indexer(1, q[None], w[None], k, 0, np.array([0]), 16, 3, 5, kp=9)
+    assert np.all(e["idx"] == -1) and np.all(e["cand"] == -1), "empty prefix selects nothing"
+    assert list(e["heads"][0]) == [0, 1, 2], "all router scores tie at 0 -> lowest heads"
+    s = o.indexer(0, q[None], w[None], k, 0, np.array([3]), 16, 3, 5)
+    assert sorted(s["idx"][0][:3]) == [0, 1, 2] and list(s["idx"][0][3:]) == [-1, -1]
+    d = o.indexer(2, q[None], w[None], k, 0, np.array([3]), 16, H_I, 5)
+    assert sorted(d["idx"][0][:3]) == [0, 1, 2] and list(d["idx"][0][3:]) == [-1, -1]
+
+
+def check_negative_weight_sign(o):
+    q, w, k = _small_clustered(7)
+    w = np.abs(w)
+    w[[1, 4]] *= -1.0  # signed weights: a negative head scores <= 0 on the router
+    r, heads = o.route(q, w, k, 300, 16, 4)
+    assert r[1] <= 0 and r[4] <= 0
+    assert 1 not in heads and 4 not in heads
+
+
+def check_planted_needles(o):
+    wl = wlmod.WORKLOADS[1]
+    inp = wlmod.shared_inputs(wl)
+    res = o.indexer(1, inp.q, inp.w, inp.k, 0, inp.n, wl.B, wl.h, wl.topk, kp=4 * wl.topk)
+    dsa = o.indexer(2, inp.q, inp.w, inp.k, 0, inp.n, wl.B, wl.h, wl.topk)
+    misa = o.indexer(0, inp.q, inp.w, inp.k, 0, inp.n, wl.B, wl.h, wl.topk)
+    for t in range(wl.T):
+        assert set(inp.needle_heads.tolist()) <= set(res["heads"][t].tolist()), "needle heads routed"
+        for out in (res, dsa, misa):
+            assert set(inp.needle_pos.tolist()) <= set(out["idx"][t].tolist()), "needle tokens selected"
+
+
+ALL_CHECKS = [
+    check_hand_example,
+    check_topk_vs_stable_argsort,
+    check_topk_with_ids,
+    check_pool_special_cases,
+    check_router_bruteforce,
+    check_scores_bruteforce,
+    check_scaling,
+    check_head_permutation,
+    check_full_routing_is_dense,
+    check_dagger_invariants,
+    check_prefix_only,
+    check_empty_and_short,
+    check_negative_weight_sign,
+    check_planted_needles,
+]

@@ -1,0 +1,52 @@
+"""Plant one plausible mistake at a time in a copy of the oracle and show the pins catch it.
+
+Each mutant is a textual edit of the oracle source (a dropped term, a wrong sign, a wrong index,
+a reversed tie rule ...), compiled into a temporary directory; the real oracle is untouched.
+"""
+import os
+
+import pytest
+
+import oracle
+import oracle_pins
+
+MUTANTS = {
+    "token score without relu": (
+        "acc += (double)w[j] * orc_relu(orc_dot_ff(q + (int64_t)j * d, k + s * d, d));",
+        "acc += (double)w[j] * (orc_dot_ff(q + (int64_t)j * d, k + s * d, d));"),
+    "router without relu": ("acc += orc_relu(orc_dot_fd(", "acc += (orc_dot_fd("),
+    "router ignores head weight": ("r[j] = (double)w[j] * acc;", "r[j] = acc;"),
+    "block sum instead of mean": ("for (int i = 0; i < d; ++i) mean[i] /= c;", "(void)c;"),
+    "partial block dropped": ("for (int64_t b = 0; b < M; ++b) acc += orc_relu(",
+                              "for (int64_t b = 0; b < n / B; ++b) acc += orc_relu("),
+    "ties to the higher index": ("if (a->i < b->i) return -1;\n  if (a->i > b->i) return 1;",
+                                 "if (a->i < b->i) return 1;\n  if (a->i > b->i) return -1;"),
+    "ascending selection": ("if (a->v > b->v) return -1;\n  if (a->v < b->v) return 1;",
+                            "if (a->v > b->v) return 1;\n  if (a->v < b->v) return -1;"),
+    "relu keeps negatives": ("return x > 0.0 ? x : 0.0;", "return x < 0.0 ? x : 0.0;"),
+    "head row stride dropped": ("orc_dot_ff(q + (int64_t)j * d, k + s * d, d)",
+                                "orc_dot_ff(q + (int64_t)j, k + s * d, d)"),
+    "weight of slot, not of head": ("acc += (double)w[j] * orc_relu(orc_dot_ff(q + (int64_t)j * d, k + s * d, d));",
+                                    "acc += (double)w[a] * orc_relu(orc_dot_ff(q + (int64_t)j * d, k + s * d, d));"),
+    "dense re-rank with half the heads": ("      for (int j = 0; j < H_I; ++j)\n        acc += (double)w[j]",
+                                          "      for (int j = 0; j < H_I / 2; ++j)\n        acc += (double)w[j]"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, tmp_path):
+    old, new = MUTANTS[name]
+    with open(oracle.SOURCE) as f:
+        src = f.read()
+    assert src.count(old) >= 1, f"mutation site not found for {name!r}"
+    mutated = tmp_path / "mutant.c"
+    mutated.write_text(src.replace(old, new))
+    lib = oracle.compile_oracle(str(mutated), str(tmp_path / "libmutant.so"), force=True)
+    orc = oracle.Oracle(lib)
+    failures = []
+    for check in oracle_pins.ALL_CHECKS:
+        try:
+            check(orc)
+        except AssertionError:
+            failures.append(check.__name__)
+    assert failures, f"no pin catches the mutant {name!r}"
