@@ -1,0 +1,361 @@
+"""Benchmark of the MISA indexer hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload ID]
+
+One step is one decode step of MISA-dagger over a batch of sequences (default: 32 sequences x
+131072 keys, H_I = 64, d = 128, B = 128, h = 8, k' = 8192, k = 2048):
+    pool the block that holds the newest key -> route (block-pooled router, top-h heads) ->
+    routed token scores -> top-k' candidates -> dense re-rank of the candidates -> top-k.
+Inputs are seeded synthetic tensors resident in HBM (the key cache of 1 GiB per GPU is larger
+than L2, so every step streams it from HBM).  Metric: scored query-tokens per second
+(T x L / step time), summed over GPUs.  With torchrun every rank runs its own batch of sequences
+(independent problems, weak scaling); the time is the max over ranks.
+
+The reference arm (--impl reference) times the CPU oracle, as it stands, on the host cores, on a
+bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_sparse_mean_b200 import workloads as W  # noqa: E402
+
+METRIC = "scored query-tokens/s (Tq x L per s) at L=128K; % of HBM / bf16 TC roofline"
+UNIT = "query-tokens/s"
+
+# DRAM traffic of the routed scoring kernel from one ncu capture (dram__bytes_read.sum +
+# dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
+# bench reports null once the kernel source has changed since.
+TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu", "sha256": None, "bytes_per_key": None,
+           "capture": None}
+
+
+def _sha(path):
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def _workload(args):
+    return W.WORKLOADS[args.workload]
+
+
+def _config(wl, extra=None):
+    c = {"workload": wl.name, "T_per_gpu": wl.T, "L": wl.L, "H_I": wl.H_I, "d": wl.d, "B": wl.B, "h": wl.h,
+         "kp": wl.kp, "topk": wl.topk, "accumulate": "f32",
+         "l2": f"inputs larger than L2 ({wl.T * wl.L * wl.d * 2 / 2**30:.2f} GiB key cache per GPU)",
+         "step": "pool newest block + route + routed scores + top-k' + dense re-rank + top-k"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+def cpu_baseline_sample(wl, seqs, threads=None):
+    """Time the oracle, as it stands, on the given sequences (one decode query each)."""
+    import oracle
+    o = oracle.get()
+    k, q, w, n, _ = W.decode_batch(wl, seqs)
+    L, d = k.shape[1], k.shape[2]
+    t0 = time.perf_counter()
+    o.indexer(oracle.MODE_DAGGER if wl.kp else oracle.MODE_MISA, q, w, k, L * d, n, wl.B, wl.h, wl.topk,
+              kp=wl.kp or 0)
+    dt = time.perf_counter() - t0
+    return dt, o.num_threads()
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle on a bounded sample of the workload."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    wl = _workload(args)
+    import oracle
+    nthr = oracle.get().num_threads()
+    per_step = max(1, min(wl.T, nthr))
+    seqs = list(range(per_step))
+    for _ in range(args.warmup):
+        cpu_baseline_sample(wl, seqs)
+    times = []
+    for _ in range(args.steps):
+        dt, thr = cpu_baseline_sample(wl, seqs)
+        times.append(dt)
+    units = per_step * wl.L
+    total = sum(times)
+    value = units * args.steps / total
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": _config(wl, {"sample_sequences_per_step": per_step}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"{per_step} of {wl.T} sequences per step, whole MISA-dagger path, "
+                                   f"double precision, OpenMP over sequences"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    from long_context_sparse_mean_b200 import binding as M
+
+    wl = _workload(args)
+    big = W.small(wl.cid, n_seq=wl.n_seq * ws, T=wl.T * ws)
+    seqs = list(range(rank * wl.T, (rank + 1) * wl.T))
+    k_h, q_h, w_h, n_h, _ = W.decode_batch(big, seqs)
+    T, L, d = k_h.shape
+    kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
+    qd = torch.from_numpy(q_h).to(torch.bfloat16).to(dev)
+    wd = torch.from_numpy(w_h).to(dev)
+    nd = torch.from_numpy(n_h).to(dev)
+    B, h, kp, kk, H_I = wl.B, wl.h, wl.kp, wl.topk, wl.H_I
+    M_ = -(-L // B)
+    stream = torch.cuda.current_stream()
+    wsp = M.Workspace(dev)
+    kbar = M.misa_pool_keys(kd, B)
+    heads = torch.empty((T, h), dtype=torch.int32, device=dev)
+    scores = torch.empty((T, L), dtype=torch.float32, device=dev)
+    cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
+    idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+    vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    score_ms = []
+    launches_per_step = 8  # pool, 3 router kernels, scores, top-k', re-rank scores, re-rank select
+
+    def step(time_scores=False):
+        M.misa_pool_keys(kd, B, kbar=kbar, block_begin=M_ - 1, block_end=M_)
+        M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
+        if time_scores:
+            ev[0].record(stream)
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
+        if time_scores:
+            ev[1].record(stream)
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False)
+        M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    # one timed pass over the step for the scoring-kernel duration (events bracket that launch)
+    for _ in range(min(args.steps, 50)):
+        step(time_scores=True)
+        torch.cuda.synchronize()
+        score_ms.append(ev[0].elapsed_time(ev[1]))
+
+    # the timed region: K whole steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if ws > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    units_per_step = T * L * ws
+    value = units_per_step * args.steps / (ms / 1000.0)
+
+    # end to end through the public API with host buffers: per step the new query q, its head
+    # weights w, the newest key of every sequence (written into the cache) and n go host->device,
+    # and the selected indices come back device->host.
+    q_pin = torch.from_numpy(q_h).to(torch.bfloat16).pin_memory()
+    w_pin = torch.from_numpy(w_h).pin_memory()
+    n_pin = torch.from_numpy(n_h).pin_memory()
+    knew_pin = torch.from_numpy(k_h[:, L - 1, :].copy()).to(torch.bfloat16).pin_memory()
+    knew_d = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    idx_pin = torch.empty((T, kk), dtype=torch.int32).pin_memory()
+    h2d = q_pin.numel() * 2 + w_pin.numel() * 4 + n_pin.numel() * 4 + knew_pin.numel() * 2
+    d2h = idx_pin.numel() * 4
+
+    def e2e_step():
+        qd.copy_(q_pin, non_blocking=True)
+        wd.copy_(w_pin, non_blocking=True)
+        nd.copy_(n_pin, non_blocking=True)
+        knew_d.copy_(knew_pin, non_blocking=True)
+        kd[:, L - 1, :].copy_(knew_d)
+        step()
+        idx_pin.copy_(idx, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        tt = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    e2e_value = units_per_step * args.steps / (e_ms / 1000.0)
+
+    # dense DSA on the same inputs (the baseline the pages compare against), not part of the step
+    dsa_ms = None
+    if not args.no_dense:
+        for _ in range(3):
+            M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=idx, vals=vals, ws=wsp)
+        torch.cuda.synchronize()
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nrep = min(args.steps, 20)
+        d0.record(stream)
+        for _ in range(nrep):
+            M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=idx, vals=vals, ws=wsp)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dsa_ms = d0.elapsed_time(d1) / nrep
+
+    if rank == 0:
+        hbm, kind = _peaks()
+        score_avg = sum(score_ms) / len(score_ms)
+        alg_bytes = T * (L * d * 2 + h * d * 2 + h * 4)
+        achieved = alg_bytes / (score_avg / 1000.0) / 1e9
+        traffic = None
+        if TRAFFIC["sha256"] and TRAFFIC["sha256"] == _sha(TRAFFIC["file"]) and TRAFFIC["bytes_per_key"]:
+            traffic = TRAFFIC["bytes_per_key"] * T * L
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU"}),
+            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_bf16_kernel)",
+                         "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
+                         "frac": achieved / hbm, "traffic": traffic,
+                         "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk.summary(),
+            "dense_dsa_same_inputs": None if dsa_ms is None else {
+                "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0)},
+        }
+        if not args.no_cpu_baseline:
+            per = max(1, min(T, os.cpu_count() or 1))
+            dt, thr = cpu_baseline_sample(wl, list(range(per)))
+            line["cpu_baseline"] = {"value": per * L / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+                                    "sample": f"{per} of {T} sequences, one pass of the whole MISA-dagger path, "
+                                              f"double precision, OpenMP over sequences"}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=4, choices=[2, 4, 5])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

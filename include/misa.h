@@ -1,0 +1,176 @@
+/*
+ * misa.h -- C ABI of the MISA indexer library (libmisa.so, CUDA, sm_100a).
+ *
+ * The method is the one on "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
+ * Inference" (gist.science/paper/2605.07363), "Technical Summary":
+ *   - "Methodology: MISA", "Lightweight Block-Pooled Router": the prefix is cut into
+ *     M = ceil(L/B) blocks of B keys, every block is summarised by the mean of its index keys,
+ *     every indexer head gets one affinity aggregated over those pooled keys, and the h best of
+ *     the H_I heads are routed;
+ *   - "Methodology: MISA", "Sparse Token Scoring": only the routed heads score every prefix
+ *     token and the top-k tokens by that reduced score are kept;
+ *   - "Hierarchical Variant (MISA-dagger)": the routed pass keeps k' > k candidates that the
+ *     dense indexer with all H_I heads re-scores, keeping the top-k;
+ *   - "Problem Statement": the dense DSA indexer scores every prefix token with all H_I heads.
+ * The pages do not write the formulas.  This library computes, for query t with prefix n_t:
+ *   kbar_b  = mean of keys [bB, min((b+1)B, n_t))             (b < M_t = ceil(n_t/B))
+ *   r_{t,j} = w_{t,j} * sum_{b < M_t} max(0, q_{t,j} . kbar_b)     (router score of head j)
+ *   R_t     = the h heads with the largest r_{t,j}                 (ties to the lower head)
+ *   I_{t,s} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . k_s)       (s < n_t)
+ *   F_{t,s} = sum_{j < H_I}  w_{t,j} * max(0, q_{t,j} . k_s)       (dense score)
+ * No scale factor is applied.  Selections order by score descending; exact ties go to the lower
+ * token index.  Scores are accumulated in fp32 (bf16 products are exact in fp32).
+ *
+ * Common conventions
+ *   - Every pointer argument is device memory owned by the caller unless stated otherwise.
+ *     Nothing is allocated inside the library; scratch comes from the caller's workspace
+ *     (size from misa_workspace_bytes), which must be 256-byte aligned.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream).
+ *     Arguments are validated on the host before any launch; on error nothing is launched.
+ *   - Layouts are dense row-major.  q is [T, H_I, d], w is [T, H_I] (fp32), n is [T] (int32).
+ *     The key cache of query t starts at k + t * k_seq_stride elements: k_seq_stride = 0 makes
+ *     all queries share one cache (prefill), k_seq_stride = L*d gives one cache per query
+ *     (batched decode).  Each cache holds L keys of d elements.
+ *   - dtype is the element type of q and k (MISA_BF16 or MISA_F32).  d must be 128.
+ *     H_I must be a multiple of 8 in [8, 128]; 1 <= h <= H_I.
+ *   - Prefix lengths n_t are read on the device: values above L count as L, values below 1 give
+ *     an empty prefix (no tokens selected; all router scores 0).
+ *   - Index outputs hold min(topk, n_t) token indices followed by -1 padding.  The selected set
+ *     is what the method defines; misa_score_topk and dsa_dense_topk write it in ascending token
+ *     order, misa_hier_rerank in the order of the candidate list.
+ *   - Errors: MISA_ERR_INVALID_ARG (null pointer, size out of range), MISA_ERR_UNSUPPORTED
+ *     (d != 128, H_I not a multiple of 8, dtype, k' too large), MISA_ERR_WORKSPACE (workspace
+ *     too small or misaligned), MISA_ERR_CUDA (a launch failed; cudaGetLastError's code is
+ *     consumed).
+ */
+#ifndef MISA_H_
+#define MISA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MISA_OK = 0,
+  MISA_ERR_INVALID_ARG = 1,
+  MISA_ERR_UNSUPPORTED = 2,
+  MISA_ERR_WORKSPACE = 3,
+  MISA_ERR_CUDA = 4
+} misa_status;
+
+typedef enum { MISA_BF16 = 0, MISA_F32 = 1 } misa_dtype;
+
+/* Operation codes for misa_workspace_bytes. */
+typedef enum {
+  MISA_OP_ROUTE = 0,
+  MISA_OP_SCORE_TOPK = 1,
+  MISA_OP_RERANK = 2,
+  MISA_OP_DENSE_TOPK = 3,
+  MISA_OP_TOPK_SELECT = 4
+} misa_op;
+
+/* Largest k' accepted by misa_hier_rerank (its candidates are ranked in shared memory). */
+#define MISA_MAX_KP 16384
+
+/* Library version, major*10000 + minor*100 + patch. */
+int misa_version(void);
+
+/* Static text for a status code. */
+const char* misa_status_str(int status);
+
+/*
+ * Workspace bytes needed by one call of `op` with these sizes (0 if it needs none).
+ * Arguments an op does not use are ignored.  Sizes <= 0 give 0.
+ */
+size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp);
+
+/*
+ * Block mean-pool of key caches ("Lightweight Block-Pooled Router": mean-pooled indexing keys
+ * over M = ceil(L/B) blocks).
+ *   k      : n_seq caches of L keys [L, d] at stride k_seq_stride elements (dtype)
+ *   kbar   : out, fp32, n_seq x [ceil(L/B), d] at stride kbar_seq_stride floats
+ *   blocks [block_begin, block_end) of every cache are written (clamped to [0, ceil(L/B)));
+ *   block b averages keys [bB, min((b+1)B, L)) (a partial last block over its valid keys).
+ * A decode loop calls it with [b, b+1) for the block that just filled.
+ */
+misa_status misa_pool_keys(const void* k, int64_t k_seq_stride, int n_seq, int L, int d, int B,
+                           int dtype, float* kbar, int64_t kbar_seq_stride, int block_begin,
+                           int block_end, void* stream);
+
+/*
+ * Block-pooled router and top-h head selection ("Lightweight Block-Pooled Router").
+ *   kbar   : fp32 block means from misa_pool_keys; query t reads kbar + t*kbar_seq_stride
+ *            (0 = shared).  Only full blocks b < floor(n_t/B) are read from it; the partial
+ *            last block of a prefix (n_t not a multiple of B) is averaged from k directly.
+ *   heads  : out [T, h] int32, routed heads in descending router score (ties: lower head)
+ *   r_opt  : out [T, H_I] fp32 router scores, or NULL
+ *   ws     : workspace of misa_workspace_bytes(MISA_OP_ROUTE, T, L, H_I, B, h, 0, 0) bytes
+ */
+misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                       const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
+                       int H_I, int d, int B, int h, int dtype, int32_t* heads, float* r_opt,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Routed-head token scores ("Sparse Token Scoring"): scores[t, s] = I_{t,s} for s < n_t.
+ *   heads  : [T, h] routed heads (any order; NULL = all H_I heads, i.e. the dense score F)
+ *   scores : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
+ */
+misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                              const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
+                              int h, int dtype, float* scores, int64_t ld_scores, void* stream);
+
+/*
+ * Top-k selection over per-query score rows ("Sparse Token Scoring": the final top-k tokens
+ * are selected on the reduced scores).  scores [T, ld_scores] fp32, entries s < n_t are read.
+ *   idx       : out [T, topk] int32, ascending token order, -1 padded
+ *   score_opt : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
+ * Scores must be finite.  No workspace is needed (pass NULL, 0).
+ */
+misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
+                             int L, int topk, int32_t* idx, float* score_opt, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Routed scoring followed by top-k: misa_token_scores then misa_topk_select.  With topk = k'
+ * this is the coarse stage of MISA-dagger ("Hierarchical Variant": enlarged candidate set).
+ *   scores_full_opt : [T, L] fp32 buffer that receives every score, or NULL to use workspace
+ *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK, T, L, ...) bytes (0 if scores_full_opt given)
+ */
+misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                            const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
+                            int h, int topk, int dtype, int32_t* idx, float* score_opt,
+                            float* scores_full_opt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * MISA-dagger fine stage ("Hierarchical Variant (MISA-dagger)": the dense indexer with all H_I
+ * heads re-scores only the k' candidates and keeps the final top-k).
+ *   cand      : [T, kp] candidate token indices; entries < 0 or >= n_t are empty slots
+ *   idx       : out [T, topk] the kept candidates (candidate-list order), -1 padded
+ *   score_opt : out [T, topk] their dense scores, or NULL
+ *   ws        : misa_workspace_bytes(MISA_OP_RERANK, T, 0, H_I, 0, 0, topk, kp) bytes
+ * Requires topk <= kp <= MISA_MAX_KP; duplicate candidates are the caller's error.
+ */
+misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                             const int32_t* n, const int32_t* cand, int T, int L, int H_I, int d,
+                             int kp, int topk, int dtype, int32_t* idx, float* score_opt, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * Dense DSA indexer ("Problem Statement": every prefix token scored with all H_I heads, top-k
+ * kept): top-k of F_{t,s} over s < n_t.  Outputs as misa_score_topk.
+ *   ws : misa_workspace_bytes(MISA_OP_DENSE_TOPK, T, L, ...) bytes
+ */
+misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                           const int32_t* n, int T, int L, int H_I, int d, int topk, int dtype,
+                           int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
+                           void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MISA_H_ */

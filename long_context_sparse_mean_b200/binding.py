@@ -1,0 +1,297 @@
+"""Python binding of libmisa.so: argument marshalling only.
+
+Each function has the name of the C entry point it calls (include/misa.h) and passes torch
+tensors' device pointers and the current CUDA stream through ctypes.  Every step of the indexer
+runs in the library's CUDA kernels; there is no fallback.  If libmisa.so is missing the import
+of this module fails.
+
+Tensor conventions (all on one CUDA device, contiguous):
+  q [T, H_I, 128] bf16 or fp32, w [T, H_I] fp32, n [T] int32 (prefix lengths),
+  k [L, 128] (one cache shared by all queries) or [T, L, 128] (cache t for query t), same dtype as q,
+  kbar [M, 128] or [T, M, 128] fp32 with M = ceil(L / B).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libmisa.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = range(5)
+BF16, F32 = 0, 1
+OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT = range(5)
+MAX_KP = 16384
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is not built: run `python -m long_context_sparse_mean_b200.build`")
+
+
+class MisaError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {_lib.misa_status_str(status).decode()} (status {status})")
+        self.status = status
+
+
+def _setup(lib):
+    P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
+    sigs = {
+        "misa_version": ([], i32),
+        "misa_status_str": ([i32], ctypes.c_char_p),
+        "misa_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32, i32], sz),
+        "misa_pool_keys": ([P, i64, i32, i32, i32, i32, i32, P, i64, i32, i32, P], i32),
+        "misa_route": ([P, P, P, i64, P, i64, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
+        "misa_token_scores": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, P, i64, P], i32),
+        "misa_topk_select": ([P, i64, P, i32, i32, i32, P, P, P, sz, P], i32),
+        "misa_score_topk": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, sz, P], i32),
+        "misa_hier_rerank": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
+        "dsa_dense_topk": ([P, P, P, i64, P, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
+    }
+    for name, (args, res) in sigs.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    return lib
+
+
+_lib = _setup(ctypes.CDLL(LIB_PATH))
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream: Optional[torch.cuda.Stream] = None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != OK:
+        raise MisaError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"q/k must be bfloat16 or float32, got {t.dtype}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _cache_geometry(k: torch.Tensor, T: int):
+    """(L, d, k_seq_stride) of a shared [L, d] or per-query [T, L, d] key cache."""
+    if k.dim() == 2:
+        return k.shape[0], k.shape[1], 0
+    if k.dim() == 3:
+        if k.shape[0] != T:
+            raise ValueError(f"per-query cache needs k.shape[0] == T ({T}), got {k.shape[0]}")
+        return k.shape[1], k.shape[2], k.shape[1] * k.shape[2]
+    raise ValueError("k must be [L, d] or [T, L, d]")
+
+
+def misa_workspace_bytes(op: int, T: int, L: int, H_I: int, B: int = 1, h: int = 0, topk: int = 0,
+                         kp: int = 0) -> int:
+    return int(_lib.misa_workspace_bytes(op, T, L, H_I, B, h, topk, kp))
+
+
+class Workspace:
+    """A reusable, 256-byte aligned device scratch buffer (grown on demand)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, nbytes: int) -> Optional[torch.Tensor]:
+        if nbytes <= 0:
+            return None
+        if self.buf is None or self.buf.numel() < nbytes:
+            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _ws(ws: Optional[Workspace], device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, block_begin: int = 0,
+                   block_end: Optional[int] = None, stream=None) -> torch.Tensor:
+    """Block means of every cache: k [L,d] or [S,L,d] -> kbar [M,d] or [S,M,d] (fp32)."""
+    _need(k, "k")
+    shared = k.dim() == 2
+    S = 1 if shared else k.shape[0]
+    L, d = k.shape[-2], k.shape[-1]
+    M = -(-L // B)
+    if kbar is None:
+        kbar = torch.empty((M, d) if shared else (S, M, d), dtype=torch.float32, device=k.device)
+    _need(kbar, "kbar", torch.float32)
+    block_end = M if block_end is None else block_end
+    _check("misa_pool_keys", _lib.misa_pool_keys(
+        _p(k), 0 if shared else L * d, S, L, d, B, _dtype_code(k), _p(kbar), 0 if shared else M * d,
+        block_begin, block_end, _stream(stream)))
+    return kbar
+
+
+def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optional[Workspace] = None,
+               want_r: bool = False, stream=None):
+    """Routed heads [T, h] (descending router score) and, if asked, router scores r [T, H_I]."""
+    for t, nm in ((q, "q"), (k, "k")):
+        _need(t, nm)
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(kbar, "kbar", torch.float32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    kbss = 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
+    if heads is None:
+        heads = torch.empty((T, h), dtype=torch.int32, device=q.device)
+    if r is None and want_r:
+        r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_ROUTE, T, L, H_I, B, h)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_route", _lib.misa_route(
+        _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r),
+        _p(buf), nbytes, _stream(stream)))
+    return heads, r
+
+
+def misa_token_scores(q, w, k, n, heads=None, out=None, stream=None) -> torch.Tensor:
+    """Scores [T, L] fp32 (entries s >= n_t untouched); heads None = all heads (dense score)."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    h = 0
+    if heads is not None:
+        _need(heads, "heads", torch.int32)
+        h = heads.shape[1]
+    if out is None:
+        out = torch.empty((T, L), dtype=torch.float32, device=q.device)
+    _need(out, "out", torch.float32)
+    _check("misa_token_scores", _lib.misa_token_scores(
+        _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, _dtype_code(q), _p(out), out.shape[1],
+        _stream(stream)))
+    return out
+
+
+def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, vals=None, want_vals=True,
+                     stream=None):
+    """Top-k per row of scores [T, ld] over entries s < min(n_t, L) -> (idx [T, k], vals [T, k])."""
+    _need(scores, "scores", torch.float32)
+    _need(n, "n", torch.int32)
+    T, ld = scores.shape
+    L = ld if L is None else L
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=scores.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=scores.device)
+    _check("misa_topk_select", _lib.misa_topk_select(
+        _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), None, 0, _stream(stream)))
+    return idx, vals
+
+
+def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_full=None, want_vals=True,
+                    ws: Optional[Workspace] = None, stream=None):
+    """Routed scoring + top-k -> (idx [T, k] ascending token order, vals [T, k])."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(heads, "heads", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    h = heads.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = 0 if scores_full is not None else misa_workspace_bytes(OP_SCORE_TOPK, T, L, H_I, 1, h, topk)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_score_topk", _lib.misa_score_topk(
+        _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, topk, _dtype_code(q), _p(idx), _p(vals),
+        _p(scores_full), _p(buf), nbytes, _stream(stream)))
+    return idx, vals
+
+
+def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals=True,
+                     ws: Optional[Workspace] = None, stream=None):
+    """MISA-dagger fine stage: dense re-score of cand [T, k'] -> (idx [T, k], vals [T, k])."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(cand, "cand", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    kp = cand.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_RERANK, T, L, H_I, 1, 0, topk, kp)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_hier_rerank", _lib.misa_hier_rerank(
+        _p(q), _p(w), _p(k), kss, _p(n), _p(cand), T, L, H_I, d, kp, topk, _dtype_code(q), _p(idx), _p(vals),
+        _p(buf), nbytes, _stream(stream)))
+    return idx, vals
+
+
+def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, ws: Optional[Workspace] = None,
+                   stream=None):
+    """Dense all-head indexer -> (idx [T, k] ascending token order, vals [T, k])."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_DENSE_TOPK, T, L, H_I, 1, 0, topk)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("dsa_dense_topk", _lib.dsa_dense_topk(
+        _p(q), _p(w), _p(k), kss, _p(n), T, L, H_I, d, topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes,
+        _stream(stream)))
+    return idx, vals
+
+
+def misa_indexer(q, w, k, kbar, n, B: int, h: int, topk: int, kp: Optional[int] = None,
+                 ws: Optional[Workspace] = None, stream=None):
+    """The whole indexer for one batch: route -> routed scoring -> top-k (MISA), or with kp given
+    route -> routed scoring -> top-k' candidates -> dense re-rank -> top-k (MISA-dagger).
+    Returns a dict with idx [T, k], vals [T, k], heads [T, h] and (MISA-dagger) cand [T, k']."""
+    heads, _ = misa_route(q, w, k, kbar, n, B, h, ws=ws, stream=stream)
+    if kp is None:
+        idx, vals = misa_score_topk(q, w, k, n, heads, topk, ws=ws, stream=stream)
+        return {"idx": idx, "vals": vals, "heads": heads}
+    cand, _ = misa_score_topk(q, w, k, n, heads, kp, want_vals=False, ws=ws, stream=stream)
+    idx, vals = misa_hier_rerank(q, w, k, n, cand, topk, ws=ws, stream=stream)
+    return {"idx": idx, "vals": vals, "heads": heads, "cand": cand}

@@ -1,0 +1,215 @@
+// C ABI of the MISA indexer library: argument checks, workspace layout, launch order.
+// The declarations and their documentation are in include/misa.h.
+#include <cuda_runtime.h>
+
+#include "../../include/misa.h"
+#include "kernels.cuh"
+
+using misa::DType;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) % kAlign) == 0; }
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Row stride of internal score buffers: L rounded up to 4 floats (16 bytes).
+int64_t score_ld(int L) { return (L + 3) / 4 * 4; }
+
+misa_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MISA_OK : MISA_ERR_CUDA;
+}
+
+misa_status check_common(const void* q, const float* w, const void* k, const int32_t* n, int T, int L,
+                         int H_I, int d, int dtype, int64_t k_seq_stride) {
+  if (T < 0 || L < 1 || k_seq_stride < 0) return MISA_ERR_INVALID_ARG;
+  if (T > 0 && (!q || !w || !k || !n)) return MISA_ERR_INVALID_ARG;
+  if (dtype != MISA_BF16 && dtype != MISA_F32) return MISA_ERR_UNSUPPORTED;
+  if (d != misa::kD) return MISA_ERR_UNSUPPORTED;
+  if (H_I < 8 || H_I > misa::kMaxHeads || H_I % 8 != 0) return MISA_ERR_UNSUPPORTED;
+  if (k_seq_stride != 0 && k_seq_stride < (int64_t)L * d) return MISA_ERR_INVALID_ARG;
+  return MISA_OK;
+}
+
+DType to_dtype(int dtype) { return dtype == MISA_F32 ? DType::F32 : DType::BF16; }
+
+cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+size_t route_ws(int T, int L, int H_I, int B) {
+  if (T <= 0 || L <= 0 || H_I <= 0 || B <= 0) return 0;
+  const size_t pm = align_up(sizeof(float) * (size_t)T * misa::kD);
+  const size_t part = align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
+  return pm + part;
+}
+
+size_t scores_ws(int T, int L) {
+  if (T <= 0 || L <= 0) return 0;
+  return align_up(sizeof(float) * (size_t)T * score_ld(L));
+}
+
+size_t rerank_ws(int T, int kp) {
+  if (T <= 0 || kp <= 0) return 0;
+  return align_up(sizeof(float) * (size_t)T * kp);
+}
+
+}  // namespace
+
+extern "C" {
+
+int misa_version(void) { return 100; }
+
+const char* misa_status_str(int status) {
+  switch (status) {
+    case MISA_OK:
+      return "ok";
+    case MISA_ERR_INVALID_ARG:
+      return "invalid argument";
+    case MISA_ERR_UNSUPPORTED:
+      return "unsupported configuration";
+    case MISA_ERR_WORKSPACE:
+      return "workspace too small or misaligned";
+    case MISA_ERR_CUDA:
+      return "CUDA launch failed";
+    default:
+      return "unknown status";
+  }
+}
+
+size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
+  (void)h;
+  (void)topk;
+  switch (op) {
+    case MISA_OP_ROUTE:
+      return route_ws(T, L, H_I, B);
+    case MISA_OP_SCORE_TOPK:
+    case MISA_OP_DENSE_TOPK:
+      return scores_ws(T, L);
+    case MISA_OP_RERANK:
+      return rerank_ws(T, kp);
+    case MISA_OP_TOPK_SELECT:
+    default:
+      return 0;
+  }
+}
+
+misa_status misa_pool_keys(const void* k, int64_t k_seq_stride, int n_seq, int L, int d, int B, int dtype,
+                           float* kbar, int64_t kbar_seq_stride, int block_begin, int block_end, void* stream) {
+  if (n_seq < 0 || L < 1 || B < 1 || k_seq_stride < 0 || kbar_seq_stride < 0) return MISA_ERR_INVALID_ARG;
+  if (dtype != MISA_BF16 && dtype != MISA_F32) return MISA_ERR_UNSUPPORTED;
+  if (d != misa::kD) return MISA_ERR_UNSUPPORTED;
+  const int M = (int)ceil_div(L, B);
+  if (n_seq > 1 && (k_seq_stride < (int64_t)L * d || kbar_seq_stride < (int64_t)M * d)) return MISA_ERR_INVALID_ARG;
+  const int b0 = block_begin < 0 ? 0 : block_begin;
+  const int b1 = block_end > M ? M : block_end;
+  if (n_seq == 0 || b1 <= b0) return MISA_OK;
+  if (!k || !kbar) return MISA_ERR_INVALID_ARG;
+  misa::launch_pool(to_dtype(dtype), k, k_seq_stride, n_seq, L, B, kbar, kbar_seq_stride, b0, b1,
+                    as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_seq_stride, const float* kbar,
+                       int64_t kbar_seq_stride, const int32_t* n, int T, int L, int H_I, int d, int B, int h,
+                       int dtype, int32_t* heads, float* r_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (B < 1 || h < 1 || h > H_I || kbar_seq_stride < 0) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!kbar || !heads) return MISA_ERR_INVALID_ARG;
+  const size_t need = route_ws(T, L, H_I, B);
+  if (!ws || ws_bytes < need || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  float* pm = static_cast<float*>(ws);
+  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * misa::kD));
+  misa::launch_route(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, T, L, H_I, B, h, heads,
+                     r_opt, pm, partial, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                              const int32_t* heads, int T, int L, int H_I, int d, int h, int dtype, float* scores,
+                              int64_t ld_scores, void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (heads && (h < 1 || h > H_I)) return MISA_ERR_INVALID_ARG;
+  if (ld_scores < L) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!scores) return MISA_ERR_INVALID_ARG;
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, heads ? h : H_I, nullptr, 0,
+                      scores, ld_scores, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T, int L, int topk,
+                             int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+  (void)ws;
+  (void)ws_bytes;
+  if (T < 0 || L < 1 || topk < 1 || ld_scores < L) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
+  misa::launch_topk_rows(scores, ld_scores, n, T, L, topk, idx, score_opt, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                            const int32_t* heads, int T, int L, int H_I, int d, int h, int topk, int dtype,
+                            int32_t* idx, float* score_opt, float* scores_full_opt, void* ws, size_t ws_bytes,
+                            void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (!heads && T > 0) return MISA_ERR_INVALID_ARG;
+  if (h < 1 || h > H_I || topk < 1) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!idx) return MISA_ERR_INVALID_ARG;
+  float* buf = scores_full_opt;
+  int64_t ld = L;
+  if (!buf) {
+    if (!ws || ws_bytes < scores_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+    buf = static_cast<float*>(ws);
+    ld = score_ld(L);
+  }
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld,
+                      as_stream(stream));
+  misa::launch_topk_rows(buf, ld, n, T, L, topk, idx, score_opt, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                             const int32_t* cand, int T, int L, int H_I, int d, int kp, int topk, int dtype,
+                             int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (topk < 1 || kp < topk) return MISA_ERR_INVALID_ARG;
+  if (kp > MISA_MAX_KP) return MISA_ERR_UNSUPPORTED;
+  if (T == 0) return MISA_OK;
+  if (!cand || !idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  float* F = static_cast<float*>(ws);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp,
+                      as_stream(stream));
+  misa::launch_topk_cand(F, cand, n, T, L, kp, topk, idx, score_opt, as_stream(stream));
+  return launch_status();
+}
+
+misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                           int T, int L, int H_I, int d, int topk, int dtype, int32_t* idx, float* score_opt,
+                           void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (topk < 1) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < scores_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  float* buf = static_cast<float*>(ws);
+  const int64_t ld = score_ld(L);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
+                      as_stream(stream));
+  misa::launch_topk_rows(buf, ld, n, T, L, topk, idx, score_opt, as_stream(stream));
+  return launch_status();
+}
+
+}  // extern "C"

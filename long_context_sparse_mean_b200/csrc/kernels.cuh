@@ -1,0 +1,37 @@
+// Internal launchers of the MISA indexer kernels (C++ linkage; the C ABI lives in capi.cu).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace misa {
+
+// Block mean-pool ("Lightweight Block-Pooled Router": mean-pooled index keys).
+void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L, int B,
+                 float* kbar, int64_t kbar_seq_stride, int b0, int b1, cudaStream_t s);
+
+// Router: partial-block means, per-chunk affinities, then sum, weight and top-h.
+int route_chunks(int L, int B);  // chunks of kRouteTile blocks per query (upper bound)
+void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                  const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
+                  int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
+                  cudaStream_t s);
+
+// Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
+// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].
+void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                   const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
+                   const int32_t* rows, int P, float* out, int64_t ld, cudaStream_t s);
+
+// Top-k of each score row (entries s < n_t), output in ascending token order.
+void launch_topk_rows(const float* scores, int64_t ld, const int32_t* n, int T, int L, int topk,
+                      int32_t* idx, float* score_opt, cudaStream_t s);
+
+// Top-k of candidate lists: values F[t, P], ids cand[t, P] (ids outside [0, n_t) are empty).
+size_t topk_cand_smem(int P);
+void launch_topk_cand(const float* F, const int32_t* cand, const int32_t* n, int T, int L, int P,
+                      int topk, int32_t* idx, float* score_opt, cudaStream_t s);
+
+}  // namespace misa

@@ -1,0 +1,134 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every function that
+include/misa.h declares, sizes workspaces, and rejects bad arguments on the host before any
+launch (these calls never reach the CUDA runtime)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_sparse_mean_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "misa.h")
+
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = range(5)
+BF16, F32 = 0, 1
+P = ctypes.c_void_p
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:misa_status|size_t|int|const char\s*\*)\s*(\w+)\s*\(", src, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    path = build.build()
+    lib = ctypes.CDLL(path)
+    from long_context_sparse_mean_b200 import binding  # sets the argtypes
+    return binding.library()
+
+
+def test_header_declares_the_indexer_calls():
+    names = declared_functions()
+    for want in ("misa_pool_keys", "misa_route", "misa_token_scores", "misa_topk_select", "misa_score_topk",
+                 "misa_hier_rerank", "dsa_dense_topk", "misa_workspace_bytes", "misa_status_str", "misa_version"):
+        assert want in names, want
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in misa.h but not exported"
+
+
+def test_status_strings_and_version(lib):
+    assert lib.misa_version() >= 100
+    for code in range(5):
+        assert lib.misa_status_str(code)
+    assert lib.misa_status_str(99) == b"unknown status"
+
+
+def test_workspace_sizes(lib):
+    ws = lib.misa_workspace_bytes
+    # router: [T,128] partial-block means + [T, ceil(ceil(L/B)/64), H_I] tile sums, each 256-aligned
+    assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4
+    assert ws(1, 32, 131072, 64, 128, 8, 8192, 0) == 32 * 131072 * 4
+    assert ws(1, 3, 1001, 64, 1, 8, 10, 0) == (3 * 1004 * 4 + 255) // 256 * 256
+    assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4
+    assert ws(3, 64, 131072, 32, 0, 0, 2048, 0) == 64 * 131072 * 4
+    assert ws(4, 64, 131072, 32, 0, 0, 2048, 0) == 0
+    assert ws(1, 0, 100, 64, 1, 8, 10, 0) == 0
+
+
+FAKE = P(0x10000)        # never dereferenced: every call below fails validation first
+MISALIGNED = P(0x10008)
+
+
+def route(lib, **kw):
+    a = dict(q=FAKE, w=FAKE, k=FAKE, kss=0, kbar=FAKE, kbss=0, n=FAKE, T=4, L=1000, H_I=64, d=128, B=64, h=8,
+             dt=BF16, heads=FAKE, r=None, ws=FAKE, wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.misa_route(a["q"], a["w"], a["k"], a["kss"], a["kbar"], a["kbss"], a["n"], a["T"], a["L"], a["H_I"],
+                          a["d"], a["B"], a["h"], a["dt"], a["heads"], a["r"], a["ws"], a["wsb"], a["s"])
+
+
+def test_router_argument_checks(lib):
+    assert route(lib, d=64) == UNSUPPORTED
+    assert route(lib, H_I=12) == UNSUPPORTED
+    assert route(lib, H_I=136) == UNSUPPORTED
+    assert route(lib, dt=7) == UNSUPPORTED
+    assert route(lib, h=0) == INVALID
+    assert route(lib, h=65) == INVALID
+    assert route(lib, B=0) == INVALID
+    assert route(lib, L=0) == INVALID
+    assert route(lib, T=-1) == INVALID
+    assert route(lib, q=None) == INVALID
+    assert route(lib, kbar=None) == INVALID
+    assert route(lib, heads=None) == INVALID
+    assert route(lib, kss=1000 * 128 - 1) == INVALID
+    assert route(lib, ws=None) == WORKSPACE
+    assert route(lib, wsb=100) == WORKSPACE
+    assert route(lib, ws=MISALIGNED) == WORKSPACE
+    assert route(lib, T=0, q=None, w=None, k=None, n=None, heads=None) == OK
+
+
+def test_scoring_and_selection_argument_checks(lib):
+    st = lib.misa_score_topk(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, 0, BF16, FAKE, None, None, FAKE,
+                             1 << 30, None)
+    assert st == INVALID  # topk < 1
+    st = lib.misa_score_topk(FAKE, FAKE, FAKE, 0, FAKE, None, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, None, FAKE,
+                             1 << 30, None)
+    assert st == INVALID  # no heads
+    st = lib.misa_score_topk(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, None, FAKE,
+                             16, None)
+    assert st == WORKSPACE
+    st = lib.misa_token_scores(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, BF16, FAKE, 999, None)
+    assert st == INVALID  # ld < L
+    st = lib.misa_topk_select(FAKE, 999, FAKE, 4, 1000, 10, FAKE, None, None, 0, None)
+    assert st == INVALID
+    st = lib.misa_topk_select(FAKE, 1000, FAKE, 4, 1000, 0, FAKE, None, None, 0, None)
+    assert st == INVALID
+    st = lib.misa_hier_rerank(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 100, 200, BF16, FAKE, None, FAKE,
+                              1 << 30, None)
+    assert st == INVALID  # k' < k
+    st = lib.misa_hier_rerank(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 100000, 64, 128, 16385, 200, BF16, FAKE, None, FAKE,
+                              1 << 30, None)
+    assert st == UNSUPPORTED  # k' above the shared-memory limit
+    st = lib.dsa_dense_topk(FAKE, FAKE, FAKE, 0, FAKE, 4, 1000, 64, 128, 10, BF16, FAKE, None, MISALIGNED, 1 << 30,
+                            None)
+    assert st == WORKSPACE
+    st = lib.misa_pool_keys(FAKE, 0, 1, 1000, 64, 64, BF16, FAKE, 0, 0, 16, None)
+    assert st == UNSUPPORTED
+    st = lib.misa_pool_keys(FAKE, 1000, 2, 1000, 128, 64, BF16, FAKE, 16 * 128, 0, 16, None)
+    assert st == INVALID  # caches overlap
+    assert lib.misa_pool_keys(FAKE, 0, 0, 1000, 128, 64, BF16, FAKE, 0, 0, 16, None) == OK
+    assert lib.misa_pool_keys(FAKE, 0, 1, 1000, 128, 64, BF16, FAKE, 0, 16, 16, None) == OK  # empty range
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    from long_context_sparse_mean_b200 import binding
+    with pytest.raises(ValueError):
+        binding.misa_pool_keys(torch.zeros(10, 128, dtype=torch.bfloat16), 4)
