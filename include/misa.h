@@ -169,6 +169,34 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
                            int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
                            void* stream);
 
+/*
+ * Capacity, in floats, of the fixed scratch array used by misa_hier_rerank_static
+ * (4 MiB per GPU that loads the library, held until the process exits).
+ */
+#define MISA_STATIC_RERANK_SCRATCH_FLOATS (1 << 20)
+
+/*
+ * misa_hier_rerank without a workspace argument, for callers that cannot allocate device
+ * memory.  The pages have no counterpart to this call; it exists for the deployment side only.
+ * Who needs it: a plugin that its host framework hands only input and output buffers (the
+ * framework owns the device memory and offers the plugin no allocator), or a latency-critical
+ * decode loop that must not risk an allocation failure, or the device synchronisation that
+ * cudaMalloc / cudaFree can cause, in the middle of a step.
+ * Same arguments, results and checks as misa_hier_rerank, minus ws and ws_bytes.  Its T * kp
+ * floats of scratch live in one array compiled into the library (MISA_STATIC_RERANK_SCRATCH_FLOATS
+ * floats per device); the call allocates nothing.
+ *   - T * kp above MISA_STATIC_RERANK_SCRATCH_FLOATS: returns MISA_ERR_WORKSPACE, nothing launched.
+ *   - All calls on a device share the array and it keeps the last call's contents; nothing in it
+ *     needs to start at zero.  Calls that overlap on the GPU (unordered streams) race on it and
+ *     give undefined results: order them on one stream or with events.
+ *   - The first call on a device looks up the array's device address with that device current
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ */
+misa_status misa_hier_rerank_static(const void* q, const float* w, const void* k,
+                                    int64_t k_seq_stride, const int32_t* n, const int32_t* cand,
+                                    int T, int L, int H_I, int d, int kp, int topk, int dtype,
+                                    int32_t* idx, float* score_opt, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -295,3 +295,31 @@ def misa_indexer(q, w, k, kbar, n, B: int, h: int, topk: int, kp: Optional[int] 
     cand, _ = misa_score_topk(q, w, k, n, heads, kp, want_vals=False, ws=ws, stream=stream)
     idx, vals = misa_hier_rerank(q, w, k, n, cand, topk, ws=ws, stream=stream)
     return {"idx": idx, "vals": vals, "heads": heads, "cand": cand}
+
+
+_lib.misa_hier_rerank_static.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int64] + [ctypes.c_void_p] * 2 + \
+    [ctypes.c_int] * 7 + [ctypes.c_void_p] * 3
+_lib.misa_hier_rerank_static.restype = ctypes.c_int
+STATIC_RERANK_SCRATCH_FLOATS = 1 << 20
+
+
+def misa_hier_rerank_static(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals=True, stream=None):
+    """misa_hier_rerank for callers that cannot allocate device memory: the library's fixed
+    scratch array replaces the workspace (T * k' <= STATIC_RERANK_SCRATCH_FLOATS).  Calls that
+    overlap on the GPU share that array and must be ordered on one stream."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(cand, "cand", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    kp = cand.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    _check("misa_hier_rerank_static", _lib.misa_hier_rerank_static(
+        _p(q), _p(w), _p(k), kss, _p(n), _p(cand), T, L, H_I, d, kp, topk, _dtype_code(q), _p(idx), _p(vals),
+        _stream(stream)))
+    return idx, vals
