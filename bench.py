@@ -40,8 +40,9 @@ UNIT = "query-tokens/s"
 # DRAM traffic of the routed scoring kernel from one ncu capture (dram__bytes_read.sum +
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
-TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu", "sha256": None, "bytes_per_key": None,
-           "capture": None}
+TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
+           "sha256": "4b425ffcef44de6292b97de3aaf2e847b519a18b5d4a943a5c8ed965993f4725",
+           "bytes_per_key": 1.0932e9 / 4194304, "capture": "profiles/score_bf16_decode_L131072_b32.md"}
 
 
 def _sha(path):
