@@ -210,18 +210,28 @@ def run_ours(args):
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     score_ms = []
-    launches_per_step = 8  # pool, 3 router kernels, scores, top-k', re-rank scores, re-rank select
+    # pool, router, scores, 4 top-k' kernels, re-rank scores + 4 selection kernels
+    launches_per_step = 12
 
-    def step(time_scores=False):
+    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+
+    def step(time_scores=False, stages=False):
+        mark = (lambda i: stage_ev[i].record(stream)) if stages else (lambda i: None)
+        mark(0)
         M.misa_pool_keys(kd, B, kbar=kbar, block_begin=M_ - 1, block_end=M_)
+        mark(1)
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
+        mark(2)
         if time_scores:
             ev[0].record(stream)
         M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
         if time_scores:
             ev[1].record(stream)
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False)
+        mark(3)
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=wsp)
+        mark(4)
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
+        mark(5)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -232,6 +242,17 @@ def run_ours(args):
         step(time_scores=True)
         torch.cuda.synchronize()
         score_ms.append(ev[0].elapsed_time(ev[1]))
+
+    # per-stage breakdown (events between the calls; separate untimed steps)
+    stage_names = ["pool_newest_block", "route", "routed_scores", "topk_kprime", "rerank"]
+    stage_acc = [0.0] * len(stage_names)
+    nst = min(args.steps, 20)
+    for _ in range(nst):
+        step(stages=True)
+        torch.cuda.synchronize()
+        for i in range(len(stage_names)):
+            stage_acc[i] += stage_ev[i].elapsed_time(stage_ev[i + 1])
+    stages_us = {nm: round(1000 * a / nst, 2) for nm, a in zip(stage_names, stage_acc)}
 
     # the timed region: K whole steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -321,12 +342,13 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU"}),
-            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_bf16_kernel)",
+            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
                          "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
+            "stages_us": stages_us,
             "clocks": clk.summary(),
             "dense_dsa_same_inputs": None if dsa_ms is None else {
                 "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0)},

@@ -36,8 +36,8 @@
  *   - Prefix lengths n_t are read on the device: values above L count as L, values below 1 give
  *     an empty prefix (no tokens selected; all router scores 0).
  *   - Index outputs hold min(topk, n_t) token indices followed by -1 padding.  The selected set
- *     is what the method defines; misa_score_topk and dsa_dense_topk write it in ascending token
- *     order, misa_hier_rerank in the order of the candidate list.
+ *     is what the method defines (and identical from run to run); the order of the indices
+ *     inside a row is not specified.
  *   - Errors: MISA_ERR_INVALID_ARG (null pointer, size out of range), MISA_ERR_UNSUPPORTED
  *     (d != 128, H_I not a multiple of 8, dtype, k' too large), MISA_ERR_WORKSPACE (workspace
  *     too small or misaligned), MISA_ERR_CUDA (a launch failed; cudaGetLastError's code is
@@ -116,8 +116,8 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
 
 /*
  * Routed-head token scores ("Sparse Token Scoring"): scores[t, s] = I_{t,s} for s < n_t.
- *   heads  : [T, h] routed heads (any order; NULL = all H_I heads, i.e. the dense score F)
- *   scores : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
+ *   heads    : [T, h] routed heads (any order; NULL = all H_I heads, i.e. the dense score F)
+ *   scores   : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -126,9 +126,10 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
 /*
  * Top-k selection over per-query score rows ("Sparse Token Scoring": the final top-k tokens
  * are selected on the reduced scores).  scores [T, ld_scores] fp32, entries s < n_t are read.
- *   idx       : out [T, topk] int32, ascending token order, -1 padded
+ *   idx       : out [T, topk] int32, -1 padded
  *   score_opt : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
- * Scores must be finite.  No workspace is needed (pass NULL, 0).
+ *   ws        : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
+ * Scores must be finite.
  */
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
                              int L, int topk, int32_t* idx, float* score_opt, void* ws,
@@ -137,8 +138,10 @@ misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32
 /*
  * Routed scoring followed by top-k: misa_token_scores then misa_topk_select.  With topk = k'
  * this is the coarse stage of MISA-dagger ("Hierarchical Variant": enlarged candidate set).
- *   scores_full_opt : [T, L] fp32 buffer that receives every score, or NULL to use workspace
- *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK, T, L, ...) bytes (0 if scores_full_opt given)
+ *   scores_full_opt : [T, L] fp32 buffer that receives every score, or NULL (scores then live in
+ *                     the workspace)
+ *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK, T, L, ...) bytes (with scores_full_opt given,
+ *        misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes suffice)
  */
 misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                             const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -149,7 +152,7 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
  * MISA-dagger fine stage ("Hierarchical Variant (MISA-dagger)": the dense indexer with all H_I
  * heads re-scores only the k' candidates and keeps the final top-k).
  *   cand      : [T, kp] candidate token indices; entries < 0 or >= n_t are empty slots
- *   idx       : out [T, topk] the kept candidates (candidate-list order), -1 padded
+ *   idx       : out [T, topk] the kept candidates, -1 padded
  *   score_opt : out [T, topk] their dense scores, or NULL
  *   ws        : misa_workspace_bytes(MISA_OP_RERANK, T, 0, H_I, 0, 0, topk, kp) bytes
  * Requires topk <= kp <= MISA_MAX_KP; duplicate candidates are the caller's error.

@@ -201,7 +201,7 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, stream=None) -> torch.Te
 
 
 def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, vals=None, want_vals=True,
-                     stream=None):
+                     ws: Optional[Workspace] = None, stream=None):
     """Top-k per row of scores [T, ld] over entries s < min(n_t, L) -> (idx [T, k], vals [T, k])."""
     _need(scores, "scores", torch.float32)
     _need(n, "n", torch.int32)
@@ -211,14 +211,16 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
         idx = torch.empty((T, topk), dtype=torch.int32, device=scores.device)
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=scores.device)
+    nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, 8)
+    buf = _ws(ws, scores.device).get(nbytes)
     _check("misa_topk_select", _lib.misa_topk_select(
-        _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), None, 0, _stream(stream)))
+        _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
     return idx, vals
 
 
 def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_full=None, want_vals=True,
                     ws: Optional[Workspace] = None, stream=None):
-    """Routed scoring + top-k -> (idx [T, k] ascending token order, vals [T, k])."""
+    """Routed scoring + top-k -> (idx [T, k], vals [T, k]); the index order is not specified."""
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
@@ -231,7 +233,8 @@ def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_fu
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
-    nbytes = 0 if scores_full is not None else misa_workspace_bytes(OP_SCORE_TOPK, T, L, H_I, 1, h, topk)
+    op = OP_TOPK_SELECT if scores_full is not None else OP_SCORE_TOPK
+    nbytes = misa_workspace_bytes(op, T, L, H_I, 1, h, topk)
     buf = _ws(ws, q.device).get(nbytes)
     _check("misa_score_topk", _lib.misa_score_topk(
         _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, topk, _dtype_code(q), _p(idx), _p(vals),
@@ -264,7 +267,7 @@ def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals
 
 def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, ws: Optional[Workspace] = None,
                    stream=None):
-    """Dense all-head indexer -> (idx [T, k] ascending token order, vals [T, k])."""
+    """Dense all-head indexer -> (idx [T, k], vals [T, k]); the index order is not specified."""
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)

@@ -44,17 +44,28 @@ size_t route_ws(int T, int L, int H_I, int B) {
   if (T <= 0 || L <= 0 || H_I <= 0 || B <= 0) return 0;
   const size_t pm = align_up(sizeof(float) * (size_t)T * misa::kD);
   const size_t part = align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
-  return pm + part;
+  const size_t done = align_up(sizeof(uint32_t) * (size_t)T);
+  return pm + part + done;
 }
 
+size_t scores_part(int T, int L) { return align_up(sizeof(float) * (size_t)T * score_ld(L)); }
+
+// misa_topk_select: histograms, per-row state and boundary pairs of the selection
+size_t select_ws(int T, int P) {
+  if (T <= 0 || P <= 0) return 0;
+  return align_up(misa::topk_rows_ws(T, P));
+}
+
+// misa_score_topk / dsa_dense_topk: [scores][selection]
 size_t scores_ws(int T, int L) {
   if (T <= 0 || L <= 0) return 0;
-  return align_up(sizeof(float) * (size_t)T * score_ld(L));
+  return scores_part(T, L) + select_ws(T, L);
 }
 
+// misa_hier_rerank: [dense scores of the candidates][selection over the candidate lists]
 size_t rerank_ws(int T, int kp) {
   if (T <= 0 || kp <= 0) return 0;
-  return align_up(sizeof(float) * (size_t)T * kp);
+  return align_up(sizeof(float) * (size_t)T * kp) + select_ws(T, kp);
 }
 
 }  // namespace
@@ -92,6 +103,7 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
     case MISA_OP_RERANK:
       return rerank_ws(T, kp);
     case MISA_OP_TOPK_SELECT:
+      return select_ws(T, L);
     default:
       return 0;
   }
@@ -123,10 +135,14 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
   if (!kbar || !heads) return MISA_ERR_INVALID_ARG;
   const size_t need = route_ws(T, L, H_I, B);
   if (!ws || ws_bytes < need || !aligned(ws)) return MISA_ERR_WORKSPACE;
-  float* pm = static_cast<float*>(ws);
-  float* partial = reinterpret_cast<float*>(static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * misa::kD));
+  char* p = static_cast<char*>(ws);
+  float* pm = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * misa::kD);
+  float* partial = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
+  uint32_t* done = reinterpret_cast<uint32_t*>(p);
   misa::launch_route(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, T, L, H_I, B, h, heads,
-                     r_opt, pm, partial, as_stream(stream));
+                     r_opt, pm, partial, done, as_stream(stream));
   return launch_status();
 }
 
@@ -146,12 +162,11 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
 
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T, int L, int topk,
                              int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   if (T < 0 || L < 1 || topk < 1 || ld_scores < L) return MISA_ERR_INVALID_ARG;
   if (T == 0) return MISA_OK;
   if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
-  misa::launch_topk_rows(scores, ld_scores, n, T, L, topk, idx, score_opt, as_stream(stream));
+  if (!ws || ws_bytes < select_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -165,16 +180,19 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
   if (h < 1 || h > H_I || topk < 1) return MISA_ERR_INVALID_ARG;
   if (T == 0) return MISA_OK;
   if (!idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < (scores_full_opt ? select_ws(T, L) : scores_ws(T, L)) || !aligned(ws))
+    return MISA_ERR_WORKSPACE;
+  char* p = static_cast<char*>(ws);
   float* buf = scores_full_opt;
   int64_t ld = L;
   if (!buf) {
-    if (!ws || ws_bytes < scores_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
-    buf = static_cast<float*>(ws);
+    buf = reinterpret_cast<float*>(p);
     ld = score_ld(L);
+    p += scores_part(T, L);
   }
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld,
                       as_stream(stream));
-  misa::launch_topk_rows(buf, ld, n, T, L, topk, idx, score_opt, as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -189,9 +207,10 @@ misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64
   if (!cand || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   float* F = static_cast<float*>(ws);
+  void* sel = static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * kp);
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp,
                       as_stream(stream));
-  misa::launch_topk_cand(F, cand, n, T, L, kp, topk, idx, score_opt, as_stream(stream));
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -204,11 +223,13 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   if (T == 0) return MISA_OK;
   if (!idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < scores_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
-  float* buf = static_cast<float*>(ws);
+  char* p = static_cast<char*>(ws);
+  float* buf = reinterpret_cast<float*>(p);
   const int64_t ld = score_ld(L);
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
                       as_stream(stream));
-  misa::launch_topk_rows(buf, ld, n, T, L, topk, idx, score_opt, as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p + scores_part(T, L), idx, score_opt,
+                         as_stream(stream));
   return launch_status();
 }
 

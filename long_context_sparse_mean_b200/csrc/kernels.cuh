@@ -17,7 +17,7 @@ int route_chunks(int L, int B);  // chunks of kRouteTile blocks per query (upper
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
                   int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
-                  cudaStream_t s);
+                  uint32_t* done, cudaStream_t s);
 
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
 // position p of query t scores token rows[t*P + p] and writes out[t*ld + p].
@@ -25,11 +25,14 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
                    const int32_t* rows, int P, float* out, int64_t ld, cudaStream_t s);
 
-// Top-k of each score row (entries s < n_t), output in ascending token order.
-void launch_topk_rows(const float* scores, int64_t ld, const int32_t* n, int T, int L, int topk,
-                      int32_t* idx, float* score_opt, cudaStream_t s);
+// Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
+// or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t)).  ws holds
+// topk_rows_ws(T, P or L) bytes, 256-byte aligned.  Output order within a row is not specified.
+size_t topk_rows_ws(int T, int P);
+void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
+                      int L, int topk, void* ws, int32_t* idx, float* score_opt, cudaStream_t s);
 
-// Top-k of candidate lists: values F[t, P], ids cand[t, P] (ids outside [0, n_t) are empty).
+// Top-k of short candidate lists in shared memory (no workspace): values F[t, P], ids cand[t, P].
 size_t topk_cand_smem(int P);
 void launch_topk_cand(const float* F, const int32_t* cand, const int32_t* n, int T, int L, int P,
                       int topk, int32_t* idx, float* score_opt, cudaStream_t s);

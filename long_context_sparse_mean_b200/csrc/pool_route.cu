@@ -7,11 +7,13 @@
 // heads are routed.  Aggregation used here: r_{t,j} = w_{t,j} * sum_b max(0, q_{t,j} . kbar_b).
 //
 // Data layout: keys [L, 128] (bf16 or fp32) per cache, pooled keys kbar [M, 128] fp32 per cache.
-// Work split for the router: one CTA per (query, tile of 64 blocks); the CTA holds the query's
-// H_I head vectors and the 64 pooled keys transposed in shared memory and every thread owns a
-// 4-head x 4-block register tile, so each pair of float4 shared loads feeds 16 FMAs.  Partial
-// sums per tile go to workspace and a one-warp-per-query kernel adds them in a fixed order
-// (deterministic), applies w and picks the top-h heads with warp shuffles.
+// bf16 queries: one kernel.  One CTA per (query, tile of 128 pooled blocks) multiplies the tile
+// with the query's H_I head vectors on the tensor cores (see route_affinity_mma_kernel); the CTA
+// whose tile holds a partial last block averages that block's keys itself; per-tile sums go to
+// workspace and the query's last tile to finish adds them in tile order (deterministic), applies
+// w and picks the top-h heads with warp shuffles.
+// fp32 queries: CUDA cores, one CTA per (query, tile of 64 blocks) with a 4-head x 4-block
+// register tile per thread, then a one-warp-per-query selection kernel.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
@@ -156,14 +158,11 @@ __device__ __forceinline__ bool head_better(float av, int aj, float bv, int bj) 
   return av > bv || (av == bv && aj < bj);
 }
 
-// One warp per query: r_j = w_j * sum over tiles; top-h heads by (r desc, j asc).
-__global__ void __launch_bounds__(32) route_select_kernel(const float* partial, const float* w,
-                                                          const int32_t* n, int L, int H_I, int B,
-                                                          int nch, int h, int32_t* heads, float* r_opt) {
-  const int t = blockIdx.x, lane = threadIdx.x;
-  const int nt = clamp_len(n[t], L);
-  const int Mt = (nt + B - 1) / B;
-  const int nc = (Mt + kRouteTile - 1) / kRouteTile;
+// One warp: r_j = w_j * (sum of the nc per-tile partial sums, in tile order), then the top-h heads
+// by (r desc, j asc) with warp shuffles.  partial_t is [nch][H_I] for this query.
+__device__ __forceinline__ void select_heads_warp(const float* partial_t, int nc, const float* w_t, int H_I, int h,
+                                                  int32_t* heads_t, float* r_t) {
+  const int lane = threadIdx.x & 31;
   float v[kMaxHeads / 32];
   bool live[kMaxHeads / 32];
 #pragma unroll
@@ -173,9 +172,9 @@ __global__ void __launch_bounds__(32) route_select_kernel(const float* partial, 
     v[i] = 0.f;
     if (live[i]) {
       float s = 0.f;
-      for (int c = 0; c < nc; ++c) s += partial[((int64_t)t * nch + c) * H_I + j];
-      v[i] = w[(int64_t)t * H_I + j] * s;
-      if (r_opt) r_opt[(int64_t)t * H_I + j] = v[i];
+      for (int c = 0; c < nc; ++c) s += __ldcg(partial_t + (int64_t)c * H_I + j);
+      v[i] = w_t[j] * s;
+      if (r_t) r_t[j] = v[i];
     }
   }
   for (int rnd = 0; rnd < h; ++rnd) {
@@ -200,10 +199,159 @@ __global__ void __launch_bounds__(32) route_select_kernel(const float* partial, 
         bj = oj;
       }
     }
-    if (lane == 0) heads[(int64_t)t * h + rnd] = bj;
+    if (lane == 0) heads_t[rnd] = bj;
 #pragma unroll
     for (int i = 0; i < kMaxHeads / 32; ++i)
       if (lane + 32 * i == bj) live[i] = false;
+  }
+}
+
+// One warp per query (fp32 path).
+__global__ void __launch_bounds__(32) route_select_kernel(const float* partial, const float* w,
+                                                          const int32_t* n, int L, int H_I, int B,
+                                                          int nch, int tile, int h, int32_t* heads,
+                                                          float* r_opt) {
+  const int t = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  const int Mt = (nt + B - 1) / B;
+  select_heads_warp(partial + (int64_t)t * nch * H_I, (Mt + tile - 1) / tile, w + (int64_t)t * H_I, H_I, h,
+                    heads + (int64_t)t * h, r_opt ? r_opt + (int64_t)t * H_I : nullptr);
+}
+
+constexpr int kRouteMmaTile = 128;  // pooled blocks per CTA of the tensor-core router (8 warps x 16)
+
+__device__ __forceinline__ void mma_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// x = hi + mid + lo exactly up to the last ~24 bits: each part is the bf16 rounding of what the
+// previous parts leave (the subtractions are exact in fp32).
+__device__ __forceinline__ void split3(float x, float& hi, float& mid, float& lo) {
+  hi = __bfloat162float(__float2bfloat16_rn(x));
+  const float r1 = x - hi;
+  mid = __bfloat162float(__float2bfloat16_rn(r1));
+  lo = r1 - mid;
+}
+
+// Tensor-core router for bf16 queries.  Per (query, tile of 128 pooled blocks): the GEMM
+// kbar[128 blocks, 128] x q^T[128, H_I] on mma.m16n8k16.  bf16 q is exact; each fp32 pooled key is
+// split into three bf16 parts and the three products are accumulated in fp32, which keeps the
+// dot products at fp32 accuracy.  The pooled keys are loaded straight into A fragments (lane
+// (g, c) of a warp holds dims 16kk + 4c .. +3 of blocks g and g+8 at k-step kk, and the q
+// fragments staged in shared memory use the same dimension order).  Epilogue: relu, sum over the
+// tile's blocks per head (quad shuffles, then a fixed-order sum over the 8 warps).
+template <int NG>
+__global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bfloat16* __restrict__ q,
+                                                                 const float* __restrict__ w,
+                                                                 const __nv_bfloat16* __restrict__ k,
+                                                                 int64_t k_seq_stride,
+                                                                 const float* __restrict__ kbar,
+                                                                 int64_t kbar_seq_stride,
+                                                                 const int32_t* __restrict__ n, int L, int B, int h,
+                                                                 int nch, float* __restrict__ partial,
+                                                                 uint32_t* __restrict__ done,
+                                                                 int32_t* __restrict__ heads, float* __restrict__ r_opt) {
+  constexpr int H = NG * 8;
+  __shared__ uint2 frag[NG][8][32];
+  __shared__ float wsum[8][H];
+  __shared__ float part[4][kD];
+  __shared__ __align__(16) float pms[kD];  // mean of the partial last block
+  __shared__ int last;
+  const int t = blockIdx.y, c0 = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  const int nfull = nt / B, Mt = (nt + B - 1) / B;
+  const int nc = (Mt + kRouteMmaTile - 1) / kRouteMmaTile;
+  const int bb = c0 * kRouteMmaTile;
+  if (bb >= Mt) {
+    if (Mt == 0 && c0 == 0 && threadIdx.x < 32)  // empty prefix: every router score is 0
+      select_heads_warp(partial, 0, w + (int64_t)t * H, H, h, heads + (int64_t)t * h,
+                        r_opt ? r_opt + (int64_t)t * H : nullptr);
+    return;
+  }
+  if (nfull < Mt && nfull >= bb && nfull < bb + kRouteMmaTile) {  // this tile holds the partial block
+    const float m = block_mean_256<DType::BF16>(k + (int64_t)t * k_seq_stride, nfull * B, nt, part);
+    if (threadIdx.x < kD) pms[threadIdx.x] = m;
+  }
+  for (int e = threadIdx.x; e < NG * 8 * 32; e += blockDim.x) {
+    const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
+    const int g = ln >> 2, c = ln & 3;
+    const __nv_bfloat16* src = q + ((int64_t)t * H + ng * 8 + g) * kD + 16 * kk + 4 * c;
+    frag[ng][kk][ln] = *reinterpret_cast<const uint2*>(src);
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const int ba = bb + warp * 16 + g, bq = ba + 8;
+  const float* kb = kbar + (int64_t)t * kbar_seq_stride;
+  const float* rowa = ba < nfull ? kb + (int64_t)ba * kD : (ba < Mt ? pms : nullptr);
+  const float* rowb = bq < nfull ? kb + (int64_t)bq * kD : (bq < Mt ? pms : nullptr);
+  float acc[NG][4];
+#pragma unroll
+  for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.f;
+#pragma unroll 2
+  for (int kk = 0; kk < 8; ++kk) {
+    const float4 xa = rowa ? *reinterpret_cast<const float4*>(rowa + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
+    const float4 xb = rowb ? *reinterpret_cast<const float4*>(rowb + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
+    float ah[4], am[4], al[4], bh[4], bm[4], bl[4];
+    split3(xa.x, ah[0], am[0], al[0]);
+    split3(xa.y, ah[1], am[1], al[1]);
+    split3(xa.z, ah[2], am[2], al[2]);
+    split3(xa.w, ah[3], am[3], al[3]);
+    split3(xb.x, bh[0], bm[0], bl[0]);
+    split3(xb.y, bh[1], bm[1], bl[1]);
+    split3(xb.z, bh[2], bm[2], bl[2]);
+    split3(xb.w, bh[3], bm[3], bl[3]);
+    const uint32_t A[3][4] = {
+        {pack_bf16x2(ah[0], ah[1]), pack_bf16x2(bh[0], bh[1]), pack_bf16x2(ah[2], ah[3]), pack_bf16x2(bh[2], bh[3])},
+        {pack_bf16x2(am[0], am[1]), pack_bf16x2(bm[0], bm[1]), pack_bf16x2(am[2], am[3]), pack_bf16x2(bm[2], bm[3])},
+        {pack_bf16x2(al[0], al[1]), pack_bf16x2(bl[0], bl[1]), pack_bf16x2(al[2], al[3]), pack_bf16x2(bl[2], bl[3])}};
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      const uint2 bf = frag[ng][kk][lane];
+#pragma unroll
+      for (int p = 0; p < 3; ++p) mma_16816(acc[ng], A[p][0], A[p][1], A[p][2], A[p][3], bf.x, bf.y);
+    }
+  }
+  const bool va = ba < Mt, vb = bq < Mt;
+#pragma unroll
+  for (int ng = 0; ng < NG; ++ng) {
+    float h0 = (va ? relu(acc[ng][0]) : 0.f) + (vb ? relu(acc[ng][2]) : 0.f);
+    float h1 = (va ? relu(acc[ng][1]) : 0.f) + (vb ? relu(acc[ng][3]) : 0.f);
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      h0 += __shfl_xor_sync(0xffffffffu, h0, o);
+      h1 += __shfl_xor_sync(0xffffffffu, h1, o);
+    }
+    if (g == 0) {
+      wsum[warp][ng * 8 + 2 * c] = h0;
+      wsum[warp][ng * 8 + 2 * c + 1] = h1;
+    }
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < H; j += blockDim.x) {
+    float s = 0.f;
+#pragma unroll
+    for (int w8 = 0; w8 < 8; ++w8) s += wsum[w8][j];
+    partial[((int64_t)t * nch + c0) * H + j] = s;
+  }
+  // the query's last tile to finish sums the tiles in order and picks the heads
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(done + t, 1u) == (uint32_t)(nc - 1);
+  __syncthreads();
+  if (last && threadIdx.x < 32) {
+    __threadfence();
+    select_heads_warp(partial + (int64_t)t * nch * H, nc, w + (int64_t)t * H, H, h, heads + (int64_t)t * h,
+                      r_opt ? r_opt + (int64_t)t * H : nullptr);
   }
 }
 
@@ -226,24 +374,52 @@ int route_chunks(int L, int B) {
 
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L, int H_I,
-                  int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial, cudaStream_t s) {
+                  int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial, uint32_t* done,
+                  cudaStream_t s) {
   if (T <= 0) return;
-  const int nch = route_chunks(L, B);
-  const size_t smem = sizeof(float) * (size_t)kD * ((H_I + 4) + (kRouteTile + 4));
+  const int M = (L + B - 1) / B;
   if (dt == DType::BF16) {
-    partial_mean_kernel<DType::BF16><<<T, 256, 0, s>>>(k, k_seq_stride, n, L, B, pm);
-    cudaFuncSetAttribute(route_affinity_kernel<DType::BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    route_affinity_kernel<DType::BF16><<<dim3(nch, T), 4 * H_I, smem, s>>>(q, kbar, kbar_seq_stride, pm, n, L,
-                                                                            H_I, B, nch, partial);
+    const int nch = (M + kRouteMmaTile - 1) / kRouteMmaTile;
+    const dim3 grid(nch, T);
+    cudaMemsetAsync(done, 0, sizeof(uint32_t) * (size_t)T, s);
+    auto qb = static_cast<const __nv_bfloat16*>(q);
+    auto kb = static_cast<const __nv_bfloat16*>(k);
+    switch (H_I / 8) {
+#define MISA_ROUTE_CASE(NGV)                                                                                  \
+  case NGV:                                                                                                   \
+    route_affinity_mma_kernel<NGV><<<grid, 256, 0, s>>>(qb, w, kb, k_seq_stride, kbar, kbar_seq_stride, n, L, B, h, \
+                                                        nch, partial, done, heads, r_opt);                    \
+    break;
+      MISA_ROUTE_CASE(1)
+      MISA_ROUTE_CASE(2)
+      MISA_ROUTE_CASE(3)
+      MISA_ROUTE_CASE(4)
+      MISA_ROUTE_CASE(5)
+      MISA_ROUTE_CASE(6)
+      MISA_ROUTE_CASE(7)
+      MISA_ROUTE_CASE(8)
+      MISA_ROUTE_CASE(9)
+      MISA_ROUTE_CASE(10)
+      MISA_ROUTE_CASE(11)
+      MISA_ROUTE_CASE(12)
+      MISA_ROUTE_CASE(13)
+      MISA_ROUTE_CASE(14)
+      MISA_ROUTE_CASE(15)
+      MISA_ROUTE_CASE(16)
+#undef MISA_ROUTE_CASE
+      default:
+        break;
+    }
   } else {
+    const int nch = route_chunks(L, B);
+    const size_t smem = sizeof(float) * (size_t)kD * ((H_I + 4) + (kRouteTile + 4));
     partial_mean_kernel<DType::F32><<<T, 256, 0, s>>>(k, k_seq_stride, n, L, B, pm);
     cudaFuncSetAttribute(route_affinity_kernel<DType::F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     route_affinity_kernel<DType::F32><<<dim3(nch, T), 4 * H_I, smem, s>>>(q, kbar, kbar_seq_stride, pm, n, L,
                                                                            H_I, B, nch, partial);
+    route_select_kernel<<<T, 32, 0, s>>>(partial, w, n, L, H_I, B, nch, kRouteTile, h, heads, r_opt);
   }
-  route_select_kernel<<<T, 32, 0, s>>>(partial, w, n, L, H_I, B, nch, h, heads, r_opt);
 }
 
 }  // namespace misa

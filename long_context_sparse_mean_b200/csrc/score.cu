@@ -7,47 +7,41 @@
 //
 // bf16 path.  Per key the work is h x 128 multiply-adds against 256 bytes read, so with h = 8 a
 // CUDA-core dot product would spend more issue slots on FMAs and shuffles than HBM allows; the
-// contraction K[rows,128] x Q[128, heads] instead runs on the tensor cores with
-// mma.m16n8k16 (bf16 in, fp32 accumulate).  Key rows are loaded straight from global memory
-// into the A-fragment registers: the dot product is invariant under any permutation of the 128
-// dimensions applied to both operands, so lane (g, c) of a warp loads the 16-byte chunks
-// c, c+4, c+8, c+12 of rows g and g+8 (every load instruction of the warp reads 8 rows x 64
-// contiguous bytes, all of each 32-byte sector used) and the query fragments staged in shared
-// memory use the same dimension order.  No shared-memory round trip for K, no ldmatrix.  The
-// epilogue applies relu, weights and sums the heads of a row inside the thread and over the 4
-// lanes of a quad, and writes one fp32 score per key.
+// contraction runs on the tensor cores instead (mma_frag.cuh: key rows go from global memory
+// straight into A fragments).  Heads are summed in ascending head index (the routed list is
+// sorted, padded to a multiple of 8 with zero-weight slots), so the routed score with h = H_I is
+// the dense score bit for bit.
 //
-// Heads are summed in ascending head index (the routed list is sorted first, padded to a
-// multiple of 8 with zero-weight slots), so the routed score with h = H_I is the dense score bit
-// for bit.  -0 is normalised to +0.
-//
-// fp32 path (q and k in fp32): one warp per key row on CUDA cores, exact fp32 products.
+// Three kernels:
+//   score_persist_kernel  decode (one cache per query): persistent, 2 CTAs per SM; the actual
+//       work (ceil(n_t/128) tiles of 128 rows per query) is flattened and split evenly over the
+//       CTAs, each taking one contiguous range.  Each warp owns 16 rows of every tile and holds
+//       the next tile in registers while the current one is multiplied.  (Measured on B200 with
+//       32 x 131072 keys: 178 us against 185 us for the grid kernel; an added bulk L2 prefetch
+//       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
+//       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
+//   score_grid_kernel     shared caches (prefill): one CTA per (query, chunk of positions).
+//   score_f32_kernel      fp32 inputs: one warp per key row on CUDA cores, exact fp32 products.
+// The top-k selection histograms the written scores in passes of its own (topk.cu): counting
+// inside these kernels cost 12-16 us per 32 x 131072 scores, more than a separate pass over the
+// L2-resident scores.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"
+#include "mma_frag.cuh"
 
 namespace misa {
 
 namespace {
 
 constexpr int kScoreThreads = 256;   // 8 warps
-constexpr int kRowsPerChunk = 1024;  // positions per CTA
+constexpr int kRowsPerChunk = 1024;  // positions per CTA of the grid kernel
+constexpr int kGatherRowsPerChunk = 256;
+constexpr int kTileRows = 128;       // persistent kernel: 8 warps x 16 rows
+constexpr int kMaxPersistQueries = 8192;
 
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2,
-                                               uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};\n"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint4 ldg_row_chunk(const __nv_bfloat16* row, int chunk) {
-  return __ldg(reinterpret_cast<const uint4*>(row) + chunk);
-}
-
-// Shared staging of one query's head list: ascending head ids (padded), weights and, for the
-// bf16 path, the B fragments in fragment order.
+// Shared staging of one query's head list: ascending head ids (padded), weights and the B
+// fragments in fragment order.
 template <int NG>
 struct HeadStage {
   uint2 frag[NG][8][32];
@@ -77,32 +71,129 @@ __device__ __forceinline__ void stage_head_list(const int32_t* heads, int h, int
   }
 }
 
+template <int NG>
+__device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat16* q, const float* w,
+                                            const int32_t* heads, int h, int H_I, int t) {
+  stage_head_list(heads, h, H_I, t, NG * 8, st.hl, &st.m);
+  __syncthreads();
+  if (threadIdx.x < NG * 8)
+    st.wsel[threadIdx.x] = (int)threadIdx.x < st.m ? w[(int64_t)t * H_I + st.hl[threadIdx.x]] : 0.f;
+  stage_q_frags<NG>(st.frag, q + (int64_t)t * H_I * kD, st.hl);
+  __syncthreads();
+}
+
 template <int NG, bool GATHER>
 __global__ void __launch_bounds__(kScoreThreads, 2)
-    score_bf16_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+    score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                         const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
+                         const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
+                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld) {
+  extern __shared__ int tile_base[];  // flattened tile prefix [T + 1]
+  __shared__ HeadStage<NG> st;
+  __shared__ uint32_t wtot[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+
+  const int per = (T + kScoreThreads - 1) / kScoreThreads;
+  const int q0 = min((int)threadIdx.x * per, T), q1 = min(q0 + per, T);
+  uint32_t mine = 0;
+  for (int t = q0; t < q1; ++t) mine += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
+  uint32_t total;
+  uint32_t run = block_exclusive_scan(mine, wtot, &total);
+  for (int t = q0; t < q1; ++t) {
+    tile_base[t] = (int)run;
+    run += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
+  }
+  if (threadIdx.x == 0) tile_base[T] = (int)total;
+  __syncthreads();
+  const int64_t tb = (int64_t)blockIdx.x * total / gridDim.x;
+  const int64_t te = (int64_t)(blockIdx.x + 1) * total / gridDim.x;
+
+  int64_t pos = tb;
+  while (pos < te) {
+    int lo = 0, hi = T - 1;  // last query whose first tile is at or before pos
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (tile_base[mid] <= pos) lo = mid;
+      else hi = mid - 1;
+    }
+    const int t = lo;
+    const int64_t seg_end = min(te, (int64_t)tile_base[t + 1]);
+    const int first = (int)(pos - tile_base[t]);
+    const int ntile = (int)(seg_end - pos);
+    const int nt = clamp_len(n[t], L);
+    const int npos = GATHER ? P : nt;
+    const int32_t* rt = GATHER ? rows + (int64_t)t * P : nullptr;
+
+    __syncthreads();  // the previous segment's fragments are no longer read
+    stage_query<NG>(st, q, w, heads, h, H_I, t);
+    float wa[NG], wb[NG];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      wa[ng] = st.wsel[ng * 8 + 2 * c];
+      wb[ng] = st.wsel[ng * 8 + 2 * c + 1];
+    }
+    const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
+    float* ot = out + (int64_t)t * ld;
+    auto row_of = [&](int j) { return (first + j) * kTileRows + warp * 16; };
+    // position p -> key row: p itself, or rows[t, p] when gathering (outside [0, n_t): empty).
+    // Gathered row ids are fetched two tiles ahead, so a tile's row loads never wait for its ids.
+    auto raw_id = [&](int p) -> int { return p < npos ? (GATHER ? __ldg(rt + p) : p) : -1; };
+    auto valid_row = [&](int r) -> int { return (r >= 0 && r < nt) ? r : -1; };
+    int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
+    int nia = GATHER && ntile > 1 ? raw_id(row_of(1) + g) : -1;
+    int nib = GATHER && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
+    auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4]) {
+      ra = valid_row(ra);
+      rb = valid_row(rb);
+      load_rows(ra >= 0 ? kt + (int64_t)ra * kD : nullptr, rb >= 0 ? kt + (int64_t)rb * kD : nullptr, c, A, B);
+    };
+    uint4 RA[4], RB[4];
+    load_ids(ida, idb, RA, RB);
+    for (int j = 0; j < ntile; ++j) {
+      uint4 NA[4], NB[4];
+      if (j + 1 < ntile) {
+        int ra, rb;
+        if (GATHER) {
+          ra = nia;
+          rb = nib;
+          nia = j + 2 < ntile ? raw_id(row_of(j + 2) + g) : -1;
+          nib = j + 2 < ntile ? raw_id(row_of(j + 2) + g + 8) : -1;
+        } else {
+          ra = raw_id(row_of(j + 1) + g);
+          rb = raw_id(row_of(j + 1) + g + 8);
+        }
+        load_ids(ra, rb, NA, NB);
+      }
+      float slo, shi;
+      score_rows<NG>(RA, RB, st.frag, wa, wb, lane, slo, shi);
+      const int r = row_of(j) + g;
+      if (c == 0 && r < npos) ot[r] = slo;
+      if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        RA[i] = NA[i];
+        RB[i] = NB[i];
+      }
+    }
+    pos = seg_end;
+  }
+}
+
+template <int NG, bool GATHER>
+__global__ void __launch_bounds__(kScoreThreads, 2)
+    score_grid_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                       const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                       const int32_t* __restrict__ heads, int h, int H_I, int L,
                       const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld) {
+  constexpr int kChunk = GATHER ? kGatherRowsPerChunk : kRowsPerChunk;
   __shared__ HeadStage<NG> st;
   const int t = blockIdx.y;
   const int nt = clamp_len(n[t], L);
   const int npos = GATHER ? P : nt;
-  const int p0 = blockIdx.x * kRowsPerChunk;
+  const int p0 = blockIdx.x * kChunk;
   if (p0 >= npos) return;
-  const int p1 = min(p0 + kRowsPerChunk, npos);
-
-  stage_head_list(heads, h, H_I, t, NG * 8, st.hl, &st.m);
-  __syncthreads();
-  if (threadIdx.x < NG * 8)
-    st.wsel[threadIdx.x] = threadIdx.x < st.m ? w[(int64_t)t * H_I + st.hl[threadIdx.x]] : 0.f;
-  for (int e = threadIdx.x; e < NG * 8 * 32; e += kScoreThreads) {
-    const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
-    const int g = ln >> 2, c = ln & 3;
-    const int base = 32 * (kk >> 1) + 8 * c + 4 * (kk & 1);
-    const __nv_bfloat16* src = q + ((int64_t)t * H_I + st.hl[ng * 8 + g]) * kD + base;
-    st.frag[ng][kk][ln] = *reinterpret_cast<const uint2*>(src);
-  }
-  __syncthreads();
+  const int p1 = min(p0 + kChunk, npos);
+  stage_query<NG>(st, q, w, heads, h, H_I, t);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
@@ -127,49 +218,20 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       va = va && sa >= 0 && sa < nt;
       vb = vb && sb >= 0 && sb < nt;
     }
-    const __nv_bfloat16* ra = kt + (int64_t)(va ? sa : 0) * kD;
-    const __nv_bfloat16* rb = kt + (int64_t)(vb ? sb : 0) * kD;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      RA[i] = va ? ldg_row_chunk(ra, 4 * i + c) : make_uint4(0, 0, 0, 0);
-      RB[i] = vb ? ldg_row_chunk(rb, 4 * i + c) : make_uint4(0, 0, 0, 0);
-    }
+    load_rows(va ? kt + (int64_t)sa * kD : nullptr, vb ? kt + (int64_t)sb * kD : nullptr, c, RA, RB);
   };
 
   int r0 = p0 + warp * 16;
   uint4 RA[4], RB[4];
-  bool va, vb;
+  bool va = false, vb = false;
   if (r0 < p1) load(r0, RA, RB, va, vb);
   for (; r0 < p1; r0 += 8 * 16) {
     uint4 NA[4], NB[4];
     bool na = false, nb = false;
     const int rn = r0 + 8 * 16;
     if (rn < p1) load(rn, NA, NB, na, nb);
-
-    float slo = 0.f, shi = 0.f;
-#pragma unroll
-    for (int ng = 0; ng < NG; ++ng) {
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        const uint4 xa = RA[kk >> 1], xb = RB[kk >> 1];
-        const uint2 bf = st.frag[ng][kk][lane];
-        if (kk & 1)
-          mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, bf.x, bf.y);
-        else
-          mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, bf.x, bf.y);
-      }
-      slo = fmaf(wa[ng], relu(acc[0]), slo);
-      slo = fmaf(wb[ng], relu(acc[1]), slo);
-      shi = fmaf(wa[ng], relu(acc[2]), shi);
-      shi = fmaf(wb[ng], relu(acc[3]), shi);
-    }
-    slo += __shfl_xor_sync(0xffffffffu, slo, 1);
-    shi += __shfl_xor_sync(0xffffffffu, shi, 1);
-    slo += __shfl_xor_sync(0xffffffffu, slo, 2);
-    shi += __shfl_xor_sync(0xffffffffu, shi, 2);
-    slo = __fadd_rn(slo, 0.0f);
-    shi = __fadd_rn(shi, 0.0f);
+    float slo, shi;
+    score_rows<NG>(RA, RB, st.frag, wa, wb, lane, slo, shi);
     if (c == 0 && va) ot[r0 + g] = slo;
     if (c == 1 && vb) ot[r0 + g + 8] = shi;
 #pragma unroll
@@ -202,7 +264,7 @@ __global__ void __launch_bounds__(kScoreThreads)
   stage_head_list(heads, h, H_I, t, heads ? h : H_I, hl, &m_sh);
   __syncthreads();
   const int m = m_sh;
-  if (threadIdx.x < m) wsel[threadIdx.x] = w[(int64_t)t * H_I + hl[threadIdx.x]];
+  if ((int)threadIdx.x < m) wsel[threadIdx.x] = w[(int64_t)t * H_I + hl[threadIdx.x]];
   for (int e = threadIdx.x; e < m * kD; e += kScoreThreads)
     qs[e] = q[((int64_t)t * H_I + hl[e / kD]) * kD + (e % kD)];
   __syncthreads();
@@ -232,18 +294,43 @@ __global__ void __launch_bounds__(kScoreThreads)
   }
 }
 
+int num_sms() {
+  static int sms = 0;
+  if (sms == 0) {
+    int dev = 0, v = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev);
+    sms = v > 0 ? v : 148;
+  }
+  return sms;
+}
+
 template <int NG>
-void launch_bf16(bool gather, dim3 grid, cudaStream_t s, const void* q, const float* w, const void* k,
-                 int64_t k_seq_stride, const int32_t* n, const int32_t* heads, int h, int H_I, int L,
+void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const float* w, const void* k,
+                 int64_t k_seq_stride, const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L,
                  const int32_t* rows, int P, float* out, int64_t ld) {
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
-  if (gather)
-    score_bf16_kernel<NG, true><<<grid, kScoreThreads, 0, s>>>(qb, w, kb, k_seq_stride, n, heads, h, H_I, L, rows,
-                                                               P, out, ld);
-  else
-    score_bf16_kernel<NG, false><<<grid, kScoreThreads, 0, s>>>(qb, w, kb, k_seq_stride, n, heads, h, H_I, L,
-                                                                rows, P, out, ld);
+  if (persist) {
+    const size_t smem = sizeof(int) * (size_t)(T + 1);
+    if (gather) {
+      cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(qb, w, kb, k_seq_stride, n, heads, h,
+                                                                                H_I, L, T, rows, P, out, ld);
+    } else {
+      cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(qb, w, kb, k_seq_stride, n, heads,
+                                                                                 h, H_I, L, T, rows, P, out, ld);
+    }
+  } else if (gather) {
+    const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
+    score_grid_kernel<NG, true><<<grid, kScoreThreads, 0, s>>>(qb, w, kb, k_seq_stride, n, heads, h, H_I, L, rows, P,
+                                                               out, ld);
+  } else {
+    const dim3 grid((L + kRowsPerChunk - 1) / kRowsPerChunk, T);
+    score_grid_kernel<NG, false><<<grid, kScoreThreads, 0, s>>>(qb, w, kb, k_seq_stride, n, heads, h, H_I, L, rows,
+                                                                P, out, ld);
+  }
 }
 
 }  // namespace
@@ -254,9 +341,9 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
   if (T <= 0) return;
   const int npos = rows ? P : L;
   if (npos <= 0) return;
-  dim3 grid((npos + kRowsPerChunk - 1) / kRowsPerChunk, T);
   const bool gather = rows != nullptr;
   if (dt == DType::F32) {
+    const dim3 grid((npos + kRowsPerChunk - 1) / kRowsPerChunk, T);
     const int m = heads ? h : H_I;
     const size_t smem = sizeof(float) * (size_t)m * kD;
     if (gather) {
@@ -270,34 +357,36 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
           static_cast<const float*>(q), w, static_cast<const float*>(k), k_seq_stride, n, heads, h, H_I, L, rows,
           P, out, ld);
     }
-    return;
-  }
-  const int m = heads ? h : H_I;
-  const int ng = (m + 7) / 8;
-  switch (ng) {
-#define MISA_NG_CASE(NGV) \
-  case NGV:               \
-    launch_bf16<NGV>(gather, grid, s, q, w, k, k_seq_stride, n, heads, h, H_I, L, rows, P, out, ld); \
+  } else {
+    const int m = heads ? h : H_I;
+    const int ng = (m + 7) / 8;
+    // persistent schedule for per-query caches and for gathered candidate lists
+    const bool persist = (gather || k_seq_stride != 0) && T <= kMaxPersistQueries;
+    switch (ng) {
+#define MISA_NG_CASE(NGV)                                                                                  \
+  case NGV:                                                                                                \
+    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld); \
     break;
-    MISA_NG_CASE(1)
-    MISA_NG_CASE(2)
-    MISA_NG_CASE(3)
-    MISA_NG_CASE(4)
-    MISA_NG_CASE(5)
-    MISA_NG_CASE(6)
-    MISA_NG_CASE(7)
-    MISA_NG_CASE(8)
-    MISA_NG_CASE(9)
-    MISA_NG_CASE(10)
-    MISA_NG_CASE(11)
-    MISA_NG_CASE(12)
-    MISA_NG_CASE(13)
-    MISA_NG_CASE(14)
-    MISA_NG_CASE(15)
-    MISA_NG_CASE(16)
+      MISA_NG_CASE(1)
+      MISA_NG_CASE(2)
+      MISA_NG_CASE(3)
+      MISA_NG_CASE(4)
+      MISA_NG_CASE(5)
+      MISA_NG_CASE(6)
+      MISA_NG_CASE(7)
+      MISA_NG_CASE(8)
+      MISA_NG_CASE(9)
+      MISA_NG_CASE(10)
+      MISA_NG_CASE(11)
+      MISA_NG_CASE(12)
+      MISA_NG_CASE(13)
+      MISA_NG_CASE(14)
+      MISA_NG_CASE(15)
+      MISA_NG_CASE(16)
 #undef MISA_NG_CASE
-    default:
-      break;
+      default:
+        break;
+    }
   }
 }
 

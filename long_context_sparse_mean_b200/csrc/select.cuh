@@ -1,0 +1,174 @@
+// Device helpers of the top-k selection.
+//
+// Selection rule ("MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference",
+// Technical Summary, "Sparse Token Scoring" and "Hierarchical Variant (MISA-dagger)": keep the k
+// best tokens): score descending, exact ties to the lower token id.  Scores become
+// order-preserving 32-bit keys (common.cuh).  Radix levels, most significant first:
+//   level 0: bits 31..20 (4096 buckets)   level 1: bits 19..10   level 2: bits 9..0
+// and, when equal keys straddle the boundary, the same three levels on (0xffffffff - id), which
+// ranks smaller ids higher.
+#pragma once
+
+#include "common.cuh"
+
+namespace misa {
+
+constexpr int kHistBins = 4096;
+
+__device__ __forceinline__ int level_shift(int l) { return l == 0 ? 20 : (l == 1 ? 10 : 0); }
+__device__ __forceinline__ int level_bins(int l) { return l == 0 ? 4096 : 1024; }
+
+struct Bucket {
+  uint32_t prefix, need, eq;
+};
+
+// Histogram increment in shared memory.  A plain atomic per item: on B200 aggregating the lanes
+// of a warp that share a bin with __match_any_sync first was three times slower on real score
+// rows (22.7 us against 7.4 us for 32 x 131072 scores; the rows spread over ~70 buckets).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
+
+// Find the bucket (of nb bins holding key bits shift..) that holds the need-th largest key among
+// those counted in hist[nb].  All threads of the block get the same answer.  `scratch` holds 32
+// words of shared memory for the scan and 3 words for the answer.
+__device__ __forceinline__ Bucket block_bucket_bits(const uint32_t* hist, int nb, int sh, uint32_t prefix,
+                                                    uint32_t need, uint32_t* scratch) {
+  const int per = (nb + (int)blockDim.x - 1) / (int)blockDim.x;
+  uint32_t local = 0;
+  for (int d = 0; d < per; ++d) {
+    const int b = nb - 1 - ((int)threadIdx.x * per + d);
+    if (b >= 0) local += hist[b];
+  }
+  uint32_t total;
+  uint32_t cum = block_exclusive_scan(local, scratch, &total);
+  for (int d = 0; d < per; ++d) {
+    const int b = nb - 1 - ((int)threadIdx.x * per + d);
+    if (b < 0) break;
+    const uint32_t hb = hist[b];
+    if (cum < need && cum + hb >= need) {
+      scratch[32] = prefix | ((uint32_t)b << sh);
+      scratch[33] = need - cum;
+      scratch[34] = hb;
+    }
+    cum += hb;
+  }
+  __syncthreads();
+  const Bucket r{scratch[32], scratch[33], scratch[34]};
+  __syncthreads();
+  return r;
+}
+
+__device__ __forceinline__ Bucket block_bucket(const uint32_t* hist, int lvl, uint32_t prefix, uint32_t need,
+                                               uint32_t* scratch) {
+  return block_bucket_bits(hist, level_bins(lvl), level_shift(lvl), prefix, need, scratch);
+}
+
+// Radix select over m items given by acc.key(i) (0 = absent) and acc.id(i).  Starts at level
+// `lvl0` with the boundary prefix/mask already fixed by earlier levels.  On return the selection
+// is: items of class 1 (surely selected) and the first `need` items of class 2 in item order.
+// hist: shared memory of kHistBins words; scratch: 35 words.
+struct SelectResult {
+  uint32_t prefix, mask, need;
+  bool by_id;
+  uint32_t prefix2, mask2, need2;
+};
+
+template <class Acc>
+__device__ SelectResult radix_select_items(const Acc& acc, int m, uint32_t need, int lvl0, uint32_t prefix,
+                                           uint32_t mask, uint32_t* hist, uint32_t* scratch) {
+  SelectResult r{prefix, mask, need, false, 0u, 0u, 0u};
+  uint32_t eq = 0;
+  bool done = false;
+  for (int lvl = lvl0; lvl < 3 && !done; ++lvl) {
+    const int nb = level_bins(lvl), sh = level_shift(lvl);
+    for (int b = threadIdx.x; b < nb; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    const int iters = (m + (int)blockDim.x - 1) / (int)blockDim.x;
+    for (int j = 0; j < iters; ++j) {
+      const int i = j * (int)blockDim.x + (int)threadIdx.x;
+      const uint32_t k = i < m ? acc.key(i) : 0u;
+      hist_add(hist, (k >> sh) & (uint32_t)(nb - 1), k != 0u && (k & r.mask) == r.prefix);
+    }
+    __syncthreads();
+    const Bucket bk = block_bucket(hist, lvl, r.prefix, r.need, scratch);
+    r.prefix = bk.prefix;
+    r.need = bk.need;
+    eq = bk.eq;
+    r.mask |= (uint32_t)(nb - 1) << sh;
+    done = eq == r.need;
+  }
+  if (eq > r.need) {  // equal keys straddle the boundary: rank them by id
+    r.by_id = true;
+    r.need2 = r.need;
+    for (int lvl = 0; lvl < 3; ++lvl) {
+      const int nb = level_bins(lvl), sh = level_shift(lvl);
+      for (int b = threadIdx.x; b < nb; b += blockDim.x) hist[b] = 0;
+      __syncthreads();
+      const int iters = (m + (int)blockDim.x - 1) / (int)blockDim.x;
+      for (int j = 0; j < iters; ++j) {
+        const int i = j * (int)blockDim.x + (int)threadIdx.x;
+        const uint32_t k = i < m ? acc.key(i) : 0u;
+        const bool in = k != 0u && (k & r.mask) == r.prefix;
+        const uint32_t k2 = in ? 0xffffffffu - acc.id(i) : 0u;
+        hist_add(hist, (k2 >> sh) & (uint32_t)(nb - 1), in && (k2 & r.mask2) == r.prefix2);
+      }
+      __syncthreads();
+      const Bucket bk = block_bucket(hist, lvl, r.prefix2, r.need2, scratch);
+      r.prefix2 = bk.prefix;
+      r.need2 = bk.need;
+      r.mask2 |= (uint32_t)(nb - 1) << sh;
+      if (bk.eq == r.need2) break;
+    }
+  }
+  return r;
+}
+
+// Class of item i under a select result: 1 surely selected, 2 selected by rank, 0 not.
+template <class Acc>
+__device__ __forceinline__ int select_class(const Acc& acc, int i, const SelectResult& r) {
+  const uint32_t k = acc.key(i);
+  if (k == 0u) return 0;
+  const uint32_t u = k & r.mask;
+  if (u > r.prefix) return 1;
+  if (u < r.prefix) return 0;
+  if (!r.by_id) return 2;
+  const uint32_t u2 = (0xffffffffu - acc.id(i)) & r.mask2;
+  return u2 > r.prefix2 ? 1 : (u2 == r.prefix2 ? 2 : 0);
+}
+
+// Write the selection in item order: out_id[pos], out_val[pos] for pos < kk (kk = selected count).
+// Every thread takes a contiguous run of items; one block scan places the runs.
+template <class Acc>
+__device__ void write_selection(const Acc& acc, int m, const SelectResult& r, bool take_all, int32_t* out_id,
+                                float* out_val, uint32_t kk, uint32_t* scratch) {
+  const uint32_t needF = r.by_id ? r.need2 : r.need;
+  const int run = (m + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int e0 = min((int)threadIdx.x * run, m), e1 = min(e0 + run, m);
+  uint32_t c1 = 0, c2 = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = take_all ? (acc.key(e) != 0u ? 1 : 0) : select_class(acc, e, r);
+    c1 += c == 1;
+    c2 += c == 2;
+  }
+  uint32_t tot;
+  uint32_t r1 = block_exclusive_scan(c1, scratch, &tot);
+  uint32_t r2 = block_exclusive_scan(c2, scratch, &tot);
+  for (int e = e0; e < e1; ++e) {
+    const int c = take_all ? (acc.key(e) != 0u ? 1 : 0) : select_class(acc, e, r);
+    uint32_t pos = 0xffffffffu;
+    if (c == 1) {
+      pos = r1 + (take_all ? 0u : min(r2, needF));
+      ++r1;
+    } else if (c == 2) {
+      if (r2 < needF) pos = r1 + r2;
+      ++r2;
+    }
+    if (pos < kk) {
+      out_id[pos] = (int32_t)acc.id(e);
+      if (out_val) out_val[pos] = key_to_float(acc.key(e));
+    }
+  }
+}
+
+}  // namespace misa

@@ -1,224 +1,317 @@
-// Top-k selection by radix select.
+// Top-k selection.
 //
 // "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM Inference", Technical Summary,
 // "Methodology: MISA", "Sparse Token Scoring": the final top-k tokens are selected on the reduced
 // scores; "Hierarchical Variant (MISA-dagger)": the k' candidates are narrowed to the top-k by
-// their dense scores.  Selection rule: score descending, exact ties to the lower token index.
+// their dense scores.  Rule: score descending, exact ties to the lower token id (select.cuh).
 //
-// Every score becomes an order-preserving 32-bit key.  Three histogram passes (11, 11 and 10
-// bits, most significant first, each counting only keys whose higher bits match the prefix found
-// so far) pin the key tau of the k-th largest element and how many elements equal to tau are
-// still needed; a pass stops early once the bucket holding the k-th element is taken whole.  A
-// last pass walks the row in index order with a block-wide scan and writes every key above
-// tau and the first `need` keys equal to tau, so the output is in ascending index order and the
-// tie rule holds exactly.  One CTA of 1024 threads per query.
-//
-// Candidate lists (re-rank) live in shared memory; if equal scores straddle the boundary, a
-// second select over the token ids (smaller id wins) settles them, so the result does not depend
-// on the order of the candidate list.
+// Rows of scores (one per query; a position p is token p, or token ids[p] for candidate lists)
+// are selected by a radix cascade over the order keys, every pass reading the rows from L2 with
+// wide loads, 4096 positions per CTA:
+//   1. level-0 pass: 4096-bucket histogram of key bits 31..20 per row; the last CTA of a row to
+//      finish (a counter per row) finds the bucket holding the k-th key and how many keys above it
+//      are taken;
+//   2. level-1 pass: histogram of bits 19..8 of the keys in that bucket; again the last CTA of the
+//      row fixes the 24-bit boundary prefix;
+//   3. partition: keys above the boundary are written out directly (slots reserved with one atomic
+//      per CTA), keys on the boundary prefix go to a short (key, id) list;
+//   4. resolve: one CTA per row ranks that list on the last 8 key bits and, for exact ties, on the
+//      token id, in shared memory (straight from global memory if the list is too long).
+// Clustered scores put about half of a 131072-key row in one level-0 bucket, which is why the
+// cascade has two histogram levels before the partition.  The selected set is exact; its order in
+// the output is not specified.
+// select_small_kernel ranks a short candidate list entirely in one CTA's shared memory; it needs
+// no workspace (used by the entry point without allocation).
 #include "kernels.cuh"
+#include "select.cuh"
 
 namespace misa {
 
 namespace {
 
-constexpr int kTopkThreads = 1024;
-constexpr int kBins = 2048;
+constexpr int kPassThreads = 256;
+constexpr int kPassItems = 16;                         // positions per thread
+constexpr int kPassChunk = kPassThreads * kPassItems;  // positions per CTA
+constexpr int kResolveThreads = 256;
+constexpr int kResolveSmemItems = 8192;  // boundary pairs ranked in shared memory
+constexpr int kSmallThreads = 1024;
+constexpr int kRec = 8;  // words of per-row state
 
-struct SelectState {
-  uint32_t prefix, mask, need, eq;  // keys k with (k & mask) == prefix are "equal"; take `need` of them
+// Per-row state rec[t][kRec]:
+//   0: level-0 CTAs finished   1: level-1 CTAs finished
+//   2: level-0 prefix (bits 31..20)   3: keys still needed inside the level-0 bucket
+//   4: 24-bit boundary prefix (bits 31..8)   5: keys still needed on the boundary prefix
+//   6: slots filled by keys above the boundary   7: boundary pairs written
+
+__device__ __forceinline__ int padded(int e) { return e + (e >> 5); }
+
+// The row positions handled by one thread of a pass CTA: 4 groups of 4 consecutive positions.
+struct RowSlice {
+  const float* row;
+  const int32_t* ids;  // null: token = position
+  int s1, nt;
+  bool vec;
+  __device__ int pos(int base, int item) const {
+    return base + 4 * ((int)threadIdx.x + (item >> 2) * kPassThreads) + (item & 3);
+  }
+  __device__ void load(int base, float (&v)[kPassItems], uint32_t (&key)[kPassItems], bool (&ok)[kPassItems]) const {
+#pragma unroll
+    for (int j = 0; j < kPassItems / 4; ++j) {
+      const int s = pos(base, 4 * j);
+      if (vec && s + 3 < s1) {
+        const float4 x = __ldcg(reinterpret_cast<const float4*>(row + s));
+        v[4 * j] = x.x;
+        v[4 * j + 1] = x.y;
+        v[4 * j + 2] = x.z;
+        v[4 * j + 3] = x.w;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[4 * j + i] = s + i < s1 ? __ldcg(row + s + i) : 0.f;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPassItems; ++i) {
+      const int s = pos(base, i);
+      bool in = s < s1;
+      if (in && ids) {
+        const int32_t id = __ldcg(ids + s);
+        in = id >= 0 && id < nt;
+      }
+      key[i] = order_key(v[i]);
+      ok[i] = in && key[i] != 0u;
+    }
+  }
+  __device__ int32_t token(int p) const { return ids ? ids[p] : p; }
 };
 
-// Radix select over `count` keys fetched by key_at(i) (key 0 = absent).  Leaves the boundary in
-// *st: keys with (key & mask) > prefix are selected, and `need` of the `eq` keys with
-// (key & mask) == prefix.  Requires need <= number of present keys.
-template <class KeyAt>
-__device__ void radix_select(KeyAt key_at, int count, uint32_t need, uint32_t* hist, uint32_t* wtot,
-                             SelectState* st) {
-  uint32_t prefix = 0, mask = 0;
-  uint32_t eq = 0;
-  const int shifts[3] = {21, 10, 0};
-  const int nbits[3] = {11, 11, 10};
-  for (int pass = 0; pass < 3; ++pass) {
-    const int nb = 1 << nbits[pass], sh = shifts[pass];
-    for (int b = threadIdx.x; b < kBins; b += blockDim.x) hist[b] = 0;
-    __syncthreads();
-    for (int i = threadIdx.x; i < count; i += blockDim.x) {
-      const uint32_t u = key_at(i);
-      if (u != 0u && (u & mask) == prefix) atomicAdd(&hist[(u >> sh) & (nb - 1)], 1u);
-    }
-    __syncthreads();
-    // Thread x owns `per` consecutive bins in descending bin order.
-    const int per = (nb + blockDim.x - 1) / blockDim.x;
-    uint32_t local = 0;
-    for (int d = 0; d < per; ++d) {
-      const int b = nb - 1 - (threadIdx.x * per + d);
-      if (b >= 0) local += hist[b];
-    }
-    uint32_t total;
-    uint32_t cum = block_exclusive_scan(local, wtot, &total);
-    for (int d = 0; d < per; ++d) {
-      const int b = nb - 1 - (threadIdx.x * per + d);
-      if (b < 0) break;
-      const uint32_t hb = hist[b];
-      if (cum < need && cum + hb >= need) {
-        st->prefix = prefix | ((uint32_t)b << sh);
-        st->need = need - cum;
-        st->eq = hb;
-      }
-      cum += hb;
-    }
-    __syncthreads();
-    prefix = st->prefix;
-    need = st->need;
-    eq = st->eq;
-    mask |= (uint32_t)(nb - 1) << sh;
-    __syncthreads();
-    if (eq == need) break;  // the boundary bucket is taken whole
-  }
-  if (threadIdx.x == 0) {
-    st->prefix = prefix;
-    st->mask = mask;
-    st->need = need;
-    st->eq = eq;
+// Histogram pass of level LVL (0: bits 31..20 of all keys; 1: bits 19..8 of the keys in the
+// level-0 bucket); the row's last CTA turns the histogram into a boundary.
+template <int LVL>
+__global__ void __launch_bounds__(kPassThreads) hist_pass_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                 const int32_t* __restrict__ ids, int P,
+                                                                 const int32_t* __restrict__ n, int L, int topk,
+                                                                 uint32_t* __restrict__ hist, uint32_t* __restrict__ rec) {
+  __shared__ uint32_t h[kHistBins];
+  __shared__ uint32_t scratch[35];
+  __shared__ int last;
+  const int t = blockIdx.y;
+  const int nt = clamp_len(n[t], L);
+  const int npos = ids ? P : nt;
+  if (!ids && npos <= topk) return;  // the whole prefix is selected
+  const int nchunks = (npos + kPassChunk - 1) / kPassChunk;
+  const int base = blockIdx.x * kPassChunk;
+  if (base >= npos) return;
+  uint32_t* rt = rec + (int64_t)t * kRec;
+  uint32_t* ht = hist + (int64_t)t * kHistBins;
+  for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) h[b] = 0;
+  const RowSlice rs{scores + (int64_t)t * ld, ids ? ids + (int64_t)t * P : nullptr, min(base + kPassChunk, npos), nt,
+                    (ld % 4) == 0};
+  float v[kPassItems];
+  uint32_t key[kPassItems];
+  bool ok[kPassItems];
+  rs.load(base, v, key, ok);
+  const uint32_t top0 = LVL == 1 ? (__ldcg(rt + 2) >> 20) : 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < kPassItems; ++i) {
+    const bool in = ok[i] && (LVL == 0 || (key[i] >> 20) == top0);
+    hist_add(h, LVL == 0 ? key[i] >> 20 : (key[i] >> 8) & 4095u, in);
   }
   __syncthreads();
+  for (int b = threadIdx.x; b < kHistBins; b += kPassThreads)
+    if (h[b]) atomicAdd(ht + b, h[b]);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(rt + LVL, 1u) == (uint32_t)(nchunks - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) h[b] = __ldcg(ht + b);
+  __syncthreads();
+  if (LVL == 0) {
+    // with a candidate list fewer than k keys may be valid: then all of them are taken
+    uint32_t local = 0;
+    for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) local += h[b];
+    uint32_t total;
+    block_exclusive_scan(local, scratch, &total);
+    const uint32_t need = min((uint32_t)topk, total);
+    const Bucket bk = block_bucket_bits(h, kHistBins, 20, 0u, need, scratch);
+    if (threadIdx.x == 0) {
+      rt[2] = need ? bk.prefix : 0xffffffffu;
+      rt[3] = need ? bk.need : 0u;
+    }
+  } else {
+    const uint32_t need = __ldcg(rt + 3);
+    const Bucket bk = block_bucket_bits(h, kHistBins, 8, __ldcg(rt + 2), need, scratch);
+    if (threadIdx.x == 0) {
+      rt[4] = need ? bk.prefix : 0xffffffffu;
+      rt[5] = need ? bk.need : 0u;
+    }
+  }
 }
 
-__global__ void __launch_bounds__(kTopkThreads) topk_rows_kernel(const float* __restrict__ scores, int64_t ld,
+__global__ void __launch_bounds__(kPassThreads) partition_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                 const int32_t* __restrict__ ids, int P,
                                                                  const int32_t* __restrict__ n, int L, int topk,
-                                                                 int32_t* __restrict__ idx,
+                                                                 uint32_t* __restrict__ rec, uint2* __restrict__ pairs,
+                                                                 int64_t pairs_ld, int32_t* __restrict__ idx,
                                                                  float* __restrict__ score_opt) {
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t wtot[32];
-  __shared__ SelectState st;
-  const int t = blockIdx.x;
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t basev[2];
+  const int t = blockIdx.y;
   const int nt = clamp_len(n[t], L);
-  const float* row = scores + (int64_t)t * ld;
+  const int npos = ids ? P : nt;
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
-  if (nt <= topk) {
-    for (int s = threadIdx.x; s < topk; s += blockDim.x) {
-      oi[s] = s < nt ? s : -1;
-      if (ov) ov[s] = s < nt ? row[s] : 0.f;
+  const float* row = scores + (int64_t)t * ld;
+  if (!ids && npos <= topk) {  // every prefix token is selected; this CTA writes its share of the slots
+    const int per = (topk + gridDim.x - 1) / gridDim.x;
+    for (int a = blockIdx.x * per + threadIdx.x; a < min(topk, (int)(blockIdx.x + 1) * per); a += kPassThreads) {
+      oi[a] = a < nt ? a : -1;
+      if (ov) ov[a] = a < nt ? row[a] : 0.f;
     }
     return;
   }
-  auto key_at = [&](int i) { return order_key(row[i]); };
-  radix_select(key_at, nt, (uint32_t)topk, hist, wtot, &st);
-  const uint32_t prefix = st.prefix, mask = st.mask, need = st.need;
-  const uint32_t n_gt = (uint32_t)topk - need;
-  uint32_t base_gt = 0, base_eq = 0;
-  for (int s0 = 0; s0 < nt; s0 += blockDim.x) {
-    const int s = s0 + threadIdx.x;
-    float v = 0.f;
-    uint32_t gt = 0, eq = 0;
-    if (s < nt) {
-      v = row[s];
-      const uint32_t key = order_key(v);
-      const uint32_t u = key & mask;
-      gt = key != 0u && u > prefix;  // key 0 (only an all-ones NaN) is never selected
-      eq = key != 0u && u == prefix;
-    }
-    uint32_t tot;
-    const uint32_t ex = block_exclusive_scan(gt | (eq << 16), wtot, &tot);
-    const uint32_t gt_before = base_gt + (ex & 0xffffu), eq_before = base_eq + (ex >> 16);
-    if (gt || (eq && eq_before < need)) {
-      const uint32_t pos = gt_before + min(eq_before, need);
-      if (pos < (uint32_t)topk) {
-        oi[pos] = s;
-        if (ov) ov[pos] = v;
+  const int base = blockIdx.x * kPassChunk;
+  if (base >= npos) return;
+  uint32_t* rt = rec + (int64_t)t * kRec;
+  const uint32_t b24 = __ldcg(rt + 4);
+  const bool none = b24 == 0xffffffffu;  // no valid key at all
+  const uint32_t prefix = b24 >> 8;
+  const RowSlice rs{row, ids ? ids + (int64_t)t * P : nullptr, min(base + kPassChunk, npos), nt, (ld % 4) == 0};
+  float v[kPassItems];
+  uint32_t key[kPassItems];
+  bool ok[kPassItems];
+  rs.load(base, v, key, ok);
+  uint32_t gtm = 0, eqm = 0;
+#pragma unroll
+  for (int i = 0; i < kPassItems; ++i) {
+    gtm |= (uint32_t)(!none && ok[i] && (key[i] >> 8) > prefix) << i;
+    eqm |= (uint32_t)(!none && ok[i] && (key[i] >> 8) == prefix) << i;
+  }
+  uint32_t tg, te;
+  uint32_t pg = block_exclusive_scan(__popc(gtm), scratch, &tg);
+  uint32_t pe = block_exclusive_scan(__popc(eqm), scratch, &te);
+  if (threadIdx.x == 0) {
+    basev[0] = tg ? atomicAdd(rt + 6, tg) : 0u;
+    basev[1] = te ? atomicAdd(rt + 7, te) : 0u;
+  }
+  __syncthreads();
+  pg += basev[0];
+  pe += basev[1];
+  uint2* pt = pairs + (int64_t)t * pairs_ld;
+#pragma unroll
+  for (int i = 0; i < kPassItems; ++i) {
+    const int p = rs.pos(base, i);
+    if ((gtm >> i) & 1u) {
+      if (pg < (uint32_t)topk) {
+        oi[pg] = rs.token(p);
+        if (ov) ov[pg] = v[i];
       }
+      ++pg;
     }
-    base_gt += tot & 0xffffu;
-    base_eq += tot >> 16;
-    if (base_gt == n_gt && base_eq >= need) break;  // uniform: every selected index is written
+    if ((eqm >> i) & 1u) {
+      if (pe < (uint32_t)pairs_ld) pt[pe] = make_uint2(key[i], (uint32_t)rs.token(p));
+      ++pe;
+    }
   }
 }
 
-// Candidate lists: F[t, P] with ids cand[t, P]; dynamic shared memory holds keys[P] and ids[P].
-__global__ void __launch_bounds__(kTopkThreads) topk_cand_kernel(const float* __restrict__ F,
-                                                                 const int32_t* __restrict__ cand,
-                                                                 const int32_t* __restrict__ n, int L, int P,
-                                                                 int topk, int32_t* __restrict__ idx,
-                                                                 float* __restrict__ score_opt) {
-  extern __shared__ uint32_t csm[];
-  uint32_t* keys = csm;       // [P] order keys, 0 = empty slot
-  uint32_t* ids = csm + P;    // [P] token ids
-  __shared__ uint32_t hist[kBins];
-  __shared__ uint32_t wtot[32];
-  __shared__ SelectState st, st2;
+struct PairList {
+  const uint2* p;
+  __device__ uint32_t key(int i) const { return p[i].x; }
+  __device__ uint32_t id(int i) const { return p[i].y; }
+};
+
+// One CTA per row: slots [n_out, n_out + need) come from the boundary pairs; the rest of the row
+// after the selection is padded with -1.
+__global__ void __launch_bounds__(kResolveThreads) resolve_kernel(const int32_t* __restrict__ n, int L, bool lists,
+                                                                  int topk, const uint32_t* __restrict__ rec,
+                                                                  const uint2* __restrict__ pairs, int64_t pairs_ld,
+                                                                  int32_t* __restrict__ idx,
+                                                                  float* __restrict__ score_opt) {
+  extern __shared__ uint2 list[];  // [kResolveSmemItems]
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t scratch[35];
+  const int t = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  if (!lists && nt <= topk) return;
+  const uint32_t* rt = rec + (int64_t)t * kRec;
+  const uint32_t n_out = min(__ldcg(rt + 6), (uint32_t)topk);
+  const int c = (int)min(__ldcg(rt + 7), (uint32_t)pairs_ld);
+  const uint32_t need = min(__ldcg(rt + 5), (uint32_t)c);
+  const uint32_t prefix = __ldcg(rt + 4);
+  int32_t* oi = idx + (int64_t)t * topk;
+  float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
+  const uint2* pt = pairs + (int64_t)t * pairs_ld;
+  const uint32_t kk = min((uint32_t)topk, n_out + need);
+  if ((uint32_t)c <= need) {
+    for (int i = threadIdx.x; i < c; i += kResolveThreads)
+      if (n_out + i < (uint32_t)topk) {
+        oi[n_out + i] = (int32_t)pt[i].y;
+        if (ov) ov[n_out + i] = key_to_float(pt[i].x);
+      }
+  } else if (c <= kResolveSmemItems) {
+    for (int i = threadIdx.x; i < c; i += kResolveThreads) list[i] = pt[i];
+    __syncthreads();
+    const PairList acc{list};
+    const SelectResult r = radix_select_items(acc, c, need, 2, prefix, 0xffffff00u, hist, scratch);
+    write_selection(acc, c, r, false, oi + n_out, ov ? ov + n_out : nullptr, need, scratch);
+  } else {
+    const PairList acc{pt};
+    const SelectResult r = radix_select_items(acc, c, need, 2, prefix, 0xffffff00u, hist, scratch);
+    write_selection(acc, c, r, false, oi + n_out, ov ? ov + n_out : nullptr, need, scratch);
+  }
+  for (int a = (int)kk + threadIdx.x; a < topk; a += kResolveThreads) {
+    oi[a] = -1;
+    if (ov) ov[a] = 0.f;
+  }
+}
+
+struct SmemItems {
+  const uint32_t* keys;
+  const uint32_t* ids;
+  __device__ uint32_t key(int i) const { return keys[padded(i)]; }
+  __device__ uint32_t id(int i) const { return ids[padded(i)]; }
+};
+
+// Top-k of candidate lists in one CTA: values F[t, P], ids cand[t, P] (ids outside [0, n_t) are
+// empty).
+__global__ void __launch_bounds__(kSmallThreads) select_small_kernel(const float* __restrict__ F,
+                                                                     const int32_t* __restrict__ cand,
+                                                                     const int32_t* __restrict__ n, int L, int P,
+                                                                     int topk, int32_t* __restrict__ idx,
+                                                                     float* __restrict__ score_opt) {
+  extern __shared__ uint32_t sm[];
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t scratch[35];
+  uint32_t* keys = sm;
+  uint32_t* ids = sm + padded(P) + 1;
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
   const float* ft = F + (int64_t)t * P;
-  const int32_t* ct = cand + (int64_t)t * P;
+  const int32_t* ctp = cand + (int64_t)t * P;
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
-  uint32_t cnt = 0;
-  for (int i = threadIdx.x; i < P; i += blockDim.x) {
-    const int32_t id = ct[i];
+  uint32_t mine = 0;
+  for (int i = threadIdx.x; i < P; i += kSmallThreads) {
+    const int32_t id = ctp[i];
     const bool ok = id >= 0 && id < nt;
-    keys[i] = ok ? order_key(ft[i]) : 0u;
-    ids[i] = ok ? (uint32_t)id : 0u;
-    cnt += ok;
+    keys[padded(i)] = ok ? order_key(ft[i]) : 0u;
+    ids[padded(i)] = ok ? (uint32_t)id : 0u;
+    mine += ok;
   }
   uint32_t nvalid;
-  block_exclusive_scan(cnt, wtot, &nvalid);
-  const uint32_t kk = (uint32_t)topk < nvalid ? (uint32_t)topk : nvalid;
-  uint32_t prefix = 0, mask = 0, need = 0;
-  bool tie_by_id = false;
-  uint32_t prefix2 = 0, mask2 = 0, need2 = 0;
-  if (kk < nvalid) {
-    radix_select([&](int i) { return keys[i]; }, P, kk, hist, wtot, &st);
-    prefix = st.prefix;
-    mask = st.mask;
-    need = st.need;
-    if (st.eq > need) {
-      // equal scores straddle the boundary: among them keep the `need` smallest ids
-      tie_by_id = true;
-      radix_select(
-          [&](int i) { return (keys[i] != 0u && (keys[i] & mask) == prefix) ? 0xffffffffu - ids[i] : 0u; }, P,
-          need, hist, wtot, &st2);
-      prefix2 = st2.prefix;
-      mask2 = st2.mask;
-      need2 = st2.need;
-    }
+  block_exclusive_scan(mine, scratch, &nvalid);
+  const uint32_t kk = min((uint32_t)topk, nvalid);
+  const SmemItems acc{keys, ids};
+  if (kk == nvalid) {
+    write_selection(acc, P, SelectResult{}, true, oi, ov, kk, scratch);
+  } else {
+    const SelectResult r = radix_select_items(acc, P, kk, 0, 0u, 0u, hist, scratch);
+    write_selection(acc, P, r, false, oi, ov, kk, scratch);
   }
-  uint32_t base = 0, base_eq2 = 0;
-  for (int i0 = 0; i0 < P; i0 += blockDim.x) {
-    const int i = i0 + threadIdx.x;
-    uint32_t sel = 0, eq2 = 0;
-    if (i < P && keys[i] != 0u) {
-      if (kk == nvalid) {
-        sel = 1;
-      } else {
-        const uint32_t u = keys[i] & mask;
-        if (u > prefix) sel = 1;
-        else if (u == prefix) {
-          if (!tie_by_id) sel = 1;  // the whole equal group is needed (eq == need)
-          else {
-            const uint32_t u2 = (0xffffffffu - ids[i]) & mask2;
-            if (u2 > prefix2) sel = 1;
-            else if (u2 == prefix2) eq2 = 1;
-          }
-        }
-      }
-    }
-    uint32_t tot;
-    const uint32_t ex = block_exclusive_scan(sel | (eq2 << 16), wtot, &tot);
-    const uint32_t eq2_before = base_eq2 + (ex >> 16);
-    if (eq2 && eq2_before < need2) sel = 1;
-    // positions: recount with the resolved flags
-    uint32_t tot2;
-    const uint32_t pos = base + block_exclusive_scan(sel, wtot, &tot2);
-    if (sel && pos < (uint32_t)topk) {
-      oi[pos] = (int32_t)ids[i];
-      if (ov) ov[pos] = key_to_float(keys[i]);
-    }
-    base += tot2;
-    base_eq2 += tot >> 16;
-  }
-  for (int a = (int)kk + threadIdx.x; a < topk; a += blockDim.x) {
+  for (int a = (int)kk + threadIdx.x; a < topk; a += kSmallThreads) {
     oi[a] = -1;
     if (ov) ov[a] = 0.f;
   }
@@ -226,20 +319,37 @@ __global__ void __launch_bounds__(kTopkThreads) topk_cand_kernel(const float* __
 
 }  // namespace
 
-void launch_topk_rows(const float* scores, int64_t ld, const int32_t* n, int T, int L, int topk, int32_t* idx,
-                      float* score_opt, cudaStream_t s) {
-  if (T <= 0) return;
-  topk_rows_kernel<<<T, kTopkThreads, 0, s>>>(scores, ld, n, L, topk, idx, score_opt);
+// Workspace of one selection: hist0 [T][4096], hist1 [T][4096], rec [T][8], pairs [T][P] (uint2).
+size_t topk_rows_ws(int T, int P) {
+  return sizeof(uint32_t) * (2 * (size_t)kHistBins + kRec) * (size_t)T + sizeof(uint2) * (size_t)T * P;
 }
 
-size_t topk_cand_smem(int P) { return sizeof(uint32_t) * 2 * (size_t)P; }
+void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
+                      int topk, void* ws, int32_t* idx, float* score_opt, cudaStream_t s) {
+  if (T <= 0) return;
+  const int npos = ids ? P : L;
+  uint32_t* hist0 = static_cast<uint32_t*>(ws);
+  uint32_t* hist1 = hist0 + (size_t)kHistBins * T;
+  uint32_t* rec = hist1 + (size_t)kHistBins * T;
+  uint2* pairs = reinterpret_cast<uint2*>(rec + (size_t)kRec * T);  // 8-byte aligned: even word count
+  cudaMemsetAsync(ws, 0, sizeof(uint32_t) * (2 * (size_t)kHistBins + kRec) * (size_t)T, s);
+  const dim3 grid((npos + kPassChunk - 1) / kPassChunk, T);
+  hist_pass_kernel<0><<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, hist0, rec);
+  hist_pass_kernel<1><<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, hist1, rec);
+  partition_kernel<<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, rec, pairs, npos, idx, score_opt);
+  const size_t smem = sizeof(uint2) * (size_t)kResolveSmemItems;
+  cudaFuncSetAttribute(resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  resolve_kernel<<<T, kResolveThreads, smem, s>>>(n, L, ids != nullptr, topk, rec, pairs, npos, idx, score_opt);
+}
+
+size_t topk_cand_smem(int P) { return sizeof(uint32_t) * 2 * (size_t)(P + P / 32 + 2); }
 
 void launch_topk_cand(const float* F, const int32_t* cand, const int32_t* n, int T, int L, int P, int topk,
                       int32_t* idx, float* score_opt, cudaStream_t s) {
   if (T <= 0) return;
   const size_t smem = topk_cand_smem(P);
-  cudaFuncSetAttribute(topk_cand_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  topk_cand_kernel<<<T, kTopkThreads, smem, s>>>(F, cand, n, L, P, topk, idx, score_opt);
+  cudaFuncSetAttribute(select_small_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  select_small_kernel<<<T, kSmallThreads, smem, s>>>(F, cand, n, L, P, topk, idx, score_opt);
 }
 
 }  // namespace misa
