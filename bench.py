@@ -202,6 +202,7 @@ def run_ours(args):
     M_ = -(-L // B)
     stream = torch.cuda.current_stream()
     wsp = M.Workspace(dev)
+    sel_ws = M.Workspace(dev)  # selection state shared by the scoring and top-k' calls
     kbar = M.misa_pool_keys(kd, B)
     heads = torch.empty((T, h), dtype=torch.int32, device=dev)
     scores = torch.empty((T, L), dtype=torch.float32, device=dev)
@@ -210,8 +211,9 @@ def run_ours(args):
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     score_ms = []
-    # pool, router, scores, 4 top-k' kernels, re-rank scores + 4 selection kernels
-    launches_per_step = 12
+    # pool, router, scores (level-0 histogram fused), partition + resolve, re-rank scores (fused
+    # histogram) + partition + resolve
+    launches_per_step = 8
 
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
 
@@ -224,11 +226,11 @@ def run_ours(args):
         mark(2)
         if time_scores:
             ev[0].record(stream)
-        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
         if time_scores:
             ev[1].record(stream)
         mark(3)
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=wsp)
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=True)
         mark(4)
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
         mark(5)

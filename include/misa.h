@@ -118,22 +118,29 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
  * Routed-head token scores ("Sparse Token Scoring"): scores[t, s] = I_{t,s} for s < n_t.
  *   heads    : [T, h] routed heads (any order; NULL = all H_I heads, i.e. the dense score F)
  *   scores   : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
+ *   select_ws, select_ws_bytes, select_topk : optional (NULL, 0, 0).  A workspace of
+ *              misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes in which the call also
+ *              leaves the first stage of a top-select_topk selection of these scores (the decode
+ *              scoring kernel builds it while it writes the scores); pass the same workspace to
+ *              misa_topk_select with ws_prepared = 1.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
-                              int h, int dtype, float* scores, int64_t ld_scores, void* stream);
+                              int h, int dtype, float* scores, int64_t ld_scores, int select_topk,
+                              void* select_ws, size_t select_ws_bytes, void* stream);
 
 /*
  * Top-k selection over per-query score rows ("Sparse Token Scoring": the final top-k tokens
  * are selected on the reduced scores).  scores [T, ld_scores] fp32, entries s < n_t are read.
- *   idx       : out [T, topk] int32, -1 padded
- *   score_opt : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
- *   ws        : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
+ *   idx         : out [T, topk] int32, -1 padded
+ *   score_opt   : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
+ *   ws          : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
+ *   ws_prepared : 1 if misa_token_scores already prepared ws for these scores and this topk
  * Scores must be finite.
  */
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
                              int L, int topk, int32_t* idx, float* score_opt, void* ws,
-                             size_t ws_bytes, void* stream);
+                             size_t ws_bytes, int ws_prepared, void* stream);
 
 /*
  * Routed scoring followed by top-k: misa_token_scores then misa_topk_select.  With topk = k'

@@ -44,8 +44,8 @@ def _setup(lib):
         "misa_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32, i32], sz),
         "misa_pool_keys": ([P, i64, i32, i32, i32, i32, i32, P, i64, i32, i32, P], i32),
         "misa_route": ([P, P, P, i64, P, i64, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
-        "misa_token_scores": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, P, i64, P], i32),
-        "misa_topk_select": ([P, i64, P, i32, i32, i32, P, P, P, sz, P], i32),
+        "misa_token_scores": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, P, i64, i32, P, sz, P], i32),
+        "misa_topk_select": ([P, i64, P, i32, i32, i32, P, P, P, sz, i32, P], i32),
         "misa_score_topk": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, sz, P], i32),
         "misa_hier_rerank": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
         "dsa_dense_topk": ([P, P, P, i64, P, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
@@ -179,8 +179,10 @@ def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optiona
     return heads, r
 
 
-def misa_token_scores(q, w, k, n, heads=None, out=None, stream=None) -> torch.Tensor:
-    """Scores [T, L] fp32 (entries s >= n_t untouched); heads None = all heads (dense score)."""
+def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, select_ws=None, stream=None):
+    """Scores [T, L] fp32 (entries s >= n_t untouched); heads None = all heads (dense score).
+    With select_topk > 0 and a Workspace, the first stage of a top-select_topk selection of the
+    scores is left in that workspace for misa_topk_select(..., ws=<same>, ws_prepared=True)."""
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
@@ -194,14 +196,20 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, stream=None) -> torch.Te
     if out is None:
         out = torch.empty((T, L), dtype=torch.float32, device=q.device)
     _need(out, "out", torch.float32)
+    buf, nbytes = None, 0
+    if select_topk > 0:
+        if select_ws is None:
+            raise ValueError("select_topk needs select_ws")
+        nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, H_I)
+        buf = select_ws.get(nbytes)
     _check("misa_token_scores", _lib.misa_token_scores(
         _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, _dtype_code(q), _p(out), out.shape[1],
-        _stream(stream)))
+        select_topk, _p(buf), nbytes, _stream(stream)))
     return out
 
 
 def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, vals=None, want_vals=True,
-                     ws: Optional[Workspace] = None, stream=None):
+                     ws: Optional[Workspace] = None, ws_prepared: bool = False, stream=None):
     """Top-k per row of scores [T, ld] over entries s < min(n_t, L) -> (idx [T, k], vals [T, k])."""
     _need(scores, "scores", torch.float32)
     _need(n, "n", torch.int32)
@@ -214,7 +222,7 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
     nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, 8)
     buf = _ws(ws, scores.device).get(nbytes)
     _check("misa_topk_select", _lib.misa_topk_select(
-        _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
+        _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), _p(buf), nbytes, int(ws_prepared), _stream(stream)))
     return idx, vals
 
 

@@ -51,7 +51,7 @@ size_t route_ws(int T, int L, int H_I, int B) {
 size_t scores_part(int T, int L) { return align_up(sizeof(float) * (size_t)T * score_ld(L)); }
 
 // misa_topk_select: histograms, per-row state and boundary pairs of the selection
-size_t select_ws(int T, int P) {
+size_t select_bytes(int T, int P) {
   if (T <= 0 || P <= 0) return 0;
   return align_up(misa::topk_rows_ws(T, P));
 }
@@ -59,13 +59,13 @@ size_t select_ws(int T, int P) {
 // misa_score_topk / dsa_dense_topk: [scores][selection]
 size_t scores_ws(int T, int L) {
   if (T <= 0 || L <= 0) return 0;
-  return scores_part(T, L) + select_ws(T, L);
+  return scores_part(T, L) + select_bytes(T, L);
 }
 
 // misa_hier_rerank: [dense scores of the candidates][selection over the candidate lists]
 size_t rerank_ws(int T, int kp) {
   if (T <= 0 || kp <= 0) return 0;
-  return align_up(sizeof(float) * (size_t)T * kp) + select_ws(T, kp);
+  return align_up(sizeof(float) * (size_t)T * kp) + select_bytes(T, kp);
 }
 
 }  // namespace
@@ -103,7 +103,7 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
     case MISA_OP_RERANK:
       return rerank_ws(T, kp);
     case MISA_OP_TOPK_SELECT:
-      return select_ws(T, L);
+      return select_bytes(T, L);
     default:
       return 0;
   }
@@ -148,25 +148,39 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
 
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
                               const int32_t* heads, int T, int L, int H_I, int d, int h, int dtype, float* scores,
-                              int64_t ld_scores, void* stream) {
+                              int64_t ld_scores, int select_topk, void* select_ws, size_t select_ws_bytes,
+                              void* stream) {
   misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
   if (st != MISA_OK) return st;
   if (heads && (h < 1 || h > H_I)) return MISA_ERR_INVALID_ARG;
   if (ld_scores < L) return MISA_ERR_INVALID_ARG;
+  if (select_ws && select_topk < 1) return MISA_ERR_INVALID_ARG;
   if (T == 0) return MISA_OK;
   if (!scores) return MISA_ERR_INVALID_ARG;
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, heads ? h : H_I, nullptr, 0,
-                      scores, ld_scores, as_stream(stream));
+  if (select_ws && (select_ws_bytes < select_bytes(T, L) || !aligned(select_ws))) return MISA_ERR_WORKSPACE;
+  const cudaStream_t s = as_stream(stream);
+  if (!select_ws) {
+    misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, heads ? h : H_I, nullptr, 0,
+                        scores, ld_scores, nullptr, s);
+    return launch_status();
+  }
+  misa::topk_rows_prepare(select_ws, T, s);
+  const misa::TopkFuse fuse = misa::topk_rows_fuse(select_ws, T, select_topk);
+  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I,
+                                         heads ? h : H_I, nullptr, 0, scores, ld_scores, &fuse, s);
+  if (!ready) misa::launch_topk_level0(scores, ld_scores, nullptr, 0, n, T, L, select_topk, select_ws, s);
   return launch_status();
 }
 
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T, int L, int topk,
-                             int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+                             int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, int ws_prepared,
+                             void* stream) {
   if (T < 0 || L < 1 || topk < 1 || ld_scores < L) return MISA_ERR_INVALID_ARG;
   if (T == 0) return MISA_OK;
   if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < select_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
-  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws, idx, score_opt, as_stream(stream));
+  if (!ws || ws_bytes < select_bytes(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws, ws_prepared != 0, idx, score_opt,
+                         as_stream(stream));
   return launch_status();
 }
 
@@ -180,7 +194,7 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
   if (h < 1 || h > H_I || topk < 1) return MISA_ERR_INVALID_ARG;
   if (T == 0) return MISA_OK;
   if (!idx) return MISA_ERR_INVALID_ARG;
-  if (!ws || ws_bytes < (scores_full_opt ? select_ws(T, L) : scores_ws(T, L)) || !aligned(ws))
+  if (!ws || ws_bytes < (scores_full_opt ? select_bytes(T, L) : scores_ws(T, L)) || !aligned(ws))
     return MISA_ERR_WORKSPACE;
   char* p = static_cast<char*>(ws);
   float* buf = scores_full_opt;
@@ -190,9 +204,11 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
     ld = score_ld(L);
     p += scores_part(T, L);
   }
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld,
-                      as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, idx, score_opt, as_stream(stream));
+  misa::topk_rows_prepare(p, T, as_stream(stream));
+  const misa::TopkFuse fuse = misa::topk_rows_fuse(p, T, topk);
+  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0,
+                                         buf, ld, &fuse, as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, ready, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -208,9 +224,11 @@ misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64
   if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   float* F = static_cast<float*>(ws);
   void* sel = static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * kp);
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp,
-                      as_stream(stream));
-  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, idx, score_opt, as_stream(stream));
+  misa::topk_rows_prepare(sel, T, as_stream(stream));
+  const misa::TopkFuse fuse = misa::topk_rows_fuse(sel, T, topk);
+  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand,
+                                         kp, F, kp, &fuse, as_stream(stream));
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, ready, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -226,10 +244,12 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   char* p = static_cast<char*>(ws);
   float* buf = reinterpret_cast<float*>(p);
   const int64_t ld = score_ld(L);
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
-                      as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p + scores_part(T, L), idx, score_opt,
-                         as_stream(stream));
+  void* sel = p + scores_part(T, L);
+  misa::topk_rows_prepare(sel, T, as_stream(stream));
+  const misa::TopkFuse fuse = misa::topk_rows_fuse(sel, T, topk);
+  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr,
+                                         0, buf, ld, &fuse, as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, sel, ready, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 

@@ -19,18 +19,34 @@ void launch_route(DType dt, const void* q, const float* w, const void* k, int64_
                   int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
                   uint32_t* done, cudaStream_t s);
 
+// Level-0 selection state the decode scoring kernel can build while it scores (select.cuh):
+// hist [T][4096] and rec [T][8], both zeroed beforehand (topk_rows_prepare).
+struct TopkFuse {
+  uint32_t* hist;
+  uint32_t* rec;
+  int topk;
+};
+
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
-// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].
-void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].  Returns true if it
+// also filled *fuse (only the persistent bf16 kernel does).
+bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
-                   const int32_t* rows, int P, float* out, int64_t ld, cudaStream_t s);
+                   const int32_t* rows, int P, float* out, int64_t ld, const TopkFuse* fuse, cudaStream_t s);
 
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
 // or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t)).  ws holds
-// topk_rows_ws(T, P or L) bytes, 256-byte aligned.  Output order within a row is not specified.
+// topk_rows_ws(T, P or L) bytes, 256-byte aligned; hist_ready: the scoring kernel already filled
+// the level-0 state in ws.  Output order within a row is not specified.
 size_t topk_rows_ws(int T, int P);
+void topk_rows_prepare(void* ws, int T, cudaStream_t s);
+TopkFuse topk_rows_fuse(void* ws, int T, int topk);
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
-                      int L, int topk, void* ws, int32_t* idx, float* score_opt, cudaStream_t s);
+                      int L, int topk, void* ws, bool hist_ready, int32_t* idx, float* score_opt,
+                      cudaStream_t s);
+// Only the level-0 state (prepare + histogram pass), for scores written without it.
+void launch_topk_level0(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
+                        int L, int topk, void* ws, cudaStream_t s);
 
 // Top-k of short candidate lists in shared memory (no workspace): values F[t, P], ids cand[t, P].
 size_t topk_cand_smem(int P);

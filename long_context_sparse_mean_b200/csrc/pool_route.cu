@@ -52,16 +52,40 @@ __device__ __forceinline__ float block_mean_256(const void* kseq, int s0, int s1
   return mean;
 }
 
+// One CTA of 1024 threads per block: 16 row groups x 64 column pairs, so a 128-key block is read
+// with every load in flight at once.
 template <DType DT>
-__global__ void __launch_bounds__(256) pool_kernel(const void* k, int64_t k_seq_stride, int L, int B,
-                                                   float* kbar, int64_t kbar_seq_stride, int b0) {
-  __shared__ float part[4][kD];
+__global__ void __launch_bounds__(1024) pool_kernel(const void* k, int64_t k_seq_stride, int L, int B,
+                                                    float* kbar, int64_t kbar_seq_stride, int b0) {
+  constexpr int RG = 16;
+  __shared__ float part[RG][kD];
   const int b = b0 + blockIdx.x, seq = blockIdx.y;
   const size_t esz = DT == DType::BF16 ? 2 : 4;
   const void* kseq = static_cast<const char*>(k) + (int64_t)seq * k_seq_stride * esz;
   const int s0 = b * B, s1 = min(s0 + B, L);
-  const float m = block_mean_256<DT>(kseq, s0, s1, part);
-  if (threadIdx.x < kD) kbar[(int64_t)seq * kbar_seq_stride + (int64_t)b * kD + threadIdx.x] = m;
+  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
+  float a0 = 0.f, a1 = 0.f;
+#pragma unroll 4
+  for (int s = s0 + rg; s < s1; s += RG) {
+    if (DT == DType::BF16) {
+      const uint32_t x = reinterpret_cast<const uint32_t*>(kseq)[(int64_t)s * (kD / 2) + cp];
+      a0 += bf16_lo(x);
+      a1 += bf16_hi(x);
+    } else {
+      const float2 x = reinterpret_cast<const float2*>(kseq)[(int64_t)s * (kD / 2) + cp];
+      a0 += x.x;
+      a1 += x.y;
+    }
+  }
+  part[rg][2 * cp] = a0;
+  part[rg][2 * cp + 1] = a1;
+  __syncthreads();
+  if (threadIdx.x < kD) {
+    float sum = 0.f;
+#pragma unroll
+    for (int r = 0; r < RG; ++r) sum += part[r][threadIdx.x];
+    kbar[(int64_t)seq * kbar_seq_stride + (int64_t)b * kD + threadIdx.x] = sum / (float)(s1 - s0);
+  }
 }
 
 // Mean of the partial last block [floor(n_t/B)*B, n_t) of every query whose prefix is not a
@@ -297,10 +321,15 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
   float acc[NG][4];
 #pragma unroll
   for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.f;
-#pragma unroll 2
+  float4 XA[8], XB[8];  // all loads of the warp's two pooled-key rows in flight at once
+#pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
-    const float4 xa = rowa ? *reinterpret_cast<const float4*>(rowa + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
-    const float4 xb = rowb ? *reinterpret_cast<const float4*>(rowb + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
+    XA[kk] = rowa ? *reinterpret_cast<const float4*>(rowa + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
+    XB[kk] = rowb ? *reinterpret_cast<const float4*>(rowb + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const float4 xa = XA[kk], xb = XB[kk];
     float ah[4], am[4], al[4], bh[4], bm[4], bl[4];
     split3(xa.x, ah[0], am[0], al[0]);
     split3(xa.y, ah[1], am[1], al[1]);
@@ -362,9 +391,9 @@ void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L
   if (b1 <= b0 || n_seq <= 0) return;
   dim3 grid(b1 - b0, n_seq);
   if (dt == DType::BF16)
-    pool_kernel<DType::BF16><<<grid, 256, 0, s>>>(k, k_seq_stride, L, B, kbar, kbar_seq_stride, b0);
+    pool_kernel<DType::BF16><<<grid, 1024, 0, s>>>(k, k_seq_stride, L, B, kbar, kbar_seq_stride, b0);
   else
-    pool_kernel<DType::F32><<<grid, 256, 0, s>>>(k, k_seq_stride, L, B, kbar, kbar_seq_stride, b0);
+    pool_kernel<DType::F32><<<grid, 1024, 0, s>>>(k, k_seq_stride, L, B, kbar, kbar_seq_stride, b0);
 }
 
 int route_chunks(int L, int B) {

@@ -29,6 +29,7 @@
 
 #include "kernels.cuh"
 #include "mma_frag.cuh"
+#include "select.cuh"
 
 namespace misa {
 
@@ -87,10 +88,15 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                          const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                          const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
-                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld) {
-  extern __shared__ int tile_base[];  // flattened tile prefix [T + 1]
+                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld,
+                         uint32_t* __restrict__ hist, uint32_t* __restrict__ rec, int topk) {
+  // dynamic: padded level-0 histogram [kHistPadded], then the flattened tile prefix [T + 1]
+  extern __shared__ uint32_t dyn[];
+  uint32_t* hsm = dyn;
+  int* tile_base = reinterpret_cast<int*>(dyn + kHistPadded);
   __shared__ HeadStage<NG> st;
-  __shared__ uint32_t wtot[32];
+  __shared__ uint32_t wtot[35];
+  __shared__ int last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
 
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
@@ -104,6 +110,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     run += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
   }
   if (threadIdx.x == 0) tile_base[T] = (int)total;
+  if (hist)
+    for (int b = threadIdx.x; b < kHistPadded; b += kScoreThreads) hsm[b] = 0;
   __syncthreads();
   const int64_t tb = (int64_t)blockIdx.x * total / gridDim.x;
   const int64_t te = (int64_t)(blockIdx.x + 1) * total / gridDim.x;
@@ -142,15 +150,19 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
     int nia = GATHER && ntile > 1 ? raw_id(row_of(1) + g) : -1;
     int nib = GATHER && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
-    auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4]) {
+    auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4], bool& va, bool& vb) {
       ra = valid_row(ra);
       rb = valid_row(rb);
+      va = ra >= 0;
+      vb = rb >= 0;
       load_rows(ra >= 0 ? kt + (int64_t)ra * kD : nullptr, rb >= 0 ? kt + (int64_t)rb * kD : nullptr, c, A, B);
     };
     uint4 RA[4], RB[4];
-    load_ids(ida, idb, RA, RB);
+    bool va, vb;
+    load_ids(ida, idb, RA, RB, va, vb);
     for (int j = 0; j < ntile; ++j) {
       uint4 NA[4], NB[4];
+      bool na = false, nb = false;
       if (j + 1 < ntile) {
         int ra, rb;
         if (GATHER) {
@@ -162,17 +174,52 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
           ra = raw_id(row_of(j + 1) + g);
           rb = raw_id(row_of(j + 1) + g + 8);
         }
-        load_ids(ra, rb, NA, NB);
+        load_ids(ra, rb, NA, NB, na, nb);
       }
       float slo, shi;
       score_rows<NG>(RA, RB, st.frag, wa, wb, lane, slo, shi);
       const int r = row_of(j) + g;
       if (c == 0 && r < npos) ot[r] = slo;
       if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
+      if (hist) {  // count the key row's score; empty gathered slots are not counted
+        const bool cnt = (c == 0 && va) || (c == 1 && vb);
+        if (cnt) atomicAdd(&hsm[hpad((int)(order_key(c == 0 ? slo : shi) >> 20))], 1u);
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         RA[i] = NA[i];
         RB[i] = NB[i];
+      }
+      va = na;
+      vb = nb;
+    }
+    if (hist) {
+      // add this segment's counts to the row's histogram; the CTA that completes the row's
+      // tiles turns it into the level-0 boundary of the selection
+      __syncthreads();
+      uint32_t* ht = hist + (int64_t)t * kHistBins;
+      for (int b = threadIdx.x; b < kHistBins; b += kScoreThreads) {
+        const uint32_t v = hsm[hpad(b)];
+        if (v) atomicAdd(ht + b, v);
+        hsm[hpad(b)] = 0;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        // fences are cumulative: after the barrier, one fence orders the whole CTA's adds
+        __threadfence();
+        const uint32_t row_tiles = (uint32_t)(tile_base[t + 1] - tile_base[t]);
+        last = atomicAdd(rec + 8 * (int64_t)t, (uint32_t)ntile) + (uint32_t)ntile == row_tiles;
+      }
+      __syncthreads();
+      if (last) {
+        __threadfence();
+        const Bucket bk = level0_boundary(ht, (uint32_t)topk, hsm, wtot);
+        if (threadIdx.x == 0) {
+          rec[8 * (int64_t)t + 2] = bk.prefix;
+          rec[8 * (int64_t)t + 3] = bk.need;
+        }
+        for (int b = threadIdx.x; b < kHistPadded; b += kScoreThreads) hsm[b] = 0;
+        __syncthreads();
       }
     }
     pos = seg_end;
@@ -308,19 +355,22 @@ int num_sms() {
 template <int NG>
 void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const float* w, const void* k,
                  int64_t k_seq_stride, const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L,
-                 const int32_t* rows, int P, float* out, int64_t ld) {
+                 const int32_t* rows, int P, float* out, int64_t ld, const TopkFuse* fuse) {
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   if (persist) {
-    const size_t smem = sizeof(int) * (size_t)(T + 1);
+    const size_t smem = sizeof(uint32_t) * ((size_t)kHistPadded + T + 1);
+    uint32_t* hist = fuse ? fuse->hist : nullptr;
+    uint32_t* rec = fuse ? fuse->rec : nullptr;
+    const int topk = fuse ? fuse->topk : 0;
     if (gather) {
       cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(qb, w, kb, k_seq_stride, n, heads, h,
-                                                                                H_I, L, T, rows, P, out, ld);
+      score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, hist, rec, topk);
     } else {
       cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(qb, w, kb, k_seq_stride, n, heads,
-                                                                                 h, H_I, L, T, rows, P, out, ld);
+      score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, hist, rec, topk);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
@@ -335,12 +385,12 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
 
 }  // namespace
 
-void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h, const int32_t* rows,
-                   int P, float* out, int64_t ld, cudaStream_t s) {
-  if (T <= 0) return;
+                   int P, float* out, int64_t ld, const TopkFuse* fuse, cudaStream_t s) {
+  if (T <= 0) return false;
   const int npos = rows ? P : L;
-  if (npos <= 0) return;
+  if (npos <= 0) return false;
   const bool gather = rows != nullptr;
   if (dt == DType::F32) {
     const dim3 grid((npos + kRowsPerChunk - 1) / kRowsPerChunk, T);
@@ -357,6 +407,7 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
           static_cast<const float*>(q), w, static_cast<const float*>(k), k_seq_stride, n, heads, h, H_I, L, rows,
           P, out, ld);
     }
+    return false;
   } else {
     const int m = heads ? h : H_I;
     const int ng = (m + 7) / 8;
@@ -365,7 +416,7 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
     switch (ng) {
 #define MISA_NG_CASE(NGV)                                                                                  \
   case NGV:                                                                                                \
-    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld); \
+    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld, fuse); \
     break;
       MISA_NG_CASE(1)
       MISA_NG_CASE(2)
@@ -387,6 +438,7 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
       default:
         break;
     }
+    return persist && fuse != nullptr;
   }
 }
 

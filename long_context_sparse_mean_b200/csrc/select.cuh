@@ -59,6 +59,54 @@ __device__ __forceinline__ Bucket block_bucket_bits(const uint32_t* hist, int nb
   return r;
 }
 
+// Shared-memory index of bin b in a padded histogram: one extra word per 16 bins, so threads that
+// each read 16 contiguous bins hit different banks.
+__device__ __forceinline__ int hpad(int b) { return b + (b >> 4); }
+constexpr int kHistPadded = kHistBins + kHistBins / 16;
+
+// Bucket search over a padded shared histogram of kHistBins bins (key bits 31..20): each thread
+// owns kHistBins / blockDim contiguous bins (at most 16), read without bank conflicts.
+__device__ __forceinline__ Bucket bucket_search_padded(const uint32_t* hp, uint32_t need, uint32_t* scratch) {
+  const int per = kHistBins / (int)blockDim.x;
+  uint32_t local = 0;
+  for (int d = 0; d < per; ++d) local += hp[hpad(kHistBins - 1 - ((int)threadIdx.x * per + d))];
+  uint32_t total;
+  uint32_t cum = block_exclusive_scan(local, scratch, &total);
+  for (int d = 0; d < per; ++d) {
+    const int b = kHistBins - 1 - ((int)threadIdx.x * per + d);
+    const uint32_t hb = hp[hpad(b)];
+    if (cum < need && cum + hb >= need) {
+      scratch[32] = (uint32_t)b << 20;
+      scratch[33] = need - cum;
+      scratch[34] = hb;
+    }
+    cum += hb;
+  }
+  __syncthreads();
+  const Bucket r{scratch[32], scratch[33], scratch[34]};
+  __syncthreads();
+  return r;
+}
+
+// Level-0 boundary of one row from its complete global histogram hist_t[kHistBins]: returns
+// (prefix of the bucket holding the k-th largest key, keys still needed from it).  With fewer
+// than k counted keys every key is taken; with none the prefix is 0xffffffff.  hp: padded
+// shared scratch of kHistPadded words.  Every thread of the block must call it.
+__device__ __forceinline__ Bucket level0_boundary(const uint32_t* hist_t, uint32_t topk, uint32_t* hp,
+                                                  uint32_t* scratch) {
+  uint32_t local = 0;
+  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) {
+    const uint32_t v = __ldcg(hist_t + b);
+    hp[hpad(b)] = v;
+    local += v;
+  }
+  uint32_t total;
+  block_exclusive_scan(local, scratch, &total);  // also orders the stores above
+  const uint32_t need = min(topk, total);
+  if (need == 0) return Bucket{0xffffffffu, 0u, 0u};
+  return bucket_search_padded(hp, need, scratch);
+}
+
 __device__ __forceinline__ Bucket block_bucket(const uint32_t* hist, int lvl, uint32_t prefix, uint32_t need,
                                                uint32_t* scratch) {
   return block_bucket_bits(hist, level_bins(lvl), level_shift(lvl), prefix, need, scratch);

@@ -5,21 +5,17 @@
 // scores; "Hierarchical Variant (MISA-dagger)": the k' candidates are narrowed to the top-k by
 // their dense scores.  Rule: score descending, exact ties to the lower token id (select.cuh).
 //
-// Rows of scores (one per query; a position p is token p, or token ids[p] for candidate lists)
-// are selected by a radix cascade over the order keys, every pass reading the rows from L2 with
-// wide loads, 4096 positions per CTA:
-//   1. level-0 pass: 4096-bucket histogram of key bits 31..20 per row; the last CTA of a row to
-//      finish (a counter per row) finds the bucket holding the k-th key and how many keys above it
-//      are taken;
-//   2. level-1 pass: histogram of bits 19..8 of the keys in that bucket; again the last CTA of the
-//      row fixes the 24-bit boundary prefix;
-//   3. partition: keys above the boundary are written out directly (slots reserved with one atomic
-//      per CTA), keys on the boundary prefix go to a short (key, id) list;
-//   4. resolve: one CTA per row ranks that list on the last 8 key bits and, for exact ties, on the
-//      token id, in shared memory (straight from global memory if the list is too long).
-// Clustered scores put about half of a 131072-key row in one level-0 bucket, which is why the
-// cascade has two histogram levels before the partition.  The selected set is exact; its order in
-// the output is not specified.
+// Rows of scores (one per query; a position p is token p, or token ids[p] for candidate lists):
+//   1. level-0 histogram: 4096 buckets of key bits 31..20 per row, and the bucket holding the k-th
+//      key.  The decode scoring kernel builds both while it writes the scores (the CTA that
+//      finishes a row's last tile finds the bucket); otherwise hist_pass_kernel does, with the
+//      same last-CTA rule, in a pass over the rows;
+//   2. partition: keys above the bucket are written out directly (slots reserved with one atomic
+//      per CTA), the bucket's keys go to a (key, id) list;
+//   3. resolve: one CTA per row ranks that list on the remaining 20 key bits and, for exact ties,
+//      on the token id, in shared memory (straight from global memory if the list is too long).
+// On the decode workloads the boundary bucket holds about a tenth of a row.  The selected set is
+// exact; its order in the output is not specified.
 // select_small_kernel ranks a short candidate list entirely in one CTA's shared memory; it needs
 // no workspace (used by the entry point without allocation).
 #include "kernels.cuh"
@@ -30,23 +26,24 @@ namespace misa {
 namespace {
 
 constexpr int kPassThreads = 256;
-constexpr int kPassItems = 16;                         // positions per thread
-constexpr int kPassChunk = kPassThreads * kPassItems;  // positions per CTA
-constexpr int kResolveThreads = 256;
-constexpr int kResolveSmemItems = 8192;  // boundary pairs ranked in shared memory
+constexpr int kRowItems = 16;   // positions per thread for score rows (4096 per CTA)
+constexpr int kListItems = 4;   // for candidate lists (1024 per CTA: more CTAs on short lists)
+constexpr int kResolveSmemItems = 24576;  // boundary pairs ranked in shared memory (192 KB)
 constexpr int kSmallThreads = 1024;
 constexpr int kRec = 8;  // words of per-row state
 
-// Per-row state rec[t][kRec]:
-//   0: level-0 CTAs finished   1: level-1 CTAs finished
-//   2: level-0 prefix (bits 31..20)   3: keys still needed inside the level-0 bucket
-//   4: 24-bit boundary prefix (bits 31..8)   5: keys still needed on the boundary prefix
+// Per-row state rec[t][kRec] (kRec and the meaning of words 0, 2, 3 are shared with the scoring
+// kernel that builds the histogram):
+//   0: tiles or CTAs that have added to the histogram
+//   2: level-0 boundary prefix (bits 31..20; 0xffffffff: no valid key)   3: keys needed from it
 //   6: slots filled by keys above the boundary   7: boundary pairs written
 
 __device__ __forceinline__ int padded(int e) { return e + (e >> 5); }
 
-// The row positions handled by one thread of a pass CTA: 4 groups of 4 consecutive positions.
+// The row positions handled by one thread of a pass CTA: ITEMS/4 groups of 4 consecutive positions.
+template <int ITEMS>
 struct RowSlice {
+  static constexpr int kChunk = kPassThreads * ITEMS;
   const float* row;
   const int32_t* ids;  // null: token = position
   int s1, nt;
@@ -54,9 +51,9 @@ struct RowSlice {
   __device__ int pos(int base, int item) const {
     return base + 4 * ((int)threadIdx.x + (item >> 2) * kPassThreads) + (item & 3);
   }
-  __device__ void load(int base, float (&v)[kPassItems], uint32_t (&key)[kPassItems], bool (&ok)[kPassItems]) const {
+  __device__ void load(int base, float (&v)[ITEMS], uint32_t (&key)[ITEMS], bool (&ok)[ITEMS]) const {
 #pragma unroll
-    for (int j = 0; j < kPassItems / 4; ++j) {
+    for (int j = 0; j < ITEMS / 4; ++j) {
       const int s = pos(base, 4 * j);
       if (vec && s + 3 < s1) {
         const float4 x = __ldcg(reinterpret_cast<const float4*>(row + s));
@@ -70,7 +67,7 @@ struct RowSlice {
       }
     }
 #pragma unroll
-    for (int i = 0; i < kPassItems; ++i) {
+    for (int i = 0; i < ITEMS; ++i) {
       const int s = pos(base, i);
       bool in = s < s1;
       if (in && ids) {
@@ -84,72 +81,54 @@ struct RowSlice {
   __device__ int32_t token(int p) const { return ids ? ids[p] : p; }
 };
 
-// Histogram pass of level LVL (0: bits 31..20 of all keys; 1: bits 19..8 of the keys in the
-// level-0 bucket); the row's last CTA turns the histogram into a boundary.
-template <int LVL>
+// Level-0 histogram pass; the row's last CTA turns the histogram into the boundary.
+template <int ITEMS>
 __global__ void __launch_bounds__(kPassThreads) hist_pass_kernel(const float* __restrict__ scores, int64_t ld,
                                                                  const int32_t* __restrict__ ids, int P,
                                                                  const int32_t* __restrict__ n, int L, int topk,
                                                                  uint32_t* __restrict__ hist, uint32_t* __restrict__ rec) {
-  __shared__ uint32_t h[kHistBins];
+  __shared__ uint32_t h[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ int last;
   const int t = blockIdx.y;
   const int nt = clamp_len(n[t], L);
   const int npos = ids ? P : nt;
   if (!ids && npos <= topk) return;  // the whole prefix is selected
-  const int nchunks = (npos + kPassChunk - 1) / kPassChunk;
-  const int base = blockIdx.x * kPassChunk;
+  constexpr int kChunk = RowSlice<ITEMS>::kChunk;
+  const int nchunks = (npos + kChunk - 1) / kChunk;
+  const int base = blockIdx.x * kChunk;
   if (base >= npos) return;
   uint32_t* rt = rec + (int64_t)t * kRec;
   uint32_t* ht = hist + (int64_t)t * kHistBins;
-  for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) h[b] = 0;
-  const RowSlice rs{scores + (int64_t)t * ld, ids ? ids + (int64_t)t * P : nullptr, min(base + kPassChunk, npos), nt,
-                    (ld % 4) == 0};
-  float v[kPassItems];
-  uint32_t key[kPassItems];
-  bool ok[kPassItems];
+  for (int b = threadIdx.x; b < kHistPadded; b += kPassThreads) h[b] = 0;
+  const RowSlice<ITEMS> rs{scores + (int64_t)t * ld, ids ? ids + (int64_t)t * P : nullptr, min(base + kChunk, npos),
+                           nt, (ld % 4) == 0};
+  float v[ITEMS];
+  uint32_t key[ITEMS];
+  bool ok[ITEMS];
   rs.load(base, v, key, ok);
-  const uint32_t top0 = LVL == 1 ? (__ldcg(rt + 2) >> 20) : 0u;
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < kPassItems; ++i) {
-    const bool in = ok[i] && (LVL == 0 || (key[i] >> 20) == top0);
-    hist_add(h, LVL == 0 ? key[i] >> 20 : (key[i] >> 8) & 4095u, in);
-  }
+  for (int i = 0; i < ITEMS; ++i) hist_add(h, (uint32_t)hpad((int)(key[i] >> 20)), ok[i]);
   __syncthreads();
   for (int b = threadIdx.x; b < kHistBins; b += kPassThreads)
-    if (h[b]) atomicAdd(ht + b, h[b]);
-  __threadfence();
+    if (h[hpad(b)]) atomicAdd(ht + b, h[hpad(b)]);
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(rt + LVL, 1u) == (uint32_t)(nchunks - 1);
+  if (threadIdx.x == 0) {
+    __threadfence();  // cumulative: orders the whole CTA's adds before the count
+    last = atomicAdd(rt, 1u) == (uint32_t)(nchunks - 1);
+  }
   __syncthreads();
   if (!last) return;
   __threadfence();
-  for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) h[b] = __ldcg(ht + b);
-  __syncthreads();
-  if (LVL == 0) {
-    // with a candidate list fewer than k keys may be valid: then all of them are taken
-    uint32_t local = 0;
-    for (int b = threadIdx.x; b < kHistBins; b += kPassThreads) local += h[b];
-    uint32_t total;
-    block_exclusive_scan(local, scratch, &total);
-    const uint32_t need = min((uint32_t)topk, total);
-    const Bucket bk = block_bucket_bits(h, kHistBins, 20, 0u, need, scratch);
-    if (threadIdx.x == 0) {
-      rt[2] = need ? bk.prefix : 0xffffffffu;
-      rt[3] = need ? bk.need : 0u;
-    }
-  } else {
-    const uint32_t need = __ldcg(rt + 3);
-    const Bucket bk = block_bucket_bits(h, kHistBins, 8, __ldcg(rt + 2), need, scratch);
-    if (threadIdx.x == 0) {
-      rt[4] = need ? bk.prefix : 0xffffffffu;
-      rt[5] = need ? bk.need : 0u;
-    }
+  const Bucket bk = level0_boundary(ht, (uint32_t)topk, h, scratch);
+  if (threadIdx.x == 0) {
+    rt[2] = bk.prefix;
+    rt[3] = bk.need;
   }
 }
 
+template <int ITEMS>
 __global__ void __launch_bounds__(kPassThreads) partition_kernel(const float* __restrict__ scores, int64_t ld,
                                                                  const int32_t* __restrict__ ids, int P,
                                                                  const int32_t* __restrict__ n, int L, int topk,
@@ -172,22 +151,23 @@ __global__ void __launch_bounds__(kPassThreads) partition_kernel(const float* __
     }
     return;
   }
-  const int base = blockIdx.x * kPassChunk;
+  constexpr int kChunk = RowSlice<ITEMS>::kChunk;
+  const int base = blockIdx.x * kChunk;
   if (base >= npos) return;
   uint32_t* rt = rec + (int64_t)t * kRec;
-  const uint32_t b24 = __ldcg(rt + 4);
-  const bool none = b24 == 0xffffffffu;  // no valid key at all
-  const uint32_t prefix = b24 >> 8;
-  const RowSlice rs{row, ids ? ids + (int64_t)t * P : nullptr, min(base + kPassChunk, npos), nt, (ld % 4) == 0};
-  float v[kPassItems];
-  uint32_t key[kPassItems];
-  bool ok[kPassItems];
+  const uint32_t b0 = __ldcg(rt + 2);
+  const bool none = b0 == 0xffffffffu;  // no valid key at all
+  const uint32_t prefix = b0 >> 20;
+  const RowSlice<ITEMS> rs{row, ids ? ids + (int64_t)t * P : nullptr, min(base + kChunk, npos), nt, (ld % 4) == 0};
+  float v[ITEMS];
+  uint32_t key[ITEMS];
+  bool ok[ITEMS];
   rs.load(base, v, key, ok);
   uint32_t gtm = 0, eqm = 0;
 #pragma unroll
-  for (int i = 0; i < kPassItems; ++i) {
-    gtm |= (uint32_t)(!none && ok[i] && (key[i] >> 8) > prefix) << i;
-    eqm |= (uint32_t)(!none && ok[i] && (key[i] >> 8) == prefix) << i;
+  for (int i = 0; i < ITEMS; ++i) {
+    gtm |= (uint32_t)(!none && ok[i] && (key[i] >> 20) > prefix) << i;
+    eqm |= (uint32_t)(!none && ok[i] && (key[i] >> 20) == prefix) << i;
   }
   uint32_t tg, te;
   uint32_t pg = block_exclusive_scan(__popc(gtm), scratch, &tg);
@@ -201,7 +181,7 @@ __global__ void __launch_bounds__(kPassThreads) partition_kernel(const float* __
   pe += basev[1];
   uint2* pt = pairs + (int64_t)t * pairs_ld;
 #pragma unroll
-  for (int i = 0; i < kPassItems; ++i) {
+  for (int i = 0; i < ITEMS; ++i) {
     const int p = rs.pos(base, i);
     if ((gtm >> i) & 1u) {
       if (pg < (uint32_t)topk) {
@@ -225,7 +205,8 @@ struct PairList {
 
 // One CTA per row: slots [n_out, n_out + need) come from the boundary pairs; the rest of the row
 // after the selection is padded with -1.
-__global__ void __launch_bounds__(kResolveThreads) resolve_kernel(const int32_t* __restrict__ n, int L, bool lists,
+template <int NT>
+__global__ void __launch_bounds__(NT) resolve_kernel(const int32_t* __restrict__ n, int L, bool lists,
                                                                   int topk, const uint32_t* __restrict__ rec,
                                                                   const uint2* __restrict__ pairs, int64_t pairs_ld,
                                                                   int32_t* __restrict__ idx,
@@ -239,30 +220,30 @@ __global__ void __launch_bounds__(kResolveThreads) resolve_kernel(const int32_t*
   const uint32_t* rt = rec + (int64_t)t * kRec;
   const uint32_t n_out = min(__ldcg(rt + 6), (uint32_t)topk);
   const int c = (int)min(__ldcg(rt + 7), (uint32_t)pairs_ld);
-  const uint32_t need = min(__ldcg(rt + 5), (uint32_t)c);
-  const uint32_t prefix = __ldcg(rt + 4);
+  const uint32_t need = min(__ldcg(rt + 3), (uint32_t)c);
+  const uint32_t prefix = __ldcg(rt + 2);
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
   const uint2* pt = pairs + (int64_t)t * pairs_ld;
   const uint32_t kk = min((uint32_t)topk, n_out + need);
   if ((uint32_t)c <= need) {
-    for (int i = threadIdx.x; i < c; i += kResolveThreads)
+    for (int i = threadIdx.x; i < c; i += NT)
       if (n_out + i < (uint32_t)topk) {
         oi[n_out + i] = (int32_t)pt[i].y;
         if (ov) ov[n_out + i] = key_to_float(pt[i].x);
       }
   } else if (c <= kResolveSmemItems) {
-    for (int i = threadIdx.x; i < c; i += kResolveThreads) list[i] = pt[i];
+    for (int i = threadIdx.x; i < c; i += NT) list[i] = pt[i];
     __syncthreads();
     const PairList acc{list};
-    const SelectResult r = radix_select_items(acc, c, need, 2, prefix, 0xffffff00u, hist, scratch);
+    const SelectResult r = radix_select_items(acc, c, need, 1, prefix, 0xfff00000u, hist, scratch);
     write_selection(acc, c, r, false, oi + n_out, ov ? ov + n_out : nullptr, need, scratch);
   } else {
     const PairList acc{pt};
-    const SelectResult r = radix_select_items(acc, c, need, 2, prefix, 0xffffff00u, hist, scratch);
+    const SelectResult r = radix_select_items(acc, c, need, 1, prefix, 0xfff00000u, hist, scratch);
     write_selection(acc, c, r, false, oi + n_out, ov ? ov + n_out : nullptr, need, scratch);
   }
-  for (int a = (int)kk + threadIdx.x; a < topk; a += kResolveThreads) {
+  for (int a = (int)kk + threadIdx.x; a < topk; a += NT) {
     oi[a] = -1;
     if (ov) ov[a] = 0.f;
   }
@@ -319,27 +300,60 @@ __global__ void __launch_bounds__(kSmallThreads) select_small_kernel(const float
 
 }  // namespace
 
-// Workspace of one selection: hist0 [T][4096], hist1 [T][4096], rec [T][8], pairs [T][P] (uint2).
+// Workspace of one selection: hist [T][4096], rec [T][kRec], pairs [T][P] (uint2).
 size_t topk_rows_ws(int T, int P) {
-  return sizeof(uint32_t) * (2 * (size_t)kHistBins + kRec) * (size_t)T + sizeof(uint2) * (size_t)T * P;
+  return sizeof(uint32_t) * ((size_t)kHistBins + kRec) * (size_t)T + sizeof(uint2) * (size_t)T * P;
+}
+
+void topk_rows_prepare(void* ws, int T, cudaStream_t s) {
+  if (T > 0) cudaMemsetAsync(ws, 0, sizeof(uint32_t) * ((size_t)kHistBins + kRec) * (size_t)T, s);
+}
+
+TopkFuse topk_rows_fuse(void* ws, int T, int topk) {
+  uint32_t* hist = static_cast<uint32_t*>(ws);
+  return TopkFuse{hist, hist + (size_t)kHistBins * T, topk};
+}
+
+void launch_topk_level0(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
+                        int topk, void* ws, cudaStream_t s) {
+  if (T <= 0) return;
+  const int npos = ids ? P : L;
+  uint32_t* hist = static_cast<uint32_t*>(ws);
+  uint32_t* rec = hist + (size_t)kHistBins * T;
+  topk_rows_prepare(ws, T, s);
+  if (ids) {
+    constexpr int C = RowSlice<kListItems>::kChunk;
+    hist_pass_kernel<kListItems><<<dim3((npos + C - 1) / C, T), kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk,
+                                                                                      hist, rec);
+  } else {
+    constexpr int C = RowSlice<kRowItems>::kChunk;
+    hist_pass_kernel<kRowItems><<<dim3((npos + C - 1) / C, T), kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk,
+                                                                                     hist, rec);
+  }
 }
 
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
-                      int topk, void* ws, int32_t* idx, float* score_opt, cudaStream_t s) {
+                      int topk, void* ws, bool hist_ready, int32_t* idx, float* score_opt, cudaStream_t s) {
   if (T <= 0) return;
   const int npos = ids ? P : L;
-  uint32_t* hist0 = static_cast<uint32_t*>(ws);
-  uint32_t* hist1 = hist0 + (size_t)kHistBins * T;
-  uint32_t* rec = hist1 + (size_t)kHistBins * T;
+  uint32_t* hist = static_cast<uint32_t*>(ws);
+  uint32_t* rec = hist + (size_t)kHistBins * T;
   uint2* pairs = reinterpret_cast<uint2*>(rec + (size_t)kRec * T);  // 8-byte aligned: even word count
-  cudaMemsetAsync(ws, 0, sizeof(uint32_t) * (2 * (size_t)kHistBins + kRec) * (size_t)T, s);
-  const dim3 grid((npos + kPassChunk - 1) / kPassChunk, T);
-  hist_pass_kernel<0><<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, hist0, rec);
-  hist_pass_kernel<1><<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, hist1, rec);
-  partition_kernel<<<grid, kPassThreads, 0, s>>>(scores, ld, ids, P, n, L, topk, rec, pairs, npos, idx, score_opt);
+  if (!hist_ready) launch_topk_level0(scores, ld, ids, P, n, T, L, topk, ws, s);
   const size_t smem = sizeof(uint2) * (size_t)kResolveSmemItems;
-  cudaFuncSetAttribute(resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  resolve_kernel<<<T, kResolveThreads, smem, s>>>(n, L, ids != nullptr, topk, rec, pairs, npos, idx, score_opt);
+  if (ids) {
+    constexpr int C = RowSlice<kListItems>::kChunk;
+    partition_kernel<kListItems><<<dim3((npos + C - 1) / C, T), kPassThreads, 0, s>>>(
+        scores, ld, ids, P, n, L, topk, rec, pairs, npos, idx, score_opt);
+    cudaFuncSetAttribute(resolve_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    resolve_kernel<256><<<T, 256, smem, s>>>(n, L, true, topk, rec, pairs, npos, idx, score_opt);
+  } else {
+    constexpr int C = RowSlice<kRowItems>::kChunk;
+    partition_kernel<kRowItems><<<dim3((npos + C - 1) / C, T), kPassThreads, 0, s>>>(
+        scores, ld, ids, P, n, L, topk, rec, pairs, npos, idx, score_opt);
+    cudaFuncSetAttribute(resolve_kernel<1024>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    resolve_kernel<1024><<<T, 1024, smem, s>>>(n, L, false, topk, rec, pairs, npos, idx, score_opt);
+  }
 }
 
 size_t topk_cand_smem(int P) { return sizeof(uint32_t) * 2 * (size_t)(P + P / 32 + 2); }

@@ -58,15 +58,15 @@ def test_workspace_sizes(lib):
     ws = lib.misa_workspace_bytes
     # router: [T,128] partial-block means + [T, ceil(ceil(L/B)/64), H_I] tile sums + [T] counters
     assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256
-    # top-k select: two [T, 4096] histograms, [T, 8] row state, [T, L] boundary (key, id) pairs
-    sel = _al(32 * (2 * 4096 + 8) * 4 + 32 * 131072 * 8)
+    # top-k select: [T, 4096] histogram, [T, 8] row state, [T, L] boundary (key, id) pairs
+    sel = _al(32 * (4096 + 8) * 4 + 32 * 131072 * 8)
     assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel
     # scoring + top-k: [T, ceil4(L)] scores in front of the select workspace
     assert ws(1, 32, 131072, 64, 128, 8, 8192, 0) == 32 * 131072 * 4 + sel
     assert ws(3, 32, 131072, 64, 0, 0, 2048, 0) == 32 * 131072 * 4 + sel
-    assert ws(1, 3, 1001, 64, 1, 8, 10, 0) == _al(3 * 1004 * 4) + _al(3 * 8200 * 4 + 3 * 1001 * 8)
+    assert ws(1, 3, 1001, 64, 1, 8, 10, 0) == _al(3 * 1004 * 4) + _al(3 * 4104 * 4 + 3 * 1001 * 8)
     # re-rank: [T, k'] dense scores + the select workspace over k' positions
-    assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + _al(32 * 8200 * 4 + 32 * 8192 * 8)
+    assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + _al(32 * 4104 * 4 + 32 * 8192 * 8)
     assert ws(1, 0, 100, 64, 1, 8, 10, 0) == 0
 
 
@@ -112,13 +112,20 @@ def test_scoring_and_selection_argument_checks(lib):
     st = lib.misa_score_topk(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, None, FAKE,
                              16, None)
     assert st == WORKSPACE
-    st = lib.misa_token_scores(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, BF16, FAKE, 999, None)
+    st = lib.misa_token_scores(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, BF16, FAKE, 999, 0, None, 0,
+                               None)
     assert st == INVALID  # ld < L
-    st = lib.misa_topk_select(FAKE, 999, FAKE, 4, 1000, 10, FAKE, None, FAKE, 1 << 30, None)
+    st = lib.misa_token_scores(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, BF16, FAKE, 1000, 0, FAKE,
+                               1 << 30, None)
+    assert st == INVALID  # a selection workspace without a k
+    st = lib.misa_token_scores(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 8, BF16, FAKE, 1000, 10, FAKE, 64,
+                               None)
+    assert st == WORKSPACE
+    st = lib.misa_topk_select(FAKE, 999, FAKE, 4, 1000, 10, FAKE, None, FAKE, 1 << 30, 0, None)
     assert st == INVALID
-    st = lib.misa_topk_select(FAKE, 1000, FAKE, 4, 1000, 0, FAKE, None, FAKE, 1 << 30, None)
+    st = lib.misa_topk_select(FAKE, 1000, FAKE, 4, 1000, 0, FAKE, None, FAKE, 1 << 30, 0, None)
     assert st == INVALID
-    st = lib.misa_topk_select(FAKE, 1000, FAKE, 4, 1000, 10, FAKE, None, FAKE, 64, None)
+    st = lib.misa_topk_select(FAKE, 1000, FAKE, 4, 1000, 10, FAKE, None, FAKE, 64, 0, None)
     assert st == WORKSPACE
     st = lib.misa_hier_rerank(FAKE, FAKE, FAKE, 0, FAKE, FAKE, 4, 1000, 64, 128, 100, 200, BF16, FAKE, None, FAKE,
                               1 << 30, None)

@@ -209,3 +209,25 @@ def test_pool_block_range_and_repeatability():
     for t in range(2):
         oa, ob = np.argsort(host(a["idx"])[t]), np.argsort(host(b["idx"])[t])
         assert np.array_equal(host(a["vals"])[t][oa], host(b["vals"])[t][ob])
+
+
+def test_prepared_selection_matches_score_topk():
+    """misa_token_scores leaving the selection's first stage in a workspace, then
+    misa_topk_select(ws_prepared) equals misa_score_topk and the plain selection, for per-query
+    caches (the scoring kernel builds the stage) and a shared cache (a separate pass does)."""
+    L_ = lib()
+    wl, k, q, w = _clustered_small(20000, 6, H_I=64, seed=21, B=128)
+    n = np.array([20000, 19999, 12345, 4097, 2048, 100], np.int32)
+    for shared in (False, True):
+        kk_ = k[0] if shared else k
+        kd, qd = dev(kk_, torch.bfloat16), dev(q, torch.bfloat16)
+        wd, nd = dev(w, torch.float32), dev(n, torch.int32)
+        heads, _ = L_.misa_route(qd, wd, kd, L_.misa_pool_keys(kd, 128), nd, 128, 8)
+        a, _ = L_.misa_score_topk(qd, wd, kd, nd, heads, 3000)
+        ws = L_.Workspace()
+        scores = L_.misa_token_scores(qd, wd, kd, nd, heads, select_topk=3000, select_ws=ws)
+        b, _ = L_.misa_topk_select(scores, nd, 3000, ws=ws, ws_prepared=True)
+        c, _ = L_.misa_topk_select(scores, nd, 3000)
+        for t in range(6):
+            sa, sb, sc = (sorted(host(x)[t].tolist()) for x in (a, b, c))
+            assert sa == sb == sc, (shared, t)
