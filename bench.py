@@ -59,6 +59,18 @@ def _peaks():
     return 6650.0, "fallback"
 
 
+def _tc_peaks():
+    """Dense bf16 tensor-core peaks in TFLOP/s: burst (a kernel timed alone) and sustained (a
+    seconds-long loop under the power cap)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"burst": float(d["bf16_tflops"]), "sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "kind": "measured"}
+    return {"burst": 1590.0, "sustained": 1400.0, "kind": "fallback"}
+
+
 class ClockSampler:
     """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
 
@@ -145,6 +157,26 @@ def cpu_baseline_sample(wl, seqs, threads=None):
     return dt, o.num_threads()
 
 
+def prefill_sample_inputs(wl, count):
+    """The last `count` queries of a shared-cache workload (the longest prefixes) and the cache."""
+    ch = wl.chunk or wl.T
+    c0 = (wl.T - 1) // ch * ch
+    q, w = W.shared_queries(wl, c0, wl.T)
+    n = W.prefix_lengths(wl, c0, wl.T)
+    return W.shared_keys(wl), q[-count:], w[-count:], n[-count:]
+
+
+def cpu_prefill_sample(wl, inputs):
+    """Time the oracle, as it stands, on a few prefill queries: route + routed scores + top-k."""
+    import oracle
+    o = oracle.get()
+    k, q, w, n = inputs
+    t0 = time.perf_counter()
+    o.indexer(oracle.MODE_MISA, q, w, k, 0, n, wl.B, wl.h, wl.topk)
+    dt = time.perf_counter() - t0
+    return dt, o.num_threads(), int(n.astype(np.int64).sum())
+
+
 def run_reference(args):
     """The reference arm: the CPU oracle on a bounded sample of the workload."""
     ws, rank, _ = _dist()
@@ -153,6 +185,8 @@ def run_reference(args):
     wl = _workload(args)
     import oracle
     nthr = oracle.get().num_threads()
+    if wl.n_seq == 1:
+        return run_reference_prefill(args, wl, nthr)
     per_step = max(1, min(wl.T, nthr))
     seqs = list(range(per_step))
     for _ in range(args.warmup):
@@ -178,6 +212,226 @@ def run_reference(args):
     return 0
 
 
+def run_reference_prefill(args, wl, nthr):
+    count = max(1, min(64, 2 * nthr))
+    inputs = prefill_sample_inputs(wl, count)
+    for _ in range(args.warmup):
+        cpu_prefill_sample(wl, inputs)
+    total, units = 0.0, 0
+    for _ in range(args.steps):
+        dt, thr, u = cpu_prefill_sample(wl, inputs)
+        total += dt
+        units += u
+    value = units / total
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1000 * total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+        "config": _config(wl, {"sample_queries_per_step": count}),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
+                         "sample": f"the last {count} of {wl.T} prefill queries per step (prefixes of "
+                                   f"{int(inputs[3].min())}-{int(inputs[3].max())} keys): route + routed scores "
+                                   f"+ top-k, double precision, OpenMP over queries; units = scored "
+                                   f"(query, key) pairs"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _gen_chunk(cid, c):
+    wl = W.WORKLOADS[cid]
+    ch = wl.chunk
+    q, w = W.shared_queries(wl, c * ch, min((c + 1) * ch, wl.T))
+    return q, w
+
+
+def run_prefill(args, wl):
+    """One step = the whole chunked causal prefill of one sequence: pool every block of the shared
+    cache once, then for each chunk of queries route, score with the routed heads on the tensor
+    cores, and select the top-k of every query."""
+    import multiprocessing as mp
+
+    ch = wl.chunk
+    nch = -(-wl.T // ch)
+    with mp.get_context("spawn").Pool(min(nch, max(1, os.cpu_count() or 1))) as pool:
+        parts = pool.starmap(_gen_chunk, [(wl.cid, c) for c in range(nch)])
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = _dist()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+    from long_context_sparse_mean_b200 import binding as M
+
+    k_h = W.shared_keys(wl)
+    n_h = W.prefix_lengths(wl)
+    L, d, T, B, h, kk = wl.L, wl.d, wl.T, wl.B, wl.h, wl.topk
+    kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
+    qd = torch.cat([torch.from_numpy(p[0]).to(torch.bfloat16) for p in parts]).to(dev)
+    wd = torch.cat([torch.from_numpy(p[1]) for p in parts]).to(dev)
+    nd = torch.from_numpy(n_h).to(dev)
+    del parts
+    stream = torch.cuda.current_stream()
+    wsp = M.Workspace(dev)
+    sel_ws = M.Workspace(dev)
+    kbar = M.misa_pool_keys(kd, B)
+    heads = torch.empty((ch, h), dtype=torch.int32, device=dev)
+    scores = torch.empty((ch, L), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+    pairs = int(n_h.astype(np.int64).sum())
+    flops = 2 * h * d * pairs
+    chunks = [(c * ch, min((c + 1) * ch, T)) for c in range(nch)]
+    score_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in chunks]
+    stage_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in chunks]
+    pool_ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+
+    def step(time_scores=False, stages=False):
+        if stages:
+            pool_ev[0].record(stream)
+        M.misa_pool_keys(kd, B, kbar=kbar)
+        if stages:
+            pool_ev[1].record(stream)
+        for c, (a, b) in enumerate(chunks):
+            qc, wc, nc = qd[a:b], wd[a:b], nd[a:b]
+            hc, sc = heads[: b - a], scores[: b - a]
+            if stages:
+                stage_ev[c][0].record(stream)
+            M.misa_route(qc, wc, kd, kbar, nc, B, h, heads=hc, ws=wsp)
+            if stages:
+                stage_ev[c][1].record(stream)
+            if time_scores:
+                score_ev[c][0].record(stream)
+            M.misa_token_scores(qc, wc, kd, nc, hc, out=sc)
+            if time_scores:
+                score_ev[c][1].record(stream)
+            if stages:
+                stage_ev[c][2].record(stream)
+            M.misa_topk_select(sc, nc, kk, idx=idx[a:b], want_vals=False, ws=sel_ws)
+            if stages:
+                stage_ev[c][3].record(stream)
+
+    # launches per step: pool + per chunk (route 1, tensor-core scores 1, selection 3)
+    launches_per_step = 1 + nch * 5
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    score_ms = 0.0
+    nsc = min(args.steps, 5)
+    for _ in range(nsc):
+        step(time_scores=True)
+        torch.cuda.synchronize()
+        score_ms += sum(e0.elapsed_time(e1) for e0, e1 in score_ev)
+    score_ms /= nsc
+    acc = {"pool_all_blocks": 0.0, "route": 0.0, "routed_scores": 0.0, "topk": 0.0}
+    nst = min(args.steps, 5)
+    for _ in range(nst):
+        step(stages=True)
+        torch.cuda.synchronize()
+        acc["pool_all_blocks"] += pool_ev[0].elapsed_time(pool_ev[1])
+        for c in range(nch):
+            e = stage_ev[c]
+            acc["route"] += e[0].elapsed_time(e[1])
+            acc["routed_scores"] += e[1].elapsed_time(e[2])
+            acc["topk"] += e[2].elapsed_time(e[3])
+    stages_us = {k_: round(1000 * v / nst, 1) for k_, v in acc.items()}
+
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            step()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    ms = t0.elapsed_time(t1)
+    if ws > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    value = pairs * ws * args.steps / (ms / 1000.0)
+
+    # end to end: every step copies the cache, the queries, their weights and n from pinned host
+    # memory and reads every query's top-k indices back
+    k_pin = torch.from_numpy(k_h).to(torch.bfloat16).pin_memory()
+    q_pin = qd.cpu().pin_memory()
+    w_pin = wd.cpu().pin_memory()
+    n_pin = torch.from_numpy(n_h).pin_memory()
+    idx_pin = torch.empty((T, kk), dtype=torch.int32).pin_memory()
+    h2d = k_pin.numel() * 2 + q_pin.numel() * 2 + w_pin.numel() * 4 + n_pin.numel() * 4
+    d2h = idx_pin.numel() * 4
+
+    def e2e_step():
+        kd.copy_(k_pin, non_blocking=True)
+        qd.copy_(q_pin, non_blocking=True)
+        wd.copy_(w_pin, non_blocking=True)
+        nd.copy_(n_pin, non_blocking=True)
+        step()
+        idx_pin.copy_(idx, non_blocking=True)
+
+    ne = max(1, min(args.steps, 5))
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(ne):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1)
+    if ws > 1:
+        tt = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    e2e_value = pairs * ws * ne / (e_ms / 1000.0)
+
+    if rank == 0:
+        peaks = _tc_peaks()
+        achieved = flops / (score_ms / 1000.0) / 1e12
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "L": L, "T": T, "chunk": ch, "H_I": wl.H_I, "d": d, "B": B, "h": h,
+                       "topk": kk, "accumulate": "f32", "causal": "n_t = t + 1",
+                       "units": f"scored (query, key) pairs, sum of n_t = {pairs} per step "
+                                f"(T x L = {T * L})",
+                       "l2": f"score rows of one chunk ({ch * L * 4 / 2**30:.1f} GiB) exceed L2; the "
+                             f"16 MiB key cache stays in L2",
+                       "parallelism": f"{ws} GPU(s), one independent sequence per GPU",
+                       "step": "pool all blocks + per chunk: route + routed scores + top-k"},
+            "roofline": {"bound": "tensor", "kernel": "routed token scoring (score_tc_kernel, tcgen05)",
+                         "achieved": achieved, "peak": peaks["sustained"], "peak_kind": peaks["kind"] + " sustained",
+                         "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
+                         "frac_of_burst_peak": achieved / peaks["burst"], "traffic": None,
+                         "algorithmic_flops_per_step": flops, "score_ms_per_step": score_ms},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches_per_step * args.steps,
+            "stages_us": stages_us,
+            "clocks": clk.summary(),
+        }
+        if not args.no_cpu_baseline:
+            count = max(1, min(64, 2 * (os.cpu_count() or 1)))
+            dt, thr, u = cpu_prefill_sample(wl, prefill_sample_inputs(wl, count))
+            line["cpu_baseline"] = {"value": u / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+                                    "sample": f"the last {count} of {T} prefill queries: route + routed scores + "
+                                              f"top-k, double precision, OpenMP over queries"}
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -190,6 +444,8 @@ def run_ours(args):
     from long_context_sparse_mean_b200 import binding as M
 
     wl = _workload(args)
+    if wl.n_seq == 1:
+        raise SystemExit("shared-cache workloads run through run_prefill")
     big = W.small(wl.cid, n_seq=wl.n_seq * ws, T=wl.T * ws)
     seqs = list(range(rank * wl.T, (rank + 1) * wl.T))
     k_h, q_h, w_h, n_h, _ = W.decode_batch(big, seqs)
@@ -373,12 +629,15 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=4, choices=[2, 4, 5])
+    ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    wl = _workload(args)
+    if wl.n_seq == 1:
+        return run_prefill(args, wl)
     return run_ours(args)
 
 

@@ -41,7 +41,8 @@
  *   - Errors: MISA_ERR_INVALID_ARG (null pointer, size out of range), MISA_ERR_UNSUPPORTED
  *     (d != 128, H_I not a multiple of 8, dtype, k' too large), MISA_ERR_WORKSPACE (workspace
  *     too small or misaligned), MISA_ERR_CUDA (a launch failed; cudaGetLastError's code is
- *     consumed).
+ *     consumed).  Errors that arise on the device after a launch are reported by
+ *     misa_device_check.
  */
 #ifndef MISA_H_
 #define MISA_H_
@@ -58,7 +59,8 @@ typedef enum {
   MISA_ERR_INVALID_ARG = 1,
   MISA_ERR_UNSUPPORTED = 2,
   MISA_ERR_WORKSPACE = 3,
-  MISA_ERR_CUDA = 4
+  MISA_ERR_CUDA = 4,
+  MISA_ERR_DEVICE_TIMEOUT = 5
 } misa_status;
 
 typedef enum { MISA_BF16 = 0, MISA_F32 = 1 } misa_dtype;
@@ -178,6 +180,18 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
                            const int32_t* n, int T, int L, int H_I, int d, int topk, int dtype,
                            int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
                            void* stream);
+
+/*
+ * Device-side status of the calls made so far on the current device.  The tensor-core scoring
+ * kernel (queries sharing one bf16 cache: k_seq_stride 0) pipelines its copies and MMAs through
+ * shared-memory barriers; every wait on them is bounded (about one second).  A wait that runs
+ * out makes the kernel stop early, leaving its outputs incomplete, and records the event in a
+ * per-device status word.  This call waits for all work on the device to finish
+ * (cudaDeviceSynchronize), then reads and clears that word.
+ *   returns MISA_OK, MISA_ERR_DEVICE_TIMEOUT (some call since the last check stopped early), or
+ *   MISA_ERR_CUDA (the synchronisation or the read failed).
+ */
+misa_status misa_device_check(void);
 
 /*
  * Capacity, in floats, of the fixed scratch array used by misa_hier_rerank_static

@@ -21,7 +21,7 @@ import torch
 PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libmisa.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA = range(5)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
 BF16, F32 = 0, 1
 OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT = range(5)
 MAX_KP = 16384
@@ -40,6 +40,7 @@ def _setup(lib):
     P, i32, i64, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t
     sigs = {
         "misa_version": ([], i32),
+        "misa_device_check": ([], i32),
         "misa_status_str": ([i32], ctypes.c_char_p),
         "misa_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32, i32], sz),
         "misa_pool_keys": ([P, i64, i32, i32, i32, i32, i32, P, i64, i32, i32, P], i32),
@@ -104,6 +105,12 @@ def _cache_geometry(k: torch.Tensor, T: int):
             raise ValueError(f"per-query cache needs k.shape[0] == T ({T}), got {k.shape[0]}")
         return k.shape[1], k.shape[2], k.shape[1] * k.shape[2]
     raise ValueError("k must be [L, d] or [T, L, d]")
+
+
+def misa_device_check() -> None:
+    """Waits for the device, then raises MisaError if a tensor-core kernel stopped early on a
+    wait that ran out since the last check (its outputs are then incomplete)."""
+    _check("misa_device_check", _lib.misa_device_check())
 
 
 def misa_workspace_bytes(op: int, T: int, L: int, H_I: int, B: int = 1, h: int = 0, topk: int = 0,

@@ -45,7 +45,8 @@ size_t route_ws(int T, int L, int H_I, int B) {
   const size_t pm = align_up(sizeof(float) * (size_t)T * misa::kD);
   const size_t part = align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
   const size_t done = align_up(sizeof(uint32_t) * (size_t)T);
-  return pm + part + done;
+  const size_t parts = align_up(sizeof(uint16_t) * 3 * (size_t)((L + B - 1) / B) * misa::kD);
+  return pm + part + done + parts;
 }
 
 size_t scores_part(int T, int L) { return align_up(sizeof(float) * (size_t)T * score_ld(L)); }
@@ -86,9 +87,19 @@ const char* misa_status_str(int status) {
       return "workspace too small or misaligned";
     case MISA_ERR_CUDA:
       return "CUDA launch failed";
+    case MISA_ERR_DEVICE_TIMEOUT:
+      return "a device-side wait ran out; outputs of some call are incomplete";
     default:
       return "unknown status";
   }
+}
+
+misa_status misa_device_check(void) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return MISA_ERR_CUDA;
+  const int v = misa::read_and_clear_tc_status();
+  const int u = misa::read_and_clear_route_tc_status();
+  if (v < 0 || u < 0) return MISA_ERR_CUDA;
+  return (v || u) ? MISA_ERR_DEVICE_TIMEOUT : MISA_OK;
 }
 
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
@@ -141,8 +152,10 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
   float* partial = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
   uint32_t* done = reinterpret_cast<uint32_t*>(p);
+  p += align_up(sizeof(uint32_t) * (size_t)T);
+  __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(p);
   misa::launch_route(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, T, L, H_I, B, h, heads,
-                     r_opt, pm, partial, done, as_stream(stream));
+                     r_opt, pm, partial, done, parts, as_stream(stream));
   return launch_status();
 }
 

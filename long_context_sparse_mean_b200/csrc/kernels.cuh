@@ -1,6 +1,7 @@
 // Internal launchers of the MISA indexer kernels (C++ linkage; the C ABI lives in capi.cu).
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,10 +15,23 @@ void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L
 
 // Router: partial-block means, per-chunk affinities, then sum, weight and top-h.
 int route_chunks(int L, int B);  // chunks of kRouteTile blocks per query (upper bound)
+// kbar_parts: [3][ceil(L/B)][128] bf16 scratch for the tensor-core router (shared cache).
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
                   int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
-                  uint32_t* done, cudaStream_t s);
+                  uint32_t* done, __nv_bfloat16* kbar_parts, cudaStream_t s);
+
+// Router on the tensor cores for queries that share one bf16 cache and its pooled keys: per-tile
+// sums over full blocks into Sp [T][nch][H_I], then route_finish.  False (nothing launched) when
+// the shapes do not suit it (H_I must divide 128).
+constexpr int kRouteTcMinQueries = 64;
+bool launch_route_tc(const void* q, const float* w, const void* k, const float* kbar, const int32_t* n, int T,
+                     int L, int H_I, int B, int h, int32_t* heads, float* r_opt, __nv_bfloat16* kbar_parts,
+                     float* Sp, int nch, cudaStream_t s);
+void launch_kbar_split(const float* kbar, int M, __nv_bfloat16* parts, cudaStream_t s);
+void launch_route_finish(const __nv_bfloat16* q, const float* w, const __nv_bfloat16* k, const int32_t* n, int T,
+                         int L, int H_I, int B, int h, const float* Sp, int nch, int tile, int32_t* heads,
+                         float* r_opt, cudaStream_t s);
 
 // Level-0 selection state the decode scoring kernel can build while it scores (select.cuh):
 // hist [T][4096] and rec [T][8], both zeroed beforehand (topk_rows_prepare).
@@ -33,6 +47,14 @@ struct TopkFuse {
 bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
                    const int32_t* rows, int P, float* out, int64_t ld, const TopkFuse* fuse, cudaStream_t s);
+
+// Tensor-core scoring for queries sharing one bf16 key cache (k_seq_stride 0, no gather).  Returns
+// false without launching when the inputs do not suit it (alignment, no TMA encoder).
+bool launch_scores_tc(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads, int T,
+                      int L, int H_I, int h, float* out, int64_t ld, cudaStream_t s);
+// Reads and clears the status word the tensor-core kernels set when a bounded wait runs out.
+int read_and_clear_tc_status();
+int read_and_clear_route_tc_status();
 
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
 // or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t)).  ws holds

@@ -16,6 +16,8 @@
 // register tile per thread, then a one-warp-per-query selection kernel.
 #include <cuda_bf16.h>
 
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace misa {
@@ -182,25 +184,11 @@ __device__ __forceinline__ bool head_better(float av, int aj, float bv, int bj) 
   return av > bv || (av == bv && aj < bj);
 }
 
-// One warp: r_j = w_j * (sum of the nc per-tile partial sums, in tile order), then the top-h heads
-// by (r desc, j asc) with warp shuffles.  partial_t is [nch][H_I] for this query.
-__device__ __forceinline__ void select_heads_warp(const float* partial_t, int nc, const float* w_t, int H_I, int h,
-                                                  int32_t* heads_t, float* r_t) {
+// One warp: the top-h heads by (r desc, j asc) with warp shuffles; lane l holds r of heads
+// l + 32 i in v[i], live[i] false past H_I.
+__device__ __forceinline__ void pick_heads_warp(float (&v)[kMaxHeads / 32], bool (&live)[kMaxHeads / 32], int h,
+                                                int32_t* heads_t) {
   const int lane = threadIdx.x & 31;
-  float v[kMaxHeads / 32];
-  bool live[kMaxHeads / 32];
-#pragma unroll
-  for (int i = 0; i < kMaxHeads / 32; ++i) {
-    const int j = lane + 32 * i;
-    live[i] = j < H_I;
-    v[i] = 0.f;
-    if (live[i]) {
-      float s = 0.f;
-      for (int c = 0; c < nc; ++c) s += __ldcg(partial_t + (int64_t)c * H_I + j);
-      v[i] = w_t[j] * s;
-      if (r_t) r_t[j] = v[i];
-    }
-  }
   for (int rnd = 0; rnd < h; ++rnd) {
     float bv = 0.f;
     int bj = 0x7fffffff;
@@ -228,6 +216,28 @@ __device__ __forceinline__ void select_heads_warp(const float* partial_t, int nc
     for (int i = 0; i < kMaxHeads / 32; ++i)
       if (lane + 32 * i == bj) live[i] = false;
   }
+}
+
+// One warp: r_j = w_j * (sum of the nc per-tile partial sums in global memory, in tile order),
+// then the top-h heads.  partial_t is [nch][H_I] for this query.
+__device__ __forceinline__ void select_heads_warp(const float* partial_t, int nc, const float* w_t, int H_I, int h,
+                                                  int32_t* heads_t, float* r_t) {
+  const int lane = threadIdx.x & 31;
+  float v[kMaxHeads / 32];
+  bool live[kMaxHeads / 32];
+#pragma unroll
+  for (int i = 0; i < kMaxHeads / 32; ++i) {
+    const int j = lane + 32 * i;
+    live[i] = j < H_I;
+    v[i] = 0.f;
+    if (live[i]) {
+      float s = 0.f;
+      for (int c = 0; c < nc; ++c) s += __ldcg(partial_t + (int64_t)c * H_I + j);
+      v[i] = w_t[j] * s;
+      if (r_t) r_t[j] = v[i];
+    }
+  }
+  pick_heads_warp(v, live, h, heads_t);
 }
 
 // One warp per query (fp32 path).
@@ -384,7 +394,85 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
   }
 }
 
+// kbar [M, 128] fp32 -> parts [3][M][128] bf16 with kbar = hi + mid + lo to fp32 accuracy (the
+// operands of the tensor-core router for one shared cache).
+__global__ void __launch_bounds__(256) kbar_split_kernel(const float* __restrict__ kbar, int64_t count,
+                                                         __nv_bfloat16* __restrict__ parts) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < count; i += (int64_t)gridDim.x * blockDim.x) {
+    float hi, mid, lo;
+    split3(kbar[i], hi, mid, lo);
+    parts[i] = __float2bfloat16_rn(hi);
+    parts[count + i] = __float2bfloat16_rn(mid);
+    parts[2 * count + i] = __float2bfloat16_rn(lo);
+  }
+}
+
+// One CTA per query, after the tensor-core router's per-tile sums Sp[t][tile][j] over full pooled
+// blocks: adds max(0, q_{t,j} . mean of the partial last block) (keys [floor(n_t/B) B, n_t),
+// averaged here), then r_j = w_j * total and the top-h heads.
+__global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* __restrict__ q,
+                                                           const float* __restrict__ w,
+                                                           const __nv_bfloat16* __restrict__ k,
+                                                           const int32_t* __restrict__ n, int L, int H_I, int B,
+                                                           int h, const float* __restrict__ Sp, int nch,
+                                                           int tile, int32_t* __restrict__ heads,
+                                                           float* __restrict__ r_opt) {
+  __shared__ float part[4][kD];
+  __shared__ __align__(16) float pm[kD];
+  __shared__ float tot[kMaxHeads];
+  const int t = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  const int nf = nt / B, c = nt % B;
+  const int ntiles = (nf + tile - 1) / tile;
+  if (c > 0) {
+    const float m = block_mean_256<DType::BF16>(k, nt - c, nt, part);
+    if (threadIdx.x < kD) pm[threadIdx.x] = m;
+  }
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = warp; j < H_I; j += 8) {
+    float d = 0.f;
+    if (c > 0) {
+      const uint2 x = *reinterpret_cast<const uint2*>(q + ((int64_t)t * H_I + j) * kD + 4 * lane);
+      const float4 p4 = *reinterpret_cast<const float4*>(pm + 4 * lane);
+      d = bf16_lo(x.x) * p4.x + bf16_hi(x.x) * p4.y + bf16_lo(x.y) * p4.z + bf16_hi(x.y) * p4.w;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+    }
+    if (lane == 0) {
+      float sum = 0.f;
+      for (int i = 0; i < ntiles; ++i) sum += __ldcg(Sp + ((int64_t)t * nch + i) * H_I + j);
+      tot[j] = sum + relu(d);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    float v[kMaxHeads / 32];
+    bool live[kMaxHeads / 32];
+#pragma unroll
+    for (int i = 0; i < kMaxHeads / 32; ++i) {
+      const int j = lane + 32 * i;
+      live[i] = j < H_I;
+      v[i] = live[i] ? w[(int64_t)t * H_I + j] * tot[j] : 0.f;
+      if (live[i] && r_opt) r_opt[(int64_t)t * H_I + j] = v[i];
+    }
+    pick_heads_warp(v, live, h, heads + (int64_t)t * h);
+  }
+}
+
 }  // namespace
+
+void launch_kbar_split(const float* kbar, int M, __nv_bfloat16* parts, cudaStream_t s) {
+  const int64_t count = (int64_t)M * kD;
+  const int grid = (int)std::min<int64_t>((count + 255) / 256, 4096);
+  if (count > 0) kbar_split_kernel<<<grid, 256, 0, s>>>(kbar, count, parts);
+}
+
+void launch_route_finish(const __nv_bfloat16* q, const float* w, const __nv_bfloat16* k, const int32_t* n, int T,
+                         int L, int H_I, int B, int h, const float* Sp, int nch, int tile, int32_t* heads,
+                         float* r_opt, cudaStream_t s) {
+  if (T > 0) route_finish_kernel<<<T, 256, 0, s>>>(q, w, k, n, L, H_I, B, h, Sp, nch, tile, heads, r_opt);
+}
 
 void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L, int B, float* kbar,
                  int64_t kbar_seq_stride, int b0, int b1, cudaStream_t s) {
@@ -404,9 +492,13 @@ int route_chunks(int L, int B) {
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L, int H_I,
                   int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial, uint32_t* done,
-                  cudaStream_t s) {
+                  __nv_bfloat16* kbar_parts, cudaStream_t s) {
   if (T <= 0) return;
   const int M = (L + B - 1) / B;
+  // many queries on one shared cache: tensor-core contraction over blocks of queries
+  if (dt == DType::BF16 && k_seq_stride == 0 && kbar_seq_stride == 0 && T >= kRouteTcMinQueries &&
+      launch_route_tc(q, w, k, kbar, n, T, L, H_I, B, h, heads, r_opt, kbar_parts, partial, route_chunks(L, B), s))
+    return;
   if (dt == DType::BF16) {
     const int nch = (M + kRouteMmaTile - 1) / kRouteMmaTile;
     const dim3 grid(nch, T);

@@ -409,6 +409,8 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
     }
     return false;
   } else {
+    // one shared cache: tensor-core contraction over blocks of queries
+    if (!gather && k_seq_stride == 0 && launch_scores_tc(q, w, k, n, heads, T, L, H_I, h, out, ld, s)) return false;
     const int m = heads ? h : H_I;
     const int ng = (m + 7) / 8;
     // persistent schedule for per-query caches and for gathered candidate lists

@@ -1,0 +1,244 @@
+// Blackwell (sm_100a) building blocks in inline PTX: shared-memory mbarriers with bounded waits,
+// TMA tile loads, asynchronous 16-byte copies, and the tcgen05 tensor-memory and MMA
+// instructions (cta_group::1, kind::f16 with fp32 accumulation).
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace misa {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---- mbarriers --------------------------------------------------------------------------------
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Makes the initialised barriers visible to the async proxy (TMA, tcgen05.commit).
+__device__ __forceinline__ void mbar_init_fence() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Arrival without release semantics: orders nothing but the arrival itself (no wait for this
+// thread's earlier global stores); for barriers that only hand back tensor memory.
+__device__ __forceinline__ void mbar_arrive_relaxed(uint32_t bar) {
+  asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// One arrival plus `bytes` of expected transaction count (completed by TMA).
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for completion of the barrier phase with the given parity.  Gives up and returns false
+// once *abort is nonzero (abort may be null) or after limit_ns nanoseconds of waiting.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                          uint64_t limit_ns) {
+  if (mbar_test(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t spin = 1;; ++spin) {
+    if (mbar_test(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if ((spin & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// ---- copies -----------------------------------------------------------------------------------
+
+// 2-D TMA tile load into shared memory; completion is counted in bytes on `bar`.
+// x (innermost coordinate) times the element size must be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+// 16-byte asynchronous global->shared copy; src_bytes < 16 zero-fills the rest.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+// Orders this thread's generic-proxy shared-memory writes before later async-proxy reads.
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// ---- tensor memory and tcgen05 MMA ------------------------------------------------------------
+
+// Warp-wide: allocates ncols TMEM columns (power of two >= 32) and writes the base to [dst].
+__device__ __forceinline__ void tmem_alloc(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor for a K-major operand in the 128-byte swizzled layout: rows of
+// 64 bf16 (128 bytes), 8-row atoms of 1024 bytes stored back to back.  Advancing the start
+// address by 32 bytes moves 16 elements along K inside the atom.
+__device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4)  // start address, 16-byte units
+         | ((uint64_t)1 << 16)                 // leading byte offset (unused with this swizzle)
+         | ((uint64_t)(1024 >> 4) << 32)       // stride byte offset: 8 rows x 128 bytes
+         | ((uint64_t)1 << 46)                 // descriptor version for tcgen05
+         | ((uint64_t)2 << 61);                // 128-byte swizzle
+}
+
+// Instruction descriptor of kind::f16: bf16 A and B (both K-major), fp32 accumulator, M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
+  return (1u << 4)                          // accumulator format fp32
+         | (1u << 7)                        // A format bf16
+         | (1u << 10)                       // B format bf16
+         | ((uint32_t)(N >> 3) << 17)       // N / 8
+         | ((uint32_t)(M >> 4) << 24);      // M / 16
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, issued by one thread.
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives once on `bar` when every MMA this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// Warp-wide: lane l reads 32 consecutive fp32 columns of TMEM lane (taddr.lane + l).
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+      : "r"(taddr));
+}
+
+// Waits for this thread's tcgen05.ld results; the registers are tied in so that no use of them
+// is scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
+               :
+               : "memory");
+}
+
+// ---- persistent schedule over (query block, tile) work -----------------------------------------
+
+// pre[b] = first flattened tile of query block b, pre[NB] = the total, in shared memory: block b
+// (queries [b QB, b QB + QB) of T) needs ceil(max over its queries of len(t) / tile) tiles.
+// len(t) must be >= 0.  Every thread of the block calls it; warp_tot is 32 words of scratch.
+template <class Len>
+__device__ __forceinline__ void block_tile_prefix(int NB, int QB, int T, int tile, Len len, uint32_t* pre,
+                                                  uint32_t* warp_tot) {
+  for (int b = threadIdx.x; b <= NB; b += blockDim.x) pre[b] = 0;
+  __syncthreads();
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const int v = len(t);
+    if (v > 0) atomicMax(pre + t / QB, (uint32_t)v);
+  }
+  __syncthreads();
+  const int per = (NB + (int)blockDim.x - 1) / (int)blockDim.x;
+  const int b0 = (int)threadIdx.x * per, b1 = min(NB, b0 + per);
+  uint32_t local = 0;
+  for (int b = b0; b < b1; ++b) {
+    const uint32_t tiles = (pre[b] + tile - 1) / tile;
+    pre[b] = tiles;
+    local += tiles;
+  }
+  uint32_t total;
+  uint32_t run = block_exclusive_scan(local, warp_tot, &total);
+  for (int b = b0; b < b1; ++b) {
+    const uint32_t x = pre[b];
+    pre[b] = run;
+    run += x;
+  }
+  if (threadIdx.x == 0) pre[NB] = total;
+  __syncthreads();
+}
+
+// Walks the (query block, tile range) segments of the flattened tile range [pos, end).
+struct TileSegments {
+  const uint32_t* pre;
+  int b;
+  uint32_t pos, end;
+  __device__ TileSegments(const uint32_t* pre_, int NB, uint32_t a, uint32_t e) : pre(pre_), pos(a), end(e) {
+    int lo = 0, hi = NB - 1;  // last block with pre[b] <= a
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (pre[mid] <= a) lo = mid;
+      else hi = mid - 1;
+    }
+    b = lo;
+  }
+  __device__ bool next(int& blk, uint32_t& lo, uint32_t& hi) {
+    if (pos >= end) return false;
+    while (pre[b + 1] <= pos) ++b;  // skip blocks without tiles
+    blk = b;
+    lo = pos - pre[b];
+    const uint32_t stop = end < pre[b + 1] ? end : pre[b + 1];
+    hi = stop - pre[b];
+    pos = stop;
+    ++b;
+    return true;
+  }
+};
+
+}  // namespace tc
+}  // namespace misa

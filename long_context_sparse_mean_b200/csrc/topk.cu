@@ -31,6 +31,7 @@ constexpr int kListItems = 4;   // for candidate lists (1024 per CTA: more CTAs 
 constexpr int kResolveSmemItems = 24576;  // boundary pairs ranked in shared memory (192 KB)
 constexpr int kSmallThreads = 1024;
 constexpr int kRec = 8;  // words of per-row state
+constexpr int kRowKernelMinRows = 256;  // from this many rows on, one CTA per row
 
 // Per-row state rec[t][kRec] (kRec and the meaning of words 0, 2, 3 are shared with the scoring
 // kernel that builds the histogram):
@@ -249,6 +250,221 @@ __global__ void __launch_bounds__(NT) resolve_kernel(const int32_t* __restrict__
   }
 }
 
+// ---- one CTA per row, for many rows (prefill chunks) ----------------------------------------
+//
+// A row of n_t scores is read by its CTA (3 CTAs per SM).  The cut comes from a sample: every
+// 16th key, ranked to 22 bits (level-0 bucket, then 10 more bits inside it), at 1.25 x the
+// expected rank of the k-th key plus a margin; one pass appends every key at or above the cut to
+// a shared-memory list (one atomic per warp and step; ~5% of a row), and an exact radix select on
+// the list keeps the top k.  The list holds
+// every selected key whenever it has at least k entries.  Otherwise (too few, or more than the
+// list holds) the row takes the exact path: full level-0 histogram, keys above the boundary
+// bucket written out, the bucket's keys ranked as above (from global memory if they overflow).
+
+constexpr int kRowThreads = 512;
+constexpr int kRowList = 6144;  // (key, id) pairs in shared memory (48 KB): 3 CTAs per SM
+constexpr int kRowSampleStride = 16;
+
+struct SmemPairs {
+  const uint2* p;
+  __device__ uint32_t key(int i) const { return p[i].x; }
+  __device__ uint32_t id(int i) const { return p[i].y; }
+};
+
+// The row in global memory restricted to one level-0 bucket (other keys read as absent).
+struct RowBucket {
+  const float* row;
+  uint32_t prefix;
+  __device__ uint32_t key(int i) const {
+    const uint32_t k = order_key(__ldcg(row + i));
+    return (k & 0xfff00000u) == prefix ? k : 0u;
+  }
+  __device__ uint32_t id(int i) const { return (uint32_t)i; }
+};
+
+// Appends, for every lane whose `take` is set, (key, id) at a slot of the list counted by *cnt
+// (one shared atomic per warp).  Returns the slot (or a value >= cap when the list is full).
+__device__ __forceinline__ void warp_append(bool take, uint32_t key, uint32_t id, uint2* list, int cap,
+                                            uint32_t* cnt) {
+  const unsigned m = __ballot_sync(0xffffffffu, take);
+  if (m == 0u) return;
+  const int lane = threadIdx.x & 31;
+  const int leader = __ffs(m) - 1;
+  uint32_t base = 0;
+  if (lane == leader) base = atomicAdd(cnt, (uint32_t)__popc(m));
+  base = __shfl_sync(0xffffffffu, base, leader);
+  const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+  if (take && pos < (uint32_t)cap) list[pos] = make_uint2(key, id);
+}
+
+// Visits positions [0, nt) of a row, four per step, with all lanes of every warp taking the same
+// number of steps (f gets position, key and a validity flag).
+template <class F>
+__device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&& f) {
+  if (vec) {
+    const int n4 = (nt + 3) / 4;
+    const int steps = (n4 + kRowThreads - 1) / kRowThreads;
+    for (int j = 0; j < steps; ++j) {
+      const int i = j * kRowThreads + (int)threadIdx.x;
+      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (4 * i + 3 < nt) {
+        x = __ldcg(reinterpret_cast<const float4*>(row) + i);
+      } else if (4 * i < nt) {
+        x.x = __ldcg(row + 4 * i);
+        if (4 * i + 1 < nt) x.y = __ldcg(row + 4 * i + 1);
+        if (4 * i + 2 < nt) x.z = __ldcg(row + 4 * i + 2);
+      }
+      const float v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int s = 4 * i + u;
+        f(s, order_key(v[u]), s < nt);
+      }
+    }
+  } else {
+    const int steps = (nt + kRowThreads - 1) / kRowThreads;
+    for (int j = 0; j < steps; ++j) {
+      const int s = j * kRowThreads + (int)threadIdx.x;
+      const float v = s < nt ? __ldcg(row + s) : 0.f;
+      f(s, order_key(v), s < nt);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads, 3) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                 const int32_t* __restrict__ n, int L, int topk,
+                                                                 int32_t* __restrict__ idx,
+                                                                 float* __restrict__ score_opt) {
+  extern __shared__ uint2 list[];  // [kRowList]
+  __shared__ uint32_t hp[kHistPadded];
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t cnt[2];
+  const int t = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  const float* row = scores + (int64_t)t * ld;
+  int32_t* oi = idx + (int64_t)t * topk;
+  float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
+  const int tid = threadIdx.x;
+  if (nt <= topk) {  // every prefix token is selected
+    for (int a = tid; a < topk; a += kRowThreads) {
+      oi[a] = a < nt ? a : -1;
+      if (ov) ov[a] = a < nt ? row[a] : 0.f;
+    }
+    return;
+  }
+  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  uint32_t kk = 0;  // slots filled
+
+  // ---- sampled cut and candidate list ----
+  bool exact = nt <= 4 * topk;
+  if (!exact) {
+    for (int b = tid; b < kHistPadded; b += kRowThreads) hp[b] = 0;
+    if (tid < 2) cnt[tid] = 0;
+    __syncthreads();
+    const int ns = (nt + kRowSampleStride - 1) / kRowSampleStride;
+    for (int i = tid; i < ns; i += kRowThreads) {
+      const uint32_t k = order_key(__ldcg(row + (int64_t)i * kRowSampleStride));
+      hist_add(hp, (uint32_t)hpad((int)(k >> 20)), k != 0u);
+    }
+    uint32_t local = 0;
+    __syncthreads();
+    for (int b = tid; b < kHistBins; b += kRowThreads) local += hp[hpad(b)];
+    uint32_t total;
+    block_exclusive_scan(local, scratch, &total);
+    const uint32_t rank = (uint32_t)((int64_t)topk * 5 * ns / (4 * (int64_t)nt)) + 32u;
+    if (total < rank) {
+      exact = true;
+    } else {
+      // cut at the rank-th sample key, to 22 bits: its level-0 bucket, then 10 more bits
+      const Bucket cut = bucket_search_padded(hp, rank, scratch);
+      for (int b = tid; b < 1024; b += kRowThreads) hp[b] = 0;
+      __syncthreads();
+      for (int i = tid; i < ns; i += kRowThreads) {
+        const uint32_t k = order_key(__ldcg(row + (int64_t)i * kRowSampleStride));
+        hist_add(hp, (k >> 10) & 1023u, k != 0u && (k & 0xfff00000u) == cut.prefix);
+      }
+      __syncthreads();
+      const Bucket cut2 = block_bucket(hp, 1, cut.prefix, cut.need, scratch);
+      const uint32_t cb = cut2.prefix >> 10;
+      row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
+        warp_append(in && k != 0u && (k >> 10) >= cb, k, (uint32_t)s, list, kRowList, &cnt[0]);
+      });
+      __syncthreads();
+      const uint32_t c = cnt[0];
+      if (c >= (uint32_t)topk && c <= (uint32_t)kRowList) {
+        const SmemPairs acc{list};
+        const SelectResult r = radix_select_items(acc, (int)c, (uint32_t)topk, 0, 0u, 0u, hp, scratch);
+        write_selection(acc, (int)c, r, false, oi, ov, (uint32_t)topk, scratch);
+        return;  // topk < n_t keys: every slot is filled
+      }
+      exact = true;
+      __syncthreads();
+    }
+  }
+
+  // ---- exact path: full level-0 histogram, boundary bucket, rank the bucket ----
+  for (int b = tid; b < kHistPadded; b += kRowThreads) hp[b] = 0;
+  if (tid < 2) cnt[tid] = 0;
+  __syncthreads();
+  row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
+    (void)s;
+    hist_add(hp, (uint32_t)hpad((int)(k >> 20)), in && k != 0u);
+  });
+  __syncthreads();
+  uint32_t local = 0;
+  for (int b = tid; b < kHistBins; b += kRowThreads) local += hp[hpad(b)];
+  uint32_t total;
+  block_exclusive_scan(local, scratch, &total);
+  const uint32_t want = min((uint32_t)topk, total);
+  if (want > 0) {
+    const Bucket bk = bucket_search_padded(hp, want, scratch);
+    const uint32_t pb = bk.prefix >> 20;
+    // keys above the bucket straight to the output, the bucket's keys to the list
+    row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
+      const bool ok = in && k != 0u;
+      const bool gt = ok && (k >> 20) > pb;
+      const unsigned m = __ballot_sync(0xffffffffu, gt);
+      if (m) {
+        const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
+        uint32_t base = 0;
+        if (lane == leader) base = atomicAdd(&cnt[1], (uint32_t)__popc(m));
+        base = __shfl_sync(0xffffffffu, base, leader);
+        const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+        if (gt && pos < (uint32_t)topk) {
+          oi[pos] = s;
+          if (ov) ov[pos] = key_to_float(k);
+        }
+      }
+      warp_append(ok && (k >> 20) == pb, k, (uint32_t)s, list, kRowList, &cnt[0]);
+    });
+    __syncthreads();
+    const uint32_t n_gt = min(cnt[1], (uint32_t)topk);
+    const uint32_t c = cnt[0];
+    const uint32_t need = min(bk.need, want - n_gt);
+    if (c <= (uint32_t)kRowList) {
+      const SmemPairs acc{list};
+      if (c <= need) {
+        for (uint32_t i = tid; i < c; i += kRowThreads) {
+          oi[n_gt + i] = (int32_t)list[i].y;
+          if (ov) ov[n_gt + i] = key_to_float(list[i].x);
+        }
+      } else {
+        const SelectResult r = radix_select_items(acc, (int)c, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
+        write_selection(acc, (int)c, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
+      }
+    } else {
+      const RowBucket acc{row, bk.prefix};
+      const SelectResult r = radix_select_items(acc, nt, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
+      write_selection(acc, nt, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
+    }
+    kk = n_gt + need;
+  }
+  for (int a = (int)kk + tid; a < topk; a += kRowThreads) {
+    oi[a] = -1;
+    if (ov) ov[a] = 0.f;
+  }
+}
+
 struct SmemItems {
   const uint32_t* keys;
   const uint32_t* ids;
@@ -335,6 +551,12 @@ void launch_topk_level0(const float* scores, int64_t ld, const int32_t* ids, int
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
                       int topk, void* ws, bool hist_ready, int32_t* idx, float* score_opt, cudaStream_t s) {
   if (T <= 0) return;
+  if (!ids && !hist_ready && T >= kRowKernelMinRows) {  // many rows: one CTA each
+    const size_t smem = sizeof(uint2) * (size_t)kRowList;
+    cudaFuncSetAttribute(row_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    row_topk_kernel<<<T, kRowThreads, smem, s>>>(scores, ld, n, L, topk, idx, score_opt);
+    return;
+  }
   const int npos = ids ? P : L;
   uint32_t* hist = static_cast<uint32_t*>(ws);
   uint32_t* rec = hist + (size_t)kHistBins * T;

@@ -12,7 +12,7 @@ from long_context_sparse_mean_b200 import build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "misa.h")
 
-OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA = range(5)
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT = range(6)
 BF16, F32 = 0, 1
 P = ctypes.c_void_p
 
@@ -34,7 +34,8 @@ def lib():
 def test_header_declares_the_indexer_calls():
     names = declared_functions()
     for want in ("misa_pool_keys", "misa_route", "misa_token_scores", "misa_topk_select", "misa_score_topk",
-                 "misa_hier_rerank", "dsa_dense_topk", "misa_workspace_bytes", "misa_status_str", "misa_version"):
+                 "misa_hier_rerank", "dsa_dense_topk", "misa_workspace_bytes", "misa_status_str", "misa_version",
+                 "misa_device_check"):
         assert want in names, want
 
 
@@ -45,8 +46,8 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings_and_version(lib):
     assert lib.misa_version() >= 100
-    for code in range(5):
-        assert lib.misa_status_str(code)
+    for code in range(6):
+        assert lib.misa_status_str(code) != b"unknown status"
     assert lib.misa_status_str(99) == b"unknown status"
 
 
@@ -57,7 +58,8 @@ def _al(x):
 def test_workspace_sizes(lib):
     ws = lib.misa_workspace_bytes
     # router: [T,128] partial-block means + [T, ceil(ceil(L/B)/64), H_I] tile sums + [T] counters
-    assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256
+    # + [3, ceil(L/B), 128] bf16 parts of the pooled keys
+    assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256 + 3 * 1024 * 128 * 2
     # top-k select: [T, 4096] histogram, [T, 8] row state, [T, L] boundary (key, id) pairs
     sel = _al(32 * (4096 + 8) * 4 + 32 * 131072 * 8)
     assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel
