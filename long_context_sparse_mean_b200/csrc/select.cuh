@@ -112,7 +112,8 @@ __device__ __forceinline__ Bucket block_bucket(const uint32_t* hist, int lvl, ui
   return block_bucket_bits(hist, level_bins(lvl), level_shift(lvl), prefix, need, scratch);
 }
 
-// Radix select over m items given by acc.key(i) (0 = absent) and acc.id(i).  Starts at level
+// Radix select over m items given by acc.key(i) (0 = absent) and acc.id(i); acc.value(i) is the
+// score written out for a selected item.  Starts at level
 // `lvl0` with the boundary prefix/mask already fixed by earlier levels.  On return the selection
 // is: items of class 1 (surely selected) and the first `need` items of class 2 in item order.
 // hist: shared memory of kHistBins words; scratch: 35 words.
@@ -214,7 +215,7 @@ __device__ void write_selection(const Acc& acc, int m, const SelectResult& r, bo
     }
     if (pos < kk) {
       out_id[pos] = (int32_t)acc.id(e);
-      if (out_val) out_val[pos] = key_to_float(acc.key(e));
+      if (out_val) out_val[pos] = acc.value(e);
     }
   }
 }

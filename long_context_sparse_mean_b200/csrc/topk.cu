@@ -202,6 +202,7 @@ struct PairList {
   const uint2* p;
   __device__ uint32_t key(int i) const { return p[i].x; }
   __device__ uint32_t id(int i) const { return p[i].y; }
+  __device__ float value(int i) const { return key_to_float(p[i].x); }
 };
 
 // One CTA per row: slots [n_out, n_out + need) come from the boundary pairs; the rest of the row
@@ -252,23 +253,46 @@ __global__ void __launch_bounds__(NT) resolve_kernel(const int32_t* __restrict__
 
 // ---- one CTA per row, for many rows (prefill chunks) ----------------------------------------
 //
-// A row of n_t scores is read by its CTA (3 CTAs per SM).  The cut comes from a sample: every
-// 16th key, ranked to 22 bits (level-0 bucket, then 10 more bits inside it), at 1.25 x the
-// expected rank of the k-th key plus a margin; one pass appends every key at or above the cut to
-// a shared-memory list (one atomic per warp and step; ~5% of a row), and an exact radix select on
-// the list keeps the top k.  The list holds
-// every selected key whenever it has at least k entries.  Otherwise (too few, or more than the
-// list holds) the row takes the exact path: full level-0 histogram, keys above the boundary
-// bucket written out, the bucket's keys ranked as above (from global memory if they overflow).
+// A row of n_t scores is read once by its CTA (2 CTAs of 512 threads per SM):
+//   1. cut: rows longer than the shared-memory list are sampled (256 evenly spaced runs of 8
+//      scores, 2048 keys); a 4096-bin histogram over the sampled key range places the sample key
+//      whose rank is the expected sample count above the k-th key plus three standard deviations
+//      and a margin, and the lower edge of its bin is the threshold value; shorter rows take every
+//      score;
+//   2. one pass appends (key, position) of every score at or above the threshold to the list
+//      (a bit mask per 32 scores a thread, one warp scan and one shared atomic per warp and
+//      batch; ~5% of a long row) and tracks the smallest and largest key;
+//   3. the list's keys are rewritten relative to the smallest so that they spread over the high
+//      bits (same order); one 4096-bin histogram finds the bucket of the k-th key; keys above it
+//      go straight to the output, the bucket's keys are ranked by one warp (when at most 32) or
+//      on the remaining bits, and, for exact ties, on the position.
+// Whenever the list holds at least k keys it holds every selected key, so the result is exact.
+// Otherwise (fewer than k at or above the cut, or more than the list holds) the row takes the
+// exact path: full level-0 histogram of the row, keys above the boundary bucket written out,
+// the bucket's keys ranked as above (from global memory if they overflow the list).
 
 constexpr int kRowThreads = 512;
-constexpr int kRowList = 6144;  // (key, id) pairs in shared memory (48 KB): 3 CTAs per SM
-constexpr int kRowSampleStride = 16;
+constexpr int kRowList = 8192;          // (key, position) pairs in shared memory (64 KB)
+constexpr int kRowSegments = 256;       // sample runs per long row
+constexpr int kRowSegLen = 8;           // scores per run (one 32-byte sector)
+constexpr int kSweepBatch = 8;          // float4 loads in flight per thread
 
 struct SmemPairs {
   const uint2* p;
   __device__ uint32_t key(int i) const { return p[i].x; }
   __device__ uint32_t id(int i) const { return p[i].y; }
+  __device__ float value(int i) const { return key_to_float(p[i].x); }
+};
+
+// A shared-memory list whose keys were rewritten as 0x80000000 | ((key - lo) << sh): the same
+// order, spread over the high bits.
+struct ShiftedPairs {
+  const uint2* p;
+  uint32_t lo;
+  int sh;
+  __device__ uint32_t key(int i) const { return p[i].x; }
+  __device__ uint32_t id(int i) const { return p[i].y; }
+  __device__ float value(int i) const { return key_to_float(((p[i].x & 0x7fffffffu) >> sh) + lo); }
 };
 
 // The row in global memory restricted to one level-0 bucket (other keys read as absent).
@@ -280,45 +304,53 @@ struct RowBucket {
     return (k & 0xfff00000u) == prefix ? k : 0u;
   }
   __device__ uint32_t id(int i) const { return (uint32_t)i; }
+  __device__ float value(int i) const { return __ldcg(row + i); }
 };
 
-// Appends, for every lane whose `take` is set, (key, id) at a slot of the list counted by *cnt
-// (one shared atomic per warp).  Returns the slot (or a value >= cap when the list is full).
-__device__ __forceinline__ void warp_append(bool take, uint32_t key, uint32_t id, uint2* list, int cap,
-                                            uint32_t* cnt) {
+// Slot for every lane whose `take` is set, counted by *cnt (one shared atomic per warp).
+__device__ __forceinline__ uint32_t warp_slot(bool take, uint32_t* cnt) {
   const unsigned m = __ballot_sync(0xffffffffu, take);
-  if (m == 0u) return;
+  if (m == 0u) return 0u;
   const int lane = threadIdx.x & 31;
   const int leader = __ffs(m) - 1;
   uint32_t base = 0;
   if (lane == leader) base = atomicAdd(cnt, (uint32_t)__popc(m));
   base = __shfl_sync(0xffffffffu, base, leader);
-  const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-  if (take && pos < (uint32_t)cap) list[pos] = make_uint2(key, id);
+  return base + (uint32_t)__popc(m & ((1u << lane) - 1u));
 }
 
 // Visits positions [0, nt) of a row, four per step, with all lanes of every warp taking the same
-// number of steps (f gets position, key and a validity flag).
+// number of steps (f gets position, key and a validity flag).  Loads are issued kSweepBatch steps
+// ahead of their use.  Used by the exact path only.
 template <class F>
 __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&& f) {
   if (vec) {
     const int n4 = (nt + 3) / 4;
     const int steps = (n4 + kRowThreads - 1) / kRowThreads;
-    for (int j = 0; j < steps; ++j) {
-      const int i = j * kRowThreads + (int)threadIdx.x;
-      float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (4 * i + 3 < nt) {
-        x = __ldcg(reinterpret_cast<const float4*>(row) + i);
-      } else if (4 * i < nt) {
-        x.x = __ldcg(row + 4 * i);
-        if (4 * i + 1 < nt) x.y = __ldcg(row + 4 * i + 1);
-        if (4 * i + 2 < nt) x.z = __ldcg(row + 4 * i + 2);
-      }
-      const float v[4] = {x.x, x.y, x.z, x.w};
+    for (int j0 = 0; j0 < steps; j0 += kSweepBatch) {
+      float4 x[kSweepBatch];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int s = 4 * i + u;
-        f(s, order_key(v[u]), s < nt);
+      for (int u = 0; u < kSweepBatch; ++u) {
+        const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
+        x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (4 * i + 3 < nt) {
+          x[u] = __ldcg(reinterpret_cast<const float4*>(row) + i);
+        } else if (4 * i < nt) {
+          x[u].x = __ldcg(row + 4 * i);
+          if (4 * i + 1 < nt) x[u].y = __ldcg(row + 4 * i + 1);
+          if (4 * i + 2 < nt) x[u].z = __ldcg(row + 4 * i + 2);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kSweepBatch; ++u) {
+        if (j0 + u >= steps) break;  // uniform across the block
+        const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
+        const float v[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int s = 4 * i + e;
+          f(s, order_key(v[e]), s < nt);
+        }
       }
     }
   } else {
@@ -331,7 +363,162 @@ __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&
   }
 }
 
-__global__ void __launch_bounds__(kRowThreads, 3) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
+// Appends (key, position) of every position s < nt whose score is >= thr to the list and folds
+// the appended keys into mm[0] (min) and mm[1] (max).  A thread reads 16 positions (4 float4) a
+// step, the next step's loads in flight while it handles the current one, and marks its
+// candidates in a bit mask; one warp scan and one shared atomic per warp and step place them.
+__device__ __forceinline__ void collect_above(const float* row, int nt, bool vec, float thr, uint2* list, int cap,
+                                              uint32_t* cnt, uint32_t* mm) {
+  constexpr int U = 4;  // float4 per thread and step
+  const int lane = threadIdx.x & 31;
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  auto load = [&](int j0, float4 (&x)[U]) {
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
+      x[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      if (vec && 4 * i + 3 < nt) {
+        x[u] = __ldcg(reinterpret_cast<const float4*>(row) + i);
+      } else if (4 * i < nt) {
+        x[u].x = __ldcg(row + 4 * i);
+        if (4 * i + 1 < nt) x[u].y = __ldcg(row + 4 * i + 1);
+        if (4 * i + 2 < nt) x[u].z = __ldcg(row + 4 * i + 2);
+        if (4 * i + 3 < nt) x[u].w = __ldcg(row + 4 * i + 3);
+      }
+    }
+  };
+  const int steps = ((nt + 3) / 4 + kRowThreads - 1) / kRowThreads;  // float4 groups a thread
+  float4 cur[U], nxt[U];
+  load(0, cur);
+  for (int j0 = 0; j0 < steps; j0 += U) {
+    if (j0 + U < steps) load(j0 + U, nxt);
+    uint32_t m = 0;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      m |= (uint32_t)(cur[u].x >= thr) << (4 * u);
+      m |= (uint32_t)(cur[u].y >= thr) << (4 * u + 1);
+      m |= (uint32_t)(cur[u].z >= thr) << (4 * u + 2);
+      m |= (uint32_t)(cur[u].w >= thr) << (4 * u + 3);
+    }
+    const uint32_t c = (uint32_t)__popc(m);
+    uint32_t incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t base = 0;
+    if (lane == 31 && incl) base = atomicAdd(cnt, incl);
+    base = __shfl_sync(0xffffffffu, base, 31);
+    if (m) {
+      uint32_t pos = base + incl - c;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int s0 = 4 * ((j0 + u) * kRowThreads + (int)threadIdx.x);
+        const float v[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          if ((m >> (4 * u + e)) & 1u) {
+            const uint32_t k = order_key(v[e]);
+            lo = min(lo, k);
+            hi = max(hi, k);
+            if (pos < (uint32_t)cap) list[pos] = make_uint2(k, (uint32_t)(s0 + e));
+            ++pos;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) cur[u] = nxt[u];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  if (lane == 0 && hi >= lo) {
+    atomicMin(&mm[0], lo);
+    atomicMax(&mm[1], hi);
+  }
+}
+
+// Ranks n <= 32 entries of list (keys descending, then ids ascending) in one warp and writes the
+// first `need` to oi/ov at their rank.
+template <class Acc>
+__device__ __forceinline__ void warp_rank_write(const uint2* list, int n, uint32_t need, const Acc& acc, int32_t* oi,
+                                                float* ov) {
+  const int lane = threadIdx.x & 31;
+  const bool mine = lane < n;
+  const uint2 e = mine ? list[lane] : make_uint2(0u, 0xffffffffu);
+  uint32_t rank = 0;
+  for (int j = 0; j < n; ++j) {
+    const uint32_t kj = __shfl_sync(0xffffffffu, e.x, j);
+    const uint32_t ij = __shfl_sync(0xffffffffu, e.y, j);
+    rank += (kj > e.x) || (kj == e.x && ij < e.y);
+  }
+  if (mine && rank < need) {
+    oi[rank] = (int32_t)e.y;
+    if (ov) ov[rank] = acc.value(lane);
+  }
+}
+
+// Top `need` of the c list entries (c >= need), keys spread (ShiftedPairs, bit 31 set): written
+// to oi/ov [0, need).  One histogram of key bits 30..19; keys above the boundary bucket go out
+// directly, the bucket's entries move to the front of the list and are ranked (one warp when
+// they are few).  hist: kHistBins words; ctr: 2 words; scratch: 35 words.
+__device__ void select_list(uint2* list, int c, uint32_t need, uint32_t lo, int sh, uint32_t* hist, uint32_t* ctr,
+                            uint32_t* scratch, int32_t* oi, float* ov) {
+  const int tid = threadIdx.x;
+  for (int b = tid; b < kHistBins; b += kRowThreads) hist[b] = 0;
+  if (tid < 2) ctr[tid] = 0;
+  __syncthreads();
+  for (int i = tid; i < c; i += kRowThreads) hist_add(hist, (list[i].x >> 19) & 4095u, true);
+  __syncthreads();
+  const Bucket bk = block_bucket_bits(hist, kHistBins, 19, 0x80000000u, need, scratch);
+  const uint32_t pb = bk.prefix >> 19;
+  const ShiftedPairs acc{list, lo, sh};
+  constexpr int kPer = kRowList / kRowThreads;
+  uint2 keep[kPer];
+  int nk = 0;
+  const int steps = (c + kRowThreads - 1) / kRowThreads;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    if (j >= steps) break;  // uniform
+    const int i = j * kRowThreads + tid;
+    const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
+    const bool gt = i < c && (e.x >> 19) > pb;
+    const uint32_t slot = warp_slot(gt, &ctr[0]);
+    if (gt) {
+      oi[slot] = (int32_t)e.y;
+      if (ov) ov[slot] = acc.value(i);
+    }
+    const bool eq = i < c && (e.x >> 19) == pb;
+    if (eq) keep[nk] = e;
+    nk += eq;
+  }
+  __syncthreads();  // every entry read
+  uint32_t total;
+  const uint32_t off = block_exclusive_scan((uint32_t)nk, scratch, &total);
+  for (int x = 0; x < kPer; ++x)
+    if (x < nk) list[off + x] = keep[x];
+  __syncthreads();
+  const uint32_t n_gt = ctr[0];
+  const uint32_t need2 = need - n_gt;
+  if (total <= need2) {
+    for (uint32_t i = tid; i < total; i += kRowThreads) {
+      oi[n_gt + i] = (int32_t)list[i].y;
+      if (ov) ov[n_gt + i] = acc.value((int)i);
+    }
+  } else if (total <= 32) {
+    if (tid < 32) warp_rank_write(list, (int)total, need2, acc, oi + n_gt, ov ? ov + n_gt : nullptr);
+  } else {
+    const SelectResult r =
+        radix_select_items(acc, (int)total, need2, 1, bk.prefix & 0xfff00000u, 0xfff00000u, hist, scratch);
+    write_selection(acc, (int)total, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need2, scratch);
+  }
+}
+
+__global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
                                                                  const int32_t* __restrict__ n, int L, int topk,
                                                                  int32_t* __restrict__ idx,
                                                                  float* __restrict__ score_opt) {
@@ -339,6 +526,7 @@ __global__ void __launch_bounds__(kRowThreads, 3) row_topk_kernel(const float* _
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t cnt[2];
+  __shared__ uint32_t mm[2];
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
   const float* row = scores + (int64_t)t * ld;
@@ -353,56 +541,89 @@ __global__ void __launch_bounds__(kRowThreads, 3) row_topk_kernel(const float* _
     return;
   }
   const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
-  uint32_t kk = 0;  // slots filled
+  if (tid < 2) cnt[tid] = 0;
+  if (tid == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
 
-  // ---- sampled cut and candidate list ----
-  bool exact = nt <= 4 * topk;
-  if (!exact) {
-    for (int b = tid; b < kHistPadded; b += kRowThreads) hp[b] = 0;
-    if (tid < 2) cnt[tid] = 0;
+  // ---- 1. the cut ----
+  bool exact = false;
+  float thr = -INFINITY;
+  constexpr int ns = kRowSegments * kRowSegLen;
+  // expected sample count above the k-th key, plus three standard deviations and a margin
+  const float mean = (float)topk * (float)ns / (float)nt;
+  const uint32_t rank = (uint32_t)(mean + 3.f * sqrtf(mean) + 8.f);
+  if (nt > kRowList && rank > (uint32_t)ns) {
+    exact = true;  // k close to n_t: the sample cannot place the cut
     __syncthreads();
-    const int ns = (nt + kRowSampleStride - 1) / kRowSampleStride;
-    for (int i = tid; i < ns; i += kRowThreads) {
-      const uint32_t k = order_key(__ldcg(row + (int64_t)i * kRowSampleStride));
-      hist_add(hp, (uint32_t)hpad((int)(k >> 20)), k != 0u);
+  } else if (nt > kRowList) {
+    const int seg = (nt / kRowSegments) & ~(kRowSegLen - 1);  // >= 32 here
+    constexpr int per = ns / kRowThreads;
+    uint32_t sk[per];
+    uint32_t slo = 0xffffffffu, shi = 0u;
+#pragma unroll
+    for (int u = 0; u < per; ++u) {
+      const int i = u * kRowThreads + tid;
+      sk[u] = order_key(__ldcg(row + (int64_t)(i / kRowSegLen) * seg + (i % kRowSegLen)));
+      slo = min(slo, sk[u]);
+      shi = max(shi, sk[u]);
     }
-    uint32_t local = 0;
+    for (int b = tid; b < kHistBins; b += kRowThreads) hp[b] = 0;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      slo = min(slo, __shfl_xor_sync(0xffffffffu, slo, o));
+      shi = max(shi, __shfl_xor_sync(0xffffffffu, shi, o));
+    }
+    __syncthreads();  // mm initialised
+    if ((tid & 31) == 0) {
+      atomicMin(&mm[0], slo);
+      atomicMax(&mm[1], shi);
+    }
     __syncthreads();
-    for (int b = tid; b < kHistBins; b += kRowThreads) local += hp[hpad(b)];
-    uint32_t total;
-    block_exclusive_scan(local, scratch, &total);
-    const uint32_t rank = (uint32_t)((int64_t)topk * 5 * ns / (4 * (int64_t)nt)) + 32u;
-    if (total < rank) {
-      exact = true;
-    } else {
-      // cut at the rank-th sample key, to 22 bits: its level-0 bucket, then 10 more bits
-      const Bucket cut = bucket_search_padded(hp, rank, scratch);
-      for (int b = tid; b < 1024; b += kRowThreads) hp[b] = 0;
-      __syncthreads();
-      for (int i = tid; i < ns; i += kRowThreads) {
-        const uint32_t k = order_key(__ldcg(row + (int64_t)i * kRowSampleStride));
-        hist_add(hp, (k >> 10) & 1023u, k != 0u && (k & 0xfff00000u) == cut.prefix);
-      }
-      __syncthreads();
-      const Bucket cut2 = block_bucket(hp, 1, cut.prefix, cut.need, scratch);
-      const uint32_t cb = cut2.prefix >> 10;
-      row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
-        warp_append(in && k != 0u && (k >> 10) >= cb, k, (uint32_t)s, list, kRowList, &cnt[0]);
-      });
-      __syncthreads();
-      const uint32_t c = cnt[0];
-      if (c >= (uint32_t)topk && c <= (uint32_t)kRowList) {
+    // 4096 bins over the sampled key range
+    slo = mm[0];
+    const uint32_t srange = mm[1] - slo;
+    const int ssh = srange >= 4096u ? 32 - __clz(srange) - 12 : 0;
+#pragma unroll
+    for (int u = 0; u < per; ++u) hist_add(hp, (sk[u] - slo) >> ssh, true);
+    __syncthreads();
+    const Bucket cut = block_bucket_bits(hp, kHistBins, ssh, 0u, rank, scratch);
+    // keys >= slo + cut.prefix are the scores >= this value
+    thr = key_to_float(slo + cut.prefix);
+    if (tid == 0) {
+      mm[0] = 0xffffffffu;
+      mm[1] = 0u;
+    }
+    __syncthreads();
+  } else {
+    __syncthreads();
+  }
+
+  // ---- 2-3. candidates and their selection ----
+  if (!exact) {
+    collect_above(row, nt, vec, thr, list, kRowList, &cnt[0], mm);
+    __syncthreads();
+    const uint32_t c = cnt[0];
+    if (c >= (uint32_t)topk && c <= (uint32_t)kRowList) {
+      const uint32_t lo = mm[0], range = mm[1] - mm[0];
+      const int sh = __clz(range) > 0 ? (range ? __clz(range) - 1 : 31) : 0;
+      if (__clz(range) > 0) {
+        for (uint32_t i = tid; i < c; i += kRowThreads) list[i].x = 0x80000000u | ((list[i].x - lo) << sh);
+        __syncthreads();
+        select_list(list, (int)c, (uint32_t)topk, lo, sh, hp, cnt, scratch, oi, ov);
+      } else {  // the keys span more than half the key range: rank them as they are
         const SmemPairs acc{list};
         const SelectResult r = radix_select_items(acc, (int)c, (uint32_t)topk, 0, 0u, 0u, hp, scratch);
         write_selection(acc, (int)c, r, false, oi, ov, (uint32_t)topk, scratch);
-        return;  // topk < n_t keys: every slot is filled
       }
-      exact = true;
-      __syncthreads();
+      return;  // topk < n_t keys: every slot is filled
     }
+    __syncthreads();
   }
 
   // ---- exact path: full level-0 histogram, boundary bucket, rank the bucket ----
+  uint32_t kk = 0;  // slots filled
   for (int b = tid; b < kHistPadded; b += kRowThreads) hp[b] = 0;
   if (tid < 2) cnt[tid] = 0;
   __syncthreads();
@@ -423,19 +644,14 @@ __global__ void __launch_bounds__(kRowThreads, 3) row_topk_kernel(const float* _
     row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
       const bool ok = in && k != 0u;
       const bool gt = ok && (k >> 20) > pb;
-      const unsigned m = __ballot_sync(0xffffffffu, gt);
-      if (m) {
-        const int lane = threadIdx.x & 31, leader = __ffs(m) - 1;
-        uint32_t base = 0;
-        if (lane == leader) base = atomicAdd(&cnt[1], (uint32_t)__popc(m));
-        base = __shfl_sync(0xffffffffu, base, leader);
-        const uint32_t pos = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-        if (gt && pos < (uint32_t)topk) {
-          oi[pos] = s;
-          if (ov) ov[pos] = key_to_float(k);
-        }
+      const uint32_t slot = warp_slot(gt, &cnt[1]);
+      if (gt && slot < (uint32_t)topk) {
+        oi[slot] = s;
+        if (ov) ov[slot] = key_to_float(k);
       }
-      warp_append(ok && (k >> 20) == pb, k, (uint32_t)s, list, kRowList, &cnt[0]);
+      const bool eq = ok && (k >> 20) == pb;
+      const uint32_t e = warp_slot(eq, &cnt[0]);
+      if (eq && e < (uint32_t)kRowList) list[e] = make_uint2(k, (uint32_t)s);
     });
     __syncthreads();
     const uint32_t n_gt = min(cnt[1], (uint32_t)topk);
@@ -470,6 +686,7 @@ struct SmemItems {
   const uint32_t* ids;
   __device__ uint32_t key(int i) const { return keys[padded(i)]; }
   __device__ uint32_t id(int i) const { return ids[padded(i)]; }
+  __device__ float value(int i) const { return key_to_float(keys[padded(i)]); }
 };
 
 // Top-k of candidate lists in one CTA: values F[t, P], ids cand[t, P] (ids outside [0, n_t) are
