@@ -16,17 +16,21 @@
 //
 // Per CTA (one per SM, persistent): a contiguous range of the flattened (query block, key tile)
 // work, balanced to within one tile.  Warp roles:
-//   warps 0-7  epilogue: tcgen05.ld of the accumulator, w * ReLU sums, masked stores (s < n_t)
-//   warp 8     query-head gather: sorts each query's head list, cp.async of the rows into the
+//   warps 0-15 epilogue (TMEM lane quarter x column quarter): tcgen05.ld of the accumulator,
+//              w * ReLU sums; a warp's (queries x 32 keys) block goes out as one TMA store from
+//              shared memory when every key is inside every prefix, else as masked stores
+//              (entries at s >= n_t are never written)
+//   warp 16    query-head gather: sorts each query's head list, cp.async of the rows into the
 //              swizzled operand layout (double-buffered across query blocks)
-//   warp 9     TMA producer: 128-key x 64-dim tiles of K into a 5-stage ring
-//   warp 10    MMA issuer (one thread) and TMEM owner: 2 accumulators of 256 fp32 columns
+//   warp 17    TMA producer: 128-key x 64-dim tiles of K into a 4-stage ring
+//   warp 18    MMA issuer (one thread) and TMEM owner: 2 accumulators of 256 fp32 columns
 // Every wait is bounded in time; a wait that runs out sets a device status word and all roles
 // leave their loops, wait for their own copies and MMAs, and free tensor memory.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -43,21 +47,23 @@ namespace {
 
 constexpr int kTileKeys = 128;                       // UMMA M: keys per accumulator (TMEM lanes)
 constexpr int kTileCols = 256;                       // UMMA N: query-head rows per block
-constexpr int kStages = 5;                           // K ring: 128 keys x 64 dims per stage
+constexpr int kStages = 4;                           // K ring: 128 keys x 64 dims per stage
 constexpr int kStageBytes = kTileKeys * 64 * 2;      // 16 KB
 constexpr int kQHalfBytes = kTileCols * 64 * 2;      // 32 KB: 64 dims of all 256 rows
 constexpr int kQBytes = 2 * kQHalfBytes;             // 64 KB per query block
 constexpr int kMaxBlocks = 2048;                     // query blocks per launch
-constexpr int kEpiWarps = 8;
-constexpr int kLoaderWarp = 8, kTmaWarp = 9, kMmaWarp = 10;
-constexpr int kThreads = 11 * 32;
+constexpr int kEpiWarps = 16;
+constexpr int kLoaderWarp = 16, kTmaWarp = 17, kMmaWarp = 18;
+constexpr int kThreads = 19 * 32;
 constexpr uint32_t kTmemCols = 512;                  // two accumulators of 256 columns
 constexpr uint64_t kWaitLimitNs = 1000000000ull;     // 1 s
 
 // Shared-memory layout (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = 0;                                          // [2][64 KB]
 constexpr int kOffK = kOffQ + 2 * kQBytes;                         // [kStages][16 KB]
-constexpr int kOffPre = kOffK + kStages * kStageBytes;             // [kMaxBlocks + 1] u32
+constexpr int kStageOutFloats = 8 * 32;                           // per epilogue warp: 8 rows x 32 keys
+constexpr int kOffOut = kOffK + kStages * kStageBytes;             // [kEpiWarps][8][32] f32 staged stores
+constexpr int kOffPre = kOffOut + kEpiWarps * kStageOutFloats * 4; // [kMaxBlocks + 1] u32
 constexpr int kOffW = kOffPre + ((kMaxBlocks + 1) * 4 + 15) / 16 * 16;  // [2][256] f32
 constexpr int kOffHead = kOffW + 2 * kTileCols * 4;                // [2][256] i32
 constexpr int kOffN = kOffHead + 2 * kTileCols * 4;                // [2][32] i32 prefix lengths
@@ -76,20 +82,22 @@ struct Bars {
   __device__ uint32_t qe(int i) const { return qempty + 8 * i; }
 };
 
-// w * ReLU of the 32 accumulator columns [32 CC, 32 CC + 32) of one epilogue thread: column c
-// belongs to query c / MP of the thread's column half; its slot c % MP feeds partial sum
-// (c % MP) % NP of that query.  wr holds the weights of the 128 columns.
-template <int MP, int NP, int CC>
-__device__ __forceinline__ void accumulate_chunk(const uint32_t (&v)[32], const float* wr, float* acc) {
+// w * ReLU of the 32 accumulator columns [32 CC, 32 CC + 32) of one epilogue thread, two columns
+// per packed fp32x2 FMA: column c (counted from the warp's first column) belongs to query c / MP
+// of the warp; its slot pair (c % MP) / 2 feeds float2 partial sum ((c % MP) / 2) % NF of that
+// query.  wr holds the weights from the warp's first column on.
+template <int MP, int NF, int CC>
+__device__ __forceinline__ void accumulate_chunk(const uint32_t (&v)[32], const float* wr, float2* acc) {
 #pragma unroll
   for (int j = 0; j < 32; j += 4) {
     const float4 wv = *reinterpret_cast<const float4*>(wr + CC * 32 + j);
-    const float wj[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
+    for (int u = 0; u < 4; u += 2) {
       const int c = CC * 32 + j + u;
-      const int x = (c / MP) * NP + (c % MP) % NP;
-      acc[x] = fmaf(wj[u], fmaxf(__uint_as_float(v[j + u]), 0.f), acc[x]);
+      const int x = (c / MP) * NF + ((c % MP) / 2) % NF;
+      const float2 r = make_float2(fmaxf(__uint_as_float(v[j + u]), 0.f), fmaxf(__uint_as_float(v[j + u + 1]), 0.f));
+      const float2 ww = u == 0 ? make_float2(wv.x, wv.y) : make_float2(wv.z, wv.w);
+      acc[x] = __ffma2_rn(ww, r, acc[x]);
     }
   }
 }
@@ -101,11 +109,11 @@ __device__ __forceinline__ void give_up(volatile int* abort) {
 
 template <int MP>
 __global__ void __launch_bounds__(kThreads, 1)
-    score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __nv_bfloat16* __restrict__ q,
-                    const float* __restrict__ w, const int32_t* __restrict__ n, const int32_t* __restrict__ heads,
-                    int h, int H_I, int L, int T, float* __restrict__ out, int64_t ld) {
+    score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap omap,
+                    int tma_store, const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                    const int32_t* __restrict__ n, const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
+                    float* __restrict__ out, int64_t ld) {
   constexpr int QT = kTileCols / MP;  // queries per block
-  constexpr int QW = 128 / MP;        // queries per epilogue warp (one column half)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* pre = reinterpret_cast<uint32_t*>(sm + kOffPre);
@@ -165,8 +173,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < kEpiWarps) {
     // ---------------- epilogue ----------------
-    const int lq = warp & 3, ch = warp >> 2;
-    constexpr int NP = QW >= 16 ? 1 : 16 / QW;  // partial sums per query: chains of 8 FMAs a tile
+    // warp = (column quarter cq, TMEM lane quarter lq); with 128 rows per query the even quarters
+    // take a whole query (128 columns) and the odd ones only hand the accumulator back
+    constexpr int CW = MP > 64 ? 128 : 64;  // columns of an active warp
+    constexpr int QW = CW / MP;              // its queries
+    constexpr int NF = MP / 8;               // float2 partial sums per query: chains of 4 a tile
+    const int lq = warp & 3, cq = warp >> 2;
+    const int col0 = cq * 64;
+    float* stage_out = reinterpret_cast<float*>(sm + kOffOut) + warp * kStageOutFloats;
+    const bool active = (col0 % CW) == 0;
     uint32_t i = 0, p = 0, lo, hi;
     int blk;
     tc::TileSegments it(pre, NB, a, e);
@@ -176,9 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         give_up(abort);
         break;
       }
-      const int tq = blk * QT + ch * QW;
-      const int* nr = nsm + pb * 32 + ch * QW;
-      const float* wr = wsm + pb * kTileCols + ch * 128;
+      const int tq = blk * QT + col0 / MP;
+      const int* nr = nsm + pb * 32 + col0 / MP;
+      const float* wr = wsm + pb * kTileCols + col0;
+      int nmin = tma_store ? 0x7fffffff : 0;  // keys below it are inside every prefix of the warp
+#pragma unroll
+      for (int l = 0; l < QW; ++l) nmin = min(nmin, nr[l]);
       bool ok = true;
       for (uint32_t tile = lo; tile < hi; ++tile, ++i) {
         const int ab = i & 1;
@@ -187,35 +205,61 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc::tc_fence_after();
-        float acc[QW * NP];
+        float2 acc[QW * NF];
 #pragma unroll
-        for (int x = 0; x < QW * NP; ++x) acc[x] = 0.f;
-        const uint32_t ta = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(ab * kTileCols + ch * 128);
-        // four 32-column loads, each overlapping the previous chunk's arithmetic
-        uint32_t va[32], vb[32];
-        tc::tmem_ld32(ta, va);
-        tc::tmem_ld_wait(va);
-        tc::tmem_ld32(ta + 32, vb);
-        accumulate_chunk<MP, NP, 0>(va, wr, acc);
-        tc::tmem_ld_wait(vb);
-        tc::tmem_ld32(ta + 64, va);
-        accumulate_chunk<MP, NP, 1>(vb, wr, acc);
-        tc::tmem_ld_wait(va);
-        tc::tmem_ld32(ta + 96, vb);
-        accumulate_chunk<MP, NP, 2>(va, wr, acc);
-        tc::tmem_ld_wait(vb);
-        accumulate_chunk<MP, NP, 3>(vb, wr, acc);
+        for (int x = 0; x < QW * NF; ++x) acc[x] = make_float2(0.f, 0.f);
+        if (active) {
+          const uint32_t ta = tmem + ((uint32_t)(lq * 32) << 16) + (uint32_t)(ab * kTileCols + col0);
+          // 32-column loads, each overlapping the previous chunk's arithmetic
+          uint32_t va[32], vb[32];
+          tc::tmem_ld32(ta, va);
+          tc::tmem_ld_wait(va);
+          tc::tmem_ld32(ta + 32, vb);
+          accumulate_chunk<MP, NF, 0>(va, wr, acc);
+          tc::tmem_ld_wait(vb);
+          if constexpr (CW == 128) {
+            tc::tmem_ld32(ta + 64, va);
+            accumulate_chunk<MP, NF, 1>(vb, wr, acc);
+            tc::tmem_ld_wait(va);
+            tc::tmem_ld32(ta + 96, vb);
+            accumulate_chunk<MP, NF, 2>(va, wr, acc);
+            tc::tmem_ld_wait(vb);
+            accumulate_chunk<MP, NF, 3>(vb, wr, acc);
+          } else {
+            accumulate_chunk<MP, NF, 1>(vb, wr, acc);
+          }
+        }
         tc::tc_fence_before();
         __syncwarp();
         if (lane == 0) tc::mbar_arrive_relaxed(bars.ae(ab));
-        const int s = (int)tile * kTileKeys + lq * 32 + lane;
+        if (active) {
+          const int s0w = (int)tile * kTileKeys + lq * 32;
+          const int s = s0w + lane;
+          float sum[QW];
 #pragma unroll
-        for (int l = 0; l < QW; ++l) {
+          for (int l = 0; l < QW; ++l) {
 #pragma unroll
-          for (int st = NP / 2; st >= 1; st >>= 1)
+            for (int st = NF / 2; st >= 1; st >>= 1)
 #pragma unroll
-            for (int x = 0; x < st; ++x) acc[l * NP + x] += acc[l * NP + x + st];
-          if (s < nr[l]) out[(int64_t)(tq + l) * ld + s] = acc[l * NP];
+              for (int x = 0; x < st; ++x) acc[l * NF + x] = __fadd2_rn(acc[l * NF + x], acc[l * NF + x + st]);
+            sum[l] = acc[l * NF].x + acc[l * NF].y;
+          }
+          if (s0w + 32 <= nmin) {  // the whole block: one TMA store
+            if (lane == 0) tc::bulk_wait_read_all();  // the previous store has read the buffer
+            __syncwarp();
+#pragma unroll
+            for (int l = 0; l < QW; ++l) stage_out[l * 32 + lane] = sum[l];
+            tc::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tc::tma_store_2d(&omap, s0w, tq, tc::smem_u32(stage_out));
+              tc::bulk_commit();
+            }
+          } else {
+#pragma unroll
+            for (int l = 0; l < QW; ++l)
+              if (s < nr[l]) out[(int64_t)(tq + l) * ld + s] = sum[l];
+          }
         }
       }
       if (!ok) {
@@ -226,6 +270,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) tc::mbar_arrive(bars.qe(pb));
       ++p;
     }
+    if (lane == 0) tc::bulk_wait_all();  // staged stores complete before the CTA exits
+    __syncwarp();
   } else if (warp == kLoaderWarp) {
     // ---------------- query-head gather ----------------
     const int m = heads ? h : H_I;
@@ -386,14 +432,19 @@ template <int MP>
 void launch_mp(const CUtensorMap& map, const __nv_bfloat16* q, const float* w, const int32_t* n,
                const int32_t* heads, int h, int H_I, int L, int T, float* out, int64_t ld, cudaStream_t s) {
   constexpr int QT = kTileCols / MP;
+  constexpr int QW = (MP > 64 ? 128 : 64) / MP;  // rows of an epilogue warp's store box
   cudaFuncSetAttribute(score_tc_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   const int grid = sm_count();
   const int per_launch = kMaxBlocks * QT;
   for (int t0 = 0; t0 < T; t0 += per_launch) {
     const int Tc = T - t0 < per_launch ? T - t0 : per_launch;
+    float* o = out + (int64_t)t0 * ld;
+    CUtensorMap omap;
+    const bool tma = tmap_f32_rows(&omap, o, (uint64_t)L, (uint64_t)Tc, (uint64_t)ld, 32, QW);
+    if (!tma) memset(&omap, 0, sizeof(omap));
     score_tc_kernel<MP><<<grid, kThreads, kSmemBytes, s>>>(
-        map, q + (int64_t)t0 * H_I * kD, w + (int64_t)t0 * H_I, n + t0, heads ? heads + (int64_t)t0 * h : nullptr,
-        h, H_I, L, Tc, out + (int64_t)t0 * ld, ld);
+        map, omap, tma ? 1 : 0, q + (int64_t)t0 * H_I * kD, w + (int64_t)t0 * H_I, n + t0,
+        heads ? heads + (int64_t)t0 * h : nullptr, h, H_I, L, Tc, o, ld);
   }
 }
 
