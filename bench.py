@@ -41,86 +41,15 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "4b425ffcef44de6292b97de3aaf2e847b519a18b5d4a943a5c8ed965993f4725",
-           "bytes_per_key": 1.0932e9 / 4194304, "capture": "profiles/score_bf16_decode_L131072_b32.md"}
-
-
-def _sha(path):
-    with open(os.path.join(ROOT, path), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()
-
-
-def _peaks():
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return float(d["hbm_gbs"]), "measured"
-    return 6650.0, "fallback"
-
-
-def _tc_peaks():
-    """Dense bf16 tensor-core peaks in TFLOP/s: burst (a kernel timed alone) and sustained (a
-    seconds-long loop under the power cap)."""
-    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return {"burst": float(d["bf16_tflops"]), "sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
-                "kind": "measured"}
-    return {"burst": 1590.0, "sustained": 1400.0, "kind": "fallback"}
-
-
-class ClockSampler:
-    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
-
-    REASONS = {
-        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
-        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
-        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
-    }
-
-    def __init__(self, index):
-        self.samples, self.reasons, self.max_mhz = [], set(), None
-        self._stop = threading.Event()
-        self._thread = None
-        try:
-            import pynvml
-            pynvml.nvmlInit()
-            self.nv = pynvml
-            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
-            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
-        except Exception:
-            self.nv = None
-
-    def _run(self):
-        while not self._stop.is_set():
-            try:
-                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
-                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for bit, name in self.REASONS.items():
-                    if r & bit and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(0.002)
-
-    def __enter__(self):
-        if self.nv is not None:
-            self._thread = threading.Thread(target=self._run, daemon=True)
-            self._thread.start()
-        return self
-
-    def __exit__(self, *a):
-        self._stop.set()
-        if self._thread:
-            self._thread.join()
-
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+           "sha256": "882fa00edb9e7424a1789c4bd4c2617855703325b29011526c34175b4253d28b",
+           "bytes_per_key": (1.074456e9 + 19.13344e6) / 4194304,
+           "capture": "profiles/score_persist_decode_L131072_b32.md"}
+# The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
+# chunk's launch; the step's traffic is that rate times the pairs the step scores.
+TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
+                   "sha256": "3aa6df1f296fc7e0cb8afde7e9ae237d607084f9533b601ca428cd9b148f33ba",
+                   "bytes_per_pair": (52.319232e6 + 984.943616e6) / 260048896,
+                   "capture": "profiles/score_tc_prefill_L65536_chunk15.md"}
 
 
 def _dist():
@@ -398,6 +327,9 @@ def run_prefill(args, wl):
     if rank == 0:
         peaks = _tc_peaks()
         achieved = flops / (score_ms / 1000.0) / 1e12
+        traffic = None
+        if TRAFFIC_PREFILL["sha256"] == _sha(TRAFFIC_PREFILL["file"]):
+            traffic = TRAFFIC_PREFILL["bytes_per_pair"] * pairs
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -413,7 +345,9 @@ def run_prefill(args, wl):
             "roofline": {"bound": "tensor", "kernel": "routed token scoring (score_tc_kernel, tcgen05)",
                          "achieved": achieved, "peak": peaks["sustained"], "peak_kind": peaks["kind"] + " sustained",
                          "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
-                         "frac_of_burst_peak": achieved / peaks["burst"], "traffic": None,
+                         "frac_of_burst_peak": achieved / peaks["burst"], "traffic": traffic,
+                         "traffic_per_launch_note": "per step (16 chunk launches): bytes per scored pair from "
+                                                    "the capture x pairs per step",
                          "algorithmic_flops_per_step": flops, "score_ms_per_step": score_ms},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
