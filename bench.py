@@ -52,6 +52,96 @@ TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
                    "capture": "profiles/score_tc_prefill_L65536_chunk15.md"}
 
 
+def _sha(path):
+    with open(os.path.join(ROOT, path), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _tc_peaks():
+    """Dense bf16 tensor-core peaks in TFLOP/s: burst (a kernel timed alone) and sustained (a
+    seconds-long loop under the power cap)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"burst": float(d["bf16_tflops"]), "sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "kind": "measured"}
+    return {"burst": 1590.0, "sustained": 1400.0, "kind": "fallback"}
+
+
+class ClockSampler:
+    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, index):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for bit, name in self.REASONS.items():
+                    if r & bit and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def _graphed(torch, step, use_graph):
+    """The step as a CUDA graph captured from the same C-ABI calls (all launches and memsets of one
+    step replayed with one call), or the plain step.  Call after warm-up: the workspaces are sized."""
+    if not use_graph:
+        return step
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    torch.cuda.synchronize()
+    return g.replay
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -268,6 +358,9 @@ def run_prefill(args, wl):
             acc["topk"] += e[2].elapsed_time(e[3])
     stages_us = {k_: round(1000 * v / nst, 1) for k_, v in acc.items()}
 
+    run_step = _graphed(torch, step, not args.no_graph)
+    for _ in range(2):
+        run_step()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:
         dist.barrier()
@@ -275,7 +368,7 @@ def run_prefill(args, wl):
     with ClockSampler(local) as clk:
         t0.record(stream)
         for _ in range(args.steps):
-            step()
+            run_step()
         t1.record(stream)
         torch.cuda.synchronize()
     if ws > 1:
@@ -341,6 +434,7 @@ def run_prefill(args, wl):
                        "l2": f"score rows of one chunk ({ch * L * 4 / 2**30:.1f} GiB) exceed L2; the "
                              f"16 MiB key cache stays in L2",
                        "parallelism": f"{ws} GPU(s), one independent sequence per GPU",
+                       "cuda_graph": not args.no_graph,
                        "step": "pool all blocks + per chunk: route + routed scores + top-k"},
             "roofline": {"bound": "tensor", "kernel": "routed token scoring (score_tc_kernel, tcgen05)",
                          "achieved": achieved, "peak": peaks["sustained"], "peak_kind": peaks["kind"] + " sustained",
@@ -447,6 +541,9 @@ def run_ours(args):
     stages_us = {nm: round(1000 * a / nst, 2) for nm, a in zip(stage_names, stage_acc)}
 
     # the timed region: K whole steps
+    run_step = _graphed(torch, step, not args.no_graph)
+    for _ in range(3):
+        run_step()
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if ws > 1:
         dist.barrier()
@@ -454,7 +551,7 @@ def run_ours(args):
     with ClockSampler(local) as clk:
         t0.record(stream)
         for _ in range(args.steps):
-            step()
+            run_step()
         t1.record(stream)
         torch.cuda.synchronize()
     if ws > 1:
@@ -533,7 +630,8 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU"}),
+            "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU",
+                                   "cuda_graph": not args.no_graph}),
             "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                          "frac": achieved / hbm, "traffic": traffic,
@@ -566,6 +664,8 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
+                                                              "the step as a CUDA graph")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
