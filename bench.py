@@ -142,6 +142,28 @@ def _graphed(torch, step, use_graph):
     return g.replay
 
 
+def rank_sequences(rank, world, per_rank):
+    """The decode sequences of one rank: a contiguous share of world x per_rank, disjoint from the
+    other ranks' (independent problems; no data-path collective)."""
+    return list(range(rank * per_rank, (rank + 1) * per_rank))
+
+
+def rank_workload(wl, rank):
+    """The workload a rank runs: rank 0 the named one, every other rank the same shapes with its own
+    seed (its own prefill sequence)."""
+    return wl if rank == 0 else W.small(wl.cid, seed=wl.seed + 7919 * rank)
+
+
+def max_over_ranks(ms, dist, device):
+    """The largest elapsed time over all ranks: the job's time (one all-reduce of one number)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return ms
+    import torch
+    tt = torch.tensor([float(ms)], device=device)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return float(tt.item())
+
+
 def _dist():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -258,8 +280,8 @@ def run_reference_prefill(args, wl, nthr):
     return 0
 
 
-def _gen_chunk(cid, c):
-    wl = W.WORKLOADS[cid]
+def _gen_chunk(cid, seed, c):
+    wl = W.small(cid, seed=seed)
     ch = wl.chunk
     q, w = W.shared_queries(wl, c * ch, min((c + 1) * ch, wl.T))
     return q, w
@@ -271,14 +293,15 @@ def run_prefill(args, wl):
     cores, and select the top-k of every query."""
     import multiprocessing as mp
 
+    ws, rank, local = _dist()
+    wl = rank_workload(wl, rank)
     ch = wl.chunk
     nch = -(-wl.T // ch)
     with mp.get_context("spawn").Pool(min(nch, max(1, os.cpu_count() or 1))) as pool:
-        parts = pool.starmap(_gen_chunk, [(wl.cid, c) for c in range(nch)])
+        parts = pool.starmap(_gen_chunk, [(wl.cid, wl.seed, c) for c in range(nch)])
     import torch
     import torch.distributed as dist
 
-    ws, rank, local = _dist()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if ws > 1:
@@ -375,9 +398,7 @@ def run_prefill(args, wl):
         dist.barrier()
     ms = t0.elapsed_time(t1)
     if ws > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, dev)
     value = pairs * ws * args.steps / (ms / 1000.0)
 
     # end to end: every step copies the cache, the queries, their weights and n from pinned host
@@ -412,9 +433,7 @@ def run_prefill(args, wl):
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
     if ws > 1:
-        tt = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
+        e_ms = max_over_ranks(e_ms, dist, dev)
     e2e_value = pairs * ws * ne / (e_ms / 1000.0)
 
     if rank == 0:
@@ -475,7 +494,7 @@ def run_ours(args):
     if wl.n_seq == 1:
         raise SystemExit("shared-cache workloads run through run_prefill")
     big = W.small(wl.cid, n_seq=wl.n_seq * ws, T=wl.T * ws)
-    seqs = list(range(rank * wl.T, (rank + 1) * wl.T))
+    seqs = rank_sequences(rank, ws, wl.T)
     k_h, q_h, w_h, n_h, _ = W.decode_batch(big, seqs)
     T, L, d = k_h.shape
     kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
@@ -558,9 +577,7 @@ def run_ours(args):
         dist.barrier()
     ms = t0.elapsed_time(t1)
     if ws > 1:
-        tt = torch.tensor([ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+        ms = max_over_ranks(ms, dist, dev)
     units_per_step = T * L * ws
     value = units_per_step * args.steps / (ms / 1000.0)
 
@@ -598,9 +615,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     e_ms = e0.elapsed_time(e1)
     if ws > 1:
-        tt = torch.tensor([e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e_ms = float(tt.item())
+        e_ms = max_over_ranks(e_ms, dist, dev)
     e2e_value = units_per_step * args.steps / (e_ms / 1000.0)
 
     # dense DSA on the same inputs (the baseline the pages compare against), not part of the step
