@@ -28,12 +28,25 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint3
 __device__ __forceinline__ int frag_dim(int kk, int c) { return 32 * (kk >> 1) + 8 * c + 4 * (kk & 1); }
 
 // Stage the B fragments of NG groups of 8 heads: frag[ng][kk][lane] = 4 bf16 of head hl[8 ng + g].
-template <int NG>
+// NT = threads of the block; every thread issues all its loads before its first store.
+template <int NG, int NT>
 __device__ __forceinline__ void stage_q_frags(uint2 (*frag)[8][32], const __nv_bfloat16* qt, const int* hl) {
-  for (int e = threadIdx.x; e < NG * 8 * 32; e += blockDim.x) {
-    const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
-    const int g = ln >> 2, c = ln & 3;
-    frag[ng][kk][ln] = *reinterpret_cast<const uint2*>(qt + (int64_t)hl[ng * 8 + g] * kD + frag_dim(kk, c));
+  constexpr int kElems = NG * 8 * 32;
+  constexpr int kPer = (kElems + NT - 1) / NT;
+  uint2 v[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = (int)threadIdx.x + i * NT;
+    if (e < kElems) {
+      const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
+      const int g = ln >> 2, c = ln & 3;
+      v[i] = *reinterpret_cast<const uint2*>(qt + (int64_t)hl[ng * 8 + g] * kD + frag_dim(kk, c));
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    const int e = (int)threadIdx.x + i * NT;
+    if (e < kElems) frag[e >> 8][(e >> 5) & 7][e & 31] = v[i];
   }
 }
 

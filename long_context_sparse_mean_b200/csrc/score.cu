@@ -52,9 +52,15 @@ struct HeadStage {
 };
 
 // Thread 0 sorts the heads; pads reuse head hl[0] with weight 0.  Head ids outside [0, H_I) are
-// clamped into range (the router never produces them).
+// clamped into range (the router never produces them).  Without a list (all heads, already in
+// order) the threads fill it together.
 __device__ __forceinline__ void stage_head_list(const int32_t* heads, int h, int H_I, int t, int slots,
                                                 int* hl, int* m_out) {
+  if (!heads) {
+    for (int a = threadIdx.x; a < slots; a += blockDim.x) hl[a] = a < H_I ? a : 0;
+    if (threadIdx.x == 0) *m_out = H_I;
+    return;
+  }
   if (threadIdx.x == 0) {
     const int m = heads ? h : H_I;
     for (int a = 0; a < m; ++a) {
@@ -79,7 +85,7 @@ __device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat
   __syncthreads();
   if (threadIdx.x < NG * 8)
     st.wsel[threadIdx.x] = (int)threadIdx.x < st.m ? w[(int64_t)t * H_I + st.hl[threadIdx.x]] : 0.f;
-  stage_q_frags<NG>(st.frag, q + (int64_t)t * H_I * kD, st.hl);
+  stage_q_frags<NG, kScoreThreads>(st.frag, q + (int64_t)t * H_I * kD, st.hl);
   __syncthreads();
 }
 
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       __syncthreads();
       if (last) {
         __threadfence();
-        const Bucket bk = level0_boundary(ht, (uint32_t)topk, hsm, wtot);
+        const Bucket bk = level0_boundary<kScoreThreads>(ht, (uint32_t)topk, hsm, wtot);
         if (threadIdx.x == 0) {
           rec[8 * (int64_t)t + 2] = bk.prefix;
           rec[8 * (int64_t)t + 3] = bk.need;

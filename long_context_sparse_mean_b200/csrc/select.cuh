@@ -92,13 +92,18 @@ __device__ __forceinline__ Bucket bucket_search_padded(const uint32_t* hp, uint3
 // (prefix of the bucket holding the k-th largest key, keys still needed from it).  With fewer
 // than k counted keys every key is taken; with none the prefix is 0xffffffff.  hp: padded
 // shared scratch of kHistPadded words.  Every thread of the block must call it.
+template <int NT>  // = blockDim.x; every thread issues its loads of the histogram together
 __device__ __forceinline__ Bucket level0_boundary(const uint32_t* hist_t, uint32_t topk, uint32_t* hp,
                                                   uint32_t* scratch) {
+  constexpr int kPer = kHistBins / NT;
+  uint32_t v[kPer];
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) v[i] = __ldcg(hist_t + threadIdx.x + i * NT);
   uint32_t local = 0;
-  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) {
-    const uint32_t v = __ldcg(hist_t + b);
-    hp[hpad(b)] = v;
-    local += v;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    hp[hpad((int)threadIdx.x + i * NT)] = v[i];
+    local += v[i];
   }
   uint32_t total;
   block_exclusive_scan(local, scratch, &total);  // also orders the stores above

@@ -122,7 +122,7 @@ __global__ void __launch_bounds__(kPassThreads) hist_pass_kernel(const float* __
   __syncthreads();
   if (!last) return;
   __threadfence();
-  const Bucket bk = level0_boundary(ht, (uint32_t)topk, h, scratch);
+  const Bucket bk = level0_boundary<kPassThreads>(ht, (uint32_t)topk, h, scratch);
   if (threadIdx.x == 0) {
     rt[2] = bk.prefix;
     rt[3] = bk.need;
