@@ -30,7 +30,7 @@ template <DType DT>
 __device__ __forceinline__ float block_mean_256(const void* kseq, int s0, int s1, float (*part)[kD]) {
   const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
   float a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
+#pragma unroll 8
   for (int s = s0 + rg; s < s1; s += 4) {
     if (DT == DType::BF16) {
       const uint32_t x = reinterpret_cast<const uint32_t*>(kseq)[(int64_t)s * (kD / 2) + cp];
@@ -232,6 +232,7 @@ __device__ __forceinline__ void select_heads_warp(const float* partial_t, int nc
     v[i] = 0.f;
     if (live[i]) {
       float s = 0.f;
+#pragma unroll 8
       for (int c = 0; c < nc; ++c) s += __ldcg(partial_t + (int64_t)c * H_I + j);
       v[i] = w_t[j] * s;
       if (r_t) r_t[j] = v[i];
@@ -316,11 +317,23 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
     const float m = block_mean_256<DType::BF16>(k + (int64_t)t * k_seq_stride, nfull * B, nt, part);
     if (threadIdx.x < kD) pms[threadIdx.x] = m;
   }
-  for (int e = threadIdx.x; e < NG * 8 * 32; e += blockDim.x) {
-    const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
-    const int g = ln >> 2, c = ln & 3;
-    const __nv_bfloat16* src = q + ((int64_t)t * H + ng * 8 + g) * kD + 16 * kk + 4 * c;
-    frag[ng][kk][ln] = *reinterpret_cast<const uint2*>(src);
+  {  // every thread issues its fragment loads together (256 threads)
+    constexpr int kPer = (NG * 8 * 32 + 255) / 256;
+    uint2 v[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = (int)threadIdx.x + 256 * i;
+      if (e < NG * 8 * 32) {
+        const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
+        const int g = ln >> 2, c = ln & 3;
+        v[i] = *reinterpret_cast<const uint2*>(q + ((int64_t)t * H + ng * 8 + g) * kD + 16 * kk + 4 * c);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int e = (int)threadIdx.x + 256 * i;
+      if (e < NG * 8 * 32) frag[e >> 8][(e >> 5) & 7][e & 31] = v[i];
+    }
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;

@@ -235,6 +235,7 @@ __global__ void __launch_bounds__(NT) resolve_kernel(const int32_t* __restrict__
         if (ov) ov[n_out + i] = key_to_float(pt[i].x);
       }
   } else if (c <= kResolveSmemItems) {
+#pragma unroll 8
     for (int i = threadIdx.x; i < c; i += NT) list[i] = pt[i];
     __syncthreads();
     const PairList acc{list};
