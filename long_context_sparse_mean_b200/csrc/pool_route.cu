@@ -422,7 +422,8 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float* __restrict
 
 // One CTA per query, after the tensor-core router's per-tile sums Sp[t][tile][j] over full pooled
 // blocks: adds max(0, q_{t,j} . mean of the partial last block) (keys [floor(n_t/B) B, n_t),
-// averaged here), then r_j = w_j * total and the top-h heads.
+// averaged here), then r_j = w_j * total and the top-h heads.  The q rows and the per-tile sums
+// are requested before the mean is formed, so their loads overlap it.
 __global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* __restrict__ q,
                                                            const float* __restrict__ w,
                                                            const __nv_bfloat16* __restrict__ k,
@@ -430,34 +431,49 @@ __global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* 
                                                            int h, const float* __restrict__ Sp, int nch,
                                                            int tile, int32_t* __restrict__ heads,
                                                            float* __restrict__ r_opt) {
+  constexpr int kHeadsPerWarp = kMaxHeads / 8;
   __shared__ float part[4][kD];
   __shared__ __align__(16) float pm[kD];
+  __shared__ float pmd[kMaxHeads];
   __shared__ float tot[kMaxHeads];
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
   const int nf = nt / B, c = nt % B;
   const int ntiles = (nf + tile - 1) / tile;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint2 qv[kHeadsPerWarp];  // lane's 4 dims of this warp's heads warp, warp + 8, ...
+#pragma unroll
+  for (int i = 0; i < kHeadsPerWarp; ++i) {
+    const int j = warp + 8 * i;
+    qv[i] = (c > 0 && j < H_I) ? *reinterpret_cast<const uint2*>(q + ((int64_t)t * H_I + j) * kD + 4 * lane)
+                               : make_uint2(0u, 0u);
+  }
+  float spsum = 0.f;
+  if ((int)threadIdx.x < H_I) {
+#pragma unroll 4
+    for (int i = 0; i < ntiles; ++i) spsum += __ldcg(Sp + ((int64_t)t * nch + i) * H_I + threadIdx.x);
+  }
   if (c > 0) {
     const float m = block_mean_256<DType::BF16>(k, nt - c, nt, part);
     if (threadIdx.x < kD) pm[threadIdx.x] = m;
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int j = warp; j < H_I; j += 8) {
-    float d = 0.f;
-    if (c > 0) {
-      const uint2 x = *reinterpret_cast<const uint2*>(q + ((int64_t)t * H_I + j) * kD + 4 * lane);
-      const float4 p4 = *reinterpret_cast<const float4*>(pm + 4 * lane);
-      d = bf16_lo(x.x) * p4.x + bf16_hi(x.x) * p4.y + bf16_lo(x.y) * p4.z + bf16_hi(x.y) * p4.w;
+  if (c > 0) {
+    const float4 p4 = *reinterpret_cast<const float4*>(pm + 4 * lane);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
-    }
-    if (lane == 0) {
-      float sum = 0.f;
-      for (int i = 0; i < ntiles; ++i) sum += __ldcg(Sp + ((int64_t)t * nch + i) * H_I + j);
-      tot[j] = sum + relu(d);
+    for (int i = 0; i < kHeadsPerWarp; ++i) {
+      const int j = warp + 8 * i;
+      if (j < H_I) {  // uniform across the warp
+        const uint2 x = qv[i];
+        float d = bf16_lo(x.x) * p4.x + bf16_hi(x.x) * p4.y + bf16_lo(x.y) * p4.z + bf16_hi(x.y) * p4.w;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if (lane == 0) pmd[j] = relu(d);
+      }
     }
   }
+  __syncthreads();
+  if ((int)threadIdx.x < H_I) tot[threadIdx.x] = spsum + (c > 0 ? pmd[threadIdx.x] : 0.f);
   __syncthreads();
   if (warp == 0) {
     float v[kMaxHeads / 32];
