@@ -514,9 +514,9 @@ def run_ours(args):
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
     score_ms = []
-    # pool, router, scores (level-0 histogram fused), partition + resolve, re-rank scores (fused
-    # histogram) + partition + resolve
-    launches_per_step = 8
+    # pool, router, scores, top-k' (one CTA per row), re-rank scores, top-k of the candidates; with
+    # the fused histogram the top-k' is partition + resolve
+    launches_per_step = 7 if args.fused_histogram else 6
 
     stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
 
@@ -529,11 +529,14 @@ def run_ours(args):
         mark(2)
         if time_scores:
             ev[0].record(stream)
-        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
+        if args.fused_histogram:
+            M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
+        else:
+            M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
         if time_scores:
             ev[1].record(stream)
         mark(3)
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=True)
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=args.fused_histogram)
         mark(4)
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
         mark(5)
@@ -679,6 +682,9 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--fused-histogram", action="store_true",
+                    help="decode: build the top-k' histogram inside the scoring kernel and select with the "
+                         "partition/resolve kernels (instead of one CTA per row)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
     args = ap.parse_args()

@@ -217,11 +217,9 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
     ld = score_ld(L);
     p += scores_part(T, L);
   }
-  misa::topk_rows_prepare(p, T, as_stream(stream));
-  const misa::TopkFuse fuse = misa::topk_rows_fuse(p, T, topk);
-  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0,
-                                         buf, ld, &fuse, as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, ready, idx, score_opt, as_stream(stream));
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld, nullptr,
+                      as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, false, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -237,11 +235,9 @@ misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64
   if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   float* F = static_cast<float*>(ws);
   void* sel = static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * kp);
-  misa::topk_rows_prepare(sel, T, as_stream(stream));
-  const misa::TopkFuse fuse = misa::topk_rows_fuse(sel, T, topk);
-  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand,
-                                         kp, F, kp, &fuse, as_stream(stream));
-  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, ready, idx, score_opt, as_stream(stream));
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp, nullptr,
+                      as_stream(stream));
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, false, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -258,11 +254,9 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   float* buf = reinterpret_cast<float*>(p);
   const int64_t ld = score_ld(L);
   void* sel = p + scores_part(T, L);
-  misa::topk_rows_prepare(sel, T, as_stream(stream));
-  const misa::TopkFuse fuse = misa::topk_rows_fuse(sel, T, topk);
-  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr,
-                                         0, buf, ld, &fuse, as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, sel, ready, idx, score_opt, as_stream(stream));
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
+                      nullptr, as_stream(stream));
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, sel, false, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 

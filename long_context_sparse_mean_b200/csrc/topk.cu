@@ -31,7 +31,8 @@ constexpr int kListItems = 4;   // for candidate lists (1024 per CTA: more CTAs 
 constexpr int kResolveSmemItems = 24576;  // boundary pairs ranked in shared memory (192 KB)
 constexpr int kSmallThreads = 1024;
 constexpr int kRec = 8;  // words of per-row state
-constexpr int kRowKernelMinRows = 256;  // from this many rows on, one CTA per row
+constexpr int kRowKernelMinRows = 256;  // from this many rows on, 2 row CTAs per SM
+constexpr int kRowListLarge = 16384;    // list of the 1024-thread row kernel (128 KB)
 
 // Per-row state rec[t][kRec] (kRec and the meaning of words 0, 2, 3 are shared with the scoring
 // kernel that builds the histogram):
@@ -252,31 +253,33 @@ __global__ void __launch_bounds__(NT) resolve_kernel(const int32_t* __restrict__
   }
 }
 
-// ---- one CTA per row, for many rows (prefill chunks) ----------------------------------------
+// ---- one CTA per row ----------------------------------------------------------------------------
 //
-// A row of n_t scores is read once by its CTA (2 CTAs of 512 threads per SM):
-//   1. cut: rows longer than the shared-memory list are sampled (256 evenly spaced runs of 8
-//      scores, 2048 keys); a 4096-bin histogram over the sampled key range places the sample key
-//      whose rank is the expected sample count above the k-th key plus three standard deviations
-//      and a margin, and the lower edge of its bin is the threshold value; shorter rows take every
-//      score;
-//   2. one pass appends (key, position) of every score at or above the threshold to the list
-//      (a bit mask per 32 scores a thread, one warp scan and one shared atomic per warp and
-//      batch; ~5% of a long row) and tracks the smallest and largest key;
+// Each row (a query's scores over its prefix, or over a list of candidate tokens) is read once by
+// its CTA: 512 threads, 2 CTAs per SM and an 8192-entry list for many rows (prefill chunks);
+// 1024 threads, 1 CTA per SM and a 16384-entry list for a few long rows (decode) and for
+// candidate lists:
+//   1. cut: rows longer than the list are sampled (256 evenly spaced runs of 8 scores, 2048
+//      keys); a 4096-bin histogram over the sampled key range places the sample key whose rank
+//      is the expected sample count above the k-th key plus three standard deviations and a
+//      margin, and the lower edge of its bin is the threshold value; shorter rows take every
+//      entry;
+//   2. one pass appends (key, token) of every entry at or above the threshold to the list (a bit
+//      mask per 16 entries a thread, one warp scan and one shared atomic per warp and step) and
+//      tracks the smallest and largest key;
 //   3. the list's keys are rewritten relative to the smallest so that they spread over the high
 //      bits (same order); one 4096-bin histogram finds the bucket of the k-th key; keys above it
 //      go straight to the output, the bucket's keys are ranked by one warp (when at most 32) or
-//      on the remaining bits, and, for exact ties, on the position.
+//      on the remaining bits, and, for exact ties, on the token.
 // Whenever the list holds at least k keys it holds every selected key, so the result is exact.
-// Otherwise (fewer than k at or above the cut, or more than the list holds) the row takes the
-// exact path: full level-0 histogram of the row, keys above the boundary bucket written out,
-// the bucket's keys ranked as above (from global memory if they overflow the list).
+// Otherwise (fewer than k at or above the cut, or more than the list holds) a score row takes the
+// exact path: full level-0 histogram of the row, keys above the boundary bucket written out, the
+// bucket's keys ranked as above (from global memory if they overflow the list).  Candidate lists
+// always fit the list.
 
-constexpr int kRowThreads = 512;
-constexpr int kRowList = 8192;          // (key, position) pairs in shared memory (64 KB)
-constexpr int kRowSegments = 256;       // sample runs per long row
-constexpr int kRowSegLen = 8;           // scores per run (one 32-byte sector)
-constexpr int kSweepBatch = 8;          // float4 loads in flight per thread
+constexpr int kRowSegments = 256;  // sample runs per long row
+constexpr int kRowSegLen = 8;      // scores per run (one 32-byte sector)
+constexpr int kSweepBatch = 8;     // float4 loads in flight per thread (exact path)
 
 struct SmemPairs {
   const uint2* p;
@@ -320,19 +323,19 @@ __device__ __forceinline__ uint32_t warp_slot(bool take, uint32_t* cnt) {
   return base + (uint32_t)__popc(m & ((1u << lane) - 1u));
 }
 
-// Visits positions [0, nt) of a row, four per step, with all lanes of every warp taking the same
-// number of steps (f gets position, key and a validity flag).  Loads are issued kSweepBatch steps
-// ahead of their use.  Used by the exact path only.
-template <class F>
+// Visits positions [0, nt) of a score row, four per step, with all lanes of every warp taking the
+// same number of steps (f gets position, key and a validity flag).  Loads are issued kSweepBatch
+// steps ahead of their use.  Used by the exact path only.
+template <int NT, class F>
 __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&& f) {
   if (vec) {
     const int n4 = (nt + 3) / 4;
-    const int steps = (n4 + kRowThreads - 1) / kRowThreads;
+    const int steps = (n4 + NT - 1) / NT;
     for (int j0 = 0; j0 < steps; j0 += kSweepBatch) {
       float4 x[kSweepBatch];
 #pragma unroll
       for (int u = 0; u < kSweepBatch; ++u) {
-        const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
+        const int i = (j0 + u) * NT + (int)threadIdx.x;
         x[u] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (4 * i + 3 < nt) {
           x[u] = __ldcg(reinterpret_cast<const float4*>(row) + i);
@@ -345,7 +348,7 @@ __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&
 #pragma unroll
       for (int u = 0; u < kSweepBatch; ++u) {
         if (j0 + u >= steps) break;  // uniform across the block
-        const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
+        const int i = (j0 + u) * NT + (int)threadIdx.x;
         const float v[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -355,40 +358,54 @@ __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&
       }
     }
   } else {
-    const int steps = (nt + kRowThreads - 1) / kRowThreads;
+    const int steps = (nt + NT - 1) / NT;
     for (int j = 0; j < steps; ++j) {
-      const int s = j * kRowThreads + (int)threadIdx.x;
+      const int s = j * NT + (int)threadIdx.x;
       const float v = s < nt ? __ldcg(row + s) : 0.f;
       f(s, order_key(v), s < nt);
     }
   }
 }
 
-// Appends (key, position) of every position s < nt whose score is >= thr to the list and folds
-// the appended keys into mm[0] (min) and mm[1] (max).  A thread reads 16 positions (4 float4) a
+// Appends (key, token) of every entry p < np whose score is >= thr to the list and folds the
+// appended keys into mm[0] (min) and mm[1] (max).  The token is p, or ids[p] for candidate lists
+// (entries whose id is outside [0, nt) are skipped).  A thread reads 16 entries (4 float4) a
 // step, the next step's loads in flight while it handles the current one, and marks its
 // candidates in a bit mask; one warp scan and one shared atomic per warp and step place them.
-__device__ __forceinline__ void collect_above(const float* row, int nt, bool vec, float thr, uint2* list, int cap,
-                                              uint32_t* cnt, uint32_t* mm) {
+template <int NT>
+__device__ __forceinline__ void collect_above(const float* row, const int32_t* ids, int np, int nt, bool vec,
+                                              float thr, uint2* list, int cap, uint32_t* cnt, uint32_t* mm) {
   constexpr int U = 4;  // float4 per thread and step
   const int lane = threadIdx.x & 31;
   uint32_t lo = 0xffffffffu, hi = 0u;
   auto load = [&](int j0, float4 (&x)[U]) {
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      const int i = (j0 + u) * kRowThreads + (int)threadIdx.x;
-      x[u] = make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      if (vec && 4 * i + 3 < nt) {
-        x[u] = __ldcg(reinterpret_cast<const float4*>(row) + i);
-      } else if (4 * i < nt) {
-        x[u].x = __ldcg(row + 4 * i);
-        if (4 * i + 1 < nt) x[u].y = __ldcg(row + 4 * i + 1);
-        if (4 * i + 2 < nt) x[u].z = __ldcg(row + 4 * i + 2);
-        if (4 * i + 3 < nt) x[u].w = __ldcg(row + 4 * i + 3);
+      const int i = (j0 + u) * NT + (int)threadIdx.x;
+      float v[4] = {NAN, NAN, NAN, NAN};  // NaN: never at or above the threshold
+      if (vec && 4 * i + 3 < np) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(row) + i);
+        v[0] = f.x;
+        v[1] = f.y;
+        v[2] = f.z;
+        v[3] = f.w;
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if (4 * i + e < np) v[e] = __ldcg(row + 4 * i + e);
       }
+      if (ids) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int p = 4 * i + e;
+          const int32_t id = p < np ? __ldcg(ids + p) : -1;
+          if (id < 0 || id >= nt) v[e] = NAN;
+        }
+      }
+      x[u] = make_float4(v[0], v[1], v[2], v[3]);
     }
   };
-  const int steps = ((nt + 3) / 4 + kRowThreads - 1) / kRowThreads;  // float4 groups a thread
+  const int steps = ((np + 3) / 4 + NT - 1) / NT;  // float4 groups a thread
   float4 cur[U], nxt[U];
   load(0, cur);
   for (int j0 = 0; j0 < steps; j0 += U) {
@@ -415,7 +432,7 @@ __device__ __forceinline__ void collect_above(const float* row, int nt, bool vec
       uint32_t pos = base + incl - c;
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int s0 = 4 * ((j0 + u) * kRowThreads + (int)threadIdx.x);
+        const int s0 = 4 * ((j0 + u) * NT + (int)threadIdx.x);
         const float v[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -423,7 +440,8 @@ __device__ __forceinline__ void collect_above(const float* row, int nt, bool vec
             const uint32_t k = order_key(v[e]);
             lo = min(lo, k);
             hi = max(hi, k);
-            if (pos < (uint32_t)cap) list[pos] = make_uint2(k, (uint32_t)(s0 + e));
+            const uint32_t tok = ids ? (uint32_t)__ldcg(ids + s0 + e) : (uint32_t)(s0 + e);
+            if (pos < (uint32_t)cap) list[pos] = make_uint2(k, tok);
             ++pos;
           }
         }
@@ -443,8 +461,8 @@ __device__ __forceinline__ void collect_above(const float* row, int nt, bool vec
   }
 }
 
-// Ranks n <= 32 entries of list (keys descending, then ids ascending) in one warp and writes the
-// first `need` to oi/ov at their rank.
+// Ranks n <= 32 entries of list (keys descending, then tokens ascending) in one warp and writes
+// the first `need` to oi/ov at their rank.
 template <class Acc>
 __device__ __forceinline__ void warp_rank_write(const uint2* list, int n, uint32_t need, const Acc& acc, int32_t* oi,
                                                 float* ov) {
@@ -467,25 +485,26 @@ __device__ __forceinline__ void warp_rank_write(const uint2* list, int n, uint32
 // to oi/ov [0, need).  One histogram of key bits 30..19; keys above the boundary bucket go out
 // directly, the bucket's entries move to the front of the list and are ranked (one warp when
 // they are few).  hist: kHistBins words; ctr: 2 words; scratch: 35 words.
+template <int NT, int LIST>
 __device__ void select_list(uint2* list, int c, uint32_t need, uint32_t lo, int sh, uint32_t* hist, uint32_t* ctr,
                             uint32_t* scratch, int32_t* oi, float* ov) {
   const int tid = threadIdx.x;
-  for (int b = tid; b < kHistBins; b += kRowThreads) hist[b] = 0;
+  for (int b = tid; b < kHistBins; b += NT) hist[b] = 0;
   if (tid < 2) ctr[tid] = 0;
   __syncthreads();
-  for (int i = tid; i < c; i += kRowThreads) hist_add(hist, (list[i].x >> 19) & 4095u, true);
+  for (int i = tid; i < c; i += NT) hist_add(hist, (list[i].x >> 19) & 4095u, true);
   __syncthreads();
   const Bucket bk = block_bucket_bits(hist, kHistBins, 19, 0x80000000u, need, scratch);
   const uint32_t pb = bk.prefix >> 19;
   const ShiftedPairs acc{list, lo, sh};
-  constexpr int kPer = kRowList / kRowThreads;
+  constexpr int kPer = LIST / NT;
   uint2 keep[kPer];
   int nk = 0;
-  const int steps = (c + kRowThreads - 1) / kRowThreads;
+  const int steps = (c + NT - 1) / NT;
 #pragma unroll
   for (int j = 0; j < kPer; ++j) {
     if (j >= steps) break;  // uniform
-    const int i = j * kRowThreads + tid;
+    const int i = j * NT + tid;
     const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
     const bool gt = i < c && (e.x >> 19) > pb;
     const uint32_t slot = warp_slot(gt, &ctr[0]);
@@ -506,7 +525,7 @@ __device__ void select_list(uint2* list, int c, uint32_t need, uint32_t lo, int 
   const uint32_t n_gt = ctr[0];
   const uint32_t need2 = need - n_gt;
   if (total <= need2) {
-    for (uint32_t i = tid; i < total; i += kRowThreads) {
+    for (uint32_t i = tid; i < total; i += NT) {
       oi[n_gt + i] = (int32_t)list[i].y;
       if (ov) ov[n_gt + i] = acc.value((int)i);
     }
@@ -519,11 +538,14 @@ __device__ void select_list(uint2* list, int c, uint32_t need, uint32_t lo, int 
   }
 }
 
-__global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
-                                                                 const int32_t* __restrict__ n, int L, int topk,
-                                                                 int32_t* __restrict__ idx,
-                                                                 float* __restrict__ score_opt) {
-  extern __shared__ uint2 list[];  // [kRowList]
+// Rows of scores [T, ld]; ids == nullptr: entry p < n_t is token p; otherwise entry p < P is token
+// ids[t P + p] (empty when outside [0, n_t)), and P <= LIST.
+template <int NT, int LIST, int MINB>
+__global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
+                                                            const int32_t* __restrict__ ids_all, int P,
+                                                            const int32_t* __restrict__ n, int L, int topk,
+                                                            int32_t* __restrict__ idx, float* __restrict__ score_opt) {
+  extern __shared__ uint2 list[];  // [LIST]
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t cnt[2];
@@ -531,11 +553,13 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
   const float* row = scores + (int64_t)t * ld;
+  const int32_t* ids = ids_all ? ids_all + (int64_t)t * P : nullptr;
+  const int np = ids ? P : nt;  // entries of the row
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
   const int tid = threadIdx.x;
-  if (nt <= topk) {  // every prefix token is selected
-    for (int a = tid; a < topk; a += kRowThreads) {
+  if (!ids && nt <= topk) {  // every prefix token is selected
+    for (int a = tid; a < topk; a += NT) {
       oi[a] = a < nt ? a : -1;
       if (ov) ov[a] = a < nt ? row[a] : 0.f;
     }
@@ -553,24 +577,24 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
   float thr = -INFINITY;
   constexpr int ns = kRowSegments * kRowSegLen;
   // expected sample count above the k-th key, plus three standard deviations and a margin
-  const float mean = (float)topk * (float)ns / (float)nt;
+  const float mean = (float)topk * (float)ns / (float)max(np, 1);
   const uint32_t rank = (uint32_t)(mean + 3.f * sqrtf(mean) + 8.f);
-  if (nt > kRowList && rank > (uint32_t)ns) {
+  if (np > LIST && rank > (uint32_t)ns) {
     exact = true;  // k close to n_t: the sample cannot place the cut
     __syncthreads();
-  } else if (nt > kRowList) {
-    const int seg = (nt / kRowSegments) & ~(kRowSegLen - 1);  // >= 32 here
-    constexpr int per = ns / kRowThreads;
+  } else if (np > LIST) {
+    const int seg = (np / kRowSegments) & ~(kRowSegLen - 1);  // >= 32 here
+    constexpr int per = ns / NT;
     uint32_t sk[per];
     uint32_t slo = 0xffffffffu, shi = 0u;
 #pragma unroll
     for (int u = 0; u < per; ++u) {
-      const int i = u * kRowThreads + tid;
+      const int i = u * NT + tid;
       sk[u] = order_key(__ldcg(row + (int64_t)(i / kRowSegLen) * seg + (i % kRowSegLen)));
       slo = min(slo, sk[u]);
       shi = max(shi, sk[u]);
     }
-    for (int b = tid; b < kHistBins; b += kRowThreads) hp[b] = 0;
+    for (int b = tid; b < kHistBins; b += NT) hp[b] = 0;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       slo = min(slo, __shfl_xor_sync(0xffffffffu, slo, o));
@@ -603,38 +627,45 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
 
   // ---- 2-3. candidates and their selection ----
   if (!exact) {
-    collect_above(row, nt, vec, thr, list, kRowList, &cnt[0], mm);
+    collect_above<NT>(row, ids, np, nt, vec, thr, list, LIST, &cnt[0], mm);
     __syncthreads();
     const uint32_t c = cnt[0];
-    if (c >= (uint32_t)topk && c <= (uint32_t)kRowList) {
+    if (np <= LIST && c <= (uint32_t)topk) {  // every valid entry is selected
+      for (uint32_t i = tid; i < (uint32_t)topk; i += NT) {
+        oi[i] = i < c ? (int32_t)list[i].y : -1;
+        if (ov) ov[i] = i < c ? key_to_float(list[i].x) : 0.f;
+      }
+      return;
+    }
+    if (c >= (uint32_t)topk && c <= (uint32_t)LIST) {
       const uint32_t lo = mm[0], range = mm[1] - mm[0];
-      const int sh = __clz(range) > 0 ? (range ? __clz(range) - 1 : 31) : 0;
       if (__clz(range) > 0) {
-        for (uint32_t i = tid; i < c; i += kRowThreads) list[i].x = 0x80000000u | ((list[i].x - lo) << sh);
+        const int sh = range ? __clz(range) - 1 : 31;
+        for (uint32_t i = tid; i < c; i += NT) list[i].x = 0x80000000u | ((list[i].x - lo) << sh);
         __syncthreads();
-        select_list(list, (int)c, (uint32_t)topk, lo, sh, hp, cnt, scratch, oi, ov);
+        select_list<NT, LIST>(list, (int)c, (uint32_t)topk, lo, sh, hp, cnt, scratch, oi, ov);
       } else {  // the keys span more than half the key range: rank them as they are
         const SmemPairs acc{list};
         const SelectResult r = radix_select_items(acc, (int)c, (uint32_t)topk, 0, 0u, 0u, hp, scratch);
         write_selection(acc, (int)c, r, false, oi, ov, (uint32_t)topk, scratch);
       }
-      return;  // topk < n_t keys: every slot is filled
+      return;  // c >= topk entries: every slot is filled
     }
     __syncthreads();
   }
 
-  // ---- exact path: full level-0 histogram, boundary bucket, rank the bucket ----
+  // ---- exact path (score rows only): full level-0 histogram, boundary bucket, rank the bucket ----
   uint32_t kk = 0;  // slots filled
-  for (int b = tid; b < kHistPadded; b += kRowThreads) hp[b] = 0;
+  for (int b = tid; b < kHistPadded; b += NT) hp[b] = 0;
   if (tid < 2) cnt[tid] = 0;
   __syncthreads();
-  row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
+  row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
     (void)s;
     hist_add(hp, (uint32_t)hpad((int)(k >> 20)), in && k != 0u);
   });
   __syncthreads();
   uint32_t local = 0;
-  for (int b = tid; b < kHistBins; b += kRowThreads) local += hp[hpad(b)];
+  for (int b = tid; b < kHistBins; b += NT) local += hp[hpad(b)];
   uint32_t total;
   block_exclusive_scan(local, scratch, &total);
   const uint32_t want = min((uint32_t)topk, total);
@@ -642,7 +673,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
     const Bucket bk = bucket_search_padded(hp, want, scratch);
     const uint32_t pb = bk.prefix >> 20;
     // keys above the bucket straight to the output, the bucket's keys to the list
-    row_sweep(row, nt, vec, [&](int s, uint32_t k, bool in) {
+    row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
       const bool ok = in && k != 0u;
       const bool gt = ok && (k >> 20) > pb;
       const uint32_t slot = warp_slot(gt, &cnt[1]);
@@ -652,16 +683,16 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
       }
       const bool eq = ok && (k >> 20) == pb;
       const uint32_t e = warp_slot(eq, &cnt[0]);
-      if (eq && e < (uint32_t)kRowList) list[e] = make_uint2(k, (uint32_t)s);
+      if (eq && e < (uint32_t)LIST) list[e] = make_uint2(k, (uint32_t)s);
     });
     __syncthreads();
     const uint32_t n_gt = min(cnt[1], (uint32_t)topk);
     const uint32_t c = cnt[0];
     const uint32_t need = min(bk.need, want - n_gt);
-    if (c <= (uint32_t)kRowList) {
+    if (c <= (uint32_t)LIST) {
       const SmemPairs acc{list};
       if (c <= need) {
-        for (uint32_t i = tid; i < c; i += kRowThreads) {
+        for (uint32_t i = tid; i < c; i += NT) {
           oi[n_gt + i] = (int32_t)list[i].y;
           if (ov) ov[n_gt + i] = key_to_float(list[i].x);
         }
@@ -676,10 +707,18 @@ __global__ void __launch_bounds__(kRowThreads, 2) row_topk_kernel(const float* _
     }
     kk = n_gt + need;
   }
-  for (int a = (int)kk + tid; a < topk; a += kRowThreads) {
+  for (int a = (int)kk + tid; a < topk; a += NT) {
     oi[a] = -1;
     if (ov) ov[a] = 0.f;
   }
+}
+
+template <int NT, int LIST, int MINB>
+void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
+                     int topk, int32_t* idx, float* score_opt, cudaStream_t s) {
+  const size_t smem = sizeof(uint2) * (size_t)LIST;
+  cudaFuncSetAttribute(row_topk_kernel<NT, LIST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt);
 }
 
 struct SmemItems {
@@ -769,11 +808,19 @@ void launch_topk_level0(const float* scores, int64_t ld, const int32_t* ids, int
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
                       int topk, void* ws, bool hist_ready, int32_t* idx, float* score_opt, cudaStream_t s) {
   if (T <= 0) return;
-  if (!ids && !hist_ready && T >= kRowKernelMinRows) {  // many rows: one CTA each
-    const size_t smem = sizeof(uint2) * (size_t)kRowList;
-    cudaFuncSetAttribute(row_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    row_topk_kernel<<<T, kRowThreads, smem, s>>>(scores, ld, n, L, topk, idx, score_opt);
-    return;
+  if (!hist_ready) {  // one CTA per row
+    if (ids) {
+      if (P <= kRowListLarge) {
+        launch_row_topk<1024, kRowListLarge, 1>(scores, ld, ids, P, n, T, L, topk, idx, score_opt, s);
+        return;
+      }
+    } else if (T >= kRowKernelMinRows) {
+      launch_row_topk<512, 8192, 2>(scores, ld, nullptr, 0, n, T, L, topk, idx, score_opt, s);
+      return;
+    } else {
+      launch_row_topk<1024, kRowListLarge, 1>(scores, ld, nullptr, 0, n, T, L, topk, idx, score_opt, s);
+      return;
+    }
   }
   const int npos = ids ? P : L;
   uint32_t* hist = static_cast<uint32_t*>(ws);
