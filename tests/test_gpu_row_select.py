@@ -1,9 +1,9 @@
-"""Top-k selection of many score rows (one CTA per row), against a stable sort of the same
-float32 values.  With exact ties going to the lower index the selected set is unique, so the sets
-must be equal.  Row kinds cover the sampled cut, the exact fallback when the sample's candidate
-list is short or overflows, rows whose boundary bucket overflows shared memory (all scores
-equal), heavy ties, negative rows, prefixes up to k (all taken) and up to 4k (exact path), and
-row strides that break 16-byte alignment."""
+"""Top-k selection of score rows (one CTA per row; for a few long rows the candidates are first
+gathered across the GPU), against a stable sort of the same float32 values.  With exact ties going
+to the lower index the selected set is unique, so the sets must be equal.  Row kinds cover the
+sampled cut, the exact fallback when the sample's candidate list is short or overflows, rows whose
+boundary bucket overflows shared memory (all scores equal), heavy ties, negative rows, prefixes up
+to k (all taken) and short rows (list only), and row strides that break 16-byte alignment."""
 import numpy as np
 import pytest
 import torch
@@ -42,11 +42,17 @@ def _rows(T, L, seed):
     return v, n
 
 
-@pytest.mark.parametrize("pad", [0, 1])
-def test_many_rows_match_stable_sort(pad):
+@pytest.mark.parametrize("T,L,pad", [
+    (320, 40000, 0),   # many rows: 2 CTAs of 512 threads per SM
+    (320, 40000, 1),   # row stride not a multiple of 16 bytes
+    (12, 40000, 0),    # a few long rows: candidates gathered across the GPU, then one CTA per row
+    (12, 40000, 1),
+    (40, 20000, 0),    # a few rows just longer than the 16384-entry list
+])
+def test_rows_match_stable_sort(T, L, pad):
     L_ = lib()
-    T, L, k = 320, 40000, 2048
-    v, n = _rows(T, L, seed=pad + 1)
+    k = 2048
+    v, n = _rows(T, L, seed=pad + 1 + T)
     buf = torch.zeros((T, L + pad), dtype=torch.float32)
     buf[:, :L] = torch.from_numpy(v)
     sd = buf.cuda()
