@@ -41,8 +41,8 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "882fa00edb9e7424a1789c4bd4c2617855703325b29011526c34175b4253d28b",
-           "bytes_per_key": (1.074456e9 + 19.13344e6) / 4194304,
+           "sha256": "bcc587b83701c4bd759dede830ba348adeea82ea2d6876db79b0ca9dd54cda2a",
+           "bytes_per_key": (1.073953e9 + 19.169792e6) / 4194304,
            "capture": "profiles/score_persist_decode_L131072_b32.md"}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
 # chunk's launch; the step's traffic is that rate times the pairs the step scores.
