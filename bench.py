@@ -41,7 +41,7 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "bcc587b83701c4bd759dede830ba348adeea82ea2d6876db79b0ca9dd54cda2a",
+           "sha256": "63ad9e52310709f8745fdb1ae7c3406bfae625c2343add5a1deb685d3bae57c2",
            "bytes_per_key": (1.073953e9 + 19.169792e6) / 4194304,
            "capture": "profiles/score_persist_decode_L131072_b32.md"}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one

@@ -59,7 +59,8 @@ int read_and_clear_route_tc_status();
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
 // or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t)).  ws holds
 // topk_rows_ws(T, P or L) bytes, 256-byte aligned; hist_ready: the scoring kernel already filled
-// the level-0 state in ws.  Output order within a row is not specified.
+// the level-0 state in ws (the partition/resolve kernels then select); otherwise one CTA per row
+// selects.  Output order within a row is not specified.
 size_t topk_rows_ws(int T, int P);
 void topk_rows_prepare(void* ws, int T, cudaStream_t s);
 TopkFuse topk_rows_fuse(void* ws, int T, int topk);

@@ -12,7 +12,7 @@
 // sorted, padded to a multiple of 8 with zero-weight slots), so the routed score with h = H_I is
 // the dense score bit for bit.
 //
-// Three kernels:
+// Three kernels here (shared bf16 caches go to score_tc.cu first):
 //   score_persist_kernel  decode (one cache per query): persistent, 2 CTAs per SM; the actual
 //       work (ceil(n_t/128) tiles of 128 rows per query) is flattened and split evenly over the
 //       CTAs, each taking one contiguous range.  Each warp owns 16 rows of every tile and holds
@@ -20,11 +20,13 @@
 //       32 x 131072 keys: 178 us against 185 us for the grid kernel; an added bulk L2 prefetch
 //       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
 //       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
-//   score_grid_kernel     shared caches (prefill): one CTA per (query, chunk of positions).
+//       On request it also builds each row's level-0 selection histogram while it writes the
+//       scores (topk.cu); the default selection reads the scores instead, which measured faster
+//       over a whole decode step (the scorer alone is 13 us faster without the histogram).
+//   score_grid_kernel     one CTA per (query, chunk of positions): shared caches when the
+//       tensor-core kernel (score_tc.cu, which takes shared bf16 caches) cannot run, and more
+//       queries than the persistent schedule takes.
 //   score_f32_kernel      fp32 inputs: one warp per key row on CUDA cores, exact fp32 products.
-// The top-k selection histograms the written scores in passes of its own (topk.cu): counting
-// inside these kernels cost 12-16 us per 32 x 131072 scores, more than a separate pass over the
-// L2-resident scores.
 #include <cuda_bf16.h>
 
 #include "kernels.cuh"

@@ -5,17 +5,19 @@
 // scores; "Hierarchical Variant (MISA-dagger)": the k' candidates are narrowed to the top-k by
 // their dense scores.  Rule: score descending, exact ties to the lower token id (select.cuh).
 //
-// Rows of scores (one per query; a position p is token p, or token ids[p] for candidate lists):
-//   1. level-0 histogram: 4096 buckets of key bits 31..20 per row, and the bucket holding the k-th
-//      key.  The decode scoring kernel builds both while it writes the scores (the CTA that
-//      finishes a row's last tile finds the bucket); otherwise hist_pass_kernel does, with the
-//      same last-CTA rule, in a pass over the rows;
-//   2. partition: keys above the bucket are written out directly (slots reserved with one atomic
-//      per CTA), the bucket's keys go to a (key, id) list;
-//   3. resolve: one CTA per row ranks that list on the remaining 20 key bits and, for exact ties,
-//      on the token id, in shared memory (straight from global memory if the list is too long).
-// On the decode workloads the boundary bucket holds about a tenth of a row.  The selected set is
-// exact; its order in the output is not specified.
+// Rows of scores (one per query; a position p is token p, or token ids[p] for candidate lists).
+// Two ways, both exact; the selected set's order in the output is not specified:
+//   * one CTA per row (row_topk_kernel, the default): a sampled cut, one pass that gathers the
+//     entries at or above it into shared memory, a selection there; an exact path for rows the
+//     sample cannot place (described with the kernel below);
+//   * after a level-0 histogram (4096 buckets of key bits 31..20 per row, and the bucket holding
+//     the k-th key) that the decode scoring kernel builds while it writes the scores (the CTA that
+//     finishes a row's last tile finds the bucket), or that hist_pass_kernel builds in a pass
+//     over the rows with the same last-CTA rule:
+//       partition: keys above the bucket are written out directly (slots reserved with one atomic
+//       per CTA), the bucket's keys go to a (key, id) list;
+//       resolve: one CTA per row ranks that list on the remaining 20 key bits and, for exact ties,
+//       on the token id, in shared memory (straight from global memory if the list is too long).
 // select_small_kernel ranks a short candidate list entirely in one CTA's shared memory; it needs
 // no workspace (used by the entry point without allocation).
 #include "kernels.cuh"
