@@ -151,3 +151,12 @@ def test_binding_rejects_host_tensors():
     from long_context_sparse_mean_b200 import binding
     with pytest.raises(ValueError):
         binding.misa_pool_keys(torch.zeros(10, 128, dtype=torch.bfloat16), 4)
+
+
+def test_device_check_reports_without_a_device(lib):
+    """misa_device_check synchronises and reads the device status word: without a usable device
+    the synchronisation fails and the call says so; with one, nothing has timed out."""
+    import torch
+    want = OK if torch.cuda.is_available() else CUDA
+    assert lib.misa_device_check() == want
+    assert lib.misa_status_str(DEVICE_TIMEOUT) != b"unknown status"
