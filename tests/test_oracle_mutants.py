@@ -3,7 +3,6 @@
 Each mutant is a textual edit of the oracle source (a dropped term, a wrong sign, a wrong index,
 a reversed tie rule ...), compiled into a temporary directory; the real oracle is untouched.
 """
-import os
 
 import pytest
 
