@@ -282,6 +282,75 @@ def check_planted_needles(o):
             assert set(inp.needle_pos.tolist()) <= set(out["idx"][t].tolist()), "needle tokens selected"
 
 
+def check_batch_matches_single_query(o):
+    """The batched drivers (router, scores, MISA, MISA-dagger, dense scores of listed tokens,
+    pooling) give per query exactly what the single-query functions give (which the brute-force
+    pins cover), for one shared cache with a different prefix per query and for one cache per
+    query."""
+    rng = np.random.default_rng(12)
+    T, H_I, d, L, B, h, kk, kp = 6, 8, 16, 90, 7, 3, 10, 25
+    q = rng.integers(-3, 4, size=(T, H_I, d)).astype(np.float32)
+    w = rng.integers(-2, 3, size=(T, H_I)).astype(np.float32)
+    shared = rng.integers(-3, 4, size=(L, d)).astype(np.float32)
+    caches = rng.integers(-3, 4, size=(T, L, d)).astype(np.float32)
+    n = np.array([0, 1, 6, 7, 50, 90], np.int32)
+    for k, kss, kt in ((shared, 0, lambda t: shared), (caches, L * d, lambda t: caches[t])):
+        r_b, h_b = o.route_batch(q, w, k, kss, n, B, h)
+        I_b = o.scores(q, w, k, kss, n, heads=h_b, ld=L)
+        misa = o.indexer(0, q, w, k, kss, n, B, h, kk)
+        dag = o.indexer(1, q, w, k, kss, n, B, h, kk, kp=kp)
+        ids = rng.integers(-2, L + 2, size=(T, 12)).astype(np.int32)
+        F_b = o.dense_scores_at(q, w, k, kss, n, ids)
+        for t in range(T):
+            nt = int(n[t])
+            r1, h1 = o.route(q[t], w[t], kt(t), nt, B, h)
+            assert np.array_equal(r_b[t], r1) and np.array_equal(h_b[t], h1), ("router", kss, t)
+            assert np.array_equal(misa["heads"][t], h1) and np.array_equal(misa["r"][t], r1), ("indexer r", kss, t)
+            I1 = o.token_scores(q[t], w[t], h1, kt(t), nt)
+            assert np.array_equal(I_b[t][:nt], I1) and np.all(np.isnan(I_b[t][nt:])), ("scores", kss, t)
+            sel, _ = o.topk(I1, kk)
+            assert np.array_equal(misa["idx"][t], sel), ("MISA top-k", kss, t)
+            cand, _ = o.topk(I1, kp)
+            assert np.array_equal(dag["cand"][t], cand), ("candidates", kss, t)
+            fin, _ = o.rerank(q[t], w[t], kt(t), nt, cand, kk)
+            assert np.array_equal(dag["idx"][t], fin), ("re-rank", kss, t)
+            F1 = o.token_scores(q[t], w[t], np.arange(H_I, dtype=np.int32), kt(t), nt)
+            want = np.array([F1[i] if 0 <= i < nt else 0.0 for i in ids[t]])
+            assert np.array_equal(F_b[t], want), ("dense scores at ids", kss, t)
+    pooled = o.pool_batch(caches, L * d, T, L, d, B)
+    for t in range(T):
+        assert np.array_equal(pooled[t], o.pool_keys(caches[t], B)), ("pool", t)
+
+
+def check_batch_against_numpy(o):
+    """Batched router (alone and inside the indexer driver) and token scores against NumPy written
+    out per query (float64, integer
+    inputs, so exact up to rounding of the block means), for a shared cache with a different prefix
+    per query and for one cache per query."""
+    rng = np.random.default_rng(13)
+    T, H_I, d, L, B, h = 5, 6, 8, 40, 6, 2
+    q = rng.integers(-3, 4, size=(T, H_I, d)).astype(np.float32)
+    w = rng.integers(-2, 3, size=(T, H_I)).astype(np.float32)
+    shared = rng.integers(-3, 4, size=(L, d)).astype(np.float32)
+    caches = rng.integers(-3, 4, size=(T, L, d)).astype(np.float32)
+    n = np.array([1, 5, 6, 23, 40], np.int32)
+    heads = np.stack([rng.permutation(H_I)[:h] for _ in range(T)]).astype(np.int32)
+    for k, kss, kt in ((shared, 0, lambda t: shared), (caches, L * d, lambda t: caches[t])):
+        r_b, _ = o.route_batch(q, w, k, kss, n, B, h)
+        r_i = o.indexer(0, q, w, k, kss, n, B, h, 3)["r"]
+        I_b = o.scores(q, w, k, kss, n, heads=heads, ld=L)
+        for t in range(T):
+            nt = int(n[t])
+            want_r = _np_router_scores(q[t], w[t], kt(t), nt, B)
+            assert np.allclose(r_b[t], want_r, rtol=1e-12, atol=1e-12), ("router", kss, t)
+            assert np.allclose(r_i[t], want_r, rtol=1e-12, atol=1e-12), ("indexer router", kss, t)
+            K = kt(t)[:nt].astype(np.float64)
+            hs = np.sort(heads[t])
+            want_I = (w[t][hs].astype(np.float64)[:, None] *
+                      np.maximum(q[t][hs].astype(np.float64) @ K.T, 0.0)).sum(axis=0)
+            assert np.allclose(I_b[t][:nt], want_I, rtol=0, atol=1e-12), ("scores", kss, t)
+
+
 ALL_CHECKS = [
     check_hand_example,
     check_topk_vs_stable_argsort,
@@ -297,4 +366,6 @@ ALL_CHECKS = [
     check_empty_and_short,
     check_negative_weight_sign,
     check_planted_needles,
+    check_batch_matches_single_query,
+    check_batch_against_numpy,
 ]

@@ -27,6 +27,11 @@ MUTANTS = {
                                 "orc_dot_ff(q + (int64_t)j, k + s * d, d)"),
     "weight of slot, not of head": ("acc += (double)w[j] * orc_relu(orc_dot_ff(q + (int64_t)j * d, k + s * d, d));",
                                     "acc += (double)w[a] * orc_relu(orc_dot_ff(q + (int64_t)j * d, k + s * d, d));"),
+    "batched driver ignores the cache stride": ("    const float* kt = k + (int64_t)t * k_seq_stride;",
+                                                "    const float* kt = k;"),
+    "batched scores use the first query's prefix": (
+        "    const int64_t nt = n[t] > 0 ? n[t] : 0;\n    orc_token_scores(q + (int64_t)t * H_I * d",
+        "    const int64_t nt = n[0] > 0 ? n[0] : 0;\n    orc_token_scores(q + (int64_t)t * H_I * d"),
     "dense re-rank with half the heads": ("      for (int j = 0; j < H_I; ++j)\n        acc += (double)w[j]",
                                           "      for (int j = 0; j < H_I / 2; ++j)\n        acc += (double)w[j]"),
 }
