@@ -122,9 +122,10 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
  *   scores   : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
  *   select_ws, select_ws_bytes, select_topk : optional (NULL, 0, 0).  A workspace of
  *              misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes in which the call also
- *              leaves the first stage of a top-select_topk selection of these scores (the decode
- *              scoring kernel builds it while it writes the scores); pass the same workspace to
- *              misa_topk_select with ws_prepared = 1.
+ *              leaves the first stage of a top-select_topk selection of these scores (the scoring
+ *              kernel for per-query bf16 caches builds it while it writes the scores, otherwise a
+ *              separate pass does); pass the same workspace to misa_topk_select with
+ *              ws_prepared = 1.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -138,7 +139,9 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
  *   score_opt   : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
  *   ws          : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
  *   ws_prepared : 1 if misa_token_scores already prepared ws for these scores and this topk
- * Scores must be finite.
+ * Scores must be finite.  Without ws_prepared one CTA per row selects (ws carries nothing between
+ * calls); with it the histogram-based selection that misa_token_scores started is completed.
+ * Both give the same set.
  */
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
                              int L, int topk, int32_t* idx, float* score_opt, void* ws,
