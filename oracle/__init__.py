@@ -7,8 +7,9 @@ here, and nothing here imports the CUDA library.
 Every function follows "MISA: Mixture of Indexer Sparse Attention for Long-Context LLM
 Inference" (gist.science/paper/2605.07363), "Technical Summary": "Methodology: MISA" (the
 block-pooled router and the sparse token scoring), "Hierarchical Variant (MISA-dagger)" and
-"Problem Statement" (the dense DSA indexer).  The C source states the formulas and the readings
-taken where the pages are silent.
+"Problem Statement" (the dense DSA indexer).  The block filter composed with MISA follows "HISA:
+Efficient Hierarchical Indexing for Fine-Grained Sparse Attention" (arXiv 2603.28458), abstract.
+The C source states the formulas and the readings taken where the pages are silent.
 """
 from __future__ import annotations
 
@@ -72,6 +73,10 @@ class Oracle:
         lib.orc_dense_scores_at.argtypes = [P, P, P, i64, P, i32, i32, i32, P, i64, P]
         lib.orc_route_batch.argtypes = [P, P, P, i64, P, i32, i32, i32, i32, i32, P, P]
         lib.orc_pool_batch.argtypes = [P, i64, i32, i64, i32, i32, P]
+        lib.orc_block_scores.argtypes = [P, P, P, i32, P, i64, i32, i32, P]
+        lib.orc_block_filter.argtypes = [P, P, P, i32, P, i64, i32, i32, i64, i64, P, P, P, P]
+        lib.orc_block_filter_batch.argtypes = [P, P, P, i64, P, i32, i32, i32, i32, i32, i64, i64, P, P,
+                                               P, P, i64, P, P, P]
         self.lib = lib
         self.path = path
 
@@ -172,6 +177,30 @@ class Oracle:
         heads = np.empty((T, h), np.int32)
         self.lib.orc_route_batch(_p(q), _p(w), _p(k), k_seq_stride, _p(n), T, H_I, d, B, h, _p(r), _p(heads))
         return r, heads
+
+    def block_scores(self, q, w, heads, k, n, B):
+        """Block-filter scores of one query: S[ceil(n/B)] with the given heads."""
+        q, w, k, heads = _f32(q), _f32(w), _f32(k), _i32(heads)
+        out = np.empty(-(-n // B), np.float64)
+        self.lib.orc_block_scores(_p(q), _p(w), _p(heads), heads.shape[0], _p(k), n, q.shape[1], B, _p(out))
+        return out
+
+    def block_filter(self, q, w, k, k_seq_stride, n, B, h, m, topk_, heads_in=None):
+        """Batched MISA with the token-axis block filter (route, keep m blocks, top-k inside them).
+
+        Returns r[T,H_I], heads[T,h], S[T,ceil(max n/B)] (NaN past each query's blocks),
+        blocks[T,m] (descending S, -1 padded), idx[T,k] and idx_v[T,k]."""
+        q, w, k, n = _f32(q), _f32(w), _f32(k), _i32(n)
+        T, H_I, d = q.shape
+        ldS = max(1, -(-int(n.max(initial=0)) // B))
+        out = {"r": np.empty((T, H_I), np.float64), "heads": np.empty((T, h), np.int32),
+               "S": np.full((T, ldS), np.nan, np.float64), "blocks": np.empty((T, m), np.int32),
+               "idx": np.empty((T, topk_), np.int32), "idx_v": np.empty((T, topk_), np.float64)}
+        hin = None if heads_in is None else _i32(heads_in)
+        self.lib.orc_block_filter_batch(_p(q), _p(w), _p(k), k_seq_stride, _p(n), T, H_I, d, B, h, m, topk_,
+                                        _p(hin), _p(out["r"]), _p(out["heads"]), _p(out["S"]), ldS,
+                                        _p(out["blocks"]), _p(out["idx"]), _p(out["idx_v"]))
+        return out
 
 
 _default = None

@@ -16,6 +16,8 @@
  *   - "Hierarchical Variant (MISA-dagger)": the routed pass keeps k' candidates, then the
  *     dense indexer with all H_I heads re-scores only those and keeps the top-k.
  *   - "Problem Statement": the dense DSA indexer scores every prefix token with all H_I heads.
+ *   - "HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse Attention" (arXiv 2603.28458),
+ *     abstract: the token-axis block filter composed with MISA (orc_block_* at the end of the file).
  * The pages never write the score formulas; this oracle fixes them as
  *     token score  I_{t,s} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . k_s)
  *     router score r_{t,j} = w_{t,j} * sum_{b < M_t} max(0, q_{t,j} . kbar_b)
@@ -300,4 +302,112 @@ void orc_pool_batch(const float* k, int64_t k_seq_stride, int n_seq, int64_t L, 
 #pragma omp parallel for schedule(dynamic, 1)
   for (int s = 0; s < n_seq; ++s)
     orc_pool_keys(k + (int64_t)s * k_seq_stride, L, d, B, kbar + (int64_t)s * M * d);
+}
+
+/*
+ * Token-axis block filter composed with MISA ("HISA: Efficient Hierarchical Indexing for
+ * Fine-Grained Sparse Attention", abstract: a block-level coarse filter scores pooled block
+ * representatives and discards regions, then the original indexer runs only inside the kept
+ * candidate blocks, and the selected tokens keep the indexer's top-k form; "MISA: Mixture of
+ * Indexer Sparse Attention ...", "Problem Statement" and "Significance and Claims": HISA saves on
+ * the token axis, MISA on the head axis, and the two are complementary).
+ * Readings where the pages are silent:
+ *   - the pooled block representative is the same block mean the router uses (partial last
+ *     block averaged over its valid keys), and a block is scored with the indexer's own formula
+ *     and the query's routed heads: S[b] = sum_{j in R, ascending} w[j] * max(0, q_j . kbar_b);
+ *     with h = H_I this is the dense indexer's block filter;
+ *   - the m best blocks are kept (value descending, ties to the lower block);
+ *   - the kept blocks' tokens of the prefix are scored with the routed heads, exactly as MISA
+ *     scores them, and the top kk of those are selected (ties to the lower token).
+ */
+void orc_block_scores(const float* q, const float* w, const int32_t* heads, int nh,
+                      const float* k, int64_t n, int d, int B, double* S) {
+  const int64_t M = (n + B - 1) / B;
+  double* kbar = (double*)malloc(sizeof(double) * (size_t)(M > 0 ? M : 1) * (size_t)d);
+  int32_t* hs = (int32_t*)malloc(sizeof(int32_t) * (size_t)(nh > 0 ? nh : 1));
+  orc_pool_keys(k, n, d, B, kbar);
+  memcpy(hs, heads, sizeof(int32_t) * (size_t)nh);
+  qsort(hs, (size_t)nh, sizeof(int32_t), orc_int_cmp);
+  for (int64_t b = 0; b < M; ++b) {
+    double acc = 0.0;
+    for (int a = 0; a < nh; ++a) {
+      const int j = hs[a];
+      acc += (double)w[j] * orc_relu(orc_dot_fd(q + (int64_t)j * d, kbar + b * d, d));
+    }
+    S[b] = acc;
+  }
+  free(kbar);
+  free(hs);
+}
+
+/*
+ * Block filter + refinement for one query with the heads heads[nh]: S[ceil(n/B)] block scores,
+ * blocks[m] the kept blocks by descending S (-1 padded), out[kk] / out_v[kk] the selected tokens.
+ */
+void orc_block_filter(const float* q, const float* w, const int32_t* heads, int nh, const float* k,
+                      int64_t n, int d, int B, int64_t m, int64_t kk, double* S, int32_t* blocks,
+                      int32_t* out, double* out_v) {
+  const int64_t M = (n + B - 1) / B;
+  orc_block_scores(q, w, heads, nh, k, n, d, B, S);
+  orc_topk(S, NULL, M, m, blocks, NULL);
+  int64_t cnt = 0;
+  for (int64_t a = 0; a < m; ++a) {
+    if (blocks[a] < 0) continue;
+    const int64_t s0 = (int64_t)blocks[a] * B;
+    cnt += ((s0 + B < n) ? s0 + B : n) - s0;
+  }
+  double* I = (double*)malloc(sizeof(double) * (size_t)(cnt > 0 ? cnt : 1));
+  int32_t* ids = (int32_t*)malloc(sizeof(int32_t) * (size_t)(cnt > 0 ? cnt : 1));
+  int64_t c = 0;
+  for (int64_t a = 0; a < m; ++a) {
+    if (blocks[a] < 0) continue;
+    const int64_t s0 = (int64_t)blocks[a] * B;
+    const int64_t s1 = (s0 + B < n) ? s0 + B : n;
+    orc_token_scores(q, w, heads, nh, k + s0 * d, s1 - s0, d, I + c);
+    for (int64_t s = s0; s < s1; ++s) ids[c++] = (int32_t)s;
+  }
+  orc_topk(I, ids, cnt, kk, out, out_v);
+  free(I);
+  free(ids);
+}
+
+/*
+ * Batched MISA + block filter over T queries (layouts as in orc_indexer_batch): route h heads
+ * (or take heads_in[T,h]), then orc_block_filter keeping m blocks and kk tokens.  Outputs (NULL
+ * to skip): r[T,H_I], heads[T,h], S[T,ldS] (entries past ceil(n_t/B) untouched), blocks[T,m],
+ * idx[T,kk], idx_v[T,kk].
+ */
+void orc_block_filter_batch(const float* q, const float* w, const float* k, int64_t k_seq_stride,
+                            const int32_t* n, int T, int H_I, int d, int B, int h, int64_t m,
+                            int64_t kk, const int32_t* heads_in, double* r_out, int32_t* heads_out,
+                            double* S_out, int64_t ldS, int32_t* blocks_out, int32_t* idx,
+                            double* idx_v) {
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int t = 0; t < T; ++t) {
+    const float* qt = q + (int64_t)t * H_I * d;
+    const float* wt = w + (int64_t)t * H_I;
+    const float* kt = k + (int64_t)t * k_seq_stride;
+    const int64_t nt = n[t] > 0 ? n[t] : 0;
+    const int64_t Mt = (nt + B - 1) / B;
+    double* r = (double*)malloc(sizeof(double) * (size_t)H_I);
+    int32_t* hd = (int32_t*)malloc(sizeof(int32_t) * (size_t)H_I);
+    double* S = (double*)malloc(sizeof(double) * (size_t)(Mt > 0 ? Mt : 1));
+    int32_t* bl = (int32_t*)malloc(sizeof(int32_t) * (size_t)(m > 0 ? m : 1));
+    if (heads_in) {
+      memcpy(hd, heads_in + (int64_t)t * h, sizeof(int32_t) * (size_t)h);
+      for (int j = 0; j < H_I; ++j) r[j] = 0.0;
+    } else {
+      orc_route(qt, wt, kt, nt, H_I, d, B, h, r, hd);
+    }
+    orc_block_filter(qt, wt, hd, h, kt, nt, d, B, m, kk, S, bl, idx + (int64_t)t * kk,
+                     idx_v ? idx_v + (int64_t)t * kk : NULL);
+    if (r_out) memcpy(r_out + (int64_t)t * H_I, r, sizeof(double) * (size_t)H_I);
+    if (heads_out) memcpy(heads_out + (int64_t)t * h, hd, sizeof(int32_t) * (size_t)h);
+    if (S_out) memcpy(S_out + (int64_t)t * ldS, S, sizeof(double) * (size_t)Mt);
+    if (blocks_out) memcpy(blocks_out + (int64_t)t * m, bl, sizeof(int32_t) * (size_t)m);
+    free(r);
+    free(hd);
+    free(S);
+    free(bl);
+  }
 }

@@ -15,7 +15,11 @@ LLM Inference", gist.science/paper/2605.07363, "Methodology: MISA" and "Hierarch
     relabelling heads permutes the router scores; h = H_I is the dense indexer bit for bit;
     k' >= n makes MISA-dagger the dense indexer, k' = k makes it MISA, and the dense top-k
     restricted to the candidates is always kept; keys past a query's prefix change nothing;
-  * a planted needle (the tiny fp32 workload) is routed and selected.
+  * a planted needle (the tiny fp32 workload) is routed and selected;
+  * the block filter composed with MISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained
+    Sparse Attention", abstract): hand-derived cases, every block kept is MISA, B = 1 turns block
+    scores into token scores, block scores sum to the routed heads' router scores, and the
+    selection is MISA's top-k restricted to the kept blocks.
 """
 from __future__ import annotations
 
@@ -351,6 +355,118 @@ def check_batch_against_numpy(o):
             assert np.allclose(I_b[t][:nt], want_I, rtol=0, atol=1e-12), ("scores", kss, t)
 
 
+def check_block_filter_hand_example(o):
+    """Hand-derived cases of the block filter composed with MISA (tests/golden/hand_example.json,
+    "block_filter"): block scores, kept blocks, selected tokens, with exact ties."""
+    g = _load_golden()
+    k = np.array(g["keys"], np.float32)
+    q = np.array(g["q"], np.float32)
+    w = np.array(g["w"], np.float32)
+    for c in g["block_filter"]["cases"]:
+        n, B, h, m, kk = c["n"], c["B"], c["h"], c["m"], c["k"]
+        res = o.block_filter(q[None], w[None], k, 0, np.array([n]), B, h, m, kk)
+        tag = f"n={n} B={B} h={h} m={m} k={kk}"
+        assert np.array_equal(res["S"][0], np.array(c["S"], np.float64)), f"block scores {tag}: {res['S'][0]}"
+        blocks = res["blocks"][0]
+        assert list(blocks[:len(c["blocks"])]) == c["blocks"] and np.all(blocks[len(c["blocks"]):] == -1), \
+            f"kept blocks {tag}: {blocks}"
+        got = res["idx"][0]
+        want = c["idx"]
+        valid = [s for s in want if s >= 0]
+        assert sorted(got[:len(valid)].tolist()) == sorted(valid) and np.all(got[len(valid):] == -1), \
+            f"selection {tag}: {got}"
+        S1 = o.block_scores(q, w, res["heads"][0], k, n, B)
+        assert np.array_equal(S1, res["S"][0]), f"single-query block scores {tag}"
+
+
+def _kept_tokens(blocks, n, B):
+    return {s for b in blocks if b >= 0 for s in range(b * B, min((b + 1) * B, n))}
+
+
+def check_block_filter_reductions(o):
+    """Keeping every block is MISA bit for bit; with B = 1 the block scores are the token scores
+    and keeping m >= k blocks is MISA again; with h = H_I and every block kept it is the dense
+    indexer."""
+    q, w, k = _small_clustered(8, H_I=8, d=16, L=300)
+    Q = np.stack([q, q[::-1], 0.5 * q])
+    W = np.stack([w, w[::-1], -w])
+    n = np.array([300, 217, 9], np.int32)
+    H_I = q.shape[0]
+    for B, h, kk in ((16, 3, 20), (7, 2, 64), (64, 5, 5)):
+        M = -(-300 // B)
+        misa = o.indexer(0, Q, W, k, 0, n, B, h, kk)
+        for m in (M, M + 3):
+            bf = o.block_filter(Q, W, k, 0, n, B, h, m, kk)
+            for key in ("r", "heads", "idx", "idx_v"):
+                assert np.array_equal(bf[key], misa[key]), f"every block kept: {key} differs (B={B})"
+        dense = o.indexer(2, Q, W, k, 0, n, B, h, kk)
+        bf = o.block_filter(Q, W, k, 0, n, B, H_I, M, kk)
+        assert np.array_equal(bf["idx"], dense["idx"]) and np.array_equal(bf["idx_v"], dense["idx_v"]), \
+            f"h = H_I with every block kept is the dense indexer (B={B})"
+    for h, kk in ((2, 10), (4, 33)):
+        misa = o.indexer(0, Q, W, k, 0, n, 1, h, kk)
+        I = o.scores(Q, W, k, 0, n, heads=misa["heads"], ld=300)
+        for m in (kk, kk + 7):
+            bf = o.block_filter(Q, W, k, 0, n, 1, h, m, kk)
+            for t in range(3):
+                nt = int(n[t])
+                assert np.array_equal(bf["S"][t][:nt], I[t][:nt]), "B = 1: block scores are token scores"
+            assert np.array_equal(bf["idx"], misa["idx"]), "B = 1 and m >= k: MISA's selection"
+
+
+def check_block_filter_invariants(o):
+    """Block scores sum to the routed heads' router scores; the kept blocks are the m best block
+    scores; the selection is MISA's top-k restricted to the kept blocks' tokens, so MISA's own
+    picks inside kept blocks survive; scaling and keys past the prefix act as for MISA; the
+    batched driver matches the single-query block scores for a shared cache and per-query caches."""
+    rng = np.random.default_rng(14)
+    T, H_I, d, L = 5, 8, 16, 260
+    q = rng.standard_normal((T, H_I, d)).astype(np.float32)
+    w = (rng.standard_normal((T, H_I)) / math.sqrt(H_I)).astype(np.float32)
+    shared = rng.standard_normal((L, d)).astype(np.float32)
+    caches = rng.standard_normal((T, L, d)).astype(np.float32)
+    n = np.array([0, 1, 37, 200, 260], np.int32)
+    for k, kss, kt in ((shared, 0, lambda t: shared), (caches, L * d, lambda t: caches[t])):
+        for B, h, m, kk in ((16, 3, 4, 20), (13, 2, 1, 8), (32, 4, 3, 100), (10, 1, 0, 5)):
+            bf = o.block_filter(q, w, k, kss, n, B, h, m, kk)
+            misa = o.indexer(0, q, w, k, kss, n, B, h, kk)
+            assert np.array_equal(bf["heads"], misa["heads"]) and np.array_equal(bf["r"], misa["r"]), "routing"
+            I = o.scores(q, w, k, kss, n, heads=bf["heads"], ld=L)
+            for t in range(T):
+                nt = int(n[t])
+                Mt = -(-nt // B)
+                S = bf["S"][t][:Mt]
+                tag = (kss, B, m, t)
+                assert np.all(np.isnan(bf["S"][t][Mt:])), tag
+                assert np.array_equal(S, o.block_scores(q[t], w[t], bf["heads"][t], kt(t), nt, B)), tag
+                routed = float(sum(misa["r"][t][j] for j in bf["heads"][t]))
+                assert abs(S.sum() - routed) <= 1e-12 * max(1.0, abs(routed)), ("sum of block scores", tag)
+                blocks = bf["blocks"][t]
+                want_b = np.argsort(-S, kind="stable")[:m]
+                assert np.array_equal(blocks[:len(want_b)], want_b) and np.all(blocks[len(want_b):] == -1), \
+                    ("kept blocks", tag)
+                kept = _kept_tokens(blocks, nt, B)
+                sel = [s for s in bf["idx"][t] if s >= 0]
+                assert set(sel) <= kept, ("selection outside the kept blocks", tag)
+                assert len(sel) == min(kk, len(kept)) and np.all(bf["idx"][t][len(sel):] == -1), tag
+                masked = np.where([s in kept for s in range(nt)], I[t][:nt], -np.inf)
+                want = np.argsort(-masked, kind="stable")[:min(kk, len(kept))]
+                assert sorted(sel) == sorted(want.tolist()), ("restricted top-k", tag)
+                assert np.array_equal(np.sort(bf["idx_v"][t][:len(sel)]), np.sort(I[t][sel])), tag
+                assert (set(misa["idx"][t].tolist()) & kept) <= set(sel), ("MISA picks in kept blocks", tag)
+    q1, w1, k1 = q[3], w[3], shared
+    base = o.block_filter(q1[None], w1[None], k1, 0, np.array([200]), 16, 3, 4, 20)
+    for name, (q2, w2, k2) in {"k": (q1, w1, 2 * k1), "q": (2 * q1, w1, k1), "w": (q1, 2 * w1, k1)}.items():
+        sc = o.block_filter(q2[None], w2[None], k2, 0, np.array([200]), 16, 3, 4, 20)
+        assert np.array_equal(sc["S"], 2 * base["S"]), f"block scores scale with {name}"
+        assert np.array_equal(sc["blocks"], base["blocks"]) and np.array_equal(sc["idx"], base["idx"]), name
+    k3 = k1.copy()
+    k3[200:] = 1000.0 * np.sign(k3[200:]) + 3.0
+    past = o.block_filter(q1[None], w1[None], k3, 0, np.array([200]), 16, 3, 4, 20)
+    for key in ("r", "heads", "S", "blocks", "idx", "idx_v"):
+        assert np.array_equal(past[key], base[key], equal_nan=True), f"keys past the prefix changed {key}"
+
+
 ALL_CHECKS = [
     check_hand_example,
     check_topk_vs_stable_argsort,
@@ -368,4 +484,7 @@ ALL_CHECKS = [
     check_planted_needles,
     check_batch_matches_single_query,
     check_batch_against_numpy,
+    check_block_filter_hand_example,
+    check_block_filter_reductions,
+    check_block_filter_invariants,
 ]

@@ -32,6 +32,23 @@ MUTANTS = {
     "batched scores use the first query's prefix": (
         "    const int64_t nt = n[t] > 0 ? n[t] : 0;\n    orc_token_scores(q + (int64_t)t * H_I * d",
         "    const int64_t nt = n[0] > 0 ? n[0] : 0;\n    orc_token_scores(q + (int64_t)t * H_I * d"),
+    "block score without relu": (
+        "acc += (double)w[j] * orc_relu(orc_dot_fd(q + (int64_t)j * d, kbar + b * d, d));",
+        "acc += (double)w[j] * (orc_dot_fd(q + (int64_t)j * d, kbar + b * d, d));"),
+    "block score ignores head weight": (
+        "acc += (double)w[j] * orc_relu(orc_dot_fd(q + (int64_t)j * d, kbar + b * d, d));",
+        "acc += orc_relu(orc_dot_fd(q + (int64_t)j * d, kbar + b * d, d));"),
+    "block score with the first heads, not the routed ones": (
+        "      const int j = hs[a];\n      acc += (double)w[j] * orc_relu(orc_dot_fd(",
+        "      const int j = a;\n      acc += (double)w[j] * orc_relu(orc_dot_fd("),
+    "partial last block never kept": ("  const int64_t M = (n + B - 1) / B;\n  orc_block_scores(",
+                                      "  const int64_t M = n / B;\n  orc_block_scores("),
+    "filter keeps the leading blocks": (
+        "  orc_topk(S, NULL, M, m, blocks, NULL);",
+        "  for (int64_t a = 0; a < m; ++a) blocks[a] = a < M ? (int32_t)a : -1;"),
+    "kept block's tokens taken from the block before": (
+        "    const int64_t s0 = (int64_t)blocks[a] * B;",
+        "    const int64_t s0 = (int64_t)(blocks[a] > 0 ? blocks[a] - 1 : 0) * B;"),
     "dense re-rank with half the heads": ("      for (int j = 0; j < H_I; ++j)\n        acc += (double)w[j]",
                                           "      for (int j = 0; j < H_I / 2; ++j)\n        acc += (double)w[j]"),
 }
