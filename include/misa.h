@@ -71,7 +71,8 @@ typedef enum {
   MISA_OP_SCORE_TOPK = 1,
   MISA_OP_RERANK = 2,
   MISA_OP_DENSE_TOPK = 3,
-  MISA_OP_TOPK_SELECT = 4
+  MISA_OP_TOPK_SELECT = 4,
+  MISA_OP_BLOCK_FILTER = 5
 } misa_op;
 
 /* Largest k' accepted by misa_hier_rerank (its candidates are ranked in shared memory). */
@@ -85,7 +86,8 @@ const char* misa_status_str(int status);
 
 /*
  * Workspace bytes needed by one call of `op` with these sizes (0 if it needs none).
- * Arguments an op does not use are ignored.  Sizes <= 0 give 0.
+ * Arguments an op does not use are ignored.  Sizes <= 0 give 0.  For MISA_OP_BLOCK_FILTER the
+ * last argument carries m, the number of kept blocks (0 when m * B exceeds MISA_MAX_KP).
  */
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp);
 
@@ -183,6 +185,36 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
                            const int32_t* n, int T, int L, int H_I, int d, int topk, int dtype,
                            int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
                            void* stream);
+
+/*
+ * Token-axis block filter composed with MISA ("HISA: Efficient Hierarchical Indexing for
+ * Fine-Grained Sparse Attention", arXiv 2603.28458, abstract: a coarse stage scores pooled block
+ * representatives and keeps candidate blocks, then the indexer scores only their tokens; "MISA",
+ * "Problem Statement" and "Significance and Claims": token-axis and head-axis savings combine).
+ * For query t with routed heads R_t (heads[t], from misa_route):
+ *   S_{t,b} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . kbar_b)     (b < M_t = ceil(n_t/B))
+ * with kbar_b the router's block means (a partial last block averaged over its valid keys); the m
+ * blocks with the largest S_{t,b} are kept (ties: lower block); their prefix tokens are scored
+ * with I_{t,s} and the top-k of those is selected (ties: lower token).  m >= M_t gives exactly
+ * misa_score_topk's selection; h = H_I gives the block filter on the dense indexer.
+ *   kbar             : fp32 block means from misa_pool_keys, 16-byte aligned; query t reads
+ *                      kbar + t*kbar_seq_stride (0 = shared; else a multiple of 4, >= M*d)
+ *   heads            : [T, h] routed heads (entries outside [0, H_I) count as weight 0)
+ *   m                : blocks kept per query, 1 <= m with m * B <= MISA_MAX_KP
+ *   block_scores_opt : out [T, ld_block_scores] fp32 S_{t,b} for b < M_t (ld >= ceil(L/B)), or NULL
+ *   blocks           : out [T, m] kept blocks, -1 padded (order unspecified)
+ *   idx, score_opt   : out [T, topk] selected tokens (-1 padded when the kept blocks hold fewer
+ *                      than topk prefix tokens) and their scores I, or NULL for score_opt
+ *   ws               : misa_workspace_bytes(MISA_OP_BLOCK_FILTER, T, L, H_I, B, h, topk, m) bytes
+ * Errors as above; m * B > MISA_MAX_KP gives MISA_ERR_UNSUPPORTED.
+ */
+misa_status misa_block_filter_topk(const void* q, const float* w, const void* k,
+                                   int64_t k_seq_stride, const float* kbar,
+                                   int64_t kbar_seq_stride, const int32_t* n,
+                                   const int32_t* heads, int T, int L, int H_I, int d, int B, int h,
+                                   int m, int topk, int dtype, float* block_scores_opt,
+                                   int64_t ld_block_scores, int32_t* blocks, int32_t* idx,
+                                   float* score_opt, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Device-side status of the calls made so far on the current device.  The tensor-core scoring

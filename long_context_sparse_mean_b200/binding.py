@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(PKG, "libmisa.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
 BF16, F32 = 0, 1
-OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT = range(5)
+OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT, OP_BLOCK_FILTER = range(6)
 MAX_KP = 16384
 
 if not os.path.exists(LIB_PATH):
@@ -50,6 +50,8 @@ def _setup(lib):
         "misa_score_topk": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, P, sz, P], i32),
         "misa_hier_rerank": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
         "dsa_dense_topk": ([P, P, P, i64, P, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
+        "misa_block_filter_topk": ([P, P, P, i64, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, i32, i32, P,
+                                    i64, P, P, P, P, sz, P], i32),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -301,12 +303,53 @@ def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, w
     return idx, vals
 
 
+def misa_block_filter_topk(q, w, k, kbar, n, heads, B: int, m: int, topk: int, idx=None, vals=None,
+                           blocks=None, block_scores=None, want_vals=True, want_block_scores=False,
+                           ws: Optional[Workspace] = None, stream=None):
+    """Block filter + routed refinement: block scores with the routed heads, the m best blocks,
+    then top-k over their tokens -> dict with idx [T, k], vals [T, k] (or None), blocks [T, m]
+    (-1 padded; order not specified) and, if asked, block_scores [T, ceil(L/B)]."""
+    _need(q, "q")
+    _need(k, "k")
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(kbar, "kbar", torch.float32)
+    _need(heads, "heads", torch.int32)
+    T, H_I, d = q.shape
+    L, _, kss = _cache_geometry(k, T)
+    kbss = 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
+    h = heads.shape[1]
+    M = -(-L // B)
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    if blocks is None:
+        blocks = torch.empty((T, m), dtype=torch.int32, device=q.device)
+    if block_scores is None and want_block_scores:
+        block_scores = torch.empty((T, M), dtype=torch.float32, device=q.device)
+    ld_bs = 0 if block_scores is None else block_scores.shape[1]
+    nbytes = misa_workspace_bytes(OP_BLOCK_FILTER, T, L, H_I, B, h, topk, m)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_block_filter_topk", _lib.misa_block_filter_topk(
+        _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), _p(heads), T, L, H_I, d, B, h, m, topk, _dtype_code(q),
+        _p(block_scores), ld_bs, _p(blocks), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
+    return {"idx": idx, "vals": vals, "blocks": blocks, "block_scores": block_scores}
+
+
 def misa_indexer(q, w, k, kbar, n, B: int, h: int, topk: int, kp: Optional[int] = None,
-                 ws: Optional[Workspace] = None, stream=None):
+                 ws: Optional[Workspace] = None, stream=None, m: Optional[int] = None):
     """The whole indexer for one batch: route -> routed scoring -> top-k (MISA), or with kp given
-    route -> routed scoring -> top-k' candidates -> dense re-rank -> top-k (MISA-dagger).
-    Returns a dict with idx [T, k], vals [T, k], heads [T, h] and (MISA-dagger) cand [T, k']."""
+    route -> routed scoring -> top-k' candidates -> dense re-rank -> top-k (MISA-dagger), or with
+    m given route -> block filter keeping m blocks -> routed scoring of their tokens -> top-k.
+    Returns a dict with idx [T, k], vals [T, k], heads [T, h], (MISA-dagger) cand [T, k'] and
+    (block filter) blocks [T, m]."""
+    if kp is not None and m is not None:
+        raise ValueError("give kp (MISA-dagger) or m (block filter), not both")
     heads, _ = misa_route(q, w, k, kbar, n, B, h, ws=ws, stream=stream)
+    if m is not None:
+        res = misa_block_filter_topk(q, w, k, kbar, n, heads, B, m, topk, ws=ws, stream=stream)
+        return {"idx": res["idx"], "vals": res["vals"], "heads": heads, "blocks": res["blocks"]}
     if kp is None:
         idx, vals = misa_score_topk(q, w, k, n, heads, topk, ws=ws, stream=stream)
         return {"idx": idx, "vals": vals, "heads": heads}

@@ -2,6 +2,8 @@
 // The declarations and their documentation are in include/misa.h.
 #include <cuda_runtime.h>
 
+#include <algorithm>
+
 #include "../../include/misa.h"
 #include "kernels.cuh"
 
@@ -69,6 +71,16 @@ size_t rerank_ws(int T, int kp) {
   return align_up(sizeof(float) * (size_t)T * kp) + select_bytes(T, kp);
 }
 
+// misa_block_filter_topk: [block scores][M_t per query][token ids of the kept blocks]
+// [their scores][selection]
+size_t block_filter_ws(int T, int L, int B, int m) {
+  if (T <= 0 || L <= 0 || B <= 0 || m <= 0 || (int64_t)m * B > MISA_MAX_KP) return 0;
+  const int M = (int)ceil_div(L, B);
+  const int64_t P = (int64_t)m * B;
+  return align_up(sizeof(float) * (size_t)T * score_ld(M)) + align_up(sizeof(int32_t) * (size_t)T) +
+         2 * align_up(sizeof(float) * (size_t)T * P) + select_bytes(T, (int)std::max<int64_t>(M, P));
+}
+
 }  // namespace
 
 extern "C" {
@@ -115,6 +127,8 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
       return rerank_ws(T, kp);
     case MISA_OP_TOPK_SELECT:
       return select_bytes(T, L);
+    case MISA_OP_BLOCK_FILTER:
+      return block_filter_ws(T, L, B, kp);
     default:
       return 0;
   }
@@ -257,6 +271,49 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
                       nullptr, as_stream(stream));
   misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, sel, false, idx, score_opt, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_block_filter_topk(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n,
+                                   const int32_t* heads, int T, int L, int H_I, int d, int B, int h, int m,
+                                   int topk, int dtype, float* block_scores_opt, int64_t ld_block_scores,
+                                   int32_t* blocks, int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (B < 1 || h < 1 || h > H_I || m < 1 || topk < 1 || kbar_seq_stride < 0) return MISA_ERR_INVALID_ARG;
+  if ((int64_t)m * B > MISA_MAX_KP) return MISA_ERR_UNSUPPORTED;
+  const int M = (int)ceil_div(L, B);
+  if (kbar_seq_stride != 0 && (kbar_seq_stride < (int64_t)M * d || kbar_seq_stride % 4 != 0))
+    return MISA_ERR_INVALID_ARG;
+  if (block_scores_opt && ld_block_scores < M) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!kbar || !heads || !blocks || !idx || (reinterpret_cast<uintptr_t>(kbar) & 15) != 0)
+    return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < block_filter_ws(T, L, B, m) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  const int P = m * B;
+  char* p = static_cast<char*>(ws);
+  float* S = block_scores_opt;
+  int64_t ldS = ld_block_scores;
+  if (!S) {
+    S = reinterpret_cast<float*>(p);
+    ldS = score_ld(M);
+  }
+  p += align_up(sizeof(float) * (size_t)T * score_ld(M));
+  int32_t* Mt = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T);
+  int32_t* rows = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(float) * (size_t)T * P);
+  float* F = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * P);
+  const cudaStream_t s = as_stream(stream);
+  misa::launch_block_scores(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, heads, T, L, H_I, B,
+                            h, S, ldS, Mt, s);
+  misa::launch_topk_rows(S, ldS, nullptr, 0, Mt, T, M, m, p, false, blocks, nullptr, s);
+  misa::launch_expand_blocks(blocks, m, n, T, L, B, rows, s);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, P, F, P, nullptr, s);
+  misa::launch_topk_rows(F, P, rows, P, n, T, L, topk, p, false, idx, score_opt, s);
   return launch_status();
 }
 

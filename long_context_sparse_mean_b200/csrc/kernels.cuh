@@ -76,4 +76,15 @@ size_t topk_cand_smem(int P);
 void launch_topk_cand(const float* F, const int32_t* cand, const int32_t* n, int T, int L, int P,
                       int topk, int32_t* idx, float* score_opt, cudaStream_t s);
 
+// Token-axis block filter composed with MISA (block_filter.cu).  Block scores of every query with
+// its routed heads: S[t, b] = sum_{j in heads[t]} w[t, j] * max(0, q[t, j] . kbar_b) for
+// b < M_t = ceil(n_t / B), where full blocks come from kbar and a partial last block is averaged
+// from k; Mt[t] receives M_t.  Entries b >= M_t are not written.
+void launch_block_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                         const float* kbar, int64_t kbar_seq_stride, const int32_t* n, const int32_t* heads, int T,
+                         int L, int H_I, int B, int h, float* S, int64_t ldS, int32_t* Mt, cudaStream_t s);
+// rows[t, a*B + i] = blocks[t, a]*B + i, or -1 for an empty slot or a token past the prefix.
+void launch_expand_blocks(const int32_t* blocks, int m, const int32_t* n, int T, int L, int B, int32_t* rows,
+                          cudaStream_t s);
+
 }  // namespace misa

@@ -11,6 +11,11 @@ Tolerances (derived from the arithmetic; the target is 1e-3 relative for fp32 ac
     (the block means are fp32 sums of up to B keys, whose rounding scales with the keys, not
     with their mean)
   * block means: |gpu - oracle| <= 2 c 2^-24 mean_{s}|k_{s,i}| + 2^-23 |oracle|  (c keys summed)
+  * block-filter score of block b with head set R (block mean of c keys):
+        |gpu - oracle| <= 1e-3 * sum_{j in R} |w_j| |q_j . kbar_b|
+                          + (1e-5 + 2 c 2^-24) * sum_{j in R} |w_j| |q_j| mean_{s in b} |k_s|
+    (the fp32 mean errs by up to 2 c 2^-24 of the mean key size, so its dot product with q_j by
+    that much of |q_j| mean |k_s|; the dot product itself by the same floor as a token score)
 Selections (top-h heads, top-k tokens): tau is the oracle's k-th value; the tie band is every item
 whose oracle value is within tol_item + tol_tau of tau.  The GPU set must have the right size, no
 duplicates, only valid ids; every oracle item outside the band must be in the GPU set and every
@@ -52,6 +57,26 @@ def router_tol(q, w, k, n, B):
     mean_norm = np.array([norms[b * B:min((b + 1) * B, n)].mean() for b in range(M)])
     D = q @ means.T
     return np.abs(w) * (SCORE_REL * np.abs(D).sum(axis=1) + SCORE_FLOOR * np.linalg.norm(q, axis=1) * mean_norm.sum())
+
+
+def block_tol(q, w, k, n, B, heads):
+    """Per-block tolerance [ceil(n/B)] of one query's block-filter scores with the given heads."""
+    q = np.asarray(q, np.float64)
+    w = np.asarray(w, np.float64)
+    K = np.asarray(k[:n], np.float64)
+    M = -(-n // B)
+    if M == 0:
+        return np.zeros(0)
+    hs = np.asarray(heads)
+    Q = q[hs]
+    W = np.abs(w[hs])
+    means = np.stack([K[b * B:min((b + 1) * B, n)].mean(axis=0) for b in range(M)])
+    norms = np.linalg.norm(K, axis=1)
+    mean_norm = np.array([norms[b * B:min((b + 1) * B, n)].mean() for b in range(M)])
+    count = np.array([min((b + 1) * B, n) - b * B for b in range(M)], np.float64)
+    A = W @ np.abs(Q @ means.T)
+    floor = (SCORE_FLOOR + 2 * count * 2.0 ** -24) * (W * np.linalg.norm(Q, axis=1)).sum() * mean_norm
+    return SCORE_REL * A + floor
 
 
 def pool_tol(k, n, B, kbar_oracle):

@@ -35,7 +35,7 @@ def test_header_declares_the_indexer_calls():
     names = declared_functions()
     for want in ("misa_pool_keys", "misa_route", "misa_token_scores", "misa_topk_select", "misa_score_topk",
                  "misa_hier_rerank", "dsa_dense_topk", "misa_workspace_bytes", "misa_status_str", "misa_version",
-                 "misa_device_check"):
+                 "misa_device_check", "misa_block_filter_topk"):
         assert want in names, want
 
 
@@ -70,6 +70,15 @@ def test_workspace_sizes(lib):
     # re-rank: [T, k'] dense scores + the select workspace over k' positions
     assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + _al(32 * 4104 * 4 + 32 * 8192 * 8)
     assert ws(1, 0, 100, 64, 1, 8, 10, 0) == 0
+    # block filter (m in the last slot): [T, ceil4(M)] block scores, [T] block counts, [T, m*B] token
+    # ids and [T, m*B] their scores, then the select workspace over max(M, m*B) positions
+    P, M = 128 * 128, 1024
+    assert ws(5, 32, 131072, 64, 128, 8, 2048, 128) == (32 * M * 4 + 256 + 2 * 32 * P * 4 +
+                                                        _al(32 * 4104 * 4 + 32 * P * 8))
+    assert ws(5, 3, 1001, 64, 7, 8, 10, 5) == (_al(3 * 144 * 4) + 256 + 2 * _al(3 * 35 * 4) +
+                                               _al(3 * 4104 * 4 + 3 * 143 * 8))
+    assert ws(5, 32, 131072, 64, 128, 8, 2048, 129) == 0  # m * B above the candidate-list limit
+    assert ws(5, 32, 131072, 64, 128, 8, 2048, 0) == 0
 
 
 FAKE = P(0x10000)        # never dereferenced: every call below fails validation first
@@ -144,6 +153,39 @@ def test_scoring_and_selection_argument_checks(lib):
     assert st == INVALID  # caches overlap
     assert lib.misa_pool_keys(FAKE, 0, 0, 1000, 128, 64, BF16, FAKE, 0, 0, 16, None) == OK
     assert lib.misa_pool_keys(FAKE, 0, 1, 1000, 128, 64, BF16, FAKE, 0, 16, 16, None) == OK  # empty range
+
+
+def block_filter(lib, **kw):
+    a = dict(q=FAKE, w=FAKE, k=FAKE, kss=0, kbar=FAKE, kbss=0, n=FAKE, heads=FAKE, T=4, L=1000, H_I=64, d=128,
+             B=64, h=8, m=4, topk=100, dt=BF16, S=None, ldS=0, blocks=FAKE, idx=FAKE, vals=None, ws=FAKE,
+             wsb=1 << 30, s=None)
+    a.update(kw)
+    return lib.misa_block_filter_topk(*(a[x] for x in ("q", "w", "k", "kss", "kbar", "kbss", "n", "heads", "T", "L",
+                                                       "H_I", "d", "B", "h", "m", "topk", "dt", "S", "ldS",
+                                                       "blocks", "idx", "vals", "ws", "wsb", "s")))
+
+
+def test_block_filter_argument_checks(lib):
+    assert block_filter(lib, d=64) == UNSUPPORTED
+    assert block_filter(lib, H_I=12) == UNSUPPORTED
+    assert block_filter(lib, m=0) == INVALID
+    assert block_filter(lib, topk=0) == INVALID
+    assert block_filter(lib, h=0) == INVALID
+    assert block_filter(lib, h=65) == INVALID
+    assert block_filter(lib, B=0) == INVALID
+    assert block_filter(lib, m=257) == UNSUPPORTED  # 257 * 64 tokens above the candidate-list limit
+    assert block_filter(lib, kbss=16 * 128 - 4) == INVALID  # pooled caches overlap
+    assert block_filter(lib, kbss=16 * 128 + 2) == INVALID  # rows not 16-byte aligned
+    assert block_filter(lib, S=FAKE, ldS=15) == INVALID  # block-score rows shorter than ceil(L/B)
+    assert block_filter(lib, kbar=None) == INVALID
+    assert block_filter(lib, kbar=MISALIGNED) == INVALID
+    assert block_filter(lib, heads=None) == INVALID
+    assert block_filter(lib, blocks=None) == INVALID
+    assert block_filter(lib, idx=None) == INVALID
+    assert block_filter(lib, ws=None) == WORKSPACE
+    assert block_filter(lib, wsb=1000) == WORKSPACE
+    assert block_filter(lib, ws=MISALIGNED) == WORKSPACE
+    assert block_filter(lib, T=0, q=None, w=None, k=None, n=None, kbar=None, heads=None) == OK
 
 
 def test_binding_rejects_host_tensors():
