@@ -13,6 +13,10 @@ than L2, so every step streams it from HBM).  Metric: scored query-tokens per se
 
 The reference arm (--impl reference) times the CPU oracle, as it stands, on the host cores, on a
 bounded sample of the same workload.
+
+--block-filter M (decode workloads) adds, outside the timed step, MISA with the token-axis block
+filter keeping M blocks per query on the same inputs (route + misa_block_filter_topk) as the
+line's "block_filter_same_inputs" object.
 """
 from __future__ import annotations
 
@@ -194,6 +198,71 @@ def cpu_baseline_sample(wl, seqs, threads=None):
               kp=wl.kp or 0)
     dt = time.perf_counter() - t0
     return dt, o.num_threads()
+
+
+def cpu_block_filter_sample(wl, seqs, m):
+    """Time the oracle's route + block filter + refinement on the given decode sequences."""
+    import oracle
+    o = oracle.get()
+    k, q, w, n, _ = W.decode_batch(wl, seqs)
+    L, d = k.shape[1], k.shape[2]
+    t0 = time.perf_counter()
+    o.block_filter(q, w, k, L * d, n, wl.B, wl.h, m, wl.topk)
+    return time.perf_counter() - t0, o.num_threads()
+
+
+def block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d):
+    """MISA with the token-axis block filter on the decode inputs of the main step, outside its
+    timed region: route + misa_block_filter_topk keeping m blocks, replayed as a CUDA graph, and
+    the block filter call alone.  Algorithmic bytes of the call per query: the M_t pooled keys
+    (fp32) and the routed q rows for the block scores, then m*B key rows (bf16), their ids and
+    scores for the refinement, and the kept-block and token outputs."""
+    m, B, h, kk = args.block_filter, wl.B, wl.h, wl.topk
+    T, L = kd.shape[0], kd.shape[1]
+    Mb = -(-L // B)
+    P = min(m, Mb) * B
+    heads = torch.empty((T, h), dtype=torch.int32, device=dev)
+    idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+    vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
+    blocks = torch.empty((T, m), dtype=torch.int32, device=dev)
+    wsp = M.Workspace(dev)
+
+    def route():
+        M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
+
+    def filt():
+        M.misa_block_filter_topk(qd, wd, kd, kbar, nd, heads, B, m, kk, idx=idx, vals=vals, blocks=blocks, ws=wsp)
+
+    def both():
+        route()
+        filt()
+
+    for _ in range(3):
+        both()
+    torch.cuda.synchronize()
+    nrep = max(1, min(args.steps, 50))
+    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    run = _graphed(torch, both, not args.no_graph)
+    for _ in range(3):
+        run()
+    e[0].record(stream)
+    for _ in range(nrep):
+        run()
+    e[1].record(stream)
+    torch.cuda.synchronize()
+    call_ms = 0.0
+    for _ in range(nrep):
+        route()
+        e[2].record(stream)
+        filt()
+        e[3].record(stream)
+        torch.cuda.synchronize()
+        call_ms += e[2].elapsed_time(e[3])
+    step_ms = e[0].elapsed_time(e[1]) / nrep
+    alg = T * (Mb * h_d * 4 + h * h_d * 2 + h * 4 + P * (h_d * 2 + 4 + 4 + 4) + m * 4 + kk * 8)
+    return {"m": m, "kept_tokens_per_query": P, "route_plus_filter_ms": step_ms,
+            "query_tokens_per_s": T * L / (step_ms / 1000.0), "call_ms": call_ms / nrep,
+            "algorithmic_bytes_per_call": alg, "launches_per_call": 5}
 
 
 def prefill_sample_inputs(wl, count):
@@ -634,6 +703,8 @@ def run_ours(args):
         torch.cuda.synchronize()
         dsa_ms = d0.elapsed_time(d1) / nrep
 
+    bf = block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d=d) if args.block_filter else None
+
     if rank == 0:
         hbm, kind = _peaks()
         score_avg = sum(score_ms) / len(score_ms)
@@ -659,6 +730,14 @@ def run_ours(args):
             "dense_dsa_same_inputs": None if dsa_ms is None else {
                 "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0)},
         }
+        if bf is not None:
+            bf["achieved_GBps"] = bf["algorithmic_bytes_per_call"] / (bf["call_ms"] / 1000.0) / 1e9
+            bf["frac_of_hbm"] = bf["achieved_GBps"] / hbm
+            if not args.no_cpu_baseline:
+                dt, thr = cpu_block_filter_sample(wl, [0], args.block_filter)
+                bf["cpu_oracle"] = {"query_tokens_per_s": L / dt, "cores": thr,
+                                    "sample": "1 sequence, route + block filter + refinement, double precision"}
+            line["block_filter_same_inputs"] = bf
         if not args.no_cpu_baseline:
             per = max(1, min(T, os.cpu_count() or 1))
             dt, thr = cpu_baseline_sample(wl, list(range(per)))
@@ -685,6 +764,9 @@ def main():
                          "partition/resolve kernels (instead of one CTA per row)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
+    ap.add_argument("--block-filter", type=int, default=0, metavar="M",
+                    help="decode: also time MISA with the token-axis block filter keeping M blocks per query "
+                         "(route + misa_block_filter_topk) on the same inputs, outside the timed step")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)

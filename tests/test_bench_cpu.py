@@ -21,7 +21,8 @@ def test_bench_module_defines_its_helpers():
     sys.path.insert(0, ROOT)
     import bench
     for name in ("ClockSampler", "_sha", "_peaks", "_tc_peaks", "_graphed", "run_ours", "run_prefill",
-                 "run_reference", "cpu_baseline_sample", "cpu_prefill_sample"):
+                 "run_reference", "cpu_baseline_sample", "cpu_prefill_sample", "block_filter_leg",
+                 "cpu_block_filter_sample"):
         assert hasattr(bench, name), name
     assert bench._sha(bench.TRAFFIC["file"])
 
@@ -35,3 +36,19 @@ def test_reference_arm_prints_a_json_line(workload):
         assert key in line, key
     assert line["value"] > 0 and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_block_filter_cpu_sample():
+    """The oracle leg of the block-filter measurement on a small decode workload."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from long_context_sparse_mean_b200 import workloads as W
+    wl = W.small(2, L=4096, n_seq=2, T=2)
+    dt, thr = bench.cpu_block_filter_sample(wl, [0], 4)
+    assert dt > 0 and thr >= 1
+
+
+def test_block_filter_flag_parses():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
+                         timeout=120, cwd=ROOT)
+    assert out.returncode == 0 and "--block-filter" in out.stdout
