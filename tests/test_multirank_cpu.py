@@ -41,7 +41,7 @@ def _rank_main(rank, world, port, out):
 def test_two_gloo_ranks_shard_and_time():
     world = 2
     port = _free_port()
-    mgr = tmp.Manager()
+    mgr = tmp.get_context("spawn").Manager()  # no fork of this (threaded) test process
     out = mgr.dict()
     tmp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
     for rank in range(world):
