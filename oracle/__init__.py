@@ -73,6 +73,8 @@ class Oracle:
         lib.orc_dense_scores_at.argtypes = [P, P, P, i64, P, i32, i32, i32, P, i64, P]
         lib.orc_route_batch.argtypes = [P, P, P, i64, P, i32, i32, i32, i32, i32, P, P]
         lib.orc_pool_batch.argtypes = [P, i64, i32, i64, i32, i32, P]
+        lib.orc_paged_gather.argtypes = [P, i64, i32, i32, P, i64, P, i32, i64, P]
+        lib.orc_paged_gather.restype = i64
         lib.orc_block_scores.argtypes = [P, P, P, i32, P, i64, i32, i32, P]
         lib.orc_block_filter.argtypes = [P, P, P, i32, P, i64, i32, i32, i64, i64, P, P, P, P]
         lib.orc_block_filter_batch.argtypes = [P, P, P, i64, P, i32, i32, i32, i32, i32, i64, i64, P, P,
@@ -177,6 +179,20 @@ class Oracle:
         heads = np.empty((T, h), np.int32)
         self.lib.orc_route_batch(_p(q), _p(w), _p(k), k_seq_stride, _p(n), T, H_I, d, B, h, _p(r), _p(heads))
         return r, heads
+
+    def paged_caches(self, pool, page_table, n, L):
+        """Logical caches [T, L, d] of sequences stored in pages: pool [num_pages, page_size, d],
+        page_table [T, max_pages] (physical page of each logical page), n [T].  Keys past each
+        prefix are zero.  Raises if a page id inside a prefix is out of range."""
+        pool, page_table, n = _f32(pool), _i32(page_table), _i32(n)
+        num_pages, page_size, d = pool.shape
+        T, max_pages = page_table.shape
+        out = np.empty((T, L, d), np.float32)
+        bad = self.lib.orc_paged_gather(_p(pool), num_pages, page_size, d, _p(page_table), max_pages, _p(n), T, L,
+                                        _p(out))
+        if bad:
+            raise ValueError(f"{bad} keys inside a prefix map to a page id outside the pool")
+        return out
 
     def block_scores(self, q, w, heads, k, n, B):
         """Block-filter scores of one query: S[ceil(n/B)] with the given heads."""

@@ -17,7 +17,9 @@
  *     dense indexer with all H_I heads re-scores only those and keeps the top-k.
  *   - "Problem Statement": the dense DSA indexer scores every prefix token with all H_I heads.
  *   - "HISA: Efficient Hierarchical Indexing for Fine-Grained Sparse Attention" (arXiv 2603.28458),
- *     abstract: the token-axis block filter composed with MISA (orc_block_* at the end of the file).
+ *     abstract: the token-axis block filter composed with MISA (orc_block_*).
+ *   - paged key caches (orc_paged_gather, at the end of the file): a storage layout for serving,
+ *     under which the definitions above apply to each sequence's logical cache.
  * The pages never write the score formulas; this oracle fixes them as
  *     token score  I_{t,s} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . k_s)
  *     router score r_{t,j} = w_{t,j} * sum_{b < M_t} max(0, q_{t,j} . kbar_b)
@@ -410,4 +412,34 @@ void orc_block_filter_batch(const float* q, const float* w, const float* k, int6
     free(S);
     free(bl);
   }
+}
+
+/*
+ * Paged key caches (a serving layout; the pages call MISA a drop-in replacement for the DSA
+ * indexer, "Key Contributions"): the keys of sequence t live in fixed-size pages of one shared
+ * pool[num_pages, page_size, d], and its logical key s is row s % page_size of physical page
+ * page_table[t][s / page_size].  The indexer's definitions apply unchanged to the logical cache.
+ * This gathers the logical cache of every sequence: out[T, L, d] receives keys s < min(n_t, L)
+ * and zeros past them; table entries of pages past the prefix are never read.  Returns the number
+ * of page ids that were out of range (their keys are left zero).
+ */
+int64_t orc_paged_gather(const float* pool, int64_t num_pages, int page_size, int d,
+                         const int32_t* page_table, int64_t max_pages, const int32_t* n, int T,
+                         int64_t L, float* out) {
+  int64_t bad = 0;
+  for (int t = 0; t < T; ++t) {
+    float* ot = out + (int64_t)t * L * d;
+    memset(ot, 0, sizeof(float) * (size_t)L * (size_t)d);
+    const int64_t nt = n[t] < 0 ? 0 : (n[t] > L ? L : n[t]);
+    for (int64_t s = 0; s < nt; ++s) {
+      const int64_t lp = s / page_size;
+      const int32_t pg = lp < max_pages ? page_table[(int64_t)t * max_pages + lp] : -1;
+      if (pg < 0 || pg >= num_pages) {
+        ++bad;
+        continue;
+      }
+      memcpy(ot + s * d, pool + ((int64_t)pg * page_size + s % page_size) * d, sizeof(float) * (size_t)d);
+    }
+  }
+  return bad;
 }

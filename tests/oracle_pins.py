@@ -19,7 +19,9 @@ LLM Inference", gist.science/paper/2605.07363, "Methodology: MISA" and "Hierarch
   * the block filter composed with MISA ("HISA: Efficient Hierarchical Indexing for Fine-Grained
     Sparse Attention", abstract): hand-derived cases, every block kept is MISA, B = 1 turns block
     scores into token scores, block scores sum to the routed heads' router scores, and the
-    selection is MISA's top-k restricted to the kept blocks.
+    selection is MISA's top-k restricted to the kept blocks;
+  * paged key caches: a shuffled pool built page by page with numpy, shared prefix pages and
+    unused table entries gather back to the contiguous caches, and every indexer agrees bit for bit.
 """
 from __future__ import annotations
 
@@ -467,6 +469,91 @@ def check_block_filter_invariants(o):
         assert np.array_equal(past[key], base[key], equal_nan=True), f"keys past the prefix changed {key}"
 
 
+def _paged(o, pool, table, n, L):
+    try:
+        return o.paged_caches(pool, table, n, L)
+    except ValueError as e:  # a mistake that reads an unused table entry shows up here
+        raise AssertionError(str(e))
+
+
+def check_paged_caches(o):
+    """Paged key caches: contiguous caches scattered page by page (numpy) into a shuffled pool with
+    spare pages, prefix pages shared between sequences and garbage table entries past each prefix,
+    gather back to the same logical caches, and every indexer (MISA, MISA-dagger, dense, block
+    filter) gives bit for bit what it gives on the contiguous caches."""
+    rng = np.random.default_rng(15)
+    T, L, d, ps, H_I = 4, 100, 16, 16, 8
+    lp = -(-L // ps)
+    caches = rng.integers(-3, 4, size=(T, L, d)).astype(np.float32)
+    caches[1, :3 * ps] = caches[0, :3 * ps]  # sequences 0 and 1 share a 48-key prefix
+    n = np.array([100, 97, 33, 0], np.int32)
+    caches_p = caches.copy()
+    for t in range(T):
+        caches_p[t, n[t]:] = 0.0
+    num_pages = T * lp + 5
+    perm = rng.permutation(num_pages)
+    pool = rng.integers(-9, 10, size=(num_pages, ps, d)).astype(np.float32)  # spare pages hold junk
+    table = np.full((T, lp + 2), -1, np.int32)
+    padded = np.zeros((T, lp * ps, d), np.float32)
+    padded[:, :L] = caches
+    for t in range(T):
+        for g in range(-(-int(n[t]) // ps)):
+            if t == 1 and g < 3:
+                table[t, g] = table[0, g]  # shared physical pages
+                continue
+            table[t, g] = perm[t * lp + g]
+            pool[table[t, g]] = padded[t, g * ps:(g + 1) * ps]
+        table[t, -(-int(n[t]) // ps):] = rng.integers(num_pages, 10 * num_pages)  # never read
+    got = _paged(o, pool, table, n, L)
+    assert np.array_equal(got, caches_p), "paged gather differs from the contiguous caches"
+    q = rng.integers(-3, 4, size=(T, H_I, d)).astype(np.float32)
+    w = rng.integers(-2, 3, size=(T, H_I)).astype(np.float32)
+    B, h, kk, kp = 7, 3, 9, 20
+    for mode, extra in ((0, {}), (1, {"kp": kp}), (2, {})):
+        a = o.indexer(mode, q, w, got, L * d, n, B, h, kk, **extra)
+        b = o.indexer(mode, q, w, caches, L * d, n, B, h, kk, **extra)
+        for key in a:
+            assert np.array_equal(a[key], b[key]), f"mode {mode}: {key} differs on the paged caches"
+    a = o.block_filter(q, w, got, L * d, n, B, h, 4, kk)
+    b = o.block_filter(q, w, caches, L * d, n, B, h, 4, kk)
+    for key in a:
+        assert np.array_equal(a[key], b[key], equal_nan=True), f"block filter: {key} differs on the paged caches"
+    bad = table.copy()
+    bad[2, 1] = num_pages + 3  # inside the prefix of sequence 2 (33 keys, 3 pages)
+    try:
+        o.paged_caches(pool, bad, n, L)
+    except ValueError:
+        pass
+    else:
+        raise AssertionError("an out-of-range page inside a prefix must be reported")
+
+
+def check_paged_hand_example(o):
+    """The hand example's five keys stored by hand in pages of two (a junk page, the partial last
+    page first, the logical pages in reverse order, junk in the unused row): the gathered cache is
+    the key list, and the indexer reproduces the hand-computed values of the golden fixture."""
+    g = _load_golden()
+    keys = np.array(g["keys"], np.float32)
+    pool = np.array([[[9, 9], [9, 9]],      # physical page 0: unused
+                     [[4, -2], [7, 7]],     # page 1: logical page 2 = {k4}, junk row
+                     [[0, 2], [-2, 4]],     # page 2: logical page 1 = {k2, k3}
+                     [[1, 0], [3, 2]]],     # page 3: logical page 0 = {k0, k1}
+                    np.float32)
+    table = np.array([[3, 2, 1], [3, 2, 0]], np.int32)
+    n = np.array([5, 4], np.int32)
+    got = _paged(o, pool, table, n, 5)
+    assert np.array_equal(got[0], keys), f"paged gather of the hand example: {got[0]}"
+    assert np.array_equal(got[1][:4], keys[:4]) and np.all(got[1][4] == 0), f"n = 4: {got[1]}"
+    q = np.array(g["q"], np.float32)
+    w = np.array(g["w"], np.float32)
+    Q, Wt = np.stack([q, q]), np.stack([w, w])
+    res = o.indexer(0, Q, Wt, got, 5 * 2, n, g["B"], 1, 2)
+    for t, qc in enumerate(g["queries"]):
+        assert np.array_equal(res["r"][t], np.array(qc["r"], np.float64)), f"paged router scores n={qc['n']}"
+        assert list(res["heads"][t]) == qc["h1"]["heads"], f"paged routed head n={qc['n']}"
+        assert sorted(res["idx"][t]) == sorted(qc["h1"]["top2"]), f"paged top-2 n={qc['n']}"
+
+
 ALL_CHECKS = [
     check_hand_example,
     check_topk_vs_stable_argsort,
@@ -487,4 +574,6 @@ ALL_CHECKS = [
     check_block_filter_hand_example,
     check_block_filter_reductions,
     check_block_filter_invariants,
+    check_paged_caches,
+    check_paged_hand_example,
 ]

@@ -49,6 +49,15 @@ MUTANTS = {
     "kept block's tokens taken from the block before": (
         "    const int64_t s0 = (int64_t)blocks[a] * B;",
         "    const int64_t s0 = (int64_t)(blocks[a] > 0 ? blocks[a] - 1 : 0) * B;"),
+    "paged gather ignores the page table": (
+        "      const int32_t pg = lp < max_pages ? page_table[(int64_t)t * max_pages + lp] : -1;",
+        "      const int32_t pg = (int32_t)((t * max_pages + lp) % num_pages);"),
+    "paged rows counted from the page's end": (
+        "(int64_t)pg * page_size + s % page_size",
+        "(int64_t)pg * page_size + (page_size - 1 - s % page_size)"),
+    "paged gather reads the page past the row's": (
+        "      const int64_t lp = s / page_size;",
+        "      const int64_t lp = s / page_size + 1;"),
     "dense re-rank with half the heads": ("      for (int j = 0; j < H_I; ++j)\n        acc += (double)w[j]",
                                           "      for (int j = 0; j < H_I / 2; ++j)\n        acc += (double)w[j]"),
 }
