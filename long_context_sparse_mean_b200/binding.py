@@ -109,6 +109,55 @@ def _cache_geometry(k: torch.Tensor, T: int):
     raise ValueError("k must be [L, d] or [T, L, d]")
 
 
+# Shape checks.  The C library sees only pointers and sizes, so a tensor smaller than the sizes
+# passed with it would be read or written past its end; these run before any device check.
+def _matrix(t, name: str, rows: int, cols: Optional[int] = None, min_cols: Optional[int] = None):
+    """t is 2-D with at least `rows` rows and exactly `cols` (or at least `min_cols`) columns."""
+    if t.dim() != 2 or t.shape[0] < rows or (cols is not None and t.shape[1] != cols) or \
+            (min_cols is not None and t.shape[1] < min_cols):
+        c = cols if cols is not None else (f">= {min_cols}" if min_cols is not None else "*")
+        raise ValueError(f"{name} must be [>= {rows}, {c}], got {tuple(t.shape)}")
+
+
+def _queries(q, w, n):
+    """(T, H_I, d) of a query batch q [T, H_I, d] with w [>= T, H_I] and n [>= T]."""
+    if q.dim() != 3:
+        raise ValueError(f"q must be [T, H_I, d], got {tuple(q.shape)}")
+    T, H_I, d = q.shape
+    _matrix(w, "w", T, H_I)
+    if n.dim() != 1 or n.shape[0] < T:
+        raise ValueError(f"n must be [>= {T}], got {tuple(n.shape)}")
+    return T, H_I, d
+
+
+def _cache(k, T: int, d: int):
+    """(L, k_seq_stride) of the key cache of a query batch whose vectors have d elements."""
+    L, dk, kss = _cache_geometry(k, T)
+    if dk != d:
+        raise ValueError(f"k rows have {dk} elements, q rows {d}")
+    return L, kss
+
+
+def _pooled(kbar, k, T: int, L: int, B: int):
+    """kbar matches the cache: [>= ceil(L/B), d] for a shared cache, [>= T, >= ceil(L/B), d] for
+    per-query caches.  Returns the pooled caches' stride in floats (0 when shared)."""
+    M = -(-L // B)
+    d = k.shape[-1]
+    if not (kbar.dim() == k.dim() and kbar.shape[-2] >= M and kbar.shape[-1] == d and
+            (kbar.dim() == 2 or kbar.shape[0] >= T)):
+        want = f"[{M}, {d}]" if k.dim() == 2 else f"[{T}, {M}, {d}]"
+        raise ValueError(f"kbar must be {want} for this cache and B = {B}, got {tuple(kbar.shape)}")
+    return 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
+
+
+def _outputs(T: int, topk: int, idx, vals):
+    """Caller-provided selection outputs hold [>= T, topk]."""
+    if idx is not None:
+        _matrix(idx, "idx", T, topk)
+    if vals is not None:
+        _matrix(vals, "vals", T, topk)
+
+
 def misa_device_check() -> None:
     """Waits for the device, then raises MisaError if a tensor-core kernel stopped early on a
     wait that ran out since the last check (its outputs are then incomplete)."""
@@ -150,11 +199,15 @@ def _ws(ws: Optional[Workspace], device) -> Workspace:
 def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, block_begin: int = 0,
                    block_end: Optional[int] = None, stream=None) -> torch.Tensor:
     """Block means of every cache: k [L,d] or [S,L,d] -> kbar [M,d] or [S,M,d] (fp32)."""
-    _need(k, "k")
+    if k.dim() not in (2, 3):
+        raise ValueError(f"k must be [L, d] or [S, L, d], got {tuple(k.shape)}")
     shared = k.dim() == 2
     S = 1 if shared else k.shape[0]
     L, d = k.shape[-2], k.shape[-1]
     M = -(-L // B)
+    if kbar is not None and tuple(kbar.shape) != ((M, d) if shared else (S, M, d)):
+        raise ValueError(f"kbar must be {[M, d] if shared else [S, M, d]}, got {tuple(kbar.shape)}")
+    _need(k, "k")
     if kbar is None:
         kbar = torch.empty((M, d) if shared else (S, M, d), dtype=torch.float32, device=k.device)
     _need(kbar, "kbar", torch.float32)
@@ -168,14 +221,18 @@ def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None,
 def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optional[Workspace] = None,
                want_r: bool = False, stream=None):
     """Routed heads [T, h] (descending router score) and, if asked, router scores r [T, H_I]."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    kbss = _pooled(kbar, k, T, L, B)
+    if heads is not None:
+        _matrix(heads, "heads", T, h)
+    if r is not None:
+        _matrix(r, "r", T, H_I)
     for t, nm in ((q, "q"), (k, "k")):
         _need(t, nm)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(kbar, "kbar", torch.float32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
-    kbss = 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
     if heads is None:
         heads = torch.empty((T, h), dtype=torch.int32, device=q.device)
     if r is None and want_r:
@@ -192,12 +249,16 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, se
     """Scores [T, L] fp32 (entries s >= n_t untouched); heads None = all heads (dense score).
     With select_topk > 0 and a Workspace, the first stage of a top-select_topk selection of the
     scores is left in that workspace for misa_topk_select(..., ws=<same>, ws_prepared=True)."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    if heads is not None:
+        _matrix(heads, "heads", T)
+    if out is not None:
+        _matrix(out, "out", T, min_cols=L)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
     h = 0
     if heads is not None:
         _need(heads, "heads", torch.int32)
@@ -220,9 +281,17 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, se
 def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, vals=None, want_vals=True,
                      ws: Optional[Workspace] = None, ws_prepared: bool = False, stream=None):
     """Top-k per row of scores [T, ld] over entries s < min(n_t, L) -> (idx [T, k], vals [T, k])."""
+    if scores.dim() != 2:
+        raise ValueError(f"scores must be [T, ld], got {tuple(scores.shape)}")
+    T, ld = scores.shape
+    if n.dim() != 1 or n.shape[0] < T:
+        raise ValueError(f"n must be [>= {T}], got {tuple(n.shape)}")
+    if idx is not None:
+        _matrix(idx, "idx", T, topk)
+    if vals is not None:
+        _matrix(vals, "vals", T, topk)
     _need(scores, "scores", torch.float32)
     _need(n, "n", torch.int32)
-    T, ld = scores.shape
     L = ld if L is None else L
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=scores.device)
@@ -238,13 +307,17 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
 def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_full=None, want_vals=True,
                     ws: Optional[Workspace] = None, stream=None):
     """Routed scoring + top-k -> (idx [T, k], vals [T, k]); the index order is not specified."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    _matrix(heads, "heads", T)
+    _outputs(T, topk, idx, vals)
+    if scores_full is not None:
+        _matrix(scores_full, "scores_full", T, L)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(heads, "heads", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
     h = heads.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -262,13 +335,15 @@ def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_fu
 def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals=True,
                      ws: Optional[Workspace] = None, stream=None):
     """MISA-dagger fine stage: dense re-score of cand [T, k'] -> (idx [T, k], vals [T, k])."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    _matrix(cand, "cand", T)
+    _outputs(T, topk, idx, vals)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(cand, "cand", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -285,12 +360,13 @@ def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals
 def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, ws: Optional[Workspace] = None,
                    stream=None):
     """Dense all-head indexer -> (idx [T, k], vals [T, k]); the index order is not specified."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    _outputs(T, topk, idx, vals)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
     if vals is None and want_vals:
@@ -309,17 +385,23 @@ def misa_block_filter_topk(q, w, k, kbar, n, heads, B: int, m: int, topk: int, i
     """Block filter + routed refinement: block scores with the routed heads, the m best blocks,
     then top-k over their tokens -> dict with idx [T, k], vals [T, k] (or None), blocks [T, m]
     (-1 padded; order not specified) and, if asked, block_scores [T, ceil(L/B)]."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    kbss = _pooled(kbar, k, T, L, B)
+    M = -(-L // B)
+    _matrix(heads, "heads", T)
+    _outputs(T, topk, idx, vals)
+    if blocks is not None:
+        _matrix(blocks, "blocks", T, m)
+    if block_scores is not None:
+        _matrix(block_scores, "block_scores", T, min_cols=M)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(kbar, "kbar", torch.float32)
     _need(heads, "heads", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
-    kbss = 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
     h = heads.shape[1]
-    M = -(-L // B)
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
     if vals is None and want_vals:
@@ -368,13 +450,15 @@ def misa_hier_rerank_static(q, w, k, n, cand, topk: int, idx=None, vals=None, wa
     """misa_hier_rerank for callers that cannot allocate device memory: the library's fixed
     scratch array replaces the workspace (T * k' <= STATIC_RERANK_SCRATCH_FLOATS).  Calls that
     overlap on the GPU share that array and must be ordered on one stream."""
+    T, H_I, d = _queries(q, w, n)
+    L, kss = _cache(k, T, d)
+    _matrix(cand, "cand", T)
+    _outputs(T, topk, idx, vals)
     _need(q, "q")
     _need(k, "k")
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(cand, "cand", torch.int32)
-    T, H_I, d = q.shape
-    L, _, kss = _cache_geometry(k, T)
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
