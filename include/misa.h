@@ -199,7 +199,8 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
  * misa_score_topk's selection; h = H_I gives the block filter on the dense indexer.
  *   kbar             : fp32 block means from misa_pool_keys, 16-byte aligned; query t reads
  *                      kbar + t*kbar_seq_stride (0 = shared; else a multiple of 4, >= M*d)
- *   heads            : [T, h] routed heads (entries outside [0, H_I) count as weight 0)
+ *   heads            : [T, h] routed heads in [0, H_I) (other ids are never dereferenced, but
+ *                      the results are then unspecified)
  *   m                : blocks kept per query, 1 <= m with m * B <= MISA_MAX_KP
  *   block_scores_opt : out [T, ld_block_scores] fp32 S_{t,b} for b < M_t (ld >= ceil(L/B)), or NULL
  *   blocks           : out [T, m] kept blocks, -1 padded (order unspecified)
