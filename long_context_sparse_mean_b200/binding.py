@@ -5,6 +5,10 @@ tensors' device pointers and the current CUDA stream through ctypes.  Every step
 runs in the library's CUDA kernels; there is no fallback.  If libmisa.so is missing the import
 of this module fails.
 
+Workspaces: a call given no Workspace uses one default buffer per device, shared by every such call
+on that device.  Calls in one stream are ordered, so that is safe there; calls on different streams
+that may overlap on the GPU must each pass their own Workspace.
+
 Tensor conventions (all on one CUDA device, contiguous):
   q [T, H_I, 128] bf16 or fp32, w [T, H_I] fp32, n [T] int32 (prefix lengths),
   k [L, 128] (one cache shared by all queries) or [T, L, 128] (cache t for query t), same dtype as q,
@@ -170,7 +174,8 @@ def misa_workspace_bytes(op: int, T: int, L: int, H_I: int, B: int = 1, h: int =
 
 
 class Workspace:
-    """A reusable, 256-byte aligned device scratch buffer (grown on demand)."""
+    """A reusable, 256-byte aligned device scratch buffer (grown on demand).  One Workspace serves
+    calls that are ordered on one stream; give each stream that may overlap another its own."""
 
     def __init__(self, device=None):
         self.device = device
