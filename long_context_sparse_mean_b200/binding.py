@@ -102,14 +102,28 @@ def _need(t: torch.Tensor, name: str, dtype=None):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
 
 
+def _need_opt(t: Optional[torch.Tensor], name: str, dtype=None):
+    if t is not None:
+        _need(t, name, dtype)
+
+
+def _on_device(*ts):
+    """Every given tensor is on the current CUDA device, where the library launches."""
+    cur = torch.cuda.current_device()
+    for t in ts:
+        if t is not None and t.get_device() != cur:
+            raise ValueError(f"every tensor must be on the current device cuda:{cur}; one is on {t.device}")
+
+
 def _cache_geometry(k: torch.Tensor, T: int):
     """(L, d, k_seq_stride) of a shared [L, d] or per-query [T, L, d] key cache."""
-    if k.dim() == 2:
-        return k.shape[0], k.shape[1], 0
-    if k.dim() == 3:
-        if k.shape[0] != T:
-            raise ValueError(f"per-query cache needs k.shape[0] == T ({T}), got {k.shape[0]}")
-        return k.shape[1], k.shape[2], k.shape[1] * k.shape[2]
+    s = k.shape
+    if len(s) == 2:
+        return s[0], s[1], 0
+    if len(s) == 3:
+        if s[0] != T:
+            raise ValueError(f"per-query cache needs k.shape[0] == T ({T}), got {s[0]}")
+        return s[1], s[2], s[1] * s[2]
     raise ValueError("k must be [L, d] or [T, L, d]")
 
 
@@ -117,20 +131,23 @@ def _cache_geometry(k: torch.Tensor, T: int):
 # passed with it would be read or written past its end; these run before any device check.
 def _matrix(t, name: str, rows: int, cols: Optional[int] = None, min_cols: Optional[int] = None):
     """t is 2-D with at least `rows` rows and exactly `cols` (or at least `min_cols`) columns."""
-    if t.dim() != 2 or t.shape[0] < rows or (cols is not None and t.shape[1] != cols) or \
-            (min_cols is not None and t.shape[1] < min_cols):
+    s = t.shape
+    if len(s) != 2 or s[0] < rows or (cols is not None and s[1] != cols) or \
+            (min_cols is not None and s[1] < min_cols):
         c = cols if cols is not None else (f">= {min_cols}" if min_cols is not None else "*")
         raise ValueError(f"{name} must be [>= {rows}, {c}], got {tuple(t.shape)}")
 
 
 def _queries(q, w, n):
     """(T, H_I, d) of a query batch q [T, H_I, d] with w [>= T, H_I] and n [>= T]."""
-    if q.dim() != 3:
-        raise ValueError(f"q must be [T, H_I, d], got {tuple(q.shape)}")
-    T, H_I, d = q.shape
+    s = q.shape
+    if len(s) != 3:
+        raise ValueError(f"q must be [T, H_I, d], got {tuple(s)}")
+    T, H_I, d = s
     _matrix(w, "w", T, H_I)
-    if n.dim() != 1 or n.shape[0] < T:
-        raise ValueError(f"n must be [>= {T}], got {tuple(n.shape)}")
+    ns = n.shape
+    if len(ns) != 1 or ns[0] < T:
+        raise ValueError(f"n must be [>= {T}], got {tuple(ns)}")
     return T, H_I, d
 
 
@@ -146,12 +163,12 @@ def _pooled(kbar, k, T: int, L: int, B: int):
     """kbar matches the cache: [>= ceil(L/B), d] for a shared cache, [>= T, >= ceil(L/B), d] for
     per-query caches.  Returns the pooled caches' stride in floats (0 when shared)."""
     M = -(-L // B)
-    d = k.shape[-1]
-    if not (kbar.dim() == k.dim() and kbar.shape[-2] >= M and kbar.shape[-1] == d and
-            (kbar.dim() == 2 or kbar.shape[0] >= T)):
-        want = f"[{M}, {d}]" if k.dim() == 2 else f"[{T}, {M}, {d}]"
-        raise ValueError(f"kbar must be {want} for this cache and B = {B}, got {tuple(kbar.shape)}")
-    return 0 if kbar.dim() == 2 else kbar.shape[1] * kbar.shape[2]
+    ks, bs = k.shape, kbar.shape
+    d = ks[-1]
+    if not (len(bs) == len(ks) and bs[-2] >= M and bs[-1] == d and (len(bs) == 2 or bs[0] >= T)):
+        want = f"[{M}, {d}]" if len(ks) == 2 else f"[{T}, {M}, {d}]"
+        raise ValueError(f"kbar must be {want} for this cache and B = {B}, got {tuple(bs)}")
+    return 0 if len(bs) == 2 else bs[1] * bs[2]
 
 
 def _outputs(T: int, topk: int, idx, vals):
@@ -216,6 +233,7 @@ def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None,
     if kbar is None:
         kbar = torch.empty((M, d) if shared else (S, M, d), dtype=torch.float32, device=k.device)
     _need(kbar, "kbar", torch.float32)
+    _on_device(k, kbar)
     block_end = M if block_end is None else block_end
     _check("misa_pool_keys", _lib.misa_pool_keys(
         _p(k), 0 if shared else L * d, S, L, d, B, _dtype_code(k), _p(kbar), 0 if shared else M * d,
@@ -233,11 +251,14 @@ def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optiona
         _matrix(heads, "heads", T, h)
     if r is not None:
         _matrix(r, "r", T, H_I)
-    for t, nm in ((q, "q"), (k, "k")):
-        _need(t, nm)
+    _need(q, "q")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(kbar, "kbar", torch.float32)
+    _need_opt(heads, "heads", torch.int32)
+    _need_opt(r, "r", torch.float32)
+    _on_device(q, k, w, n, kbar, heads, r)
     if heads is None:
         heads = torch.empty((T, h), dtype=torch.int32, device=q.device)
     if r is None and want_r:
@@ -261,13 +282,15 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, se
     if out is not None:
         _matrix(out, "out", T, min_cols=L)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
+    _need_opt(out, "out", torch.float32)
     h = 0
     if heads is not None:
         _need(heads, "heads", torch.int32)
         h = heads.shape[1]
+    _on_device(q, k, w, n, heads, out)
     if out is None:
         out = torch.empty((T, L), dtype=torch.float32, device=q.device)
     _need(out, "out", torch.float32)
@@ -297,6 +320,9 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
         _matrix(vals, "vals", T, topk)
     _need(scores, "scores", torch.float32)
     _need(n, "n", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(scores, n, idx, vals)
     L = ld if L is None else L
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=scores.device)
@@ -319,10 +345,14 @@ def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_fu
     if scores_full is not None:
         _matrix(scores_full, "scores_full", T, L)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(heads, "heads", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _need_opt(scores_full, "scores_full", torch.float32)
+    _on_device(q, k, w, n, heads, idx, vals, scores_full)
     h = heads.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -345,10 +375,13 @@ def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals
     _matrix(cand, "cand", T)
     _outputs(T, topk, idx, vals)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(cand, "cand", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, k, w, n, cand, idx, vals)
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -369,9 +402,12 @@ def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, w
     L, kss = _cache(k, T, d)
     _outputs(T, topk, idx, vals)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, k, w, n, idx, vals)
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
     if vals is None and want_vals:
@@ -401,11 +437,16 @@ def misa_block_filter_topk(q, w, k, kbar, n, heads, B: int, m: int, topk: int, i
     if block_scores is not None:
         _matrix(block_scores, "block_scores", T, min_cols=M)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(kbar, "kbar", torch.float32)
     _need(heads, "heads", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _need_opt(blocks, "blocks", torch.int32)
+    _need_opt(block_scores, "block_scores", torch.float32)
+    _on_device(q, k, w, n, kbar, heads, idx, vals, blocks, block_scores)
     h = heads.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -460,10 +501,13 @@ def misa_hier_rerank_static(q, w, k, n, cand, topk: int, idx=None, vals=None, wa
     _matrix(cand, "cand", T)
     _outputs(T, topk, idx, vals)
     _need(q, "q")
-    _need(k, "k")
+    _need(k, "k", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(cand, "cand", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, k, w, n, cand, idx, vals)
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)

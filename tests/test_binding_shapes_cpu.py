@@ -78,3 +78,21 @@ def test_wrong_shapes_are_rejected_first():
     _shape_error(lambda: M.misa_block_filter_topk(q, w, k, kbar, n, heads, B, 4, 10,
                                                   block_scores=_t(T, MB - 1)), "block_scores must be")
     _shape_error(lambda: M.misa_block_filter_topk(q, w, k, kbar, n, heads, 4, 4, 10), "kbar must be")  # B mismatch
+
+
+def test_device_check_rejects_a_tensor_on_another_gpu(monkeypatch):
+    """The library launches on the current device, so a tensor on another GPU is refused before
+    its pointer reaches a kernel."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+
+    class OnGpu:
+        def __init__(self, index):
+            self.index = index
+            self.device = f"cuda:{index}"
+
+        def get_device(self):
+            return self.index
+
+    M._on_device(OnGpu(0), None, OnGpu(0))
+    with pytest.raises(ValueError, match="current device cuda:0"):
+        M._on_device(OnGpu(0), OnGpu(1))
