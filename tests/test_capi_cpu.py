@@ -202,3 +202,35 @@ def test_device_check_reports_without_a_device(lib):
     want = OK if torch.cuda.is_available() else CUDA
     assert lib.misa_device_check() == want
     assert lib.misa_status_str(DEVICE_TIMEOUT) != b"unknown status"
+
+
+def test_a_c_program_compiles_links_and_calls_the_library(tmp_path):
+    """include/misa.h is plain C (C99, no C++ names): a C program includes it, links libmisa.so and
+    calls entry points that need no GPU (version, status text, workspace sizes, argument checks)."""
+    import subprocess
+    lib_path = build.build()
+    src = tmp_path / "use_misa.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include "misa.h"
+int main(void) {
+  if (misa_version() < 100) return 1;
+  if (misa_workspace_bytes(MISA_OP_SCORE_TOPK, 0, 100, 64, 1, 8, 10, 0) != 0) return 2;
+  if (misa_workspace_bytes(MISA_OP_RERANK, 4, 0, 64, 0, 0, 10, 100) == 0) return 3;
+  /* d = 64 is refused on the host, before any launch */
+  misa_status st = misa_route((const void*)0x10000, (const float*)0x10000, (const void*)0x10000, 0,
+                              (const float*)0x10000, 0, (const int32_t*)0x10000, 4, 1000, 64, 64, 64, 8,
+                              MISA_BF16, (int32_t*)0x10000, NULL, (void*)0x10000, 1u << 30, NULL);
+  if (st != MISA_ERR_UNSUPPORTED) return 4;
+  printf("%s\n", misa_status_str(st));
+  return 0;
+}
+""")
+    exe = tmp_path / "use_misa"
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(lib_path)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", inc, str(src), "-L", libdir, "-lmisa",
+                    f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert out.returncode == 0, (out.returncode, out.stderr)
+    assert out.stdout.strip() == "unsupported configuration"
