@@ -556,6 +556,7 @@ def misa_pool_keys_paged(pool, page_table, B: int, L: Optional[int] = None, kbar
     if kbar is None:
         kbar = torch.empty((S, M, d), dtype=torch.float32, device=pool.device)
     _need(kbar, "kbar", torch.float32)
+    _on_device(pool, page_table, kbar)
     block_end = M if block_end is None else block_end
     _check("misa_pool_keys_paged", _lib.misa_pool_keys_paged(
         _p(pool), num_pages, page_size, _p(page_table), max_pages, S, L, d, B, _dtype_code(pool), _p(kbar), M * d,
@@ -576,11 +577,14 @@ def misa_route_paged(q, w, pool, page_table, kbar, n, B: int, h: int, L: Optiona
     if r is not None:
         _matrix(r, "r", T, H_I)
     _need(q, "q")
-    _need(pool, "pool")
+    _need(pool, "pool", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(kbar, "kbar", torch.float32)
     _need(page_table, "page_table", torch.int32)
+    _need_opt(heads, "heads", torch.int32)
+    _need_opt(r, "r", torch.float32)
+    _on_device(q, pool, w, n, kbar, page_table, heads, r)
     if heads is None:
         heads = torch.empty((T, h), dtype=torch.int32, device=q.device)
     if r is None and want_r:
@@ -602,11 +606,14 @@ def misa_score_topk_paged(q, w, pool, page_table, n, heads, topk: int, L: Option
     _matrix(heads, "heads", T)
     _outputs(T, topk, idx, vals)
     _need(q, "q")
-    _need(pool, "pool")
+    _need(pool, "pool", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(heads, "heads", torch.int32)
     _need(page_table, "page_table", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, pool, w, n, heads, page_table, idx, vals)
     h = heads.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
@@ -628,11 +635,14 @@ def misa_hier_rerank_paged(q, w, pool, page_table, n, cand, topk: int, L: Option
     _matrix(cand, "cand", T)
     _outputs(T, topk, idx, vals)
     _need(q, "q")
-    _need(pool, "pool")
+    _need(pool, "pool", q.dtype)
     _need(w, "w", torch.float32)
     _need(n, "n", torch.int32)
     _need(cand, "cand", torch.int32)
     _need(page_table, "page_table", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, pool, w, n, cand, page_table, idx, vals)
     kp = cand.shape[1]
     if idx is None:
         idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
