@@ -72,7 +72,10 @@ typedef enum {
   MISA_OP_RERANK = 2,
   MISA_OP_DENSE_TOPK = 3,
   MISA_OP_TOPK_SELECT = 4,
-  MISA_OP_BLOCK_FILTER = 5
+  MISA_OP_BLOCK_FILTER = 5,
+  MISA_OP_ROUTE_PAGED = 6,
+  MISA_OP_SCORE_TOPK_PAGED = 7,
+  MISA_OP_RERANK_PAGED = 8
 } misa_op;
 
 /* Largest k' accepted by misa_hier_rerank (its candidates are ranked in shared memory). */
@@ -215,6 +218,51 @@ misa_status misa_block_filter_topk(const void* q, const float* w, const void* k,
                                    const int32_t* heads, int T, int L, int H_I, int d, int B, int h,
                                    int m, int topk, int dtype, float* block_scores_opt,
                                    int64_t ld_block_scores, int32_t* blocks, int32_t* idx,
+                                   float* score_opt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Paged key caches.  Serving stores each sequence's keys in fixed-size pages of one pool shared by
+ * all sequences (the pages call MISA a drop-in replacement for the DSA indexer, "Key
+ * Contributions"; this is the layout such a replacement reads).  The *_paged calls compute exactly
+ * what their contiguous counterparts compute on each sequence's logical cache:
+ *   pool       : [num_pages, page_size, d] keys (dtype); num_pages * page_size < 2^31
+ *   page_table : [T, max_pages] int32; logical key s of query t's sequence is row s % page_size of
+ *                physical page page_table[t][s / page_size].  Entries for pages past a prefix are
+ *                never read.  max_pages * page_size >= L (L: the longest prefix, as elsewhere).
+ *   n          : [T] prefix lengths, as elsewhere.
+ * A page id outside [0, num_pages) inside a prefix is never dereferenced: its keys read as zero
+ * (pooling, router) or the token is left out of scoring; results are then unspecified.
+ * kbar is one pooled cache per query ([T, ceil(L/B), d] at kbar_seq_stride >= ceil(L/B) * d), as
+ * written by misa_pool_keys_paged.  Queries that share a sequence repeat its table row.
+ */
+/* misa_pool_keys through page tables (page_table rows are the n_seq sequences). */
+misa_status misa_pool_keys_paged(const void* pool, int64_t num_pages, int page_size,
+                                 const int32_t* page_table, int64_t max_pages, int n_seq, int L,
+                                 int d, int B, int dtype, float* kbar, int64_t kbar_seq_stride,
+                                 int block_begin, int block_end, void* stream);
+
+/* misa_route on paged caches.
+ *   ws : misa_workspace_bytes(MISA_OP_ROUTE_PAGED, T, L, H_I, B, h, 0, 0) bytes */
+misa_status misa_route_paged(const void* q, const float* w, const void* pool, int64_t num_pages,
+                             int page_size, const int32_t* page_table, int64_t max_pages,
+                             const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T,
+                             int L, int H_I, int d, int B, int h, int dtype, int32_t* heads,
+                             float* r_opt, void* ws, size_t ws_bytes, void* stream);
+
+/* misa_score_topk on paged caches (with topk = k', the MISA-dagger coarse stage).
+ *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK_PAGED, T, L, H_I, 0, h, topk, 0) bytes */
+misa_status misa_score_topk_paged(const void* q, const float* w, const void* pool, int64_t num_pages,
+                                  int page_size, const int32_t* page_table, int64_t max_pages,
+                                  const int32_t* n, const int32_t* heads, int T, int L, int H_I,
+                                  int d, int h, int topk, int dtype, int32_t* idx, float* score_opt,
+                                  void* ws, size_t ws_bytes, void* stream);
+
+/* misa_hier_rerank on paged caches.
+ *   ws : misa_workspace_bytes(MISA_OP_RERANK_PAGED, T, 0, H_I, 0, 0, topk, kp) bytes */
+misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* pool, int64_t num_pages,
+                                   int page_size, const int32_t* page_table, int64_t max_pages,
+                                   const int32_t* n, const int32_t* cand, int T, int L, int H_I,
+                                   int d, int kp, int topk, int dtype, int32_t* idx,
                                    float* score_opt, void* ws, size_t ws_bytes, void* stream);
 
 /*

@@ -27,7 +27,8 @@ LIB_PATH = os.path.join(PKG, "libmisa.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
 BF16, F32 = 0, 1
-OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT, OP_BLOCK_FILTER = range(6)
+(OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT, OP_BLOCK_FILTER, OP_ROUTE_PAGED,
+ OP_SCORE_TOPK_PAGED, OP_RERANK_PAGED) = range(9)
 MAX_KP = 16384
 
 if not os.path.exists(LIB_PATH):
@@ -56,6 +57,13 @@ def _setup(lib):
         "dsa_dense_topk": ([P, P, P, i64, P, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
         "misa_block_filter_topk": ([P, P, P, i64, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, i32, i32, P,
                                     i64, P, P, P, P, sz, P], i32),
+        "misa_pool_keys_paged": ([P, i64, i32, P, i64, i32, i32, i32, i32, i32, P, i64, i32, i32, P], i32),
+        "misa_route_paged": ([P, P, P, i64, i32, P, i64, P, i64, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz,
+                              P], i32),
+        "misa_score_topk_paged": ([P, P, P, i64, i32, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz,
+                                   P], i32),
+        "misa_hier_rerank_paged": ([P, P, P, i64, i32, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz,
+                                    P], i32),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -517,3 +525,145 @@ def misa_hier_rerank_static(q, w, k, n, cand, topk: int, idx=None, vals=None, wa
         _p(q), _p(w), _p(k), kss, _p(n), _p(cand), T, L, H_I, d, kp, topk, _dtype_code(q), _p(idx), _p(vals),
         _stream(stream)))
     return idx, vals
+
+
+# ---- paged key caches: pool [num_pages, page_size, d], page_table [T, max_pages] int32 ----------
+
+def _paged_geometry(pool, page_table, T: int, d: int, L: Optional[int]):
+    """(num_pages, page_size, max_pages, L) of a paged cache; L defaults to what the table covers."""
+    if pool.dim() != 3 or pool.shape[2] != d:
+        raise ValueError(f"pool must be [num_pages, page_size, {d}], got {tuple(pool.shape)}")
+    _matrix(page_table, "page_table", T)
+    num_pages, page_size = pool.shape[0], pool.shape[1]
+    max_pages = page_table.shape[1]
+    L = max_pages * page_size if L is None else L
+    if L > max_pages * page_size:
+        raise ValueError(f"a table of {max_pages} pages of {page_size} keys cannot hold L = {L}")
+    return num_pages, page_size, max_pages, L
+
+
+def misa_pool_keys_paged(pool, page_table, B: int, L: Optional[int] = None, kbar=None, block_begin: int = 0,
+                         block_end: Optional[int] = None, stream=None):
+    """Block means of every sequence's logical cache through its page table -> kbar [S, M, d]."""
+    S = page_table.shape[0]
+    num_pages, page_size, max_pages, L = _paged_geometry(pool, page_table, S, pool.shape[-1], L)
+    d = pool.shape[2]
+    M = -(-L // B)
+    if kbar is not None and tuple(kbar.shape) != (S, M, d):
+        raise ValueError(f"kbar must be {[S, M, d]}, got {tuple(kbar.shape)}")
+    _need(pool, "pool")
+    _need(page_table, "page_table", torch.int32)
+    if kbar is None:
+        kbar = torch.empty((S, M, d), dtype=torch.float32, device=pool.device)
+    _need(kbar, "kbar", torch.float32)
+    _on_device(pool, page_table, kbar)
+    block_end = M if block_end is None else block_end
+    _check("misa_pool_keys_paged", _lib.misa_pool_keys_paged(
+        _p(pool), num_pages, page_size, _p(page_table), max_pages, S, L, d, B, _dtype_code(pool), _p(kbar), M * d,
+        block_begin, block_end, _stream(stream)))
+    return kbar
+
+
+def misa_route_paged(q, w, pool, page_table, kbar, n, B: int, h: int, L: Optional[int] = None, heads=None, r=None,
+                     ws: Optional[Workspace] = None, want_r: bool = False, stream=None):
+    """misa_route on paged caches -> (heads [T, h], r [T, H_I] or None)."""
+    T, H_I, d = _queries(q, w, n)
+    num_pages, page_size, max_pages, L = _paged_geometry(pool, page_table, T, d, L)
+    M = -(-L // B)
+    if kbar.dim() != 3 or kbar.shape[0] < T or kbar.shape[1] < M or kbar.shape[2] != d:
+        raise ValueError(f"kbar must be [{T}, {M}, {d}], got {tuple(kbar.shape)}")
+    if heads is not None:
+        _matrix(heads, "heads", T, h)
+    if r is not None:
+        _matrix(r, "r", T, H_I)
+    _need(q, "q")
+    _need(pool, "pool", q.dtype)
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(kbar, "kbar", torch.float32)
+    _need(page_table, "page_table", torch.int32)
+    _need_opt(heads, "heads", torch.int32)
+    _need_opt(r, "r", torch.float32)
+    _on_device(q, pool, w, n, kbar, page_table, heads, r)
+    if heads is None:
+        heads = torch.empty((T, h), dtype=torch.int32, device=q.device)
+    if r is None and want_r:
+        r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_ROUTE_PAGED, T, L, H_I, B, h)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_route_paged", _lib.misa_route_paged(
+        _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(kbar),
+        kbar.shape[1] * kbar.shape[2], _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r), _p(buf), nbytes,
+        _stream(stream)))
+    return heads, r
+
+
+def misa_score_topk_paged(q, w, pool, page_table, n, heads, topk: int, L: Optional[int] = None, idx=None, vals=None,
+                          want_vals=True, ws: Optional[Workspace] = None, stream=None):
+    """misa_score_topk on paged caches -> (idx [T, k], vals [T, k]); logical token indices."""
+    T, H_I, d = _queries(q, w, n)
+    num_pages, page_size, max_pages, L = _paged_geometry(pool, page_table, T, d, L)
+    _matrix(heads, "heads", T)
+    _outputs(T, topk, idx, vals)
+    _need(q, "q")
+    _need(pool, "pool", q.dtype)
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(heads, "heads", torch.int32)
+    _need(page_table, "page_table", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, pool, w, n, heads, page_table, idx, vals)
+    h = heads.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_SCORE_TOPK_PAGED, T, L, H_I, 0, h, topk)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_score_topk_paged", _lib.misa_score_topk_paged(
+        _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(heads), T, L, H_I, d, h,
+        topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
+    return idx, vals
+
+
+def misa_hier_rerank_paged(q, w, pool, page_table, n, cand, topk: int, L: Optional[int] = None, idx=None,
+                           vals=None, want_vals=True, ws: Optional[Workspace] = None, stream=None):
+    """misa_hier_rerank on paged caches: dense re-score of logical candidates cand [T, k']."""
+    T, H_I, d = _queries(q, w, n)
+    num_pages, page_size, max_pages, L = _paged_geometry(pool, page_table, T, d, L)
+    _matrix(cand, "cand", T)
+    _outputs(T, topk, idx, vals)
+    _need(q, "q")
+    _need(pool, "pool", q.dtype)
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(cand, "cand", torch.int32)
+    _need(page_table, "page_table", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, pool, w, n, cand, page_table, idx, vals)
+    kp = cand.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_RERANK_PAGED, T, L, H_I, 0, 0, topk, kp)
+    buf = _ws(ws, q.device).get(nbytes)
+    _check("misa_hier_rerank_paged", _lib.misa_hier_rerank_paged(
+        _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(cand), T, L, H_I, d, kp,
+        topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
+    return idx, vals
+
+
+def misa_indexer_paged(q, w, pool, page_table, kbar, n, B: int, h: int, topk: int, kp: Optional[int] = None,
+                       L: Optional[int] = None, ws: Optional[Workspace] = None, stream=None):
+    """misa_indexer on paged caches (MISA, or MISA-dagger with kp given)."""
+    heads, _ = misa_route_paged(q, w, pool, page_table, kbar, n, B, h, L=L, ws=ws, stream=stream)
+    if kp is None:
+        idx, vals = misa_score_topk_paged(q, w, pool, page_table, n, heads, topk, L=L, ws=ws, stream=stream)
+        return {"idx": idx, "vals": vals, "heads": heads}
+    cand, _ = misa_score_topk_paged(q, w, pool, page_table, n, heads, kp, L=L, want_vals=False, ws=ws,
+                                    stream=stream)
+    idx, vals = misa_hier_rerank_paged(q, w, pool, page_table, n, cand, topk, L=L, ws=ws, stream=stream)
+    return {"idx": idx, "vals": vals, "heads": heads, "cand": cand}

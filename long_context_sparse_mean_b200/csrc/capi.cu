@@ -81,6 +81,35 @@ size_t block_filter_ws(int T, int L, int B, int m) {
          2 * align_up(sizeof(float) * (size_t)T * P) + select_bytes(T, (int)std::max<int64_t>(M, P));
 }
 
+// Paged caches: [physical rows of the positions scored][n_phys] in front of each op's own layout.
+size_t paged_rows_part(int T, int P) {
+  return align_up(sizeof(int32_t) * (size_t)T * P) + align_up(sizeof(int32_t) * (size_t)T);
+}
+
+size_t route_paged_ws(int T, int L, int H_I, int B) {
+  if (T <= 0 || L <= 0 || H_I <= 0 || B <= 0) return 0;
+  return route_ws(T, L, H_I, B) + align_up(sizeof(float) * (size_t)T * misa::kD);
+}
+
+size_t score_topk_paged_ws(int T, int L) {
+  if (T <= 0 || L <= 0) return 0;
+  return paged_rows_part(T, L) + scores_ws(T, L);
+}
+
+size_t rerank_paged_ws(int T, int kp) {
+  if (T <= 0 || kp <= 0) return 0;
+  return paged_rows_part(T, kp) + rerank_ws(T, kp);
+}
+
+misa_status check_paged(const void* pool, int64_t num_pages, int page_size, const int32_t* page_table,
+                        int64_t max_pages, int L, int T) {
+  if (num_pages < 1 || page_size < 1 || max_pages < 1) return MISA_ERR_INVALID_ARG;
+  if ((int64_t)L > max_pages * page_size) return MISA_ERR_INVALID_ARG;  // the table cannot cover L keys
+  if (num_pages * (int64_t)page_size > INT32_MAX) return MISA_ERR_UNSUPPORTED;
+  if (T > 0 && (!pool || !page_table)) return MISA_ERR_INVALID_ARG;
+  return MISA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -129,6 +158,12 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
       return select_bytes(T, L);
     case MISA_OP_BLOCK_FILTER:
       return block_filter_ws(T, L, B, kp);
+    case MISA_OP_ROUTE_PAGED:
+      return route_paged_ws(T, L, H_I, B);
+    case MISA_OP_SCORE_TOPK_PAGED:
+      return score_topk_paged_ws(T, L);
+    case MISA_OP_RERANK_PAGED:
+      return rerank_paged_ws(T, kp);
     default:
       return 0;
   }
@@ -169,7 +204,7 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
   p += align_up(sizeof(uint32_t) * (size_t)T);
   __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(p);
   misa::launch_route(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, T, L, H_I, B, h, heads,
-                     r_opt, pm, partial, done, parts, as_stream(stream));
+                     r_opt, pm, partial, done, parts, nullptr, as_stream(stream));
   return launch_status();
 }
 
@@ -314,6 +349,116 @@ misa_status misa_block_filter_topk(const void* q, const float* w, const void* k,
   misa::launch_expand_blocks(blocks, m, n, T, L, B, rows, s);
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, P, F, P, nullptr, s);
   misa::launch_topk_rows(F, P, rows, P, n, T, L, topk, p, false, idx, score_opt, s);
+  return launch_status();
+}
+
+misa_status misa_pool_keys_paged(const void* pool, int64_t num_pages, int page_size, const int32_t* page_table,
+                                 int64_t max_pages, int n_seq, int L, int d, int B, int dtype, float* kbar,
+                                 int64_t kbar_seq_stride, int block_begin, int block_end, void* stream) {
+  if (n_seq < 0 || L < 1 || B < 1 || kbar_seq_stride < 0) return MISA_ERR_INVALID_ARG;
+  if (dtype != MISA_BF16 && dtype != MISA_F32) return MISA_ERR_UNSUPPORTED;
+  if (d != misa::kD) return MISA_ERR_UNSUPPORTED;
+  misa_status st = check_paged(pool, num_pages, page_size, page_table, max_pages, L, n_seq);
+  if (st != MISA_OK) return st;
+  const int M = (int)ceil_div(L, B);
+  if (n_seq > 1 && kbar_seq_stride < (int64_t)M * d) return MISA_ERR_INVALID_ARG;
+  const int b0 = block_begin < 0 ? 0 : block_begin;
+  const int b1 = block_end > M ? M : block_end;
+  if (n_seq == 0 || b1 <= b0) return MISA_OK;
+  if (!kbar) return MISA_ERR_INVALID_ARG;
+  misa::launch_pool_paged(to_dtype(dtype), pool, num_pages, page_size, page_table, max_pages, n_seq, L, B, kbar,
+                          kbar_seq_stride, b0, b1, as_stream(stream));
+  return launch_status();
+}
+
+misa_status misa_route_paged(const void* q, const float* w, const void* pool, int64_t num_pages, int page_size,
+                             const int32_t* page_table, int64_t max_pages, const float* kbar, int64_t kbar_seq_stride,
+                             const int32_t* n, int T, int L, int H_I, int d, int B, int h, int dtype, int32_t* heads,
+                             float* r_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, pool, n, T, L, H_I, d, dtype, 0);
+  if (st != MISA_OK) return st;
+  st = check_paged(pool, num_pages, page_size, page_table, max_pages, L, T);
+  if (st != MISA_OK) return st;
+  if (B < 1 || h < 1 || h > H_I) return MISA_ERR_INVALID_ARG;
+  const int M = (int)ceil_div(L, B);
+  if (T > 1 && kbar_seq_stride < (int64_t)M * d) return MISA_ERR_INVALID_ARG;  // one pooled cache per query
+  if (T == 0) return MISA_OK;
+  if (!kbar || !heads) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < route_paged_ws(T, L, H_I, B) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  char* p = static_cast<char*>(ws);
+  float* pm = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * misa::kD);
+  float* partial = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * misa::route_chunks(L, B) * H_I);
+  uint32_t* done = reinterpret_cast<uint32_t*>(p);
+  p += align_up(sizeof(uint32_t) * (size_t)T);
+  __nv_bfloat16* parts = reinterpret_cast<__nv_bfloat16*>(p);
+  p += align_up(sizeof(uint16_t) * 3 * (size_t)M * misa::kD);
+  float* pm_in = reinterpret_cast<float*>(p);
+  const cudaStream_t s = as_stream(stream);
+  misa::launch_partial_mean_paged(to_dtype(dtype), pool, num_pages, page_size, page_table, max_pages, n, T, L, B,
+                                  pm_in, s);
+  misa::launch_route(to_dtype(dtype), q, w, pool, 0, kbar, kbar_seq_stride, n, T, L, H_I, B, h, heads, r_opt, pm,
+                     partial, done, parts, pm_in, s);
+  return launch_status();
+}
+
+misa_status misa_score_topk_paged(const void* q, const float* w, const void* pool, int64_t num_pages, int page_size,
+                                  const int32_t* page_table, int64_t max_pages, const int32_t* n,
+                                  const int32_t* heads, int T, int L, int H_I, int d, int h, int topk, int dtype,
+                                  int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, pool, n, T, L, H_I, d, dtype, 0);
+  if (st != MISA_OK) return st;
+  st = check_paged(pool, num_pages, page_size, page_table, max_pages, L, T);
+  if (st != MISA_OK) return st;
+  if (!heads && T > 0) return MISA_ERR_INVALID_ARG;
+  if (h < 1 || h > H_I || topk < 1) return MISA_ERR_INVALID_ARG;
+  if (T == 0) return MISA_OK;
+  if (!idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < score_topk_paged_ws(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  char* p = static_cast<char*>(ws);
+  int32_t* rows = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T * L);
+  int32_t* n_phys = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T);
+  float* buf = reinterpret_cast<float*>(p);
+  const int64_t ld = score_ld(L);
+  p += scores_part(T, L);
+  const int pool_rows = (int)(num_pages * page_size);
+  const cudaStream_t s = as_stream(stream);
+  misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, nullptr, L, rows, n_phys, s);
+  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, heads, T, pool_rows, H_I, h, rows, L, buf, ld, nullptr,
+                      s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, false, idx, score_opt, s);
+  return launch_status();
+}
+
+misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* pool, int64_t num_pages, int page_size,
+                                   const int32_t* page_table, int64_t max_pages, const int32_t* n,
+                                   const int32_t* cand, int T, int L, int H_I, int d, int kp, int topk, int dtype,
+                                   int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, pool, n, T, L, H_I, d, dtype, 0);
+  if (st != MISA_OK) return st;
+  st = check_paged(pool, num_pages, page_size, page_table, max_pages, L, T);
+  if (st != MISA_OK) return st;
+  if (topk < 1 || kp < topk) return MISA_ERR_INVALID_ARG;
+  if (kp > MISA_MAX_KP) return MISA_ERR_UNSUPPORTED;
+  if (T == 0) return MISA_OK;
+  if (!cand || !idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < rerank_paged_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  char* p = static_cast<char*>(ws);
+  int32_t* rows = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T * kp);
+  int32_t* n_phys = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T);
+  float* F = reinterpret_cast<float*>(p);
+  void* sel = p + align_up(sizeof(float) * (size_t)T * kp);
+  const int pool_rows = (int)(num_pages * page_size);
+  const cudaStream_t s = as_stream(stream);
+  misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, cand, kp, rows, n_phys, s);
+  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, nullptr, T, pool_rows, H_I, H_I, rows, kp, F, kp,
+                      nullptr, s);
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, false, idx, score_opt, s);
   return launch_status();
 }
 

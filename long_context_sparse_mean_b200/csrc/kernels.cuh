@@ -16,10 +16,12 @@ void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L
 // Router: partial-block means, per-chunk affinities, then sum, weight and top-h.
 int route_chunks(int L, int B);  // chunks of kRouteTile blocks per query (upper bound)
 // kbar_parts: [3][ceil(L/B)][128] bf16 scratch for the tensor-core router (shared cache).
+// pm_in: [T][128] means of each query's partial last block computed beforehand (paged caches),
+// or nullptr to average them from k.
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
                   int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
-                  uint32_t* done, __nv_bfloat16* kbar_parts, cudaStream_t s);
+                  uint32_t* done, __nv_bfloat16* kbar_parts, const float* pm_in, cudaStream_t s);
 
 // Router on the tensor cores for queries that share one bf16 cache and its pooled keys: per-tile
 // sums over full blocks into Sp [T][nch][H_I], then route_finish.  False (nothing launched) when
@@ -86,5 +88,18 @@ void launch_block_scores(DType dt, const void* q, const float* w, const void* k,
 // rows[t, a*B + i] = blocks[t, a]*B + i, or -1 for an empty slot or a token past the prefix.
 void launch_expand_blocks(const int32_t* blocks, int m, const int32_t* n, int T, int L, int B, int32_t* rows,
                           cudaStream_t s);
+
+// Paged key caches (paged.cu): pool [num_pages, page_size, 128], table [T][max_pages].
+// rows[t, p] = physical pool row of logical token p (ids == nullptr) or ids[t, p] when it lies in
+// [0, n_t) and its page is in range, else -1; n_phys[t] = num_pages * page_size.
+void launch_paged_rows(const int32_t* table, int64_t max_pages, int64_t num_pages, int page_size, const int32_t* n,
+                       int T, int L, const int32_t* ids, int P, int32_t* rows, int32_t* n_phys, cudaStream_t s);
+// Block means of logical blocks [b0, b1) of every sequence (as launch_pool).
+void launch_pool_paged(DType dt, const void* pool, int64_t num_pages, int page_size, const int32_t* table,
+                       int64_t max_pages, int n_seq, int L, int B, float* kbar, int64_t kbar_seq_stride, int b0,
+                       int b1, cudaStream_t s);
+// pm[t] = mean of the partial last block of query t's prefix (untouched when n_t is a multiple of B).
+void launch_partial_mean_paged(DType dt, const void* pool, int64_t num_pages, int page_size, const int32_t* table,
+                               int64_t max_pages, const int32_t* n, int T, int L, int B, float* pm, cudaStream_t s);
 
 }  // namespace misa

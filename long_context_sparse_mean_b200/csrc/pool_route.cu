@@ -295,7 +295,8 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
                                                                  const int32_t* __restrict__ n, int L, int B, int h,
                                                                  int nch, float* __restrict__ partial,
                                                                  uint32_t* __restrict__ done,
-                                                                 int32_t* __restrict__ heads, float* __restrict__ r_opt) {
+                                                                 int32_t* __restrict__ heads, float* __restrict__ r_opt,
+                                                                 const float* __restrict__ pm_in) {
   constexpr int H = NG * 8;
   __shared__ uint2 frag[NG][8][32];
   __shared__ float wsum[8][H];
@@ -314,8 +315,12 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
     return;
   }
   if (nfull < Mt && nfull >= bb && nfull < bb + kRouteMmaTile) {  // this tile holds the partial block
-    const float m = block_mean_256<DType::BF16>(k + (int64_t)t * k_seq_stride, nfull * B, nt, part);
-    if (threadIdx.x < kD) pms[threadIdx.x] = m;
+    if (pm_in) {  // averaged beforehand (paged caches)
+      if (threadIdx.x < kD) pms[threadIdx.x] = pm_in[(int64_t)t * kD + threadIdx.x];
+    } else {
+      const float m = block_mean_256<DType::BF16>(k + (int64_t)t * k_seq_stride, nfull * B, nt, part);
+      if (threadIdx.x < kD) pms[threadIdx.x] = m;
+    }
   }
   {  // every thread issues its fragment loads together (256 threads)
     constexpr int kPer = (NG * 8 * 32 + 255) / 256;
@@ -521,11 +526,11 @@ int route_chunks(int L, int B) {
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L, int H_I,
                   int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial, uint32_t* done,
-                  __nv_bfloat16* kbar_parts, cudaStream_t s) {
+                  __nv_bfloat16* kbar_parts, const float* pm_in, cudaStream_t s) {
   if (T <= 0) return;
   const int M = (L + B - 1) / B;
   // many queries on one shared cache: tensor-core contraction over blocks of queries
-  if (dt == DType::BF16 && k_seq_stride == 0 && kbar_seq_stride == 0 && T >= kRouteTcMinQueries &&
+  if (dt == DType::BF16 && !pm_in && k_seq_stride == 0 && kbar_seq_stride == 0 && T >= kRouteTcMinQueries &&
       launch_route_tc(q, w, k, kbar, n, T, L, H_I, B, h, heads, r_opt, kbar_parts, partial, route_chunks(L, B), s))
     return;
   if (dt == DType::BF16) {
@@ -538,7 +543,7 @@ void launch_route(DType dt, const void* q, const float* w, const void* k, int64_
 #define MISA_ROUTE_CASE(NGV)                                                                                  \
   case NGV:                                                                                                   \
     route_affinity_mma_kernel<NGV><<<grid, 256, 0, s>>>(qb, w, kb, k_seq_stride, kbar, kbar_seq_stride, n, L, B, h, \
-                                                        nch, partial, done, heads, r_opt);                    \
+                                                        nch, partial, done, heads, r_opt, pm_in);             \
     break;
       MISA_ROUTE_CASE(1)
       MISA_ROUTE_CASE(2)
@@ -563,7 +568,10 @@ void launch_route(DType dt, const void* q, const float* w, const void* k, int64_
   } else {
     const int nch = route_chunks(L, B);
     const size_t smem = sizeof(float) * (size_t)kD * ((H_I + 4) + (kRouteTile + 4));
-    partial_mean_kernel<DType::F32><<<T, 256, 0, s>>>(k, k_seq_stride, n, L, B, pm);
+    if (pm_in)
+      pm = const_cast<float*>(pm_in);
+    else
+      partial_mean_kernel<DType::F32><<<T, 256, 0, s>>>(k, k_seq_stride, n, L, B, pm);
     cudaFuncSetAttribute(route_affinity_kernel<DType::F32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     route_affinity_kernel<DType::F32><<<dim3(nch, T), 4 * H_I, smem, s>>>(q, kbar, kbar_seq_stride, pm, n, L,

@@ -35,7 +35,8 @@ def test_header_declares_the_indexer_calls():
     names = declared_functions()
     for want in ("misa_pool_keys", "misa_route", "misa_token_scores", "misa_topk_select", "misa_score_topk",
                  "misa_hier_rerank", "dsa_dense_topk", "misa_workspace_bytes", "misa_status_str", "misa_version",
-                 "misa_device_check", "misa_block_filter_topk"):
+                 "misa_device_check", "misa_block_filter_topk", "misa_pool_keys_paged", "misa_route_paged",
+                 "misa_score_topk_paged", "misa_hier_rerank_paged"):
         assert want in names, want
 
 
@@ -186,6 +187,42 @@ def test_block_filter_argument_checks(lib):
     assert block_filter(lib, wsb=1000) == WORKSPACE
     assert block_filter(lib, ws=MISALIGNED) == WORKSPACE
     assert block_filter(lib, T=0, q=None, w=None, k=None, n=None, kbar=None, heads=None) == OK
+
+
+def test_paged_workspaces_and_argument_checks(lib):
+    ws = lib.misa_workspace_bytes
+    # route: the contiguous router's workspace plus [T, 128] partial-block means
+    assert ws(6, 32, 131072, 64, 128, 8, 0, 0) == ws(0, 32, 131072, 64, 128, 8, 0, 0) + 32 * 128 * 4
+    # scoring + top-k: [T, L] physical rows and [T] row counts in front of the contiguous layout
+    assert ws(7, 32, 131072, 64, 0, 8, 8192, 0) == 32 * 131072 * 4 + 256 + ws(1, 32, 131072, 64, 0, 8, 8192, 0)
+    # re-rank: [T, k'] physical rows and [T] row counts in front of the contiguous layout
+    assert ws(8, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + 256 + ws(2, 32, 0, 64, 0, 0, 2048, 8192)
+
+    def score(**kw):
+        a = dict(q=FAKE, w=FAKE, pool=FAKE, num_pages=100, ps=64, table=FAKE, max_pages=20, n=FAKE, heads=FAKE, T=4,
+                 L=1000, H_I=64, d=128, h=8, topk=10, dt=BF16, idx=FAKE, vals=None, ws=FAKE, wsb=1 << 30, s=None)
+        a.update(kw)
+        return lib.misa_score_topk_paged(*(a[x] for x in ("q", "w", "pool", "num_pages", "ps", "table", "max_pages",
+                                                          "n", "heads", "T", "L", "H_I", "d", "h", "topk", "dt",
+                                                          "idx", "vals", "ws", "wsb", "s")))
+    assert score(L=1281) == INVALID           # 20 pages of 64 keys hold 1280
+    assert score(table=None) == INVALID
+    assert score(pool=None) == INVALID
+    assert score(ps=0) == INVALID
+    assert score(num_pages=1 << 26) == UNSUPPORTED  # pool rows past int32
+    assert score(heads=None) == INVALID
+    assert score(wsb=1000) == WORKSPACE
+    assert score(T=0, q=None, w=None, pool=None, n=None, heads=None, table=None) == OK
+    st = lib.misa_hier_rerank_paged(FAKE, FAKE, FAKE, 100, 64, FAKE, 20, FAKE, FAKE, 4, 1000, 64, 128, 100, 200, BF16,
+                                    FAKE, None, FAKE, 1 << 30, None)
+    assert st == INVALID  # k' < k
+    st = lib.misa_route_paged(FAKE, FAKE, FAKE, 100, 64, FAKE, 20, FAKE, 0, FAKE, 4, 1000, 64, 128, 64, 8, BF16, FAKE,
+                              None, FAKE, 1 << 30, None)
+    assert st == INVALID  # queries need their own pooled caches
+    st = lib.misa_pool_keys_paged(FAKE, 100, 64, FAKE, 20, 2, 1000, 128, 64, BF16, FAKE, 16 * 128 - 1, 0, 16, None)
+    assert st == INVALID  # pooled caches overlap
+    assert lib.misa_pool_keys_paged(FAKE, 100, 64, FAKE, 20, 2, 1000, 128, 64, BF16, FAKE, 16 * 128, 16, 16,
+                                    None) == OK  # empty block range
 
 
 def test_binding_rejects_host_tensors():
