@@ -16,7 +16,8 @@ bounded sample of the same workload.
 
 --block-filter M (decode workloads) adds, outside the timed step, MISA with the token-axis block
 filter keeping M blocks per query on the same inputs (route + misa_block_filter_topk) as the
-line's "block_filter_same_inputs" object.
+line's "block_filter_same_inputs" object; --paged PAGE_SIZE adds the same MISA-dagger step on the
+inputs stored in shuffled pages ("paged_same_inputs").
 """
 from __future__ import annotations
 
@@ -263,6 +264,55 @@ def block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d)
     return {"m": m, "kept_tokens_per_query": P, "route_plus_filter_ms": step_ms,
             "query_tokens_per_s": T * L / (step_ms / 1000.0), "call_ms": call_ms / nrep,
             "algorithmic_bytes_per_call": alg, "launches_per_call": 5}
+
+
+def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev):
+    """MISA-dagger on the same decode inputs stored in pages of one shared pool, outside the timed
+    step: the caches are copied page by page into a shuffled pool (page_size keys a page), then
+    route + routed scores + top-k' + re-rank + top-k through the *_paged calls are replayed as a
+    CUDA graph (pooling, like the main step's newest block, refreshes one block per sequence)."""
+    ps = args.paged
+    T, L, d = kd.shape
+    B, h, kp, kk = wl.B, wl.h, wl.kp, wl.topk
+    lp = -(-L // ps)
+    g = torch.Generator(device="cpu").manual_seed(20261200 + ps)
+    perm = torch.randperm(T * lp, generator=g).to(dev)
+    pool = torch.zeros((T * lp, ps, d), dtype=kd.dtype, device=dev)
+    padded = torch.zeros((T, lp * ps, d), dtype=kd.dtype, device=dev)
+    padded[:, :L] = kd
+    pool[perm] = padded.reshape(T * lp, ps, d)
+    del padded
+    table = perm.reshape(T, lp).to(torch.int32).contiguous()
+    kbar = M.misa_pool_keys_paged(pool, table, B, L=L)
+    M_ = -(-L // B)
+    heads = torch.empty((T, h), dtype=torch.int32, device=dev)
+    cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
+    idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+    vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
+    wsp = M.Workspace(dev)
+
+    def step():
+        M.misa_pool_keys_paged(pool, table, B, L=L, kbar=kbar, block_begin=M_ - 1, block_end=M_)
+        M.misa_route_paged(qd, wd, pool, table, kbar, nd, B, h, L=L, heads=heads, ws=wsp)
+        M.misa_score_topk_paged(qd, wd, pool, table, nd, heads, kp, L=L, idx=cand, want_vals=False, ws=wsp)
+        M.misa_hier_rerank_paged(qd, wd, pool, table, nd, cand, kk, L=L, idx=idx, vals=vals, ws=wsp)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    run = _graphed(torch, step, not args.no_graph)
+    for _ in range(3):
+        run()
+    nrep = max(1, min(args.steps, 50))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(nrep):
+        run()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / nrep
+    return {"page_size": ps, "pages_per_sequence": lp, "ms_per_step": ms,
+            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 9}
 
 
 def prefill_sample_inputs(wl, count):
@@ -704,6 +754,7 @@ def run_ours(args):
         dsa_ms = d0.elapsed_time(d1) / nrep
 
     bf = block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d=d) if args.block_filter else None
+    paged = paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev) if args.paged else None
 
     if rank == 0:
         hbm, kind = _peaks()
@@ -738,6 +789,8 @@ def run_ours(args):
                 bf["cpu_oracle"] = {"query_tokens_per_s": L / dt, "cores": thr,
                                     "sample": "1 sequence, route + block filter + refinement, double precision"}
             line["block_filter_same_inputs"] = bf
+        if paged is not None:
+            line["paged_same_inputs"] = paged
         if not args.no_cpu_baseline:
             per = max(1, min(T, os.cpu_count() or 1))
             dt, thr = cpu_baseline_sample(wl, list(range(per)))
@@ -764,6 +817,9 @@ def main():
                          "partition/resolve kernels (instead of one CTA per row)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
+    ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
+                    help="decode: also time the MISA-dagger step on the same inputs stored in shuffled pages of "
+                         "PAGE_SIZE keys (the *_paged calls), outside the timed step")
     ap.add_argument("--block-filter", type=int, default=0, metavar="M",
                     help="decode: also time MISA with the token-axis block filter keeping M blocks per query "
                          "(route + misa_block_filter_topk) on the same inputs, outside the timed step")

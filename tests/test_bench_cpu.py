@@ -22,7 +22,7 @@ def test_bench_module_defines_its_helpers():
     import bench
     for name in ("ClockSampler", "_sha", "_peaks", "_tc_peaks", "_graphed", "run_ours", "run_prefill",
                  "run_reference", "cpu_baseline_sample", "cpu_prefill_sample", "block_filter_leg",
-                 "cpu_block_filter_sample"):
+                 "cpu_block_filter_sample", "paged_leg"):
         assert hasattr(bench, name), name
     assert bench._sha(bench.TRAFFIC["file"])
 
@@ -51,4 +51,4 @@ def test_block_filter_cpu_sample():
 def test_block_filter_flag_parses():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--help"], capture_output=True, text=True,
                          timeout=120, cwd=ROOT)
-    assert out.returncode == 0 and "--block-filter" in out.stdout
+    assert out.returncode == 0 and "--block-filter" in out.stdout and "--paged" in out.stdout
