@@ -5,9 +5,9 @@ tensors' device pointers and the current CUDA stream through ctypes.  Every step
 runs in the library's CUDA kernels; there is no fallback.  If libmisa.so is missing the import
 of this module fails.
 
-Workspaces: a call given no Workspace uses one default buffer per device, shared by every such call
-on that device.  Calls in one stream are ordered, so that is safe there; calls on different streams
-that may overlap on the GPU must each pass their own Workspace.
+Workspaces: a call given no Workspace uses a default buffer of its device and stream, shared only by
+calls ordered on that stream, so calls on different streams never share scratch.  A Workspace passed
+explicitly must likewise serve one stream at a time.
 
 Tensor conventions (all on one CUDA device, contiguous):
   q [T, H_I, 128] bf16 or fp32, w [T, H_I] fp32, n [T] int32 (prefix lengths),
@@ -217,13 +217,17 @@ class Workspace:
 _default_ws = {}
 
 
-def _ws(ws: Optional[Workspace], device) -> Workspace:
+def _ws(ws: Optional[Workspace], device, stream=None) -> Workspace:
+    """The caller's Workspace, or the default one of (device, stream): calls ordered on one stream
+    share it, calls on different streams never do."""
     if ws is not None:
         return ws
-    key = str(device)
-    if key not in _default_ws:
-        _default_ws[key] = Workspace(device)
-    return _default_ws[key]
+    st = stream if stream is not None else torch.cuda.current_stream(device)
+    key = (str(device), int(st.cuda_stream))
+    w = _default_ws.get(key)
+    if w is None:
+        w = _default_ws[key] = Workspace(device)
+    return w
 
 
 def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, block_begin: int = 0,
@@ -272,7 +276,7 @@ def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optiona
     if r is None and want_r:
         r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_ROUTE, T, L, H_I, B, h)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_route", _lib.misa_route(
         _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r),
         _p(buf), nbytes, _stream(stream)))
@@ -337,7 +341,7 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=scores.device)
     nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, 8)
-    buf = _ws(ws, scores.device).get(nbytes)
+    buf = _ws(ws, scores.device, stream).get(nbytes)
     _check("misa_topk_select", _lib.misa_topk_select(
         _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), _p(buf), nbytes, int(ws_prepared), _stream(stream)))
     return idx, vals
@@ -368,7 +372,7 @@ def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_fu
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     op = OP_TOPK_SELECT if scores_full is not None else OP_SCORE_TOPK
     nbytes = misa_workspace_bytes(op, T, L, H_I, 1, h, topk)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_score_topk", _lib.misa_score_topk(
         _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, topk, _dtype_code(q), _p(idx), _p(vals),
         _p(scores_full), _p(buf), nbytes, _stream(stream)))
@@ -396,7 +400,7 @@ def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_RERANK, T, L, H_I, 1, 0, topk, kp)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_hier_rerank", _lib.misa_hier_rerank(
         _p(q), _p(w), _p(k), kss, _p(n), _p(cand), T, L, H_I, d, kp, topk, _dtype_code(q), _p(idx), _p(vals),
         _p(buf), nbytes, _stream(stream)))
@@ -421,7 +425,7 @@ def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, w
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_DENSE_TOPK, T, L, H_I, 1, 0, topk)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("dsa_dense_topk", _lib.dsa_dense_topk(
         _p(q), _p(w), _p(k), kss, _p(n), T, L, H_I, d, topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes,
         _stream(stream)))
@@ -466,7 +470,7 @@ def misa_block_filter_topk(q, w, k, kbar, n, heads, B: int, m: int, topk: int, i
         block_scores = torch.empty((T, M), dtype=torch.float32, device=q.device)
     ld_bs = 0 if block_scores is None else block_scores.shape[1]
     nbytes = misa_workspace_bytes(OP_BLOCK_FILTER, T, L, H_I, B, h, topk, m)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_block_filter_topk", _lib.misa_block_filter_topk(
         _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), _p(heads), T, L, H_I, d, B, h, m, topk, _dtype_code(q),
         _p(block_scores), ld_bs, _p(blocks), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
@@ -590,7 +594,7 @@ def misa_route_paged(q, w, pool, page_table, kbar, n, B: int, h: int, L: Optiona
     if r is None and want_r:
         r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_ROUTE_PAGED, T, L, H_I, B, h)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_route_paged", _lib.misa_route_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(kbar),
         kbar.shape[1] * kbar.shape[2], _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r), _p(buf), nbytes,
@@ -620,7 +624,7 @@ def misa_score_topk_paged(q, w, pool, page_table, n, heads, topk: int, L: Option
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_SCORE_TOPK_PAGED, T, L, H_I, 0, h, topk)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_score_topk_paged", _lib.misa_score_topk_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(heads), T, L, H_I, d, h,
         topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
@@ -649,7 +653,7 @@ def misa_hier_rerank_paged(q, w, pool, page_table, n, cand, topk: int, L: Option
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_RERANK_PAGED, T, L, H_I, 0, 0, topk, kp)
-    buf = _ws(ws, q.device).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes)
     _check("misa_hier_rerank_paged", _lib.misa_hier_rerank_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(cand), T, L, H_I, d, kp,
         topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))

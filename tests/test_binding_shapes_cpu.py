@@ -96,3 +96,24 @@ def test_device_check_rejects_a_tensor_on_another_gpu(monkeypatch):
     M._on_device(OnGpu(0), None, OnGpu(0))
     with pytest.raises(ValueError, match="current device cuda:0"):
         M._on_device(OnGpu(0), OnGpu(1))
+
+
+def test_default_workspaces_are_per_stream(monkeypatch):
+    """Calls given no Workspace share the default one of their device and stream only."""
+    class FakeStream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    current = FakeStream(11)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: current)
+    monkeypatch.setattr(M, "_default_ws", {})
+    a = M._ws(None, "cpu")
+    assert M._ws(None, "cpu") is a, "one stream: one default workspace"
+    assert M._ws(None, "cpu", FakeStream(11)) is a, "the same stream given explicitly"
+    b = M._ws(None, "cpu", FakeStream(12))
+    assert b is not a, "another stream gets its own"
+    current = FakeStream(12)
+    assert M._ws(None, "cpu") is b
+    mine = M.Workspace("cpu")
+    assert M._ws(mine, "cpu") is mine, "a caller's Workspace is used as given"
+    assert a.get(64).numel() >= 64 and b.get(16) is not a.get(16)
