@@ -7,7 +7,9 @@ of this module fails.
 
 Workspaces: a call given no Workspace uses a default buffer of its device and stream, shared only by
 calls ordered on that stream, so calls on different streams never share scratch.  A Workspace passed
-explicitly must likewise serve one stream at a time.
+explicitly must likewise serve one stream at a time.  Default buffers are kept for the life of the
+process, each as large as the largest call made on its stream; release_default_workspaces() frees
+them.
 
 Tensor conventions (all on one CUDA device, contiguous):
   q [T, H_I, 128] bf16 or fp32, w [T, H_I] fp32, n [T] int32 (prefix lengths),
@@ -200,18 +202,35 @@ def misa_workspace_bytes(op: int, T: int, L: int, H_I: int, B: int = 1, h: int =
 
 class Workspace:
     """A reusable, 256-byte aligned device scratch buffer (grown on demand).  One Workspace serves
-    calls that are ordered on one stream; give each stream that may overlap another its own."""
+    calls that are ordered on one stream; give each stream that may overlap another its own.
+
+    The buffer is allocated on the stream of the call that needs it, so the caching allocator
+    hands its memory to no other tensor while that stream's kernels may still use it.  A call on
+    another stream marks the buffer as used there too (record_stream, outside graph capture), so
+    a buffer that is replaced later returns to the allocator only after the work of every stream
+    that used it."""
 
     def __init__(self, device=None):
         self.device = device
         self.buf = None
+        self._home = None  # raw handle of the stream the buffer was allocated on
 
-    def get(self, nbytes: int) -> Optional[torch.Tensor]:
+    def get(self, nbytes: int, stream=None) -> Optional[torch.Tensor]:
         if nbytes <= 0:
             return None
+        st = stream if stream is not None else torch.cuda.current_stream(self.device)
         if self.buf is None or self.buf.numel() < nbytes:
-            self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+            with torch.cuda.stream(st):
+                self.buf = torch.empty(nbytes, dtype=torch.uint8, device=self.device or "cuda")
+            self._home = int(st.cuda_stream)
+        elif int(st.cuda_stream) != self._home and not torch.cuda.is_current_stream_capturing():
+            self.buf.record_stream(st)
         return self.buf
+
+    def release(self) -> None:
+        """Drop the buffer (its memory goes back to torch's caching allocator)."""
+        self.buf = None
+        self._home = None
 
 
 _default_ws = {}
@@ -219,7 +238,8 @@ _default_ws = {}
 
 def _ws(ws: Optional[Workspace], device, stream=None) -> Workspace:
     """The caller's Workspace, or the default one of (device, stream): calls ordered on one stream
-    share it, calls on different streams never do."""
+    share it, calls on different streams never do.  Default workspaces stay allocated (each as
+    large as the largest call made on its stream) until release_default_workspaces()."""
     if ws is not None:
         return ws
     st = stream if stream is not None else torch.cuda.current_stream(device)
@@ -228,6 +248,15 @@ def _ws(ws: Optional[Workspace], device, stream=None) -> Workspace:
     if w is None:
         w = _default_ws[key] = Workspace(device)
     return w
+
+
+def release_default_workspaces() -> None:
+    """Free every default workspace (for example after a run on many external streams, whose
+    handles could otherwise be reused by unrelated streams that then inherit a large buffer).
+    Synchronises the device first, so no kernel still uses them."""
+    if _default_ws:
+        torch.cuda.synchronize()
+    _default_ws.clear()
 
 
 def misa_pool_keys(k: torch.Tensor, B: int, kbar: Optional[torch.Tensor] = None, block_begin: int = 0,
@@ -276,7 +305,7 @@ def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optiona
     if r is None and want_r:
         r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_ROUTE, T, L, H_I, B, h)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_route", _lib.misa_route(
         _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r),
         _p(buf), nbytes, _stream(stream)))
@@ -311,7 +340,7 @@ def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, se
         if select_ws is None:
             raise ValueError("select_topk needs select_ws")
         nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, H_I)
-        buf = select_ws.get(nbytes)
+        buf = select_ws.get(nbytes, stream)
     _check("misa_token_scores", _lib.misa_token_scores(
         _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, _dtype_code(q), _p(out), out.shape[1],
         select_topk, _p(buf), nbytes, _stream(stream)))
@@ -341,7 +370,7 @@ def misa_topk_select(scores, n, topk: int, L: Optional[int] = None, idx=None, va
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=scores.device)
     nbytes = misa_workspace_bytes(OP_TOPK_SELECT, T, L, 8)
-    buf = _ws(ws, scores.device, stream).get(nbytes)
+    buf = _ws(ws, scores.device, stream).get(nbytes, stream)
     _check("misa_topk_select", _lib.misa_topk_select(
         _p(scores), ld, _p(n), T, L, topk, _p(idx), _p(vals), _p(buf), nbytes, int(ws_prepared), _stream(stream)))
     return idx, vals
@@ -372,7 +401,7 @@ def misa_score_topk(q, w, k, n, heads, topk: int, idx=None, vals=None, scores_fu
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     op = OP_TOPK_SELECT if scores_full is not None else OP_SCORE_TOPK
     nbytes = misa_workspace_bytes(op, T, L, H_I, 1, h, topk)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_score_topk", _lib.misa_score_topk(
         _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, topk, _dtype_code(q), _p(idx), _p(vals),
         _p(scores_full), _p(buf), nbytes, _stream(stream)))
@@ -400,7 +429,7 @@ def misa_hier_rerank(q, w, k, n, cand, topk: int, idx=None, vals=None, want_vals
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_RERANK, T, L, H_I, 1, 0, topk, kp)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_hier_rerank", _lib.misa_hier_rerank(
         _p(q), _p(w), _p(k), kss, _p(n), _p(cand), T, L, H_I, d, kp, topk, _dtype_code(q), _p(idx), _p(vals),
         _p(buf), nbytes, _stream(stream)))
@@ -425,7 +454,7 @@ def dsa_dense_topk(q, w, k, n, topk: int, idx=None, vals=None, want_vals=True, w
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_DENSE_TOPK, T, L, H_I, 1, 0, topk)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("dsa_dense_topk", _lib.dsa_dense_topk(
         _p(q), _p(w), _p(k), kss, _p(n), T, L, H_I, d, topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes,
         _stream(stream)))
@@ -470,7 +499,7 @@ def misa_block_filter_topk(q, w, k, kbar, n, heads, B: int, m: int, topk: int, i
         block_scores = torch.empty((T, M), dtype=torch.float32, device=q.device)
     ld_bs = 0 if block_scores is None else block_scores.shape[1]
     nbytes = misa_workspace_bytes(OP_BLOCK_FILTER, T, L, H_I, B, h, topk, m)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_block_filter_topk", _lib.misa_block_filter_topk(
         _p(q), _p(w), _p(k), kss, _p(kbar), kbss, _p(n), _p(heads), T, L, H_I, d, B, h, m, topk, _dtype_code(q),
         _p(block_scores), ld_bs, _p(blocks), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
@@ -594,7 +623,7 @@ def misa_route_paged(q, w, pool, page_table, kbar, n, B: int, h: int, L: Optiona
     if r is None and want_r:
         r = torch.empty((T, H_I), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_ROUTE_PAGED, T, L, H_I, B, h)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_route_paged", _lib.misa_route_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(kbar),
         kbar.shape[1] * kbar.shape[2], _p(n), T, L, H_I, d, B, h, _dtype_code(q), _p(heads), _p(r), _p(buf), nbytes,
@@ -624,7 +653,7 @@ def misa_score_topk_paged(q, w, pool, page_table, n, heads, topk: int, L: Option
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_SCORE_TOPK_PAGED, T, L, H_I, 0, h, topk)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_score_topk_paged", _lib.misa_score_topk_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(heads), T, L, H_I, d, h,
         topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))
@@ -653,7 +682,7 @@ def misa_hier_rerank_paged(q, w, pool, page_table, n, cand, topk: int, L: Option
     if vals is None and want_vals:
         vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
     nbytes = misa_workspace_bytes(OP_RERANK_PAGED, T, L, H_I, 0, 0, topk, kp)
-    buf = _ws(ws, q.device, stream).get(nbytes)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
     _check("misa_hier_rerank_paged", _lib.misa_hier_rerank_paged(
         _p(q), _p(w), _p(pool), num_pages, page_size, _p(page_table), max_pages, _p(n), _p(cand), T, L, H_I, d, kp,
         topk, _dtype_code(q), _p(idx), _p(vals), _p(buf), nbytes, _stream(stream)))

@@ -116,4 +116,55 @@ def test_default_workspaces_are_per_stream(monkeypatch):
     assert M._ws(None, "cpu") is b
     mine = M.Workspace("cpu")
     assert M._ws(mine, "cpu") is mine, "a caller's Workspace is used as given"
-    assert a.get(64).numel() >= 64 and b.get(16) is not a.get(16)
+
+
+def test_workspace_buffers_belong_to_the_stream_that_uses_them(monkeypatch):
+    """A workspace buffer is allocated on the stream of the call that grows it, and a call on
+    another stream marks it as used there (so the allocator recycles it only after that stream's
+    work), except while a CUDA graph is being captured."""
+    import contextlib
+
+    class FakeStream:
+        def __init__(self, handle):
+            self.cuda_stream = handle
+
+    class FakeBuf:
+        def __init__(self, n):
+            self.n, self.uses = n, []
+
+        def numel(self):
+            return self.n
+
+        def record_stream(self, st):
+            self.uses.append(st.cuda_stream)
+
+    entered = []
+
+    @contextlib.contextmanager
+    def fake_stream_ctx(st):
+        entered.append(st.cuda_stream)
+        yield
+
+    capturing = [False]
+    monkeypatch.setattr(torch.cuda, "stream", fake_stream_ctx)
+    monkeypatch.setattr(torch.cuda, "is_current_stream_capturing", lambda: capturing[0])
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda device=None: FakeStream(5))
+    monkeypatch.setattr(torch, "empty", lambda n, **kw: FakeBuf(n))
+    ws = M.Workspace("cpu")
+    assert ws.get(0) is None
+    b1 = ws.get(64)
+    assert entered == [5] and b1.numel() == 64, "allocated on the current stream"
+    assert ws.get(32, FakeStream(5)) is b1 and b1.uses == [], "same stream: no record"
+    assert ws.get(32, FakeStream(9)) is b1 and b1.uses == [9], "another stream is recorded"
+    capturing[0] = True
+    ws.get(32, FakeStream(10))
+    assert b1.uses == [9], "no record_stream while capturing"
+    capturing[0] = False
+    b2 = ws.get(128, FakeStream(9))
+    assert b2 is not b1 and entered == [5, 9], "a larger buffer is allocated on the calling stream"
+    ws.release()
+    assert ws.buf is None
+    monkeypatch.setattr(M, "_default_ws", {"x": ws})
+    monkeypatch.setattr(torch.cuda, "synchronize", lambda: None)
+    M.release_default_workspaces()
+    assert M._default_ws == {}
