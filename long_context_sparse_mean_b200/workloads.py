@@ -23,10 +23,17 @@ Value distributions
 * needles (config 1): two seeded heads j1, j2 get w = +1 for every query and
   q_{t,j} = 4 u_j + xi; four keys (two per head) at seeded positions inside every query's
   prefix are k = 40 u_j.
-* needles (config 4): 64 keys per sequence at seeded distinct positions, each
-  k = alpha * q_{t,j*} / |q_{t,j*}| for a seeded head j* with w_{t,j*} > 0, where alpha is
-  4 x the largest background key norm of that sequence (so q_hat . k_needle is at least
-  4 x q_hat . k_s for every background key).
+* needles (config 4): 64 keys per sequence at seeded distinct positions.  Needle p points along
+  a direction u_p that has a positive component along q_{j*} for a seeded head j* among the
+  query's heads with the larger positive weights, and a negative one along every head with a
+  negative weight (u_p is q_{j*} with its projection on those heads' span removed, plus a small
+  step against each of them).  Its length alpha_p makes w_{j*} (q_{j*} . k_p) at least 3 x
+  S = 3 x (sum over heads with w_j > 0 of w_j |q_j|) x (largest background key norm); alpha_p is
+  also at least 4 x that largest key norm.  After bf16 rounding the generator asserts both sign
+  conditions on the stored key.  These are sign and norm conditions on the inputs, not index
+  scores: every term of a needle's dense score with a negative weight is then zero and the term
+  of head j* alone exceeds 2 S, while no background key can score above S, so the dense top-k
+  (k >= 64) holds every needle.
 
 Every generator is keyed by (config seed, stream name, index) through numpy's SeedSequence, so
 one sequence or one query chunk can be regenerated on its own.
@@ -113,9 +120,13 @@ def round_bf16(x: np.ndarray) -> np.ndarray:
     float32 -> bfloat16 conversion is exact.  Inputs are finite.
     """
     x = np.ascontiguousarray(x, dtype=np.float32)
-    u = x.view(np.uint32).astype(np.uint64)
-    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
-    return u.astype(np.uint32).view(np.float32)
+    u = x.view(np.uint32)
+    # finite inputs stay below 0xff800000, so adding at most 0x8000 cannot wrap in 32 bits
+    r = (u >> 16) & np.uint32(1)
+    r += np.uint32(0x7FFF)
+    r += u
+    r &= np.uint32(0xFFFF0000)
+    return r.view(np.float32)
 
 
 def _finish(wl: Workload, x: np.ndarray) -> np.ndarray:
@@ -144,7 +155,9 @@ def head_prefs(wl: Workload) -> list:
 def _clustered_keys(wl: Workload, g: np.random.Generator, n: int, C: np.ndarray) -> np.ndarray:
     z = g.integers(0, N_CLUSTERS, size=n)
     xi = g.standard_normal((n, wl.d), dtype=np.float32)
-    return C[z].astype(np.float32) + (0.5 / math.sqrt(wl.d)) * xi
+    xi *= np.float32(0.5 / math.sqrt(wl.d))
+    xi += C.astype(np.float32)[z]
+    return xi
 
 
 def _clustered_queries(wl: Workload, g: np.random.Generator, nq: int, C: np.ndarray, prefs) -> np.ndarray:
@@ -265,14 +278,46 @@ def decode_sequence(wl: Workload, s: int) -> DecodeSequence:
     if wl.needles == "uniform64":
         gn = _rng(wl, "needles", s)
         pos = np.sort(gn.choice(wl.L, size=64, replace=False))
-        alpha = 4.0 * float(np.sqrt((k.astype(np.float64) ** 2).sum(axis=1)).max())
-        positive = np.nonzero(w > 0)[0]
-        for p in pos:
-            j = int(gn.choice(positive))
-            qj = q[j].astype(np.float64)
-            k[p] = (alpha / np.linalg.norm(qj)) * qj
-        k = _finish(wl, k)
+        k[pos] = _needle_keys(wl, gn, q, w, k, len(pos))
     return DecodeSequence(k=k, q=q, w=w, n=wl.L, needle_pos=pos)
+
+
+def _needle_keys(wl: Workload, g: np.random.Generator, q: np.ndarray, w: np.ndarray, k: np.ndarray,
+                 count: int) -> np.ndarray:
+    """Keys of `count` planted needles for one decode query (module docstring, config 4).
+
+    Only signs and norms of the inputs are used: the direction of needle p is orthogonal to, then
+    stepped against, the query vectors of the heads with negative weight, and its length follows
+    from the weights, the query norms and the largest background key norm."""
+    q64 = q.astype(np.float64)
+    w64 = w.astype(np.float64)
+    qn = np.linalg.norm(q64, axis=1)
+    kmax = float(np.sqrt(np.einsum("ij,ij->i", k, k, dtype=np.float64).max()))
+    pos_w = np.nonzero(w64 > 0)[0]
+    strong = pos_w[w64[pos_w] >= np.median(w64[pos_w])]
+    neg = np.nonzero(w64 < 0)[0]
+    S = float((w64[pos_w] * qn[pos_w]).sum()) * kmax
+    N = q64[neg]  # [m, d]
+    basis = np.linalg.qr(N.T)[0] if len(neg) else np.zeros((wl.d, 0))
+    out = np.empty((count, wl.d), np.float32)
+    for a in range(count):
+        j = int(g.choice(strong))
+        u = q64[j] - basis @ (basis.T @ q64[j])  # no component along any negative head
+        un = np.linalg.norm(u)
+        if len(neg):
+            # a step against every negative head: N u = -0.02 |q_j'| |u| for each of them
+            u = u + np.linalg.lstsq(N, -0.02 * qn[neg] * un, rcond=None)[0]
+        u /= np.linalg.norm(u)
+        proj = float(q64[j] @ u)
+        alpha = max(3.0 * S / (w64[j] * proj), 4.0 * kmax)
+        key = _finish(wl, (alpha * u)[None, :])[0]
+        kd = key.astype(np.float64)
+        if len(neg) and not np.all(N @ kd < 0.0):
+            raise RuntimeError("needle key projects positively on a negative-weight head")
+        if not w64[j] * float(q64[j] @ kd) > 2.0 * S:
+            raise RuntimeError("needle key too short")
+        out[a] = key
+    return out
 
 
 def decode_batch(wl: Workload, seqs=None):

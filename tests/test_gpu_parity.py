@@ -1,9 +1,12 @@
 """CUDA path against the CPU oracle on the five workloads, at full size.
 
 The GPU runs every workload whole, in the launch configuration the benchmark uses.  The oracle
-checks every query of the decode workloads it can afford (all of configs 1, 2 and 4; a seeded
-sample of config 5; a seeded sample of prefill queries spread over every chunk, including the
-first and last positions and block edges).
+checks every query of the decode workloads (configs 1, 2, 4 and 5, the dense indexer on every
+sequence too) and, in prefill, every query of the first and last 128-query tile of the first and
+last chunk plus block and chunk edges and seeded queries spread over every chunk.  A few queries
+sharing one 128K cache (the multi-query decode regime on the tensor cores) run the whole
+MISA-dagger path.  On the 128K MISA-dagger workload the planted needles must all be in the GPU's
+dense top-k.
 
 Per sampled query:
   * pooled keys, router scores and routed heads against the oracle (tie band on r);
@@ -149,8 +152,13 @@ def _decode_case(name, wl, check_seqs, dense_seqs=(), run_dagger=None):
             ious.append(_iou(fin_h[s] if run_dagger else sel_h[s], gd[s]))
         extra["iou_vs_dense"] = float(np.mean(ious))
         if needles[0] is not None:
-            extra["needle_recall_dense_gpu"] = float(np.mean([len(set(needles[s]) & set(gd[s])) / len(needles[s])
-                                                              for s in dense_seqs]))
+            rec = [len(set(needles[s]) & set(gd[s])) / len(needles[s]) for s in dense_seqs]
+            extra["needle_recall_dense_gpu"] = float(np.mean(rec))
+            # the planted needles outscore every background key under the dense indexer
+            assert min(rec) == 1.0, f"{name}: dense top-k misses planted needles (recall {rec})"
+            if run_dagger:
+                extra["needle_recall_misa_gpu"] = float(np.mean(
+                    [len(set(needles[s]) & set(sel_h[s])) / len(needles[s]) for s in range(S)]))
     report(name, checked_queries=len(check_seqs), **stats, **extra)
     return stats
 
@@ -207,27 +215,34 @@ def test_config1_tiny_fp32():
 
 def test_config2_decode_32k():
     wl = W.WORKLOADS[2]
-    _decode_case("cfg2_decode_32k", wl, list(range(wl.n_seq)), dense_seqs=[0, 1], run_dagger=False)
+    every = list(range(wl.n_seq))
+    _decode_case("cfg2_decode_32k", wl, every, dense_seqs=every, run_dagger=False)
 
 
 def test_config4_misa_dagger_128k():
     wl = W.WORKLOADS[4]
-    _decode_case("cfg4_misa_dagger_128k", wl, list(range(wl.n_seq)), dense_seqs=[0, 1, 2, 3])
+    every = list(range(wl.n_seq))
+    _decode_case("cfg4_misa_dagger_128k", wl, every, dense_seqs=every)
 
 
 def test_config5_glm5_128k():
     wl = W.WORKLOADS[5]
-    rng = np.random.default_rng(5)
-    check = sorted(set([0, wl.n_seq - 1] + rng.choice(wl.n_seq, 6, replace=False).tolist()))
-    _decode_case("cfg5_glm5_128k", wl, check, dense_seqs=check[:4], run_dagger=False)
+    every = list(range(wl.n_seq))
+    _decode_case("cfg5_glm5_128k", wl, every, dense_seqs=every, run_dagger=False)
 
 
 def _prefill_sample(wl):
+    """Every query of the first and the last 128-query tile of the first and the last chunk, block
+    and chunk edges, and seeded queries spread over the whole prefill."""
+    ch = wl.chunk
+    tiles = []
+    for c0 in (0, wl.T - ch):
+        tiles += list(range(c0, c0 + 128)) + list(range(c0 + ch - 128, c0 + ch))
     fixed = [0, 1, 2, 63, 64, 127, 128, 129, 255, 256, 4095, 4096, 4097, 8191, 32767, 32768, 65407, 65408,
              65534, 65535]
     rng = np.random.default_rng(3)
-    extra = rng.choice(wl.T, 16, replace=False).tolist()
-    return sorted(set(t for t in fixed + extra if t < wl.T))
+    extra = rng.choice(wl.T, 64, replace=False).tolist()
+    return sorted(set(t for t in tiles + fixed + extra if t < wl.T))
 
 
 def test_config3_prefill_64k():
@@ -269,3 +284,37 @@ def test_config3_prefill_64k():
         og = {"r": orc["r"][a], "heads": orc["heads"][a], "I": I_o[a], "top_I": orc["idx"][a]}
         _check_query("cfg3", wl, t, q[a], w[a], k, int(n[a]), gpu, og, stats)
     report("cfg3_prefill_64k", checked_queries=len(ts), **stats)
+
+
+def test_shared_cache_few_queries_128k_misa_dagger():
+    """Four queries on one shared 131072-key bf16 cache (speculative or multi-token decode) through
+    the whole MISA-dagger path: router, routed scores on the tensor cores, top-k', dense re-rank."""
+    wl = W.small(3, name="shared_L131072_T4", L=131072, T=4, chunk=None, kp=8192)
+    L_ = lib()
+    inp = W.shared_inputs(wl)
+    dt = kdtype(wl)
+    kd, qd = dev(inp.k, dt), dev(inp.q, dt)
+    wd, nd = dev(inp.w, torch.float32), dev(inp.n, torch.int32)
+    B, h, kk, kp = wl.B, wl.h, wl.topk, wl.kp
+    kbar = L_.misa_pool_keys(kd, B)
+    res = L_.misa_indexer(qd, wd, kd, kbar, nd, B, h, kk, kp=kp)
+    _, r = L_.misa_route(qd, wd, kd, kbar, nd, B, h, want_r=True)
+    o = oracle.get()
+    orc = o.indexer(oracle.MODE_DAGGER, inp.q, inp.w, inp.k, 0, inp.n, B, h, kk, kp=kp)
+    oh = dev(orc["heads"], torch.int32)
+    I_oh = host(L_.misa_token_scores(qd, wd, kd, nd, oh))
+    idx_oh, _ = L_.misa_score_topk(qd, wd, kd, nd, oh, kp)
+    fo, fv = L_.misa_hier_rerank(qd, wd, kd, nd, dev(orc["cand"], torch.int32), kk)
+    I_o = o.scores(inp.q, inp.w, inp.k, 0, inp.n, heads=orc["heads"], ld=wl.L)
+    F_c = o.dense_scores_at(inp.q, inp.w, inp.k, 0, inp.n, orc["cand"])
+    stats = dict(head_swaps=0, token_swaps=0, e2e_token_swaps=0, e2e_skipped_head_band=0, rerank_swaps=0,
+                 e2e_final_swaps=0, e2e_final_skipped_cand_band=0)
+    hh, rr, cc, ff = host(res["heads"]), host(r), host(res["cand"]), host(res["idx"])
+    iohh, fo_h, fv_h = host(idx_oh), host(fo), host(fv)
+    for t in range(wl.T):
+        gpu = {"r": rr[t], "heads": hh[t], "I_oh": I_oh[t], "idx_oh": iohh[t], "sel": cc[t], "fin_oc": fo_h[t],
+               "fin_oc_v": fv_h[t], "fin": ff[t]}
+        og = {"r": orc["r"][t], "heads": orc["heads"][t], "I": I_o[t], "top_I": orc["cand"][t]}
+        _check_query("shared_L131072_T4", wl, t, inp.q[t], inp.w[t], inp.k, int(inp.n[t]), gpu, og, stats,
+                     {"F_cand": F_c[t], "fin": orc["idx"][t]})
+    report("shared_L131072_T4_misa_dagger", checked_queries=wl.T, **stats)
