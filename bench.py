@@ -11,13 +11,21 @@ than L2, so every step streams it from HBM).  Metric: scored query-tokens per se
 (T x L / step time), summed over GPUs.  With torchrun every rank runs its own batch of sequences
 (independent problems, weak scaling); the time is the max over ranks.
 
+On one GPU the same run also measures, outside the timed step and reported as keys of the same
+JSON line:
+  dense_dsa_same_inputs     the dense indexer on the decode inputs, and the MISA-dagger:dense ratio
+  block_filter_same_inputs  MISA with the token-axis block filter (--block-filter M blocks, 128)
+  paged_same_inputs         the MISA-dagger step on the inputs stored in shuffled pages
+                            (--paged PAGE_SIZE, 64), checked against the contiguous step
+  prefill                   the chunked causal prefill (65536 queries on one 65536-key cache,
+                            chunks of 4096): the whole step, the tensor-core scorer's TFLOP/s,
+                            and the dense indexer over the same chunks
+  glm5_decode               64 sequences x 131072 keys, H_I = 32, B = 256: the MISA step against
+                            the dense indexer on the same inputs (time ratio, token IoU)
+(--no-legs skips the last two, 0 turns off the first ones).
+
 The reference arm (--impl reference) times the CPU oracle, as it stands, on the host cores, on a
 bounded sample of the same workload.
-
---block-filter M (decode workloads) adds, outside the timed step, MISA with the token-axis block
-filter keeping M blocks per query on the same inputs (route + misa_block_filter_topk) as the
-line's "block_filter_same_inputs" object; --paged PAGE_SIZE adds the same MISA-dagger step on the
-inputs stored in shuffled pages ("paged_same_inputs").
 """
 from __future__ import annotations
 
@@ -45,19 +53,21 @@ UNIT = "query-tokens/s"
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
            "sha256": "63ad9e52310709f8745fdb1ae7c3406bfae625c2343add5a1deb685d3bae57c2",
-           "bytes_per_key": (1.073953e9 + 19.169792e6) / 4194304,
-           "capture": "profiles/score_persist_decode_L131072_b32.md"}
+           "bytes_per_key": (1.073953e9 + 19.169792e6) / 4194304}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
 # chunk's launch; the step's traffic is that rate times the pairs the step scores.
 TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
                    "sha256": "3aa6df1f296fc7e0cb8afde7e9ae237d607084f9533b601ca428cd9b148f33ba",
-                   "bytes_per_pair": (52.319232e6 + 984.943616e6) / 260048896,
-                   "capture": "profiles/score_tc_prefill_L65536_chunk15.md"}
+                   "bytes_per_pair": (52.319232e6 + 984.943616e6) / 260048896}
 
 
 def _sha(path):
     with open(os.path.join(ROOT, path), "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()
+
+
+def _traffic(entry, key, units):
+    return entry[key] * units if entry["sha256"] == _sha(entry["file"]) else None
 
 
 def _peaks():
@@ -82,7 +92,7 @@ def _tc_peaks():
 
 
 class ClockSampler:
-    """Polls SM clock and clock-event reasons through NVML while the timed region runs."""
+    """Polls SM clock and clock-event reasons through NVML while the measured region runs."""
 
     REASONS = {
         0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
@@ -113,7 +123,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception:
                 pass
-            time.sleep(0.002)
+            time.sleep(0.001)
 
     def __enter__(self):
         if self.nv is not None:
@@ -126,11 +136,12 @@ class ClockSampler:
         if self._thread:
             self._thread.join()
 
-    def summary(self):
-        if not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
-        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
-                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+    def summary(self, window=None):
+        s = {"sm_mhz": statistics.median(self.samples) if self.samples else None, "sm_max_mhz": self.max_mhz,
+             "reasons": sorted(self.reasons), "samples": len(self.samples)}
+        if window:
+            s["window"] = window
+        return s
 
 
 def _graphed(torch, step, use_graph):
@@ -143,6 +154,17 @@ def _graphed(torch, step, use_graph):
         step()
     torch.cuda.synchronize()
     return g.replay
+
+
+def _event_ms(torch, stream, fn, reps):
+    """Average device time of fn() over reps back-to-back calls (CUDA events on `stream`)."""
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
 
 
 def rank_sequences(rank, world, per_rank):
@@ -182,17 +204,82 @@ def _config(wl, extra=None):
     c = {"workload": wl.name, "T_per_gpu": wl.T, "L": wl.L, "H_I": wl.H_I, "d": wl.d, "B": wl.B, "h": wl.h,
          "kp": wl.kp, "topk": wl.topk, "accumulate": "f32",
          "l2": f"inputs larger than L2 ({wl.T * wl.L * wl.d * 2 / 2**30:.2f} GiB key cache per GPU)",
-         "step": "pool newest block + route + routed scores + top-k' + dense re-rank + top-k"}
+         "step": ("pool newest block + route + routed scores + top-k' + dense re-rank + top-k" if wl.kp else
+                  "pool newest block + route + routed scores + top-k")}
     if extra:
         c.update(extra)
     return c
 
 
-def cpu_baseline_sample(wl, seqs, threads=None):
-    """Time the oracle, as it stands, on the given sequences (one decode query each)."""
+# ---- seeded inputs, drawn in parallel by spawned worker processes -----------------------------------
+
+def _pool_processes():
+    return max(1, min(32, os.cpu_count() or 1))
+
+
+def _gen_decode_into(task):
+    """Worker: draw one decode sequence and store its keys as bf16 bits in the shared block."""
+    from multiprocessing import shared_memory
+    cid, over, s, slot, shm_name, shape = task
+    wl = W.small(cid, **over)
+    seq = W.decode_sequence(wl, s)
+    shm = shared_memory.SharedMemory(name=shm_name)
+    try:
+        arr = np.ndarray(shape, dtype=np.uint16, buffer=shm.buf)
+        arr[slot] = (seq.k.view(np.uint32) >> 16).astype(np.uint16)
+    finally:
+        shm.close()
+    return slot, seq.q, seq.w, seq.n, seq.needle_pos
+
+
+class DecodeInputs:
+    """Keys of a decode batch as bf16 bits [S, L, d] in shared memory, queries, weights, prefix
+    lengths and needle positions."""
+
+    def __init__(self, wl, seqs, pool):
+        from multiprocessing import shared_memory
+        S, L, d = len(seqs), wl.L, wl.d
+        self.shape = (S, L, d)
+        self.shm = shared_memory.SharedMemory(create=True, size=max(1, S * L * d * 2))
+        over = {f: getattr(wl, f) for f in wl.__dataclass_fields__ if f != "cid"}
+        tasks = [(wl.cid, over, s, a, self.shm.name, self.shape) for a, s in enumerate(seqs)]
+        res = sorted(pool.map(_gen_decode_into, tasks), key=lambda r: r[0])
+        self.k_bits = np.ndarray(self.shape, dtype=np.uint16, buffer=self.shm.buf)
+        self.q = np.stack([r[1] for r in res])
+        self.w = np.stack([r[2] for r in res])
+        self.n = np.array([r[3] for r in res], dtype=np.int32)
+        self.needles = [r[4] for r in res]
+
+    def k_f32(self, rows):
+        """Keys of the given batch rows as float32 (exactly the bf16 values)."""
+        return (self.k_bits[rows].astype(np.uint32) << 16).view(np.float32)
+
+    def k_device(self, torch, dev):
+        t = torch.from_numpy(self.k_bits.view(np.int16)).to(dev)
+        return t.view(torch.bfloat16)
+
+    def close(self):
+        self.k_bits = None
+        self.shm.close()
+        self.shm.unlink()
+
+
+def _gen_chunk(cid, seed, c, over=None):
+    wl = W.small(cid, seed=seed, **(over or {}))
+    ch = wl.chunk
+    q, w = W.shared_queries(wl, c * ch, min((c + 1) * ch, wl.T))
+    return q, w
+
+
+def cpu_baseline_sample(wl, seqs, threads=None, inputs=None):
+    """Time the oracle, as it stands, on the given sequences (one decode query each).  inputs:
+    (k, q, w, n) of exactly those sequences, or None to draw them."""
     import oracle
     o = oracle.get()
-    k, q, w, n, _ = W.decode_batch(wl, seqs)
+    if inputs is None:
+        k, q, w, n, _ = W.decode_batch(wl, seqs)
+    else:
+        k, q, w, n = inputs
     L, d = k.shape[1], k.shape[2]
     t0 = time.perf_counter()
     o.indexer(oracle.MODE_DAGGER if wl.kp else oracle.MODE_MISA, q, w, k, L * d, n, wl.B, wl.h, wl.topk,
@@ -201,11 +288,14 @@ def cpu_baseline_sample(wl, seqs, threads=None):
     return dt, o.num_threads()
 
 
-def cpu_block_filter_sample(wl, seqs, m):
+def cpu_block_filter_sample(wl, seqs, m, inputs=None):
     """Time the oracle's route + block filter + refinement on the given decode sequences."""
     import oracle
     o = oracle.get()
-    k, q, w, n, _ = W.decode_batch(wl, seqs)
+    if inputs is None:
+        k, q, w, n, _ = W.decode_batch(wl, seqs)
+    else:
+        k, q, w, n = inputs
     L, d = k.shape[1], k.shape[2]
     t0 = time.perf_counter()
     o.block_filter(q, w, k, L * d, n, wl.B, wl.h, m, wl.topk)
@@ -242,35 +332,26 @@ def block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d)
         both()
     torch.cuda.synchronize()
     nrep = max(1, min(args.steps, 50))
-    e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
     run = _graphed(torch, both, not args.no_graph)
     for _ in range(3):
         run()
-    e[0].record(stream)
-    for _ in range(nrep):
-        run()
-    e[1].record(stream)
-    torch.cuda.synchronize()
-    call_ms = 0.0
-    for _ in range(nrep):
-        route()
-        e[2].record(stream)
-        filt()
-        e[3].record(stream)
-        torch.cuda.synchronize()
-        call_ms += e[2].elapsed_time(e[3])
-    step_ms = e[0].elapsed_time(e[1]) / nrep
+    step_ms = _event_ms(torch, stream, run, nrep)
+    route()
+    call_ms = _event_ms(torch, stream, filt, nrep)
     alg = T * (Mb * h_d * 4 + h * h_d * 2 + h * 4 + P * (h_d * 2 + 4 + 4 + 4) + m * 4 + kk * 8)
     return {"m": m, "kept_tokens_per_query": P, "route_plus_filter_ms": step_ms,
-            "query_tokens_per_s": T * L / (step_ms / 1000.0), "call_ms": call_ms / nrep,
+            "query_tokens_per_s": T * L / (step_ms / 1000.0), "call_ms": call_ms,
             "algorithmic_bytes_per_call": alg, "launches_per_call": 5}
 
 
-def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev):
+def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     """MISA-dagger on the same decode inputs stored in pages of one shared pool, outside the timed
     step: the caches are copied page by page into a shuffled pool (page_size keys a page), then
     route + routed scores + top-k' + re-rank + top-k through the *_paged calls are replayed as a
-    CUDA graph (pooling, like the main step's newest block, refreshes one block per sequence)."""
+    CUDA graph (pooling, like the main step's newest block, refreshes one block per sequence).
+    The final selection is compared with the contiguous step's (ref_idx) on the same inputs; the
+    paged routed-scoring call is timed alone against its algorithmic bytes (the key rows and the
+    page-table entries it reads)."""
     ps = args.paged
     T, L, d = kd.shape
     B, h, kp, kk = wl.B, wl.h, wl.kp, wl.topk
@@ -291,28 +372,36 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev):
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     wsp = M.Workspace(dev)
 
+    def score():
+        M.misa_score_topk_paged(qd, wd, pool, table, nd, heads, kp, L=L, idx=cand, want_vals=False, ws=wsp)
+
     def step():
         M.misa_pool_keys_paged(pool, table, B, L=L, kbar=kbar, block_begin=M_ - 1, block_end=M_)
         M.misa_route_paged(qd, wd, pool, table, kbar, nd, B, h, L=L, heads=heads, ws=wsp)
-        M.misa_score_topk_paged(qd, wd, pool, table, nd, heads, kp, L=L, idx=cand, want_vals=False, ws=wsp)
+        score()
         M.misa_hier_rerank_paged(qd, wd, pool, table, nd, cand, kk, L=L, idx=idx, vals=vals, ws=wsp)
 
     for _ in range(3):
         step()
     torch.cuda.synchronize()
+    same = None
+    if ref_idx is not None:
+        same = bool(torch.equal(torch.sort(idx, dim=1).values, torch.sort(ref_idx, dim=1).values))
     run = _graphed(torch, step, not args.no_graph)
     for _ in range(3):
         run()
     nrep = max(1, min(args.steps, 50))
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(nrep):
-        run()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / nrep
+    ms = _event_ms(torch, stream, run, nrep)
+    score_ms = _event_ms(torch, stream, score, nrep)
+    hbm, kind = _peaks()
+    alg = T * (L * d * 2 + lp * 4)
     return {"page_size": ps, "pages_per_sequence": lp, "ms_per_step": ms,
-            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 9}
+            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 9,
+            "matches_contiguous": same,
+            "routed_scoring_call": {"ms": score_ms, "algorithmic_bytes": alg,
+                                    "achieved_GBps": alg / (score_ms / 1000.0) / 1e9,
+                                    "frac_of_hbm": alg / (score_ms / 1000.0) / 1e9 / hbm, "peak_kind": kind,
+                                    "launches": 3}}
 
 
 def prefill_sample_inputs(wl, count):
@@ -335,6 +424,8 @@ def cpu_prefill_sample(wl, inputs):
     return dt, o.num_threads(), int(n.astype(np.int64).sum())
 
 
+# ---- the reference arm: the oracle on the host cores -------------------------------------------------
+
 def run_reference(args):
     """The reference arm: the CPU oracle on a bounded sample of the workload."""
     ws, rank, _ = _dist()
@@ -347,11 +438,12 @@ def run_reference(args):
         return run_reference_prefill(args, wl, nthr)
     per_step = max(1, min(wl.T, nthr))
     seqs = list(range(per_step))
+    k, q, w, n, _ = W.decode_batch(wl, seqs)
     for _ in range(args.warmup):
-        cpu_baseline_sample(wl, seqs)
+        cpu_baseline_sample(wl, seqs, inputs=(k, q, w, n))
     times = []
     for _ in range(args.steps):
-        dt, thr = cpu_baseline_sample(wl, seqs)
+        dt, thr = cpu_baseline_sample(wl, seqs, inputs=(k, q, w, n))
         times.append(dt)
     units = per_step * wl.L
     total = sum(times)
@@ -362,8 +454,9 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
         "config": _config(wl, {"sample_sequences_per_step": per_step}),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": thr, "kind": "oracle",
-                         "sample": f"{per_step} of {wl.T} sequences per step, whole MISA-dagger path, "
-                                   f"double precision, OpenMP over sequences"},
+                         "sample": f"{per_step} of {wl.T} sequences per step, whole "
+                                   f"{'MISA-dagger' if wl.kp else 'MISA'} path, double precision, OpenMP over "
+                                   f"sequences"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -397,34 +490,20 @@ def run_reference_prefill(args, wl, nthr):
     return 0
 
 
-def _gen_chunk(cid, seed, c):
-    wl = W.small(cid, seed=seed)
-    ch = wl.chunk
-    q, w = W.shared_queries(wl, c * ch, min((c + 1) * ch, wl.T))
-    return q, w
+# ---- chunked causal prefill (shared cache) ------------------------------------------------------------
 
-
-def run_prefill(args, wl):
+def prefill_measure(args, wl, dev, gen_pool, steps, warmup, dist=None, ws=1, want_e2e=True, want_dense=True,
+                    want_cpu=True):
     """One step = the whole chunked causal prefill of one sequence: pool every block of the shared
     cache once, then for each chunk of queries route, score with the routed heads on the tensor
-    cores, and select the top-k of every query."""
-    import multiprocessing as mp
-
-    ws, rank, local = _dist()
-    wl = rank_workload(wl, rank)
-    ch = wl.chunk
-    nch = -(-wl.T // ch)
-    with mp.get_context("spawn").Pool(min(nch, max(1, os.cpu_count() or 1))) as pool:
-        parts = pool.starmap(_gen_chunk, [(wl.cid, wl.seed, c) for c in range(nch)])
+    cores, and select the top-k of every query.  Returns the measurements as a dict."""
     import torch
-    import torch.distributed as dist
-
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
     from long_context_sparse_mean_b200 import binding as M
 
+    ch = wl.chunk
+    nch = -(-wl.T // ch)
+    over = {f: getattr(wl, f) for f in wl.__dataclass_fields__ if f not in ("cid", "seed")}
+    parts = gen_pool.starmap(_gen_chunk, [(wl.cid, wl.seed, c, over) for c in range(nch)])
     k_h = W.shared_keys(wl)
     n_h = W.prefix_lengths(wl)
     L, d, T, B, h, kk = wl.L, wl.d, wl.T, wl.B, wl.h, wl.topk
@@ -472,42 +551,44 @@ def run_prefill(args, wl):
             if stages:
                 stage_ev[c][3].record(stream)
 
-    # launches per step: pool + per chunk (route 1, tensor-core scores 1, selection 3)
+    # launches per step: pool + per chunk (route 1, tensor-core scores 1, selection 1); the router
+    # of a shared cache is kbar_split + route_tc + route_finish (3)
     launches_per_step = 1 + nch * 5
-    for _ in range(max(3, args.warmup)):
+    for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
 
-    score_ms = 0.0
-    nsc = min(args.steps, 5)
-    for _ in range(nsc):
-        step(time_scores=True)
-        torch.cuda.synchronize()
-        score_ms += sum(e0.elapsed_time(e1) for e0, e1 in score_ev)
-    score_ms /= nsc
-    acc = {"pool_all_blocks": 0.0, "route": 0.0, "routed_scores": 0.0, "topk": 0.0}
-    nst = min(args.steps, 5)
-    for _ in range(nst):
-        step(stages=True)
-        torch.cuda.synchronize()
-        acc["pool_all_blocks"] += pool_ev[0].elapsed_time(pool_ev[1])
-        for c in range(nch):
-            e = stage_ev[c]
-            acc["route"] += e[0].elapsed_time(e[1])
-            acc["routed_scores"] += e[1].elapsed_time(e[2])
-            acc["topk"] += e[2].elapsed_time(e[3])
-    stages_us = {k_: round(1000 * v / nst, 1) for k_, v in acc.items()}
+    clk = ClockSampler(dev.index)
+    with clk:
+        score_ms = 0.0
+        nsc = max(1, min(steps, 5))
+        for _ in range(nsc):
+            step(time_scores=True)
+            torch.cuda.synchronize()
+            score_ms += sum(e0.elapsed_time(e1) for e0, e1 in score_ev)
+        score_ms /= nsc
+        acc = {"pool_all_blocks": 0.0, "route": 0.0, "routed_scores": 0.0, "topk": 0.0}
+        nst = max(1, min(steps, 5))
+        for _ in range(nst):
+            step(stages=True)
+            torch.cuda.synchronize()
+            acc["pool_all_blocks"] += pool_ev[0].elapsed_time(pool_ev[1])
+            for c in range(nch):
+                e = stage_ev[c]
+                acc["route"] += e[0].elapsed_time(e[1])
+                acc["routed_scores"] += e[1].elapsed_time(e[2])
+                acc["topk"] += e[2].elapsed_time(e[3])
+        stages_us = {k_: round(1000 * v / nst, 1) for k_, v in acc.items()}
 
-    run_step = _graphed(torch, step, not args.no_graph)
-    for _ in range(2):
-        run_step()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+        run_step = _graphed(torch, step, not args.no_graph)
+        for _ in range(2):
+            run_step()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         t0.record(stream)
-        for _ in range(args.steps):
+        for _ in range(steps):
             run_step()
         t1.record(stream)
         torch.cuda.synchronize()
@@ -516,111 +597,254 @@ def run_prefill(args, wl):
     ms = t0.elapsed_time(t1)
     if ws > 1:
         ms = max_over_ranks(ms, dist, dev)
-    value = pairs * ws * args.steps / (ms / 1000.0)
+    out = {"ms": ms, "steps": steps, "pairs": pairs, "flops": flops, "score_ms": score_ms, "stages_us": stages_us,
+           "launches_per_step": launches_per_step, "clocks": clk.summary("score, stage and timed passes")}
 
-    # end to end: every step copies the cache, the queries, their weights and n from pinned host
-    # memory and reads every query's top-k indices back
-    k_pin = torch.from_numpy(k_h).to(torch.bfloat16).pin_memory()
-    q_pin = qd.cpu().pin_memory()
-    w_pin = wd.cpu().pin_memory()
-    n_pin = torch.from_numpy(n_h).pin_memory()
-    idx_pin = torch.empty((T, kk), dtype=torch.int32).pin_memory()
-    h2d = k_pin.numel() * 2 + q_pin.numel() * 2 + w_pin.numel() * 4 + n_pin.numel() * 4
-    d2h = idx_pin.numel() * 4
+    if want_e2e:
+        # end to end: every step copies the cache, the queries, their weights and n from pinned host
+        # memory and reads every query's top-k indices back
+        k_pin = torch.from_numpy(k_h).to(torch.bfloat16).pin_memory()
+        q_pin = qd.cpu().pin_memory()
+        w_pin = wd.cpu().pin_memory()
+        n_pin = torch.from_numpy(n_h).pin_memory()
+        idx_pin = torch.empty((T, kk), dtype=torch.int32).pin_memory()
+        h2d = k_pin.numel() * 2 + q_pin.numel() * 2 + w_pin.numel() * 4 + n_pin.numel() * 4
+        d2h = idx_pin.numel() * 4
 
-    def e2e_step():
-        kd.copy_(k_pin, non_blocking=True)
-        qd.copy_(q_pin, non_blocking=True)
-        wd.copy_(w_pin, non_blocking=True)
-        nd.copy_(n_pin, non_blocking=True)
-        step()
-        idx_pin.copy_(idx, non_blocking=True)
+        def e2e_step():
+            kd.copy_(k_pin, non_blocking=True)
+            qd.copy_(q_pin, non_blocking=True)
+            wd.copy_(w_pin, non_blocking=True)
+            nd.copy_(n_pin, non_blocking=True)
+            run_step()
+            idx_pin.copy_(idx, non_blocking=True)
 
-    ne = max(1, min(args.steps, 5))
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    if ws > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(ne):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
-    if ws > 1:
-        e_ms = max_over_ranks(e_ms, dist, dev)
-    e2e_value = pairs * ws * ne / (e_ms / 1000.0)
+        ne = max(1, min(steps, 5))
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if ws > 1:
+            dist.barrier()
+        e_ms = _event_ms(torch, stream, e2e_step, ne) * ne
+        if ws > 1:
+            e_ms = max_over_ranks(e_ms, dist, dev)
+        out["e2e"] = {"ms": e_ms, "steps": ne, "h2d": h2d, "d2h": d2h}
 
+    if want_dense:
+        # the dense indexer over the same chunks (all H_I heads on the tensor cores, then top-k)
+        didx = torch.empty((ch, kk), dtype=torch.int32, device=dev)
+
+        def dense_step():
+            for a, b in chunks:
+                M.dsa_dense_topk(qd[a:b], wd[a:b], kd, nd[a:b], kk, idx=didx[: b - a], want_vals=False, ws=wsp)
+
+        dense_step()
+        torch.cuda.synchronize()
+        run_dense = _graphed(torch, dense_step, not args.no_graph)
+        run_dense()
+        dense_ms = _event_ms(torch, stream, run_dense, max(1, min(steps, 3)))
+        out["dense"] = {"ms_per_step": dense_ms, "pairs_per_s": pairs / (dense_ms / 1000.0),
+                        "misa_over_dense_time": (ms / steps) / dense_ms,
+                        "dense_speedup_of_misa": dense_ms / (ms / steps),
+                        "launches_per_step": nch * 2}
+    if want_cpu and not args.no_cpu_baseline:
+        count = max(1, min(64, 2 * (os.cpu_count() or 1)))
+        dt, thr, u = cpu_prefill_sample(wl, prefill_sample_inputs(wl, count))
+        out["cpu_baseline"] = {"value": u / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
+                               "sample": f"the last {count} of {T} prefill queries: route + routed scores + "
+                                         f"top-k, double precision, OpenMP over queries"}
+    return out
+
+
+def _prefill_roofline(wl, r):
+    peaks = _tc_peaks()
+    achieved = r["flops"] / (r["score_ms"] / 1000.0) / 1e12
+    return {"bound": "tensor", "kernel": "routed token scoring (score_tc_kernel, tcgen05)",
+            "achieved": achieved, "peak": peaks["burst"], "peak_kind": peaks["kind"] + " burst", "unit": "TFLOP/s",
+            "frac": achieved / peaks["burst"], "frac_of_sustained_peak": achieved / peaks["sustained"],
+            "sustained_peak": peaks["sustained"],
+            "traffic": _traffic(TRAFFIC_PREFILL, "bytes_per_pair", r["pairs"]),
+            "traffic_note": "per step (one scorer launch per 4096-query chunk): DRAM bytes per scored pair from "
+                            "one chunk's ncu capture x pairs per step",
+            "algorithmic_flops_per_step": r["flops"], "score_ms_per_step": r["score_ms"],
+            "peak_choice": "burst: the scorer is event-timed per chunk launch (about 0.3 ms each)"}
+
+
+def _prefill_config(wl, ws, args):
+    L, T, ch, pairs = wl.L, wl.T, wl.chunk, int(W.prefix_lengths(wl).astype(np.int64).sum())
+    return {"workload": wl.name, "L": L, "T": T, "chunk": ch, "H_I": wl.H_I, "d": wl.d, "B": wl.B, "h": wl.h,
+            "topk": wl.topk, "accumulate": "f32", "causal": "n_t = t + 1",
+            "units": f"scored (query, key) pairs, sum of n_t = {pairs} per step (T x L = {T * L})",
+            "l2": f"score rows of one chunk ({ch * L * 4 / 2**30:.1f} GiB) exceed L2; the 16 MiB key cache stays "
+                  f"in L2",
+            "parallelism": f"{ws} GPU(s), one independent sequence per GPU", "cuda_graph": not args.no_graph,
+            "step": "pool all blocks + per chunk: route + routed scores + top-k"}
+
+
+def run_prefill(args, wl):
+    """The prefill workload as the main line (--workload 3)."""
+    import multiprocessing as mp
+
+    ws, rank, local = _dist()
+    wl = rank_workload(wl, rank)
+    with mp.get_context("spawn").Pool(_pool_processes()) as gen_pool:
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dev = torch.device("cuda", local)
+        if ws > 1:
+            dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
+        r = prefill_measure(args, wl, dev, gen_pool, args.steps, args.warmup, dist if ws > 1 else None, ws,
+                            want_dense=not args.no_dense, want_cpu=rank == 0)
     if rank == 0:
-        peaks = _tc_peaks()
-        achieved = flops / (score_ms / 1000.0) / 1e12
-        traffic = None
-        if TRAFFIC_PREFILL["sha256"] == _sha(TRAFFIC_PREFILL["file"]):
-            traffic = TRAFFIC_PREFILL["bytes_per_pair"] * pairs
+        e = r["e2e"]
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": wl.name, "L": L, "T": T, "chunk": ch, "H_I": wl.H_I, "d": d, "B": B, "h": h,
-                       "topk": kk, "accumulate": "f32", "causal": "n_t = t + 1",
-                       "units": f"scored (query, key) pairs, sum of n_t = {pairs} per step "
-                                f"(T x L = {T * L})",
-                       "l2": f"score rows of one chunk ({ch * L * 4 / 2**30:.1f} GiB) exceed L2; the "
-                             f"16 MiB key cache stays in L2",
-                       "parallelism": f"{ws} GPU(s), one independent sequence per GPU",
-                       "cuda_graph": not args.no_graph,
-                       "step": "pool all blocks + per chunk: route + routed scores + top-k"},
-            "roofline": {"bound": "tensor", "kernel": "routed token scoring (score_tc_kernel, tcgen05)",
-                         "achieved": achieved, "peak": peaks["sustained"], "peak_kind": peaks["kind"] + " sustained",
-                         "unit": "TFLOP/s", "frac": achieved / peaks["sustained"],
-                         "frac_of_burst_peak": achieved / peaks["burst"], "traffic": traffic,
-                         "traffic_per_launch_note": "per step (16 chunk launches): bytes per scored pair from "
-                                                    "the capture x pairs per step",
-                         "algorithmic_flops_per_step": flops, "score_ms_per_step": score_ms},
-            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches_per_step * args.steps,
-            "stages_us": stages_us,
-            "clocks": clk.summary(),
+            "metric": METRIC, "value": r["pairs"] * ws * args.steps / (r["ms"] / 1000.0), "unit": UNIT,
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": _prefill_config(wl, ws, args),
+            "roofline": _prefill_roofline(wl, r),
+            "e2e": {"value": r["pairs"] * ws * e["steps"] / (e["ms"] / 1000.0), "unit": UNIT,
+                    "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]},
+            "gpu_launches": r["launches_per_step"] * args.steps,
+            "stages_us": r["stages_us"],
+            "clocks": r["clocks"],
         }
-        if not args.no_cpu_baseline:
-            count = max(1, min(64, 2 * (os.cpu_count() or 1)))
-            dt, thr, u = cpu_prefill_sample(wl, prefill_sample_inputs(wl, count))
-            line["cpu_baseline"] = {"value": u / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
-                                    "sample": f"the last {count} of {T} prefill queries: route + routed scores + "
-                                              f"top-k, double precision, OpenMP over queries"}
+        if "dense" in r:
+            line["dense_dsa_same_inputs"] = r["dense"]
+        if "cpu_baseline" in r:
+            line["cpu_baseline"] = r["cpu_baseline"]
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.destroy_process_group()
     return 0
 
 
+# ---- decode legs ------------------------------------------------------------------------------------
+
+def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
+    """MISA (routed top-k, no re-rank) against the dense indexer on one decode workload, outside the
+    main timed step: the step (pool the newest block + route + routed scores + top-k) replayed as a
+    CUDA graph, the routed scorer launch alone against its algorithmic bytes, the dense indexer on
+    the same inputs, and the token IoU of the two selections."""
+    inp = DecodeInputs(wl, list(range(wl.T)), gen_pool)
+    try:
+        kd = inp.k_device(torch, dev)
+    finally:
+        inp.close()
+    qd = torch.from_numpy(inp.q).to(torch.bfloat16).to(dev)
+    wd = torch.from_numpy(inp.w).to(dev)
+    nd = torch.from_numpy(inp.n).to(dev)
+    T, L, d = kd.shape
+    B, h, kk = wl.B, wl.h, wl.topk
+    M_ = -(-L // B)
+    stream = torch.cuda.current_stream()
+    wsp, sel_ws = M.Workspace(dev), M.Workspace(dev)
+    kbar = M.misa_pool_keys(kd, B)
+    heads = torch.empty((T, h), dtype=torch.int32, device=dev)
+    scores = torch.empty((T, L), dtype=torch.float32, device=dev)
+    idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+    didx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+
+    def route():
+        M.misa_pool_keys(kd, B, kbar=kbar, block_begin=M_ - 1, block_end=M_)
+        M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
+
+    def score():
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
+
+    def step():
+        route()
+        score()
+        M.misa_topk_select(scores, nd, kk, idx=idx, want_vals=False, ws=sel_ws)
+
+    def dense():
+        M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=didx, want_vals=False, ws=wsp)
+
+    for _ in range(3):
+        step()
+        dense()
+    torch.cuda.synchronize()
+    a, b = idx.cpu().numpy(), didx.cpu().numpy()
+    ious = [len(np.intersect1d(a[t][a[t] >= 0], b[t][b[t] >= 0])) /
+            max(1, len(np.union1d(a[t][a[t] >= 0], b[t][b[t] >= 0]))) for t in range(T)]
+    run = _graphed(torch, step, not args.no_graph)
+    run_dense = _graphed(torch, dense, not args.no_graph)
+    for _ in range(3):
+        run()
+        run_dense()
+    nrep = max(3, min(steps, 50))
+    clk = ClockSampler(dev.index)
+    with clk:
+        ms = _event_ms(torch, stream, run, nrep)
+        dense_ms = _event_ms(torch, stream, run_dense, nrep)
+        route()
+        score_ms = _event_ms(torch, stream, score, nrep)
+    hbm, kind = _peaks()
+    alg = T * (L * d * 2 + h * d * 2 + h * 4)
+    res = {"workload": wl.name, "T": T, "L": L, "H_I": wl.H_I, "B": B, "h": h, "topk": kk,
+           "ms_per_step": ms, "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 4,
+           "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
+                        "achieved": alg / (score_ms / 1000.0) / 1e9, "peak": hbm, "peak_kind": kind,
+                        "unit": "GB/s", "frac": alg / (score_ms / 1000.0) / 1e9 / hbm,
+                        "algorithmic_bytes_per_launch": alg, "avg_launch_ms": score_ms},
+           "dense": {"ms_per_call": dense_ms, "query_tokens_per_s": T * L / (dense_ms / 1000.0),
+                     "launches_per_call": 2},
+           "misa_over_dense_time": ms / dense_ms, "dense_speedup_of_misa": dense_ms / ms,
+           "iou_vs_dense": float(np.mean(ious)), "iou_vs_dense_min": float(np.min(ious)),
+           "clocks": clk.summary("step, dense and scorer timing passes")}
+    del kd, qd, wd, nd, kbar, scores
+    return res
+
+
 def run_ours(args):
+    import multiprocessing as mp
+
+    ws, rank, local = _dist()
+    wl = _workload(args)
+    if wl.n_seq == 1:
+        raise SystemExit("shared-cache workloads run through run_prefill")
+    gen_pool = mp.get_context("spawn").Pool(_pool_processes())
+    try:
+        return _run_ours(args, ws, rank, local, wl, gen_pool)
+    finally:
+        gen_pool.close()
+        gen_pool.join()
+
+
+def _run_ours(args, ws, rank, local, wl, gen_pool):
+    big = W.small(wl.cid, n_seq=wl.n_seq * ws, T=wl.T * ws)
+    seqs = rank_sequences(rank, ws, wl.T)
+    inp = DecodeInputs(big, seqs, gen_pool)
+
     import torch
     import torch.distributed as dist
 
-    ws, rank, local = _dist()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if ws > 1:
         dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
     from long_context_sparse_mean_b200 import binding as M
 
-    wl = _workload(args)
-    if wl.n_seq == 1:
-        raise SystemExit("shared-cache workloads run through run_prefill")
-    big = W.small(wl.cid, n_seq=wl.n_seq * ws, T=wl.T * ws)
-    seqs = rank_sequences(rank, ws, wl.T)
-    k_h, q_h, w_h, n_h, _ = W.decode_batch(big, seqs)
-    T, L, d = k_h.shape
-    kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
-    qd = torch.from_numpy(q_h).to(torch.bfloat16).to(dev)
-    wd = torch.from_numpy(w_h).to(dev)
-    nd = torch.from_numpy(n_h).to(dev)
+    kd = inp.k_device(torch, dev)
+    T, L, d = inp.shape
     B, h, kp, kk, H_I = wl.B, wl.h, wl.kp, wl.topk, wl.H_I
     M_ = -(-L // B)
     stream = torch.cuda.current_stream()
+    # q, w and n live in one device staging block, so the end-to-end step fills them (and the newest
+    # key of every sequence) with one host-to-device copy
+    q_bytes, w_bytes, n_bytes, knew_bytes = T * H_I * d * 2, T * H_I * 4, T * 4, T * d * 2
+    offs = np.cumsum([0] + [(x + 255) // 256 * 256 for x in (q_bytes, w_bytes, n_bytes, knew_bytes)])
+    stage_d = torch.empty(int(offs[-1]), dtype=torch.uint8, device=dev)
+    qd = stage_d[offs[0]:offs[0] + q_bytes].view(torch.bfloat16).view(T, H_I, d)
+    wd = stage_d[offs[1]:offs[1] + w_bytes].view(torch.float32).view(T, H_I)
+    nd = stage_d[offs[2]:offs[2] + n_bytes].view(torch.int32)
+    knew_d = stage_d[offs[3]:offs[3] + knew_bytes].view(torch.bfloat16).view(T, d)
+    qd.copy_(torch.from_numpy(inp.q).to(torch.bfloat16))
+    wd.copy_(torch.from_numpy(inp.w))
+    nd.copy_(torch.from_numpy(inp.n))
+    knew_d.copy_(kd[:, L - 1, :])
     wsp = M.Workspace(dev)
     sel_ws = M.Workspace(dev)  # selection state shared by the scoring and top-k' calls
     kbar = M.misa_pool_keys(kd, B)
@@ -662,32 +886,33 @@ def run_ours(args):
         step()
     torch.cuda.synchronize()
 
-    # one timed pass over the step for the scoring-kernel duration (events bracket that launch)
-    for _ in range(min(args.steps, 50)):
-        step(time_scores=True)
-        torch.cuda.synchronize()
-        score_ms.append(ev[0].elapsed_time(ev[1]))
+    clk = ClockSampler(local)
+    with clk:
+        # one timed pass over the step for the scoring-kernel duration (events bracket that launch)
+        for _ in range(min(args.steps, 50)):
+            step(time_scores=True)
+            torch.cuda.synchronize()
+            score_ms.append(ev[0].elapsed_time(ev[1]))
 
-    # per-stage breakdown (events between the calls; separate untimed steps)
-    stage_names = ["pool_newest_block", "route", "routed_scores", "topk_kprime", "rerank"]
-    stage_acc = [0.0] * len(stage_names)
-    nst = min(args.steps, 20)
-    for _ in range(nst):
-        step(stages=True)
-        torch.cuda.synchronize()
-        for i in range(len(stage_names)):
-            stage_acc[i] += stage_ev[i].elapsed_time(stage_ev[i + 1])
-    stages_us = {nm: round(1000 * a / nst, 2) for nm, a in zip(stage_names, stage_acc)}
+        # per-stage breakdown (events between the calls; separate untimed steps)
+        stage_names = ["pool_newest_block", "route", "routed_scores", "topk_kprime", "rerank"]
+        stage_acc = [0.0] * len(stage_names)
+        nst = min(args.steps, 20)
+        for _ in range(nst):
+            step(stages=True)
+            torch.cuda.synchronize()
+            for i in range(len(stage_names)):
+                stage_acc[i] += stage_ev[i].elapsed_time(stage_ev[i + 1])
+        stages_us = {nm: round(1000 * a / nst, 2) for nm, a in zip(stage_names, stage_acc)}
 
-    # the timed region: K whole steps
-    run_step = _graphed(torch, step, not args.no_graph)
-    for _ in range(3):
-        run_step()
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if ws > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+        # the timed region: K whole steps
+        run_step = _graphed(torch, step, not args.no_graph)
+        for _ in range(3):
+            run_step()
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         t0.record(stream)
         for _ in range(args.steps):
             run_step()
@@ -700,26 +925,22 @@ def run_ours(args):
         ms = max_over_ranks(ms, dist, dev)
     units_per_step = T * L * ws
     value = units_per_step * args.steps / (ms / 1000.0)
+    ref_idx = idx.clone()
 
-    # end to end through the public API with host buffers: per step the new query q, its head
-    # weights w, the newest key of every sequence (written into the cache) and n go host->device,
-    # and the selected indices come back device->host.
-    q_pin = torch.from_numpy(q_h).to(torch.bfloat16).pin_memory()
-    w_pin = torch.from_numpy(w_h).pin_memory()
-    n_pin = torch.from_numpy(n_h).pin_memory()
-    knew_pin = torch.from_numpy(k_h[:, L - 1, :].copy()).to(torch.bfloat16).pin_memory()
-    knew_d = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+    # end to end through the public API with host buffers: per step the new queries q, their head
+    # weights w, the prefix lengths n and the newest key of every sequence go host->device in one
+    # copy from pinned memory (the key is then written into the cache), the step runs, and the
+    # selected indices come back device->host.
+    stage_pin = torch.empty(int(offs[-1]), dtype=torch.uint8).pin_memory()
+    stage_pin.copy_(stage_d.cpu())
     idx_pin = torch.empty((T, kk), dtype=torch.int32).pin_memory()
-    h2d = q_pin.numel() * 2 + w_pin.numel() * 4 + n_pin.numel() * 4 + knew_pin.numel() * 2
+    h2d = q_bytes + w_bytes + n_bytes + knew_bytes
     d2h = idx_pin.numel() * 4
 
     def e2e_step():
-        qd.copy_(q_pin, non_blocking=True)
-        wd.copy_(w_pin, non_blocking=True)
-        nd.copy_(n_pin, non_blocking=True)
-        knew_d.copy_(knew_pin, non_blocking=True)
+        stage_d.copy_(stage_pin, non_blocking=True)
         kd[:, L - 1, :].copy_(knew_d)
-        step()
+        run_step()
         idx_pin.copy_(idx, non_blocking=True)
 
     for _ in range(3):
@@ -727,13 +948,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    e_ms = e0.elapsed_time(e1)
+    e_ms = _event_ms(torch, stream, e2e_step, args.steps) * args.steps
     if ws > 1:
         e_ms = max_over_ranks(e_ms, dist, dev)
     e2e_value = units_per_step * args.steps / (e_ms / 1000.0)
@@ -741,29 +956,26 @@ def run_ours(args):
     # dense DSA on the same inputs (the baseline the pages compare against), not part of the step
     dsa_ms = None
     if not args.no_dense:
+        didx = torch.empty((T, kk), dtype=torch.int32, device=dev)
+        dvals = torch.empty((T, kk), dtype=torch.float32, device=dev)
         for _ in range(3):
-            M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=idx, vals=vals, ws=wsp)
+            M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=didx, vals=dvals, ws=wsp)
         torch.cuda.synchronize()
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        nrep = min(args.steps, 20)
-        d0.record(stream)
-        for _ in range(nrep):
-            M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=idx, vals=vals, ws=wsp)
-        d1.record(stream)
-        torch.cuda.synchronize()
-        dsa_ms = d0.elapsed_time(d1) / nrep
+        dsa_ms = _event_ms(torch, stream, lambda: M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=didx, vals=dvals, ws=wsp),
+                           min(args.steps, 20))
 
-    bf = block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d=d) if args.block_filter else None
-    paged = paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev) if args.paged else None
+    single = ws == 1
+    bf = block_filter_leg(args, torch, M, qd, wd, kd, kbar, nd, wl, stream, dev, h_d=d) \
+        if args.block_filter and single else None
+    paged = paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=ref_idx) \
+        if args.paged and wl.kp and single else None
 
+    line = None
     if rank == 0:
         hbm, kind = _peaks()
         score_avg = sum(score_ms) / len(score_ms)
         alg_bytes = T * (L * d * 2 + h * d * 2 + h * 4)
         achieved = alg_bytes / (score_avg / 1000.0) / 1e9
-        traffic = None
-        if TRAFFIC["sha256"] and TRAFFIC["sha256"] == _sha(TRAFFIC["file"]) and TRAFFIC["bytes_per_key"]:
-            traffic = TRAFFIC["bytes_per_key"] * T * L
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -772,20 +984,23 @@ def run_ours(args):
                                    "cuda_graph": not args.no_graph}),
             "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
-                         "frac": achieved / hbm, "traffic": traffic,
+                         "frac": achieved / hbm,
+                         "traffic": _traffic(TRAFFIC, "bytes_per_key", T * L),
                          "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,
-            "clocks": clk.summary(),
+            "clocks": clk.summary("scorer, stage and timed passes"),
             "dense_dsa_same_inputs": None if dsa_ms is None else {
-                "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0)},
+                "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0),
+                "misa_dagger_step_over_dense_call": (ms / args.steps) / dsa_ms},
         }
         if bf is not None:
             bf["achieved_GBps"] = bf["algorithmic_bytes_per_call"] / (bf["call_ms"] / 1000.0) / 1e9
             bf["frac_of_hbm"] = bf["achieved_GBps"] / hbm
             if not args.no_cpu_baseline:
-                dt, thr = cpu_block_filter_sample(wl, [0], args.block_filter)
+                dt, thr = cpu_block_filter_sample(wl, [0], args.block_filter,
+                                                  inputs=(inp.k_f32([0]), inp.q[:1], inp.w[:1], inp.n[:1]))
                 bf["cpu_oracle"] = {"query_tokens_per_s": L / dt, "cores": thr,
                                     "sample": "1 sequence, route + block filter + refinement, double precision"}
             line["block_filter_same_inputs"] = bf
@@ -793,13 +1008,46 @@ def run_ours(args):
             line["paged_same_inputs"] = paged
         if not args.no_cpu_baseline:
             per = max(1, min(T, os.cpu_count() or 1))
-            dt, thr = cpu_baseline_sample(wl, list(range(per)))
+            rows = list(range(per))
+            dt, thr = cpu_baseline_sample(wl, rows, inputs=(inp.k_f32(rows), inp.q[:per], inp.w[:per], inp.n[:per]))
             line["cpu_baseline"] = {"value": per * L / dt, "unit": UNIT, "cores": thr, "kind": "oracle",
                                     "sample": f"{per} of {T} sequences, one pass of the whole MISA-dagger path, "
                                               f"double precision, OpenMP over sequences"}
-        print(json.dumps(line), flush=True)
+    inp.close()
     if ws > 1:
         dist.destroy_process_group()
+
+    if rank == 0 and single and not args.no_legs:
+        # further workloads on the same GPU, outside the timed step
+        del kd, stage_d, qd, wd, nd, knew_d, kbar, scores, cand, idx, vals, ref_idx
+        wsp = sel_ws = None
+        M.release_default_workspaces()
+        torch.cuda.empty_cache()
+        legs = {}
+        try:
+            r = prefill_measure(args, W.WORKLOADS[3], dev, gen_pool, max(1, min(args.steps, 5)), 2,
+                                want_e2e=False, want_dense=not args.no_dense)
+            pre = {"config": _prefill_config(W.WORKLOADS[3], 1, args),
+                   "metric": "scored (query, key) pairs per second",
+                   "value": r["pairs"] * r["steps"] / (r["ms"] / 1000.0), "ms_per_step": r["ms"] / r["steps"],
+                   "steps": r["steps"], "roofline": _prefill_roofline(W.WORKLOADS[3], r),
+                   "stages_us": r["stages_us"], "gpu_launches_per_step": r["launches_per_step"],
+                   "clocks": r["clocks"]}
+            if "dense" in r:
+                pre["dense_same_inputs"] = r["dense"]
+            if "cpu_baseline" in r:
+                pre["cpu_baseline"] = r["cpu_baseline"]
+            legs["prefill"] = pre
+        except Exception as exc:  # a failed leg is reported, the headline stands
+            legs["prefill"] = {"error": f"{type(exc).__name__}: {exc}"}
+        torch.cuda.empty_cache()
+        try:
+            legs["glm5_decode"] = misa_decode_leg(args, torch, M, W.WORKLOADS[5], dev, gen_pool, args.steps)
+        except Exception as exc:
+            legs["glm5_decode"] = {"error": f"{type(exc).__name__}: {exc}"}
+        line.update(legs)
+    if line is not None:
+        print(json.dumps(line), flush=True)
     return 0
 
 
@@ -812,17 +1060,19 @@ def main():
     ap.add_argument("--workload", type=int, default=4, choices=[2, 3, 4, 5])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-legs", action="store_true",
+                    help="decode: skip the prefill and GLM-5-shaped decode legs that follow the main line")
     ap.add_argument("--fused-histogram", action="store_true",
                     help="decode: build the top-k' histogram inside the scoring kernel and select with the "
                          "partition/resolve kernels (instead of one CTA per row)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
-    ap.add_argument("--paged", type=int, default=0, metavar="PAGE_SIZE",
+    ap.add_argument("--paged", type=int, default=64, metavar="PAGE_SIZE",
                     help="decode: also time the MISA-dagger step on the same inputs stored in shuffled pages of "
-                         "PAGE_SIZE keys (the *_paged calls), outside the timed step")
-    ap.add_argument("--block-filter", type=int, default=0, metavar="M",
+                         "PAGE_SIZE keys (the *_paged calls), outside the timed step (0: off)")
+    ap.add_argument("--block-filter", type=int, default=128, metavar="M",
                     help="decode: also time MISA with the token-axis block filter keeping M blocks per query "
-                         "(route + misa_block_filter_topk) on the same inputs, outside the timed step")
+                         "(route + misa_block_filter_topk) on the same inputs, outside the timed step (0: off)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
