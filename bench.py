@@ -4,8 +4,11 @@
 
 One step is one decode step of MISA-dagger over a batch of sequences (default: 32 sequences x
 131072 keys, H_I = 64, d = 128, B = 128, h = 8, k' = 8192, k = 2048):
-    pool the block that holds the newest key -> route (block-pooled router, top-h heads) ->
-    routed token scores -> top-k' candidates -> dense re-rank of the candidates -> top-k.
+    route (block-pooled router, top-h heads; the block holding the newest key is averaged from the
+    keys) -> routed token scores, with a sampled cut and candidate lists for the top-k' ->
+    top-k' candidates -> dense re-rank of the candidates -> top-k.
+(A block is pooled once the prefix has moved past it, once every B = 128 steps of a sequence; the
+step does not repeat it.)
 Inputs are seeded synthetic tensors resident in HBM (the key cache of 1 GiB per GPU is larger
 than L2, so every step streams it from HBM).  Metric: scored query-tokens per second
 (T x L / step time), summed over GPUs.  With torchrun every rank runs its own batch of sequences
@@ -204,8 +207,8 @@ def _config(wl, extra=None):
     c = {"workload": wl.name, "T_per_gpu": wl.T, "L": wl.L, "H_I": wl.H_I, "d": wl.d, "B": wl.B, "h": wl.h,
          "kp": wl.kp, "topk": wl.topk, "accumulate": "f32",
          "l2": f"inputs larger than L2 ({wl.T * wl.L * wl.d * 2 / 2**30:.2f} GiB key cache per GPU)",
-         "step": ("pool newest block + route + routed scores + top-k' + dense re-rank + top-k" if wl.kp else
-                  "pool newest block + route + routed scores + top-k")}
+         "step": ("route + routed scores (sampled cut, candidate lists) + top-k' + dense re-rank + top-k" if wl.kp
+                  else "route + routed scores (sampled cut, candidate lists) + top-k")}
     if extra:
         c.update(extra)
     return c
@@ -348,7 +351,7 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     """MISA-dagger on the same decode inputs stored in pages of one shared pool, outside the timed
     step: the caches are copied page by page into a shuffled pool (page_size keys a page), then
     route + routed scores + top-k' + re-rank + top-k through the *_paged calls are replayed as a
-    CUDA graph (pooling, like the main step's newest block, refreshes one block per sequence).
+    CUDA graph (as in the main step, the router averages each prefix's last block from the keys).
     The final selection is compared with the contiguous step's (ref_idx) on the same inputs; the
     paged routed-scoring call is timed alone against its algorithmic bytes (the key rows and the
     page-table entries it reads)."""
@@ -365,7 +368,6 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     del padded
     table = perm.reshape(T, lp).to(torch.int32).contiguous()
     kbar = M.misa_pool_keys_paged(pool, table, B, L=L)
-    M_ = -(-L // B)
     heads = torch.empty((T, h), dtype=torch.int32, device=dev)
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
@@ -376,7 +378,6 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
         M.misa_score_topk_paged(qd, wd, pool, table, nd, heads, kp, L=L, idx=cand, want_vals=False, ws=wsp)
 
     def step():
-        M.misa_pool_keys_paged(pool, table, B, L=L, kbar=kbar, block_begin=M_ - 1, block_end=M_)
         M.misa_route_paged(qd, wd, pool, table, kbar, nd, B, h, L=L, heads=heads, ws=wsp)
         score()
         M.misa_hier_rerank_paged(qd, wd, pool, table, nd, cand, kk, L=L, idx=idx, vals=vals, ws=wsp)
@@ -396,7 +397,7 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     hbm, kind = _peaks()
     alg = T * (L * d * 2 + lp * 4)
     return {"page_size": ps, "pages_per_sequence": lp, "ms_per_step": ms,
-            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 9,
+            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 8,
             "matches_contiguous": same,
             "routed_scoring_call": {"ms": score_ms, "algorithmic_bytes": alg,
                                     "achieved_GBps": alg / (score_ms / 1000.0) / 1e9,
@@ -725,9 +726,9 @@ def run_prefill(args, wl):
 
 def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     """MISA (routed top-k, no re-rank) against the dense indexer on one decode workload, outside the
-    main timed step: the step (pool the newest block + route + routed scores + top-k) replayed as a
-    CUDA graph, the routed scorer launch alone against its algorithmic bytes, the dense indexer on
-    the same inputs, and the token IoU of the two selections."""
+    main timed step: the step (route + routed scores + top-k) replayed as a CUDA graph, the routed
+    scoring call alone against its algorithmic bytes, the dense indexer on the same inputs, and the
+    token IoU of the two selections."""
     inp = DecodeInputs(wl, list(range(wl.T)), gen_pool)
     try:
         kd = inp.k_device(torch, dev)
@@ -738,7 +739,6 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     nd = torch.from_numpy(inp.n).to(dev)
     T, L, d = kd.shape
     B, h, kk = wl.B, wl.h, wl.topk
-    M_ = -(-L // B)
     stream = torch.cuda.current_stream()
     wsp, sel_ws = M.Workspace(dev), M.Workspace(dev)
     kbar = M.misa_pool_keys(kd, B)
@@ -748,16 +748,15 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     didx = torch.empty((T, kk), dtype=torch.int32, device=dev)
 
     def route():
-        M.misa_pool_keys(kd, B, kbar=kbar, block_begin=M_ - 1, block_end=M_)
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
 
     def score():
-        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kk, select_ws=sel_ws)
 
     def step():
         route()
         score()
-        M.misa_topk_select(scores, nd, kk, idx=idx, want_vals=False, ws=sel_ws)
+        M.misa_topk_select(scores, nd, kk, idx=idx, want_vals=False, ws=sel_ws, ws_prepared=True)
 
     def dense():
         M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=didx, want_vals=False, ws=wsp)
@@ -784,8 +783,10 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     hbm, kind = _peaks()
     alg = T * (L * d * 2 + h * d * 2 + h * 4)
     res = {"workload": wl.name, "T": T, "L": L, "H_I": wl.H_I, "B": B, "h": h, "topk": kk,
+           "step": "route + routed scores (sampled cut, candidate lists) + top-k",
            "ms_per_step": ms, "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 4,
-           "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
+           "roofline": {"bound": "hbm", "kernel": "routed scoring call: sampled cut (list_cut_kernel) + "
+                                                  "score_persist_kernel with candidate lists",
                         "achieved": alg / (score_ms / 1000.0) / 1e9, "peak": hbm, "peak_kind": kind,
                         "unit": "GB/s", "frac": alg / (score_ms / 1000.0) / 1e9 / hbm,
                         "algorithmic_bytes_per_launch": alg, "avg_launch_ms": score_ms},
@@ -830,7 +831,6 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     kd = inp.k_device(torch, dev)
     T, L, d = inp.shape
     B, h, kp, kk, H_I = wl.B, wl.h, wl.kp, wl.topk, wl.H_I
-    M_ = -(-L // B)
     stream = torch.cuda.current_stream()
     # q, w and n live in one device staging block, so the end-to-end step fills them (and the newest
     # key of every sequence) with one host-to-device copy
@@ -853,34 +853,27 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
-    score_ms = []
-    # pool, router, scores, top-k' (one CTA per row), re-rank scores, top-k of the candidates; with
-    # the fused histogram the top-k' is partition + resolve
-    launches_per_step = 7 if args.fused_histogram else 6
+    # kernels per step: router, sampled cut, routed scorer (with candidate lists), top-k' (one CTA
+    # per row), re-rank scorer, top-k of the candidates (plus two small memsets)
+    launches_per_step = 6
 
-    stage_ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
-
-    def step(time_scores=False, stages=False):
-        mark = (lambda i: stage_ev[i].record(stream)) if stages else (lambda i: None)
-        mark(0)
-        M.misa_pool_keys(kd, B, kbar=kbar, block_begin=M_ - 1, block_end=M_)
-        mark(1)
+    def route():
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
-        mark(2)
-        if time_scores:
-            ev[0].record(stream)
-        if args.fused_histogram:
-            M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
-        else:
-            M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
-        if time_scores:
-            ev[1].record(stream)
-        mark(3)
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=args.fused_histogram)
-        mark(4)
+
+    def score():
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
+
+    def select():
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=True)
+
+    def rerank():
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
-        mark(5)
+
+    def step():
+        route()
+        score()
+        select()
+        rerank()
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -888,22 +881,19 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
 
     clk = ClockSampler(local)
     with clk:
-        # one timed pass over the step for the scoring-kernel duration (events bracket that launch)
-        for _ in range(min(args.steps, 50)):
-            step(time_scores=True)
-            torch.cuda.synchronize()
-            score_ms.append(ev[0].elapsed_time(ev[1]))
-
-        # per-stage breakdown (events between the calls; separate untimed steps)
-        stage_names = ["pool_newest_block", "route", "routed_scores", "topk_kprime", "rerank"]
-        stage_acc = [0.0] * len(stage_names)
-        nst = min(args.steps, 20)
-        for _ in range(nst):
-            step(stages=True)
-            torch.cuda.synchronize()
-            for i in range(len(stage_names)):
-                stage_acc[i] += stage_ev[i].elapsed_time(stage_ev[i + 1])
-        stages_us = {nm: round(1000 * a / nst, 2) for nm, a in zip(stage_names, stage_acc)}
+        # each stage alone, replayed back to back as its own graph (the device time of its launches,
+        # no host gaps); the routed scoring call is the roofline's kernel
+        nrep = max(3, min(args.steps, 20))
+        stages_us = {}
+        for nm, fn in (("route", route), ("routed_scores", score), ("topk_kprime", select), ("rerank", rerank)):
+            g = _graphed(torch, fn, not args.no_graph)
+            g()
+            stages_us[nm] = round(1000 * _event_ms(torch, stream, g, nrep), 2)
+            if nm == "routed_scores":
+                score_avg = stages_us[nm] / 1000.0
+            del g
+        step()  # the stages above reran on the same inputs; leave one whole step's state behind
+        torch.cuda.synchronize()
 
         # the timed region: K whole steps
         run_step = _graphed(torch, step, not args.no_graph)
@@ -973,7 +963,6 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     line = None
     if rank == 0:
         hbm, kind = _peaks()
-        score_avg = sum(score_ms) / len(score_ms)
         alg_bytes = T * (L * d * 2 + h * d * 2 + h * 4)
         achieved = alg_bytes / (score_avg / 1000.0) / 1e9
         line = {
@@ -982,11 +971,14 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU",
                                    "cuda_graph": not args.no_graph}),
-            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
+            "roofline": {"bound": "hbm", "kernel": "routed scoring call: sampled cut (list_cut_kernel) + "
+                                                   "score_persist_kernel with candidate lists",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                          "frac": achieved / hbm,
                          "traffic": _traffic(TRAFFIC, "bytes_per_key", T * L),
-                         "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg},
+                         "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg,
+                         "timing": "the call replayed back to back as a CUDA graph, CUDA events on its stream; "
+                                   "its time includes the sampled cut (2048 keys a query) and the list appends"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,
@@ -1062,9 +1054,6 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-legs", action="store_true",
                     help="decode: skip the prefill and GLM-5-shaped decode legs that follow the main line")
-    ap.add_argument("--fused-histogram", action="store_true",
-                    help="decode: build the top-k' histogram inside the scoring kernel and select with the "
-                         "partition/resolve kernels (instead of one CTA per row)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
     ap.add_argument("--paged", type=int, default=64, metavar="PAGE_SIZE",

@@ -101,7 +101,9 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
  *   kbar   : out, fp32, n_seq x [ceil(L/B), d] at stride kbar_seq_stride floats
  *   blocks [block_begin, block_end) of every cache are written (clamped to [0, ceil(L/B)));
  *   block b averages keys [bB, min((b+1)B, L)) (a partial last block over its valid keys).
- * A decode loop calls it with [b, b+1) for the block that just filled.
+ * The router and the block filter average the last block of every prefix from the keys
+ * themselves, so a decode loop calls this with [b, b+1) once its prefix has moved past block b
+ * (once every B steps), not for the block that holds the newest key.
  */
 misa_status misa_pool_keys(const void* k, int64_t k_seq_stride, int n_seq, int L, int d, int B,
                            int dtype, float* kbar, int64_t kbar_seq_stride, int block_begin,
@@ -110,8 +112,9 @@ misa_status misa_pool_keys(const void* k, int64_t k_seq_stride, int n_seq, int L
 /*
  * Block-pooled router and top-h head selection ("Lightweight Block-Pooled Router").
  *   kbar   : fp32 block means from misa_pool_keys; query t reads kbar + t*kbar_seq_stride
- *            (0 = shared).  Only full blocks b < floor(n_t/B) are read from it; the partial
- *            last block of a prefix (n_t not a multiple of B) is averaged from k directly.
+ *            (0 = shared).  Only blocks b < M_t - 1 are read from it; the last block of a prefix,
+ *            keys [(M_t - 1) B, n_t) (full or partial), is averaged from k directly, so it may
+ *            hold the newest keys without being pooled.
  *   heads  : out [T, h] int32, routed heads in descending router score (ties: lower head)
  *   r_opt  : out [T, H_I] fp32 router scores, or NULL
  *   ws     : workspace of misa_workspace_bytes(MISA_OP_ROUTE, T, L, H_I, B, h, 0, 0) bytes
@@ -127,10 +130,15 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
  *   scores   : out fp32 [T, ld_scores], ld_scores >= L; entries s >= n_t are not written.
  *   select_ws, select_ws_bytes, select_topk : optional (NULL, 0, 0).  A workspace of
  *              misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes in which the call also
- *              leaves the first stage of a top-select_topk selection of these scores (the scoring
- *              kernel for per-query bf16 caches builds it while it writes the scores, otherwise a
- *              separate pass does); pass the same workspace to misa_topk_select with
- *              ws_prepared = 1.
+ *              prepares a top-select_topk selection of these scores; pass the same workspace to
+ *              misa_topk_select with ws_prepared = 1.  For one bf16 cache per query it first
+ *              scores a sample of each prefix (256 evenly spaced runs of 8 keys) to place a cut
+ *              that at least select_topk scores reach with overwhelming likelihood, then appends
+ *              every score at or above the cut to a candidate list of up to 16384 entries per
+ *              query while it writes the scores; the selection ranks that list and takes an exact
+ *              pass over the score row whenever the list cannot hold the answer (too few entries
+ *              or too many), so the result never depends on the sample.  Other caches leave no
+ *              list and the selection works from the scores alone.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -144,17 +152,18 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
  *   score_opt   : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
  *   ws          : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
  *   ws_prepared : 1 if misa_token_scores already prepared ws for these scores and this topk
- * Scores must be finite.  Without ws_prepared one CTA per row selects (ws carries nothing between
- * calls); with it the histogram-based selection that misa_token_scores started is completed.
- * Both give the same set.
+ * Scores must be finite.  One CTA per row selects; without ws_prepared it finds the row's
+ * candidates itself (a sampled cut and a pass over the row), with it it starts from the candidate
+ * list misa_token_scores left in ws.  Both give the same set.
  */
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
                              int L, int topk, int32_t* idx, float* score_opt, void* ws,
                              size_t ws_bytes, int ws_prepared, void* stream);
 
 /*
- * Routed scoring followed by top-k: misa_token_scores then misa_topk_select.  With topk = k'
- * this is the coarse stage of MISA-dagger ("Hierarchical Variant": enlarged candidate set).
+ * Routed scoring followed by top-k: misa_token_scores (preparing the selection) then
+ * misa_topk_select.  With topk = k' this is the coarse stage of MISA-dagger ("Hierarchical
+ * Variant": enlarged candidate set).
  *   scores_full_opt : [T, L] fp32 buffer that receives every score, or NULL (scores then live in
  *                     the workspace)
  *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK, T, L, ...) bytes (with scores_full_opt given,
@@ -196,12 +205,13 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
  * "Problem Statement" and "Significance and Claims": token-axis and head-axis savings combine).
  * For query t with routed heads R_t (heads[t], from misa_route):
  *   S_{t,b} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . kbar_b)     (b < M_t = ceil(n_t/B))
- * with kbar_b the router's block means (a partial last block averaged over its valid keys); the m
+ * with kbar_b the router's block means (the last block, full or partial, averaged from k); the m
  * blocks with the largest S_{t,b} are kept (ties: lower block); their prefix tokens are scored
  * with I_{t,s} and the top-k of those is selected (ties: lower token).  m >= M_t gives exactly
  * misa_score_topk's selection; h = H_I gives the block filter on the dense indexer.
  *   kbar             : fp32 block means from misa_pool_keys, 16-byte aligned; query t reads
- *                      kbar + t*kbar_seq_stride (0 = shared; else a multiple of 4, >= M*d)
+ *                      kbar + t*kbar_seq_stride (0 = shared; else a multiple of 4, >= M*d);
+ *                      blocks b < M_t - 1 only, as misa_route
  *   heads            : [T, h] routed heads in [0, H_I) (other ids are never dereferenced, but
  *                      the results are then unspecified)
  *   m                : blocks kept per query, 1 <= m with m * B <= MISA_MAX_KP

@@ -314,8 +314,9 @@ def misa_route(q, w, k, kbar, n, B: int, h: int, heads=None, r=None, ws: Optiona
 
 def misa_token_scores(q, w, k, n, heads=None, out=None, select_topk: int = 0, select_ws=None, stream=None):
     """Scores [T, L] fp32 (entries s >= n_t untouched); heads None = all heads (dense score).
-    With select_topk > 0 and a Workspace, the first stage of a top-select_topk selection of the
-    scores is left in that workspace for misa_topk_select(..., ws=<same>, ws_prepared=True)."""
+    With select_topk > 0 and a Workspace, a top-select_topk selection of the scores is prepared in
+    that workspace (for one bf16 cache per query: a sampled cut and the candidate list of every
+    query) for misa_topk_select(..., ws=<same>, ws_prepared=True)."""
     T, H_I, d = _queries(q, w, n)
     L, kss = _cache(k, T, d)
     if heads is not None:

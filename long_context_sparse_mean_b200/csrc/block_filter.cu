@@ -8,7 +8,7 @@
 //
 // Composition computed here, for query t with routed heads R_t:
 //   S_{t,b} = sum_{j in R_t} w_{t,j} * max(0, q_{t,j} . kbar_b)      (b < M_t = ceil(n_t/B))
-// with kbar_b the router's block means (the partial last block averaged over its valid keys).  The
+// with kbar_b the router's block means (the last block, full or partial, averaged from the keys).  The
 // m best blocks are kept by the per-row top-k, expand_blocks_kernel turns them into token ids, and
 // the gather scorer and the per-row top-k score and select those tokens with the routed heads.
 //
@@ -28,7 +28,7 @@ constexpr int kBlocksPerCta = 64;        // pooled blocks per CTA (8 per warp)
 // Block scores of one query over pooled blocks [blockIdx.x * 64, +64) ∩ [0, M_t).  The routed
 // heads' q rows are staged in shared memory as fp32 (dynamic, h * 128 floats).  A warp takes one
 // pooled block at a time: lane l holds columns 4l..4l+3 of kbar_b, each head's dot product is a
-// warp reduction.  The CTA whose range holds a partial last block first averages that block's keys.
+// warp reduction.  The CTA whose range holds the last block first averages that block's keys.
 template <DType DT>
 __global__ void __launch_bounds__(kBlockScoreThreads) block_score_kernel(
     const void* __restrict__ q, const float* __restrict__ w, const void* __restrict__ k, int64_t k_seq_stride,
@@ -38,11 +38,11 @@ __global__ void __launch_bounds__(kBlockScoreThreads) block_score_kernel(
   extern __shared__ __align__(16) float qs[];  // [h][kD]
   __shared__ float ws_[kMaxHeads];
   __shared__ __align__(16) float pmean[kD];
-  __shared__ float part[2][kD];
+  __shared__ float part[16 * kD];
   const int t = blockIdx.y;
   const int nt = clamp_len(n[t], L);
   const int Mt = (nt + B - 1) / B;
-  const int nfull = nt / B;  // blocks read from kbar; block nfull (if < Mt) is partial
+  const int nfull = kbar_blocks(nt, B);  // blocks read from kbar; block nfull (< Mt) is the last
   if (blockIdx.x == 0 && threadIdx.x == 0) Mt_out[t] = Mt;
   const int b0 = blockIdx.x * kBlocksPerCta;
   if (b0 >= Mt) return;
@@ -65,19 +65,12 @@ __global__ void __launch_bounds__(kBlockScoreThreads) block_score_kernel(
     }
     qs[e] = v;
   }
-  // mean of the partial last block [nfull * B, nt): 2 row groups x 128 columns
+  // mean of the last block [nfull * B, nt)
   if (nfull < Mt && nfull >= b0 && nfull < b1) {
-    const int col = tid & (kD - 1), rg = tid >> 7;
-    const int s0 = nfull * B;
-    float acc = 0.f;
-    for (int s = s0 + rg; s < nt; s += 2) {
-      const int64_t off = (int64_t)t * k_seq_stride + (int64_t)s * kD + col;
-      acc += DT == DType::BF16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(k)[off])
-                               : static_cast<const float*>(k)[off];
-    }
-    part[rg][col] = acc;
-    __syncthreads();
-    if (tid < kD) pmean[tid] = (part[0][tid] + part[1][tid]) / (float)(nt - s0);
+    const size_t esz = DT == DType::BF16 ? 2 : 4;
+    const void* kseq = static_cast<const char*>(k) + (int64_t)t * k_seq_stride * esz;
+    const float m = block_mean_rows<DT>(kseq, nfull * B, nt, part);
+    if (tid < kD) pmean[tid] = m;
   }
   __syncthreads();
 

@@ -53,11 +53,15 @@ size_t route_ws(int T, int L, int H_I, int B) {
 
 size_t scores_part(int T, int L) { return align_up(sizeof(float) * (size_t)T * score_ld(L)); }
 
-// misa_topk_select: histograms, per-row state and boundary pairs of the selection
+// misa_topk_select / misa_token_scores' selection state: the candidate lists of the rows, their
+// cuts and the sample they come from (the per-row selection itself needs no workspace)
 size_t select_bytes(int T, int P) {
   if (T <= 0 || P <= 0) return 0;
-  return align_up(misa::topk_rows_ws(T, P));
+  return align_up(misa::list_state_bytes(T));
 }
+
+// Per-query bf16 caches take the candidate-list top-k: sampled cut, lists appended by the scorer.
+bool list_path(int dtype, int64_t k_seq_stride) { return dtype == MISA_BF16 && k_seq_stride != 0; }
 
 // misa_score_topk / dsa_dense_topk: [scores][selection]
 size_t scores_ws(int T, int L) {
@@ -221,16 +225,18 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
   if (!scores) return MISA_ERR_INVALID_ARG;
   if (select_ws && (select_ws_bytes < select_bytes(T, L) || !aligned(select_ws))) return MISA_ERR_WORKSPACE;
   const cudaStream_t s = as_stream(stream);
+  const int m = heads ? h : H_I;
   if (!select_ws) {
-    misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, heads ? h : H_I, nullptr, 0,
-                        scores, ld_scores, nullptr, s);
+    misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0, scores,
+                        ld_scores, nullptr, s);
     return launch_status();
   }
-  misa::topk_rows_prepare(select_ws, T, s);
-  const misa::TopkFuse fuse = misa::topk_rows_fuse(select_ws, T, select_topk);
-  const bool ready = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I,
-                                         heads ? h : H_I, nullptr, 0, scores, ld_scores, &fuse, s);
-  if (!ready) misa::launch_topk_level0(scores, ld_scores, nullptr, 0, n, T, L, select_topk, select_ws, s);
+  const misa::ListState lst = misa::list_state(select_ws, T);
+  if (list_path(dtype, k_seq_stride)) misa::launch_list_cut(q, w, k, k_seq_stride, n, heads, T, L, H_I, m, select_topk,
+                                                            lst, s);
+  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0,
+                                          scores, ld_scores, list_path(dtype, k_seq_stride) ? &lst : nullptr, s);
+  if (!listed) misa::mark_no_lists(lst, T, s);
   return launch_status();
 }
 
@@ -241,7 +247,8 @@ misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32
   if (T == 0) return MISA_OK;
   if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < select_bytes(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
-  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws, ws_prepared != 0, idx, score_opt,
+  const misa::ListState lst = misa::list_state(ws, T);
+  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws_prepared ? &lst : nullptr, idx, score_opt,
                          as_stream(stream));
   return launch_status();
 }
@@ -266,9 +273,13 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
     ld = score_ld(L);
     p += scores_part(T, L);
   }
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld, nullptr,
-                      as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, false, idx, score_opt, as_stream(stream));
+  const cudaStream_t s = as_stream(stream);
+  const misa::ListState lst = misa::list_state(p, T);
+  const bool lp = list_path(dtype, k_seq_stride);
+  if (lp) misa::launch_list_cut(q, w, k, k_seq_stride, n, heads, T, L, H_I, h, topk, lst, s);
+  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0,
+                                          buf, ld, lp ? &lst : nullptr, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);
   return launch_status();
 }
 
@@ -283,10 +294,9 @@ misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64
   if (!cand || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   float* F = static_cast<float*>(ws);
-  void* sel = static_cast<char*>(ws) + align_up(sizeof(float) * (size_t)T * kp);
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp, nullptr,
                       as_stream(stream));
-  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, false, idx, score_opt, as_stream(stream));
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, nullptr, idx, score_opt, as_stream(stream));
   return launch_status();
 }
 
@@ -302,10 +312,13 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   char* p = static_cast<char*>(ws);
   float* buf = reinterpret_cast<float*>(p);
   const int64_t ld = score_ld(L);
-  void* sel = p + scores_part(T, L);
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld,
-                      nullptr, as_stream(stream));
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, sel, false, idx, score_opt, as_stream(stream));
+  const misa::ListState lst = misa::list_state(p + scores_part(T, L), T);
+  const cudaStream_t s = as_stream(stream);
+  const bool lp = list_path(dtype, k_seq_stride);
+  if (lp) misa::launch_list_cut(q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, topk, lst, s);
+  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr,
+                                          0, buf, ld, lp ? &lst : nullptr, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);
   return launch_status();
 }
 
@@ -345,10 +358,10 @@ misa_status misa_block_filter_topk(const void* q, const float* w, const void* k,
   const cudaStream_t s = as_stream(stream);
   misa::launch_block_scores(to_dtype(dtype), q, w, k, k_seq_stride, kbar, kbar_seq_stride, n, heads, T, L, H_I, B,
                             h, S, ldS, Mt, s);
-  misa::launch_topk_rows(S, ldS, nullptr, 0, Mt, T, M, m, p, false, blocks, nullptr, s);
+  misa::launch_topk_rows(S, ldS, nullptr, 0, Mt, T, M, m, nullptr, blocks, nullptr, s);
   misa::launch_expand_blocks(blocks, m, n, T, L, B, rows, s);
   misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, P, F, P, nullptr, s);
-  misa::launch_topk_rows(F, P, rows, P, n, T, L, topk, p, false, idx, score_opt, s);
+  misa::launch_topk_rows(F, P, rows, P, n, T, L, topk, nullptr, idx, score_opt, s);
   return launch_status();
 }
 
@@ -429,7 +442,7 @@ misa_status misa_score_topk_paged(const void* q, const float* w, const void* poo
   misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, nullptr, L, rows, n_phys, s);
   misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, heads, T, pool_rows, H_I, h, rows, L, buf, ld, nullptr,
                       s);
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, p, false, idx, score_opt, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, nullptr, idx, score_opt, s);
   return launch_status();
 }
 
@@ -452,13 +465,12 @@ misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* po
   int32_t* n_phys = reinterpret_cast<int32_t*>(p);
   p += align_up(sizeof(int32_t) * (size_t)T);
   float* F = reinterpret_cast<float*>(p);
-  void* sel = p + align_up(sizeof(float) * (size_t)T * kp);
   const int pool_rows = (int)(num_pages * page_size);
   const cudaStream_t s = as_stream(stream);
   misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, cand, kp, rows, n_phys, s);
   misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, nullptr, T, pool_rows, H_I, H_I, rows, kp, F, kp,
                       nullptr, s);
-  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, sel, false, idx, score_opt, s);
+  misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, nullptr, idx, score_opt, s);
   return launch_status();
 }
 

@@ -35,6 +35,63 @@ __device__ __forceinline__ float relu(float x) { return fmaxf(x, 0.0f); }
 // Clamp a device-side prefix length to [0, L].
 __device__ __forceinline__ int clamp_len(int n, int L) { return n < 0 ? 0 : (n > L ? L : n); }
 
+// Pooled blocks of a prefix of nt keys that are read from the pooled-key cache: every block but
+// the last.  The last block, keys [kbar_blocks(nt, B) * B, nt) (full or partial), is averaged from
+// the keys by the kernel that needs it, so a decode loop pools a block once its prefix has moved
+// past it, and the newest key is always seen.
+__device__ __forceinline__ int kbar_blocks(int nt, int B) { return nt > 0 ? (nt - 1) / B : 0; }
+
+// Mean of key rows [s0, s1) of one cache ([*, 128], bf16 or fp32), all 256 threads of the block:
+// every thread owns one 16-byte column chunk of a row group and issues the loads of up to 128 rows
+// at once.  part: shared scratch of 16 x 128 floats.  Returns the mean of column threadIdx.x in
+// threads 0..127 (IEEE division by the count); every thread must call it (it synchronises).
+template <DType DT>
+__device__ __forceinline__ float block_mean_rows(const void* kseq, int s0, int s1, float* part) {
+  constexpr int EPC = DT == DType::BF16 ? 8 : 4;  // elements per 16-byte chunk
+  constexpr int CPR = kD / EPC;                   // chunks per row
+  constexpr int RG = 256 / CPR;                   // row groups
+  constexpr int IT = 128 / RG;                    // rows a thread loads per batch
+  const int cc = threadIdx.x % CPR, rg = threadIdx.x / CPR;
+  const uint4* base = reinterpret_cast<const uint4*>(kseq);
+  float acc[EPC];
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) acc[e] = 0.f;
+  for (int s = s0 + rg; s < s1; s += RG * IT) {
+    uint4 x[IT];
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      const int r = s + i * RG;
+      x[i] = r < s1 ? __ldg(base + (int64_t)r * CPR + cc) : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int i = 0; i < IT; ++i) {
+      const uint32_t u[4] = {x[i].x, x[i].y, x[i].z, x[i].w};
+      if (DT == DType::BF16) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          acc[2 * e] += __uint_as_float(u[e] << 16);
+          acc[2 * e + 1] += __uint_as_float(u[e] & 0xffff0000u);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] += __uint_as_float(u[e]);
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < EPC; ++e) part[rg * kD + cc * EPC + e] = acc[e];
+  __syncthreads();
+  float mean = 0.f;
+  if (threadIdx.x < kD) {
+    float sum = 0.f;
+#pragma unroll
+    for (int g = 0; g < RG; ++g) sum += part[g * kD + threadIdx.x];
+    mean = sum / (float)(s1 - s0);
+  }
+  __syncthreads();  // part may be reused right after
+  return mean;
+}
+
 // Exclusive scan over the threads of a block (blockDim.x a multiple of 32, at most 1024).
 // `warp_tot` is shared scratch of 32 words.  Returns the exclusive prefix; *total gets the sum.
 __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot,

@@ -6,6 +6,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "select.cuh"
 
 namespace misa {
 
@@ -13,18 +14,19 @@ namespace misa {
 void launch_pool(DType dt, const void* k, int64_t k_seq_stride, int n_seq, int L, int B,
                  float* kbar, int64_t kbar_seq_stride, int b0, int b1, cudaStream_t s);
 
-// Router: partial-block means, per-chunk affinities, then sum, weight and top-h.
+// Router: last-block means, per-chunk affinities, then sum, weight and top-h.
 int route_chunks(int L, int B);  // chunks of kRouteTile blocks per query (upper bound)
-// kbar_parts: [3][ceil(L/B)][128] bf16 scratch for the tensor-core router (shared cache).
-// pm_in: [T][128] means of each query's partial last block computed beforehand (paged caches),
-// or nullptr to average them from k.
+// Blocks below kbar_blocks(n_t, B) are read from kbar, the last block of each prefix is averaged
+// from the keys.  kbar_parts: [3][ceil(L/B)][128] bf16 scratch for the tensor-core router (shared
+// cache).  pm_in: [T][128] means of each query's last block computed beforehand (paged caches), or
+// nullptr to average them from k.
 void launch_route(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                   const float* kbar, int64_t kbar_seq_stride, const int32_t* n, int T, int L,
                   int H_I, int B, int h, int32_t* heads, float* r_opt, float* pm, float* partial,
                   uint32_t* done, __nv_bfloat16* kbar_parts, const float* pm_in, cudaStream_t s);
 
 // Router on the tensor cores for queries that share one bf16 cache and its pooled keys: per-tile
-// sums over full blocks into Sp [T][nch][H_I], then route_finish.  False (nothing launched) when
+// sums over the blocks below kbar_blocks(n_t, B) into Sp [T][nch][H_I], then route_finish.  False (nothing launched) when
 // the shapes do not suit it (H_I must divide 128).
 constexpr int kRouteTcMinQueries = 64;
 bool launch_route_tc(const void* q, const float* w, const void* k, const float* kbar, const int32_t* n, int T,
@@ -35,20 +37,36 @@ void launch_route_finish(const __nv_bfloat16* q, const float* w, const __nv_bflo
                          int L, int H_I, int B, int h, const float* Sp, int nch, int tile, int32_t* heads,
                          float* r_opt, cudaStream_t s);
 
-// Level-0 selection state the decode scoring kernel can build while it scores (select.cuh):
-// hist [T][4096] and rec [T][8], both zeroed beforehand (topk_rows_prepare).
-struct TopkFuse {
-  uint32_t* hist;
-  uint32_t* rec;
-  int topk;
+// Candidate lists of a top-k over per-query caches, built while the scores are written (select.cuh
+// holds the sizes): a cut per query from a sample of its keys scored beforehand, then every score
+// at or above the cut is appended as (order key, token) to the query's list.
+struct ListState {
+  uint32_t* cnt;     // [T] entries appended (also past cap); kNoList: no list for this row
+  float* tau;        // [T] cut: -inf takes every entry, +inf none (the row goes the exact way)
+  uint32_t* arrive;  // [T] sample CTAs done (zeroed before the sample kernel)
+  float* sample;     // [T][kSampleRuns * kSampleRunLen] sample scores
+  uint2* list;       // [T][cap]
+  int cap;
 };
+size_t list_state_bytes(int T);
+ListState list_state(void* ws, int T);
+// cnt = kNoList for every row (scores written without lists).
+void mark_no_lists(const ListState& l, int T, cudaStream_t s);
+
+// The cut of every query for a top-topk of its routed (heads) or dense (heads == nullptr) scores
+// over one bf16 cache per query: scores kSampleRuns runs of kSampleRunLen keys spread over the
+// prefix, sets tau and zeroes cnt.  Prefixes of at most cap keys take every entry.
+void launch_list_cut(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                     const int32_t* heads, int T, int L, int H_I, int h, int topk, const ListState& l,
+                     cudaStream_t s);
 
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
-// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].  Returns true if it
-// also filled *fuse (only the persistent bf16 kernel does).
+// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].  With lst (bf16, one
+// cache per query, no gather: the persistent kernel) every score at or above lst->tau[t] is also
+// appended to the query's list; returns whether it was.
 bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
-                   const int32_t* rows, int P, float* out, int64_t ld, const TopkFuse* fuse, cudaStream_t s);
+                   const int32_t* rows, int P, float* out, int64_t ld, const ListState* lst, cudaStream_t s);
 
 // Tensor-core scoring for queries sharing one bf16 key cache (k_seq_stride 0, no gather).  Returns
 // false without launching when the inputs do not suit it (alignment, no TMA encoder).
@@ -59,19 +77,11 @@ int read_and_clear_tc_status();
 int read_and_clear_route_tc_status();
 
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
-// or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t)).  ws holds
-// topk_rows_ws(T, P or L) bytes, 256-byte aligned; hist_ready: the scoring kernel already filled
-// the level-0 state in ws (the partition/resolve kernels then select); otherwise one CTA per row
-// selects.  Output order within a row is not specified.
-size_t topk_rows_ws(int T, int P);
-void topk_rows_prepare(void* ws, int T, cudaStream_t s);
-TopkFuse topk_rows_fuse(void* ws, int T, int topk);
+// or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t); P <= 16384).  lst: the
+// candidate lists launch_scores appended for these rows (or nullptr).  One CTA per row, no
+// workspace.  Output order within a row is not specified.
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
-                      int L, int topk, void* ws, bool hist_ready, int32_t* idx, float* score_opt,
-                      cudaStream_t s);
-// Only the level-0 state (prepare + histogram pass), for scores written without it.
-void launch_topk_level0(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
-                        int L, int topk, void* ws, cudaStream_t s);
+                      int L, int topk, const ListState* lst, int32_t* idx, float* score_opt, cudaStream_t s);
 
 // Top-k of short candidate lists in shared memory (no workspace): values F[t, P], ids cand[t, P].
 size_t topk_cand_smem(int P);
@@ -80,8 +90,8 @@ void launch_topk_cand(const float* F, const int32_t* cand, const int32_t* n, int
 
 // Token-axis block filter composed with MISA (block_filter.cu).  Block scores of every query with
 // its routed heads: S[t, b] = sum_{j in heads[t]} w[t, j] * max(0, q[t, j] . kbar_b) for
-// b < M_t = ceil(n_t / B), where full blocks come from kbar and a partial last block is averaged
-// from k; Mt[t] receives M_t.  Entries b >= M_t are not written.
+// b < M_t = ceil(n_t / B), where blocks below kbar_blocks(n_t, B) come from kbar and the last block
+// is averaged from k; Mt[t] receives M_t.  Entries b >= M_t are not written.
 void launch_block_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                          const float* kbar, int64_t kbar_seq_stride, const int32_t* n, const int32_t* heads, int T,
                          int L, int H_I, int B, int h, float* S, int64_t ldS, int32_t* Mt, cudaStream_t s);
@@ -98,7 +108,7 @@ void launch_paged_rows(const int32_t* table, int64_t max_pages, int64_t num_page
 void launch_pool_paged(DType dt, const void* pool, int64_t num_pages, int page_size, const int32_t* table,
                        int64_t max_pages, int n_seq, int L, int B, float* kbar, int64_t kbar_seq_stride, int b0,
                        int b1, cudaStream_t s);
-// pm[t] = mean of the partial last block of query t's prefix (untouched when n_t is a multiple of B).
+// pm[t] = mean of the last block of query t's prefix (full or partial; untouched for an empty prefix).
 void launch_partial_mean_paged(DType dt, const void* pool, int64_t num_pages, int page_size, const int32_t* table,
                                int64_t max_pages, const int32_t* n, int T, int L, int B, float* pm, cudaStream_t s);
 

@@ -91,7 +91,8 @@ __global__ void __launch_bounds__(1024) pool_paged_kernel(const void* __restrict
     kbar[(int64_t)seq * kbar_seq_stride + (int64_t)b * kD + threadIdx.x] = part[0][threadIdx.x] / (float)(s1 - s0);
 }
 
-// pm[t] = mean of logical keys [floor(n_t/B) B, n_t) when n_t is not a multiple of B (256 threads).
+// pm[t] = mean of the last block of query t's prefix, logical keys [kbar_blocks(n_t, B) B, n_t)
+// (full or partial; untouched for an empty prefix), 256 threads.
 template <DType DT>
 __global__ void __launch_bounds__(256) partial_mean_paged_kernel(const void* __restrict__ pool, int64_t num_pages,
                                                                  int page_size, const int32_t* __restrict__ table,
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(256) partial_mean_paged_kernel(const void* __r
   __shared__ float part[4][kD];
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
-  const int c = nt % B;
+  const int c = nt - kbar_blocks(nt, B) * B;
   if (c == 0) return;
   paged_sum<DT, 4>(pool, table, max_pages, num_pages, page_size, t, nt - c, nt, part);
   if (threadIdx.x < kD) pm[(int64_t)t * kD + threadIdx.x] = part[0][threadIdx.x] / (float)c;

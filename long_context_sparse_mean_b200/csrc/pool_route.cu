@@ -7,9 +7,12 @@
 // heads are routed.  Aggregation used here: r_{t,j} = w_{t,j} * sum_b max(0, q_{t,j} . kbar_b).
 //
 // Data layout: keys [L, 128] (bf16 or fp32) per cache, pooled keys kbar [M, 128] fp32 per cache.
+// Every router path reads the pooled keys of all blocks of a prefix but the last from kbar and
+// averages the last block (full or partial) from the keys, so the newest key is always seen and a
+// decode loop pools a block only once the prefix has moved past it.
 // bf16 queries: one kernel.  One CTA per (query, tile of 128 pooled blocks) multiplies the tile
 // with the query's H_I head vectors on the tensor cores (see route_affinity_mma_kernel); the CTA
-// whose tile holds a partial last block averages that block's keys itself; per-tile sums go to
+// whose tile holds the last block averages that block's keys itself; per-tile sums go to
 // workspace and the query's last tile to finish adds them in tile order (deterministic), applies
 // w and picks the top-h heads with warp shuffles.
 // fp32 queries: CUDA cores, one CTA per (query, tile of 64 blocks) with a 4-head x 4-block
@@ -23,36 +26,6 @@
 namespace misa {
 
 namespace {
-
-// Sum of key rows [s0, s1) of one cache, 256 threads: 4 row groups x 64 column pairs.
-// Returns, in threads 0..127, the mean of column threadIdx.x (IEEE division by the count).
-template <DType DT>
-__device__ __forceinline__ float block_mean_256(const void* kseq, int s0, int s1, float (*part)[kD]) {
-  const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
-  float a0 = 0.f, a1 = 0.f;
-#pragma unroll 8
-  for (int s = s0 + rg; s < s1; s += 4) {
-    if (DT == DType::BF16) {
-      const uint32_t x = reinterpret_cast<const uint32_t*>(kseq)[(int64_t)s * (kD / 2) + cp];
-      a0 += bf16_lo(x);
-      a1 += bf16_hi(x);
-    } else {
-      const float2 x = reinterpret_cast<const float2*>(kseq)[(int64_t)s * (kD / 2) + cp];
-      a0 += x.x;
-      a1 += x.y;
-    }
-  }
-  part[rg][2 * cp] = a0;
-  part[rg][2 * cp + 1] = a1;
-  __syncthreads();
-  float mean = 0.f;
-  if (threadIdx.x < kD) {
-    const int i = threadIdx.x;
-    const float sum = ((part[0][i] + part[1][i]) + part[2][i]) + part[3][i];
-    mean = sum / (float)(s1 - s0);
-  }
-  return mean;
-}
 
 // One CTA of 1024 threads per block: 16 row groups x 64 column pairs, so a 128-key block is read
 // with every load in flight at once.
@@ -90,19 +63,17 @@ __global__ void __launch_bounds__(1024) pool_kernel(const void* k, int64_t k_seq
   }
 }
 
-// Mean of the partial last block [floor(n_t/B)*B, n_t) of every query whose prefix is not a
-// multiple of B.
+// Mean of the last block [kbar_blocks(n_t, B) * B, n_t) of every query's prefix (full or partial).
 template <DType DT>
 __global__ void __launch_bounds__(256) partial_mean_kernel(const void* k, int64_t k_seq_stride,
                                                            const int32_t* n, int L, int B, float* pm) {
-  __shared__ float part[4][kD];
+  __shared__ float part[16 * kD];
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
-  const int c = nt % B;
-  if (c == 0) return;
+  if (nt == 0) return;
   const size_t esz = DT == DType::BF16 ? 2 : 4;
   const void* kseq = static_cast<const char*>(k) + (int64_t)t * k_seq_stride * esz;
-  const float m = block_mean_256<DT>(kseq, nt - c, nt, part);
+  const float m = block_mean_rows<DT>(kseq, kbar_blocks(nt, B) * B, nt, part);
   if (threadIdx.x < kD) pm[(int64_t)t * kD + threadIdx.x] = m;
 }
 
@@ -116,7 +87,7 @@ __global__ void __launch_bounds__(512) route_affinity_kernel(const void* q, cons
   extern __shared__ __align__(16) float smem[];
   const int t = blockIdx.y, c = blockIdx.x;
   const int nt = clamp_len(n[t], L);
-  const int nfull = nt / B, Mt = (nt + B - 1) / B;
+  const int nfull = kbar_blocks(nt, B), Mt = (nt + B - 1) / B;  // block nfull (< Mt) is the last
   const int bb = c * kRouteTile;
   if (bb >= Mt) return;
   const int QS = H_I + 4, KS = kRouteTile + 4;
@@ -139,7 +110,7 @@ __global__ void __launch_bounds__(512) route_affinity_kernel(const void* q, cons
     const int bl = e / kD, dd = e % kD, b = bb + bl;
     float v = 0.f;
     if (b < nfull) v = kb[(int64_t)b * kD + dd];
-    else if (b < Mt) v = pm[(int64_t)t * kD + dd];  // the partial last block
+    else if (b < Mt) v = pm[(int64_t)t * kD + dd];  // the last block, averaged from the keys
     kT[dd * KS + bl] = v;
   }
   __syncthreads();
@@ -283,8 +254,12 @@ __device__ __forceinline__ void split3(float x, float& hi, float& mid, float& lo
 // split into three bf16 parts and the three products are accumulated in fp32, which keeps the
 // dot products at fp32 accuracy.  The pooled keys are loaded straight into A fragments (lane
 // (g, c) of a warp holds dims 16kk + 4c .. +3 of blocks g and g+8 at k-step kk, and the q
-// fragments staged in shared memory use the same dimension order).  Epilogue: relu, sum over the
-// tile's blocks per head (quad shuffles, then a fixed-order sum over the 8 warps).
+// fragments staged in shared memory use the same dimension order).  Blocks below
+// kbar_blocks(n_t, B) come from kbar; the last block of the prefix is averaged from the keys by
+// the CTA whose tile holds it (pm_in: averaged beforehand).  Every thread issues its pooled-key
+// loads first, then the q-fragment loads, then (one CTA per query) the last block's key loads,
+// so the three overlap.  Epilogue: relu, sum over the tile's blocks per head (quad shuffles, then
+// a fixed-order sum over the 8 warps).
 template <int NG>
 __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bfloat16* __restrict__ q,
                                                                  const float* __restrict__ w,
@@ -300,12 +275,12 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
   constexpr int H = NG * 8;
   __shared__ uint2 frag[NG][8][32];
   __shared__ float wsum[8][H];
-  __shared__ float part[4][kD];
-  __shared__ __align__(16) float pms[kD];  // mean of the partial last block
+  __shared__ float part[16 * kD];
+  __shared__ __align__(16) float pms[kD];  // mean of the last block
   __shared__ int last;
   const int t = blockIdx.y, c0 = blockIdx.x;
   const int nt = clamp_len(n[t], L);
-  const int nfull = nt / B, Mt = (nt + B - 1) / B;
+  const int nk = kbar_blocks(nt, B), Mt = (nt + B - 1) / B;
   const int nc = (Mt + kRouteMmaTile - 1) / kRouteMmaTile;
   const int bb = c0 * kRouteMmaTile;
   if (bb >= Mt) {
@@ -314,15 +289,20 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
                         r_opt ? r_opt + (int64_t)t * H : nullptr);
     return;
   }
-  if (nfull < Mt && nfull >= bb && nfull < bb + kRouteMmaTile) {  // this tile holds the partial block
-    if (pm_in) {  // averaged beforehand (paged caches)
-      if (threadIdx.x < kD) pms[threadIdx.x] = pm_in[(int64_t)t * kD + threadIdx.x];
-    } else {
-      const float m = block_mean_256<DType::BF16>(k + (int64_t)t * k_seq_stride, nfull * B, nt, part);
-      if (threadIdx.x < kD) pms[threadIdx.x] = m;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  const int ba = bb + warp * 16 + g, bq = ba + 8;
+  const float* kb = kbar + (int64_t)t * kbar_seq_stride;
+  float4 XA[8], XB[8];  // the warp's two pooled-key rows, all loads in flight at once
+  {
+    const float* rowa = ba < nk ? kb + (int64_t)ba * kD : nullptr;
+    const float* rowb = bq < nk ? kb + (int64_t)bq * kD : nullptr;
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      XA[kk] = rowa ? __ldg(reinterpret_cast<const float4*>(rowa + 16 * kk + 4 * c)) : make_float4(0, 0, 0, 0);
+      XB[kk] = rowb ? __ldg(reinterpret_cast<const float4*>(rowb + 16 * kk + 4 * c)) : make_float4(0, 0, 0, 0);
     }
   }
-  {  // every thread issues its fragment loads together (256 threads)
+  {  // q fragments: every thread issues its loads together (256 threads)
     constexpr int kPer = (NG * 8 * 32 + 255) / 256;
     uint2 v[kPer];
 #pragma unroll
@@ -330,8 +310,8 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
       const int e = (int)threadIdx.x + 256 * i;
       if (e < NG * 8 * 32) {
         const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
-        const int g = ln >> 2, c = ln & 3;
-        v[i] = *reinterpret_cast<const uint2*>(q + ((int64_t)t * H + ng * 8 + g) * kD + 16 * kk + 4 * c);
+        const int gg = ln >> 2, cc = ln & 3;
+        v[i] = __ldg(reinterpret_cast<const uint2*>(q + ((int64_t)t * H + ng * 8 + gg) * kD + 16 * kk + 4 * cc));
       }
     }
 #pragma unroll
@@ -340,21 +320,26 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
       if (e < NG * 8 * 32) frag[e >> 8][(e >> 5) & 7][e & 31] = v[i];
     }
   }
+  if (nk >= bb && nk < bb + kRouteMmaTile) {  // this tile holds the last block
+    if (pm_in) {  // averaged beforehand (paged caches)
+      if (threadIdx.x < kD) pms[threadIdx.x] = pm_in[(int64_t)t * kD + threadIdx.x];
+    } else {
+      const float m = block_mean_rows<DType::BF16>(k + (int64_t)t * k_seq_stride, nk * B, nt, part);
+      if (threadIdx.x < kD) pms[threadIdx.x] = m;
+    }
+  }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  const int ba = bb + warp * 16 + g, bq = ba + 8;
-  const float* kb = kbar + (int64_t)t * kbar_seq_stride;
-  const float* rowa = ba < nfull ? kb + (int64_t)ba * kD : (ba < Mt ? pms : nullptr);
-  const float* rowb = bq < nfull ? kb + (int64_t)bq * kD : (bq < Mt ? pms : nullptr);
+  if (ba == nk) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) XA[kk] = *reinterpret_cast<const float4*>(pms + 16 * kk + 4 * c);
+  }
+  if (bq == nk) {
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) XB[kk] = *reinterpret_cast<const float4*>(pms + 16 * kk + 4 * c);
+  }
   float acc[NG][4];
 #pragma unroll
   for (int ng = 0; ng < NG; ++ng) acc[ng][0] = acc[ng][1] = acc[ng][2] = acc[ng][3] = 0.f;
-  float4 XA[8], XB[8];  // all loads of the warp's two pooled-key rows in flight at once
-#pragma unroll
-  for (int kk = 0; kk < 8; ++kk) {
-    XA[kk] = rowa ? *reinterpret_cast<const float4*>(rowa + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
-    XB[kk] = rowb ? *reinterpret_cast<const float4*>(rowb + 16 * kk + 4 * c) : make_float4(0, 0, 0, 0);
-  }
 #pragma unroll
   for (int kk = 0; kk < 8; ++kk) {
     const float4 xa = XA[kk], xb = XB[kk];
@@ -425,10 +410,10 @@ __global__ void __launch_bounds__(256) kbar_split_kernel(const float* __restrict
   }
 }
 
-// One CTA per query, after the tensor-core router's per-tile sums Sp[t][tile][j] over full pooled
-// blocks: adds max(0, q_{t,j} . mean of the partial last block) (keys [floor(n_t/B) B, n_t),
-// averaged here), then r_j = w_j * total and the top-h heads.  The q rows and the per-tile sums
-// are requested before the mean is formed, so their loads overlap it.
+// One CTA per query, after the tensor-core router's per-tile sums Sp[t][tile][j] over the pooled
+// blocks below kbar_blocks(n_t, B): adds max(0, q_{t,j} . mean of the last block) (keys
+// [kbar_blocks(n_t, B) B, n_t), averaged here), then r_j = w_j * total and the top-h heads.  The q
+// rows and the per-tile sums are requested before the mean is formed, so their loads overlap it.
 __global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* __restrict__ q,
                                                            const float* __restrict__ w,
                                                            const __nv_bfloat16* __restrict__ k,
@@ -437,13 +422,13 @@ __global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* 
                                                            int tile, int32_t* __restrict__ heads,
                                                            float* __restrict__ r_opt) {
   constexpr int kHeadsPerWarp = kMaxHeads / 8;
-  __shared__ float part[4][kD];
+  __shared__ float part[16 * kD];
   __shared__ __align__(16) float pm[kD];
   __shared__ float pmd[kMaxHeads];
   __shared__ float tot[kMaxHeads];
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
-  const int nf = nt / B, c = nt % B;
+  const int nf = kbar_blocks(nt, B), c = nt - nf * B;  // c keys in the last block (0: empty prefix)
   const int ntiles = (nf + tile - 1) / tile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint2 qv[kHeadsPerWarp];  // lane's 4 dims of this warp's heads warp, warp + 8, ...
@@ -459,7 +444,7 @@ __global__ void __launch_bounds__(256) route_finish_kernel(const __nv_bfloat16* 
     for (int i = 0; i < ntiles; ++i) spsum += __ldcg(Sp + ((int64_t)t * nch + i) * H_I + threadIdx.x);
   }
   if (c > 0) {
-    const float m = block_mean_256<DType::BF16>(k, nt - c, nt, part);
+    const float m = block_mean_rows<DType::BF16>(k, nt - c, nt, part);
     if (threadIdx.x < kD) pm[threadIdx.x] = m;
   }
   __syncthreads();

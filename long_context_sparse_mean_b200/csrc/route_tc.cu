@@ -6,8 +6,9 @@
 // over the mean-pooled keys of its prefix, r_{t,j} = w_{t,j} sum_{b < M_t} max(0, q_{t,j} . kbar_b).
 //
 // This kernel computes, per tile of 256 pooled blocks, Sp[t][tile][j] = the sum over the tile's
-// full blocks b < floor(n_t / B) of max(0, q_{t,j} . kbar_b); route_finish (pool_route.cu) adds
-// the partial last block, w, and picks the top-h.  As a contraction: A = the H_I query-head rows
+// blocks b < kbar_blocks(n_t, B) (every block of the prefix but the last) of
+// max(0, q_{t,j} . kbar_b); route_finish (pool_route.cu) adds the last block, averaged from the
+// keys, applies w and picks the top-h.  As a contraction: A = the H_I query-head rows
 // of 128 / H_I consecutive queries [128 rows x 128 dims], contiguous in q and loaded by TMA;
 // B = 256 pooled keys in three bf16 parts (kbar = hi + mid + lo to fp32 accuracy, so the dot
 // products keep the accuracy of fp32 pooled keys) [256 x 128] each; D = A (hi + mid + lo)^T
@@ -90,7 +91,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int QR = kRows / H_I;  // queries per block
   const int NB = (T + QR - 1) / QR;
 
-  tc::block_tile_prefix(NB, QR, T, kBlocks, [&](int t) { return clamp_len(__ldg(n + t), L) / B; }, pre, warp_tot);
+  tc::block_tile_prefix(NB, QR, T, kBlocks, [&](int t) { return kbar_blocks(clamp_len(__ldg(n + t), L), B); }, pre,
+                        warp_tot);
   const uint64_t W = pre[NB];
   const uint32_t a = (uint32_t)(W * blockIdx.x / gridDim.x);
   const uint32_t e = (uint32_t)(W * (blockIdx.x + 1) / gridDim.x);
@@ -136,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     while (ok && it.next(blk, lo, hi)) {
       const int t = blk * QR + qi;
       const bool real = qi < QR && t < T;
-      const int nf = real ? clamp_len(__ldg(n + t), L) / B : 0;
+      const int nf = real ? kbar_blocks(clamp_len(__ldg(n + t), L), B) : 0;
       for (uint32_t tile = lo; tile < hi; ++tile, ++i) {
         const int ab = i & 1;
         if (!tc::mbar_wait(accfull + 8 * ab, (i >> 1) & 1, abort, kWaitLimitNs)) {

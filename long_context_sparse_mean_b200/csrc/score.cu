@@ -20,9 +20,10 @@
 //       32 x 131072 keys: 178 us against 185 us for the grid kernel; an added bulk L2 prefetch
 //       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
 //       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
-//       On request it also builds each row's level-0 selection histogram while it writes the
-//       scores (topk.cu); the default selection reads the scores instead, which measured faster
-//       over a whole decode step (the scorer alone is 13 us faster without the histogram).
+//       For a top-k of the scores it can also append every score at or above a per-query cut to
+//       the query's candidate list while it writes the scores (one ballot and at most one atomic
+//       per warp and tile), so the selection ranks a list of about 1.4 k entries instead of
+//       sweeping the row; list_cut_kernel places the cut beforehand from a sample of the keys.
 //   score_grid_kernel     one CTA per (query, chunk of positions): shared caches when the
 //       tensor-core kernel (score_tc.cu, which takes shared bf16 caches) cannot run, and more
 //       queries than the persistent schedule takes.
@@ -97,14 +98,11 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
                          const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                          const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
                          const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld,
-                         uint32_t* __restrict__ hist, uint32_t* __restrict__ rec, int topk) {
-  // dynamic: padded level-0 histogram [kHistPadded], then the flattened tile prefix [T + 1]
-  extern __shared__ uint32_t dyn[];
-  uint32_t* hsm = dyn;
-  int* tile_base = reinterpret_cast<int*>(dyn + kHistPadded);
+                         const float* __restrict__ tau, uint2* __restrict__ lists, uint32_t* __restrict__ lcnt,
+                         int cap) {
+  extern __shared__ int tile_base[];  // [T + 1] flattened tile prefix
   __shared__ HeadStage<NG> st;
   __shared__ uint32_t wtot[35];
-  __shared__ int last;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
 
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
@@ -118,8 +116,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     run += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
   }
   if (threadIdx.x == 0) tile_base[T] = (int)total;
-  if (hist)
-    for (int b = threadIdx.x; b < kHistPadded; b += kScoreThreads) hsm[b] = 0;
   __syncthreads();
   const int64_t tb = (int64_t)blockIdx.x * total / gridDim.x;
   const int64_t te = (int64_t)(blockIdx.x + 1) * total / gridDim.x;
@@ -139,6 +135,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const int nt = clamp_len(n[t], L);
     const int npos = GATHER ? P : nt;
     const int32_t* rt = GATHER ? rows + (int64_t)t * P : nullptr;
+    const float cut = lists ? __ldg(tau + t) : 0.f;
+    uint2* lt = lists ? lists + (int64_t)t * cap : nullptr;
 
     __syncthreads();  // the previous segment's fragments are no longer read
     stage_query<NG>(st, q, w, heads, h, H_I, t);
@@ -189,9 +187,19 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       const int r = row_of(j) + g;
       if (c == 0 && r < npos) ot[r] = slo;
       if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
-      if (hist) {  // count the key row's score; empty gathered slots are not counted
-        const bool cnt = (c == 0 && va) || (c == 1 && vb);
-        if (cnt) atomicAdd(&hsm[hpad((int)(order_key(c == 0 ? slo : shi) >> 20))], 1u);
+      if (!GATHER && lists) {
+        // the key rows of this tile whose score reaches the cut join the query's candidate list
+        const float v = c == 0 ? slo : shi;
+        const bool keep = (c == 0 ? va : (c == 1 && vb)) && v >= cut;
+        const unsigned m = __ballot_sync(0xffffffffu, keep);
+        if (m) {  // uniform across the warp
+          const int leader = __ffs(m) - 1;
+          uint32_t base = 0;
+          if (lane == leader) base = atomicAdd(lcnt + t, (uint32_t)__popc(m));
+          base = __shfl_sync(0xffffffffu, base, leader);
+          const uint32_t slot = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
+          if (keep && slot < (uint32_t)cap) lt[slot] = make_uint2(order_key(v), (uint32_t)(c == 0 ? r : r + 8));
+        }
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -201,36 +209,81 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       va = na;
       vb = nb;
     }
-    if (hist) {
-      // add this segment's counts to the row's histogram; the CTA that completes the row's
-      // tiles turns it into the level-0 boundary of the selection
-      __syncthreads();
-      uint32_t* ht = hist + (int64_t)t * kHistBins;
-      for (int b = threadIdx.x; b < kHistBins; b += kScoreThreads) {
-        const uint32_t v = hsm[hpad(b)];
-        if (v) atomicAdd(ht + b, v);
-        hsm[hpad(b)] = 0;
-      }
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        // fences are cumulative: after the barrier, one fence orders the whole CTA's adds
-        __threadfence();
-        const uint32_t row_tiles = (uint32_t)(tile_base[t + 1] - tile_base[t]);
-        last = atomicAdd(rec + 8 * (int64_t)t, (uint32_t)ntile) + (uint32_t)ntile == row_tiles;
-      }
-      __syncthreads();
-      if (last) {
-        __threadfence();
-        const Bucket bk = level0_boundary<kScoreThreads>(ht, (uint32_t)topk, hsm, wtot);
-        if (threadIdx.x == 0) {
-          rec[8 * (int64_t)t + 2] = bk.prefix;
-          rec[8 * (int64_t)t + 3] = bk.need;
-        }
-        for (int b = threadIdx.x; b < kHistPadded; b += kScoreThreads) hsm[b] = 0;
-        __syncthreads();
-      }
-    }
     pos = seg_end;
+  }
+}
+
+// Sampled cut of each query's scores for a top-k (one bf16 cache per query): CTA cb of query t
+// scores the sample runs [16 cb, 16 cb + 16) (warp w: runs 16 cb + 2w and 16 cb + 2w + 1, one run
+// of 8 consecutive keys per half of its 16-row MMA group) with the query's head list into
+// l.sample; the query's last CTA to finish places the cut from all 2048 sample scores (the sample
+// rank that the row top-k would use) and zeroes the list count.  Rows of at most cap keys take
+// every entry (cut -inf); rows whose top-k the sample cannot place take none (cut +inf), so their
+// selection takes the exact path.
+constexpr int kCutCtas = kSampleRuns / 16;
+
+template <int NG>
+__global__ void __launch_bounds__(kScoreThreads)
+    list_cut_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                    const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
+                    const int32_t* __restrict__ heads, int h, int H_I, int L, int topk, ListState l) {
+  __shared__ union Smem {  // the head list while scoring, the cut's histogram after
+    HeadStage<NG> st;
+    uint32_t hist[kHistBins];
+  } sm_u;
+  HeadStage<NG>& st = sm_u.st;
+  uint32_t* hist = sm_u.hist;
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t mm[2];
+  __shared__ int last;
+  constexpr int ns = kSampleRuns * kSampleRunLen;
+  const int t = blockIdx.y, cb = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  const uint32_t rank = sample_rank(topk, nt);
+  if (nt <= l.cap || rank > (uint32_t)ns) {
+    if (cb == 0 && threadIdx.x == 0) {
+      l.tau[t] = nt <= l.cap ? -INFINITY : INFINITY;
+      l.cnt[t] = 0u;
+    }
+    return;
+  }
+  stage_query<NG>(st, q, w, heads, h, H_I, t);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  float wa[NG], wb[NG];
+#pragma unroll
+  for (int ng = 0; ng < NG; ++ng) {
+    wa[ng] = st.wsel[ng * 8 + 2 * c];
+    wb[ng] = st.wsel[ng * 8 + 2 * c + 1];
+  }
+  const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);  // >= 64: nt > cap
+  const int ra = 16 * cb + 2 * warp, rb = ra + 1;
+  const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
+  uint4 A[4], Bq[4];
+  load_rows(kt + ((int64_t)ra * seg + g) * kD, kt + ((int64_t)rb * seg + g) * kD, c, A, Bq);
+  float slo, shi;
+  score_rows<NG>(A, Bq, st.frag, wa, wb, lane, slo, shi);
+  float* sm = l.sample + (int64_t)t * ns;
+  if (c == 0) sm[ra * kSampleRunLen + g] = slo;
+  if (c == 1) sm[rb * kSampleRunLen + g] = shi;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(l.arrive + t, 1u) == (uint32_t)(kCutCtas - 1);
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  constexpr int per = ns / kScoreThreads;
+  uint32_t sk[per];
+#pragma unroll
+  for (int u = 0; u < per; ++u) sk[u] = order_key(__ldcg(sm + u * kScoreThreads + threadIdx.x));
+  if (threadIdx.x == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+  const float cut = sample_cut<per>(sk, rank, hist, mm, scratch);
+  if (threadIdx.x == 0) {
+    l.tau[t] = cut;
+    l.cnt[t] = 0u;
+    l.arrive[t] = 0u;
   }
 }
 
@@ -363,22 +416,23 @@ int num_sms() {
 template <int NG>
 void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const float* w, const void* k,
                  int64_t k_seq_stride, const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L,
-                 const int32_t* rows, int P, float* out, int64_t ld, const TopkFuse* fuse) {
+                 const int32_t* rows, int P, float* out, int64_t ld, const ListState* lst) {
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   if (persist) {
-    const size_t smem = sizeof(uint32_t) * ((size_t)kHistPadded + T + 1);
-    uint32_t* hist = fuse ? fuse->hist : nullptr;
-    uint32_t* rec = fuse ? fuse->rec : nullptr;
-    const int topk = fuse ? fuse->topk : 0;
+    const size_t smem = sizeof(int) * ((size_t)T + 1);
+    const float* tau = lst ? lst->tau : nullptr;
+    uint2* lists = lst ? lst->list : nullptr;
+    uint32_t* lcnt = lst ? lst->cnt : nullptr;
+    const int cap = lst ? lst->cap : 0;
     if (gather) {
       cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, hist, rec, topk);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, nullptr, nullptr, nullptr, 0);
     } else {
       cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, hist, rec, topk);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, tau, lists, lcnt, cap);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
@@ -391,11 +445,19 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
   }
 }
 
+template <int NG>
+void launch_cut(cudaStream_t s, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L, int topk, const ListState& l) {
+  list_cut_kernel<NG><<<dim3(kCutCtas, T), kScoreThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(q), w,
+                                                                  static_cast<const __nv_bfloat16*>(k), k_seq_stride,
+                                                                  n, heads, h, H_I, L, topk, l);
+}
+
 }  // namespace
 
 bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h, const int32_t* rows,
-                   int P, float* out, int64_t ld, const TopkFuse* fuse, cudaStream_t s) {
+                   int P, float* out, int64_t ld, const ListState* lst, cudaStream_t s) {
   if (T <= 0) return false;
   const int npos = rows ? P : L;
   if (npos <= 0) return false;
@@ -416,39 +478,72 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
           P, out, ld);
     }
     return false;
-  } else {
-    // one shared cache: tensor-core contraction over blocks of queries
-    if (!gather && k_seq_stride == 0 && launch_scores_tc(q, w, k, n, heads, T, L, H_I, h, out, ld, s)) return false;
-    const int m = heads ? h : H_I;
-    const int ng = (m + 7) / 8;
-    // persistent schedule for per-query caches and for gathered candidate lists
-    const bool persist = (gather || k_seq_stride != 0) && T <= kMaxPersistQueries;
-    switch (ng) {
+  }
+  // one shared cache: tensor-core contraction over blocks of queries
+  if (!gather && k_seq_stride == 0 && launch_scores_tc(q, w, k, n, heads, T, L, H_I, h, out, ld, s)) return false;
+  const int m = heads ? h : H_I;
+  const int ng = (m + 7) / 8;
+  // persistent schedule for per-query caches and for gathered candidate lists
+  const bool persist = (gather || k_seq_stride != 0) && T <= kMaxPersistQueries;
+  const ListState* l = persist && !gather ? lst : nullptr;
+  switch (ng) {
 #define MISA_NG_CASE(NGV)                                                                                  \
   case NGV:                                                                                                \
-    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld, fuse); \
+    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld, l); \
     break;
-      MISA_NG_CASE(1)
-      MISA_NG_CASE(2)
-      MISA_NG_CASE(3)
-      MISA_NG_CASE(4)
-      MISA_NG_CASE(5)
-      MISA_NG_CASE(6)
-      MISA_NG_CASE(7)
-      MISA_NG_CASE(8)
-      MISA_NG_CASE(9)
-      MISA_NG_CASE(10)
-      MISA_NG_CASE(11)
-      MISA_NG_CASE(12)
-      MISA_NG_CASE(13)
-      MISA_NG_CASE(14)
-      MISA_NG_CASE(15)
-      MISA_NG_CASE(16)
+    MISA_NG_CASE(1)
+    MISA_NG_CASE(2)
+    MISA_NG_CASE(3)
+    MISA_NG_CASE(4)
+    MISA_NG_CASE(5)
+    MISA_NG_CASE(6)
+    MISA_NG_CASE(7)
+    MISA_NG_CASE(8)
+    MISA_NG_CASE(9)
+    MISA_NG_CASE(10)
+    MISA_NG_CASE(11)
+    MISA_NG_CASE(12)
+    MISA_NG_CASE(13)
+    MISA_NG_CASE(14)
+    MISA_NG_CASE(15)
+    MISA_NG_CASE(16)
 #undef MISA_NG_CASE
-      default:
-        break;
-    }
-    return persist && fuse != nullptr;
+    default:
+      break;
+  }
+  return l != nullptr;
+}
+
+void launch_list_cut(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                     const int32_t* heads, int T, int L, int H_I, int h, int topk, const ListState& l,
+                     cudaStream_t s) {
+  if (T <= 0) return;
+  cudaMemsetAsync(l.arrive, 0, sizeof(uint32_t) * (size_t)T, s);
+  const int m = heads ? h : H_I;
+  switch ((m + 7) / 8) {
+#define MISA_CUT_CASE(NGV)                                                     \
+  case NGV:                                                                    \
+    launch_cut<NGV>(s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, topk, l); \
+    break;
+    MISA_CUT_CASE(1)
+    MISA_CUT_CASE(2)
+    MISA_CUT_CASE(3)
+    MISA_CUT_CASE(4)
+    MISA_CUT_CASE(5)
+    MISA_CUT_CASE(6)
+    MISA_CUT_CASE(7)
+    MISA_CUT_CASE(8)
+    MISA_CUT_CASE(9)
+    MISA_CUT_CASE(10)
+    MISA_CUT_CASE(11)
+    MISA_CUT_CASE(12)
+    MISA_CUT_CASE(13)
+    MISA_CUT_CASE(14)
+    MISA_CUT_CASE(15)
+    MISA_CUT_CASE(16)
+#undef MISA_CUT_CASE
+    default:
+      break;
   }
 }
 

@@ -15,6 +15,14 @@ namespace misa {
 
 constexpr int kHistBins = 4096;
 
+// Sampled cut of a long row: kSampleRuns evenly spaced runs of kSampleRunLen consecutive entries.
+constexpr int kSampleRuns = 256;
+constexpr int kSampleRunLen = 8;  // one 32-byte sector of fp32 scores
+// Candidate lists the decode scoring kernel appends (entries per query), and the count that marks
+// a row without one.
+constexpr int kListCap = 16384;
+constexpr uint32_t kNoList = 0xffffffffu;
+
 __device__ __forceinline__ int level_shift(int l) { return l == 0 ? 20 : (l == 1 ? 10 : 0); }
 __device__ __forceinline__ int level_bins(int l) { return l == 0 ? 4096 : 1024; }
 
@@ -112,9 +120,69 @@ __device__ __forceinline__ Bucket level0_boundary(const uint32_t* hist_t, uint32
   return bucket_search_padded(hp, need, scratch);
 }
 
+// Sample rank whose score cuts a row of np entries for a top-k: the expected number of samples
+// above the k-th entry plus three standard deviations and a margin.  Above
+// kSampleRuns * kSampleRunLen the sample cannot place the cut.
+__host__ __device__ __forceinline__ uint32_t sample_rank(int topk, int np) {
+  const float ns = (float)(kSampleRuns * kSampleRunLen);
+  const float mean = (float)topk * ns / (float)(np > 1 ? np : 1);
+  return (uint32_t)(mean + 3.f * sqrtf(mean) + 8.f);
+}
+
+// Smallest lo and largest hi over the block into mm[0] and mm[1], which hold 0xffffffff and 0 on
+// entry.  Every thread calls it; it synchronises before its shared atomics, the caller after.
+__device__ __forceinline__ void block_min_max(uint32_t lo, uint32_t hi, uint32_t* mm) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    lo = min(lo, __shfl_xor_sync(0xffffffffu, lo, o));
+    hi = max(hi, __shfl_xor_sync(0xffffffffu, hi, o));
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) {
+    atomicMin(&mm[0], lo);
+    atomicMax(&mm[1], hi);
+  }
+}
+
+// Cut from a sample of keys: the lower edge of the bin (4096 bins over the sample's key range) holding the rank-th largest sample key, so at
+// least `rank` sample keys are at or above the returned value.  PER keys per thread; hist: 4096
+// words of shared memory; mm: 2 words holding 0xffffffff and 0 on entry (and again on return);
+// scratch: 35 words.  Every thread calls it.
+template <int PER>
+__device__ __forceinline__ float sample_cut(const uint32_t (&sk)[PER], uint32_t rank, uint32_t* hist, uint32_t* mm,
+                                            uint32_t* scratch);
+
 __device__ __forceinline__ Bucket block_bucket(const uint32_t* hist, int lvl, uint32_t prefix, uint32_t need,
                                                uint32_t* scratch) {
   return block_bucket_bits(hist, level_bins(lvl), level_shift(lvl), prefix, need, scratch);
+}
+
+template <int PER>
+__device__ __forceinline__ float sample_cut(const uint32_t (&sk)[PER], uint32_t rank, uint32_t* hist, uint32_t* mm,
+                                            uint32_t* scratch) {
+  uint32_t slo = 0xffffffffu, shi = 0u;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) {
+    slo = min(slo, sk[u]);
+    shi = max(shi, sk[u]);
+  }
+  block_min_max(slo, shi, mm);
+  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  slo = mm[0];
+  const uint32_t srange = mm[1] - slo;
+  const int ssh = srange >= 4096u ? 32 - __clz(srange) - 12 : 0;
+#pragma unroll
+  for (int u = 0; u < PER; ++u) hist_add(hist, (sk[u] - slo) >> ssh, true);
+  __syncthreads();
+  const Bucket cut = block_bucket_bits(hist, kHistBins, ssh, 0u, rank, scratch);
+  if (threadIdx.x == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+  __syncthreads();
+  // keys >= slo + cut.prefix are the scores >= this value
+  return key_to_float(slo + cut.prefix);
 }
 
 // Radix select over m items given by acc.key(i) (0 = absent) and acc.id(i); acc.value(i) is the

@@ -61,23 +61,24 @@ def test_workspace_sizes(lib):
     # router: [T,128] partial-block means + [T, ceil(ceil(L/B)/64), H_I] tile sums + [T] counters
     # + [3, ceil(L/B), 128] bf16 parts of the pooled keys
     assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256 + 3 * 1024 * 128 * 2
-    # top-k select: [T, 4096] histogram, [T, 8] row state, [T, L] boundary (key, id) pairs
-    sel = _al(32 * (4096 + 8) * 4 + 32 * 131072 * 8)
-    assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel
+    # top-k select: candidate-list state per query: count, cut and arrival counter [T] each, the
+    # sample [T, 2048] and the list [T, 16384] (key, token) pairs, each piece 256-byte aligned
+    def sel(T):
+        return 3 * _al(T * 4) + _al(T * 2048 * 4) + _al(T * 16384 * 8)
+    assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel(32)
+    assert ws(4, 32, 7, 64, 0, 0, 2048, 0) == sel(32), "independent of the row length"
     # scoring + top-k: [T, ceil4(L)] scores in front of the select workspace
-    assert ws(1, 32, 131072, 64, 128, 8, 8192, 0) == 32 * 131072 * 4 + sel
-    assert ws(3, 32, 131072, 64, 0, 0, 2048, 0) == 32 * 131072 * 4 + sel
-    assert ws(1, 3, 1001, 64, 1, 8, 10, 0) == _al(3 * 1004 * 4) + _al(3 * 4104 * 4 + 3 * 1001 * 8)
-    # re-rank: [T, k'] dense scores + the select workspace over k' positions
-    assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + _al(32 * 4104 * 4 + 32 * 8192 * 8)
+    assert ws(1, 32, 131072, 64, 128, 8, 8192, 0) == 32 * 131072 * 4 + sel(32)
+    assert ws(3, 32, 131072, 64, 0, 0, 2048, 0) == 32 * 131072 * 4 + sel(32)
+    assert ws(1, 3, 1001, 64, 1, 8, 10, 0) == _al(3 * 1004 * 4) + sel(3)
+    # re-rank: [T, k'] dense scores + the select workspace
+    assert ws(2, 32, 0, 64, 0, 0, 2048, 8192) == 32 * 8192 * 4 + sel(32)
     assert ws(1, 0, 100, 64, 1, 8, 10, 0) == 0
     # block filter (m in the last slot): [T, ceil4(M)] block scores, [T] block counts, [T, m*B] token
-    # ids and [T, m*B] their scores, then the select workspace over max(M, m*B) positions
+    # ids and [T, m*B] their scores, then the select workspace
     P, M = 128 * 128, 1024
-    assert ws(5, 32, 131072, 64, 128, 8, 2048, 128) == (32 * M * 4 + 256 + 2 * 32 * P * 4 +
-                                                        _al(32 * 4104 * 4 + 32 * P * 8))
-    assert ws(5, 3, 1001, 64, 7, 8, 10, 5) == (_al(3 * 144 * 4) + 256 + 2 * _al(3 * 35 * 4) +
-                                               _al(3 * 4104 * 4 + 3 * 143 * 8))
+    assert ws(5, 32, 131072, 64, 128, 8, 2048, 128) == (32 * M * 4 + 256 + 2 * 32 * P * 4 + sel(32))
+    assert ws(5, 3, 1001, 64, 7, 8, 10, 5) == (_al(3 * 144 * 4) + 256 + 2 * _al(3 * 35 * 4) + sel(3))
     assert ws(5, 32, 131072, 64, 128, 8, 2048, 129) == 0  # m * B above the candidate-list limit
     assert ws(5, 32, 131072, 64, 128, 8, 2048, 0) == 0
 
