@@ -60,7 +60,8 @@ typedef enum {
   MISA_ERR_UNSUPPORTED = 2,
   MISA_ERR_WORKSPACE = 3,
   MISA_ERR_CUDA = 4,
-  MISA_ERR_DEVICE_TIMEOUT = 5
+  MISA_ERR_DEVICE_TIMEOUT = 5,
+  MISA_ERR_BAD_INDEX = 6
 } misa_status;
 
 typedef enum { MISA_BF16 = 0, MISA_F32 = 1 } misa_dtype;
@@ -131,14 +132,15 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
  *   select_ws, select_ws_bytes, select_topk : optional (NULL, 0, 0).  A workspace of
  *              misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes in which the call also
  *              prepares a top-select_topk selection of these scores; pass the same workspace to
- *              misa_topk_select with ws_prepared = 1.  For one bf16 cache per query it first
- *              scores a sample of each prefix (256 evenly spaced runs of 8 keys) to place a cut
- *              that at least select_topk scores reach with overwhelming likelihood, then appends
- *              every score at or above the cut to a candidate list of up to 16384 entries per
- *              query while it writes the scores; the selection ranks that list and takes an exact
- *              pass over the score row whenever the list cannot hold the answer (too few entries
- *              or too many), so the result never depends on the sample.  Other caches leave no
- *              list and the selection works from the scores alone.
+ *              misa_topk_select with ws_prepared = 1.  For one bf16 cache per query the scoring
+ *              kernel builds a candidate list of up to 16384 entries per query as it goes: every
+ *              run of a query's keys it scores keeps the entries at or above a cut placed on the
+ *              run's own scores (its share of select_topk, 1.5 times over) and raises the query's
+ *              cut key to that cut, so every score at or above the query's cut key is listed.  The
+ *              selection ranks those entries and takes an exact pass over the score row whenever
+ *              they cannot hold the answer (fewer than select_topk, or the list overflowed), so
+ *              the result never depends on how the cuts fell.  Other caches, and batches whose
+ *              lists would not fit, leave no list and the selection works from the scores alone.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -281,11 +283,36 @@ misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* po
  * shared-memory barriers; every wait on them is bounded (about one second).  A wait that runs
  * out makes the kernel stop early, leaving its outputs incomplete, and records the event in a
  * per-device status word.  This call waits for all work on the device to finish
- * (cudaDeviceSynchronize), then reads and clears that word.
- *   returns MISA_OK, MISA_ERR_DEVICE_TIMEOUT (some call since the last check stopped early), or
+ * (cudaDeviceSynchronize), then reads and clears that word (and, in the bounds-checked build,
+ * the counts of skipped out-of-range ids described below).
+ *   returns MISA_OK, MISA_ERR_DEVICE_TIMEOUT (some call since the last check stopped early),
+ *   MISA_ERR_BAD_INDEX (bounds-checked build: out-of-range ids were seen and skipped), or
  *   MISA_ERR_CUDA (the synchronisation or the read failed).
  */
 misa_status misa_device_check(void);
+
+/*
+ * Bounds-checked build.  libmisa_checked.so (python -m long_context_sparse_mean_b200.build
+ * --checked) is the same library compiled with MISA_CHECKED: every id that a kernel skips because
+ * it lies outside its range is also counted on the device, by kind:
+ *   out[0] routed head ids outside [0, H_I)            (scoring and block-filter calls)
+ *   out[1] candidate token ids outside [0, n_t), other than the empty marker -1 (re-rank calls,
+ *          paged or not; the header's "empty slot" rule still applies: they are skipped)
+ *   out[2] page-table entries inside a prefix outside [0, num_pages) (paged calls; per key row
+ *          read through the entry)
+ * The counts are occurrences seen, not distinct ids.  In both builds such ids are never
+ * dereferenced.  misa_device_check returns MISA_ERR_BAD_INDEX (after MISA_ERR_DEVICE_TIMEOUT,
+ * which takes precedence) when any count is nonzero, and clears them.
+ */
+/* 1 for the bounds-checked build, 0 otherwise. */
+int misa_checked_build(void);
+
+/*
+ * Waits for the device (cudaDeviceSynchronize), then writes the counts of skipped out-of-range
+ * ids since the last read into out[3] (kinds as above; zeros in the normal build) and clears them.
+ * Returns MISA_OK, MISA_ERR_INVALID_ARG (out is NULL) or MISA_ERR_CUDA.
+ */
+misa_status misa_bad_index_counts(unsigned int* out);
 
 /*
  * Capacity, in floats, of the fixed scratch array used by misa_hier_rerank_static

@@ -25,9 +25,10 @@ from typing import Optional
 import torch
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "libmisa.so")
+# MISA_LIBRARY=checked selects the bounds-checked build (libmisa_checked.so, misa.h).
+LIB_PATH = os.path.join(PKG, "libmisa_checked.so" if os.environ.get("MISA_LIBRARY") == "checked" else "libmisa.so")
 
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_BAD_INDEX = range(7)
 BF16, F32 = 0, 1
 (OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT, OP_BLOCK_FILTER, OP_ROUTE_PAGED,
  OP_SCORE_TOPK_PAGED, OP_RERANK_PAGED) = range(9)
@@ -48,6 +49,8 @@ def _setup(lib):
     sigs = {
         "misa_version": ([], i32),
         "misa_device_check": ([], i32),
+        "misa_checked_build": ([], i32),
+        "misa_bad_index_counts": ([P], i32),
         "misa_status_str": ([i32], ctypes.c_char_p),
         "misa_workspace_bytes": ([i32, i32, i32, i32, i32, i32, i32, i32], sz),
         "misa_pool_keys": ([P, i64, i32, i32, i32, i32, i32, P, i64, i32, i32, P], i32),
@@ -193,6 +196,18 @@ def misa_device_check() -> None:
     """Waits for the device, then raises MisaError if a tensor-core kernel stopped early on a
     wait that ran out since the last check (its outputs are then incomplete)."""
     _check("misa_device_check", _lib.misa_device_check())
+
+
+def misa_bad_index_counts():
+    """Counts of skipped out-of-range ids since the last read, (heads, candidates, pages); all zero
+    unless the bounds-checked library is loaded.  Waits for the device; clears the counts."""
+    out = (ctypes.c_uint * 3)()
+    _check("misa_bad_index_counts", _lib.misa_bad_index_counts(out))
+    return tuple(int(x) for x in out)
+
+
+def checked_build() -> bool:
+    return bool(_lib.misa_checked_build())
 
 
 def misa_workspace_bytes(op: int, T: int, L: int, H_I: int, B: int = 1, h: int = 0, topk: int = 0,

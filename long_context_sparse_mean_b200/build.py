@@ -1,9 +1,11 @@
 """Build libmisa.so in-tree with nvcc for sm_100a (B200).
 
-    python -m long_context_sparse_mean_b200.build [--force] [--ptxas-verbose]
+    python -m long_context_sparse_mean_b200.build [--force] [--ptxas-verbose] [--checked]
 
 Every .cu file under csrc/ is compiled to an object in parallel, then linked into
-long_context_sparse_mean_b200/libmisa.so (CUDA runtime linked statically).
+long_context_sparse_mean_b200/libmisa.so (CUDA runtime linked statically).  --checked builds the
+bounds-checked variant libmisa_checked.so instead (MISA_CHECKED: out-of-range ids are counted on
+the device as they are skipped; include/misa.h, misa_bad_index_counts).
 """
 from __future__ import annotations
 
@@ -20,6 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libmisa.so")
+LIB_CHECKED = os.path.join(PKG, "libmisa_checked.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",
@@ -41,22 +44,24 @@ def _deps():
     return _sources() + glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "misa.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
-def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) -> str:
-    if not force and up_to_date():
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True, checked: bool = False) -> str:
+    lib = LIB_CHECKED if checked else LIB
+    if not force and up_to_date(lib):
+        return lib
+    objdir = os.path.join(BUILD, "checked") if checked else BUILD
+    os.makedirs(objdir, exist_ok=True)
     nvcc = _nvcc()
-    extra = ["-Xptxas", "-v"] if ptxas_verbose else []
+    extra = (["-Xptxas", "-v"] if ptxas_verbose else []) + (["-DMISA_CHECKED=1"] if checked else [])
 
     def compile_one(src):
-        obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
@@ -69,19 +74,20 @@ def build(force: bool = False, ptxas_verbose: bool = False, quiet: bool = True) 
         for _, err in results:
             if err:
                 sys.stderr.write(err)
-    tmp = LIB + f".tmp{os.getpid()}"
+    tmp = lib + f".tmp{os.getpid()}"
     cmd = [nvcc, *ARCH, "-shared", "-o", tmp, *[o for o, _ in results], "-lcudart_static", "-lrt", "-ldl",
            "-lpthread"]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--ptxas-verbose", action="store_true")
+    ap.add_argument("--checked", action="store_true", help="build the bounds-checked libmisa_checked.so")
     a = ap.parse_args()
-    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, quiet=False))
+    print(build(force=a.force, ptxas_verbose=a.ptxas_verbose, quiet=False, checked=a.checked))

@@ -52,6 +52,7 @@ __global__ void __launch_bounds__(kBlockScoreThreads) block_score_kernel(
   // routed heads: weight (0 for an index outside [0, H_I)) and q row in fp32
   for (int a = tid; a < h; a += kBlockScoreThreads) {
     const int j = heads[(int64_t)t * h + a];
+    count_bad_id(kBadHead, blockIdx.x == 0 && (j < 0 || j >= H_I));  // once per query
     ws_[a] = (j >= 0 && j < H_I) ? w[(int64_t)t * H_I + j] : 0.f;
   }
   for (int e = tid; e < h * kD; e += kBlockScoreThreads) {
@@ -135,5 +136,7 @@ void launch_expand_blocks(const int32_t* blocks, int m, const int32_t* n, int T,
   const dim3 grid((P + 255) / 256, T);
   expand_blocks_kernel<<<grid, 256, 0, s>>>(blocks, m, n, L, B, rows);
 }
+
+MISA_BAD_ID_READER(read_and_clear_bad_ids_block_filter)
 
 }  // namespace misa

@@ -53,14 +53,14 @@ size_t route_ws(int T, int L, int H_I, int B) {
 
 size_t scores_part(int T, int L) { return align_up(sizeof(float) * (size_t)T * score_ld(L)); }
 
-// misa_topk_select / misa_token_scores' selection state: the candidate lists of the rows, their
-// cuts and the sample they come from (the per-row selection itself needs no workspace)
+// misa_topk_select / misa_token_scores' selection state: the candidate lists of the rows and their
+// counts and cut keys (the per-row selection itself needs no workspace)
 size_t select_bytes(int T, int P) {
   if (T <= 0 || P <= 0) return 0;
   return align_up(misa::list_state_bytes(T));
 }
 
-// Per-query bf16 caches take the candidate-list top-k: sampled cut, lists appended by the scorer.
+// Per-query bf16 caches take the candidate-list top-k: the scorer builds the lists.
 bool list_path(int dtype, int64_t k_seq_stride) { return dtype == MISA_BF16 && k_seq_stride != 0; }
 
 // misa_score_topk / dsa_dense_topk: [scores][selection]
@@ -134,17 +134,43 @@ const char* misa_status_str(int status) {
       return "CUDA launch failed";
     case MISA_ERR_DEVICE_TIMEOUT:
       return "a device-side wait ran out; outputs of some call are incomplete";
+    case MISA_ERR_BAD_INDEX:
+      return "out-of-range ids were seen and skipped (bounds-checked build)";
     default:
       return "unknown status";
   }
+}
+
+namespace {
+bool read_bad_ids(unsigned int* out) {
+  for (int i = 0; i < misa::kBadIdKinds; ++i) out[i] = 0;
+  return misa::read_and_clear_bad_ids_score(out) && misa::read_and_clear_bad_ids_paged(out) &&
+         misa::read_and_clear_bad_ids_block_filter(out);
+}
+}  // namespace
+
+int misa_checked_build(void) {
+#ifdef MISA_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+misa_status misa_bad_index_counts(unsigned int* out) {
+  if (!out) return MISA_ERR_INVALID_ARG;
+  if (cudaDeviceSynchronize() != cudaSuccess) return MISA_ERR_CUDA;
+  return read_bad_ids(out) ? MISA_OK : MISA_ERR_CUDA;
 }
 
 misa_status misa_device_check(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return MISA_ERR_CUDA;
   const int v = misa::read_and_clear_tc_status();
   const int u = misa::read_and_clear_route_tc_status();
-  if (v < 0 || u < 0) return MISA_ERR_CUDA;
-  return (v || u) ? MISA_ERR_DEVICE_TIMEOUT : MISA_OK;
+  unsigned int bad[misa::kBadIdKinds];
+  if (v < 0 || u < 0 || !read_bad_ids(bad)) return MISA_ERR_CUDA;
+  if (v || u) return MISA_ERR_DEVICE_TIMEOUT;
+  return (bad[0] || bad[1] || bad[2]) ? MISA_ERR_BAD_INDEX : MISA_OK;
 }
 
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
@@ -231,9 +257,7 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
                         ld_scores, nullptr, s);
     return launch_status();
   }
-  const misa::ListState lst = misa::list_state(select_ws, T);
-  if (list_path(dtype, k_seq_stride)) misa::launch_list_cut(q, w, k, k_seq_stride, n, heads, T, L, H_I, m, select_topk,
-                                                            lst, s);
+  const misa::ListState lst = misa::list_state(select_ws, T, select_topk);
   const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0,
                                           scores, ld_scores, list_path(dtype, k_seq_stride) ? &lst : nullptr, s);
   if (!listed) misa::mark_no_lists(lst, T, s);
@@ -247,7 +271,7 @@ misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32
   if (T == 0) return MISA_OK;
   if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < select_bytes(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
-  const misa::ListState lst = misa::list_state(ws, T);
+  const misa::ListState lst = misa::list_state(ws, T, topk);
   misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws_prepared ? &lst : nullptr, idx, score_opt,
                          as_stream(stream));
   return launch_status();
@@ -274,9 +298,8 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
     p += scores_part(T, L);
   }
   const cudaStream_t s = as_stream(stream);
-  const misa::ListState lst = misa::list_state(p, T);
+  const misa::ListState lst = misa::list_state(p, T, topk);
   const bool lp = list_path(dtype, k_seq_stride);
-  if (lp) misa::launch_list_cut(q, w, k, k_seq_stride, n, heads, T, L, H_I, h, topk, lst, s);
   const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0,
                                           buf, ld, lp ? &lst : nullptr, s);
   misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);
@@ -312,10 +335,9 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   char* p = static_cast<char*>(ws);
   float* buf = reinterpret_cast<float*>(p);
   const int64_t ld = score_ld(L);
-  const misa::ListState lst = misa::list_state(p + scores_part(T, L), T);
+  const misa::ListState lst = misa::list_state(p + scores_part(T, L), T, topk);
   const cudaStream_t s = as_stream(stream);
   const bool lp = list_path(dtype, k_seq_stride);
-  if (lp) misa::launch_list_cut(q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, topk, lst, s);
   const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr,
                                           0, buf, ld, lp ? &lst : nullptr, s);
   misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);

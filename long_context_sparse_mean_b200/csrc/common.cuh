@@ -13,6 +13,37 @@ constexpr int kRouteTile = 64;   // router blocks per CTA tile
 // Element type of q and k.
 enum class DType : int { BF16 = 0, F32 = 1 };
 
+// Bounds-checked build (compiled with MISA_CHECKED): every id a kernel skips because it lies
+// outside its range is counted by kind in its translation unit's counters, which the C ABI reads
+// (misa_device_check, misa_bad_index_counts).  Such ids are never dereferenced in either build.
+enum BadIdKind : int {
+  kBadHead = 0,       // a routed head id outside [0, H_I)
+  kBadCandidate = 1,  // a candidate token id outside [0, n_t) other than the empty marker -1
+  kBadPage = 2,       // a page-table entry inside a prefix outside [0, num_pages)
+  kBadIdKinds = 3
+};
+#ifdef MISA_CHECKED
+static __device__ unsigned int g_bad_ids[kBadIdKinds];
+__device__ __forceinline__ void count_bad_id(int kind, bool bad) {
+  if (bad) atomicAdd(&g_bad_ids[kind], 1u);
+}
+// Host side: adds this translation unit's counters to out[kBadIdKinds] and clears them; false if
+// the copy failed.
+#define MISA_BAD_ID_READER(name)                                                          \
+  bool name(unsigned int* out) {                                                          \
+    unsigned int v[kBadIdKinds] = {0, 0, 0};                                              \
+    if (cudaMemcpyFromSymbol(v, g_bad_ids, sizeof(v)) != cudaSuccess) return false;       \
+    const unsigned int z[kBadIdKinds] = {0, 0, 0};                                        \
+    if (cudaMemcpyToSymbol(g_bad_ids, z, sizeof(z)) != cudaSuccess) return false;         \
+    for (int i = 0; i < kBadIdKinds; ++i) out[i] += v[i];                                 \
+    return true;                                                                          \
+  }
+#else
+__device__ __forceinline__ void count_bad_id(int, bool) {}
+#define MISA_BAD_ID_READER(name) \
+  bool name(unsigned int*) { return true; }
+#endif
+
 // Order-preserving map of a finite fp32 value onto uint32: a > b  <=>  key(a) > key(b), and
 // -0 and +0 map to the same key (they are the same score).
 __device__ __forceinline__ uint32_t order_key(float f) {

@@ -37,33 +37,28 @@ void launch_route_finish(const __nv_bfloat16* q, const float* w, const __nv_bflo
                          int L, int H_I, int B, int h, const float* Sp, int nch, int tile, int32_t* heads,
                          float* r_opt, cudaStream_t s);
 
-// Candidate lists of a top-k over per-query caches, built while the scores are written (select.cuh
-// holds the sizes): a cut per query from a sample of its keys scored beforehand, then every score
-// at or above the cut is appended as (order key, token) to the query's list.
+// Candidate lists of a top-k over per-query caches, built by the scoring kernel while it scores
+// (select.cuh holds the sizes).  Every CTA that scores a run of a query's keys places a cut on the
+// run's own scores (its share of the top-k, 1.5 times over, plus 16), appends the run's entries at
+// or above the cut to the query's list and raises the query's cut key to its own cut; every key
+// at or above the query's final cut key is then in the list.
 struct ListState {
   uint32_t* cnt;     // [T] entries appended (also past cap); kNoList: no list for this row
-  float* tau;        // [T] cut: -inf takes every entry, +inf none (the row goes the exact way)
-  uint32_t* arrive;  // [T] sample CTAs done (zeroed before the sample kernel)
-  float* sample;     // [T][kSampleRuns * kSampleRunLen] sample scores
-  uint2* list;       // [T][cap]
+  uint32_t* cutkey;  // [T] largest cut, as an order key, any CTA used for the row (right after cnt)
+  uint2* list;       // [T][cap] (order key, token)
   int cap;
+  int topk;
 };
 size_t list_state_bytes(int T);
-ListState list_state(void* ws, int T);
+ListState list_state(void* ws, int T, int topk);
 // cnt = kNoList for every row (scores written without lists).
 void mark_no_lists(const ListState& l, int T, cudaStream_t s);
 
-// The cut of every query for a top-topk of its routed (heads) or dense (heads == nullptr) scores
-// over one bf16 cache per query: scores kSampleRuns runs of kSampleRunLen keys spread over the
-// prefix, sets tau and zeroes cnt.  Prefixes of at most cap keys take every entry.
-void launch_list_cut(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
-                     const int32_t* heads, int T, int L, int H_I, int h, int topk, const ListState& l,
-                     cudaStream_t s);
-
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
 // position p of query t scores token rows[t*P + p] and writes out[t*ld + p].  With lst (bf16, one
-// cache per query, no gather: the persistent kernel) every score at or above lst->tau[t] is also
-// appended to the query's list; returns whether it was.
+// cache per query, no gather: the persistent kernel, when the lists are expected to fit) the
+// candidate lists of a top-lst->topk are built too; returns whether they were (otherwise the
+// caller marks the rows as having none).
 bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
                    const int32_t* rows, int P, float* out, int64_t ld, const ListState* lst, cudaStream_t s);
@@ -75,6 +70,11 @@ bool launch_scores_tc(const void* q, const float* w, const void* k, const int32_
 // Reads and clears the status word the tensor-core kernels set when a bounded wait runs out.
 int read_and_clear_tc_status();
 int read_and_clear_route_tc_status();
+// Bounds-checked build: add each file's counts of skipped out-of-range ids to out[kBadIdKinds] and
+// clear them (always true and nothing added in the normal build).
+bool read_and_clear_bad_ids_score(unsigned int* out);
+bool read_and_clear_bad_ids_paged(unsigned int* out);
+bool read_and_clear_bad_ids_block_filter(unsigned int* out);
 
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
 // or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t); P <= 16384).  lst: the

@@ -18,13 +18,17 @@ namespace misa {
 
 namespace {
 
-// Physical row of logical key s of sequence t, or -1 (page past the table or out of the pool).
+// Physical row of logical key s of sequence t, or -1 (page past the table or out of the pool; a
+// bounds-checked build counts an out-of-pool page when `count` is set).
 __device__ __forceinline__ int64_t paged_row(const int32_t* table, int64_t max_pages, int64_t num_pages,
-                                             int page_size, int t, int64_t s) {
+                                             int page_size, int t, int64_t s, bool count) {
   const int64_t lp = s / page_size;
   if (lp >= max_pages) return -1;
   const int32_t pg = __ldg(table + (int64_t)t * max_pages + lp);
-  if (pg < 0 || pg >= num_pages) return -1;
+  if (pg < 0 || pg >= num_pages) {
+    count_bad_id(kBadPage, count);
+    return -1;
+  }
   return (int64_t)pg * page_size + s % page_size;
 }
 
@@ -39,7 +43,8 @@ __global__ void paged_rows_kernel(const int32_t* __restrict__ table, int64_t max
   if (p >= P) return;
   const int nt = clamp_len(n[t], L);
   const int64_t s = ids ? (int64_t)ids[(int64_t)t * P + p] : (int64_t)p;
-  const int64_t r = (s >= 0 && s < nt) ? paged_row(table, max_pages, num_pages, page_size, t, s) : -1;
+  count_bad_id(kBadCandidate, ids && s != -1 && (s < 0 || s >= nt));
+  const int64_t r = (s >= 0 && s < nt) ? paged_row(table, max_pages, num_pages, page_size, t, s, true) : -1;
   rows[(int64_t)t * P + p] = (int32_t)r;
 }
 
@@ -53,7 +58,7 @@ __device__ __forceinline__ void paged_sum(const void* pool, const int32_t* table
   const int cp = threadIdx.x & 63, rg = threadIdx.x >> 6;
   float a0 = 0.f, a1 = 0.f;
   for (int s = s0 + rg; s < s1; s += RG) {
-    const int64_t r = paged_row(table, max_pages, num_pages, page_size, t, s);
+    const int64_t r = paged_row(table, max_pages, num_pages, page_size, t, s, cp == 0);  // one count per row
     if (r < 0) continue;
     if (DT == DType::BF16) {
       const uint32_t x = __ldg(reinterpret_cast<const uint32_t*>(pool) + r * (kD / 2) + cp);
@@ -140,5 +145,7 @@ void launch_partial_mean_paged(DType dt, const void* pool, int64_t num_pages, in
     partial_mean_paged_kernel<DType::F32><<<T, 256, 0, s>>>(pool, num_pages, page_size, table, max_pages, n, L, B,
                                                             pm);
 }
+
+MISA_BAD_ID_READER(read_and_clear_bad_ids_paged)
 
 }  // namespace misa

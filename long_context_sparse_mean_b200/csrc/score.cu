@@ -20,10 +20,12 @@
 //       32 x 131072 keys: 178 us against 185 us for the grid kernel; an added bulk L2 prefetch
 //       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
 //       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
-//       For a top-k of the scores it can also append every score at or above a per-query cut to
-//       the query's candidate list while it writes the scores (one ballot and at most one atomic
-//       per warp and tile), so the selection ranks a list of about 1.4 k entries instead of
-//       sweeping the row; list_cut_kernel places the cut beforehand from a sample of the keys.
+//       For a top-k of the scores it can also build each query's candidate list: after a run of
+//       a query's tiles the CTA places a cut on the run's scores (a histogram over their key
+//       range; the run's share of the top-k, 1.5 times over, plus 16 entries), appends the run's
+//       entries at or above it to the query's list (one global atomic per run) and raises the
+//       query's cut key, so the selection ranks a list of about 1.5 k entries instead of
+//       sweeping the row (three passes over the run's scores, read back from L2).
 //   score_grid_kernel     one CTA per (query, chunk of positions): shared caches when the
 //       tensor-core kernel (score_tc.cu, which takes shared bf16 caches) cannot run, and more
 //       queries than the persistent schedule takes.
@@ -64,11 +66,16 @@ __device__ __forceinline__ void stage_head_list(const int32_t* heads, int h, int
     if (threadIdx.x == 0) *m_out = H_I;
     return;
   }
+  // every id is loaded at once (one per thread), then one thread sorts them in shared memory
+  for (int a = threadIdx.x; a < h; a += blockDim.x) {
+    int v = heads[(int64_t)t * h + a];
+    count_bad_id(kBadHead, v < 0 || v >= H_I);
+    hl[a] = v < 0 ? 0 : (v >= H_I ? H_I - 1 : v);  // out-of-range ids are clamped, never dereferenced
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    const int m = heads ? h : H_I;
-    for (int a = 0; a < m; ++a) {
-      int v = heads ? heads[(int64_t)t * h + a] : a;
-      v = v < 0 ? 0 : (v >= H_I ? H_I - 1 : v);  // out-of-range ids are clamped, never dereferenced
+    for (int a = 1; a < h; ++a) {
+      const int v = hl[a];
       int b = a;
       while (b > 0 && hl[b - 1] > v) {
         hl[b] = hl[b - 1];
@@ -76,8 +83,8 @@ __device__ __forceinline__ void stage_head_list(const int32_t* heads, int h, int
       }
       hl[b] = v;
     }
-    for (int a = m; a < slots; ++a) hl[a] = hl[0];
-    *m_out = m;
+    for (int a = h; a < slots; ++a) hl[a] = hl[0];
+    *m_out = h;
   }
 }
 
@@ -92,17 +99,75 @@ __device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat
   __syncthreads();
 }
 
+// Candidate list of one run of a query's scores, [s0, s1) of row `ot` (written by this CTA): a cut
+// r-th from the top of the run (r = its share of the top-k, 1.5 times over, plus 16), placed with a
+// 4096-bin histogram over the run's key range [kmin, kmax] (every thread's keys, reduced here) at
+// the lower edge of the bin holding the r-th largest; every entry at or above the cut is appended
+// to the query's list lt (one global atomic for the run) and the query's cut key is raised to it.
+// Prefixes of at most cap keys keep every entry.  All threads of the CTA call it.
+__device__ __forceinline__ void segment_list(const float* ot, int t, int s0, int s1, int nt, uint32_t kmin,
+                                             uint32_t kmax, uint32_t* hist, uint32_t* mm, uint32_t* scratch,
+                                             uint32_t* sbase, uint2* lt, uint32_t* lcnt, uint32_t* lcut, int cap,
+                                             int topk) {
+  const int len = s1 - s0;
+  block_min_max(kmin, kmax, mm);
+  __syncthreads();  // also: the run's scores are visible to the whole CTA
+  uint32_t cut = 0u;  // order key; 0 keeps every entry
+  if (nt > cap) {
+    const float share = 1.5f * (float)topk * (float)len / (float)nt;
+    const int r = min(len, (int)ceilf(share) + 16);
+    if (r < len) {
+      const uint32_t lo = mm[0], range = mm[1] - mm[0];
+      const int sh = range >= 4096u ? 32 - __clz(range) - 12 : 0;
+      for (int b = threadIdx.x; b < kHistBins; b += kScoreThreads) hist[b] = 0;
+      __syncthreads();
+#pragma unroll 4
+      for (int i = threadIdx.x; i < len; i += kScoreThreads)
+        hist_add(hist, (order_key(__ldcg(ot + s0 + i)) - lo) >> sh, true);
+      __syncthreads();
+      cut = lo + block_bucket_bits(hist, kHistBins, sh, 0u, (uint32_t)r, scratch).prefix;
+    }
+  }
+  uint32_t mine = 0;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < len; i += kScoreThreads) mine += order_key(__ldcg(ot + s0 + i)) >= cut;
+  uint32_t total;
+  uint32_t slot = block_exclusive_scan(mine, scratch, &total);
+  if (threadIdx.x == 0) {
+    *sbase = atomicAdd(lcnt + t, total);
+    atomicMax(lcut + t, cut);
+  }
+  __syncthreads();
+  slot += *sbase;
+#pragma unroll 4
+  for (int i = threadIdx.x; i < len; i += kScoreThreads) {
+    const uint32_t k = order_key(__ldcg(ot + s0 + i));
+    if (k >= cut) {
+      if (slot < (uint32_t)cap) lt[slot] = make_uint2(k, (uint32_t)(s0 + i));
+      ++slot;
+    }
+  }
+  if (threadIdx.x == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+}
+
 template <int NG, bool GATHER>
 __global__ void __launch_bounds__(kScoreThreads, 2)
     score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                          const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                          const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
                          const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld,
-                         const float* __restrict__ tau, uint2* __restrict__ lists, uint32_t* __restrict__ lcnt,
-                         int cap) {
-  extern __shared__ int tile_base[];  // [T + 1] flattened tile prefix
+                         uint2* __restrict__ lists, uint32_t* __restrict__ lcnt, uint32_t* __restrict__ lcut,
+                         int cap, int topk) {
+  // dynamic: [T + 1] flattened tile prefix, then (candidate lists) a 4096-bin histogram
+  extern __shared__ int tile_base[];
+  uint32_t* hist = reinterpret_cast<uint32_t*>(tile_base + ((T + 1 + 3) & ~3));
   __shared__ HeadStage<NG> st;
   __shared__ uint32_t wtot[35];
+  __shared__ uint32_t mm[2];
+  __shared__ uint32_t sbase;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
 
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
@@ -135,10 +200,13 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const int nt = clamp_len(n[t], L);
     const int npos = GATHER ? P : nt;
     const int32_t* rt = GATHER ? rows + (int64_t)t * P : nullptr;
-    const float cut = lists ? __ldg(tau + t) : 0.f;
-    uint2* lt = lists ? lists + (int64_t)t * cap : nullptr;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;  // order keys of the scores this thread writes (lists)
 
     __syncthreads();  // the previous segment's fragments are no longer read
+    if (threadIdx.x == 0) {
+      mm[0] = 0xffffffffu;
+      mm[1] = 0u;
+    }
     stage_query<NG>(st, q, w, heads, h, H_I, t);
     float wa[NG], wb[NG];
 #pragma unroll
@@ -151,7 +219,13 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     auto row_of = [&](int j) { return (first + j) * kTileRows + warp * 16; };
     // position p -> key row: p itself, or rows[t, p] when gathering (outside [0, n_t): empty).
     // Gathered row ids are fetched two tiles ahead, so a tile's row loads never wait for its ids.
-    auto raw_id = [&](int p) -> int { return p < npos ? (GATHER ? __ldg(rt + p) : p) : -1; };
+    auto raw_id = [&](int p) -> int {
+      if (p >= npos) return -1;
+      if (!GATHER) return p;
+      const int id = __ldg(rt + p);
+      count_bad_id(kBadCandidate, c == 0 && id != -1 && (id < 0 || id >= nt));  // one lane of the quad
+      return id;
+    };
     auto valid_row = [&](int r) -> int { return (r >= 0 && r < nt) ? r : -1; };
     int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
     int nia = GATHER && ntile > 1 ? raw_id(row_of(1) + g) : -1;
@@ -187,19 +261,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       const int r = row_of(j) + g;
       if (c == 0 && r < npos) ot[r] = slo;
       if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
-      if (!GATHER && lists) {
-        // the key rows of this tile whose score reaches the cut join the query's candidate list
-        const float v = c == 0 ? slo : shi;
-        const bool keep = (c == 0 ? va : (c == 1 && vb)) && v >= cut;
-        const unsigned m = __ballot_sync(0xffffffffu, keep);
-        if (m) {  // uniform across the warp
-          const int leader = __ffs(m) - 1;
-          uint32_t base = 0;
-          if (lane == leader) base = atomicAdd(lcnt + t, (uint32_t)__popc(m));
-          base = __shfl_sync(0xffffffffu, base, leader);
-          const uint32_t slot = base + (uint32_t)__popc(m & ((1u << lane) - 1u));
-          if (keep && slot < (uint32_t)cap) lt[slot] = make_uint2(order_key(v), (uint32_t)(c == 0 ? r : r + 8));
-        }
+      if (!GATHER && lists && c < 2 && r + 8 * c < npos) {
+        const uint32_t kk = order_key(c == 0 ? slo : shi);
+        kmin = min(kmin, kk);
+        kmax = max(kmax, kk);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -209,81 +274,9 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       va = na;
       vb = nb;
     }
+    if (!GATHER && lists) segment_list(ot, t, first * kTileRows, min((first + ntile) * kTileRows, nt), nt, kmin,
+                                       kmax, hist, mm, wtot, &sbase, lists + (int64_t)t * cap, lcnt, lcut, cap, topk);
     pos = seg_end;
-  }
-}
-
-// Sampled cut of each query's scores for a top-k (one bf16 cache per query): CTA cb of query t
-// scores the sample runs [16 cb, 16 cb + 16) (warp w: runs 16 cb + 2w and 16 cb + 2w + 1, one run
-// of 8 consecutive keys per half of its 16-row MMA group) with the query's head list into
-// l.sample; the query's last CTA to finish places the cut from all 2048 sample scores (the sample
-// rank that the row top-k would use) and zeroes the list count.  Rows of at most cap keys take
-// every entry (cut -inf); rows whose top-k the sample cannot place take none (cut +inf), so their
-// selection takes the exact path.
-constexpr int kCutCtas = kSampleRuns / 16;
-
-template <int NG>
-__global__ void __launch_bounds__(kScoreThreads)
-    list_cut_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
-                    const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
-                    const int32_t* __restrict__ heads, int h, int H_I, int L, int topk, ListState l) {
-  __shared__ union Smem {  // the head list while scoring, the cut's histogram after
-    HeadStage<NG> st;
-    uint32_t hist[kHistBins];
-  } sm_u;
-  HeadStage<NG>& st = sm_u.st;
-  uint32_t* hist = sm_u.hist;
-  __shared__ uint32_t scratch[35];
-  __shared__ uint32_t mm[2];
-  __shared__ int last;
-  constexpr int ns = kSampleRuns * kSampleRunLen;
-  const int t = blockIdx.y, cb = blockIdx.x;
-  const int nt = clamp_len(n[t], L);
-  const uint32_t rank = sample_rank(topk, nt);
-  if (nt <= l.cap || rank > (uint32_t)ns) {
-    if (cb == 0 && threadIdx.x == 0) {
-      l.tau[t] = nt <= l.cap ? -INFINITY : INFINITY;
-      l.cnt[t] = 0u;
-    }
-    return;
-  }
-  stage_query<NG>(st, q, w, heads, h, H_I, t);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
-  float wa[NG], wb[NG];
-#pragma unroll
-  for (int ng = 0; ng < NG; ++ng) {
-    wa[ng] = st.wsel[ng * 8 + 2 * c];
-    wb[ng] = st.wsel[ng * 8 + 2 * c + 1];
-  }
-  const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);  // >= 64: nt > cap
-  const int ra = 16 * cb + 2 * warp, rb = ra + 1;
-  const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
-  uint4 A[4], Bq[4];
-  load_rows(kt + ((int64_t)ra * seg + g) * kD, kt + ((int64_t)rb * seg + g) * kD, c, A, Bq);
-  float slo, shi;
-  score_rows<NG>(A, Bq, st.frag, wa, wb, lane, slo, shi);
-  float* sm = l.sample + (int64_t)t * ns;
-  if (c == 0) sm[ra * kSampleRunLen + g] = slo;
-  if (c == 1) sm[rb * kSampleRunLen + g] = shi;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(l.arrive + t, 1u) == (uint32_t)(kCutCtas - 1);
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  constexpr int per = ns / kScoreThreads;
-  uint32_t sk[per];
-#pragma unroll
-  for (int u = 0; u < per; ++u) sk[u] = order_key(__ldcg(sm + u * kScoreThreads + threadIdx.x));
-  if (threadIdx.x == 0) {
-    mm[0] = 0xffffffffu;
-    mm[1] = 0u;
-  }
-  const float cut = sample_cut<per>(sk, rank, hist, mm, scratch);
-  if (threadIdx.x == 0) {
-    l.tau[t] = cut;
-    l.cnt[t] = 0u;
-    l.arrive[t] = 0u;
   }
 }
 
@@ -420,19 +413,20 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   if (persist) {
-    const size_t smem = sizeof(int) * ((size_t)T + 1);
-    const float* tau = lst ? lst->tau : nullptr;
-    uint2* lists = lst ? lst->list : nullptr;
-    uint32_t* lcnt = lst ? lst->cnt : nullptr;
-    const int cap = lst ? lst->cap : 0;
+    size_t smem = sizeof(int) * (size_t)((T + 1 + 3) & ~3);
+    if (lst) {
+      smem += sizeof(uint32_t) * kHistBins;
+      cudaMemsetAsync(lst->cnt, 0, sizeof(uint32_t) * 2 * (size_t)T, s);  // counts and cut keys
+    }
     if (gather) {
       cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, nullptr, nullptr, nullptr, 0);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, nullptr, nullptr, nullptr, 0, 0);
     } else {
       cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, tau, lists, lcnt, cap);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, lst ? lst->list : nullptr,
+          lst ? lst->cnt : nullptr, lst ? lst->cutkey : nullptr, lst ? lst->cap : 0, lst ? lst->topk : 0);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
@@ -445,12 +439,12 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
   }
 }
 
-template <int NG>
-void launch_cut(cudaStream_t s, const void* q, const float* w, const void* k, int64_t k_seq_stride,
-                const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L, int topk, const ListState& l) {
-  list_cut_kernel<NG><<<dim3(kCutCtas, T), kScoreThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(q), w,
-                                                                  static_cast<const __nv_bfloat16*>(k), k_seq_stride,
-                                                                  n, heads, h, H_I, L, topk, l);
+// Whether candidate lists of a top-k suit a launch: every CTA's run of a query adds up to 16
+// entries beyond its share of 1.5 k, so the expected list must stay well inside the cap.
+bool lists_fit(const ListState* lst, int T) {
+  if (!lst || T <= 0) return false;
+  const double ctas_per_query = (2.0 * num_sms() + T - 1) / T + 2.0;
+  return 1.5 * lst->topk + 16.0 * ctas_per_query <= 0.9 * lst->cap;
 }
 
 }  // namespace
@@ -485,7 +479,7 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
   const int ng = (m + 7) / 8;
   // persistent schedule for per-query caches and for gathered candidate lists
   const bool persist = (gather || k_seq_stride != 0) && T <= kMaxPersistQueries;
-  const ListState* l = persist && !gather ? lst : nullptr;
+  const ListState* l = persist && !gather && lists_fit(lst, T) ? lst : nullptr;
   switch (ng) {
 #define MISA_NG_CASE(NGV)                                                                                  \
   case NGV:                                                                                                \
@@ -514,37 +508,6 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
   return l != nullptr;
 }
 
-void launch_list_cut(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
-                     const int32_t* heads, int T, int L, int H_I, int h, int topk, const ListState& l,
-                     cudaStream_t s) {
-  if (T <= 0) return;
-  cudaMemsetAsync(l.arrive, 0, sizeof(uint32_t) * (size_t)T, s);
-  const int m = heads ? h : H_I;
-  switch ((m + 7) / 8) {
-#define MISA_CUT_CASE(NGV)                                                     \
-  case NGV:                                                                    \
-    launch_cut<NGV>(s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, topk, l); \
-    break;
-    MISA_CUT_CASE(1)
-    MISA_CUT_CASE(2)
-    MISA_CUT_CASE(3)
-    MISA_CUT_CASE(4)
-    MISA_CUT_CASE(5)
-    MISA_CUT_CASE(6)
-    MISA_CUT_CASE(7)
-    MISA_CUT_CASE(8)
-    MISA_CUT_CASE(9)
-    MISA_CUT_CASE(10)
-    MISA_CUT_CASE(11)
-    MISA_CUT_CASE(12)
-    MISA_CUT_CASE(13)
-    MISA_CUT_CASE(14)
-    MISA_CUT_CASE(15)
-    MISA_CUT_CASE(16)
-#undef MISA_CUT_CASE
-    default:
-      break;
-  }
-}
+MISA_BAD_ID_READER(read_and_clear_bad_ids_score)
 
 }  // namespace misa

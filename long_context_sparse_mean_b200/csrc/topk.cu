@@ -325,15 +325,17 @@ __device__ void select_list_linear(uint2* list, int c, uint32_t need, uint32_t l
 // Rows of scores [T, ld]; ids == nullptr: entry p < n_t is token p; otherwise entry p < P is token
 // ids[t P + p] (empty when outside [0, n_t)), and P <= LIST.  lists (optional): the candidate lists
 // the decode scoring kernel appended, [T][lcap] (key, token) with lcnt[t] entries (kNoList: the row
-// has none); a row whose count lies in [topk, lcap] is selected from its list, any other count
-// sends the row to the exact path.
+// has none) and every key at or above lcut[t] among them; a row whose list has at least topk
+// entries at or above lcut[t] and lost none past lcap is selected from those entries, any other row
+// takes the exact path.
 template <int NT, int LIST, int MINB>
 __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
                                                             const int32_t* __restrict__ ids_all, int P,
                                                             const int32_t* __restrict__ n, int L, int topk,
                                                             int32_t* __restrict__ idx, float* __restrict__ score_opt,
                                                             const uint2* __restrict__ lists,
-                                                            const uint32_t* __restrict__ lcnt, int lcap) {
+                                                            const uint32_t* __restrict__ lcnt,
+                                                            const uint32_t* __restrict__ lcut, int lcap) {
   extern __shared__ uint2 list[];  // [LIST]
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
@@ -368,20 +370,29 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
     c_in = __ldcg(lcnt + t);
     if (c_in != kNoList) {
       listed = c_in >= (uint32_t)topk && c_in <= (uint32_t)min(lcap, LIST);
-      exact = !listed;  // too few at or above the cut, or entries dropped past the list's end
+      exact = !listed;  // too few entries, or entries dropped past the list's end
     }
   }
-  if (listed) {  // copy the scoring kernel's list
+  if (listed) {  // copy the scoring kernel's list: the entries at or above the row's cut key
     const uint2* src = lists + (int64_t)t * lcap;
+    const uint32_t cut = __ldcg(lcut + t);
     uint32_t lo = 0xffffffffu, hi = 0u;
-    for (uint32_t i = tid; i < c_in; i += NT) {
-      const uint2 e = __ldcg(src + i);
-      list[i] = e;
-      lo = min(lo, e.x);
-      hi = max(hi, e.x);
+    for (uint32_t i0 = 0; i0 < c_in; i0 += NT) {
+      const uint32_t i = i0 + tid;
+      const uint2 e = i < c_in ? __ldcg(src + i) : make_uint2(0u, 0u);
+      const bool keep = i < c_in && e.x >= cut;
+      const uint32_t slot = warp_slot(keep, &cnt[0]);
+      if (keep) {
+        list[slot] = e;
+        lo = min(lo, e.x);
+        hi = max(hi, e.x);
+      }
     }
     block_min_max(lo, hi, mm);
-    if (tid == 0) cnt[0] = c_in;
+    __syncthreads();
+    // fewer than k entries at or above the cut: the list cannot hold the answer
+    exact = cnt[0] < (uint32_t)topk;
+    listed = !exact;
     __syncthreads();
   } else if (!exact) {
     float thr = -INFINITY;
@@ -493,7 +504,7 @@ void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P,
   cudaFuncSetAttribute(row_topk_kernel<NT, LIST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt,
                                                       lst ? lst->list : nullptr, lst ? lst->cnt : nullptr,
-                                                      lst ? lst->cap : 0);
+                                                      lst ? lst->cutkey : nullptr, lst ? lst->cap : 0);
 }
 
 struct SmemItems {
@@ -548,34 +559,25 @@ __global__ void __launch_bounds__(kSmallThreads) select_small_kernel(const float
 
 }  // namespace
 
-// Candidate-list state of one selection (kernels.cuh): cnt [T], tau [T], arrive [T],
-// sample [T][kSampleRuns * kSampleRunLen] fp32, list [T][kListCap] (key, token); each piece
-// 256-byte aligned.
+// Candidate-list state of one selection (kernels.cuh): cnt [T] and cutkey [T] in one piece, then
+// list [T][kListCap] (key, token); each piece 256-byte aligned.
 namespace {
 size_t al(size_t x) { return (x + 255) / 256 * 256; }
 }  // namespace
 
 size_t list_state_bytes(int T) {
   if (T <= 0) return 0;
-  const size_t t = (size_t)T;
-  return 3 * al(sizeof(uint32_t) * t) + al(sizeof(float) * t * kSampleRuns * kSampleRunLen) +
-         al(sizeof(uint2) * t * kListCap);
+  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(uint2) * (size_t)T * kListCap);
 }
 
-ListState list_state(void* ws, int T) {
+ListState list_state(void* ws, int T, int topk) {
   char* p = static_cast<char*>(ws);
-  const size_t t = (size_t)T;
   ListState l;
   l.cnt = reinterpret_cast<uint32_t*>(p);
-  p += al(sizeof(uint32_t) * t);
-  l.tau = reinterpret_cast<float*>(p);
-  p += al(sizeof(uint32_t) * t);
-  l.arrive = reinterpret_cast<uint32_t*>(p);
-  p += al(sizeof(uint32_t) * t);
-  l.sample = reinterpret_cast<float*>(p);
-  p += al(sizeof(float) * t * kSampleRuns * kSampleRunLen);
-  l.list = reinterpret_cast<uint2*>(p);
+  l.cutkey = l.cnt + T;
+  l.list = reinterpret_cast<uint2*>(p + al(sizeof(uint32_t) * 2 * (size_t)T));
   l.cap = kListCap;
+  l.topk = topk;
   return l;
 }
 

@@ -12,7 +12,7 @@ from long_context_sparse_mean_b200 import build
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "misa.h")
 
-OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT = range(6)
+OK, INVALID, UNSUPPORTED, WORKSPACE, CUDA, DEVICE_TIMEOUT, BAD_INDEX = range(7)
 BF16, F32 = 0, 1
 P = ctypes.c_void_p
 
@@ -47,7 +47,7 @@ def test_every_declared_symbol_is_exported(lib):
 
 def test_status_strings_and_version(lib):
     assert lib.misa_version() >= 100
-    for code in range(6):
+    for code in range(7):
         assert lib.misa_status_str(code) != b"unknown status"
     assert lib.misa_status_str(99) == b"unknown status"
 
@@ -61,10 +61,10 @@ def test_workspace_sizes(lib):
     # router: [T,128] partial-block means + [T, ceil(ceil(L/B)/64), H_I] tile sums + [T] counters
     # + [3, ceil(L/B), 128] bf16 parts of the pooled keys
     assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256 + 3 * 1024 * 128 * 2
-    # top-k select: candidate-list state per query: count, cut and arrival counter [T] each, the
-    # sample [T, 2048] and the list [T, 16384] (key, token) pairs, each piece 256-byte aligned
+    # top-k select: candidate-list state per query: count and cut key [2, T] in one piece, then the
+    # list [T, 16384] of (key, token) pairs, each piece 256-byte aligned
     def sel(T):
-        return 3 * _al(T * 4) + _al(T * 2048 * 4) + _al(T * 16384 * 8)
+        return _al(T * 8) + _al(T * 16384 * 8)
     assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel(32)
     assert ws(4, 32, 7, 64, 0, 0, 2048, 0) == sel(32), "independent of the row length"
     # scoring + top-k: [T, ceil4(L)] scores in front of the select workspace
@@ -272,3 +272,19 @@ int main(void) {
     out = subprocess.run([str(exe)], capture_output=True, text=True)
     assert out.returncode == 0, (out.returncode, out.stderr)
     assert out.stdout.strip() == "unsupported configuration"
+
+
+def test_bounds_checked_build_exports_the_same_calls():
+    """libmisa_checked.so (MISA_CHECKED) exports every call misa.h declares and says it is the checked
+    build; the normal library says it is not, and both refuse a null count buffer on the host."""
+    checked = ctypes.CDLL(build.build(checked=True))
+    for name in declared_functions():
+        assert hasattr(checked, name), f"{name} missing from the checked build"
+    checked.misa_checked_build.restype = ctypes.c_int
+    checked.misa_bad_index_counts.argtypes = [P]
+    checked.misa_bad_index_counts.restype = ctypes.c_int
+    assert checked.misa_checked_build() == 1
+    assert checked.misa_bad_index_counts(None) == INVALID
+    normal = ctypes.CDLL(build.build())
+    normal.misa_checked_build.restype = ctypes.c_int
+    assert normal.misa_checked_build() == 0
