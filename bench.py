@@ -494,25 +494,30 @@ def run_reference_prefill(args, wl, nthr):
 # ---- chunked causal prefill (shared cache) ------------------------------------------------------------
 
 def prefill_measure(args, wl, dev, gen_pool, steps, warmup, dist=None, ws=1, want_e2e=True, want_dense=True,
-                    want_cpu=True):
+                    want_cpu=True, fused=False, inputs=None):
     """One step = the whole chunked causal prefill of one sequence: pool every block of the shared
     cache once, then for each chunk of queries route, score with the routed heads on the tensor
-    cores, and select the top-k of every query.  Returns the measurements as a dict."""
+    cores, and select the top-k of every query (fused: scoring and selection in one call that writes
+    no score rows, misa_score_topk_fused).  Returns the measurements as a dict; inputs: the device
+    tensors of an earlier call, to measure the other path on the same inputs."""
     import torch
     from long_context_sparse_mean_b200 import binding as M
 
     ch = wl.chunk
     nch = -(-wl.T // ch)
-    over = {f: getattr(wl, f) for f in wl.__dataclass_fields__ if f not in ("cid", "seed")}
-    parts = gen_pool.starmap(_gen_chunk, [(wl.cid, wl.seed, c, over) for c in range(nch)])
     k_h = W.shared_keys(wl)
     n_h = W.prefix_lengths(wl)
     L, d, T, B, h, kk = wl.L, wl.d, wl.T, wl.B, wl.h, wl.topk
-    kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
-    qd = torch.cat([torch.from_numpy(p[0]).to(torch.bfloat16) for p in parts]).to(dev)
-    wd = torch.cat([torch.from_numpy(p[1]) for p in parts]).to(dev)
-    nd = torch.from_numpy(n_h).to(dev)
-    del parts
+    if inputs is None:
+        over = {f: getattr(wl, f) for f in wl.__dataclass_fields__ if f not in ("cid", "seed")}
+        parts = gen_pool.starmap(_gen_chunk, [(wl.cid, wl.seed, c, over) for c in range(nch)])
+        kd = torch.from_numpy(k_h).to(torch.bfloat16).to(dev)
+        qd = torch.cat([torch.from_numpy(p[0]).to(torch.bfloat16) for p in parts]).to(dev)
+        wd = torch.cat([torch.from_numpy(p[1]) for p in parts]).to(dev)
+        nd = torch.from_numpy(n_h).to(dev)
+        del parts
+    else:
+        kd, qd, wd, nd = inputs
     stream = torch.cuda.current_stream()
     wsp = M.Workspace(dev)
     sel_ws = M.Workspace(dev)
@@ -543,18 +548,23 @@ def prefill_measure(args, wl, dev, gen_pool, steps, warmup, dist=None, ws=1, wan
                 stage_ev[c][1].record(stream)
             if time_scores:
                 score_ev[c][0].record(stream)
-            M.misa_token_scores(qc, wc, kd, nc, hc, out=sc)
+            if fused:
+                M.misa_score_topk_fused(qc, wc, kd, nc, hc, kk, idx=idx[a:b], want_vals=False, ws=sel_ws)
+            else:
+                M.misa_token_scores(qc, wc, kd, nc, hc, out=sc)
             if time_scores:
                 score_ev[c][1].record(stream)
             if stages:
                 stage_ev[c][2].record(stream)
-            M.misa_topk_select(sc, nc, kk, idx=idx[a:b], want_vals=False, ws=sel_ws)
+            if not fused:
+                M.misa_topk_select(sc, nc, kk, idx=idx[a:b], want_vals=False, ws=sel_ws)
             if stages:
                 stage_ev[c][3].record(stream)
 
-    # launches per step: pool + per chunk (route 1, tensor-core scores 1, selection 1); the router
-    # of a shared cache is kbar_split + route_tc + route_finish (3)
-    launches_per_step = 1 + nch * 5
+    # launches per step: pool + per chunk: the router (pooled-key split, tensor-core router, finish)
+    # and scores + selection, or fused: sample, cuts, compact scores, list selection and the two
+    # launches of the exact redo (empty unless a list could not answer)
+    launches_per_step = 1 + nch * (3 + (6 if fused else 2))
     for _ in range(max(3, warmup)):
         step()
     torch.cuda.synchronize()
@@ -599,7 +609,8 @@ def prefill_measure(args, wl, dev, gen_pool, steps, warmup, dist=None, ws=1, wan
     if ws > 1:
         ms = max_over_ranks(ms, dist, dev)
     out = {"ms": ms, "steps": steps, "pairs": pairs, "flops": flops, "score_ms": score_ms, "stages_us": stages_us,
-           "launches_per_step": launches_per_step, "clocks": clk.summary("score, stage and timed passes")}
+           "launches_per_step": launches_per_step, "clocks": clk.summary("score, stage and timed passes"),
+           "inputs": (kd, qd, wd, nd), "idx": idx}
 
     if want_e2e:
         # end to end: every step copies the cache, the queries, their weights and n from pinned host
@@ -697,14 +708,14 @@ def run_prefill(args, wl):
         if ws > 1:
             dist.init_process_group("nccl", device_id=dev, timeout=__import__("datetime").timedelta(seconds=120))
         r = prefill_measure(args, wl, dev, gen_pool, args.steps, args.warmup, dist if ws > 1 else None, ws,
-                            want_dense=not args.no_dense, want_cpu=rank == 0)
+                            want_dense=not args.no_dense, want_cpu=rank == 0, fused=args.fused)
     if rank == 0:
         e = r["e2e"]
         line = {
             "metric": METRIC, "value": r["pairs"] * ws * args.steps / (r["ms"] / 1000.0), "unit": UNIT,
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup, "ms_per_step": r["ms"] / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": _prefill_config(wl, ws, args),
+            "config": dict(_prefill_config(wl, ws, args), fused=bool(args.fused)),
             "roofline": _prefill_roofline(wl, r),
             "e2e": {"value": r["pairs"] * ws * e["steps"] / (e["ms"] / 1000.0), "unit": UNIT,
                     "h2d_bytes_per_step": e["h2d"], "d2h_bytes_per_step": e["d2h"]},
@@ -1029,6 +1040,18 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
                 pre["dense_same_inputs"] = r["dense"]
             if "cpu_baseline" in r:
                 pre["cpu_baseline"] = r["cpu_baseline"]
+            # the same step with scoring and selection fused (no score rows), on the same inputs
+            f = prefill_measure(args, W.WORKLOADS[3], dev, gen_pool, max(1, min(args.steps, 5)), 2,
+                                want_e2e=False, want_dense=False, want_cpu=False, fused=True, inputs=r["inputs"])
+            same = bool(torch.equal(torch.sort(f["idx"], dim=1).values, torch.sort(r["idx"], dim=1).values))
+            pre["fused"] = {"ms_per_step": f["ms"] / f["steps"],
+                            "value": f["pairs"] * f["steps"] / (f["ms"] / 1000.0),
+                            "scoring_and_selection_ms_per_step": f["score_ms"],
+                            "effective_TFLOPs": f["flops"] / (f["score_ms"] / 1000.0) / 1e12,
+                            "stages_us": f["stages_us"], "gpu_launches_per_step": f["launches_per_step"],
+                            "matches_unfused": same, "clocks": f["clocks"],
+                            "speedup_over_unfused_step": r["ms"] / r["steps"] / (f["ms"] / f["steps"])}
+            del r, f
             legs["prefill"] = pre
         except Exception as exc:  # a failed leg is reported, the headline stands
             legs["prefill"] = {"error": f"{type(exc).__name__}: {exc}"}
@@ -1054,6 +1077,8 @@ def main():
     ap.add_argument("--no-dense", action="store_true")
     ap.add_argument("--no-legs", action="store_true",
                     help="decode: skip the prefill and GLM-5-shaped decode legs that follow the main line")
+    ap.add_argument("--fused", action="store_true",
+                    help="prefill main line: score and select each chunk with misa_score_topk_fused (no score rows)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
     ap.add_argument("--paged", type=int, default=64, metavar="PAGE_SIZE",

@@ -76,7 +76,8 @@ typedef enum {
   MISA_OP_BLOCK_FILTER = 5,
   MISA_OP_ROUTE_PAGED = 6,
   MISA_OP_SCORE_TOPK_PAGED = 7,
-  MISA_OP_RERANK_PAGED = 8
+  MISA_OP_RERANK_PAGED = 8,
+  MISA_OP_SCORE_TOPK_FUSED = 9
 } misa_op;
 
 /* Largest k' accepted by misa_hier_rerank (its candidates are ranked in shared memory). */
@@ -276,6 +277,26 @@ misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* po
                                    const int32_t* n, const int32_t* cand, int T, int L, int H_I,
                                    int d, int kp, int topk, int dtype, int32_t* idx,
                                    float* score_opt, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * misa_score_topk for queries that share one bf16 key cache (chunked prefill), without writing
+ * score rows ("Sparse Token Scoring": the top-k tokens by the routed score).  The tensor-core
+ * scorer first scores every 32nd tile of 128 keys of each prefix; each query's cut is placed on that
+ * sample (the expected number of sampled scores above the k-th, plus three standard deviations and
+ * a margin); a second pass over every key appends only the scores at or above the cut to a list of
+ * 4k entries per query, from which the top-k is selected.  A query whose list holds fewer than
+ * min(k, n_t) entries or overflowed is redone exactly on the device by the unfused scorer and
+ * selection, so the selected set is always misa_score_topk's.
+ *   k  : one shared cache [L, d] (k_seq_stride 0), bf16 like q
+ *   ws : misa_workspace_bytes(MISA_OP_SCORE_TOPK_FUSED, T, L, H_I, 0, h, topk, 0) bytes (it also
+ *        holds score rows for the queries that are redone)
+ * Requires 4 * topk <= 16384 (else MISA_ERR_UNSUPPORTED); other arguments and outputs as
+ * misa_score_topk.
+ */
+misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, const int32_t* n,
+                                  const int32_t* heads, int T, int L, int H_I, int d, int h,
+                                  int topk, int dtype, int32_t* idx, float* score_opt, void* ws,
+                                  size_t ws_bytes, void* stream);
 
 /*
  * Device-side status of the calls made so far on the current device.  The tensor-core scoring

@@ -175,7 +175,6 @@ misa_status misa_device_check(void) {
 
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
   (void)h;
-  (void)topk;
   switch (op) {
     case MISA_OP_ROUTE:
       return route_ws(T, L, H_I, B);
@@ -194,6 +193,8 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
       return score_topk_paged_ws(T, L);
     case MISA_OP_RERANK_PAGED:
       return rerank_paged_ws(T, kp);
+    case MISA_OP_SCORE_TOPK_FUSED:
+      return T > 0 && L > 0 && misa::fused_cap(topk) > 0 ? align_up(misa::fused_ws_bytes(T, L, topk)) : 0;
     default:
       return 0;
   }
@@ -493,6 +494,28 @@ misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* po
   misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, nullptr, T, pool_rows, H_I, H_I, rows, kp, F, kp,
                       nullptr, s);
   misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, nullptr, idx, score_opt, s);
+  return launch_status();
+}
+
+misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, const int32_t* n,
+                                  const int32_t* heads, int T, int L, int H_I, int d, int h, int topk, int dtype,
+                                  int32_t* idx, float* score_opt, void* ws, size_t ws_bytes, void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, 0);
+  if (st != MISA_OK) return st;
+  if (!heads && T > 0) return MISA_ERR_INVALID_ARG;
+  if (h < 1 || h > H_I || topk < 1) return MISA_ERR_INVALID_ARG;
+  if (dtype != MISA_BF16 || misa::fused_cap(topk) == 0) return MISA_ERR_UNSUPPORTED;
+  if (T == 0) return MISA_OK;
+  if (!idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < misa::fused_ws_bytes(T, L, topk) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  const cudaStream_t s = as_stream(stream);
+  float* rows = nullptr;
+  int64_t ld = 0;
+  if (!misa::launch_score_topk_fused(q, w, k, n, heads, T, L, H_I, h, topk, ws, idx, score_opt, &rows, &ld, s)) {
+    // the tensor-core scorer cannot take these inputs: every query by the unfused path
+    misa::launch_scores(misa::DType::BF16, q, w, k, 0, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, nullptr, s);
+    misa::launch_topk_rows(rows, ld, nullptr, 0, n, T, L, topk, nullptr, idx, score_opt, s);
+  }
   return launch_status();
 }
 

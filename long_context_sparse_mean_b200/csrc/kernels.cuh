@@ -48,9 +48,12 @@ struct ListState {
   uint2* list;       // [T][cap] (order key, token)
   int cap;
   int topk;
+  // Lists without score rows behind them (fused prefill): a row the list cannot answer is not
+  // selected; redo[t] receives n_t for it (0 for the rows answered) and the caller redoes it.
+  int32_t* redo = nullptr;
 };
-size_t list_state_bytes(int T);
-ListState list_state(void* ws, int T, int topk);
+size_t list_state_bytes(int T, int cap = kListCap);
+ListState list_state(void* ws, int T, int topk, int cap = kListCap);
 // cnt = kNoList for every row (scores written without lists).
 void mark_no_lists(const ListState& l, int T, cudaStream_t s);
 
@@ -81,7 +84,34 @@ bool read_and_clear_bad_ids_block_filter(unsigned int* out);
 // candidate lists launch_scores appended for these rows (or nullptr).  One CTA per row, no
 // workspace.  Output order within a row is not specified.
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T,
-                      int L, int topk, const ListState* lst, int32_t* idx, float* score_opt, cudaStream_t s);
+                      int L, int topk, const ListState* lst, int32_t* idx, float* score_opt, cudaStream_t s,
+                      const int32_t* only = nullptr);
+// only (optional): rows with only[t] <= 0 are skipped and keep their outputs.
+
+// The tensor-core scorer's other output modes (score_tc.cu), for queries sharing one bf16 cache:
+// every tile_stride-th key tile of each prefix (tiles 0, S, 2S, ...), written packed (sampled tile i
+// of row t goes to sample[t, 128 i .. 128 i + 127]); or no score row at all, every score at or above
+// tau[t] appended as (order key, token) to query t's list (lists [T][cap], lcnt[t] counting every
+// such score, also past cap).  False (nothing launched) when the inputs do not suit the kernel.
+bool launch_scores_tc_sample(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads,
+                             int T, int L, int H_I, int h, int tile_stride, float* sample, int64_t ld,
+                             cudaStream_t s);
+bool launch_scores_tc_compact(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads,
+                              int T, int L, int H_I, int h, const float* tau, uint2* lists, uint32_t* lcnt, int cap,
+                              cudaStream_t s);
+
+// Routed scoring + top-k for queries sharing one bf16 cache without score rows (fused.cu): a sample
+// pass over every kFusedStride-th key tile, a cut per query from its sample, the compact pass, the
+// selection from the lists, and an exact redo of the queries whose list could not answer.
+constexpr int kFusedStride = 32;
+int fused_cap(int topk);                    // list entries per query (0: topk unsupported)
+int64_t fused_sample_cols(int L);           // packed sample columns of a cache of L keys
+size_t fused_ws_bytes(int T, int L, int topk);
+// False (after launching part of it) when the tensor-core scorer cannot take these inputs; the
+// caller then runs the unfused path on the same workspace's score rows.
+bool launch_score_topk_fused(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads,
+                             int T, int L, int H_I, int h, int topk, void* ws, int32_t* idx, float* score_opt,
+                             float** rows_out, int64_t* ld_out, cudaStream_t s);
 
 // Top-k of short candidate lists in shared memory (no workspace): values F[t, P], ids cand[t, P].
 size_t topk_cand_smem(int P);

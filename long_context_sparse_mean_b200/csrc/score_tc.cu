@@ -67,7 +67,8 @@ constexpr int kOffPre = kOffOut + kEpiWarps * kStageOutFloats * 4; // [kMaxBlock
 constexpr int kOffW = kOffPre + ((kMaxBlocks + 1) * 4 + 15) / 16 * 16;  // [2][256] f32
 constexpr int kOffHead = kOffW + 2 * kTileCols * 4;                // [2][256] i32
 constexpr int kOffN = kOffHead + 2 * kTileCols * 4;                // [2][32] i32 prefix lengths
-constexpr int kOffBar = kOffN + 2 * 32 * 4;                        // mbarriers
+constexpr int kOffTau = kOffN + 2 * 32 * 4;                        // [2][32] f32 cuts (compact mode)
+constexpr int kOffBar = kOffTau + 2 * 32 * 4;                      // mbarriers
 constexpr int kNumBars = 2 * kStages + 2 + 2 + 2 + 2 + 1;
 constexpr int kOffMisc = kOffBar + kNumBars * 8;                   // tmem base, abort, scan scratch
 constexpr int kSmemBytes = kOffMisc + 4 * 36 + 1024;               // + alignment slack
@@ -107,13 +108,25 @@ __device__ __forceinline__ void give_up(volatile int* abort) {
   atomicExch(&g_tc_status, 1);
 }
 
-template <int MP>
+// Output modes of the scorer:
+//   kRows     score rows: out[t, s] for s < n_t (entries past the prefix are not written)
+//   kSample   every tile_stride-th key tile only (tiles 0, S, 2S, ...), packed: sampled tile i of a
+//             row goes to columns [128 i, 128 i + 128) of out
+//   kCompact  no score row: each score at or above tau[t] is appended as (order key, token) to the
+//             query's candidate list (lists [T][cap]); lcnt[t] counts every such score, also past
+//             cap (then the list is incomplete and the caller redoes the query)
+enum { kRows = 0, kSample = 1, kCompact = 2 };
+
+template <int MP, int FM>
 __global__ void __launch_bounds__(kThreads, 1)
     score_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap omap,
                     int tma_store, const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                     const int32_t* __restrict__ n, const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
-                    float* __restrict__ out, int64_t ld) {
+                    float* __restrict__ out, int64_t ld, int tile_stride, const float* __restrict__ tau,
+                    uint2* __restrict__ lists, uint32_t* __restrict__ lcnt, int cap) {
   constexpr int QT = kTileCols / MP;  // queries per block
+  // key tile of work tile `tile` (the sample takes every tile_stride-th)
+  auto key_tile = [&](uint32_t tile) -> int { return FM == kSample ? (int)tile * tile_stride : (int)tile; };
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint32_t* pre = reinterpret_cast<uint32_t*>(sm + kOffPre);
@@ -121,6 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* shead = reinterpret_cast<int*>(sm + kOffHead);  // sorted head of every B row
   int* hraw = shead + kTileCols;                         // the same, as given
   int* nsm = reinterpret_cast<int*>(sm + kOffN);         // n_t of the block's queries
+  float* tsm = reinterpret_cast<float*>(sm + kOffTau);   // tau_t of the block's queries (compact mode)
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile int* abort = reinterpret_cast<volatile int*>(misc + 1);
@@ -130,7 +144,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NB = (T + QT - 1) / QT;
 
   // ---- key tiles per query block and their prefix ----
-  tc::block_tile_prefix(NB, QT, T, kTileKeys, [&](int t) { return clamp_len(__ldg(n + t), L); }, pre, warp_tot);
+  tc::block_tile_prefix(NB, QT, T, kTileKeys, [&](int t) {
+    const int nt = clamp_len(__ldg(n + t), L);
+    if (FM != kSample) return nt;
+    const int kt = (nt + kTileKeys - 1) / kTileKeys;                   // key tiles of the prefix
+    return (kt + tile_stride - 1) / tile_stride * kTileKeys;           // sampled tiles, as a length
+  }, pre, warp_tot);
   const uint64_t W = pre[NB];
   const uint32_t a = (uint32_t)(W * blockIdx.x / gridDim.x);
   const uint32_t e = (uint32_t)(W * (blockIdx.x + 1) / gridDim.x);
@@ -233,8 +252,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
         if (lane == 0) tc::mbar_arrive_relaxed(bars.ae(ab));
         if (active) {
-          const int s0w = (int)tile * kTileKeys + lq * 32;
+          const int s0w = key_tile(tile) * kTileKeys + lq * 32;  // first key of the warp's 32
           const int s = s0w + lane;
+          const int c0w = FM == kSample ? (int)tile * kTileKeys + lq * 32 : s0w;  // its output column
           float sum[QW];
 #pragma unroll
           for (int l = 0; l < QW; ++l) {
@@ -244,7 +264,29 @@ __global__ void __launch_bounds__(kThreads, 1)
               for (int x = 0; x < st; ++x) acc[l * NF + x] = __fadd2_rn(acc[l * NF + x], acc[l * NF + x + st]);
             sum[l] = acc[l * NF].x + acc[l * NF].y;
           }
-          if (s0w + 32 <= nmin) {  // the whole block: one TMA store
+          if (FM == kCompact) {
+            // one ballot per query, then lane l reserves query l's slots: the warp's atomics to its
+            // QW lists go out as one instruction, one round trip per tile
+            const float* tr = tsm + pb * 32 + col0 / MP;
+            unsigned mk[QW];
+            uint32_t want = 0;
+#pragma unroll
+            for (int l = 0; l < QW; ++l) {
+              mk[l] = __ballot_sync(0xffffffffu, s < nr[l] && sum[l] >= tr[l]);
+              if (lane == l) want = (uint32_t)__popc(mk[l]);
+            }
+            uint32_t got = 0;
+            if (lane < QW && want) got = atomicAdd(lcnt + tq + lane, want);
+            const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+            for (int l = 0; l < QW; ++l) {
+              const uint32_t base = __shfl_sync(0xffffffffu, got, l);
+              if ((mk[l] >> lane) & 1u) {
+                const uint32_t pos = base + (uint32_t)__popc(mk[l] & below);
+                if (pos < (uint32_t)cap) lists[(int64_t)(tq + l) * cap + pos] = make_uint2(order_key(sum[l]), (uint32_t)s);
+              }
+            }
+          } else if (s0w + 32 <= nmin) {  // the whole block: one TMA store
             if (lane == 0) tc::bulk_wait_read_all();  // the previous store has read the buffer
             __syncwarp();
 #pragma unroll
@@ -252,13 +294,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-              tc::tma_store_2d(&omap, s0w, tq, tc::smem_u32(stage_out));
+              tc::tma_store_2d(&omap, c0w, tq, tc::smem_u32(stage_out));
               tc::bulk_commit();
             }
           } else {
 #pragma unroll
             for (int l = 0; l < QW; ++l)
-              if (s < nr[l]) out[(int64_t)(tq + l) * ld + s] = sum[l];
+              if (s < nr[l]) out[(int64_t)(tq + l) * ld + c0w + lane] = sum[l];
           }
         }
       }
@@ -317,6 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int qi = lane; qi < QT; qi += 32) {
         const int t = t0 + qi;
         nsm[pb * 32 + qi] = t < T ? clamp_len(__ldg(n + t), L) : 0;
+        if (FM == kCompact) tsm[pb * 32 + qi] = t < T ? __ldg(tau + t) : INFINITY;
       }
       // weights; padding slots repeat the query's first head with weight 0
       for (int idx = lane; idx < kTileCols; idx += 32) {
@@ -361,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               break;
             }
             tc::mbar_arrive_expect_tx(bars.kf(st), kStageBytes);
-            tc::tma_load_2d(kbase + st * kStageBytes, &kmap, half * 64, (int)tile * kTileKeys, bars.kf(st));
+            tc::tma_load_2d(kbase + st * kStageBytes, &kmap, half * 64, key_tile(tile) * kTileKeys, bars.kf(st));
           }
         }
       }
@@ -428,24 +471,73 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int MP>
+// Output buffers of one scorer call: out [T, ld] with out_cols columns written at most (score
+// rows, or the packed sample), or the candidate lists of compact mode.
+struct TcOut {
+  float* out;
+  int64_t ld;
+  int64_t out_cols;
+  int tile_stride;
+  const float* tau;
+  uint2* lists;
+  uint32_t* lcnt;
+  int cap;
+};
+
+template <int MP, int FM>
 void launch_mp(const CUtensorMap& map, const __nv_bfloat16* q, const float* w, const int32_t* n,
-               const int32_t* heads, int h, int H_I, int L, int T, float* out, int64_t ld, cudaStream_t s) {
+               const int32_t* heads, int h, int H_I, int L, int T, const TcOut& o, cudaStream_t s) {
   constexpr int QT = kTileCols / MP;
   constexpr int QW = (MP > 64 ? 128 : 64) / MP;  // rows of an epilogue warp's store box
-  cudaFuncSetAttribute(score_tc_kernel<MP>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  cudaFuncSetAttribute(score_tc_kernel<MP, FM>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   const int grid = sm_count();
   const int per_launch = kMaxBlocks * QT;
   for (int t0 = 0; t0 < T; t0 += per_launch) {
     const int Tc = T - t0 < per_launch ? T - t0 : per_launch;
-    float* o = out + (int64_t)t0 * ld;
+    float* ot = FM == kCompact ? nullptr : o.out + (int64_t)t0 * o.ld;
     CUtensorMap omap;
-    const bool tma = tmap_f32_rows(&omap, o, (uint64_t)L, (uint64_t)Tc, (uint64_t)ld, 32, QW);
+    const bool tma = FM != kCompact &&
+                     tmap_f32_rows(&omap, ot, (uint64_t)o.out_cols, (uint64_t)Tc, (uint64_t)o.ld, 32, QW);
     if (!tma) memset(&omap, 0, sizeof(omap));
-    score_tc_kernel<MP><<<grid, kThreads, kSmemBytes, s>>>(
+    score_tc_kernel<MP, FM><<<grid, kThreads, kSmemBytes, s>>>(
         map, omap, tma ? 1 : 0, q + (int64_t)t0 * H_I * kD, w + (int64_t)t0 * H_I, n + t0,
-        heads ? heads + (int64_t)t0 * h : nullptr, h, H_I, L, Tc, o, ld);
+        heads ? heads + (int64_t)t0 * h : nullptr, h, H_I, L, Tc, ot, o.ld, o.tile_stride,
+        FM == kCompact ? o.tau + t0 : nullptr, FM == kCompact ? o.lists + (int64_t)t0 * o.cap : nullptr,
+        FM == kCompact ? o.lcnt + t0 : nullptr, o.cap);
   }
+}
+
+template <int FM>
+bool launch_tc_mode(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads, int T,
+                    int L, int H_I, int h, const TcOut& o, cudaStream_t s) {
+  if (T <= 0 || L <= 0) return true;
+  if (reinterpret_cast<uintptr_t>(q) & 15) return false;
+  CUtensorMap map;
+  if (!tmap_rows128_bf16(&map, k, (uint64_t)L, kTileKeys)) return false;
+  const int m = heads ? h : H_I;
+  int mp = 8;
+  while (mp < m) mp <<= 1;
+  const auto* qb = static_cast<const __nv_bfloat16*>(q);
+  switch (mp) {
+    case 8:
+      launch_mp<8, FM>(map, qb, w, n, heads, h, H_I, L, T, o, s);
+      break;
+    case 16:
+      launch_mp<16, FM>(map, qb, w, n, heads, h, H_I, L, T, o, s);
+      break;
+    case 32:
+      launch_mp<32, FM>(map, qb, w, n, heads, h, H_I, L, T, o, s);
+      break;
+    case 64:
+      launch_mp<64, FM>(map, qb, w, n, heads, h, H_I, L, T, o, s);
+      break;
+    case 128:
+      launch_mp<128, FM>(map, qb, w, n, heads, h, H_I, L, T, o, s);
+      break;
+    default:
+      return false;
+  }
+  return true;
 }
 
 }  // namespace
@@ -461,34 +553,23 @@ int sm_count() {
 
 bool launch_scores_tc(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads, int T,
                       int L, int H_I, int h, float* out, int64_t ld, cudaStream_t s) {
-  if (T <= 0 || L <= 0) return true;
-  if (reinterpret_cast<uintptr_t>(q) & 15) return false;
-  CUtensorMap map;
-  if (!tmap_rows128_bf16(&map, k, (uint64_t)L, kTileKeys)) return false;
-  const int m = heads ? h : H_I;
-  int mp = 8;
-  while (mp < m) mp <<= 1;
-  const auto* qb = static_cast<const __nv_bfloat16*>(q);
-  switch (mp) {
-    case 8:
-      launch_mp<8>(map, qb, w, n, heads, h, H_I, L, T, out, ld, s);
-      break;
-    case 16:
-      launch_mp<16>(map, qb, w, n, heads, h, H_I, L, T, out, ld, s);
-      break;
-    case 32:
-      launch_mp<32>(map, qb, w, n, heads, h, H_I, L, T, out, ld, s);
-      break;
-    case 64:
-      launch_mp<64>(map, qb, w, n, heads, h, H_I, L, T, out, ld, s);
-      break;
-    case 128:
-      launch_mp<128>(map, qb, w, n, heads, h, H_I, L, T, out, ld, s);
-      break;
-    default:
-      return false;
-  }
-  return true;
+  const TcOut o{out, ld, L, 1, nullptr, nullptr, nullptr, 0};
+  return launch_tc_mode<kRows>(q, w, k, n, heads, T, L, H_I, h, o, s);
+}
+
+bool launch_scores_tc_sample(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads,
+                             int T, int L, int H_I, int h, int tile_stride, float* sample, int64_t ld,
+                             cudaStream_t s) {
+  const int64_t cols = (int64_t)((L + kTileKeys - 1) / kTileKeys + tile_stride - 1) / tile_stride * kTileKeys;
+  const TcOut o{sample, ld, cols, tile_stride, nullptr, nullptr, nullptr, 0};
+  return launch_tc_mode<kSample>(q, w, k, n, heads, T, L, H_I, h, o, s);
+}
+
+bool launch_scores_tc_compact(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads,
+                              int T, int L, int H_I, int h, const float* tau, uint2* lists, uint32_t* lcnt, int cap,
+                              cudaStream_t s) {
+  const TcOut o{nullptr, 0, 0, 1, tau, lists, lcnt, cap};
+  return launch_tc_mode<kCompact>(q, w, k, n, heads, T, L, H_I, h, o, s);
 }
 
 int read_and_clear_tc_status() {

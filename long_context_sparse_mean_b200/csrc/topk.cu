@@ -324,10 +324,12 @@ __device__ void select_list_linear(uint2* list, int c, uint32_t need, uint32_t l
 
 // Rows of scores [T, ld]; ids == nullptr: entry p < n_t is token p; otherwise entry p < P is token
 // ids[t P + p] (empty when outside [0, n_t)), and P <= LIST.  lists (optional): the candidate lists
-// the decode scoring kernel appended, [T][lcap] (key, token) with lcnt[t] entries (kNoList: the row
-// has none) and every key at or above lcut[t] among them; a row whose list has at least topk
-// entries at or above lcut[t] and lost none past lcap is selected from those entries, any other row
-// takes the exact path.
+// a scoring kernel appended, [T][lcap] (key, token) with lcnt[t] entries (kNoList: the row has
+// none) and every key at or above lcut[t] among them; a row whose list has at least
+// min(topk, n_t) entries at or above lcut[t] and lost none past lcap is selected from those
+// entries.  Any other row takes the exact path over its scores, or, with no score rows behind the
+// lists (scores == nullptr), is left unselected with redo[t] = n_t (redo[t] = 0 for the rows
+// answered).  only (optional): rows with only[t] <= 0 are skipped and keep their outputs.
 template <int NT, int LIST, int MINB>
 __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restrict__ scores, int64_t ld,
                                                             const int32_t* __restrict__ ids_all, int P,
@@ -335,28 +337,31 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
                                                             int32_t* __restrict__ idx, float* __restrict__ score_opt,
                                                             const uint2* __restrict__ lists,
                                                             const uint32_t* __restrict__ lcnt,
-                                                            const uint32_t* __restrict__ lcut, int lcap) {
+                                                            const uint32_t* __restrict__ lcut, int lcap,
+                                                            int32_t* __restrict__ redo,
+                                                            const int32_t* __restrict__ only) {
   extern __shared__ uint2 list[];  // [LIST]
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t cnt[2];
   __shared__ uint32_t mm[2];
   const int t = blockIdx.x;
+  if (only && only[t] <= 0) return;
   const int nt = clamp_len(n[t], L);
-  const float* row = scores + (int64_t)t * ld;
+  const float* row = scores ? scores + (int64_t)t * ld : nullptr;
   const int32_t* ids = ids_all ? ids_all + (int64_t)t * P : nullptr;
   const int np = ids ? P : nt;  // entries of the row
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
   const int tid = threadIdx.x;
-  if (!ids && nt <= topk) {  // every prefix token is selected
+  if (!ids && nt <= topk && row) {  // every prefix token is selected
     for (int a = tid; a < topk; a += NT) {
       oi[a] = a < nt ? a : -1;
       if (ov) ov[a] = a < nt ? row[a] : 0.f;
     }
     return;
   }
-  const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+  const bool vec = row && (reinterpret_cast<uintptr_t>(row) & 15) == 0;
   if (tid < 2) cnt[tid] = 0;
   if (tid == 0) {
     mm[0] = 0xffffffffu;
@@ -364,12 +369,14 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
   }
 
   // ---- 1. candidates ----
+  // the answer needs min(topk, n_t) entries (a prefix of at most topk keys is selected whole)
+  const uint32_t need = (uint32_t)((!ids && nt < topk) ? nt : topk);
   bool exact = false, listed = false;
   uint32_t c_in = 0;
   if (lists) {
     c_in = __ldcg(lcnt + t);
     if (c_in != kNoList) {
-      listed = c_in >= (uint32_t)topk && c_in <= (uint32_t)min(lcap, LIST);
+      listed = c_in >= need && c_in <= (uint32_t)min(lcap, LIST);
       exact = !listed;  // too few entries, or entries dropped past the list's end
     }
   }
@@ -390,8 +397,8 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
     }
     block_min_max(lo, hi, mm);
     __syncthreads();
-    // fewer than k entries at or above the cut: the list cannot hold the answer
-    exact = cnt[0] < (uint32_t)topk;
+    // fewer than the needed entries at or above the cut: the list cannot hold the answer
+    exact = cnt[0] < need;
     listed = !exact;
     __syncthreads();
   } else if (!exact) {
@@ -419,12 +426,14 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
   } else {
     __syncthreads();
   }
+  if (redo && tid == 0) redo[t] = exact ? nt : 0;
+  if (exact && !row) return;  // no score rows behind the list: the caller redoes this row
 
   // ---- 2. selection from the candidates ----
   if (!exact) {
     __syncthreads();
     const uint32_t c = cnt[0];
-    if (!listed && np <= LIST && c <= (uint32_t)topk) {  // every valid entry is selected
+    if ((!listed || need < (uint32_t)topk) && np <= LIST && c <= (uint32_t)topk) {  // every entry is selected
       for (uint32_t i = tid; i < (uint32_t)topk; i += NT) {
         oi[i] = i < c ? (int32_t)list[i].y : -1;
         if (ov) ov[i] = i < c ? key_to_float(list[i].x) : 0.f;
@@ -499,12 +508,14 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
 
 template <int NT, int LIST, int MINB>
 void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
-                     int topk, int32_t* idx, float* score_opt, const ListState* lst, cudaStream_t s) {
+                     int topk, int32_t* idx, float* score_opt, const ListState* lst, const int32_t* only,
+                     cudaStream_t s) {
   const size_t smem = sizeof(uint2) * (size_t)LIST;
   cudaFuncSetAttribute(row_topk_kernel<NT, LIST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt,
                                                       lst ? lst->list : nullptr, lst ? lst->cnt : nullptr,
-                                                      lst ? lst->cutkey : nullptr, lst ? lst->cap : 0);
+                                                      lst ? lst->cutkey : nullptr, lst ? lst->cap : 0,
+                                                      lst ? lst->redo : nullptr, only);
 }
 
 struct SmemItems {
@@ -565,18 +576,18 @@ namespace {
 size_t al(size_t x) { return (x + 255) / 256 * 256; }
 }  // namespace
 
-size_t list_state_bytes(int T) {
+size_t list_state_bytes(int T, int cap) {
   if (T <= 0) return 0;
-  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(uint2) * (size_t)T * kListCap);
+  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(uint2) * (size_t)T * cap);
 }
 
-ListState list_state(void* ws, int T, int topk) {
+ListState list_state(void* ws, int T, int topk, int cap) {
   char* p = static_cast<char*>(ws);
   ListState l;
   l.cnt = reinterpret_cast<uint32_t*>(p);
   l.cutkey = l.cnt + T;
   l.list = reinterpret_cast<uint2*>(p + al(sizeof(uint32_t) * 2 * (size_t)T));
-  l.cap = kListCap;
+  l.cap = cap;
   l.topk = topk;
   return l;
 }
@@ -586,12 +597,13 @@ void mark_no_lists(const ListState& l, int T, cudaStream_t s) {
 }
 
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,
-                      int topk, const ListState* lst, int32_t* idx, float* score_opt, cudaStream_t s) {
+                      int topk, const ListState* lst, int32_t* idx, float* score_opt, cudaStream_t s,
+                      const int32_t* only) {
   if (T <= 0) return;
-  if (!ids && !lst && T >= kRowKernelMinRows)
-    launch_row_topk<512, 8192, 2>(scores, ld, nullptr, 0, n, T, L, topk, idx, score_opt, nullptr, s);
+  if (!ids && (!lst || lst->cap <= 8192) && T >= kRowKernelMinRows)
+    launch_row_topk<512, 8192, 2>(scores, ld, nullptr, 0, n, T, L, topk, idx, score_opt, lst, only, s);
   else
-    launch_row_topk<1024, kRowListLarge, 1>(scores, ld, ids, P, n, T, L, topk, idx, score_opt, lst, s);
+    launch_row_topk<1024, kRowListLarge, 1>(scores, ld, ids, P, n, T, L, topk, idx, score_opt, lst, only, s);
 }
 
 size_t topk_cand_smem(int P) { return sizeof(uint32_t) * 2 * (size_t)(P + P / 32 + 2); }
