@@ -6,10 +6,10 @@
 // path writes every score row (4 bytes per scored pair) and reads it back to select; here:
 //   1. the tensor-core scorer scores every kFusedStride-th key tile of each prefix (the sample,
 //      1/32 of the work), written packed;
-//   2. fused_cut_kernel places each query's cut from its sample: the lower edge of the bin (4096
-//      bins over the sample's key range) holding the sample entry whose rank is the expected
-//      sample count above the k-th score plus three standard deviations and a margin; prefixes of
-//      at most cap keys take every key;
+//   2. fused_cut_kernel places each query's cut from its sample: the smallest score of the linear
+//      bin (4096 bins over the sample's score range) holding the sample entry whose rank is the
+//      expected sample count above the k-th score plus three standard deviations and a margin;
+//      prefixes of at most cap keys take every key;
 //   3. the scorer runs over every key tile in compact mode: each score at or above its query's cut
 //      is appended as (order key, token) to the query's list of cap = 4k entries, no score row;
 //   4. the per-row top-k selects each query from its list;
@@ -72,14 +72,15 @@ __global__ void __launch_bounds__(kCutThreads) fused_cut_kernel(const int32_t* _
     hi = max(hi, k);
   }
   block_min_max(lo, hi, mm);
-  for (int b = threadIdx.x; b < kHistBins; b += kCutThreads) hist[b] = 0;
   __syncthreads();
   lo = mm[0];
-  const uint32_t range = mm[1] - lo;
-  const int sh = range >= 4096u ? 32 - __clz(range) - 12 : 0;
-  for (int i = threadIdx.x; i < ns; i += kCutThreads) hist_add(hist, (order_key(__ldg(st + i)) - lo) >> sh, true);
+  hi = mm[1];
   __syncthreads();
-  const uint32_t cut = lo + block_bucket_bits(hist, kHistBins, sh, 0u, rank, scratch).prefix;
+  const uint32_t cut = linear_cut(
+      [&](auto f) {
+        for (int i = threadIdx.x; i < ns; i += kCutThreads) f(order_key(__ldg(st + i)));
+      },
+      lo, hi, rank, hist, mm, scratch);
   if (threadIdx.x == 0) {
     tau[t] = key_to_float(cut);
     cutkey[t] = cut;

@@ -21,11 +21,11 @@
 //       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
 //       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
 //       For a top-k of the scores it can also build each query's candidate list: after a run of
-//       a query's tiles the CTA places a cut on the run's scores (a histogram over their key
-//       range; the run's share of the top-k, 1.5 times over, plus 16 entries), appends the run's
-//       entries at or above it to the query's list (one global atomic per run) and raises the
-//       query's cut key, so the selection ranks a list of about 1.5 k entries instead of
-//       sweeping the row (three passes over the run's scores, read back from L2).
+//       a query's tiles the CTA places a cut on the run's scores (4096 bins linear in the score;
+//       the run's share of the top-k, 1.5 times over, plus 16 entries), appends the run's entries
+//       at or above it to the query's list (one global atomic per run) and raises the query's
+//       cut key, so the selection ranks a list of about 1.5 k entries instead of sweeping the
+//       row (three passes over the run's scores, read back from L2).
 //   score_grid_kernel     one CTA per (query, chunk of positions): shared caches when the
 //       tensor-core kernel (score_tc.cu, which takes shared bf16 caches) cannot run, and more
 //       queries than the persistent schedule takes.
@@ -99,38 +99,65 @@ __device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat
   __syncthreads();
 }
 
+// Calls f(order key, position) for every score of p[0, len) the calling thread owns, reading from L2
+// with eight 16-byte loads in flight per thread (scalar loads when p is not 16-byte aligned).
+template <class F>
+__device__ __forceinline__ void run_each(const float* p, int len, F&& f) {
+  constexpr int U = 8;
+  int done = 0;
+  if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
+    const int n4 = len / 4;
+    const float4* p4 = reinterpret_cast<const float4*>(p);
+    for (int j0 = threadIdx.x; j0 < n4; j0 += U * kScoreThreads) {
+      float4 x[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * kScoreThreads;
+        x[u] = j < n4 ? __ldcg(p4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u * kScoreThreads;
+        if (j < n4) {
+          f(order_key(x[u].x), 4 * j);
+          f(order_key(x[u].y), 4 * j + 1);
+          f(order_key(x[u].z), 4 * j + 2);
+          f(order_key(x[u].w), 4 * j + 3);
+        }
+      }
+    }
+    done = n4 * 4;
+  }
+#pragma unroll 8
+  for (int i = done + threadIdx.x; i < len; i += kScoreThreads) f(order_key(__ldcg(p + i)), i);
+}
+
 // Candidate list of one run of a query's scores, [s0, s1) of row `ot` (written by this CTA): a cut
-// r-th from the top of the run (r = its share of the top-k, 1.5 times over, plus 16), placed with a
-// 4096-bin histogram over the run's key range [kmin, kmax] (every thread's keys, reduced here) at
-// the lower edge of the bin holding the r-th largest; every entry at or above the cut is appended
-// to the query's list lt (one global atomic for the run) and the query's cut key is raised to it.
-// Prefixes of at most cap keys keep every entry.  All threads of the CTA call it.
+// r-th from the top of the run (r = its share of the top-k, 1.5 times over, plus 16), the smallest
+// key of the linear bin holding the r-th largest (linear_cut over the run's score range, from every
+// thread's smallest and largest key); every entry at or above the cut is appended to the query's
+// list lt (one global atomic for the run) and the query's cut key is raised to it.  Prefixes of at
+// most cap keys keep every entry.  All threads of the CTA call it.
 __device__ __forceinline__ void segment_list(const float* ot, int t, int s0, int s1, int nt, uint32_t kmin,
                                              uint32_t kmax, uint32_t* hist, uint32_t* mm, uint32_t* scratch,
                                              uint32_t* sbase, uint2* lt, uint32_t* lcnt, uint32_t* lcut, int cap,
                                              int topk) {
   const int len = s1 - s0;
+  const float* p = ot + s0;
   block_min_max(kmin, kmax, mm);
   __syncthreads();  // also: the run's scores are visible to the whole CTA
+  const uint32_t lo = mm[0], hi = mm[1];
+  __syncthreads();
   uint32_t cut = 0u;  // order key; 0 keeps every entry
   if (nt > cap) {
     const float share = 1.5f * (float)topk * (float)len / (float)nt;
     const int r = min(len, (int)ceilf(share) + 16);
-    if (r < len) {
-      const uint32_t lo = mm[0], range = mm[1] - mm[0];
-      const int sh = range >= 4096u ? 32 - __clz(range) - 12 : 0;
-      for (int b = threadIdx.x; b < kHistBins; b += kScoreThreads) hist[b] = 0;
-      __syncthreads();
-#pragma unroll 4
-      for (int i = threadIdx.x; i < len; i += kScoreThreads)
-        hist_add(hist, (order_key(__ldcg(ot + s0 + i)) - lo) >> sh, true);
-      __syncthreads();
-      cut = lo + block_bucket_bits(hist, kHistBins, sh, 0u, (uint32_t)r, scratch).prefix;
-    }
+    if (r < len)
+      cut = linear_cut([&](auto f) { run_each(p, len, [&](uint32_t k, int) { f(k); }); }, lo, hi, (uint32_t)r, hist,
+                       mm, scratch);
   }
   uint32_t mine = 0;
-#pragma unroll 4
-  for (int i = threadIdx.x; i < len; i += kScoreThreads) mine += order_key(__ldcg(ot + s0 + i)) >= cut;
+  run_each(p, len, [&](uint32_t k, int) { mine += k >= cut; });
   uint32_t total;
   uint32_t slot = block_exclusive_scan(mine, scratch, &total);
   if (threadIdx.x == 0) {
@@ -139,14 +166,12 @@ __device__ __forceinline__ void segment_list(const float* ot, int t, int s0, int
   }
   __syncthreads();
   slot += *sbase;
-#pragma unroll 4
-  for (int i = threadIdx.x; i < len; i += kScoreThreads) {
-    const uint32_t k = order_key(__ldcg(ot + s0 + i));
+  run_each(p, len, [&](uint32_t k, int i) {
     if (k >= cut) {
       if (slot < (uint32_t)cap) lt[slot] = make_uint2(k, (uint32_t)(s0 + i));
       ++slot;
     }
-  }
+  });
   if (threadIdx.x == 0) {
     mm[0] = 0xffffffffu;
     mm[1] = 0u;

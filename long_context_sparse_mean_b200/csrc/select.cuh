@@ -144,10 +144,50 @@ __device__ __forceinline__ void block_min_max(uint32_t lo, uint32_t hi, uint32_t
   }
 }
 
-// Cut from a sample of keys: the lower edge of the bin (4096 bins over the sample's key range) holding the rank-th largest sample key, so at
-// least `rank` sample keys are at or above the returned value.  PER keys per thread; hist: 4096
-// words of shared memory; mm: 2 words holding 0xffffffff and 0 on entry (and again on return);
-// scratch: 35 words.  Every thread calls it.
+// Linear bin of an order key's score: 4096 bins over [vlo, vlo + 4096 / scale].  Non-decreasing in
+// the score (the subtraction and the multiplication by a positive scale keep order under
+// round-to-nearest), so every entry of a higher bin is at least every entry of a lower one.
+__device__ __forceinline__ uint32_t linear_bin(uint32_t key, float vlo, float scale) {
+  const float x = (key_to_float(key) - vlo) * scale;
+  return (uint32_t)min(__float2int_rz(x), kHistBins - 1);
+}
+
+// Cut for the r-th largest of a set of keys spread over the block: each(f) calls f(key) for every
+// key of the calling thread; lo and hi are the block's smallest and largest key.  Returns the
+// smallest key of the linear bin (4096 bins between the scores of lo and hi) that holds the r-th
+// largest key, so at least r keys are at or above it and at most one bin's worth more; a set of
+// one value (or a range too wide to bin) returns lo, which keeps every key.  hist: 4096 words of
+// shared memory; mm: 2 words; scratch: 35 words.  Every thread calls it.
+template <class Each>
+__device__ __forceinline__ uint32_t linear_cut(Each each, uint32_t lo, uint32_t hi, uint32_t r, uint32_t* hist,
+                                               uint32_t* mm, uint32_t* scratch) {
+  const float vlo = key_to_float(lo), vhi = key_to_float(hi);
+  const float scale = (float)kHistBins / (vhi - vlo);
+  if (!(vhi > vlo) || !(scale > 0.f) || !(scale < 3.0e38f)) return lo;
+  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  each([&](uint32_t k) { hist_add(hist, linear_bin(k, vlo, scale), true); });
+  __syncthreads();
+  const uint32_t b = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch).prefix;
+  if (threadIdx.x == 0) mm[0] = 0xffffffffu;
+  __syncthreads();
+  uint32_t mn = 0xffffffffu;
+  each([&](uint32_t k) {
+    if (linear_bin(k, vlo, scale) == b) mn = min(mn, k);
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+  if ((threadIdx.x & 31) == 0) atomicMin(&mm[0], mn);
+  __syncthreads();
+  const uint32_t cut = mm[0];
+  __syncthreads();
+  return cut;
+}
+
+// Cut from a sample of keys: the smallest score of the linear bin holding the rank-th largest
+// sample key (linear_cut), so at least `rank` sample keys are at or above the returned value.  PER
+// keys per thread; hist: 4096 words of shared memory; mm: 2 words holding 0xffffffff and 0 on entry
+// (and again on return); scratch: 35 words.  Every thread calls it.
 template <int PER>
 __device__ __forceinline__ float sample_cut(const uint32_t (&sk)[PER], uint32_t rank, uint32_t* hist, uint32_t* mm,
                                             uint32_t* scratch);
@@ -167,22 +207,22 @@ __device__ __forceinline__ float sample_cut(const uint32_t (&sk)[PER], uint32_t 
     shi = max(shi, sk[u]);
   }
   block_min_max(slo, shi, mm);
-  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
   __syncthreads();
   slo = mm[0];
-  const uint32_t srange = mm[1] - slo;
-  const int ssh = srange >= 4096u ? 32 - __clz(srange) - 12 : 0;
-#pragma unroll
-  for (int u = 0; u < PER; ++u) hist_add(hist, (sk[u] - slo) >> ssh, true);
+  shi = mm[1];
   __syncthreads();
-  const Bucket cut = block_bucket_bits(hist, kHistBins, ssh, 0u, rank, scratch);
+  const uint32_t cut = linear_cut(
+      [&](auto f) {
+#pragma unroll
+        for (int u = 0; u < PER; ++u) f(sk[u]);
+      },
+      slo, shi, rank, hist, mm, scratch);
   if (threadIdx.x == 0) {
     mm[0] = 0xffffffffu;
     mm[1] = 0u;
   }
   __syncthreads();
-  // keys >= slo + cut.prefix are the scores >= this value
-  return key_to_float(slo + cut.prefix);
+  return key_to_float(cut);  // the scores >= this value are the keys >= cut
 }
 
 // Radix select over m items given by acc.key(i) (0 = absent) and acc.id(i); acc.value(i) is the

@@ -248,14 +248,6 @@ __device__ __forceinline__ void warp_rank_write(const uint2* list, int n, uint32
   }
 }
 
-// Linear bin of a score: 4096 bins over [vlo, vlo + 4096 / scale].  Non-decreasing in v (the
-// subtraction and the multiplication by a positive scale keep order under round-to-nearest), so
-// every entry of a higher bin is at least every entry of a lower one.
-__device__ __forceinline__ uint32_t linear_bin(uint32_t key, float vlo, float scale) {
-  const float x = (key_to_float(key) - vlo) * scale;
-  return (uint32_t)min(__float2int_rz(x), kHistBins - 1);
-}
-
 // Top `need` of the c list entries (c >= need) in shared memory, written to oi/ov [0, need).
 // lo/hi: the smallest and largest key in the list.  One histogram of 4096 bins linear in the score
 // finds the bin of the need-th entry; entries of higher bins go out directly, the boundary bin's
