@@ -5,8 +5,8 @@
 One step is one decode step of MISA-dagger over a batch of sequences (default: 32 sequences x
 131072 keys, H_I = 64, d = 128, B = 128, h = 8, k' = 8192, k = 2048):
     route (block-pooled router, top-h heads; the block holding the newest key is averaged from the
-    keys) -> routed token scores, building candidate lists for the top-k' -> top-k' candidates ->
-    dense re-rank of the candidates -> top-k.
+    keys) -> routed token scores -> candidate lists of the score rows and top-k' -> dense re-rank
+    of the candidates (tensor cores) -> top-k.
 (A block is pooled once the prefix has moved past it, once every B = 128 steps of a sequence; the
 step does not repeat it.)
 Inputs are seeded synthetic tensors resident in HBM (the key cache of 1 GiB per GPU is larger
@@ -207,8 +207,8 @@ def _config(wl, extra=None):
     c = {"workload": wl.name, "T_per_gpu": wl.T, "L": wl.L, "H_I": wl.H_I, "d": wl.d, "B": wl.B, "h": wl.h,
          "kp": wl.kp, "topk": wl.topk, "accumulate": "f32",
          "l2": f"inputs larger than L2 ({wl.T * wl.L * wl.d * 2 / 2**30:.2f} GiB key cache per GPU)",
-         "step": ("route + routed scores (with candidate lists) + top-k' + dense re-rank + top-k" if wl.kp
-                  else "route + routed scores (with candidate lists) + top-k")}
+         "step": ("route + routed scores + candidate lists and top-k' + dense re-rank + top-k" if wl.kp
+                  else "route + routed scores + candidate lists and top-k")}
     if extra:
         c.update(extra)
     return c
@@ -762,12 +762,12 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
 
     def score():
-        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kk, select_ws=sel_ws)
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
 
     def step():
         route()
         score()
-        M.misa_topk_select(scores, nd, kk, idx=idx, want_vals=False, ws=sel_ws, ws_prepared=True)
+        M.misa_topk_select(scores, nd, kk, idx=idx, want_vals=False, ws=sel_ws)
 
     def dense():
         M.dsa_dense_topk(qd, wd, kd, nd, kk, idx=didx, want_vals=False, ws=wsp)
@@ -794,10 +794,9 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     hbm, kind = _peaks()
     alg = T * (L * d * 2 + h * d * 2 + h * 4)
     res = {"workload": wl.name, "T": T, "L": L, "H_I": wl.H_I, "B": B, "h": h, "topk": kk,
-           "step": "route + routed scores (with candidate lists) + top-k",
+           "step": "route + routed scores + candidate lists and top-k",
            "ms_per_step": ms, "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 4,
-           "roofline": {"bound": "hbm", "kernel": "routed scoring call: score_persist_kernel building the "
-                                                  "candidate lists (one memset before it)",
+           "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                         "achieved": alg / (score_ms / 1000.0) / 1e9, "peak": hbm, "peak_kind": kind,
                         "unit": "GB/s", "frac": alg / (score_ms / 1000.0) / 1e9 / hbm,
                         "algorithmic_bytes_per_launch": alg, "avg_launch_ms": score_ms},
@@ -864,18 +863,18 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
-    # kernels per step: router, routed scorer (building the candidate lists), top-k' (one CTA per
-    # row), re-rank scorer, top-k of the candidates (plus two small memsets)
-    launches_per_step = 5
+    # kernels per step: router, routed scorer, candidate lists and top-k' (one CTA per row), re-rank
+    # scorer, top-k of the candidates (plus two small memsets)
+    launches_per_step = 6
 
     def route():
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
 
     def score():
-        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores, select_topk=kp, select_ws=sel_ws)
+        M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
 
     def select():
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws, ws_prepared=True)
+        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws)
 
     def rerank():
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
@@ -982,14 +981,13 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU",
                                    "cuda_graph": not args.no_graph}),
-            "roofline": {"bound": "hbm", "kernel": "routed scoring call: score_persist_kernel building the "
-                                                   "candidate lists (one memset before it)",
+            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                          "frac": achieved / hbm,
                          "traffic": _traffic(TRAFFIC, "bytes_per_key", T * L),
                          "algorithmic_bytes_per_launch": alg_bytes, "avg_launch_ms": score_avg,
-                         "timing": "the call replayed back to back as a CUDA graph, CUDA events on its stream; "
-                                   "its time includes the candidate lists (per-run cuts and appends)"},
+                         "timing": "the scoring call (one launch) replayed back to back as a CUDA graph, CUDA "
+                                   "events on its stream"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,

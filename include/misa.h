@@ -133,15 +133,16 @@ misa_status misa_route(const void* q, const float* w, const void* k, int64_t k_s
  *   select_ws, select_ws_bytes, select_topk : optional (NULL, 0, 0).  A workspace of
  *              misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes in which the call also
  *              prepares a top-select_topk selection of these scores; pass the same workspace to
- *              misa_topk_select with ws_prepared = 1.  For one bf16 cache per query the scoring
- *              kernel builds a candidate list of up to 16384 entries per query as it goes: every
- *              run of a query's keys it scores keeps the entries at or above a cut placed on the
- *              run's own scores (its share of select_topk, 1.5 times over) and raises the query's
- *              cut key to that cut, so every score at or above the query's cut key is listed.  The
- *              selection ranks those entries and takes an exact pass over the score row whenever
- *              they cannot hold the answer (fewer than select_topk, or the list overflowed), so
- *              the result never depends on how the cuts fell.  Other caches, and batches whose
- *              lists would not fit, leave no list and the selection works from the scores alone.
+ *              misa_topk_select with ws_prepared = 1.  For fewer than 256 rows longer than
+ *              16384 entries it builds a candidate list per query right after the scores: one
+ *              CTA per row places the row's cut from a sample of its scores (256 evenly spaced
+ *              runs of 8; the rank of the expected count above the select_topk-th score plus
+ *              three standard deviations), then CTAs over chunks of 8192 scores append every
+ *              score at or above it.  The selection ranks those entries and takes an exact pass
+ *              over the score row whenever they cannot hold the answer (fewer than select_topk,
+ *              or the list overflowed), so the result never depends on where the cut fell.
+ *              Shorter rows, many rows and rows whose lists would not fit get no list and are
+ *              selected from the scores.
  */
 misa_status misa_token_scores(const void* q, const float* w, const void* k, int64_t k_seq_stride,
                               const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
@@ -155,9 +156,9 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
  *   score_opt   : out [T, topk] fp32 score of each selected token (0 for padding), or NULL
  *   ws          : misa_workspace_bytes(MISA_OP_TOPK_SELECT, T, L, ...) bytes
  *   ws_prepared : 1 if misa_token_scores already prepared ws for these scores and this topk
- * Scores must be finite.  One CTA per row selects; without ws_prepared it finds the row's
- * candidates itself (a sampled cut and a pass over the row), with it it starts from the candidate
- * list misa_token_scores left in ws.  Both give the same set.
+ * Scores must be finite.  Without ws_prepared the call first builds the candidate lists of long
+ * rows itself (as misa_token_scores does); then one CTA per row selects, from its list or, for rows
+ * without one, from a sampled cut and a pass over the row.  Both give the same set.
  */
 misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32_t* n, int T,
                              int L, int topk, int32_t* idx, float* score_opt, void* ws,
@@ -299,9 +300,10 @@ misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, 
                                   size_t ws_bytes, void* stream);
 
 /*
- * Device-side status of the calls made so far on the current device.  The tensor-core scoring
- * kernel (queries sharing one bf16 cache: k_seq_stride 0) pipelines its copies and MMAs through
- * shared-memory barriers; every wait on them is bounded (about one second).  A wait that runs
+ * Device-side status of the calls made so far on the current device.  The tensor-core kernels
+ * (scoring and routing queries that share one bf16 cache, and the re-rank of gathered candidates)
+ * pipeline their copies and MMAs through shared-memory barriers; every wait on them is bounded
+ * (about one second).  A wait that runs
  * out makes the kernel stop early, leaving its outputs incomplete, and records the event in a
  * per-device status word.  This call waits for all work on the device to finish
  * (cudaDeviceSynchronize), then reads and clears that word (and, in the bounds-checked build,

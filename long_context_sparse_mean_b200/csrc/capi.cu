@@ -60,9 +60,6 @@ size_t select_bytes(int T, int P) {
   return align_up(misa::list_state_bytes(T));
 }
 
-// Per-query bf16 caches take the candidate-list top-k: the scorer builds the lists.
-bool list_path(int dtype, int64_t k_seq_stride) { return dtype == MISA_BF16 && k_seq_stride != 0; }
-
 // misa_score_topk / dsa_dense_topk: [scores][selection]
 size_t scores_ws(int T, int L) {
   if (T <= 0 || L <= 0) return 0;
@@ -145,7 +142,7 @@ namespace {
 bool read_bad_ids(unsigned int* out) {
   for (int i = 0; i < misa::kBadIdKinds; ++i) out[i] = 0;
   return misa::read_and_clear_bad_ids_score(out) && misa::read_and_clear_bad_ids_paged(out) &&
-         misa::read_and_clear_bad_ids_block_filter(out);
+         misa::read_and_clear_bad_ids_block_filter(out) && misa::read_and_clear_bad_ids_rerank_tc(out);
 }
 }  // namespace
 
@@ -167,9 +164,10 @@ misa_status misa_device_check(void) {
   if (cudaDeviceSynchronize() != cudaSuccess) return MISA_ERR_CUDA;
   const int v = misa::read_and_clear_tc_status();
   const int u = misa::read_and_clear_route_tc_status();
+  const int x = misa::read_and_clear_rerank_tc_status();
   unsigned int bad[misa::kBadIdKinds];
-  if (v < 0 || u < 0 || !read_bad_ids(bad)) return MISA_ERR_CUDA;
-  if (v || u) return MISA_ERR_DEVICE_TIMEOUT;
+  if (v < 0 || u < 0 || x < 0 || !read_bad_ids(bad)) return MISA_ERR_CUDA;
+  if (v || u || x) return MISA_ERR_DEVICE_TIMEOUT;
   return (bad[0] || bad[1] || bad[2]) ? MISA_ERR_BAD_INDEX : MISA_OK;
 }
 
@@ -253,15 +251,9 @@ misa_status misa_token_scores(const void* q, const float* w, const void* k, int6
   if (select_ws && (select_ws_bytes < select_bytes(T, L) || !aligned(select_ws))) return MISA_ERR_WORKSPACE;
   const cudaStream_t s = as_stream(stream);
   const int m = heads ? h : H_I;
-  if (!select_ws) {
-    misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0, scores,
-                        ld_scores, nullptr, s);
-    return launch_status();
-  }
-  const misa::ListState lst = misa::list_state(select_ws, T, select_topk);
-  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0,
-                                          scores, ld_scores, list_path(dtype, k_seq_stride) ? &lst : nullptr, s);
-  if (!listed) misa::mark_no_lists(lst, T, s);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, m, nullptr, 0, scores, ld_scores,
+                      s);
+  if (select_ws) misa::launch_list_build(scores, ld_scores, n, T, L, misa::list_state(select_ws, T, select_topk), s);
   return launch_status();
 }
 
@@ -273,8 +265,9 @@ misa_status misa_topk_select(const float* scores, int64_t ld_scores, const int32
   if (!scores || !n || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < select_bytes(T, L) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   const misa::ListState lst = misa::list_state(ws, T, topk);
-  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, ws_prepared ? &lst : nullptr, idx, score_opt,
-                         as_stream(stream));
+  const cudaStream_t s = as_stream(stream);
+  if (!ws_prepared) misa::launch_list_build(scores, ld_scores, n, T, L, lst, s);
+  misa::launch_topk_rows(scores, ld_scores, nullptr, 0, n, T, L, topk, &lst, idx, score_opt, s);
   return launch_status();
 }
 
@@ -300,10 +293,9 @@ misa_status misa_score_topk(const void* q, const float* w, const void* k, int64_
   }
   const cudaStream_t s = as_stream(stream);
   const misa::ListState lst = misa::list_state(p, T, topk);
-  const bool lp = list_path(dtype, k_seq_stride);
-  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0,
-                                          buf, ld, lp ? &lst : nullptr, s);
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, buf, ld, s);
+  misa::launch_list_build(buf, ld, n, T, L, lst, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, &lst, idx, score_opt, s);
   return launch_status();
 }
 
@@ -318,7 +310,7 @@ misa_status misa_hier_rerank(const void* q, const float* w, const void* k, int64
   if (!cand || !idx) return MISA_ERR_INVALID_ARG;
   if (!ws || ws_bytes < rerank_ws(T, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
   float* F = static_cast<float*>(ws);
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp, nullptr,
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp,
                       as_stream(stream));
   misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, nullptr, idx, score_opt, as_stream(stream));
   return launch_status();
@@ -338,10 +330,9 @@ misa_status dsa_dense_topk(const void* q, const float* w, const void* k, int64_t
   const int64_t ld = score_ld(L);
   const misa::ListState lst = misa::list_state(p + scores_part(T, L), T, topk);
   const cudaStream_t s = as_stream(stream);
-  const bool lp = list_path(dtype, k_seq_stride);
-  const bool listed = misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr,
-                                          0, buf, ld, lp ? &lst : nullptr, s);
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, listed ? &lst : nullptr, idx, score_opt, s);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, nullptr, 0, buf, ld, s);
+  misa::launch_list_build(buf, ld, n, T, L, lst, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, &lst, idx, score_opt, s);
   return launch_status();
 }
 
@@ -383,7 +374,7 @@ misa_status misa_block_filter_topk(const void* q, const float* w, const void* k,
                             h, S, ldS, Mt, s);
   misa::launch_topk_rows(S, ldS, nullptr, 0, Mt, T, M, m, nullptr, blocks, nullptr, s);
   misa::launch_expand_blocks(blocks, m, n, T, L, B, rows, s);
-  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, P, F, P, nullptr, s);
+  misa::launch_scores(to_dtype(dtype), q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, P, F, P, s);
   misa::launch_topk_rows(F, P, rows, P, n, T, L, topk, nullptr, idx, score_opt, s);
   return launch_status();
 }
@@ -463,9 +454,10 @@ misa_status misa_score_topk_paged(const void* q, const float* w, const void* poo
   const int pool_rows = (int)(num_pages * page_size);
   const cudaStream_t s = as_stream(stream);
   misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, nullptr, L, rows, n_phys, s);
-  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, heads, T, pool_rows, H_I, h, rows, L, buf, ld, nullptr,
-                      s);
-  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, nullptr, idx, score_opt, s);
+  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, heads, T, pool_rows, H_I, h, rows, L, buf, ld, s);
+  const misa::ListState lst = misa::list_state(p, T, topk);
+  misa::launch_list_build(buf, ld, n, T, L, lst, s);
+  misa::launch_topk_rows(buf, ld, nullptr, 0, n, T, L, topk, &lst, idx, score_opt, s);
   return launch_status();
 }
 
@@ -491,8 +483,7 @@ misa_status misa_hier_rerank_paged(const void* q, const float* w, const void* po
   const int pool_rows = (int)(num_pages * page_size);
   const cudaStream_t s = as_stream(stream);
   misa::launch_paged_rows(page_table, max_pages, num_pages, page_size, n, T, L, cand, kp, rows, n_phys, s);
-  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, nullptr, T, pool_rows, H_I, H_I, rows, kp, F, kp,
-                      nullptr, s);
+  misa::launch_scores(to_dtype(dtype), q, w, pool, 0, n_phys, nullptr, T, pool_rows, H_I, H_I, rows, kp, F, kp, s);
   misa::launch_topk_rows(F, kp, cand, kp, n, T, L, topk, nullptr, idx, score_opt, s);
   return launch_status();
 }
@@ -513,7 +504,7 @@ misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, 
   int64_t ld = 0;
   if (!misa::launch_score_topk_fused(q, w, k, n, heads, T, L, H_I, h, topk, ws, idx, score_opt, &rows, &ld, s)) {
     // the tensor-core scorer cannot take these inputs: every query by the unfused path
-    misa::launch_scores(misa::DType::BF16, q, w, k, 0, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, nullptr, s);
+    misa::launch_scores(misa::DType::BF16, q, w, k, 0, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, s);
     misa::launch_topk_rows(rows, ld, nullptr, 0, n, T, L, topk, nullptr, idx, score_opt, s);
   }
   return launch_status();

@@ -6,13 +6,13 @@
 // path writes every score row (4 bytes per scored pair) and reads it back to select; here:
 //   1. the tensor-core scorer scores every kFusedStride-th key tile of each prefix (the sample,
 //      1/32 of the work), written packed;
-//   2. fused_cut_kernel places each query's cut from its sample: the smallest score of the linear
-//      bin (4096 bins over the sample's score range) holding the sample entry whose rank is the
-//      expected sample count above the k-th score plus three standard deviations and a margin;
-//      prefixes of at most cap keys take every key;
+//   2. fused_cut_kernel places each query's cut from its sample, one warp per query: the lower
+//      edge of the narrow bin (rounds of 1024 bins over the key range) holding the sample entry
+//      whose rank is the expected sample count above the k-th score plus three standard
+//      deviations and a margin; prefixes of at most cap keys take every key;
 //   3. the scorer runs over every key tile in compact mode: each score at or above its query's cut
 //      is appended as (order key, token) to the query's list of cap = 4k entries, no score row;
-//   4. the per-row top-k selects each query from its list;
+//   4. one warp per query selects from its list (list_select_warp_kernel);
 //   5. a query whose list holds fewer than min(k, n_t) entries or lost some past cap is redone
 //      exactly: the rows scorer and the per-row top-k, restricted to those queries (both launches
 //      find nothing to do when every list answered).
@@ -22,27 +22,28 @@
 #include <math.h>
 
 #include "kernels.cuh"
+#include "warp_select.cuh"
 
 namespace misa {
 
 namespace {
 
-constexpr int kCutThreads = 256;
-
 size_t al(size_t x) { return (x + 255) / 256 * 256; }
 
-// One CTA per query: cut[t] (and the list's cut key) from the packed sample row of query t.
-__global__ void __launch_bounds__(kCutThreads) fused_cut_kernel(const int32_t* __restrict__ n, int L, int topk,
-                                                                int cap, const float* __restrict__ sample,
-                                                                int64_t ld_sample, float* __restrict__ tau,
-                                                                uint32_t* __restrict__ cutkey) {
-  __shared__ uint32_t hist[kHistBins];
-  __shared__ uint32_t scratch[35];
-  __shared__ uint32_t mm[2];
-  const int t = blockIdx.x;
+// One warp per query: cut[t] (and the list's cut key) from the packed sample row of query t, the
+// lower edge of the narrow bin holding the sample entry of the given rank (warp_sample_cut).
+__global__ void __launch_bounds__(32 * kSelWarps, 3) fused_cut_kernel(const int32_t* __restrict__ n, int L, int T,
+                                                                   int topk, int cap,
+                                                                   const float* __restrict__ sample,
+                                                                   int64_t ld_sample, float* __restrict__ tau,
+                                                                   uint32_t* __restrict__ cutkey) {
+  __shared__ uint32_t hist[kSelWarps][kWarpBinWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelWarps + warp;
+  if (t >= T) return;  // uniform across the warp
   const int nt = clamp_len(n[t], L);
   if (nt <= cap) {  // the list takes every key
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
       tau[t] = -INFINITY;
       cutkey[t] = 0u;
     }
@@ -54,34 +55,15 @@ __global__ void __launch_bounds__(kCutThreads) fused_cut_kernel(const int32_t* _
   const float mean = (float)topk * (float)ns / (float)nt;
   const uint32_t rank = (uint32_t)(mean + 3.f * sqrtf(mean) + 8.f);
   if (rank > (uint32_t)ns) {  // the sample cannot place the cut: no list, the query is redone
-    if (threadIdx.x == 0) {
+    if (lane == 0) {
       tau[t] = INFINITY;
       cutkey[t] = 0xffffffffu;
     }
     return;
   }
   const float* st = sample + (int64_t)t * ld_sample;
-  if (threadIdx.x == 0) {
-    mm[0] = 0xffffffffu;
-    mm[1] = 0u;
-  }
-  uint32_t lo = 0xffffffffu, hi = 0u;
-  for (int i = threadIdx.x; i < ns; i += kCutThreads) {
-    const uint32_t k = order_key(__ldg(st + i));
-    lo = min(lo, k);
-    hi = max(hi, k);
-  }
-  block_min_max(lo, hi, mm);
-  __syncthreads();
-  lo = mm[0];
-  hi = mm[1];
-  __syncthreads();
-  const uint32_t cut = linear_cut(
-      [&](auto f) {
-        for (int i = threadIdx.x; i < ns; i += kCutThreads) f(order_key(__ldg(st + i)));
-      },
-      lo, hi, rank, hist, mm, scratch);
-  if (threadIdx.x == 0) {
+  const uint32_t cut = warp_sample_cut(ns, [&](int i) { return order_key(__ldg(st + i)); }, rank, hist[warp]);
+  if (lane == 0) {
     tau[t] = key_to_float(cut);
     cutkey[t] = cut;
   }
@@ -90,7 +72,6 @@ __global__ void __launch_bounds__(kCutThreads) fused_cut_kernel(const int32_t* _
 struct FusedWs {
   ListState lst;
   float* tau;      // [T]
-  int32_t* redo;   // [T] n_t of a query to redo, else 0
   float* sample;   // [T][fused_sample_cols(L)]
   int64_t ld_sample;
   float* rows;     // [T][ld] score rows of redone queries
@@ -105,14 +86,11 @@ FusedWs carve(void* ws, int T, int L, int topk) {
   p += list_state_bytes(T, cap);
   f.tau = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * (size_t)T);
-  f.redo = reinterpret_cast<int32_t*>(p);
-  p += al(sizeof(int32_t) * (size_t)T);
   f.ld_sample = fused_sample_cols(L);
   f.sample = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * (size_t)T * f.ld_sample);
   f.ld = (L + 3) / 4 * 4;
   f.rows = reinterpret_cast<float*>(p);
-  f.lst.redo = f.redo;
   return f;
 }
 
@@ -131,7 +109,7 @@ int64_t fused_sample_cols(int L) {
 size_t fused_ws_bytes(int T, int L, int topk) {
   if (T <= 0 || L <= 0 || fused_cap(topk) == 0) return 0;
   const int64_t ld = (L + 3) / 4 * 4;
-  return list_state_bytes(T, fused_cap(topk)) + 2 * al(sizeof(float) * (size_t)T) +
+  return list_state_bytes(T, fused_cap(topk)) + al(sizeof(float) * (size_t)T) +
          al(sizeof(float) * (size_t)T * fused_sample_cols(L)) + al(sizeof(float) * (size_t)T * ld);
 }
 
@@ -144,13 +122,14 @@ bool launch_score_topk_fused(const void* q, const float* w, const void* k, const
   if (T <= 0) return true;
   cudaMemsetAsync(f.lst.cnt, 0, sizeof(uint32_t) * 2 * (size_t)T, s);  // counts and cut keys
   if (!launch_scores_tc_sample(q, w, k, n, heads, T, L, H_I, h, kFusedStride, f.sample, f.ld_sample, s)) return false;
-  fused_cut_kernel<<<T, kCutThreads, 0, s>>>(n, L, topk, f.lst.cap, f.sample, f.ld_sample, f.tau, f.lst.cutkey);
+  fused_cut_kernel<<<(T + kSelWarps - 1) / kSelWarps, 32 * kSelWarps, 0, s>>>(n, L, T, topk, f.lst.cap, f.sample,
+                                                                              f.ld_sample, f.tau, f.lst.cutkey);
   if (!launch_scores_tc_compact(q, w, k, n, heads, T, L, H_I, h, f.tau, f.lst.list, f.lst.cnt, f.lst.cap, s))
     return false;
-  launch_topk_rows(nullptr, 0, nullptr, 0, n, T, L, topk, &f.lst, idx, score_opt, s);
+  launch_list_select_warp(n, T, L, topk, f.lst, idx, score_opt, s);
   // exact redo of the queries whose list could not answer: rows and selection restricted to them
-  if (!launch_scores_tc(q, w, k, f.redo, heads, T, L, H_I, h, f.rows, f.ld, s)) return false;
-  launch_topk_rows(f.rows, f.ld, nullptr, 0, f.redo, T, L, topk, nullptr, idx, score_opt, s, f.redo);
+  if (!launch_scores_tc(q, w, k, f.lst.redo, heads, T, L, H_I, h, f.rows, f.ld, s)) return false;
+  launch_topk_rows(f.rows, f.ld, nullptr, 0, f.lst.redo, T, L, topk, nullptr, idx, score_opt, s, f.lst.redo);
   return true;
 }
 

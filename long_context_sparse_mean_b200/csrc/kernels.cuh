@@ -37,47 +37,68 @@ void launch_route_finish(const __nv_bfloat16* q, const float* w, const __nv_bflo
                          int L, int H_I, int B, int h, const float* Sp, int nch, int tile, int32_t* heads,
                          float* r_opt, cudaStream_t s);
 
-// Candidate lists of a top-k over per-query caches, built by the scoring kernel while it scores
-// (select.cuh holds the sizes).  Every CTA that scores a run of a query's keys places a cut on the
-// run's own scores (its share of the top-k, 1.5 times over, plus 16), appends the run's entries at
-// or above the cut to the query's list and raises the query's cut key to its own cut; every key
-// at or above the query's final cut key is then in the list.
+// Candidate lists of a top-k over long score rows (select.cuh holds the sizes), built after the
+// scores are written: list_cut_kernel places each row's cut from a sample of its scores (the row
+// kernel's own sample and rank), list_sweep_kernel appends every entry at or above it with CTAs over
+// chunks of 8192 scores; the per-row selection ranks the list's entries at or above the row's cut.
 struct ListState {
   uint32_t* cnt;     // [T] entries appended (also past cap); kNoList: no list for this row
-  uint32_t* cutkey;  // [T] largest cut, as an order key, any CTA used for the row (right after cnt)
-  uint2* list;       // [T][cap] (order key, token)
+  uint32_t* cutkey;  // [T] the row's cut as an order key: every score at or above it is listed, and
+                     // every list entry is at or above it (right after cnt)
+  uint2* list;       // [T][stride] (order key, token); the first cap entries of a row are used
   int cap;
   int topk;
-  // Lists without score rows behind them (fused prefill): a row the list cannot answer is not
-  // selected; redo[t] receives n_t for it (0 for the rows answered) and the caller redoes it.
+  // [T] n_t of a row the list could not answer (0 for the rows answered): the row is redone from
+  // its scores (or, with no score rows behind the lists, by the caller)
   int32_t* redo = nullptr;
+  int64_t stride = kListCap;
+  // Lists built from score rows of fewer than 256 queries also keep a histogram of their entries:
+  // hist[t][b] counts the entries with min((key - cutkey[t]) >> shift[t], 4095) = b, so the
+  // selection finds the bin of the k-th entry without a pass of its own.  nullptr otherwise.
+  uint32_t* hist = nullptr;  // [T][4096]
+  uint32_t* shift = nullptr;  // [T]
 };
 size_t list_state_bytes(int T, int cap = kListCap);
 ListState list_state(void* ws, int T, int topk, int cap = kListCap);
-// cnt = kNoList for every row (scores written without lists).
+// cnt = kNoList for every row (no lists).
 void mark_no_lists(const ListState& l, int T, cudaStream_t s);
+// Builds the candidate lists of score rows [T, ld] (entries s < min(n_t, L)) for fewer than 256
+// rows longer than the list (per row: unless the sample cannot place the cut or the list is not
+// expected to fit; those rows get kNoList): the cut from the row kernel's sample by one CTA per
+// row, then list_sweep_kernel.  Otherwise marks every row as having none.  Returns whether the list
+// kernels ran.  list_state gives rows of 256 or more queries a cap of 8192.
+bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T, int L, const ListState& l,
+                       cudaStream_t s);
+// One warp per row: the top-k of each row's list (exact, ties to the lower token); rows the list
+// cannot answer get l.redo[t] = n_t and no output, the others l.redo[t] = 0.
+void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const ListState& l, int32_t* idx,
+                             float* score_opt, cudaStream_t s);
 
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
-// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].  With lst (bf16, one
-// cache per query, no gather: the persistent kernel, when the lists are expected to fit) the
-// candidate lists of a top-lst->topk are built too; returns whether they were (otherwise the
-// caller marks the rows as having none).
-bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+// position p of query t scores token rows[t*P + p] and writes out[t*ld + p].
+void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h,
-                   const int32_t* rows, int P, float* out, int64_t ld, const ListState* lst, cudaStream_t s);
+                   const int32_t* rows, int P, float* out, int64_t ld, cudaStream_t s);
 
 // Tensor-core scoring for queries sharing one bf16 key cache (k_seq_stride 0, no gather).  Returns
 // false without launching when the inputs do not suit it (alignment, no TMA encoder).
 bool launch_scores_tc(const void* q, const float* w, const void* k, const int32_t* n, const int32_t* heads, int T,
                       int L, int H_I, int h, float* out, int64_t ld, cudaStream_t s);
+// Dense scores of gathered candidates on the tensor cores (rerank_tc.cu): out[t, p] = F of token
+// cand[t, p] (0 when outside [0, n_t)) for p < P, bf16 q and k.  False (nothing launched) when the
+// inputs do not suit it (H_I a multiple of 16 in [16, 128], 16-byte aligned rows).
+bool launch_rerank_tc(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n, int T,
+                      int L, int H_I, const int32_t* cand, int P, float* out, int64_t ld, cudaStream_t s);
 // Reads and clears the status word the tensor-core kernels set when a bounded wait runs out.
 int read_and_clear_tc_status();
 int read_and_clear_route_tc_status();
+int read_and_clear_rerank_tc_status();
 // Bounds-checked build: add each file's counts of skipped out-of-range ids to out[kBadIdKinds] and
 // clear them (always true and nothing added in the normal build).
 bool read_and_clear_bad_ids_score(unsigned int* out);
 bool read_and_clear_bad_ids_paged(unsigned int* out);
 bool read_and_clear_bad_ids_block_filter(unsigned int* out);
+bool read_and_clear_bad_ids_rerank_tc(unsigned int* out);
 
 // Top-k of each row of scores [T, ld]: positions p < n_t are tokens p (ids == nullptr, P unused),
 // or positions p < P are tokens ids[t*P + p] (empty when outside [0, n_t); P <= 16384).  lst: the

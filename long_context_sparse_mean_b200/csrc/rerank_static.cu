@@ -78,7 +78,7 @@ extern "C" misa_status misa_hier_rerank_static(const void* q, const float* w, co
   if (st != MISA_OK) return st;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   const misa::DType dt = dtype == MISA_F32 ? misa::DType::F32 : misa::DType::BF16;
-  misa::launch_scores(dt, q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp, nullptr, s);
+  misa::launch_scores(dt, q, w, k, k_seq_stride, n, nullptr, T, L, H_I, H_I, cand, kp, F, kp, s);
   misa::launch_topk_cand(F, cand, n, T, L, kp, topk, idx, score_opt, s);
   return cudaGetLastError() == cudaSuccess ? MISA_OK : MISA_ERR_CUDA;
 }

@@ -20,12 +20,6 @@
 //       32 x 131072 keys: 178 us against 185 us for the grid kernel; an added bulk L2 prefetch
 //       of the rows four tiles ahead made it slower, 202 us, and was dropped.)
 //       The same schedule serves gathered candidate lists (re-rank): positions instead of rows.
-//       For a top-k of the scores it can also build each query's candidate list: after a run of
-//       a query's tiles the CTA places a cut on the run's scores (4096 bins linear in the score;
-//       the run's share of the top-k, 1.5 times over, plus 16 entries), appends the run's entries
-//       at or above it to the query's list (one global atomic per run) and raises the query's
-//       cut key, so the selection ranks a list of about 1.5 k entries instead of sweeping the
-//       row (three passes over the run's scores, read back from L2).
 //   score_grid_kernel     one CTA per (query, chunk of positions): shared caches when the
 //       tensor-core kernel (score_tc.cu, which takes shared bf16 caches) cannot run, and more
 //       queries than the persistent schedule takes.
@@ -99,100 +93,15 @@ __device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat
   __syncthreads();
 }
 
-// Calls f(order key, position) for every score of p[0, len) the calling thread owns, reading from L2
-// with eight 16-byte loads in flight per thread (scalar loads when p is not 16-byte aligned).
-template <class F>
-__device__ __forceinline__ void run_each(const float* p, int len, F&& f) {
-  constexpr int U = 8;
-  int done = 0;
-  if ((reinterpret_cast<uintptr_t>(p) & 15) == 0) {
-    const int n4 = len / 4;
-    const float4* p4 = reinterpret_cast<const float4*>(p);
-    for (int j0 = threadIdx.x; j0 < n4; j0 += U * kScoreThreads) {
-      float4 x[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * kScoreThreads;
-        x[u] = j < n4 ? __ldcg(p4 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int j = j0 + u * kScoreThreads;
-        if (j < n4) {
-          f(order_key(x[u].x), 4 * j);
-          f(order_key(x[u].y), 4 * j + 1);
-          f(order_key(x[u].z), 4 * j + 2);
-          f(order_key(x[u].w), 4 * j + 3);
-        }
-      }
-    }
-    done = n4 * 4;
-  }
-#pragma unroll 8
-  for (int i = done + threadIdx.x; i < len; i += kScoreThreads) f(order_key(__ldcg(p + i)), i);
-}
-
-// Candidate list of one run of a query's scores, [s0, s1) of row `ot` (written by this CTA): a cut
-// r-th from the top of the run (r = its share of the top-k, 1.5 times over, plus 16), the smallest
-// key of the linear bin holding the r-th largest (linear_cut over the run's score range, from every
-// thread's smallest and largest key); every entry at or above the cut is appended to the query's
-// list lt (one global atomic for the run) and the query's cut key is raised to it.  Prefixes of at
-// most cap keys keep every entry.  All threads of the CTA call it.
-__device__ __forceinline__ void segment_list(const float* ot, int t, int s0, int s1, int nt, uint32_t kmin,
-                                             uint32_t kmax, uint32_t* hist, uint32_t* mm, uint32_t* scratch,
-                                             uint32_t* sbase, uint2* lt, uint32_t* lcnt, uint32_t* lcut, int cap,
-                                             int topk) {
-  const int len = s1 - s0;
-  const float* p = ot + s0;
-  block_min_max(kmin, kmax, mm);
-  __syncthreads();  // also: the run's scores are visible to the whole CTA
-  const uint32_t lo = mm[0], hi = mm[1];
-  __syncthreads();
-  uint32_t cut = 0u;  // order key; 0 keeps every entry
-  if (nt > cap) {
-    const float share = 1.5f * (float)topk * (float)len / (float)nt;
-    const int r = min(len, (int)ceilf(share) + 16);
-    if (r < len)
-      cut = linear_cut([&](auto f) { run_each(p, len, [&](uint32_t k, int) { f(k); }); }, lo, hi, (uint32_t)r, hist,
-                       mm, scratch);
-  }
-  uint32_t mine = 0;
-  run_each(p, len, [&](uint32_t k, int) { mine += k >= cut; });
-  uint32_t total;
-  uint32_t slot = block_exclusive_scan(mine, scratch, &total);
-  if (threadIdx.x == 0) {
-    *sbase = atomicAdd(lcnt + t, total);
-    atomicMax(lcut + t, cut);
-  }
-  __syncthreads();
-  slot += *sbase;
-  run_each(p, len, [&](uint32_t k, int i) {
-    if (k >= cut) {
-      if (slot < (uint32_t)cap) lt[slot] = make_uint2(k, (uint32_t)(s0 + i));
-      ++slot;
-    }
-  });
-  if (threadIdx.x == 0) {
-    mm[0] = 0xffffffffu;
-    mm[1] = 0u;
-  }
-}
-
 template <int NG, bool GATHER>
 __global__ void __launch_bounds__(kScoreThreads, 2)
     score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                          const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                          const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
-                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld,
-                         uint2* __restrict__ lists, uint32_t* __restrict__ lcnt, uint32_t* __restrict__ lcut,
-                         int cap, int topk) {
-  // dynamic: [T + 1] flattened tile prefix, then (candidate lists) a 4096-bin histogram
-  extern __shared__ int tile_base[];
-  uint32_t* hist = reinterpret_cast<uint32_t*>(tile_base + ((T + 1 + 3) & ~3));
+                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld) {
+  extern __shared__ int tile_base[];  // [T + 1] flattened tile prefix
   __shared__ HeadStage<NG> st;
   __shared__ uint32_t wtot[35];
-  __shared__ uint32_t mm[2];
-  __shared__ uint32_t sbase;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
 
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
@@ -225,13 +134,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const int nt = clamp_len(n[t], L);
     const int npos = GATHER ? P : nt;
     const int32_t* rt = GATHER ? rows + (int64_t)t * P : nullptr;
-    uint32_t kmin = 0xffffffffu, kmax = 0u;  // order keys of the scores this thread writes (lists)
 
     __syncthreads();  // the previous segment's fragments are no longer read
-    if (threadIdx.x == 0) {
-      mm[0] = 0xffffffffu;
-      mm[1] = 0u;
-    }
     stage_query<NG>(st, q, w, heads, h, H_I, t);
     float wa[NG], wb[NG];
 #pragma unroll
@@ -286,11 +190,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       const int r = row_of(j) + g;
       if (c == 0 && r < npos) ot[r] = slo;
       if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
-      if (!GATHER && lists && c < 2 && r + 8 * c < npos) {
-        const uint32_t kk = order_key(c == 0 ? slo : shi);
-        kmin = min(kmin, kk);
-        kmax = max(kmax, kk);
-      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         RA[i] = NA[i];
@@ -299,8 +198,6 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       va = na;
       vb = nb;
     }
-    if (!GATHER && lists) segment_list(ot, t, first * kTileRows, min((first + ntile) * kTileRows, nt), nt, kmin,
-                                       kmax, hist, mm, wtot, &sbase, lists + (int64_t)t * cap, lcnt, lcut, cap, topk);
     pos = seg_end;
   }
 }
@@ -434,24 +331,19 @@ int num_sms() {
 template <int NG>
 void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const float* w, const void* k,
                  int64_t k_seq_stride, const int32_t* n, const int32_t* heads, int h, int H_I, int T, int L,
-                 const int32_t* rows, int P, float* out, int64_t ld, const ListState* lst) {
+                 const int32_t* rows, int P, float* out, int64_t ld) {
   auto qb = static_cast<const __nv_bfloat16*>(q);
   auto kb = static_cast<const __nv_bfloat16*>(k);
   if (persist) {
-    size_t smem = sizeof(int) * (size_t)((T + 1 + 3) & ~3);
-    if (lst) {
-      smem += sizeof(uint32_t) * kHistBins;
-      cudaMemsetAsync(lst->cnt, 0, sizeof(uint32_t) * 2 * (size_t)T, s);  // counts and cut keys
-    }
+    const size_t smem = sizeof(int) * ((size_t)T + 1);
     if (gather) {
       cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, nullptr, nullptr, nullptr, 0, 0);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld);
     } else {
       cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, lst ? lst->list : nullptr,
-          lst ? lst->cnt : nullptr, lst ? lst->cutkey : nullptr, lst ? lst->cap : 0, lst ? lst->topk : 0);
+          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
@@ -464,22 +356,14 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
   }
 }
 
-// Whether candidate lists of a top-k suit a launch: every CTA's run of a query adds up to 16
-// entries beyond its share of 1.5 k, so the expected list must stay well inside the cap.
-bool lists_fit(const ListState* lst, int T) {
-  if (!lst || T <= 0) return false;
-  const double ctas_per_query = (2.0 * num_sms() + T - 1) / T + 2.0;
-  return 1.5 * lst->topk + 16.0 * ctas_per_query <= 0.9 * lst->cap;
-}
-
 }  // namespace
 
-bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,
                    const int32_t* n, const int32_t* heads, int T, int L, int H_I, int h, const int32_t* rows,
-                   int P, float* out, int64_t ld, const ListState* lst, cudaStream_t s) {
-  if (T <= 0) return false;
+                   int P, float* out, int64_t ld, cudaStream_t s) {
+  if (T <= 0) return;
   const int npos = rows ? P : L;
-  if (npos <= 0) return false;
+  if (npos <= 0) return;
   const bool gather = rows != nullptr;
   if (dt == DType::F32) {
     const dim3 grid((npos + kRowsPerChunk - 1) / kRowsPerChunk, T);
@@ -496,19 +380,20 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
           static_cast<const float*>(q), w, static_cast<const float*>(k), k_seq_stride, n, heads, h, H_I, L, rows,
           P, out, ld);
     }
-    return false;
+    return;
   }
   // one shared cache: tensor-core contraction over blocks of queries
-  if (!gather && k_seq_stride == 0 && launch_scores_tc(q, w, k, n, heads, T, L, H_I, h, out, ld, s)) return false;
+  if (!gather && k_seq_stride == 0 && launch_scores_tc(q, w, k, n, heads, T, L, H_I, h, out, ld, s)) return;
+  // dense scores of gathered candidates (MISA-dagger re-rank): tensor-core contraction per 128 rows
+  if (gather && !heads && launch_rerank_tc(q, w, k, k_seq_stride, n, T, L, H_I, rows, P, out, ld, s)) return;
   const int m = heads ? h : H_I;
   const int ng = (m + 7) / 8;
   // persistent schedule for per-query caches and for gathered candidate lists
   const bool persist = (gather || k_seq_stride != 0) && T <= kMaxPersistQueries;
-  const ListState* l = persist && !gather && lists_fit(lst, T) ? lst : nullptr;
   switch (ng) {
-#define MISA_NG_CASE(NGV)                                                                                  \
-  case NGV:                                                                                                \
-    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld, l); \
+#define MISA_NG_CASE(NGV)                                                                               \
+  case NGV:                                                                                             \
+    launch_bf16<NGV>(gather, persist, s, q, w, k, k_seq_stride, n, heads, h, H_I, T, L, rows, P, out, ld); \
     break;
     MISA_NG_CASE(1)
     MISA_NG_CASE(2)
@@ -530,7 +415,6 @@ bool launch_scores(DType dt, const void* q, const float* w, const void* k, int64
     default:
       break;
   }
-  return l != nullptr;
 }
 
 MISA_BAD_ID_READER(read_and_clear_bad_ids_score)

@@ -152,39 +152,77 @@ __device__ __forceinline__ uint32_t linear_bin(uint32_t key, float vlo, float sc
   return (uint32_t)min(__float2int_rz(x), kHistBins - 1);
 }
 
-// Cut for the r-th largest of a set of keys spread over the block: each(f) calls f(key) for every
-// key of the calling thread; lo and hi are the block's smallest and largest key.  Returns the
-// smallest key of the linear bin (4096 bins between the scores of lo and hi) that holds the r-th
-// largest key, so at least r keys are at or above it and at most one bin's worth more; a set of
-// one value (or a range too wide to bin) returns lo, which keeps every key.  hist: 4096 words of
-// shared memory; mm: 2 words; scratch: 35 words.  Every thread calls it.
-template <class Each>
-__device__ __forceinline__ uint32_t linear_cut(Each each, uint32_t lo, uint32_t hi, uint32_t r, uint32_t* hist,
-                                               uint32_t* mm, uint32_t* scratch) {
-  const float vlo = key_to_float(lo), vhi = key_to_float(hi);
-  const float scale = (float)kHistBins / (vhi - vlo);
-  if (!(vhi > vlo) || !(scale > 0.f) || !(scale < 3.0e38f)) return lo;
-  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
-  __syncthreads();
-  each([&](uint32_t k) { hist_add(hist, linear_bin(k, vlo, scale), true); });
-  __syncthreads();
-  const uint32_t b = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch).prefix;
+// Smallest key among the calling threads' keys that `take` accepts, over the block (0xffffffff for
+// none).  mm[0] is used; every thread calls it.
+template <class Each, class Take>
+__device__ __forceinline__ uint32_t block_min_of(Each each, Take take, uint32_t* mm) {
   if (threadIdx.x == 0) mm[0] = 0xffffffffu;
   __syncthreads();
   uint32_t mn = 0xffffffffu;
   each([&](uint32_t k) {
-    if (linear_bin(k, vlo, scale) == b) mn = min(mn, k);
+    if (take(k)) mn = min(mn, k);
   });
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
   if ((threadIdx.x & 31) == 0) atomicMin(&mm[0], mn);
   __syncthreads();
-  const uint32_t cut = mm[0];
+  const uint32_t v = mm[0];
   __syncthreads();
-  return cut;
+  return v;
 }
 
-// Cut from a sample of keys: the smallest score of the linear bin holding the rank-th largest
+// Cut for the r-th largest of a set of keys spread over the block: each(f) calls f(key) for every
+// key of the calling thread; lo and hi are the block's smallest and largest key.  Returns the
+// smallest key of a narrow bin holding the r-th largest key, so at least r keys are at or above it
+// and only that bin's keys beyond.  Round 1 bins the key range itself in 4096 bins: order keys are
+// close to logarithmic in the score within one sign, so a few outliers (far larger scores) do not
+// crowd the bulk of the set into a few bins.  When the boundary bin still holds more than 64 keys
+// (scores of both signs put 8 bins in a factor of two), round 2 bins that bin's own score range
+// linearly.  A set of one value returns lo, which keeps every key.  hist: 4096 words of shared
+// memory; mm: 2 words; scratch: 35 words.  Every thread calls it.
+template <class Each>
+__device__ __forceinline__ uint32_t linear_cut(Each each, uint32_t lo, uint32_t hi, uint32_t r, uint32_t* hist,
+                                               uint32_t* mm, uint32_t* scratch) {
+  if (hi <= lo) return lo;
+  const uint32_t range = hi - lo;
+  const int sh = range >= 4096u ? 32 - __clz(range) - 12 : 0;
+  for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  each([&](uint32_t k) { hist_add(hist, (k - lo) >> sh, true); });
+  __syncthreads();
+  const Bucket bk = block_bucket_bits(hist, kHistBins, sh, 0u, r, scratch);
+  const uint32_t b = bk.prefix >> sh;
+  auto in_bin = [&](uint32_t k) { return ((k - lo) >> sh) == b; };
+  if (bk.eq <= 64u) return block_min_of(each, in_bin, mm);
+  // round 2: the boundary bin's keys, 4096 bins linear in their score
+  if (threadIdx.x == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+  uint32_t blo = 0xffffffffu, bhi = 0u;
+  each([&](uint32_t k) {
+    if (in_bin(k)) {
+      blo = min(blo, k);
+      bhi = max(bhi, k);
+    }
+  });
+  block_min_max(blo, bhi, mm);
+  __syncthreads();
+  blo = mm[0];
+  bhi = mm[1];
+  __syncthreads();
+  const float vlo = key_to_float(blo), vhi = key_to_float(bhi);
+  const float scale = (float)kHistBins / (vhi - vlo);
+  if (!(vhi > vlo) || !(scale > 0.f) || !(scale < 3.0e38f)) return blo;
+  for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+  __syncthreads();
+  each([&](uint32_t k) { hist_add(hist, linear_bin(k, vlo, scale), in_bin(k)); });
+  __syncthreads();
+  const uint32_t b2 = block_bucket_bits(hist, kHistBins, 0, 0u, bk.need, scratch).prefix;
+  return block_min_of(each, [&](uint32_t k) { return in_bin(k) && linear_bin(k, vlo, scale) == b2; }, mm);
+}
+
+// Cut from a sample of keys: the smallest score of the narrow bin holding the rank-th largest
 // sample key (linear_cut), so at least `rank` sample keys are at or above the returned value.  PER
 // keys per thread; hist: 4096 words of shared memory; mm: 2 words holding 0xffffffff and 0 on entry
 // (and again on return); scratch: 35 words.  Every thread calls it.

@@ -10,15 +10,20 @@
 // specified.  The candidates of a row (the entries that can still be selected) reach a list in
 // shared memory in one of two ways:
 //   * from the row: a sampled cut, then one pass that gathers the entries at or above it;
-//   * from a candidate list the decode scoring kernel already appended while it scored (every
-//     score at or above a cut taken from a sample of the keys beforehand, score.cu), copied in.
-// The list is then ranked with 4096 bins that are linear in the score between its smallest and
-// largest entry, so the bin holding the k-th entry is small and one warp ranks it.  A row whose
+//   * from a candidate list built beforehand, copied in: for a few long rows, one CTA per row
+//     places the row's cut from the same sample (list_cut_kernel) and CTAs over chunks of 8192
+//     scores append the entries at or above it (list_sweep_kernel), so the pass over the row runs
+//     on every SM instead of one per row.
+// Candidate lists without score rows (the fused prefill scorer's) are ranked one warp per row
+// (list_select_warp_kernel).
+// The list is then ranked by rounds of 4096-bin histograms over what is left of its key range,
+// which find the k-th key exactly; one pass writes the selection.  A row whose
 // candidates cannot be trusted to hold the selection takes an exact path over the whole row.
 // select_small_kernel ranks a short candidate list entirely in one CTA's shared memory; it needs
 // no workspace (used by the entry point without allocation).
 #include "kernels.cuh"
 #include "select.cuh"
+#include "warp_select.cuh"
 
 namespace misa {
 
@@ -37,18 +42,16 @@ __device__ __forceinline__ int padded(int e) { return e + (e >> 5); }
 // one CTA: 512 threads, 2 CTAs per SM and an 8192-entry list for many rows (prefill chunks);
 // 1024 threads, 1 CTA per SM and a 16384-entry list for a few long rows (decode), for candidate
 // lists and for rows whose candidates the scoring kernel already gathered:
-//   1. candidates: rows whose scoring kernel appended a candidate list (every score at or above a
-//      cut sampled from the keys, score.cu) copy that list in.  Otherwise rows longer than the
+//   1. candidates: rows with a candidate list (list_cut_kernel and list_sweep_kernel, below: every
+//      score at or above the row's cut key) copy the entries at or above the cut key in.  Otherwise rows longer than the
 //      list are sampled (256 evenly spaced runs of 8 scores, 2048 keys) and a 4096-bin histogram
 //      over the sampled key range places the sample key whose rank is the expected sample count
 //      above the k-th key plus three standard deviations and a margin; the lower edge of its bin
 //      is the threshold value (shorter rows take every entry), and one pass appends (key, token)
 //      of every entry at or above it to the list (a bit mask per 16 entries a thread, one warp
 //      scan and one shared atomic per warp and step), tracking the smallest and largest key;
-//   2. selection (select_list_linear): 4096 bins linear in the score between the list's smallest
-//      and largest value; one histogram finds the bin of the k-th entry, entries in higher bins go
-//      straight to the output, the boundary bin's entries are ranked by one warp (when at most 32)
-//      or by a radix select on their keys, exact ties by token.
+//   2. selection (select_list_exact): rounds of 4096 bins over what is left of the list's key range
+//      find the k-th key; exact ties there go to the lower tokens; one pass writes the selection.
 // Whenever the list holds at least k keys and every entry at or above its cut, it holds every
 // selected key, so the result is exact.  Otherwise (fewer than k at or above the cut, or more than
 // the list holds) a score row takes the exact path: full level-0 histogram of the row, keys above
@@ -228,89 +231,135 @@ __device__ __forceinline__ void collect_above(const float* row, const int32_t* i
   }
 }
 
-// Ranks n <= 32 entries of list (keys descending, then tokens ascending) in one warp and writes
-// the first `need` to oi/ov at their rank.
-template <class Acc>
-__device__ __forceinline__ void warp_rank_write(const uint2* list, int n, uint32_t need, const Acc& acc, int32_t* oi,
-                                                float* ov) {
-  const int lane = threadIdx.x & 31;
-  const bool mine = lane < n;
-  const uint2 e = mine ? list[lane] : make_uint2(0u, 0xffffffffu);
-  uint32_t rank = 0;
-  for (int j = 0; j < n; ++j) {
-    const uint32_t kj = __shfl_sync(0xffffffffu, e.x, j);
-    const uint32_t ij = __shfl_sync(0xffffffffu, e.y, j);
-    rank += (kj > e.x) || (kj == e.x && ij < e.y);
+// The r-th largest (1 <= r <= count) of the keys the block's threads visit, all within [lo, hi].
+// Round 0 bins the scores linearly over [value(lo), value(hi)] (4096 bins; smooth score
+// distributions spread evenly, so the shared-memory atomics rarely collide, where order keys crowd
+// the bulk of a set that spans both signs into a few bins); the boundary bin's own key range then
+// takes rounds of 4096 key bins until a bin holds exactly the missing count (*all = true: every key
+// of the bin is taken; the result is the bin's smallest key) or is one key wide (*all = false: the
+// result is that key; ties with it may straddle the r-th place).  each(g) calls g(key, counted) for
+// every member on the calling thread.  *above: the count of keys above the result's bin.  LINEAR
+// false skips round 0 (keys that are not order keys of finite scores).  hist: kHistBins words;
+// mm: 2 words; scratch: 35 words.
+template <bool LINEAR, class Each>
+__device__ __forceinline__ uint32_t block_rth_largest(Each each, uint32_t lo, uint32_t hi, uint32_t r, uint32_t* hist,
+                                                      uint32_t* mm, uint32_t* scratch, uint32_t* above, bool* all) {
+  uint32_t gt = 0;
+  const float vlo = key_to_float(lo), vhi = key_to_float(hi);
+  const float scale = (float)kHistBins / (vhi - vlo);
+  if (LINEAR && hi > lo && vhi > vlo && scale > 0.f && scale < 3.0e38f) {
+    for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    each([&](uint32_t k, bool counted) {
+      if (counted) atomicAdd(&hist[linear_bin(k, vlo, scale)], 1u);
+    });
+    __syncthreads();
+    const Bucket bk = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch);
+    gt += r - bk.need;
+    r = bk.need;
+    // the bin's key range (linear_bin is monotone: lower bins hold smaller scores only)
+    if (threadIdx.x == 0) {
+      mm[0] = 0xffffffffu;
+      mm[1] = 0u;
+    }
+    __syncthreads();
+    uint32_t blo = 0xffffffffu, bhi = 0u;
+    each([&](uint32_t k, bool counted) {
+      if (counted && linear_bin(k, vlo, scale) == bk.prefix) {
+        blo = min(blo, k);
+        bhi = max(bhi, k);
+      }
+    });
+    block_min_max(blo, bhi, mm);
+    __syncthreads();
+    lo = mm[0];
+    hi = mm[1];
+    __syncthreads();
+    if (bk.eq == r) {
+      *above = gt;
+      *all = true;
+      return lo;
+    }
   }
-  if (mine && rank < need) {
-    oi[rank] = (int32_t)e.y;
-    if (ov) ov[rank] = acc.value(lane);
+  uint32_t base = lo, range = hi - lo;
+  for (;;) {
+    const int sh = range >= (uint32_t)kHistBins ? 32 - __clz(range) - 12 : 0;
+    for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    each([&](uint32_t v, bool counted) {
+      if (counted && v >= base && v - base <= range) atomicAdd(&hist[(v - base) >> sh], 1u);
+    });
+    __syncthreads();
+    const Bucket bk = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch);  // bin in prefix
+    gt += r - bk.need;
+    r = bk.need;
+    const uint32_t edge = base + (bk.prefix << sh);
+    if (bk.eq == r || sh == 0) {
+      *above = gt;
+      *all = bk.eq == r;
+      return edge;
+    }
+    range = min(range - (bk.prefix << sh), (1u << sh) - 1u);
+    base = edge;
   }
 }
 
-// Top `need` of the c list entries (c >= need) in shared memory, written to oi/ov [0, need).
-// lo/hi: the smallest and largest key in the list.  One histogram of 4096 bins linear in the score
-// finds the bin of the need-th entry; entries of higher bins go out directly, the boundary bin's
-// entries move to the front of the list and are ranked on their keys (one warp when they are
-// few), exact ties by token.  When the value range is empty or not finite the list is ranked on
-// its keys directly.  hist: kHistBins words; ctr: 2 words; scratch: 35 words.
-template <int NT, int LIST>
-__device__ void select_list_linear(uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
-                                   uint32_t* ctr, uint32_t* scratch, int32_t* oi, float* ov) {
+// Top `need` of the c list entries (c >= need, keys within [lo, hi]) in shared memory, written to
+// oi/ov [0, need) in no particular order: block_rth_largest finds the need-th key kstar, exact ties
+// at kstar that straddle the place go to the lower tokens (a second search over the tied entries'
+// tokens), and one pass writes every entry above kstar and the tied ones taken.  The list is only
+// read.  ctr: 2 words; scratch: 35 words.
+template <int NT>
+__device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
+                                  uint32_t* ctr, uint32_t* mm, uint32_t* scratch, int32_t* oi, float* ov) {
   const int tid = threadIdx.x;
-  const SmemPairs acc{list};
-  const float vlo = key_to_float(lo), vhi = key_to_float(hi);
-  const float scale = (float)kHistBins / (vhi - vlo);
-  if (!(vhi > vlo) || !(scale > 0.f) || !(scale < 3.0e38f)) {
-    const SelectResult r = radix_select_items(acc, c, need, 0, 0u, 0u, hist, scratch);
-    write_selection(acc, c, r, false, oi, ov, need, scratch);
-    return;
+  uint32_t above;
+  bool all;
+  const uint32_t kstar = block_rth_largest<true>(
+      [&](auto g) {
+        for (int i = tid; i < c; i += NT) g(list[i].x, true);
+      },
+      lo, hi, need, hist, mm, scratch, &above, &all);
+  uint32_t tok = 0xffffffffu;  // tied entries at kstar taken: every one (all), else tokens <= tok
+  if (!all) {
+    if (tid == 0) {
+      mm[0] = 0xffffffffu;
+      mm[1] = 0u;
+    }
+    __syncthreads();
+    uint32_t tlo = 0xffffffffu, thi = 0u;
+    for (int i = tid; i < c; i += NT)
+      if (list[i].x == kstar) {
+        tlo = min(tlo, 0xffffffffu - list[i].y);
+        thi = max(thi, 0xffffffffu - list[i].y);
+      }
+    block_min_max(tlo, thi, mm);
+    __syncthreads();
+    tlo = mm[0];
+    thi = mm[1];
+    uint32_t a2;
+    bool all2;
+    tok = 0xffffffffu - block_rth_largest<false>(
+                            [&](auto g) {
+                              for (int i = tid; i < c; i += NT) {
+                                const uint2 e = list[i];
+                                g(0xffffffffu - e.y, e.x == kstar);
+                              }
+                            },
+                            tlo, thi, need - above, hist, mm, scratch, &a2, &all2);
   }
-  for (int b = tid; b < kHistBins; b += NT) hist[b] = 0;
-  if (tid < 2) ctr[tid] = 0;
+  if (tid == 0) ctr[0] = 0;
   __syncthreads();
-  for (int i = tid; i < c; i += NT) hist_add(hist, linear_bin(list[i].x, vlo, scale), true);
-  __syncthreads();
-  const Bucket bk = block_bucket_bits(hist, kHistBins, 0, 0u, need, scratch);
-  const uint32_t pb = bk.prefix;  // boundary bin
-  constexpr int kPer = LIST / NT;
-  uint2 keep[kPer];
-  int nk = 0;
   const int steps = (c + NT - 1) / NT;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) {
-    if (j >= steps) break;  // uniform
+  for (int j = 0; j < steps; ++j) {
     const int i = j * NT + tid;
     const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
-    const uint32_t bin = i < c ? linear_bin(e.x, vlo, scale) : 0u;
-    const bool gt = i < c && bin > pb;
-    const uint32_t slot = warp_slot(gt, &ctr[0]);
-    if (gt) {
+    const bool sel = i < c && (e.x > kstar || (e.x == kstar && (all || e.y <= tok)));
+    const uint32_t slot = warp_slot(sel, &ctr[0]);
+    if (sel) {
       oi[slot] = (int32_t)e.y;
       if (ov) ov[slot] = key_to_float(e.x);
     }
-    const bool eq = i < c && bin == pb;
-    if (eq) keep[nk] = e;
-    nk += eq;
-  }
-  __syncthreads();  // every entry read
-  uint32_t total;
-  const uint32_t off = block_exclusive_scan((uint32_t)nk, scratch, &total);
-  for (int x = 0; x < kPer; ++x)
-    if (x < nk) list[off + x] = keep[x];
-  __syncthreads();
-  const uint32_t n_gt = ctr[0];
-  const uint32_t need2 = need - n_gt;
-  if (total <= need2) {
-    for (uint32_t i = tid; i < total; i += NT) {
-      oi[n_gt + i] = (int32_t)list[i].y;
-      if (ov) ov[n_gt + i] = key_to_float(list[i].x);
-    }
-  } else if (total <= 32) {
-    if (tid < 32) warp_rank_write(list, (int)total, need2, acc, oi + n_gt, ov ? ov + n_gt : nullptr);
-  } else {
-    const SelectResult r = radix_select_items(acc, (int)total, need2, 0, 0u, 0u, hist, scratch);
-    write_selection(acc, (int)total, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need2, scratch);
   }
 }
 
@@ -330,8 +379,10 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
                                                             const uint2* __restrict__ lists,
                                                             const uint32_t* __restrict__ lcnt,
                                                             const uint32_t* __restrict__ lcut, int lcap,
-                                                            int32_t* __restrict__ redo,
-                                                            const int32_t* __restrict__ only) {
+                                                            int64_t lstride, int32_t* __restrict__ redo,
+                                                            const int32_t* __restrict__ only,
+                                                            const uint32_t* __restrict__ lhist,
+                                                            const uint32_t* __restrict__ lshift) {
   extern __shared__ uint2 list[];  // [LIST]
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
@@ -372,26 +423,81 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
       exact = !listed;  // too few entries, or entries dropped past the list's end
     }
   }
-  if (listed) {  // copy the scoring kernel's list: the entries at or above the row's cut key
-    const uint2* src = lists + (int64_t)t * lcap;
-    const uint32_t cut = __ldcg(lcut + t);
+  if (listed && lhist && __ldcg(lcut + t) != 0x80000000u) {
+    // the list's histogram (bins of the key above the cut) gives the bin of the k-th entry; one pass
+    // over the list writes the entries of higher bins out and keeps the bin's own entries, which
+    // are ranked next.  (A cut at +0.0 takes the copy below: a -0.0 score passes the sweep's float
+    // compare but sits below the cut key, outside the histogram.)
+    for (int b = tid; b < kHistBins; b += NT) hp[b] = __ldcg(lhist + (int64_t)t * kHistBins + b);
+    __syncthreads();
+    const Bucket bk = block_bucket_bits(hp, kHistBins, 0, 0u, (uint32_t)topk, scratch);
+    const uint32_t cut = __ldcg(lcut + t), sh = __ldcg(lshift + t);
+    const uint2* src = lists + (int64_t)t * lstride;
     uint32_t lo = 0xffffffffu, hi = 0u;
-    for (uint32_t i0 = 0; i0 < c_in; i0 += NT) {
-      const uint32_t i = i0 + tid;
-      const uint2 e = i < c_in ? __ldcg(src + i) : make_uint2(0u, 0u);
-      const bool keep = i < c_in && e.x >= cut;
-      const uint32_t slot = warp_slot(keep, &cnt[0]);
-      if (keep) {
-        list[slot] = e;
-        lo = min(lo, e.x);
-        hi = max(hi, e.x);
+    for (uint32_t i0 = 0; i0 < c_in; i0 += 4 * NT) {
+      uint2 e[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * NT + tid;
+        e[u] = i < c_in ? __ldcg(src + i) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * NT + tid;
+        const bool valid = i < c_in && e[u].x >= cut;
+        const uint32_t bin = min((e[u].x - cut) >> sh, (uint32_t)(kHistBins - 1));
+        const bool gt = valid && bin > bk.prefix, in = valid && bin == bk.prefix;
+        const uint32_t slot = warp_slot(gt, &cnt[0]);
+        if (gt) {
+          oi[slot] = (int32_t)e[u].y;
+          if (ov) ov[slot] = key_to_float(e[u].x);
+        }
+        const uint32_t s2 = warp_slot(in, &cnt[1]);
+        if (in) {
+          list[s2] = e[u];
+          lo = min(lo, e[u].x);
+          hi = max(hi, e[u].x);
+        }
       }
     }
     block_min_max(lo, hi, mm);
     __syncthreads();
-    // fewer than the needed entries at or above the cut: the list cannot hold the answer
-    exact = cnt[0] < need;
-    listed = !exact;
+    const uint32_t n_gt = (uint32_t)topk - bk.need, c2 = cnt[1];
+    if (c2 == bk.need) {
+      for (uint32_t i = tid; i < c2; i += NT) {
+        oi[n_gt + i] = (int32_t)list[i].y;
+        if (ov) ov[n_gt + i] = key_to_float(list[i].x);
+      }
+    } else {
+      const uint32_t blo = mm[0], bhi = mm[1];
+      __syncthreads();  // mm is reused as scratch
+      select_list_exact<NT>(list, (int)c2, bk.need, blo, bhi, hp, cnt, mm, scratch, oi + n_gt, ov ? ov + n_gt : nullptr);
+    }
+    if (redo && tid == 0) redo[t] = 0;
+    return;
+  }
+  if (listed) {  // copy the list in: every entry of a built list is at or above the row's cut
+    const uint2* src = lists + (int64_t)t * lstride;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (uint32_t i0 = 0; i0 < c_in; i0 += 4 * NT) {
+      uint2 e[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * NT + tid;
+        e[u] = i < c_in ? __ldcg(src + i) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t i = i0 + u * NT + tid;
+        if (i < c_in) {
+          list[i] = e[u];
+          lo = min(lo, e[u].x);
+          hi = max(hi, e[u].x);
+        }
+      }
+    }
+    if (tid == 0) cnt[0] = c_in;
+    block_min_max(lo, hi, mm);
     __syncthreads();
   } else if (!exact) {
     float thr = -INFINITY;
@@ -433,7 +539,9 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
       return;
     }
     if (c >= (uint32_t)topk && c <= (uint32_t)LIST) {
-      select_list_linear<NT, LIST>(list, (int)c, (uint32_t)topk, mm[0], mm[1], hp, cnt, scratch, oi, ov);
+      const uint32_t lo = mm[0], hi = mm[1];
+      __syncthreads();  // mm is reused as scratch
+      select_list_exact<NT>(list, (int)c, (uint32_t)topk, lo, hi, hp, cnt, mm, scratch, oi, ov);
       return;  // c >= topk entries: every slot is filled
     }
     __syncthreads();
@@ -507,7 +615,165 @@ void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P,
   row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt,
                                                       lst ? lst->list : nullptr, lst ? lst->cnt : nullptr,
                                                       lst ? lst->cutkey : nullptr, lst ? lst->cap : 0,
-                                                      lst ? lst->redo : nullptr, only);
+                                                      lst ? lst->stride : 0, lst ? lst->redo : nullptr, only,
+                                                      lst ? lst->hist : nullptr, lst ? lst->shift : nullptr);
+}
+
+// ---- candidate lists of long score rows --------------------------------------------------------
+
+constexpr int kCutThreads = 1024;
+constexpr int kSweepThreads = 256;
+constexpr int kSweepPer = 32;                              // scores per thread (8 x float4)
+constexpr int kSweepChunk = kSweepThreads * kSweepPer;     // 8192 scores per CTA
+
+// One CTA per row: the row's cut from the same sample the row kernel takes (256 evenly spaced runs
+// of 8 scores; rank: the expected sample count above the k-th score plus three standard
+// deviations and a margin), as an order key in lcut[t], and lcnt[t] = 0.  Rows of at most cap
+// entries, rows whose sample cannot place the cut and rows whose list is not expected to fit get
+// no list (lcnt[t] = kNoList) and take the row kernel's own path.
+__global__ void __launch_bounds__(kCutThreads) list_cut_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                const int32_t* __restrict__ n, int L, int topk,
+                                                                int cap, uint32_t* __restrict__ lcnt,
+                                                                uint32_t* __restrict__ lcut,
+                                                                uint32_t* __restrict__ lhist,
+                                                                uint32_t* __restrict__ lshift) {
+  __shared__ uint32_t hist[kHistBins];
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t mm[2];
+  __shared__ uint32_t smax;
+  const int t = blockIdx.x;
+  const int nt = clamp_len(n[t], L);
+  constexpr int ns = kSampleRuns * kSampleRunLen;
+  const uint32_t rank = sample_rank(topk, nt);
+  // the list is expected to hold about rank / ns of the row; keep a tenth of the cap in reserve
+  if (nt <= cap || rank > (uint32_t)ns || (double)rank * nt > 0.9 * (double)cap * ns) {
+    if (threadIdx.x == 0) lcnt[t] = kNoList;
+    return;
+  }
+  const float* row = scores + (int64_t)t * ld;
+  const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);
+  constexpr int per = ns / kCutThreads;
+  uint32_t sk[per];
+  uint32_t mx = 0u;
+#pragma unroll
+  for (int u = 0; u < per; ++u) {
+    const int i = u * kCutThreads + (int)threadIdx.x;
+    sk[u] = order_key(__ldcg(row + (int64_t)(i / kSampleRunLen) * seg + (i % kSampleRunLen)));
+    mx = max(mx, sk[u]);
+  }
+  for (int b = threadIdx.x; b < kHistBins; b += kCutThreads) lhist[(int64_t)t * kHistBins + b] = 0u;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if (threadIdx.x == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+    smax = 0u;
+  }
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) atomicMax(&smax, mx);
+  const float thr = sample_cut<per>(sk, rank, hist, mm, scratch);  // synchronises first
+  if (threadIdx.x == 0) {
+    const uint32_t cut = order_key(thr);
+    // histogram bins: the sampled range above the cut in 4096 bins (larger keys go to the top bin)
+    const uint32_t range = smax > cut ? smax - cut : 0u;
+    lcnt[t] = 0u;
+    lcut[t] = cut;
+    lshift[t] = range >= (uint32_t)kHistBins ? (uint32_t)(32 - __clz(range) - 12) : 0u;
+  }
+}
+
+// One CTA per (chunk of 8192 scores, row): every entry at or above the row's cut goes to the row's
+// list; one block scan and one atomic per CTA place them (entries past cap are counted, not
+// written).  Scores are compared as floats with the cut's value (the same order as their keys).
+__global__ void __launch_bounds__(kSweepThreads, 4) list_sweep_kernel(const float* __restrict__ scores, int64_t ld,
+                                                                      const int32_t* __restrict__ n, int L,
+                                                                      uint2* __restrict__ lists, int64_t stride,
+                                                                      uint32_t* __restrict__ lcnt,
+                                                                      const uint32_t* __restrict__ lcut, int cap,
+                                                                      uint32_t* __restrict__ lhist,
+                                                                      const uint32_t* __restrict__ lshift) {
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t sbase;
+  const int t = blockIdx.y;
+  const int nt = clamp_len(n[t], L);
+  const int s0 = blockIdx.x * kSweepChunk;
+  if (s0 >= nt || __ldcg(lcnt + t) == kNoList) return;  // uniform across the block
+  const int len = min(kSweepChunk, nt - s0);
+  const float* row = scores + (int64_t)t * ld + s0;
+  const float thr = key_to_float(__ldcg(lcut + t));
+  const int tid = threadIdx.x;
+  // element 4 (u * 256 + tid) + e of the chunk is v[4 u + e] and bit 4 u + e of the mask
+  float v[kSweepPer];
+  if (len == kSweepChunk && (reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+#pragma unroll
+    for (int u = 0; u < kSweepPer / 4; ++u) {
+      const float4 x = __ldcg(reinterpret_cast<const float4*>(row) + u * kSweepThreads + tid);
+      v[4 * u] = x.x;
+      v[4 * u + 1] = x.y;
+      v[4 * u + 2] = x.z;
+      v[4 * u + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < kSweepPer; ++i) {
+      const int p = 4 * ((i >> 2) * kSweepThreads + tid) + (i & 3);
+      v[i] = p < len ? __ldcg(row + p) : -INFINITY;  // never at or above a cut of a finite score
+    }
+  }
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < kSweepPer; ++i) m |= (uint32_t)(v[i] >= thr) << i;
+  uint32_t total;
+  uint32_t slot = block_exclusive_scan((uint32_t)__popc(m), scratch, &total);
+  if (tid == 0) sbase = total ? atomicAdd(lcnt + t, total) : 0u;
+  __syncthreads();
+  if (!m) return;
+  slot += sbase;
+  uint2* lt = lists + (int64_t)t * stride;
+  const uint32_t cut = __ldcg(lcut + t), sh = __ldcg(lshift + t);
+  uint32_t* ht = lhist + (int64_t)t * kHistBins;
+#pragma unroll
+  for (int i = 0; i < kSweepPer; ++i)
+    if ((m >> i) & 1u) {
+      const uint32_t k = order_key(v[i]);
+      if (slot < (uint32_t)cap) lt[slot] = make_uint2(k, (uint32_t)(s0 + 4 * ((i >> 2) * kSweepThreads + tid) + (i & 3)));
+      ++slot;
+      // a list entry is at or above the cut key (a -0.0 score against a +0.0 cut is not counted)
+      if (k >= cut) atomicAdd(ht + min((k - cut) >> sh, (uint32_t)(kHistBins - 1)), 1u);
+    }
+}
+
+// One warp per row: the top-k of the row's candidate list (warp_list_select).  A row without a
+// list, whose list lost entries past cap, or whose list holds fewer than min(k, n_t) entries at or
+// above its cut gets redo[t] = n_t and no output; the others redo[t] = 0.
+__global__ void __launch_bounds__(32 * kSelWarps, 3) list_select_warp_kernel(const int32_t* __restrict__ n, int L, int T,
+                                                                          int topk, const uint2* __restrict__ lists,
+                                                                          int64_t stride, int cap,
+                                                                          const uint32_t* __restrict__ lcnt,
+                                                                          const uint32_t* __restrict__ lcut,
+                                                                          int32_t* __restrict__ redo,
+                                                                          int32_t* __restrict__ idx,
+                                                                          float* __restrict__ score_opt) {
+  __shared__ uint32_t hist[kSelWarps][kWarpBinWords];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kSelWarps + warp;
+  if (t >= T) return;  // uniform across the warp
+  const int nt = clamp_len(n[t], L);
+  const uint32_t c = __ldcg(lcnt + t);
+  int32_t* oi = idx + (int64_t)t * topk;
+  float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
+  if (nt == 0) {  // empty prefix: nothing to select
+    for (int a = lane; a < topk; a += 32) {
+      oi[a] = -1;
+      if (ov) ov[a] = 0.f;
+    }
+    if (lane == 0) redo[t] = 0;
+    return;
+  }
+  bool ok = c <= (uint32_t)cap;  // kNoList, or entries lost past cap: redone
+  if (ok) ok = warp_list_select(lists + (int64_t)t * stride, (int)c, __ldcg(lcut + t), (uint32_t)min(topk, nt), topk,
+                                hist[warp], oi, ov);
+  if (lane == 0) redo[t] = ok ? 0 : nt;
 }
 
 struct SmemItems {
@@ -570,7 +836,9 @@ size_t al(size_t x) { return (x + 255) / 256 * 256; }
 
 size_t list_state_bytes(int T, int cap) {
   if (T <= 0) return 0;
-  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(uint2) * (size_t)T * cap);
+  const size_t hist = T < kRowKernelMinRows ? al(sizeof(uint32_t) * (size_t)T * kHistBins) + al(sizeof(uint32_t) * T) : 0;
+  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(int32_t) * (size_t)T) + al(sizeof(uint2) * (size_t)T * cap) +
+         hist;
 }
 
 ListState list_state(void* ws, int T, int topk, int cap) {
@@ -578,10 +846,45 @@ ListState list_state(void* ws, int T, int topk, int cap) {
   ListState l;
   l.cnt = reinterpret_cast<uint32_t*>(p);
   l.cutkey = l.cnt + T;
-  l.list = reinterpret_cast<uint2*>(p + al(sizeof(uint32_t) * 2 * (size_t)T));
-  l.cap = cap;
+  p += al(sizeof(uint32_t) * 2 * (size_t)T);
+  l.redo = reinterpret_cast<int32_t*>(p);
+  p += al(sizeof(int32_t) * (size_t)T);
+  l.list = reinterpret_cast<uint2*>(p);
+  p += al(sizeof(uint2) * (size_t)T * cap);
+  if (T < kRowKernelMinRows) {
+    l.hist = reinterpret_cast<uint32_t*>(p);
+    p += al(sizeof(uint32_t) * (size_t)T * kHistBins);
+    l.shift = reinterpret_cast<uint32_t*>(p);
+  }
+  // many rows take the 512-thread row kernel, whose list holds 8192 entries
+  l.cap = T >= kRowKernelMinRows && cap > 8192 ? 8192 : cap;
+  l.stride = cap;
   l.topk = topk;
   return l;
+}
+
+bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T, int L, const ListState& l,
+                       cudaStream_t s) {
+  if (T <= 0) return false;
+  // lists pay off for a few rows longer than the row kernel's own list: the pass over each row is
+  // spread over every SM instead of one CTA per row; many rows fill the GPU with row CTAs already
+  // (measured: lists built for prefill chunks of 4096 rows were slower than the row kernel alone)
+  if (T >= kRowKernelMinRows || L <= l.cap) {
+    mark_no_lists(l, T, s);
+    return false;
+  }
+  list_cut_kernel<<<T, kCutThreads, 0, s>>>(scores, ld, n, L, l.topk, l.cap, l.cnt, l.cutkey, l.hist, l.shift);
+  const int chunks = (L + kSweepChunk - 1) / kSweepChunk;
+  list_sweep_kernel<<<dim3(chunks, T), kSweepThreads, 0, s>>>(scores, ld, n, L, l.list, l.stride, l.cnt, l.cutkey,
+                                                              l.cap, l.hist, l.shift);
+  return true;
+}
+
+void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const ListState& l, int32_t* idx,
+                             float* score_opt, cudaStream_t s) {
+  if (T <= 0) return;
+  list_select_warp_kernel<<<(T + kSelWarps - 1) / kSelWarps, 32 * kSelWarps, 0, s>>>(
+      n, L, T, topk, l.list, l.stride, l.cap, l.cnt, l.cutkey, l.redo, idx, score_opt);
 }
 
 void mark_no_lists(const ListState& l, int T, cudaStream_t s) {

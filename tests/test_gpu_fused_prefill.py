@@ -10,7 +10,8 @@ selections must be the same sets with the same values.  Cases:
     redone exactly;
   * a cache of equal keys: every score ties with the cut, every list overflows, the redo keeps the
     lowest token indices;
-  * prefixes of at most 4k keys, which skip the cut and list every key.
+  * prefixes of at most 4k keys, which skip the cut and list every key;
+  * one strong key repeated 3000 times: the k-th place falls inside an exact tie held by the list.
 """
 import numpy as np
 import pytest
@@ -108,3 +109,25 @@ def test_short_prefixes_take_every_key():
     hd = dev(_heads(256, wl.H_I, wl.h, 9), torch.int32)
     _same(L_, dev(q, torch.bfloat16), dev(w, torch.float32), dev(k, torch.bfloat16), dev(n, torch.int32), hd, 2048,
           "short prefixes")
+
+
+def test_ties_across_the_kth_place_are_ranked_by_token():
+    """3000 copies of one strong key among random keys (queries with positive entries, so the copy
+    scores far above the rest): each list holds all copies under its cap, the k-th place falls inside
+    the tie, and the k lowest tokens among the copies are selected."""
+    L_ = lib()
+    L, T, H_I, h, topk = 40000, 64, 64, 8, 2048
+    g = np.random.default_rng(8)
+    k = W.round_bf16(0.3 * g.standard_normal((L, 128)).astype(np.float32))
+    pos = np.sort(g.choice(L, 3000, replace=False))
+    k[pos] = W.round_bf16(np.abs(g.standard_normal((1, 128))).astype(np.float32))
+    q = W.round_bf16(np.abs(g.standard_normal((T, H_I, 128))).astype(np.float32))
+    w = np.abs(g.standard_normal((T, H_I))).astype(np.float32) / 8
+    n = np.linspace(32000, L, T).astype(np.int32)
+    hd = dev(_heads(T, H_I, h, 10), torch.int32)
+    got = _same(L_, dev(q, torch.bfloat16), dev(w, torch.float32), dev(k, torch.bfloat16), dev(n, torch.int32), hd,
+                topk, "ties at the k-th place")
+    for t in range(T):
+        tied = pos[pos < n[t]]
+        assert len(tied) > topk
+        assert sorted(got[t].tolist()) == tied[:topk].tolist(), "the lowest tokens of the tie"
