@@ -52,11 +52,6 @@ struct ListState {
   // its scores (or, with no score rows behind the lists, by the caller)
   int32_t* redo = nullptr;
   int64_t stride = kListCap;
-  // Lists built from score rows of fewer than 256 queries also keep a histogram of their entries:
-  // hist[t][b] counts the entries with min((key - cutkey[t]) >> shift[t], 4095) = b, so the
-  // selection finds the bin of the k-th entry without a pass of its own.  nullptr otherwise.
-  uint32_t* hist = nullptr;  // [T][4096]
-  uint32_t* shift = nullptr;  // [T]
 };
 size_t list_state_bytes(int T, int cap = kListCap);
 ListState list_state(void* ws, int T, int topk, int cap = kListCap);

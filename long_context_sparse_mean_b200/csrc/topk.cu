@@ -380,9 +380,7 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
                                                             const uint32_t* __restrict__ lcnt,
                                                             const uint32_t* __restrict__ lcut, int lcap,
                                                             int64_t lstride, int32_t* __restrict__ redo,
-                                                            const int32_t* __restrict__ only,
-                                                            const uint32_t* __restrict__ lhist,
-                                                            const uint32_t* __restrict__ lshift) {
+                                                            const int32_t* __restrict__ only) {
   extern __shared__ uint2 list[];  // [LIST]
   __shared__ uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
@@ -422,59 +420,6 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
       listed = c_in >= need && c_in <= (uint32_t)min(lcap, LIST);
       exact = !listed;  // too few entries, or entries dropped past the list's end
     }
-  }
-  if (listed && lhist && __ldcg(lcut + t) != 0x80000000u) {
-    // the list's histogram (bins of the key above the cut) gives the bin of the k-th entry; one pass
-    // over the list writes the entries of higher bins out and keeps the bin's own entries, which
-    // are ranked next.  (A cut at +0.0 takes the copy below: a -0.0 score passes the sweep's float
-    // compare but sits below the cut key, outside the histogram.)
-    for (int b = tid; b < kHistBins; b += NT) hp[b] = __ldcg(lhist + (int64_t)t * kHistBins + b);
-    __syncthreads();
-    const Bucket bk = block_bucket_bits(hp, kHistBins, 0, 0u, (uint32_t)topk, scratch);
-    const uint32_t cut = __ldcg(lcut + t), sh = __ldcg(lshift + t);
-    const uint2* src = lists + (int64_t)t * lstride;
-    uint32_t lo = 0xffffffffu, hi = 0u;
-    for (uint32_t i0 = 0; i0 < c_in; i0 += 4 * NT) {
-      uint2 e[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t i = i0 + u * NT + tid;
-        e[u] = i < c_in ? __ldcg(src + i) : make_uint2(0u, 0u);
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t i = i0 + u * NT + tid;
-        const bool valid = i < c_in && e[u].x >= cut;
-        const uint32_t bin = min((e[u].x - cut) >> sh, (uint32_t)(kHistBins - 1));
-        const bool gt = valid && bin > bk.prefix, in = valid && bin == bk.prefix;
-        const uint32_t slot = warp_slot(gt, &cnt[0]);
-        if (gt) {
-          oi[slot] = (int32_t)e[u].y;
-          if (ov) ov[slot] = key_to_float(e[u].x);
-        }
-        const uint32_t s2 = warp_slot(in, &cnt[1]);
-        if (in) {
-          list[s2] = e[u];
-          lo = min(lo, e[u].x);
-          hi = max(hi, e[u].x);
-        }
-      }
-    }
-    block_min_max(lo, hi, mm);
-    __syncthreads();
-    const uint32_t n_gt = (uint32_t)topk - bk.need, c2 = cnt[1];
-    if (c2 == bk.need) {
-      for (uint32_t i = tid; i < c2; i += NT) {
-        oi[n_gt + i] = (int32_t)list[i].y;
-        if (ov) ov[n_gt + i] = key_to_float(list[i].x);
-      }
-    } else {
-      const uint32_t blo = mm[0], bhi = mm[1];
-      __syncthreads();  // mm is reused as scratch
-      select_list_exact<NT>(list, (int)c2, bk.need, blo, bhi, hp, cnt, mm, scratch, oi + n_gt, ov ? ov + n_gt : nullptr);
-    }
-    if (redo && tid == 0) redo[t] = 0;
-    return;
   }
   if (listed) {  // copy the list in: every entry of a built list is at or above the row's cut
     const uint2* src = lists + (int64_t)t * lstride;
@@ -615,8 +560,7 @@ void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P,
   row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt,
                                                       lst ? lst->list : nullptr, lst ? lst->cnt : nullptr,
                                                       lst ? lst->cutkey : nullptr, lst ? lst->cap : 0,
-                                                      lst ? lst->stride : 0, lst ? lst->redo : nullptr, only,
-                                                      lst ? lst->hist : nullptr, lst ? lst->shift : nullptr);
+                                                      lst ? lst->stride : 0, lst ? lst->redo : nullptr, only);
 }
 
 // ---- candidate lists of long score rows --------------------------------------------------------
@@ -634,13 +578,10 @@ constexpr int kSweepChunk = kSweepThreads * kSweepPer;     // 8192 scores per CT
 __global__ void __launch_bounds__(kCutThreads) list_cut_kernel(const float* __restrict__ scores, int64_t ld,
                                                                 const int32_t* __restrict__ n, int L, int topk,
                                                                 int cap, uint32_t* __restrict__ lcnt,
-                                                                uint32_t* __restrict__ lcut,
-                                                                uint32_t* __restrict__ lhist,
-                                                                uint32_t* __restrict__ lshift) {
+                                                                uint32_t* __restrict__ lcut) {
   __shared__ uint32_t hist[kHistBins];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t mm[2];
-  __shared__ uint32_t smax;
   const int t = blockIdx.x;
   const int nt = clamp_len(n[t], L);
   constexpr int ns = kSampleRuns * kSampleRunLen;
@@ -654,31 +595,20 @@ __global__ void __launch_bounds__(kCutThreads) list_cut_kernel(const float* __re
   const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);
   constexpr int per = ns / kCutThreads;
   uint32_t sk[per];
-  uint32_t mx = 0u;
 #pragma unroll
   for (int u = 0; u < per; ++u) {
     const int i = u * kCutThreads + (int)threadIdx.x;
     sk[u] = order_key(__ldcg(row + (int64_t)(i / kSampleRunLen) * seg + (i % kSampleRunLen)));
-    mx = max(mx, sk[u]);
   }
-  for (int b = threadIdx.x; b < kHistBins; b += kCutThreads) lhist[(int64_t)t * kHistBins + b] = 0u;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
   if (threadIdx.x == 0) {
     mm[0] = 0xffffffffu;
     mm[1] = 0u;
-    smax = 0u;
   }
   __syncthreads();
-  if ((threadIdx.x & 31) == 0) atomicMax(&smax, mx);
-  const float thr = sample_cut<per>(sk, rank, hist, mm, scratch);  // synchronises first
+  const float thr = sample_cut<per>(sk, rank, hist, mm, scratch);
   if (threadIdx.x == 0) {
-    const uint32_t cut = order_key(thr);
-    // histogram bins: the sampled range above the cut in 4096 bins (larger keys go to the top bin)
-    const uint32_t range = smax > cut ? smax - cut : 0u;
     lcnt[t] = 0u;
-    lcut[t] = cut;
-    lshift[t] = range >= (uint32_t)kHistBins ? (uint32_t)(32 - __clz(range) - 12) : 0u;
+    lcut[t] = order_key(thr);
   }
 }
 
@@ -689,9 +619,7 @@ __global__ void __launch_bounds__(kSweepThreads, 4) list_sweep_kernel(const floa
                                                                       const int32_t* __restrict__ n, int L,
                                                                       uint2* __restrict__ lists, int64_t stride,
                                                                       uint32_t* __restrict__ lcnt,
-                                                                      const uint32_t* __restrict__ lcut, int cap,
-                                                                      uint32_t* __restrict__ lhist,
-                                                                      const uint32_t* __restrict__ lshift) {
+                                                                      const uint32_t* __restrict__ lcut, int cap) {
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t sbase;
   const int t = blockIdx.y;
@@ -730,16 +658,12 @@ __global__ void __launch_bounds__(kSweepThreads, 4) list_sweep_kernel(const floa
   if (!m) return;
   slot += sbase;
   uint2* lt = lists + (int64_t)t * stride;
-  const uint32_t cut = __ldcg(lcut + t), sh = __ldcg(lshift + t);
-  uint32_t* ht = lhist + (int64_t)t * kHistBins;
 #pragma unroll
   for (int i = 0; i < kSweepPer; ++i)
     if ((m >> i) & 1u) {
-      const uint32_t k = order_key(v[i]);
-      if (slot < (uint32_t)cap) lt[slot] = make_uint2(k, (uint32_t)(s0 + 4 * ((i >> 2) * kSweepThreads + tid) + (i & 3)));
+      if (slot < (uint32_t)cap)
+        lt[slot] = make_uint2(order_key(v[i]), (uint32_t)(s0 + 4 * ((i >> 2) * kSweepThreads + tid) + (i & 3)));
       ++slot;
-      // a list entry is at or above the cut key (a -0.0 score against a +0.0 cut is not counted)
-      if (k >= cut) atomicAdd(ht + min((k - cut) >> sh, (uint32_t)(kHistBins - 1)), 1u);
     }
 }
 
@@ -836,9 +760,7 @@ size_t al(size_t x) { return (x + 255) / 256 * 256; }
 
 size_t list_state_bytes(int T, int cap) {
   if (T <= 0) return 0;
-  const size_t hist = T < kRowKernelMinRows ? al(sizeof(uint32_t) * (size_t)T * kHistBins) + al(sizeof(uint32_t) * T) : 0;
-  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(int32_t) * (size_t)T) + al(sizeof(uint2) * (size_t)T * cap) +
-         hist;
+  return al(sizeof(uint32_t) * 2 * (size_t)T) + al(sizeof(int32_t) * (size_t)T) + al(sizeof(uint2) * (size_t)T * cap);
 }
 
 ListState list_state(void* ws, int T, int topk, int cap) {
@@ -850,12 +772,6 @@ ListState list_state(void* ws, int T, int topk, int cap) {
   l.redo = reinterpret_cast<int32_t*>(p);
   p += al(sizeof(int32_t) * (size_t)T);
   l.list = reinterpret_cast<uint2*>(p);
-  p += al(sizeof(uint2) * (size_t)T * cap);
-  if (T < kRowKernelMinRows) {
-    l.hist = reinterpret_cast<uint32_t*>(p);
-    p += al(sizeof(uint32_t) * (size_t)T * kHistBins);
-    l.shift = reinterpret_cast<uint32_t*>(p);
-  }
   // many rows take the 512-thread row kernel, whose list holds 8192 entries
   l.cap = T >= kRowKernelMinRows && cap > 8192 ? 8192 : cap;
   l.stride = cap;
@@ -873,10 +789,10 @@ bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T,
     mark_no_lists(l, T, s);
     return false;
   }
-  list_cut_kernel<<<T, kCutThreads, 0, s>>>(scores, ld, n, L, l.topk, l.cap, l.cnt, l.cutkey, l.hist, l.shift);
+  list_cut_kernel<<<T, kCutThreads, 0, s>>>(scores, ld, n, L, l.topk, l.cap, l.cnt, l.cutkey);
   const int chunks = (L + kSweepChunk - 1) / kSweepChunk;
   list_sweep_kernel<<<dim3(chunks, T), kSweepThreads, 0, s>>>(scores, ld, n, L, l.list, l.stride, l.cnt, l.cutkey,
-                                                              l.cap, l.hist, l.shift);
+                                                              l.cap);
   return true;
 }
 

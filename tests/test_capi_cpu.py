@@ -62,10 +62,9 @@ def test_workspace_sizes(lib):
     # + [3, ceil(L/B), 128] bf16 parts of the pooled keys
     assert ws(0, 32, 131072, 64, 128, 8, 0, 0) == 32 * 128 * 4 + 32 * 16 * 64 * 4 + 256 + 3 * 1024 * 128 * 2
     # top-k select: candidate-list state per query: count and cut key [2, T] in one piece, the redo
-    # flags [T], the list [T, 16384] of (key, token) pairs, and below 256 queries the list's
-    # histogram [T, 4096] and bin shift [T], each piece 256-byte aligned
+    # flags [T] and the list [T, 16384] of (key, token) pairs, each piece 256-byte aligned
     def sel(T):
-        return _al(T * 8) + _al(T * 4) + _al(T * 16384 * 8) + (_al(T * 4096 * 4) + _al(T * 4) if T < 256 else 0)
+        return _al(T * 8) + _al(T * 4) + _al(T * 16384 * 8)
     assert ws(4, 32, 131072, 64, 0, 0, 2048, 0) == sel(32)
     assert ws(4, 32, 7, 64, 0, 0, 2048, 0) == sel(32), "independent of the row length"
     # scoring + top-k: [T, ceil4(L)] scores in front of the select workspace
