@@ -55,13 +55,13 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "63ad9e52310709f8745fdb1ae7c3406bfae625c2343add5a1deb685d3bae57c2",
-           "bytes_per_key": (1.073953e9 + 19.169792e6) / 4194304}
+           "sha256": "b2832ee84d6757b5ca450b10cbc4e73539f154c83556b905b3f97f9e44d9ae61",
+           "bytes_per_key": (1.073897e9 + 18.633472e6) / 4194304}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
 # chunk's launch; the step's traffic is that rate times the pairs the step scores.
 TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
-                   "sha256": "3aa6df1f296fc7e0cb8afde7e9ae237d607084f9533b601ca428cd9b148f33ba",
-                   "bytes_per_pair": (52.319232e6 + 984.943616e6) / 260048896}
+                   "sha256": "c4db6753fea8fcc662f8a92e3f98af9f7ade68f519c2221d137c1b4b0fb06537",
+                   "bytes_per_pair": (56.73728e6 + 984.10624e6) / 260048896}
 
 
 def _sha(path):
@@ -397,12 +397,12 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     hbm, kind = _peaks()
     alg = T * (L * d * 2 + lp * 4)
     return {"page_size": ps, "pages_per_sequence": lp, "ms_per_step": ms,
-            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 8,
+            "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 10,
             "matches_contiguous": same,
             "routed_scoring_call": {"ms": score_ms, "algorithmic_bytes": alg,
                                     "achieved_GBps": alg / (score_ms / 1000.0) / 1e9,
                                     "frac_of_hbm": alg / (score_ms / 1000.0) / 1e9 / hbm, "peak_kind": kind,
-                                    "launches": 3}}
+                                    "launches": 5}}
 
 
 def prefill_sample_inputs(wl, count):
@@ -795,13 +795,13 @@ def misa_decode_leg(args, torch, M, wl, dev, gen_pool, steps):
     alg = T * (L * d * 2 + h * d * 2 + h * 4)
     res = {"workload": wl.name, "T": T, "L": L, "H_I": wl.H_I, "B": B, "h": h, "topk": kk,
            "step": "route + routed scores + candidate lists and top-k",
-           "ms_per_step": ms, "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 4,
+           "ms_per_step": ms, "query_tokens_per_s": T * L / (ms / 1000.0), "launches_per_step": 5,
            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
                         "achieved": alg / (score_ms / 1000.0) / 1e9, "peak": hbm, "peak_kind": kind,
                         "unit": "GB/s", "frac": alg / (score_ms / 1000.0) / 1e9 / hbm,
                         "algorithmic_bytes_per_launch": alg, "avg_launch_ms": score_ms},
            "dense": {"ms_per_call": dense_ms, "query_tokens_per_s": T * L / (dense_ms / 1000.0),
-                     "launches_per_call": 2},
+                     "launches_per_call": 4},
            "misa_over_dense_time": ms / dense_ms, "dense_speedup_of_misa": dense_ms / ms,
            "iou_vs_dense": float(np.mean(ious)), "iou_vs_dense_min": float(np.min(ious)),
            "clocks": clk.summary("step, dense and scorer timing passes")}
@@ -863,9 +863,9 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
-    # kernels per step: router, routed scorer, candidate lists and top-k' (one CTA per row), re-rank
-    # scorer, top-k of the candidates (plus two small memsets)
-    launches_per_step = 6
+    # kernels per step: router, routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank,
+    # top-k of the candidates
+    launches_per_step = 7
 
     def route():
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
