@@ -6,6 +6,30 @@
 
 namespace misa {
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start while the previous
+// kernel on its stream is finishing; pdl_wait() (at the top of such a kernel, before it reads
+// anything the previous kernel writes) waits for that kernel to complete and its memory to be
+// visible, and pdl_trigger() lets the next kernel launch its CTAs early.  Both are no-ops in a
+// kernel launched the ordinary way.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <class... KArgs, class... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 constexpr int kD = 128;          // index-key width handled by every kernel
 constexpr int kMaxHeads = 128;   // largest indexer-head pool H_I
 constexpr int kRouteTile = 64;   // router blocks per CTA tile

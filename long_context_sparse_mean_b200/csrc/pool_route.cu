@@ -279,6 +279,8 @@ __global__ void __launch_bounds__(256) route_affinity_mma_kernel(const __nv_bflo
   __shared__ __align__(16) float pms[kD];  // mean of the last block
   __shared__ int last;
   const int t = blockIdx.y, c0 = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int nt = clamp_len(n[t], L);
   const int nk = kbar_blocks(nt, B), Mt = (nt + B - 1) / B;
   const int nc = (Mt + kRouteMmaTile - 1) / kRouteMmaTile;
@@ -527,8 +529,8 @@ void launch_route(DType dt, const void* q, const float* w, const void* k, int64_
     switch (H_I / 8) {
 #define MISA_ROUTE_CASE(NGV)                                                                                  \
   case NGV:                                                                                                   \
-    route_affinity_mma_kernel<NGV><<<grid, 256, 0, s>>>(qb, w, kb, k_seq_stride, kbar, kbar_seq_stride, n, L, B, h, \
-                                                        nch, partial, done, heads, r_opt, pm_in);             \
+    launch_pdl(route_affinity_mma_kernel<NGV>, grid, 256, 0, s, qb, w, kb, k_seq_stride, kbar, kbar_seq_stride, n, L, \
+               B, h, nch, partial, done, heads, r_opt, pm_in);                                                \
     break;
       MISA_ROUTE_CASE(1)
       MISA_ROUTE_CASE(2)

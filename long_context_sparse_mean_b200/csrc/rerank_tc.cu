@@ -105,6 +105,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile uint32_t* tmem_slot = misc;
   volatile int* abort = reinterpret_cast<volatile int*>(misc + 1);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
 
   const int ntile = (P + kRows - 1) / kRows;
   const int64_t W = (int64_t)T * ntile;
@@ -348,7 +350,7 @@ bool launch_rerank_tc(const void* q, const float* w, const void* k, int64_t k_se
   const int64_t work = (int64_t)T * ((P + kRows - 1) / kRows);
   const int grid = (int)(work < sm_count() ? work : sm_count());
   cudaFuncSetAttribute(rerank_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-  rerank_tc_kernel<<<grid, kThreads, kSmemBytes, s>>>(static_cast<const __nv_bfloat16*>(q), w,
+  launch_pdl(rerank_tc_kernel, grid, kThreads, kSmemBytes, s, static_cast<const __nv_bfloat16*>(q), w,
                                                       static_cast<const __nv_bfloat16*>(k), k_seq_stride, n, L, T,
                                                       H_I, cand, P, out, ld);
   return true;

@@ -103,6 +103,8 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
   __shared__ HeadStage<NG> st;
   __shared__ uint32_t wtot[35];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  pdl_wait();
+  pdl_trigger();
 
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
   const int q0 = min((int)threadIdx.x * per, T), q1 = min(q0 + per, T);
@@ -338,12 +340,12 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
     const size_t smem = sizeof(int) * ((size_t)T + 1);
     if (gather) {
       cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      score_persist_kernel<NG, true><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld);
+      launch_pdl(score_persist_kernel<NG, true>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb, k_seq_stride, n,
+                 heads, h, H_I, L, T, rows, P, out, ld);
     } else {
       cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      score_persist_kernel<NG, false><<<2 * num_sms(), kScoreThreads, smem, s>>>(
-          qb, w, kb, k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld);
+      launch_pdl(score_persist_kernel<NG, false>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb, k_seq_stride, n,
+                 heads, h, H_I, L, T, rows, P, out, ld);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);

@@ -387,6 +387,8 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
   __shared__ uint32_t cnt[2];
   __shared__ uint32_t mm[2];
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   if (only && only[t] <= 0) return;
   const int nt = clamp_len(n[t], L);
   const float* row = scores ? scores + (int64_t)t * ld : nullptr;
@@ -557,7 +559,7 @@ void launch_row_topk(const float* scores, int64_t ld, const int32_t* ids, int P,
                      cudaStream_t s) {
   const size_t smem = sizeof(uint2) * (size_t)LIST;
   cudaFuncSetAttribute(row_topk_kernel<NT, LIST, MINB>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  row_topk_kernel<NT, LIST, MINB><<<T, NT, smem, s>>>(scores, ld, ids, P, n, L, topk, idx, score_opt,
+  launch_pdl(row_topk_kernel<NT, LIST, MINB>, T, NT, smem, s, scores, ld, ids, P, n, L, topk, idx, score_opt,
                                                       lst ? lst->list : nullptr, lst ? lst->cnt : nullptr,
                                                       lst ? lst->cutkey : nullptr, lst ? lst->cap : 0,
                                                       lst ? lst->stride : 0, lst ? lst->redo : nullptr, only);
@@ -583,6 +585,8 @@ __global__ void __launch_bounds__(kCutThreads) list_cut_kernel(const float* __re
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t mm[2];
   const int t = blockIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int nt = clamp_len(n[t], L);
   constexpr int ns = kSampleRuns * kSampleRunLen;
   const uint32_t rank = sample_rank(topk, nt);
@@ -623,6 +627,8 @@ __global__ void __launch_bounds__(kSweepThreads, 4) list_sweep_kernel(const floa
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t sbase;
   const int t = blockIdx.y;
+  pdl_wait();
+  pdl_trigger();
   const int nt = clamp_len(n[t], L);
   const int s0 = blockIdx.x * kSweepChunk;
   if (s0 >= nt || __ldcg(lcnt + t) == kNoList) return;  // uniform across the block
@@ -789,10 +795,10 @@ bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T,
     mark_no_lists(l, T, s);
     return false;
   }
-  list_cut_kernel<<<T, kCutThreads, 0, s>>>(scores, ld, n, L, l.topk, l.cap, l.cnt, l.cutkey);
+  launch_pdl(list_cut_kernel, T, kCutThreads, 0, s, scores, ld, n, L, l.topk, l.cap, l.cnt, l.cutkey);
   const int chunks = (L + kSweepChunk - 1) / kSweepChunk;
-  list_sweep_kernel<<<dim3(chunks, T), kSweepThreads, 0, s>>>(scores, ld, n, L, l.list, l.stride, l.cnt, l.cutkey,
-                                                              l.cap);
+  launch_pdl(list_sweep_kernel, dim3(chunks, T), kSweepThreads, 0, s, scores, ld, n, L, l.list, l.stride, l.cnt,
+             l.cutkey, l.cap);
   return true;
 }
 
