@@ -288,3 +288,33 @@ def test_bounds_checked_build_exports_the_same_calls():
     normal = ctypes.CDLL(build.build())
     normal.misa_checked_build.restype = ctypes.c_int
     assert normal.misa_checked_build() == 0
+
+
+def test_fused_prefill_workspace_and_argument_checks(lib):
+    """misa_score_topk_fused: workspace = candidate-list state (counts and cut keys [2, T], redo flags
+    [T], lists [T, 4k] of (key, token) pairs) + the cut [T] + the packed sample [T, ceil(ceil(L/128)/32)
+    * 128] + score rows [T, ceil4(L)] for the queries that are redone; k above 4096 (lists over 16384
+    entries) and fp32 inputs are unsupported."""
+    ws = lib.misa_workspace_bytes
+    T, L, k = 4096, 65536, 2048
+    cols = -(-(-(-L // 128)) // 32) * 128
+    want = (_al(T * 8) + _al(T * 4) + _al(T * 4 * k * 8) + _al(T * 4) + _al(T * cols * 4) +
+            _al(T * (-(-L // 4) * 4) * 4))
+    assert ws(9, T, L, 64, 128, 8, k, 0) == want
+    assert ws(9, 3, 1001, 64, 128, 8, 10, 0) == (_al(24) + _al(12) + _al(3 * 40 * 8) + _al(12) + _al(3 * 128 * 4) +
+                                                 _al(3 * 1004 * 4))
+    assert ws(9, T, L, 64, 128, 8, 4097, 0) == 0, "lists of more than 16384 entries"
+    f = lib.misa_score_topk_fused
+    st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, F32, FAKE, None, FAKE, 1 << 30, None)
+    assert st == UNSUPPORTED  # fp32 inputs take the unfused calls
+    st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 8, 4097, BF16, FAKE, None, FAKE, 1 << 30, None)
+    assert st == UNSUPPORTED
+    st = f(FAKE, FAKE, FAKE, FAKE, None, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, FAKE, 1 << 30, None)
+    assert st == INVALID  # no heads
+    st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 65, 10, BF16, FAKE, None, FAKE, 1 << 30, None)
+    assert st == INVALID  # h > H_I
+    st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, FAKE, 64, None)
+    assert st == WORKSPACE
+    st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, MISALIGNED, 1 << 30, None)
+    assert st == WORKSPACE
+    assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1000, 64, 128, 8, 10, BF16, FAKE, None, None, 0, None) == OK
