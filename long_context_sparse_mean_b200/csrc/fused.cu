@@ -12,7 +12,9 @@
 //      deviations and a margin; prefixes of at most cap keys take every key;
 //   3. the scorer runs over every key tile in compact mode: each score at or above its query's cut
 //      is appended as (order key, token) to the query's list of cap = 4k entries, no score row;
-//   4. one warp per query selects from its list (list_select_warp_kernel);
+//   4. one warp per query selects from its list (list_select_warp_kernel): the list's scores lie
+//      mostly between the cut and the sample's largest score, so one pass bins them linearly and a
+//      second writes the selection, ranking only the k-th entry's bin;
 //   5. a query whose list holds fewer than min(k, n_t) entries or lost some past cap is redone
 //      exactly: the rows scorer and the per-row top-k, restricted to those queries (both launches
 //      find nothing to do when every list answered).
@@ -36,7 +38,8 @@ __global__ void __launch_bounds__(32 * kSelWarps, 3) fused_cut_kernel(const int3
                                                                    int topk, int cap,
                                                                    const float* __restrict__ sample,
                                                                    int64_t ld_sample, float* __restrict__ tau,
-                                                                   uint32_t* __restrict__ cutkey) {
+                                                                   uint32_t* __restrict__ cutkey,
+                                                                   float* __restrict__ shi) {
   __shared__ uint32_t hist[kSelWarps][kWarpBinWords];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kSelWarps + warp;
@@ -62,16 +65,20 @@ __global__ void __launch_bounds__(32 * kSelWarps, 3) fused_cut_kernel(const int3
     return;
   }
   const float* st = sample + (int64_t)t * ld_sample;
-  const uint32_t cut = warp_sample_cut(ns, [&](int i) { return order_key(__ldg(st + i)); }, rank, hist[warp]);
+  uint32_t smax;
+  const uint32_t cut =
+      warp_sample_cut(ns, [&](int i) { return order_key(__ldg(st + i)); }, rank, hist[warp], &smax);
   if (lane == 0) {
     tau[t] = key_to_float(cut);
     cutkey[t] = cut;
+    shi[t] = key_to_float(smax);
   }
 }
 
 struct FusedWs {
   ListState lst;
   float* tau;      // [T]
+  float* shi;      // [T] the sample's largest score
   float* sample;   // [T][fused_sample_cols(L)]
   int64_t ld_sample;
   float* rows;     // [T][ld] score rows of redone queries
@@ -85,6 +92,8 @@ FusedWs carve(void* ws, int T, int L, int topk) {
   f.lst = list_state(p, T, topk, cap);
   p += list_state_bytes(T, cap);
   f.tau = reinterpret_cast<float*>(p);
+  p += al(sizeof(float) * (size_t)T);
+  f.shi = reinterpret_cast<float*>(p);
   p += al(sizeof(float) * (size_t)T);
   f.ld_sample = fused_sample_cols(L);
   f.sample = reinterpret_cast<float*>(p);
@@ -109,7 +118,7 @@ int64_t fused_sample_cols(int L) {
 size_t fused_ws_bytes(int T, int L, int topk) {
   if (T <= 0 || L <= 0 || fused_cap(topk) == 0) return 0;
   const int64_t ld = (L + 3) / 4 * 4;
-  return list_state_bytes(T, fused_cap(topk)) + al(sizeof(float) * (size_t)T) +
+  return list_state_bytes(T, fused_cap(topk)) + 2 * al(sizeof(float) * (size_t)T) +
          al(sizeof(float) * (size_t)T * fused_sample_cols(L)) + al(sizeof(float) * (size_t)T * ld);
 }
 
@@ -123,10 +132,10 @@ bool launch_score_topk_fused(const void* q, const float* w, const void* k, const
   cudaMemsetAsync(f.lst.cnt, 0, sizeof(uint32_t) * 2 * (size_t)T, s);  // counts and cut keys
   if (!launch_scores_tc_sample(q, w, k, n, heads, T, L, H_I, h, kFusedStride, f.sample, f.ld_sample, s)) return false;
   fused_cut_kernel<<<(T + kSelWarps - 1) / kSelWarps, 32 * kSelWarps, 0, s>>>(n, L, T, topk, f.lst.cap, f.sample,
-                                                                              f.ld_sample, f.tau, f.lst.cutkey);
+                                                                              f.ld_sample, f.tau, f.lst.cutkey, f.shi);
   if (!launch_scores_tc_compact(q, w, k, n, heads, T, L, H_I, h, f.tau, f.lst.list, f.lst.cnt, f.lst.cap, s))
     return false;
-  launch_list_select_warp(n, T, L, topk, f.lst, idx, score_opt, s);
+  launch_list_select_warp(n, T, L, topk, f.lst, idx, score_opt, s, f.shi);
   // exact redo of the queries whose list could not answer: rows and selection restricted to them
   if (!launch_scores_tc(q, w, k, f.lst.redo, heads, T, L, H_I, h, f.rows, f.ld, s)) return false;
   launch_topk_rows(f.rows, f.ld, nullptr, 0, f.lst.redo, T, L, topk, nullptr, idx, score_opt, s, f.lst.redo);

@@ -65,9 +65,11 @@ void mark_no_lists(const ListState& l, int T, cudaStream_t s);
 bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T, int L, const ListState& l,
                        cudaStream_t s);
 // One warp per row: the top-k of each row's list (exact, ties to the lower token); rows the list
-// cannot answer get l.redo[t] = n_t and no output, the others l.redo[t] = 0.
+// cannot answer get l.redo[t] = n_t and no output, the others l.redo[t] = 0.  hi (optional): per row
+// the largest score of the sample that placed the cut, which bounds most of the list's entries
+// and lets two passes over the list do (the general rounds otherwise).
 void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const ListState& l, int32_t* idx,
-                             float* score_opt, cudaStream_t s);
+                             float* score_opt, cudaStream_t s, const float* hi = nullptr);
 
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
 // position p of query t scores token rows[t*P + p] and writes out[t*ld + p].

@@ -683,8 +683,10 @@ __global__ void __launch_bounds__(32 * kSelWarps, 3) list_select_warp_kernel(con
                                                                           const uint32_t* __restrict__ lcut,
                                                                           int32_t* __restrict__ redo,
                                                                           int32_t* __restrict__ idx,
-                                                                          float* __restrict__ score_opt) {
+                                                                          float* __restrict__ score_opt,
+                                                                          const float* __restrict__ lhi) {
   __shared__ uint32_t hist[kSelWarps][kWarpBinWords];
+  __shared__ uint2 bnd[kSelWarps][kWarpBound];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kSelWarps + warp;
   if (t >= T) return;  // uniform across the warp
@@ -701,8 +703,17 @@ __global__ void __launch_bounds__(32 * kSelWarps, 3) list_select_warp_kernel(con
     return;
   }
   bool ok = c <= (uint32_t)cap;  // kNoList, or entries lost past cap: redone
-  if (ok) ok = warp_list_select(lists + (int64_t)t * stride, (int)c, __ldcg(lcut + t), (uint32_t)min(topk, nt), topk,
-                                hist[warp], oi, ov);
+  if (ok) {
+    const uint2* lt = lists + (int64_t)t * stride;
+    const uint32_t cut = __ldcg(lcut + t), need = (uint32_t)min(topk, nt);
+    // two passes when the list's score range is known (a cut placed from a sample), else the
+    // general rounds
+    int r = 2;
+    if (lhi && cut != 0u && cut != 0xffffffffu)
+      r = warp_list_select_binned(lt, (int)c, cut, key_to_float(cut), __ldcg(lhi + t), need, topk, hist[warp],
+                                  bnd[warp], oi, ov);
+    ok = r == 1 || (r == 2 && warp_list_select(lt, (int)c, cut, need, topk, hist[warp], oi, ov));
+  }
   if (lane == 0) redo[t] = ok ? 0 : nt;
 }
 
@@ -803,10 +814,10 @@ bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T,
 }
 
 void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const ListState& l, int32_t* idx,
-                             float* score_opt, cudaStream_t s) {
+                             float* score_opt, cudaStream_t s, const float* hi) {
   if (T <= 0) return;
   list_select_warp_kernel<<<(T + kSelWarps - 1) / kSelWarps, 32 * kSelWarps, 0, s>>>(
-      n, L, T, topk, l.list, l.stride, l.cap, l.cnt, l.cutkey, l.redo, idx, score_opt);
+      n, L, T, topk, l.list, l.stride, l.cap, l.cnt, l.cutkey, l.redo, idx, score_opt, hi);
 }
 
 void mark_no_lists(const ListState& l, int T, cudaStream_t s) {

@@ -135,7 +135,8 @@ __device__ __forceinline__ void warp_min_max(uint32_t& lo, uint32_t& hi) {
 // rank-th largest key, so at least rank sample keys are at or above it.  key(i) is sample key i
 // < ns (rank <= ns).
 template <class Key>
-__device__ __forceinline__ uint32_t warp_sample_cut(int ns, Key key, uint32_t rank, uint32_t* h) {
+__device__ __forceinline__ uint32_t warp_sample_cut(int ns, Key key, uint32_t rank, uint32_t* h,
+                                                    uint32_t* smax = nullptr) {
   auto load = [&](int i) { return make_uint2(key(i), 0u); };
   uint32_t lo = 0xffffffffu, hi = 0u;
   warp_each(ns, load, [&](int i, uint2 e) {
@@ -145,10 +146,86 @@ __device__ __forceinline__ uint32_t warp_sample_cut(int ns, Key key, uint32_t ra
     }
   });
   warp_min_max(lo, hi);
+  if (smax) *smax = hi;
   uint32_t above;
   bool all;
   return warp_rth_largest([&](auto g) { warp_each(ns, load, [&](int i, uint2 e) { g(e.x, i < ns); }); }, lo, hi,
                           rank, h, &above, &all);
+}
+
+// Top-k of a candidate list whose entries (keys at or above cut; key 0 is an empty slot) lie
+// mostly in [vlo, vhi] (the cut's score and the largest score of the sample that placed it;
+// larger scores go to the top bin), in two passes: one bins the entries linearly in 1024 bins,
+// the other writes the entries of the bins above the need-th entry's bin and keeps that bin's own
+// entries in bnd (kWarpBound of them at most), where a rank count (score, then token) orders them.
+// Returns 0 when fewer than need entries qualify, 2 when the bin holds more than kWarpBound
+// entries or the range is empty (nothing written in either case), 1 when the selection is written
+// to oi/ov [0, need) and padding to [need, topk).
+constexpr int kWarpBound = 128;
+__device__ __forceinline__ int warp_list_select_binned(const uint2* lt, int c, uint32_t cut, float vlo, float vhi,
+                                                       uint32_t need, int topk, uint32_t* h, uint2* bnd,
+                                                       int32_t* oi, float* ov) {
+  const int lane = threadIdx.x & 31;
+  const float scale = (float)kWarpBins / (vhi - vlo);
+  if (!(vhi > vlo) || !(scale > 0.f) || !(scale < 3.0e38f)) return 2;
+  auto load = [&](int i) { return __ldcg(lt + i); };
+  auto valid = [&](int i, uint2 e) { return i < c && e.x != 0u && e.x >= cut; };
+  auto bin = [&](uint32_t k) {
+    return (uint32_t)max(0, min(__float2int_rz((key_to_float(k) - vlo) * scale), kWarpBins - 1));
+  };
+#pragma unroll
+  for (int j = 0; j < (kWarpBinWords + 31) / 32; ++j)
+    if (32 * j + lane < kWarpBinWords) h[32 * j + lane] = 0u;
+  __syncwarp();
+  uint32_t cnt = 0;
+  warp_each(c, load, [&](int i, uint2 e) {
+    if (valid(i, e)) {
+      atomicAdd(&h[warp_bin_word(bin(e.x))], 1u);
+      ++cnt;
+    }
+  });
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
+  if (cnt < need) return 0;
+  __syncwarp();
+  const WarpBin wb = warp_bin(h, need);
+  if (wb.in > (uint32_t)kWarpBound) return 2;
+  const uint32_t need_in = need - wb.above;
+  const uint32_t below = (1u << lane) - 1u;
+  uint32_t pg = 0, pb = 0;
+  warp_each(c, load, [&](int i, uint2 e) {
+    const bool ok = valid(i, e);
+    const uint32_t b = ok ? bin(e.x) : 0u;
+    const bool gt = ok && b > wb.bin, eq = ok && b == wb.bin;
+    const unsigned mg = __ballot_sync(0xffffffffu, gt), me = __ballot_sync(0xffffffffu, eq);
+    if (gt) {
+      const uint32_t s = pg + (uint32_t)__popc(mg & below);
+      oi[s] = (int32_t)e.y;
+      if (ov) ov[s] = key_to_float(e.x);
+    }
+    if (eq) bnd[pb + (uint32_t)__popc(me & below)] = e;
+    pg += (uint32_t)__popc(mg);
+    pb += (uint32_t)__popc(me);
+  });
+  __syncwarp();
+  // the bin's entries: rank by score, then token; the first need_in are taken
+  for (uint32_t j = lane; j < wb.in; j += 32) {
+    const uint2 m = bnd[j];
+    uint32_t r = 0;
+    for (uint32_t i = 0; i < wb.in; ++i) {
+      const uint2 o = bnd[i];
+      r += (o.x > m.x) || (o.x == m.x && o.y < m.y);
+    }
+    if (r < need_in) {
+      oi[wb.above + r] = (int32_t)m.y;
+      if (ov) ov[wb.above + r] = key_to_float(m.x);
+    }
+  }
+  for (int a = (int)need + lane; a < topk; a += 32) {
+    oi[a] = -1;
+    if (ov) ov[a] = 0.f;
+  }
+  return 1;
 }
 
 // Top-k of one query's candidate list lt[0, c) of (order key, token): the entries with a key at or

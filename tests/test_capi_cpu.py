@@ -292,16 +292,16 @@ def test_bounds_checked_build_exports_the_same_calls():
 
 def test_fused_prefill_workspace_and_argument_checks(lib):
     """misa_score_topk_fused: workspace = candidate-list state (counts and cut keys [2, T], redo flags
-    [T], lists [T, 4k] of (key, token) pairs) + the cut [T] + the packed sample [T, ceil(ceil(L/128)/32)
-    * 128] + score rows [T, ceil4(L)] for the queries that are redone; k above 4096 (lists over 16384
-    entries) and fp32 inputs are unsupported."""
+    [T], lists [T, 4k] of (key, token) pairs) + the cut [T] + the sample's largest score [T] + the
+    packed sample [T, ceil(ceil(L/128)/32) * 128] + score rows [T, ceil4(L)] for the queries that are
+    redone; k above 4096 (lists over 16384 entries) and fp32 inputs are unsupported."""
     ws = lib.misa_workspace_bytes
     T, L, k = 4096, 65536, 2048
     cols = -(-(-(-L // 128)) // 32) * 128
-    want = (_al(T * 8) + _al(T * 4) + _al(T * 4 * k * 8) + _al(T * 4) + _al(T * cols * 4) +
+    want = (_al(T * 8) + _al(T * 4) + _al(T * 4 * k * 8) + 2 * _al(T * 4) + _al(T * cols * 4) +
             _al(T * (-(-L // 4) * 4) * 4))
     assert ws(9, T, L, 64, 128, 8, k, 0) == want
-    assert ws(9, 3, 1001, 64, 128, 8, 10, 0) == (_al(24) + _al(12) + _al(3 * 40 * 8) + _al(12) + _al(3 * 128 * 4) +
+    assert ws(9, 3, 1001, 64, 128, 8, 10, 0) == (_al(24) + _al(12) + _al(3 * 40 * 8) + 2 * _al(12) + _al(3 * 128 * 4) +
                                                  _al(3 * 1004 * 4))
     assert ws(9, T, L, 64, 128, 8, 4097, 0) == 0, "lists of more than 16384 entries"
     f = lib.misa_score_topk_fused
