@@ -55,8 +55,8 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "b2832ee84d6757b5ca450b10cbc4e73539f154c83556b905b3f97f9e44d9ae61",
-           "bytes_per_key": (1.073897e9 + 18.633472e6) / 4194304}
+           "sha256": "563bd1e63154ff27fd27781231e980992b784b507515b6f567ad79c3cbb1fc8d",
+           "bytes_per_key": (1.073898e9 + 19.067648e6) / 4194304}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
 # chunk's launch; the step's traffic is that rate times the pairs the step scores.
 TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
