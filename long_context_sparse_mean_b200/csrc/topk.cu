@@ -231,56 +231,16 @@ __device__ __forceinline__ void collect_above(const float* row, const int32_t* i
   }
 }
 
-// The r-th largest (1 <= r <= count) of the keys the block's threads visit, all within [lo, hi].
-// Round 0 bins the scores linearly over [value(lo), value(hi)] (4096 bins; smooth score
-// distributions spread evenly, so the shared-memory atomics rarely collide, where order keys crowd
-// the bulk of a set that spans both signs into a few bins); the boundary bin's own key range then
-// takes rounds of 4096 key bins until a bin holds exactly the missing count (*all = true: every key
-// of the bin is taken; the result is the bin's smallest key) or is one key wide (*all = false: the
-// result is that key; ties with it may straddle the r-th place).  each(g) calls g(key, counted) for
-// every member on the calling thread.  *above: the count of keys above the result's bin.  LINEAR
-// false skips round 0 (keys that are not order keys of finite scores).  hist: kHistBins words;
-// mm: 2 words; scratch: 35 words.
-template <bool LINEAR, class Each>
+// The r-th largest (1 <= r <= count) of the keys the block's threads visit, all within [lo, hi]:
+// rounds of 4096 key bins over what is left of the range until a bin holds exactly the missing
+// count (*all = true: every key of the bin is taken; the result is the bin's lower edge) or is one
+// key wide (*all = false: the result is that key).  each(g) calls g(key, counted) for every member
+// on the calling thread.  *above: the count of keys above the result's bin.  hist: kHistBins
+// words; scratch: 35 words.
+template <class Each>
 __device__ __forceinline__ uint32_t block_rth_largest(Each each, uint32_t lo, uint32_t hi, uint32_t r, uint32_t* hist,
-                                                      uint32_t* mm, uint32_t* scratch, uint32_t* above, bool* all) {
+                                                      uint32_t* scratch, uint32_t* above, bool* all) {
   uint32_t gt = 0;
-  const float vlo = key_to_float(lo), vhi = key_to_float(hi);
-  const float scale = (float)kHistBins / (vhi - vlo);
-  if (LINEAR && hi > lo && vhi > vlo && scale > 0.f && scale < 3.0e38f) {
-    for (int b = threadIdx.x; b < kHistBins; b += blockDim.x) hist[b] = 0;
-    __syncthreads();
-    each([&](uint32_t k, bool counted) {
-      if (counted) atomicAdd(&hist[linear_bin(k, vlo, scale)], 1u);
-    });
-    __syncthreads();
-    const Bucket bk = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch);
-    gt += r - bk.need;
-    r = bk.need;
-    // the bin's key range (linear_bin is monotone: lower bins hold smaller scores only)
-    if (threadIdx.x == 0) {
-      mm[0] = 0xffffffffu;
-      mm[1] = 0u;
-    }
-    __syncthreads();
-    uint32_t blo = 0xffffffffu, bhi = 0u;
-    each([&](uint32_t k, bool counted) {
-      if (counted && linear_bin(k, vlo, scale) == bk.prefix) {
-        blo = min(blo, k);
-        bhi = max(bhi, k);
-      }
-    });
-    block_min_max(blo, bhi, mm);
-    __syncthreads();
-    lo = mm[0];
-    hi = mm[1];
-    __syncthreads();
-    if (bk.eq == r) {
-      *above = gt;
-      *all = true;
-      return lo;
-    }
-  }
   uint32_t base = lo, range = hi - lo;
   for (;;) {
     const int sh = range >= (uint32_t)kHistBins ? 32 - __clz(range) - 12 : 0;
@@ -305,56 +265,135 @@ __device__ __forceinline__ uint32_t block_rth_largest(Each each, uint32_t lo, ui
 }
 
 // Top `need` of the c list entries (c >= need, keys within [lo, hi]) in shared memory, written to
-// oi/ov [0, need) in no particular order: block_rth_largest finds the need-th key kstar, exact ties
-// at kstar that straddle the place go to the lower tokens (a second search over the tied entries'
-// tokens), and one pass writes every entry above kstar and the tied ones taken.  The list is only
-// read.  ctr: 2 words; scratch: 35 words.
+// oi/ov [0, need) in no particular order.  Rounds of 4096 bins narrow a key interval [ilo, ihi]
+// that holds the need-th entry: the first round bins the keys themselves when they share one sign
+// (order keys are close to logarithmic in the score, so outliers do not crowd the bulk into a few
+// bins) and bins linearly in the score otherwise; later rounds bin the interval's keys.  Once the
+// interval holds at most 256 entries (or one key), one pass writes every entry above it and moves
+// the interval's entries into the histogram's words (hist: 16-byte aligned), where a rank count
+// (score, then token) places them.  An exact tie of more than 2048 entries at one key takes the
+// lowest tokens by a search over the tokens.  The list is only read.  ctr: 2 words; mm: 2 words;
+// scratch: 35 words.
 template <int NT>
 __device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
                                   uint32_t* ctr, uint32_t* mm, uint32_t* scratch, int32_t* oi, float* ov) {
+  constexpr uint32_t kRank = 256;            // interval entries a rank count orders
+  constexpr uint32_t kBuf = kHistBins / 2;   // (key, token) pairs the histogram's words hold
   const int tid = threadIdx.x;
-  uint32_t above;
-  bool all;
-  const uint32_t kstar = block_rth_largest<true>(
-      [&](auto g) {
-        for (int i = tid; i < c; i += NT) g(list[i].x, true);
-      },
-      lo, hi, need, hist, mm, scratch, &above, &all);
-  uint32_t tok = 0xffffffffu;  // tied entries at kstar taken: every one (all), else tokens <= tok
-  if (!all) {
-    if (tid == 0) {
-      mm[0] = 0xffffffffu;
-      mm[1] = 0u;
+  uint32_t ilo = lo, ihi = hi, r = need, eq = (uint32_t)c;
+  const bool one_sign = lo >= 0x80000000u || hi < 0x80000000u;
+  for (int round = 0; round < 4 && eq > kRank && ihi > ilo; ++round) {
+    const float vlo = key_to_float(ilo);
+    const float scale = (float)kHistBins / (key_to_float(ihi) - vlo);
+    const bool lin = round == 0 && !one_sign && scale > 0.f && scale < 3.0e38f;
+    const uint32_t range = ihi - ilo;
+    const int sh = range >= (uint32_t)kHistBins ? 32 - __clz(range) - 12 : 0;
+    auto bin_of = [&](uint32_t k) { return lin ? linear_bin(k, vlo, scale) : (k - ilo) >> sh; };
+    for (int b = tid; b < kHistBins; b += NT) hist[b] = 0;
+    __syncthreads();
+    for (int i = tid; i < c; i += NT) {
+      const uint32_t k = list[i].x;
+      if (k >= ilo && k <= ihi) atomicAdd(&hist[bin_of(k)], 1u);
     }
     __syncthreads();
-    uint32_t tlo = 0xffffffffu, thi = 0u;
-    for (int i = tid; i < c; i += NT)
-      if (list[i].x == kstar) {
-        tlo = min(tlo, 0xffffffffu - list[i].y);
-        thi = max(thi, 0xffffffffu - list[i].y);
+    const Bucket bk = block_bucket_bits(hist, kHistBins, 0, 0u, r, scratch);  // bin in prefix
+    r = bk.need;
+    eq = bk.eq;
+    if (lin) {  // the bin's key range (linear_bin is monotone)
+      if (tid == 0) {
+        mm[0] = 0xffffffffu;
+        mm[1] = 0u;
       }
-    block_min_max(tlo, thi, mm);
-    __syncthreads();
-    tlo = mm[0];
-    thi = mm[1];
-    uint32_t a2;
-    bool all2;
-    tok = 0xffffffffu - block_rth_largest<false>(
-                            [&](auto g) {
-                              for (int i = tid; i < c; i += NT) {
-                                const uint2 e = list[i];
-                                g(0xffffffffu - e.y, e.x == kstar);
-                              }
-                            },
-                            tlo, thi, need - above, hist, mm, scratch, &a2, &all2);
+      __syncthreads();
+      uint32_t blo = 0xffffffffu, bhi = 0u;
+      for (int i = tid; i < c; i += NT) {
+        const uint32_t k = list[i].x;
+        if (k >= ilo && k <= ihi && bin_of(k) == bk.prefix) {
+          blo = min(blo, k);
+          bhi = max(bhi, k);
+        }
+      }
+      block_min_max(blo, bhi, mm);
+      __syncthreads();
+      ilo = mm[0];
+      ihi = mm[1];
+      __syncthreads();
+    } else {
+      const uint32_t base = ilo + (bk.prefix << sh);
+      ihi = min(ihi, base + ((1u << sh) - 1u));
+      ilo = base;
+    }
   }
+  const uint32_t n_gt = need - r;  // entries above the interval, all taken
+  if (eq <= kBuf) {
+    uint2* bl = reinterpret_cast<uint2*>(hist);
+    if (tid == 0) {
+      ctr[0] = 0;
+      ctr[1] = 0;
+    }
+    __syncthreads();
+    const int steps = (c + NT - 1) / NT;
+    for (int j = 0; j < steps; ++j) {
+      const int i = j * NT + tid;
+      const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
+      const bool gt = i < c && e.x > ihi, in = i < c && e.x >= ilo && e.x <= ihi;
+      const uint32_t slot = warp_slot(gt, &ctr[0]);
+      if (gt) {
+        oi[slot] = (int32_t)e.y;
+        if (ov) ov[slot] = key_to_float(e.x);
+      }
+      const uint32_t s2 = warp_slot(in, &ctr[1]);
+      if (in) bl[s2] = e;
+    }
+    __syncthreads();
+    for (uint32_t j = tid; j < eq; j += NT) {
+      const uint2 m = bl[j];
+      uint32_t rk = 0;
+      for (uint32_t i = 0; i < eq; ++i) {
+        const uint2 o = bl[i];
+        rk += (o.x > m.x) || (o.x == m.x && o.y < m.y);
+      }
+      if (rk < r) {
+        oi[n_gt + rk] = (int32_t)m.y;
+        if (ov) ov[n_gt + rk] = key_to_float(m.x);
+      }
+    }
+    return;
+  }
+  // more than kBuf entries share the key ilo == ihi: the r lowest tokens among them, as the largest
+  // values of 0xffffffff - token
+  if (tid == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+  __syncthreads();
+  uint32_t tlo = 0xffffffffu, thi = 0u;
+  for (int i = tid; i < c; i += NT)
+    if (list[i].x == ilo) {
+      tlo = min(tlo, 0xffffffffu - list[i].y);
+      thi = max(thi, 0xffffffffu - list[i].y);
+    }
+  block_min_max(tlo, thi, mm);
+  __syncthreads();
+  tlo = mm[0];
+  thi = mm[1];
+  uint32_t a2;
+  bool all2;
+  const uint32_t tok = 0xffffffffu - block_rth_largest(
+                                         [&](auto g) {
+                                           for (int i = tid; i < c; i += NT) {
+                                             const uint2 e = list[i];
+                                             g(0xffffffffu - e.y, e.x == ilo);
+                                           }
+                                         },
+                                         tlo, thi, r, hist, scratch, &a2, &all2);
   if (tid == 0) ctr[0] = 0;
   __syncthreads();
   const int steps = (c + NT - 1) / NT;
   for (int j = 0; j < steps; ++j) {
     const int i = j * NT + tid;
     const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
-    const bool sel = i < c && (e.x > kstar || (e.x == kstar && (all || e.y <= tok)));
+    const bool sel = i < c && (e.x > ihi || (e.x == ilo && e.y <= tok));
     const uint32_t slot = warp_slot(sel, &ctr[0]);
     if (sel) {
       oi[slot] = (int32_t)e.y;
@@ -382,7 +421,7 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
                                                             int64_t lstride, int32_t* __restrict__ redo,
                                                             const int32_t* __restrict__ only) {
   extern __shared__ uint2 list[];  // [LIST]
-  __shared__ uint32_t hp[kHistPadded];
+  __shared__ __align__(16) uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t cnt[2];
   __shared__ uint32_t mm[2];
@@ -467,7 +506,48 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
     } else {
       __syncthreads();
     }
-    if (!exact) collect_above<NT>(row, ids, np, nt, vec, thr, list, LIST, &cnt[0], mm);
+    if (!exact && ids && np <= LIST) {
+      // a candidate list: every entry with a valid token is kept; four entries a thread and step,
+      // one block scan places a step's entries (no per-entry atomics or reloads)
+      uint32_t lo = 0xffffffffu, hi = 0u, base = 0;
+      const bool vec4 = vec && (reinterpret_cast<uintptr_t>(ids) & 15) == 0;
+      for (int p0 = 0; p0 < np; p0 += 4 * NT) {
+        const int p = p0 + 4 * tid;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        int32_t id[4] = {-1, -1, -1, -1};
+        if (vec4 && p + 3 < np) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(row + p));
+          const int4 y = __ldcg(reinterpret_cast<const int4*>(ids + p));
+          v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+          id[0] = y.x, id[1] = y.y, id[2] = y.z, id[3] = y.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (p + e < np) {
+              v[e] = __ldcg(row + p + e);
+              id[e] = __ldcg(ids + p + e);
+            }
+        }
+        uint32_t m = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) m |= (uint32_t)(id[e] >= 0 && id[e] < nt) << e;
+        uint32_t total;
+        uint32_t pos = base + block_exclusive_scan((uint32_t)__popc(m), scratch, &total);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          if ((m >> e) & 1u) {
+            const uint32_t k = order_key(v[e]);
+            lo = min(lo, k);
+            hi = max(hi, k);
+            list[pos++] = make_uint2(k, (uint32_t)id[e]);
+          }
+        base += total;
+      }
+      if (tid == 0) cnt[0] = base;
+      block_min_max(lo, hi, mm);
+    } else if (!exact) {
+      collect_above<NT>(row, ids, np, nt, vec, thr, list, LIST, &cnt[0], mm);
+    }
   } else {
     __syncthreads();
   }
