@@ -137,14 +137,16 @@ __device__ __forceinline__ void row_sweep(const float* row, int nt, bool vec, F&
   }
 }
 
-// Appends (key, token) of every entry p < np whose score is >= thr to the list and folds the
-// appended keys into mm[0] (min) and mm[1] (max).  The token is p, or ids[p] for candidate lists
-// (entries whose id is outside [0, nt) are skipped).  A thread reads 16 entries (4 float4) a
-// step, the next step's loads in flight while it handles the current one, and marks its
-// candidates in a bit mask; one warp scan and one shared atomic per warp and step place them.
+// Appends (key, token p) of every entry p < np of a score row whose score is >= thr to the list and
+// folds the appended keys into mm[0] (min) and mm[1] (max).  A thread reads 16 entries (4 float4) a
+// step, the next step's loads in flight while it handles the current one, and marks its candidates
+// in a bit mask; one warp scan and one shared atomic per warp and step place them.  The lanes then
+// take their candidates one per round (lowest set bit, its value picked from the 16 by a select
+// tree), as many rounds as the lane with the most candidates needs, which for a sampled cut is two
+// or three instead of a pass over all 16 bits.
 template <int NT>
-__device__ __forceinline__ void collect_above(const float* row, const int32_t* ids, int np, int nt, bool vec,
-                                              float thr, uint2* list, int cap, uint32_t* cnt, uint32_t* mm) {
+__device__ __forceinline__ void collect_above(const float* row, int np, bool vec, float thr, uint2* list, int cap,
+                                              uint32_t* cnt, uint32_t* mm) {
   constexpr int U = 4;  // float4 per thread and step
   const int lane = threadIdx.x & 31;
   uint32_t lo = 0xffffffffu, hi = 0u;
@@ -152,27 +154,15 @@ __device__ __forceinline__ void collect_above(const float* row, const int32_t* i
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const int i = (j0 + u) * NT + (int)threadIdx.x;
-      float v[4] = {NAN, NAN, NAN, NAN};  // NaN: never at or above the threshold
       if (vec && 4 * i + 3 < np) {
-        const float4 f = __ldcg(reinterpret_cast<const float4*>(row) + i);
-        v[0] = f.x;
-        v[1] = f.y;
-        v[2] = f.z;
-        v[3] = f.w;
+        x[u] = __ldcg(reinterpret_cast<const float4*>(row) + i);
       } else {
+        float v[4] = {NAN, NAN, NAN, NAN};  // NaN: never at or above the threshold
 #pragma unroll
         for (int e = 0; e < 4; ++e)
           if (4 * i + e < np) v[e] = __ldcg(row + 4 * i + e);
+        x[u] = make_float4(v[0], v[1], v[2], v[3]);
       }
-      if (ids) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int p = 4 * i + e;
-          const int32_t id = p < np ? __ldcg(ids + p) : -1;
-          if (id < 0 || id >= nt) v[e] = NAN;
-        }
-      }
-      x[u] = make_float4(v[0], v[1], v[2], v[3]);
     }
   };
   const int steps = ((np + 3) / 4 + NT - 1) / NT;  // float4 groups a thread
@@ -198,23 +188,21 @@ __device__ __forceinline__ void collect_above(const float* row, const int32_t* i
     uint32_t base = 0;
     if (lane == 31 && incl) base = atomicAdd(cnt, incl);
     base = __shfl_sync(0xffffffffu, base, 31);
-    if (m) {
-      uint32_t pos = base + incl - c;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int s0 = 4 * ((j0 + u) * NT + (int)threadIdx.x);
-        const float v[4] = {cur[u].x, cur[u].y, cur[u].z, cur[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          if ((m >> (4 * u + e)) & 1u) {
-            const uint32_t k = order_key(v[e]);
-            lo = min(lo, k);
-            hi = max(hi, k);
-            const uint32_t tok = ids ? (uint32_t)__ldcg(ids + s0 + e) : (uint32_t)(s0 + e);
-            if (pos < (uint32_t)cap) list[pos] = make_uint2(k, tok);
-            ++pos;
-          }
-        }
+    uint32_t pos = base + incl - c;
+    const uint32_t rounds = __reduce_max_sync(0xffffffffu, c);
+    for (uint32_t r = 0; r < rounds; ++r) {
+      if (m) {
+        const int b = __ffs(m) - 1;
+        m &= m - 1u;
+        // entry b: float4 b >> 2, component b & 3
+        const float4 q = (b & 8) ? ((b & 4) ? cur[3] : cur[2]) : ((b & 4) ? cur[1] : cur[0]);
+        const float v = (b & 2) ? ((b & 1) ? q.w : q.z) : ((b & 1) ? q.y : q.x);
+        const uint32_t k = order_key(v);
+        lo = min(lo, k);
+        hi = max(hi, k);
+        const uint32_t tok = (uint32_t)(4 * ((j0 + (b >> 2)) * NT + (int)threadIdx.x) + (b & 3));
+        if (pos < (uint32_t)cap) list[pos] = make_uint2(k, tok);
+        ++pos;
       }
     }
 #pragma unroll
@@ -506,7 +494,7 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
     } else {
       __syncthreads();
     }
-    if (!exact && ids && np <= LIST) {
+    if (!exact && ids) {  // P <= LIST (checked on the host)
       // a candidate list: every entry with a valid token is kept; four entries a thread and step,
       // one block scan places a step's entries (no per-entry atomics or reloads)
       uint32_t lo = 0xffffffffu, hi = 0u, base = 0;
@@ -546,7 +534,7 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
       if (tid == 0) cnt[0] = base;
       block_min_max(lo, hi, mm);
     } else if (!exact) {
-      collect_above<NT>(row, ids, np, nt, vec, thr, list, LIST, &cnt[0], mm);
+      collect_above<NT>(row, np, vec, thr, list, LIST, &cnt[0], mm);
     }
   } else {
     __syncthreads();
