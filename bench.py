@@ -863,9 +863,11 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
-    # kernels per step: router, routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank,
-    # top-k of the candidates
-    launches_per_step = 7
+    fused = args.dagger == "fused" and kp is not None
+    # kernels per step.  Fused: router, sampled scores, list cut, routed scorer keeping the dense
+    # scores of the tokens at or above the cut, the two selections (one CTA per row).  Unfused: router,
+    # routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank, top-k of the candidates.
+    launches_per_step = 5 if fused else 7
 
     def route():
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
@@ -879,11 +881,21 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     def rerank():
         M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
 
-    def step():
+    def fused_rest():
+        M.misa_hier_topk_fused(qd, wd, kd, nd, heads, kp, kk, idx=idx, vals=vals, ws=sel_ws)
+
+    def step_unfused():
         route()
         score()
         select()
         rerank()
+
+    def step_fused():
+        route()
+        fused_rest()
+
+    step = step_fused if fused else step_unfused
+    other_step = step_unfused if fused else (step_fused if kp is not None else None)
 
     for _ in range(max(3, args.warmup)):
         step()
@@ -895,12 +907,22 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         # no host gaps); the routed scoring call is the roofline's kernel
         nrep = max(3, min(args.steps, 20))
         stages_us = {}
-        for nm, fn in (("route", route), ("routed_scores", score), ("topk_kprime", select), ("rerank", rerank)):
+        stage_fns = [("route", route), ("routed_scores", score)]
+        stage_fns += [("scores_and_selections_fused", fused_rest)] if fused else \
+            [("topk_kprime", select), ("rerank", rerank)]
+        for nm, fn in stage_fns:
             g = _graphed(torch, fn, not args.no_graph)
             g()
             stages_us[nm] = round(1000 * _event_ms(torch, stream, g, nrep), 2)
             if nm == "routed_scores":
                 score_avg = stages_us[nm] / 1000.0
+            del g
+        # the other composition of the same MISA-dagger step, for comparison (not the headline)
+        other_ms = None
+        if other_step is not None:
+            g = _graphed(torch, other_step, not args.no_graph)
+            g()
+            other_ms = _event_ms(torch, stream, g, nrep)
             del g
         step()  # the stages above reran on the same inputs; leave one whole step's state behind
         torch.cuda.synchronize()
@@ -991,6 +1013,9 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,
+            "dagger_step": "fused (misa_route + misa_hier_topk_fused)" if fused else
+                           "unfused (misa_route, misa_token_scores, misa_topk_select, misa_hier_rerank)",
+            "other_dagger_step_ms": other_ms,
             "clocks": clk.summary("scorer, stage and timed passes"),
             "dense_dsa_same_inputs": None if dsa_ms is None else {
                 "ms_per_call": dsa_ms, "query_tokens_per_s": T * L / (dsa_ms / 1000.0),
@@ -1077,6 +1102,9 @@ def main():
                     help="decode: skip the prefill and GLM-5-shaped decode legs that follow the main line")
     ap.add_argument("--fused", action="store_true",
                     help="prefill main line: score and select each chunk with misa_score_topk_fused (no score rows)")
+    ap.add_argument("--dagger", choices=["fused", "unfused"], default="fused",
+                    help="MISA-dagger decode step: one call for scores and both selections (fused), or the "
+                         "separate scoring, top-k' and re-rank calls (unfused; the other is timed beside it)")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
     ap.add_argument("--paged", type=int, default=64, metavar="PAGE_SIZE",

@@ -77,7 +77,8 @@ typedef enum {
   MISA_OP_ROUTE_PAGED = 6,
   MISA_OP_SCORE_TOPK_PAGED = 7,
   MISA_OP_RERANK_PAGED = 8,
-  MISA_OP_SCORE_TOPK_FUSED = 9
+  MISA_OP_SCORE_TOPK_FUSED = 9,
+  MISA_OP_HIER_FUSED = 10
 } misa_op;
 
 /* Largest k' accepted by misa_hier_rerank (its candidates are ranked in shared memory). */
@@ -298,6 +299,34 @@ misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, 
                                   const int32_t* heads, int T, int L, int H_I, int d, int h,
                                   int topk, int dtype, int32_t* idx, float* score_opt, void* ws,
                                   size_t ws_bytes, void* stream);
+
+/*
+ * MISA-dagger for decode batches with one key cache per query, without gathering the candidates
+ * ("Hierarchical Variant (MISA-dagger)": the top-k' tokens by the routed score are re-scored with
+ * all H_I heads and the top-k of that dense score is kept).  The result is misa_score_topk with
+ * topk = k' followed by misa_hier_rerank on its candidates, up to the rounding of the dense scores
+ * (a different summation on the tensor cores: near-ties at the k-th dense score may be ordered
+ * differently).  For fewer than 256 queries longer than 16384 keys and h <= 8, the list cut's sample
+ * of each prefix (256 evenly spaced runs of 8 keys) is scored first, each query's cut is placed on
+ * it (the expected number of sampled scores above the k'-th, plus three standard deviations and a
+ * margin), and one pass over the keys writes every routed score and keeps each token at or above
+ * the cut with its dense score, computed from the key row the pass already holds; the top-k' of
+ * those by the routed score and the top-k of them by the dense score are then selected.  A query
+ * whose kept tokens are fewer than k' or overflow 16384 is answered exactly from its score row on
+ * the device (the dense scores of its k' candidates computed there), so the selected set never
+ * depends on the sample.  Other shapes take that exact way for every query.
+ *   k         : per-query caches [T, L, d] (k_seq_stride >= L * d), bf16 like q
+ *   heads     : [T, h] routed heads (misa_route)
+ *   idx       : out [T, topk] the kept tokens (order not specified), -1 padded when n_t < topk
+ *   score_opt : out [T, topk] their dense scores, or NULL
+ *   ws        : misa_workspace_bytes(MISA_OP_HIER_FUSED, T, L, H_I, 0, h, topk, kp) bytes
+ * Requires topk <= kp <= MISA_MAX_KP (else MISA_ERR_INVALID_ARG / MISA_ERR_UNSUPPORTED); a shared
+ * cache (k_seq_stride 0) or fp32 inputs give MISA_ERR_UNSUPPORTED.
+ */
+misa_status misa_hier_topk_fused(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                                 const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d,
+                                 int h, int kp, int topk, int dtype, int32_t* idx, float* score_opt,
+                                 void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Device-side status of the calls made so far on the current device.  The tensor-core kernels

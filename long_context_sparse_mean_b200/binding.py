@@ -31,7 +31,7 @@ LIB_PATH = os.path.join(PKG, "libmisa_checked.so" if os.environ.get("MISA_LIBRAR
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE_TIMEOUT, ERR_BAD_INDEX = range(7)
 BF16, F32 = 0, 1
 (OP_ROUTE, OP_SCORE_TOPK, OP_RERANK, OP_DENSE_TOPK, OP_TOPK_SELECT, OP_BLOCK_FILTER, OP_ROUTE_PAGED,
- OP_SCORE_TOPK_PAGED, OP_RERANK_PAGED, OP_SCORE_TOPK_FUSED) = range(10)
+ OP_SCORE_TOPK_PAGED, OP_RERANK_PAGED, OP_SCORE_TOPK_FUSED, OP_HIER_FUSED) = range(11)
 MAX_KP = 16384
 
 if not os.path.exists(LIB_PATH):
@@ -70,6 +70,7 @@ def _setup(lib):
         "misa_hier_rerank_paged": ([P, P, P, i64, i32, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz,
                                     P], i32),
         "misa_score_topk_fused": ([P, P, P, P, P, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
+        "misa_hier_topk_fused": ([P, P, P, i64, P, P, i32, i32, i32, i32, i32, i32, i32, i32, P, P, P, sz, P], i32),
     }
     for name, (args, res) in sigs.items():
         f = getattr(lib, name)
@@ -453,6 +454,38 @@ def misa_score_topk_fused(q, w, k, n, heads, topk: int, idx=None, vals=None, wan
     _check("misa_score_topk_fused", _lib.misa_score_topk_fused(
         _p(q), _p(w), _p(k), _p(n), _p(heads), T, L, H_I, d, h, topk, BF16, _p(idx), _p(vals), _p(buf), nbytes,
         _stream(stream)))
+    return idx, vals
+
+
+def misa_hier_topk_fused(q, w, k, n, heads, kp: int, topk: int, idx=None, vals=None, want_vals=True,
+                         ws: Optional[Workspace] = None, stream=None):
+    """MISA-dagger for per-query bf16 caches k [T, L, d] in one call: routed scores, top-k' by them,
+    dense scores of those k' kept while the keys are read once, top-k of the dense score ->
+    (idx [T, k], vals [T, k])."""
+    T, H_I, d = _queries(q, w, n)
+    if k.dim() != 3:
+        raise ValueError(f"k must be per-query caches [T, L, d], got {tuple(k.shape)}")
+    L, kss = _cache(k, T, d)
+    _matrix(heads, "heads", T)
+    _outputs(T, topk, idx, vals)
+    _need(q, "q", torch.bfloat16)
+    _need(k, "k", torch.bfloat16)
+    _need(w, "w", torch.float32)
+    _need(n, "n", torch.int32)
+    _need(heads, "heads", torch.int32)
+    _need_opt(idx, "idx", torch.int32)
+    _need_opt(vals, "vals", torch.float32)
+    _on_device(q, k, w, n, heads, idx, vals)
+    h = heads.shape[1]
+    if idx is None:
+        idx = torch.empty((T, topk), dtype=torch.int32, device=q.device)
+    if vals is None and want_vals:
+        vals = torch.empty((T, topk), dtype=torch.float32, device=q.device)
+    nbytes = misa_workspace_bytes(OP_HIER_FUSED, T, L, H_I, 0, h, topk, kp)
+    buf = _ws(ws, q.device, stream).get(nbytes, stream)
+    _check("misa_hier_topk_fused", _lib.misa_hier_topk_fused(
+        _p(q), _p(w), _p(k), kss, _p(n), _p(heads), T, L, H_I, d, h, kp, topk, BF16, _p(idx), _p(vals), _p(buf),
+        nbytes, _stream(stream)))
     return idx, vals
 
 

@@ -171,6 +171,15 @@ misa_status misa_device_check(void) {
   return (bad[0] || bad[1] || bad[2]) ? MISA_ERR_BAD_INDEX : MISA_OK;
 }
 
+// misa_hier_topk_fused: [score rows][list counts][cuts][dense lists (entries, dense scores)]
+// [candidates][their dense scores]
+size_t hier_fused_ws(int T, int L, int kp) {
+  if (T <= 0 || L <= 0 || kp <= 0) return 0;
+  const size_t cap = misa::kListCap;
+  return scores_part(T, L) + 2 * align_up(sizeof(uint32_t) * (size_t)T) + align_up(sizeof(uint2) * (size_t)T * cap) +
+         align_up(sizeof(float) * (size_t)T * cap) + 2 * align_up(sizeof(int32_t) * (size_t)T * kp);
+}
+
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
   (void)h;
   switch (op) {
@@ -193,6 +202,8 @@ size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int top
       return rerank_paged_ws(T, kp);
     case MISA_OP_SCORE_TOPK_FUSED:
       return T > 0 && L > 0 && misa::fused_cap(topk) > 0 ? align_up(misa::fused_ws_bytes(T, L, topk)) : 0;
+    case MISA_OP_HIER_FUSED:
+      return hier_fused_ws(T, L, kp);
     default:
       return 0;
   }
@@ -507,6 +518,55 @@ misa_status misa_score_topk_fused(const void* q, const float* w, const void* k, 
     misa::launch_scores(misa::DType::BF16, q, w, k, 0, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, s);
     misa::launch_topk_rows(rows, ld, nullptr, 0, n, T, L, topk, nullptr, idx, score_opt, s);
   }
+  return launch_status();
+}
+
+misa_status misa_hier_topk_fused(const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                                 const int32_t* n, const int32_t* heads, int T, int L, int H_I, int d, int h, int kp,
+                                 int topk, int dtype, int32_t* idx, float* score_opt, void* ws, size_t ws_bytes,
+                                 void* stream) {
+  misa_status st = check_common(q, w, k, n, T, L, H_I, d, dtype, k_seq_stride);
+  if (st != MISA_OK) return st;
+  if (!heads && T > 0) return MISA_ERR_INVALID_ARG;
+  if (h < 1 || h > H_I || topk < 1 || kp < topk) return MISA_ERR_INVALID_ARG;
+  if (kp > MISA_MAX_KP) return MISA_ERR_UNSUPPORTED;
+  if (dtype != MISA_BF16 || k_seq_stride == 0) return MISA_ERR_UNSUPPORTED;
+  if (T == 0) return MISA_OK;
+  if (!idx) return MISA_ERR_INVALID_ARG;
+  if (!ws || ws_bytes < hier_fused_ws(T, L, kp) || !aligned(ws)) return MISA_ERR_WORKSPACE;
+  const cudaStream_t s = as_stream(stream);
+  const int64_t ld = score_ld(L);
+  char* p = static_cast<char*>(ws);
+  float* rows = reinterpret_cast<float*>(p);
+  p += scores_part(T, L);
+  misa::DenseList dl{};
+  dl.cnt = reinterpret_cast<uint32_t*>(p);
+  p += align_up(sizeof(uint32_t) * (size_t)T);
+  uint32_t* cut = reinterpret_cast<uint32_t*>(p);
+  dl.cut = cut;
+  p += align_up(sizeof(uint32_t) * (size_t)T);
+  dl.cap = misa::kListCap;
+  dl.stride = misa::kListCap;
+  dl.list = reinterpret_cast<uint2*>(p);
+  p += align_up(sizeof(uint2) * (size_t)T * dl.cap);
+  dl.f = reinterpret_cast<float*>(p);
+  p += align_up(sizeof(float) * (size_t)T * dl.cap);
+  int32_t* ctok = reinterpret_cast<int32_t*>(p);
+  p += align_up(sizeof(int32_t) * (size_t)T * kp);
+  float* cf = reinterpret_cast<float*>(p);
+  // lists for a few long rows (many rows fill the GPU with one CTA per row already); the scorer's
+  // shared memory must fit two CTAs per SM
+  const bool lists = T <= misa::kDenseListMaxRows && L > dl.cap && h <= 8 &&
+                     misa::dense_list_smem(T, H_I) <= misa::kDenseListMaxSmem;
+  if (lists) {
+    misa::launch_scores_sample(q, w, k, k_seq_stride, n, heads, T, L, H_I, h, dl.cap, rows, ld, s);
+    misa::launch_list_cut(rows, ld, n, T, L, kp, dl.cap, dl.cnt, cut, s);
+    misa::launch_scores_dense_list(q, w, k, k_seq_stride, n, heads, T, L, H_I, h, rows, ld, dl, s);
+  } else {
+    cudaMemsetAsync(dl.cnt, 0xff, sizeof(uint32_t) * (size_t)T, s);  // kNoList: every row from its score row
+    misa::launch_scores(misa::DType::BF16, q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, s);
+  }
+  misa::launch_hier_select(rows, ld, n, T, L, kp, topk, dl, q, w, k, k_seq_stride, H_I, ctok, cf, idx, score_opt, s);
   return launch_status();
 }
 

@@ -71,6 +71,44 @@ bool launch_list_build(const float* scores, int64_t ld, const int32_t* n, int T,
 void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const ListState& l, int32_t* idx,
                              float* score_opt, cudaStream_t s, const float* hi = nullptr);
 
+// MISA-dagger decode in one pass over the keys ("Hierarchical Variant (MISA-dagger)"), for one
+// cache per query, h <= 8 and bf16: launch_scores_sample scores the list cut's sample of every row
+// longer than the cap (kSampleRuns runs of kSampleRunLen tokens, into the score rows at those
+// tokens), launch_list_cut places each row's cut on it (with topk = k'), launch_scores_dense_list
+// writes every routed score and appends each token at or above the cut with its dense score over
+// all H_I heads (computed from the key row the scorer already holds: nothing is gathered), and
+// launch_hier_select takes per row the top-k' by the routed score, then the top-k of those by the
+// dense score.
+struct DenseList {
+  uint2* list;          // [T][stride] (order key of the routed score, token)
+  float* f;             // [T][stride] the dense score of the same token
+  uint32_t* cnt;        // [T] entries appended (also past cap); kNoList: no list for this row
+  const uint32_t* cut;  // [T] the row's cut as an order key
+  int64_t stride;
+  int cap;
+};
+constexpr size_t kDenseListMaxSmem = 110 * 1024;  // dynamic shared memory of the list scorer (2 CTAs per SM)
+constexpr int kDenseListMaxRows = 255;            // lists pay off for a few rows (one CTA per row fills the GPU)
+size_t dense_list_smem(int T, int H_I);
+// False (nothing launched) unless h <= 8, per-query caches and T <= 8192.
+bool launch_scores_sample(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                          const int32_t* heads, int T, int L, int H_I, int h, int cap, float* out, int64_t ld,
+                          cudaStream_t s);
+// Rows whose cnt[t] is kNoList get their scores only.  False (nothing launched) as above, or when
+// the shared memory would not fit.
+bool launch_scores_dense_list(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                              const int32_t* heads, int T, int L, int H_I, int h, float* out, int64_t ld,
+                              const DenseList& dl, cudaStream_t s);
+// The cut of list_cut_kernel alone (cnt[t] = 0 and cut[t], or cnt[t] = kNoList).
+void launch_list_cut(const float* scores, int64_t ld, const int32_t* n, int T, int L, int topk, int cap,
+                     uint32_t* lcnt, uint32_t* lcut, cudaStream_t s);
+// One CTA per row (kp <= 16384): idx [T, topk] (score_opt: the dense scores) from the dense lists, or
+// for a row they cannot answer, from its score row (exact top-k', dense scores of the candidates
+// computed here).  ctok / cf: [T][kp] scratch.
+void launch_hier_select(const float* scores, int64_t ld, const int32_t* n, int T, int L, int kp, int topk,
+                        const DenseList& dl, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                        int H_I, int32_t* ctok, float* cf, int32_t* idx, float* score_opt, cudaStream_t s);
+
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
 // position p of query t scores token rows[t*P + p] and writes out[t*ld + p].
 void launch_scores(DType dt, const void* q, const float* w, const void* k, int64_t k_seq_stride,

@@ -50,6 +50,18 @@ __device__ __forceinline__ void stage_q_frags(uint2 (*frag)[8][32], const __nv_b
   }
 }
 
+// The B fragments of all H_I heads in head order, ngf = ceil(H_I / 8) groups (slots past H_I repeat
+// head 0; their weight is 0), by the NT threads of the block.  Same layout as stage_q_frags.
+template <int NT>
+__device__ __forceinline__ void stage_all_head_frags(uint2 (*frag)[8][32], const __nv_bfloat16* qt, int H_I,
+                                                     int ngf) {
+  for (int e = (int)threadIdx.x; e < ngf * 256; e += NT) {
+    const int ng = e >> 8, kk = (e >> 5) & 7, ln = e & 31;
+    const int hd = ng * 8 + (ln >> 2);
+    frag[ng][kk][ln] = *reinterpret_cast<const uint2*>(qt + (int64_t)(hd < H_I ? hd : 0) * kD + frag_dim(kk, ln & 3));
+  }
+}
+
 // Load the A data of one 16-row group: rows ra (lane row g) and rb (row g+8); null = zeros.
 __device__ __forceinline__ void load_rows(const __nv_bfloat16* ra, const __nv_bfloat16* rb, int c, uint4 (&A)[4],
                                           uint4 (&Bq)[4]) {
@@ -82,6 +94,38 @@ __device__ __forceinline__ void score_rows(const uint4 (&A)[4], const uint4 (&Bq
     slo = fmaf(wb[ng], relu(acc[1]), slo);
     shi = fmaf(wa[ng], relu(acc[2]), shi);
     shi = fmaf(wb[ng], relu(acc[3]), shi);
+  }
+  slo += __shfl_xor_sync(0xffffffffu, slo, 1);
+  shi += __shfl_xor_sync(0xffffffffu, shi, 1);
+  slo += __shfl_xor_sync(0xffffffffu, slo, 2);
+  shi += __shfl_xor_sync(0xffffffffu, shi, 2);
+  s_lo = __fadd_rn(slo, 0.0f);
+  s_hi = __fadd_rn(shi, 0.0f);
+}
+
+// score_rows for a run-time number of head groups ng_count, weights from shared memory (wsel[8 ng +
+// e] for slot e of group ng): the same operations in the same order, so the result is score_rows<NG>
+// bit for bit.
+__device__ __forceinline__ void score_rows_rt(const uint4 (&A)[4], const uint4 (&Bq)[4], const uint2 (*frag)[8][32],
+                                              const float* wsel, int ng_count, int lane, float& s_lo, float& s_hi) {
+  const int c = lane & 3;
+  float slo = 0.f, shi = 0.f;
+  for (int ng = 0; ng < ng_count; ++ng) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint4 xa = A[kk >> 1], xb = Bq[kk >> 1];
+      const uint2 bf = frag[ng][kk][lane];
+      if (kk & 1)
+        mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, bf.x, bf.y);
+      else
+        mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, bf.x, bf.y);
+    }
+    const float wa = wsel[ng * 8 + 2 * c], wb = wsel[ng * 8 + 2 * c + 1];
+    slo = fmaf(wa, relu(acc[0]), slo);
+    slo = fmaf(wb, relu(acc[1]), slo);
+    shi = fmaf(wa, relu(acc[2]), shi);
+    shi = fmaf(wb, relu(acc[3]), shi);
   }
   slo += __shfl_xor_sync(0xffffffffu, slo, 1);
   shi += __shfl_xor_sync(0xffffffffu, shi, 1);

@@ -93,28 +93,58 @@ __device__ __forceinline__ void stage_query(HeadStage<NG>& st, const __nv_bfloat
   __syncthreads();
 }
 
-template <int NG, bool GATHER>
+// Work of the persistent scorer.
+enum : int {
+  kModeRows = 0,    // every prefix position of each query: out[t, p] for p < n_t
+  kModeGather = 1,  // gathered candidates: out[t, p] = score of token rows[t, p] for p < P
+  kModeSample = 2,  // only the list cut's sample of each row longer than the list cap (kSampleRuns
+                    // evenly spaced runs of kSampleRunLen tokens): out[t, s] at those tokens s
+  kModeList = 3,    // as kModeRows, and every token whose score is at or above its row's cut is
+                    // appended to the row's list with its dense score over all H_I heads
+};
+
+// Per-warp staging of kModeList: key rows at or above the cut wait here (a ring of 32 rows of
+// 256 bytes, plus their (order key, token)) until 16 of them fill one tensor-core group.
+constexpr int kRing = 32;
+
+template <int NG, int MODE>
 __global__ void __launch_bounds__(kScoreThreads, 2)
     score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                          const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, const int32_t* __restrict__ n,
                          const int32_t* __restrict__ heads, int h, int H_I, int L, int T,
-                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld) {
-  extern __shared__ int tile_base[];  // [T + 1] flattened tile prefix
+                         const int32_t* __restrict__ rows, int P, float* __restrict__ out, int64_t ld,
+                         DenseList dl) {
+  extern __shared__ __align__(16) uint8_t dsm[];
+  int* tile_base = reinterpret_cast<int*>(dsm);  // [T + 1] flattened tile prefix
   __shared__ HeadStage<NG> st;
   __shared__ uint32_t wtot[35];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  // kModeList: all heads' fragments and weights, and this warp's ring (after the tile prefix)
+  const int ngf = (H_I + 7) / 8;
+  uint8_t* lsm = dsm + (((size_t)T + 1) * sizeof(int) + 15) / 16 * 16;
+  uint2(*frag_all)[8][32] = reinterpret_cast<uint2(*)[8][32]>(lsm);
+  float* wall = reinterpret_cast<float*>(lsm + (size_t)ngf * 8 * 32 * sizeof(uint2));
+  uint8_t* ring = lsm + (size_t)ngf * 8 * 32 * sizeof(uint2) + kMaxHeads * sizeof(float) +
+                  (size_t)warp * kRing * (kD * 2 + sizeof(uint2));
+  uint2* meta = reinterpret_cast<uint2*>(ring + kRing * kD * 2);
   pdl_wait();
   pdl_trigger();
 
+  // positions of query t: n_t (rows, list), P (gather), the sample of a row longer than the cap
+  auto npos_of = [&](int nt) {
+    if (MODE == kModeGather) return P;
+    if (MODE == kModeSample) return nt > dl.cap ? kSampleRuns * kSampleRunLen : 0;
+    return nt;
+  };
   const int per = (T + kScoreThreads - 1) / kScoreThreads;
   const int q0 = min((int)threadIdx.x * per, T), q1 = min(q0 + per, T);
   uint32_t mine = 0;
-  for (int t = q0; t < q1; ++t) mine += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
+  for (int t = q0; t < q1; ++t) mine += (npos_of(clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
   uint32_t total;
   uint32_t run = block_exclusive_scan(mine, wtot, &total);
   for (int t = q0; t < q1; ++t) {
     tile_base[t] = (int)run;
-    run += ((GATHER ? P : clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
+    run += (npos_of(clamp_len(n[t], L)) + kTileRows - 1) / kTileRows;
   }
   if (threadIdx.x == 0) tile_base[T] = (int)total;
   __syncthreads();
@@ -134,10 +164,22 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const int first = (int)(pos - tile_base[t]);
     const int ntile = (int)(seg_end - pos);
     const int nt = clamp_len(n[t], L);
-    const int npos = GATHER ? P : nt;
-    const int32_t* rt = GATHER ? rows + (int64_t)t * P : nullptr;
+    const int npos = npos_of(nt);
+    const int32_t* rt = MODE == kModeGather ? rows + (int64_t)t * P : nullptr;
+    const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);  // kModeSample: run spacing
+    // kModeList: the row's cut (no list: nothing is appended)
+    bool listing = false;
+    uint32_t cutk = 0;
+    if (MODE == kModeList) {
+      listing = __ldcg(dl.cnt + t) != kNoList;
+      cutk = __ldcg(dl.cut + t);
+    }
 
     __syncthreads();  // the previous segment's fragments are no longer read
+    if (MODE == kModeList && listing) {
+      stage_all_head_frags<kScoreThreads>(frag_all, q + (int64_t)t * H_I * kD, H_I, ngf);
+      for (int e = threadIdx.x; e < ngf * 8; e += kScoreThreads) wall[e] = e < H_I ? w[(int64_t)t * H_I + e] : 0.f;
+    }
     stage_query<NG>(st, q, w, heads, h, H_I, t);
     float wa[NG], wb[NG];
 #pragma unroll
@@ -148,35 +190,65 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
     float* ot = out + (int64_t)t * ld;
     auto row_of = [&](int j) { return (first + j) * kTileRows + warp * 16; };
-    // position p -> key row: p itself, or rows[t, p] when gathering (outside [0, n_t): empty).
-    // Gathered row ids are fetched two tiles ahead, so a tile's row loads never wait for its ids.
+    // position p -> key row: p itself, the p-th sampled token, or rows[t, p] when gathering
+    // (outside [0, n_t): empty).  Gathered row ids are fetched two tiles ahead, so a tile's row
+    // loads never wait for its ids.
     auto raw_id = [&](int p) -> int {
       if (p >= npos) return -1;
-      if (!GATHER) return p;
+      if (MODE == kModeSample) return (p / kSampleRunLen) * seg + (p % kSampleRunLen);
+      if (MODE != kModeGather) return p;
       const int id = __ldg(rt + p);
       count_bad_id(kBadCandidate, c == 0 && id != -1 && (id < 0 || id >= nt));  // one lane of the quad
       return id;
     };
     auto valid_row = [&](int r) -> int { return (r >= 0 && r < nt) ? r : -1; };
     int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
-    int nia = GATHER && ntile > 1 ? raw_id(row_of(1) + g) : -1;
-    int nib = GATHER && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
-    auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4], bool& va, bool& vb) {
+    int nia = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g) : -1;
+    int nib = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
+    auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4]) {
       ra = valid_row(ra);
       rb = valid_row(rb);
-      va = ra >= 0;
-      vb = rb >= 0;
       load_rows(ra >= 0 ? kt + (int64_t)ra * kD : nullptr, rb >= 0 ? kt + (int64_t)rb * kD : nullptr, c, A, B);
     };
+    // kModeList: the staged rows [head, head + ns) of the ring; flush scores the first m <= 16 of
+    // them with all heads and appends them to the row's list (one atomic per flush)
+    int ns = 0, head = 0;
+    auto flush = [&](int m) {
+      __syncwarp();
+      const int sa = (head + g) & (kRing - 1), sb = (head + g + 8) & (kRing - 1);
+      uint4 A[4], B[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        A[i] = g < m ? *reinterpret_cast<const uint4*>(ring + sa * kD * 2 + (4 * i + c) * 16) : make_uint4(0, 0, 0, 0);
+        B[i] = g + 8 < m ? *reinterpret_cast<const uint4*>(ring + sb * kD * 2 + (4 * i + c) * 16)
+                         : make_uint4(0, 0, 0, 0);
+      }
+      float flo, fhi;
+      score_rows_rt(A, B, frag_all, wall, ngf, lane, flo, fhi);
+      uint32_t base = 0;
+      if (lane == 0) base = atomicAdd(dl.cnt + t, (uint32_t)m);
+      base = __shfl_sync(0xffffffffu, base, 0);
+      uint2* lt = dl.list + (int64_t)t * dl.stride;
+      float* ft = dl.f + (int64_t)t * dl.stride;
+      if (c == 0 && g < m && base + g < (uint32_t)dl.cap) {
+        lt[base + g] = meta[sa];
+        ft[base + g] = flo;
+      }
+      if (c == 1 && g + 8 < m && base + g + 8 < (uint32_t)dl.cap) {
+        lt[base + g + 8] = meta[sb];
+        ft[base + g + 8] = fhi;
+      }
+      __syncwarp();  // the slots are read before they are written again
+      head = (head + m) & (kRing - 1);
+      ns -= m;
+    };
     uint4 RA[4], RB[4];
-    bool va, vb;
-    load_ids(ida, idb, RA, RB, va, vb);
+    load_ids(ida, idb, RA, RB);
     for (int j = 0; j < ntile; ++j) {
       uint4 NA[4], NB[4];
-      bool na = false, nb = false;
+      int ra = -1, rb = -1;
       if (j + 1 < ntile) {
-        int ra, rb;
-        if (GATHER) {
+        if (MODE == kModeGather) {
           ra = nia;
           rb = nib;
           nia = j + 2 < ntile ? raw_id(row_of(j + 2) + g) : -1;
@@ -185,21 +257,53 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
           ra = raw_id(row_of(j + 1) + g);
           rb = raw_id(row_of(j + 1) + g + 8);
         }
-        load_ids(ra, rb, NA, NB, na, nb);
+        load_ids(ra, rb, NA, NB);
       }
       float slo, shi;
       score_rows<NG>(RA, RB, st.frag, wa, wb, lane, slo, shi);
       const int r = row_of(j) + g;
-      if (c == 0 && r < npos) ot[r] = slo;
-      if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
+      if (MODE == kModeSample) {
+        if (c == 0 && ida >= 0) ot[ida] = slo;
+        if (c == 1 && idb >= 0) ot[idb] = shi;
+      } else {
+        if (c == 0 && r < npos) ot[r] = slo;
+        if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
+      }
+      if (MODE == kModeList && listing) {
+        const bool pa = r < npos && order_key(slo) >= cutk;
+        const bool pb = r + 8 < npos && order_key(shi) >= cutk;
+        const uint32_t ba = __ballot_sync(0xffffffffu, pa && c == 0);  // bit 4 g': row g' passes
+        const uint32_t bb = __ballot_sync(0xffffffffu, pb && c == 0);
+        if (ba | bb) {
+          const uint32_t below = (1u << (4 * g)) - 1u;
+          const int na = __popc(ba);
+          if (pa) {
+            const int sl = (head + ns + __popc(ba & below)) & (kRing - 1);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(ring + sl * kD * 2 + (4 * i + c) * 16) = RA[i];
+            if (c == 0) meta[sl] = make_uint2(order_key(slo), (uint32_t)r);
+          }
+          if (pb) {
+            const int sl = (head + ns + na + __popc(bb & below)) & (kRing - 1);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(ring + sl * kD * 2 + (4 * i + c) * 16) = RB[i];
+            if (c == 0) meta[sl] = make_uint2(order_key(shi), (uint32_t)(r + 8));
+          }
+          ns += na + __popc(bb);
+          if (ns >= 16) flush(16);
+        }
+      }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         RA[i] = NA[i];
         RB[i] = NB[i];
       }
-      va = na;
-      vb = nb;
+      if (MODE == kModeSample) {
+        ida = ra;
+        idb = rb;
+      }
     }
+    if (MODE == kModeList && listing && ns > 0) flush(ns);
     pos = seg_end;
   }
 }
@@ -338,14 +442,17 @@ void launch_bf16(bool gather, bool persist, cudaStream_t s, const void* q, const
   auto kb = static_cast<const __nv_bfloat16*>(k);
   if (persist) {
     const size_t smem = sizeof(int) * ((size_t)T + 1);
+    const DenseList none{};
     if (gather) {
-      cudaFuncSetAttribute(score_persist_kernel<NG, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(score_persist_kernel<NG, true>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb, k_seq_stride, n,
-                 heads, h, H_I, L, T, rows, P, out, ld);
+      cudaFuncSetAttribute(score_persist_kernel<NG, kModeGather>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      launch_pdl(score_persist_kernel<NG, kModeGather>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb,
+                 k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, none);
     } else {
-      cudaFuncSetAttribute(score_persist_kernel<NG, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      launch_pdl(score_persist_kernel<NG, false>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb, k_seq_stride, n,
-                 heads, h, H_I, L, T, rows, P, out, ld);
+      cudaFuncSetAttribute(score_persist_kernel<NG, kModeRows>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+      launch_pdl(score_persist_kernel<NG, kModeRows>, 2 * num_sms(), kScoreThreads, smem, s, qb, w, kb,
+                 k_seq_stride, n, heads, h, H_I, L, T, rows, P, out, ld, none);
     }
   } else if (gather) {
     const dim3 grid((P + kGatherRowsPerChunk - 1) / kGatherRowsPerChunk, T);
@@ -417,6 +524,39 @@ void launch_scores(DType dt, const void* q, const float* w, const void* k, int64
     default:
       break;
   }
+}
+
+size_t dense_list_smem(int T, int H_I) {
+  const int ngf = (H_I + 7) / 8;
+  return ((size_t)T + 1) * sizeof(int) + 15 + (size_t)ngf * 8 * 32 * sizeof(uint2) + kMaxHeads * sizeof(float) +
+         (size_t)(kScoreThreads / 32) * kRing * (kD * 2 + sizeof(uint2));
+}
+
+bool launch_scores_sample(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                          const int32_t* heads, int T, int L, int H_I, int h, int cap, float* out, int64_t ld,
+                          cudaStream_t s) {
+  if (h < 1 || h > 8 || T < 1 || T > kMaxPersistQueries || k_seq_stride == 0) return false;
+  DenseList dl{};
+  dl.cap = cap;
+  const size_t smem = sizeof(int) * ((size_t)T + 1);
+  cudaFuncSetAttribute(score_persist_kernel<1, kModeSample>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(score_persist_kernel<1, kModeSample>, 2 * num_sms(), kScoreThreads, smem, s,
+             static_cast<const __nv_bfloat16*>(q), w, static_cast<const __nv_bfloat16*>(k), k_seq_stride, n, heads, h,
+             H_I, L, T, static_cast<const int32_t*>(nullptr), 0, out, ld, dl);
+  return true;
+}
+
+bool launch_scores_dense_list(const void* q, const float* w, const void* k, int64_t k_seq_stride, const int32_t* n,
+                              const int32_t* heads, int T, int L, int H_I, int h, float* out, int64_t ld,
+                              const DenseList& dl, cudaStream_t s) {
+  if (h < 1 || h > 8 || T < 1 || T > kMaxPersistQueries || k_seq_stride == 0 || H_I > kMaxHeads) return false;
+  const size_t smem = dense_list_smem(T, H_I);
+  if (smem > kDenseListMaxSmem) return false;
+  cudaFuncSetAttribute(score_persist_kernel<1, kModeList>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(score_persist_kernel<1, kModeList>, 2 * num_sms(), kScoreThreads, smem, s,
+             static_cast<const __nv_bfloat16*>(q), w, static_cast<const __nv_bfloat16*>(k), k_seq_stride, n, heads, h,
+             H_I, L, T, static_cast<const int32_t*>(nullptr), 0, out, ld, dl);
+  return true;
 }
 
 MISA_BAD_ID_READER(read_and_clear_bad_ids_score)

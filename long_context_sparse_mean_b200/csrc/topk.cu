@@ -22,6 +22,7 @@
 // select_small_kernel ranks a short candidate list entirely in one CTA's shared memory; it needs
 // no workspace (used by the entry point without allocation).
 #include "kernels.cuh"
+#include "mma_frag.cuh"
 #include "select.cuh"
 #include "warp_select.cuh"
 
@@ -252,21 +253,21 @@ __device__ __forceinline__ uint32_t block_rth_largest(Each each, uint32_t lo, ui
   }
 }
 
-// Top `need` of the c list entries (c >= need, keys within [lo, hi]) in shared memory, written to
-// oi/ov [0, need) in no particular order.  Rounds of 4096 bins narrow a key interval [ilo, ihi]
+// Top `need` of the c list entries (c >= need, keys within [lo, hi]) in shared memory, handed to
+// emit(slot, i) (list entry i goes to output slot < need; every slot once, in no particular order).  Rounds of 4096 bins narrow a key interval [ilo, ihi]
 // that holds the need-th entry: the first round bins the keys themselves when they share one sign
 // (order keys are close to logarithmic in the score, so outliers do not crowd the bulk into a few
 // bins) and bins linearly in the score otherwise; later rounds bin the interval's keys.  Once the
 // interval holds at most 256 entries (or one key), one pass writes every entry above it and moves
-// the interval's entries into the histogram's words (hist: 16-byte aligned), where a rank count
-// (score, then token) places them.  An exact tie of more than 2048 entries at one key takes the
+// the interval's entries (key, list index) into the histogram's words (hist: 16-byte aligned),
+// where a rank count (score, then token) places them.  An exact tie of more than 2048 entries at one key takes the
 // lowest tokens by a search over the tokens.  The list is only read.  ctr: 2 words; mm: 2 words;
 // scratch: 35 words.
-template <int NT>
-__device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
-                                  uint32_t* ctr, uint32_t* mm, uint32_t* scratch, int32_t* oi, float* ov) {
+template <int NT, class Emit>
+__device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi,
+                                       uint32_t* hist, uint32_t* ctr, uint32_t* mm, uint32_t* scratch, Emit emit) {
   constexpr uint32_t kRank = 256;            // interval entries a rank count orders
-  constexpr uint32_t kBuf = kHistBins / 2;   // (key, token) pairs the histogram's words hold
+  constexpr uint32_t kBuf = kHistBins / 2;   // (key, list index) pairs the histogram's words hold
   const int tid = threadIdx.x;
   uint32_t ilo = lo, ihi = hi, r = need, eq = (uint32_t)c;
   const bool one_sign = lo >= 0x80000000u || hi < 0x80000000u;
@@ -326,25 +327,20 @@ __device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint3
       const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
       const bool gt = i < c && e.x > ihi, in = i < c && e.x >= ilo && e.x <= ihi;
       const uint32_t slot = warp_slot(gt, &ctr[0]);
-      if (gt) {
-        oi[slot] = (int32_t)e.y;
-        if (ov) ov[slot] = key_to_float(e.x);
-      }
+      if (gt) emit(slot, (uint32_t)i);
       const uint32_t s2 = warp_slot(in, &ctr[1]);
-      if (in) bl[s2] = e;
+      if (in) bl[s2] = make_uint2(e.x, (uint32_t)i);
     }
     __syncthreads();
     for (uint32_t j = tid; j < eq; j += NT) {
       const uint2 m = bl[j];
+      const uint32_t mt = list[m.y].y;
       uint32_t rk = 0;
       for (uint32_t i = 0; i < eq; ++i) {
         const uint2 o = bl[i];
-        rk += (o.x > m.x) || (o.x == m.x && o.y < m.y);
+        rk += (o.x > m.x) || (o.x == m.x && list[o.y].y < mt);
       }
-      if (rk < r) {
-        oi[n_gt + rk] = (int32_t)m.y;
-        if (ov) ov[n_gt + rk] = key_to_float(m.x);
-      }
+      if (rk < r) emit(n_gt + rk, m.y);
     }
     return;
   }
@@ -383,10 +379,84 @@ __device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint3
     const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
     const bool sel = i < c && (e.x > ihi || (e.x == ilo && e.y <= tok));
     const uint32_t slot = warp_slot(sel, &ctr[0]);
-    if (sel) {
-      oi[slot] = (int32_t)e.y;
-      if (ov) ov[slot] = key_to_float(e.x);
+    if (sel) emit(slot, (uint32_t)i);
+  }
+}
+
+// select_list_exact_emit writing token and value: oi[slot] (and ov[slot]).
+template <int NT>
+__device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
+                                  uint32_t* ctr, uint32_t* mm, uint32_t* scratch, int32_t* oi, float* ov) {
+  select_list_exact_emit<NT>(list, c, need, lo, hi, hist, ctr, mm, scratch, [&](uint32_t slot, uint32_t i) {
+    const uint2 e = list[i];
+    oi[slot] = (int32_t)e.y;
+    if (ov) ov[slot] = key_to_float(e.x);
+  });
+}
+
+// Exact top-k of the score row [0, nt) by one CTA (tie: lower token): a full level-0 histogram of
+// the keys, the keys above the boundary bucket written out, the bucket's keys ranked from the list
+// (or from global memory when they overflow it).  Slots past the selection get -1 (and 0).
+// list: LIST entries; hp: kHistPadded words; cnt: 2 words; scratch: 35 words.
+template <int NT, int LIST>
+__device__ void row_exact_topk(const float* row, int nt, bool vec, int topk, uint2* list, uint32_t* hp, uint32_t* cnt,
+                               uint32_t* scratch, int32_t* oi, float* ov) {
+  const int tid = threadIdx.x;
+  uint32_t kk = 0;  // slots filled
+  for (int b = tid; b < kHistPadded; b += NT) hp[b] = 0;
+  if (tid < 2) cnt[tid] = 0;
+  __syncthreads();
+  row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
+    (void)s;
+    hist_add(hp, (uint32_t)hpad((int)(k >> 20)), in && k != 0u);
+  });
+  __syncthreads();
+  uint32_t local = 0;
+  for (int b = tid; b < kHistBins; b += NT) local += hp[hpad(b)];
+  uint32_t total;
+  block_exclusive_scan(local, scratch, &total);
+  const uint32_t want = min((uint32_t)topk, total);
+  if (want > 0) {
+    const Bucket bk = bucket_search_padded(hp, want, scratch);
+    const uint32_t pb = bk.prefix >> 20;
+    // keys above the bucket straight to the output, the bucket's keys to the list
+    row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
+      const bool ok = in && k != 0u;
+      const bool gt = ok && (k >> 20) > pb;
+      const uint32_t slot = warp_slot(gt, &cnt[1]);
+      if (gt && slot < (uint32_t)topk) {
+        oi[slot] = s;
+        if (ov) ov[slot] = key_to_float(k);
+      }
+      const bool eq = ok && (k >> 20) == pb;
+      const uint32_t e = warp_slot(eq, &cnt[0]);
+      if (eq && e < (uint32_t)LIST) list[e] = make_uint2(k, (uint32_t)s);
+    });
+    __syncthreads();
+    const uint32_t n_gt = min(cnt[1], (uint32_t)topk);
+    const uint32_t c = cnt[0];
+    const uint32_t need = min(bk.need, want - n_gt);
+    if (c <= (uint32_t)LIST) {
+      const SmemPairs acc{list};
+      if (c <= need) {
+        for (uint32_t i = tid; i < c; i += NT) {
+          oi[n_gt + i] = (int32_t)list[i].y;
+          if (ov) ov[n_gt + i] = key_to_float(list[i].x);
+        }
+      } else {
+        const SelectResult r = radix_select_items(acc, (int)c, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
+        write_selection(acc, (int)c, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
+      }
+    } else {
+      const RowBucket acc{row, bk.prefix};
+      const SelectResult r = radix_select_items(acc, nt, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
+      write_selection(acc, nt, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
     }
+    kk = n_gt + need;
+  }
+  for (int a = (int)kk + tid; a < topk; a += NT) {
+    oi[a] = -1;
+    if (ov) ov[a] = 0.f;
   }
 }
 
@@ -562,63 +632,8 @@ __global__ void __launch_bounds__(NT, MINB) row_topk_kernel(const float* __restr
     __syncthreads();
   }
 
-  // ---- exact path (score rows only): full level-0 histogram, boundary bucket, rank the bucket ----
-  uint32_t kk = 0;  // slots filled
-  for (int b = tid; b < kHistPadded; b += NT) hp[b] = 0;
-  if (tid < 2) cnt[tid] = 0;
-  __syncthreads();
-  row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
-    (void)s;
-    hist_add(hp, (uint32_t)hpad((int)(k >> 20)), in && k != 0u);
-  });
-  __syncthreads();
-  uint32_t local = 0;
-  for (int b = tid; b < kHistBins; b += NT) local += hp[hpad(b)];
-  uint32_t total;
-  block_exclusive_scan(local, scratch, &total);
-  const uint32_t want = min((uint32_t)topk, total);
-  if (want > 0) {
-    const Bucket bk = bucket_search_padded(hp, want, scratch);
-    const uint32_t pb = bk.prefix >> 20;
-    // keys above the bucket straight to the output, the bucket's keys to the list
-    row_sweep<NT>(row, nt, vec, [&](int s, uint32_t k, bool in) {
-      const bool ok = in && k != 0u;
-      const bool gt = ok && (k >> 20) > pb;
-      const uint32_t slot = warp_slot(gt, &cnt[1]);
-      if (gt && slot < (uint32_t)topk) {
-        oi[slot] = s;
-        if (ov) ov[slot] = key_to_float(k);
-      }
-      const bool eq = ok && (k >> 20) == pb;
-      const uint32_t e = warp_slot(eq, &cnt[0]);
-      if (eq && e < (uint32_t)LIST) list[e] = make_uint2(k, (uint32_t)s);
-    });
-    __syncthreads();
-    const uint32_t n_gt = min(cnt[1], (uint32_t)topk);
-    const uint32_t c = cnt[0];
-    const uint32_t need = min(bk.need, want - n_gt);
-    if (c <= (uint32_t)LIST) {
-      const SmemPairs acc{list};
-      if (c <= need) {
-        for (uint32_t i = tid; i < c; i += NT) {
-          oi[n_gt + i] = (int32_t)list[i].y;
-          if (ov) ov[n_gt + i] = key_to_float(list[i].x);
-        }
-      } else {
-        const SelectResult r = radix_select_items(acc, (int)c, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
-        write_selection(acc, (int)c, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
-      }
-    } else {
-      const RowBucket acc{row, bk.prefix};
-      const SelectResult r = radix_select_items(acc, nt, need, 1, bk.prefix, 0xfff00000u, hp, scratch);
-      write_selection(acc, nt, r, false, oi + n_gt, ov ? ov + n_gt : nullptr, need, scratch);
-    }
-    kk = n_gt + need;
-  }
-  for (int a = (int)kk + tid; a < topk; a += NT) {
-    oi[a] = -1;
-    if (ov) ov[a] = 0.f;
-  }
+  // ---- exact path (score rows only) ----
+  row_exact_topk<NT, LIST>(row, nt, vec, topk, list, hp, cnt, scratch, oi, ov);
 }
 
 template <int NT, int LIST, int MINB>
@@ -890,6 +905,137 @@ void launch_list_select_warp(const int32_t* n, int T, int L, int topk, const Lis
 
 void mark_no_lists(const ListState& l, int T, cudaStream_t s) {
   if (T > 0) cudaMemsetAsync(l.cnt, 0xff, sizeof(uint32_t) * (size_t)T, s);
+}
+
+// ---- MISA-dagger selection over dense lists -----------------------------------------------------
+
+// One CTA per row: the top-k' of the row's dense list by the routed score (ties to the lower token)
+// with their dense scores, then the top-k of those by the dense score.  A row its list cannot
+// answer (no list, fewer than k' entries, entries lost past the cap) takes the exact top-k' of its
+// routed score row and scores those candidates with all H_I heads here (as the scorer does, one
+// warp per 16 candidates on the tensor cores).  ctok / cf: [T][kp] scratch for the k' candidates.
+template <int NT, int LIST>
+__global__ void __launch_bounds__(NT, 1)
+    hier_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n, int L, int kp,
+                       int topk, DenseList dl, const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
+                       const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, int H_I, int32_t* __restrict__ ctok,
+                       float* __restrict__ cf, int32_t* __restrict__ idx, float* __restrict__ score_opt) {
+  extern __shared__ uint2 list[];  // [LIST]
+  __shared__ __align__(16) uint32_t hp[kHistPadded];
+  __shared__ uint32_t scratch[35];
+  __shared__ uint32_t cnt[2];
+  __shared__ uint32_t mm[2];
+  const int t = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  const int nt = clamp_len(n[t], L);
+  const float* row = scores + (int64_t)t * ld;
+  int32_t* ct = ctok + (int64_t)t * kp;
+  float* cft = cf + (int64_t)t * kp;
+  int32_t* oi = idx + (int64_t)t * topk;
+  float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
+  const int c1 = min(kp, nt);  // candidates
+  const uint32_t c_in = __ldcg(dl.cnt + t);
+  const bool listed = c_in != kNoList && c_in >= (uint32_t)kp && c_in <= (uint32_t)min(dl.cap, LIST);
+  if (tid == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+
+  // ---- 1. the k' candidates and their dense scores, into ct / cft ----
+  if (listed) {
+    const uint2* src = dl.list + (int64_t)t * dl.stride;
+    uint32_t lo = 0xffffffffu, hi = 0u;
+    for (uint32_t i = tid; i < c_in; i += NT) {
+      const uint2 e = __ldcg(src + i);
+      list[i] = e;
+      lo = min(lo, e.x);
+      hi = max(hi, e.x);
+    }
+    block_min_max(lo, hi, mm);
+    __syncthreads();
+    lo = mm[0];
+    hi = mm[1];
+    __syncthreads();  // mm is reused as scratch
+    const float* fsrc = dl.f + (int64_t)t * dl.stride;
+    select_list_exact_emit<NT>(list, (int)c_in, (uint32_t)kp, lo, hi, hp, cnt, mm, scratch,
+                               [&](uint32_t slot, uint32_t i) {
+                                 ct[slot] = (int32_t)list[i].y;
+                                 cft[slot] = __ldcg(fsrc + i);
+                               });
+  } else {
+    if (nt <= kp) {
+      for (int p = tid; p < nt; p += NT) ct[p] = p;
+    } else {
+      const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
+      row_exact_topk<NT, LIST>(row, nt, vec, kp, list, hp, cnt, scratch, ct, nullptr);
+    }
+    __syncthreads();  // the candidates are written; the list's memory is free
+    const int ngf = (H_I + 7) / 8;
+    uint2(*frag)[8][32] = reinterpret_cast<uint2(*)[8][32]>(list);
+    float* wall = reinterpret_cast<float*>(list + ngf * 8 * 32);
+    stage_all_head_frags<NT>(frag, q + (int64_t)t * H_I * kD, H_I, ngf);
+    for (int e = tid; e < ngf * 8; e += NT) wall[e] = e < H_I ? w[(int64_t)t * H_I + e] : 0.f;
+    __syncthreads();
+    const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
+    const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
+    for (int s0 = warp * 16; s0 < c1; s0 += (NT / 32) * 16) {
+      const int ra = s0 + g < c1 ? __ldcg(ct + s0 + g) : -1;
+      const int rb = s0 + g + 8 < c1 ? __ldcg(ct + s0 + g + 8) : -1;
+      uint4 A[4], B[4];
+      load_rows(ra >= 0 && ra < nt ? kt + (int64_t)ra * kD : nullptr, rb >= 0 && rb < nt ? kt + (int64_t)rb * kD : nullptr,
+                c, A, B);
+      float flo, fhi;
+      score_rows_rt(A, B, frag, wall, ngf, lane, flo, fhi);
+      if (c == 0 && s0 + g < c1) cft[s0 + g] = flo;
+      if (c == 1 && s0 + g + 8 < c1) cft[s0 + g + 8] = fhi;
+    }
+  }
+  __syncthreads();  // ct / cft written by this block
+
+  // ---- 2. the top-k of the candidates by the dense score ----
+  if (tid == 0) {
+    mm[0] = 0xffffffffu;
+    mm[1] = 0u;
+  }
+  uint32_t lo = 0xffffffffu, hi = 0u;
+  for (int i = tid; i < c1; i += NT) {
+    const uint32_t key = order_key(__ldcg(cft + i));
+    list[i] = make_uint2(key, (uint32_t)__ldcg(ct + i));
+    lo = min(lo, key);
+    hi = max(hi, key);
+  }
+  block_min_max(lo, hi, mm);
+  __syncthreads();
+  if (c1 <= topk) {  // every candidate is selected
+    for (int i = tid; i < topk; i += NT) {
+      oi[i] = i < c1 ? (int32_t)list[i].y : -1;
+      if (ov) ov[i] = i < c1 ? key_to_float(list[i].x) : 0.f;
+    }
+    return;
+  }
+  lo = mm[0];
+  hi = mm[1];
+  __syncthreads();  // mm is reused as scratch
+  select_list_exact<NT>(list, c1, (uint32_t)topk, lo, hi, hp, cnt, mm, scratch, oi, ov);
+}
+
+void launch_list_cut(const float* scores, int64_t ld, const int32_t* n, int T, int L, int topk, int cap,
+                     uint32_t* lcnt, uint32_t* lcut, cudaStream_t s) {
+  if (T <= 0) return;
+  launch_pdl(list_cut_kernel, T, kCutThreads, 0, s, scores, ld, n, L, topk, cap, lcnt, lcut);
+}
+
+void launch_hier_select(const float* scores, int64_t ld, const int32_t* n, int T, int L, int kp, int topk,
+                        const DenseList& dl, const void* q, const float* w, const void* k, int64_t k_seq_stride,
+                        int H_I, int32_t* ctok, float* cf, int32_t* idx, float* score_opt, cudaStream_t s) {
+  if (T <= 0) return;
+  constexpr int NT = 1024, LIST = kRowListLarge;
+  const size_t smem = sizeof(uint2) * (size_t)LIST;
+  cudaFuncSetAttribute(hier_select_kernel<NT, LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  launch_pdl(hier_select_kernel<NT, LIST>, T, NT, smem, s, scores, ld, n, L, kp, topk, dl,
+             static_cast<const __nv_bfloat16*>(q), w, static_cast<const __nv_bfloat16*>(k), k_seq_stride, H_I, ctok,
+             cf, idx, score_opt);
 }
 
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,

@@ -318,3 +318,32 @@ def test_fused_prefill_workspace_and_argument_checks(lib):
     st = f(FAKE, FAKE, FAKE, FAKE, FAKE, 4, 1000, 64, 128, 8, 10, BF16, FAKE, None, MISALIGNED, 1 << 30, None)
     assert st == WORKSPACE
     assert f(FAKE, FAKE, FAKE, FAKE, FAKE, 0, 1000, 64, 128, 8, 10, BF16, FAKE, None, None, 0, None) == OK
+
+
+def test_hier_fused_workspace_and_argument_checks(lib):
+    """misa_hier_topk_fused: workspace = score rows [T, ceil4(L)] + list counts and cuts [2, T] +
+    dense lists [T, 16384] of (key, token) pairs and their dense scores + the k' candidates and their
+    dense scores [2, T, k']; shared caches, fp32 inputs and k' above 16384 are unsupported."""
+    ws = lib.misa_workspace_bytes
+    T, L, kp, k = 32, 131072, 8192, 2048
+    cap = 16384
+    want = _al(T * L * 4) + 2 * _al(T * 4) + _al(T * cap * 8) + _al(T * cap * 4) + 2 * _al(T * kp * 4)
+    assert ws(10, T, L, 64, 0, 8, k, kp) == want
+    assert ws(10, 3, 1001, 64, 0, 8, 10, 20) == (_al(3 * 1004 * 4) + 2 * _al(12) + _al(3 * cap * 8) +
+                                                 _al(3 * cap * 4) + 2 * _al(3 * 20 * 4))
+    assert ws(10, 0, L, 64, 0, 8, k, kp) == 0
+    f = lib.misa_hier_topk_fused
+    S = 1000 * 128
+    args = lambda **o: dict(dict(q=FAKE, w=FAKE, k=FAKE, kss=S, n=FAKE, heads=FAKE, T=4, L=1000, H=64, d=128, h=8,
+                                 kp=40, topk=10, dt=BF16, idx=FAKE, v=None, ws=FAKE, wsb=1 << 30, s=None), **o)
+    call = lambda a: f(*a.values())
+    assert call(args(dt=F32)) == UNSUPPORTED
+    assert call(args(kss=0)) == UNSUPPORTED  # one shared cache
+    assert call(args(kp=16385)) == UNSUPPORTED
+    assert call(args(kp=9)) == INVALID  # k' < k
+    assert call(args(heads=None)) == INVALID
+    assert call(args(h=65)) == INVALID
+    assert call(args(kss=999 * 128)) == INVALID  # stride below L * d
+    assert call(args(wsb=64)) == WORKSPACE
+    assert call(args(ws=MISALIGNED)) == WORKSPACE
+    assert call(args(T=0, ws=None, wsb=0)) == OK
