@@ -172,12 +172,12 @@ misa_status misa_device_check(void) {
 }
 
 // misa_hier_topk_fused: [score rows][list counts][cuts][dense lists (entries, dense scores)]
-// [candidates][their dense scores]
+// [candidates of the rows the lists cannot answer]
 size_t hier_fused_ws(int T, int L, int kp) {
   if (T <= 0 || L <= 0 || kp <= 0) return 0;
   const size_t cap = misa::kListCap;
   return scores_part(T, L) + 2 * align_up(sizeof(uint32_t) * (size_t)T) + align_up(sizeof(uint2) * (size_t)T * cap) +
-         align_up(sizeof(float) * (size_t)T * cap) + 2 * align_up(sizeof(int32_t) * (size_t)T * kp);
+         align_up(sizeof(float) * (size_t)T * cap) + align_up(sizeof(int32_t) * (size_t)T * kp);
 }
 
 size_t misa_workspace_bytes(int op, int T, int L, int H_I, int B, int h, int topk, int kp) {
@@ -552,8 +552,6 @@ misa_status misa_hier_topk_fused(const void* q, const float* w, const void* k, i
   dl.f = reinterpret_cast<float*>(p);
   p += align_up(sizeof(float) * (size_t)T * dl.cap);
   int32_t* ctok = reinterpret_cast<int32_t*>(p);
-  p += align_up(sizeof(int32_t) * (size_t)T * kp);
-  float* cf = reinterpret_cast<float*>(p);
   // lists for a few long rows (many rows fill the GPU with one CTA per row already); the scorer's
   // shared memory must fit two CTAs per SM
   const bool lists = T <= misa::kDenseListMaxRows && L > dl.cap && h <= 8 &&
@@ -566,7 +564,7 @@ misa_status misa_hier_topk_fused(const void* q, const float* w, const void* k, i
     cudaMemsetAsync(dl.cnt, 0xff, sizeof(uint32_t) * (size_t)T, s);  // kNoList: every row from its score row
     misa::launch_scores(misa::DType::BF16, q, w, k, k_seq_stride, n, heads, T, L, H_I, h, nullptr, 0, rows, ld, s);
   }
-  misa::launch_hier_select(rows, ld, n, T, L, kp, topk, dl, q, w, k, k_seq_stride, H_I, ctok, cf, idx, score_opt, s);
+  misa::launch_hier_select(rows, ld, n, T, L, kp, topk, dl, q, w, k, k_seq_stride, H_I, ctok, idx, score_opt, s);
   return launch_status();
 }
 

@@ -104,10 +104,10 @@ void launch_list_cut(const float* scores, int64_t ld, const int32_t* n, int T, i
                      uint32_t* lcnt, uint32_t* lcut, cudaStream_t s);
 // One CTA per row (kp <= 16384): idx [T, topk] (score_opt: the dense scores) from the dense lists, or
 // for a row they cannot answer, from its score row (exact top-k', dense scores of the candidates
-// computed here).  ctok / cf: [T][kp] scratch.
+// computed here).  ctok: [T][kp] scratch.
 void launch_hier_select(const float* scores, int64_t ld, const int32_t* n, int T, int L, int kp, int topk,
                         const DenseList& dl, const void* q, const float* w, const void* k, int64_t k_seq_stride,
-                        int H_I, int32_t* ctok, float* cf, int32_t* idx, float* score_opt, cudaStream_t s);
+                        int H_I, int32_t* ctok, int32_t* idx, float* score_opt, cudaStream_t s);
 
 // Token scores with a head list (heads == nullptr: all H_I heads).  rows != nullptr gathers:
 // position p of query t scores token rows[t*P + p] and writes out[t*ld + p].

@@ -107,6 +107,39 @@ enum : int {
 // 256 bytes, plus their (order key, token)) until 16 of them fill one tensor-core group.
 constexpr int kRing = 32;
 
+// kModeList: the first m <= 16 rows staged in a warp's ring (slots head .. head + m - 1, mod kRing)
+// scored with all heads (frag / wall: ngf head groups) and appended to row t's list with one atomic
+// (entries past the cap are counted, not written).  Called by the whole warp; rare (once per 16
+// rows at or above the cut), so it is kept out of line, away from the scoring loop's registers.
+__device__ __noinline__ void flush_ring(const uint8_t* ring, const uint2* meta, int head, int m,
+                                        const uint2 (*frag)[8][32], const float* wall, int ngf, DenseList dl, int t) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+  __syncwarp();
+  const int sa = (head + g) & (kRing - 1), sb = (head + g + 8) & (kRing - 1);
+  uint4 A[4], B[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    A[i] = g < m ? *reinterpret_cast<const uint4*>(ring + sa * kD * 2 + (4 * i + c) * 16) : make_uint4(0, 0, 0, 0);
+    B[i] = g + 8 < m ? *reinterpret_cast<const uint4*>(ring + sb * kD * 2 + (4 * i + c) * 16) : make_uint4(0, 0, 0, 0);
+  }
+  float flo, fhi;
+  score_rows_rt(A, B, frag, wall, ngf, lane, flo, fhi);
+  uint32_t base = 0;
+  if (lane == 0) base = atomicAdd(dl.cnt + t, (uint32_t)m);
+  base = __shfl_sync(0xffffffffu, base, 0);
+  uint2* lt = dl.list + (int64_t)t * dl.stride;
+  float* ft = dl.f + (int64_t)t * dl.stride;
+  if (c == 0 && g < m && base + g < (uint32_t)dl.cap) {
+    lt[base + g] = meta[sa];
+    ft[base + g] = flo;
+  }
+  if (c == 1 && g + 8 < m && base + g + 8 < (uint32_t)dl.cap) {
+    lt[base + g + 8] = meta[sb];
+    ft[base + g + 8] = fhi;
+  }
+  __syncwarp();  // the slots are read before they are written again
+}
+
 template <int NG, int MODE>
 __global__ void __launch_bounds__(kScoreThreads, 2)
     score_persist_kernel(const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
@@ -169,26 +202,13 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
     const int seg = (nt / kSampleRuns) & ~(kSampleRunLen - 1);  // kModeSample: run spacing
     // kModeList: the row's cut (no list: nothing is appended)
     bool listing = false;
-    uint32_t cutk = 0;
+    float cutv = 0.f;  // compared as a float: the same order as the keys (the cut is a finite score)
     if (MODE == kModeList) {
       listing = __ldcg(dl.cnt + t) != kNoList;
-      cutk = __ldcg(dl.cut + t);
+      cutv = key_to_float(__ldcg(dl.cut + t));
     }
 
-    __syncthreads();  // the previous segment's fragments are no longer read
-    if (MODE == kModeList && listing) {
-      stage_all_head_frags<kScoreThreads>(frag_all, q + (int64_t)t * H_I * kD, H_I, ngf);
-      for (int e = threadIdx.x; e < ngf * 8; e += kScoreThreads) wall[e] = e < H_I ? w[(int64_t)t * H_I + e] : 0.f;
-    }
-    stage_query<NG>(st, q, w, heads, h, H_I, t);
-    float wa[NG], wb[NG];
-#pragma unroll
-    for (int ng = 0; ng < NG; ++ng) {
-      wa[ng] = st.wsel[ng * 8 + 2 * c];
-      wb[ng] = st.wsel[ng * 8 + 2 * c + 1];
-    }
     const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
-    float* ot = out + (int64_t)t * ld;
     auto row_of = [&](int j) { return (first + j) * kTileRows + warp * 16; };
     // position p -> key row: p itself, the p-th sampled token, or rows[t, p] when gathering
     // (outside [0, n_t): empty).  Gathered row ids are fetched two tiles ahead, so a tile's row
@@ -202,49 +222,42 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
       return id;
     };
     auto valid_row = [&](int r) -> int { return (r >= 0 && r < nt) ? r : -1; };
-    int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
-    int nia = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g) : -1;
-    int nib = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
     auto load_ids = [&](int ra, int rb, uint4 (&A)[4], uint4 (&B)[4]) {
       ra = valid_row(ra);
       rb = valid_row(rb);
       load_rows(ra >= 0 ? kt + (int64_t)ra * kD : nullptr, rb >= 0 ? kt + (int64_t)rb * kD : nullptr, c, A, B);
     };
+    // the first tile's rows are read while the query's heads are staged
+    int ida = raw_id(row_of(0) + g), idb = raw_id(row_of(0) + g + 8);
+    int nia = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g) : -1;
+    int nib = MODE == kModeGather && ntile > 1 ? raw_id(row_of(1) + g + 8) : -1;
+    uint4 RA[4], RB[4];
+    load_ids(ida, idb, RA, RB);
+
+    __syncthreads();  // the previous segment's fragments are no longer read
+    if (MODE == kModeList && listing) {
+      stage_all_head_frags<kScoreThreads>(frag_all, q + (int64_t)t * H_I * kD, H_I, ngf);
+      for (int e = threadIdx.x; e < ngf * 8; e += kScoreThreads) wall[e] = e < H_I ? w[(int64_t)t * H_I + e] : 0.f;
+    }
+    stage_query<NG>(st, q, w, heads, h, H_I, t);
+    float wa[NG], wb[NG];
+#pragma unroll
+    for (int ng = 0; ng < NG; ++ng) {
+      wa[ng] = st.wsel[ng * 8 + 2 * c];
+      wb[ng] = st.wsel[ng * 8 + 2 * c + 1];
+    }
+    float* ot = out + (int64_t)t * ld;
     // kModeList: the staged rows [head, head + ns) of the ring; flush scores the first m <= 16 of
     // them with all heads and appends them to the row's list (one atomic per flush)
     int ns = 0, head = 0;
     auto flush = [&](int m) {
-      __syncwarp();
-      const int sa = (head + g) & (kRing - 1), sb = (head + g + 8) & (kRing - 1);
-      uint4 A[4], B[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        A[i] = g < m ? *reinterpret_cast<const uint4*>(ring + sa * kD * 2 + (4 * i + c) * 16) : make_uint4(0, 0, 0, 0);
-        B[i] = g + 8 < m ? *reinterpret_cast<const uint4*>(ring + sb * kD * 2 + (4 * i + c) * 16)
-                         : make_uint4(0, 0, 0, 0);
-      }
-      float flo, fhi;
-      score_rows_rt(A, B, frag_all, wall, ngf, lane, flo, fhi);
-      uint32_t base = 0;
-      if (lane == 0) base = atomicAdd(dl.cnt + t, (uint32_t)m);
-      base = __shfl_sync(0xffffffffu, base, 0);
-      uint2* lt = dl.list + (int64_t)t * dl.stride;
-      float* ft = dl.f + (int64_t)t * dl.stride;
-      if (c == 0 && g < m && base + g < (uint32_t)dl.cap) {
-        lt[base + g] = meta[sa];
-        ft[base + g] = flo;
-      }
-      if (c == 1 && g + 8 < m && base + g + 8 < (uint32_t)dl.cap) {
-        lt[base + g + 8] = meta[sb];
-        ft[base + g + 8] = fhi;
-      }
-      __syncwarp();  // the slots are read before they are written again
+      flush_ring(ring, meta, head, m, frag_all, wall, ngf, dl, t);
       head = (head + m) & (kRing - 1);
       ns -= m;
     };
-    uint4 RA[4], RB[4];
-    load_ids(ida, idb, RA, RB);
     for (int j = 0; j < ntile; ++j) {
+      // the rows staged by the previous tile, before the next tile's loads are in flight
+      if (MODE == kModeList && listing && ns >= 16) flush(16);
       uint4 NA[4], NB[4];
       int ra = -1, rb = -1;
       if (j + 1 < ntile) {
@@ -270,11 +283,12 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
         if (c == 1 && r + 8 < npos) ot[r + 8] = shi;
       }
       if (MODE == kModeList && listing) {
-        const bool pa = r < npos && order_key(slo) >= cutk;
-        const bool pb = r + 8 < npos && order_key(shi) >= cutk;
-        const uint32_t ba = __ballot_sync(0xffffffffu, pa && c == 0);  // bit 4 g': row g' passes
-        const uint32_t bb = __ballot_sync(0xffffffffu, pb && c == 0);
-        if (ba | bb) {
+        const bool pa = r < npos && slo >= cutv;
+        const bool pb = r + 8 < npos && shi >= cutv;
+        // bit 4 g' (lane (g', 0)): row g' passes; bit 4 g' + 1 (lane (g', 1)): row g' + 8
+        const uint32_t bab = __ballot_sync(0xffffffffu, c == 0 ? pa : (c == 1 && pb));
+        if (bab) {
+          const uint32_t ba = bab & 0x11111111u, bb = (bab >> 1) & 0x11111111u;
           const uint32_t below = (1u << (4 * g)) - 1u;
           const int na = __popc(ba);
           if (pa) {
@@ -289,8 +303,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
             for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4*>(ring + sl * kD * 2 + (4 * i + c) * 16) = RB[i];
             if (c == 0) meta[sl] = make_uint2(order_key(shi), (uint32_t)(r + 8));
           }
-          ns += na + __popc(bb);
-          if (ns >= 16) flush(16);
+          ns += na + __popc(bb);  // at most 31: the ring holds them
         }
       }
 #pragma unroll
@@ -303,7 +316,10 @@ __global__ void __launch_bounds__(kScoreThreads, 2)
         idb = rb;
       }
     }
-    if (MODE == kModeList && listing && ns > 0) flush(ns);
+    if (MODE == kModeList && listing) {
+      if (ns >= 16) flush(16);
+      if (ns > 0) flush(ns);
+    }
     pos = seg_end;
   }
 }

@@ -254,20 +254,21 @@ __device__ __forceinline__ uint32_t block_rth_largest(Each each, uint32_t lo, ui
 }
 
 // Top `need` of the c list entries (c >= need, keys within [lo, hi]) in shared memory, handed to
-// emit(slot, i) (list entry i goes to output slot < need; every slot once, in no particular order).  Rounds of 4096 bins narrow a key interval [ilo, ihi]
+// emit(slot, i, entry) (list entry i goes to output slot < need; every slot once, in no particular
+// order).  Rounds of 4096 bins narrow a key interval [ilo, ihi]
 // that holds the need-th entry: the first round bins the keys themselves when they share one sign
 // (order keys are close to logarithmic in the score, so outliers do not crowd the bulk into a few
 // bins) and bins linearly in the score otherwise; later rounds bin the interval's keys.  Once the
 // interval holds at most 256 entries (or one key), one pass writes every entry above it and moves
-// the interval's entries (key, list index) into the histogram's words (hist: 16-byte aligned),
-// where a rank count (score, then token) places them.  An exact tie of more than 2048 entries at one key takes the
-// lowest tokens by a search over the tokens.  The list is only read.  ctr: 2 words; mm: 2 words;
+// the interval's entries and their list indices into the histogram's words (hist: 16-byte
+// aligned), where a rank count (score, then token) places them.  An exact tie of more than 1365
+// entries at one key takes the lowest tokens by a search over the tokens.  The list is only read.  ctr: 2 words; mm: 2 words;
 // scratch: 35 words.
 template <int NT, class Emit>
 __device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi,
                                        uint32_t* hist, uint32_t* ctr, uint32_t* mm, uint32_t* scratch, Emit emit) {
   constexpr uint32_t kRank = 256;            // interval entries a rank count orders
-  constexpr uint32_t kBuf = kHistBins / 2;   // (key, list index) pairs the histogram's words hold
+  constexpr uint32_t kBuf = kHistBins / 3;   // (key, token) pairs and their list indices the histogram holds
   const int tid = threadIdx.x;
   uint32_t ilo = lo, ihi = hi, r = need, eq = (uint32_t)c;
   const bool one_sign = lo >= 0x80000000u || hi < 0x80000000u;
@@ -316,6 +317,7 @@ __device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, 
   const uint32_t n_gt = need - r;  // entries above the interval, all taken
   if (eq <= kBuf) {
     uint2* bl = reinterpret_cast<uint2*>(hist);
+    uint32_t* bi = hist + 2 * kBuf;
     if (tid == 0) {
       ctr[0] = 0;
       ctr[1] = 0;
@@ -327,20 +329,22 @@ __device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, 
       const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
       const bool gt = i < c && e.x > ihi, in = i < c && e.x >= ilo && e.x <= ihi;
       const uint32_t slot = warp_slot(gt, &ctr[0]);
-      if (gt) emit(slot, (uint32_t)i);
+      if (gt) emit(slot, (uint32_t)i, e);
       const uint32_t s2 = warp_slot(in, &ctr[1]);
-      if (in) bl[s2] = make_uint2(e.x, (uint32_t)i);
+      if (in) {
+        bl[s2] = e;
+        bi[s2] = (uint32_t)i;
+      }
     }
     __syncthreads();
     for (uint32_t j = tid; j < eq; j += NT) {
       const uint2 m = bl[j];
-      const uint32_t mt = list[m.y].y;
       uint32_t rk = 0;
       for (uint32_t i = 0; i < eq; ++i) {
         const uint2 o = bl[i];
-        rk += (o.x > m.x) || (o.x == m.x && list[o.y].y < mt);
+        rk += (o.x > m.x) || (o.x == m.x && o.y < m.y);
       }
-      if (rk < r) emit(n_gt + rk, m.y);
+      if (rk < r) emit(n_gt + rk, bi[j], m);
     }
     return;
   }
@@ -379,7 +383,7 @@ __device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, 
     const uint2 e = i < c ? list[i] : make_uint2(0u, 0u);
     const bool sel = i < c && (e.x > ihi || (e.x == ilo && e.y <= tok));
     const uint32_t slot = warp_slot(sel, &ctr[0]);
-    if (sel) emit(slot, (uint32_t)i);
+    if (sel) emit(slot, (uint32_t)i, e);
   }
 }
 
@@ -387,8 +391,7 @@ __device__ void select_list_exact_emit(const uint2* list, int c, uint32_t need, 
 template <int NT>
 __device__ void select_list_exact(const uint2* list, int c, uint32_t need, uint32_t lo, uint32_t hi, uint32_t* hist,
                                   uint32_t* ctr, uint32_t* mm, uint32_t* scratch, int32_t* oi, float* ov) {
-  select_list_exact_emit<NT>(list, c, need, lo, hi, hist, ctr, mm, scratch, [&](uint32_t slot, uint32_t i) {
-    const uint2 e = list[i];
+  select_list_exact_emit<NT>(list, c, need, lo, hi, hist, ctr, mm, scratch, [&](uint32_t slot, uint32_t, uint2 e) {
     oi[slot] = (int32_t)e.y;
     if (ov) ov[slot] = key_to_float(e.x);
   });
@@ -909,18 +912,23 @@ void mark_no_lists(const ListState& l, int T, cudaStream_t s) {
 
 // ---- MISA-dagger selection over dense lists -----------------------------------------------------
 
-// One CTA per row: the top-k' of the row's dense list by the routed score (ties to the lower token)
-// with their dense scores, then the top-k of those by the dense score.  A row its list cannot
-// answer (no list, fewer than k' entries, entries lost past the cap) takes the exact top-k' of its
-// routed score row and scores those candidates with all H_I heads here (as the scorer does, one
-// warp per 16 candidates on the tensor cores).  ctok / cf: [T][kp] scratch for the k' candidates.
+// One CTA per row: the top-k' of the row's dense list by the routed score (ties to the lower token),
+// then the top-k of those by their dense score.  Both selections stay in shared memory: the list's
+// entries and dense scores are copied in, the first selection marks its entries, one compaction
+// pass rewrites the marked ones as (dense score key, token) in place, and the second selection
+// writes the output.  A row its list cannot answer (no list, fewer than k' entries, entries lost
+// past the cap) takes the exact top-k' of its routed score row (into ctok, [T][kp] scratch) and
+// scores those candidates with all H_I heads here (as the scorer does: one warp per 16 candidates
+// on the tensor cores).
 template <int NT, int LIST>
 __global__ void __launch_bounds__(NT, 1)
     hier_select_kernel(const float* __restrict__ scores, int64_t ld, const int32_t* __restrict__ n, int L, int kp,
                        int topk, DenseList dl, const __nv_bfloat16* __restrict__ q, const float* __restrict__ w,
                        const __nv_bfloat16* __restrict__ k, int64_t k_seq_stride, int H_I, int32_t* __restrict__ ctok,
-                       float* __restrict__ cf, int32_t* __restrict__ idx, float* __restrict__ score_opt) {
-  extern __shared__ uint2 list[];  // [LIST]
+                       int32_t* __restrict__ idx, float* __restrict__ score_opt) {
+  extern __shared__ uint2 list[];                                    // [LIST]
+  float* fl = reinterpret_cast<float*>(list + LIST);                 // [LIST] dense scores
+  uint32_t* mark = reinterpret_cast<uint32_t*>(fl + LIST);           // [LIST / 32] selected entries
   __shared__ __align__(16) uint32_t hp[kHistPadded];
   __shared__ uint32_t scratch[35];
   __shared__ uint32_t cnt[2];
@@ -929,9 +937,6 @@ __global__ void __launch_bounds__(NT, 1)
   pdl_wait();
   pdl_trigger();
   const int nt = clamp_len(n[t], L);
-  const float* row = scores + (int64_t)t * ld;
-  int32_t* ct = ctok + (int64_t)t * kp;
-  float* cft = cf + (int64_t)t * kp;
   int32_t* oi = idx + (int64_t)t * topk;
   float* ov = score_opt ? score_opt + (int64_t)t * topk : nullptr;
   const int c1 = min(kp, nt);  // candidates
@@ -942,41 +947,56 @@ __global__ void __launch_bounds__(NT, 1)
     mm[1] = 0u;
   }
 
-  // ---- 1. the k' candidates and their dense scores, into ct / cft ----
+  // ---- 1. the k' candidates as (dense score key, token) in list[0, c1) ----
   if (listed) {
     const uint2* src = dl.list + (int64_t)t * dl.stride;
+    const float* fsrc = dl.f + (int64_t)t * dl.stride;
     uint32_t lo = 0xffffffffu, hi = 0u;
     for (uint32_t i = tid; i < c_in; i += NT) {
       const uint2 e = __ldcg(src + i);
       list[i] = e;
+      fl[i] = __ldcg(fsrc + i);
       lo = min(lo, e.x);
       hi = max(hi, e.x);
     }
+    for (uint32_t i = tid; i < (c_in + 31) / 32; i += NT) mark[i] = 0u;
     block_min_max(lo, hi, mm);
     __syncthreads();
     lo = mm[0];
     hi = mm[1];
     __syncthreads();  // mm is reused as scratch
-    const float* fsrc = dl.f + (int64_t)t * dl.stride;
     select_list_exact_emit<NT>(list, (int)c_in, (uint32_t)kp, lo, hi, hp, cnt, mm, scratch,
-                               [&](uint32_t slot, uint32_t i) {
-                                 ct[slot] = (int32_t)list[i].y;
-                                 cft[slot] = __ldcg(fsrc + i);
-                               });
+                               [&](uint32_t, uint32_t i, uint2) { atomicOr(&mark[i >> 5], 1u << (i & 31)); });
+    __syncthreads();
+    // compaction in place, NT entries a step: every entry moves down (or stays), so a step only
+    // overwrites entries its threads have read (the barrier between reads and writes)
+    uint32_t base = 0;
+    for (uint32_t i0 = 0; i0 < c_in; i0 += NT) {
+      const uint32_t i = i0 + tid;
+      const bool sel = i < c_in && ((mark[i >> 5] >> (i & 31)) & 1u);
+      const uint2 e = sel ? list[i] : make_uint2(0u, 0u);
+      const float v = sel ? fl[i] : 0.f;
+      uint32_t total;
+      const uint32_t pos = base + block_exclusive_scan((uint32_t)sel, scratch, &total);
+      __syncthreads();
+      if (sel) list[pos] = make_uint2(order_key(v), e.y);
+      base += total;
+    }
   } else {
+    int32_t* ct = ctok + (int64_t)t * kp;
     if (nt <= kp) {
       for (int p = tid; p < nt; p += NT) ct[p] = p;
     } else {
+      const float* row = scores + (int64_t)t * ld;
       const bool vec = (reinterpret_cast<uintptr_t>(row) & 15) == 0;
       row_exact_topk<NT, LIST>(row, nt, vec, kp, list, hp, cnt, scratch, ct, nullptr);
     }
-    __syncthreads();  // the candidates are written; the list's memory is free
     const int ngf = (H_I + 7) / 8;
-    uint2(*frag)[8][32] = reinterpret_cast<uint2(*)[8][32]>(list);
-    float* wall = reinterpret_cast<float*>(list + ngf * 8 * 32);
+    uint2(*frag)[8][32] = reinterpret_cast<uint2(*)[8][32]>(fl);  // the dense-score array is free here
+    float* wall = reinterpret_cast<float*>(fl) + ngf * 8 * 32 * 2;
     stage_all_head_frags<NT>(frag, q + (int64_t)t * H_I * kD, H_I, ngf);
     for (int e = tid; e < ngf * 8; e += NT) wall[e] = e < H_I ? w[(int64_t)t * H_I + e] : 0.f;
-    __syncthreads();
+    __syncthreads();  // the candidates are written (global memory, this block) and the heads staged
     const int warp = tid >> 5, lane = tid & 31, g = lane >> 2, c = lane & 3;
     const __nv_bfloat16* kt = k + (int64_t)t * k_seq_stride;
     for (int s0 = warp * 16; s0 < c1; s0 += (NT / 32) * 16) {
@@ -987,11 +1007,11 @@ __global__ void __launch_bounds__(NT, 1)
                 c, A, B);
       float flo, fhi;
       score_rows_rt(A, B, frag, wall, ngf, lane, flo, fhi);
-      if (c == 0 && s0 + g < c1) cft[s0 + g] = flo;
-      if (c == 1 && s0 + g + 8 < c1) cft[s0 + g + 8] = fhi;
+      if (c == 0 && s0 + g < c1) list[s0 + g] = make_uint2(order_key(flo), (uint32_t)ra);
+      if (c == 1 && s0 + g + 8 < c1) list[s0 + g + 8] = make_uint2(order_key(fhi), (uint32_t)rb);
     }
   }
-  __syncthreads();  // ct / cft written by this block
+  __syncthreads();
 
   // ---- 2. the top-k of the candidates by the dense score ----
   if (tid == 0) {
@@ -1000,10 +1020,8 @@ __global__ void __launch_bounds__(NT, 1)
   }
   uint32_t lo = 0xffffffffu, hi = 0u;
   for (int i = tid; i < c1; i += NT) {
-    const uint32_t key = order_key(__ldcg(cft + i));
-    list[i] = make_uint2(key, (uint32_t)__ldcg(ct + i));
-    lo = min(lo, key);
-    hi = max(hi, key);
+    lo = min(lo, list[i].x);
+    hi = max(hi, list[i].x);
   }
   block_min_max(lo, hi, mm);
   __syncthreads();
@@ -1028,14 +1046,14 @@ void launch_list_cut(const float* scores, int64_t ld, const int32_t* n, int T, i
 
 void launch_hier_select(const float* scores, int64_t ld, const int32_t* n, int T, int L, int kp, int topk,
                         const DenseList& dl, const void* q, const float* w, const void* k, int64_t k_seq_stride,
-                        int H_I, int32_t* ctok, float* cf, int32_t* idx, float* score_opt, cudaStream_t s) {
+                        int H_I, int32_t* ctok, int32_t* idx, float* score_opt, cudaStream_t s) {
   if (T <= 0) return;
   constexpr int NT = 1024, LIST = kRowListLarge;
-  const size_t smem = sizeof(uint2) * (size_t)LIST;
+  const size_t smem = (sizeof(uint2) + sizeof(float)) * (size_t)LIST + sizeof(uint32_t) * (LIST / 32);
   cudaFuncSetAttribute(hier_select_kernel<NT, LIST>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   launch_pdl(hier_select_kernel<NT, LIST>, T, NT, smem, s, scores, ld, n, L, kp, topk, dl,
              static_cast<const __nv_bfloat16*>(q), w, static_cast<const __nv_bfloat16*>(k), k_seq_stride, H_I, ctok,
-             cf, idx, score_opt);
+             idx, score_opt);
 }
 
 void launch_topk_rows(const float* scores, int64_t ld, const int32_t* ids, int P, const int32_t* n, int T, int L,

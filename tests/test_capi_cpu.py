@@ -322,15 +322,15 @@ def test_fused_prefill_workspace_and_argument_checks(lib):
 
 def test_hier_fused_workspace_and_argument_checks(lib):
     """misa_hier_topk_fused: workspace = score rows [T, ceil4(L)] + list counts and cuts [2, T] +
-    dense lists [T, 16384] of (key, token) pairs and their dense scores + the k' candidates and their
-    dense scores [2, T, k']; shared caches, fp32 inputs and k' above 16384 are unsupported."""
+    dense lists [T, 16384] of (key, token) pairs and their dense scores + the k' candidates [T, k']
+    of rows the lists cannot answer; shared caches, fp32 inputs and k' above 16384 are unsupported."""
     ws = lib.misa_workspace_bytes
     T, L, kp, k = 32, 131072, 8192, 2048
     cap = 16384
-    want = _al(T * L * 4) + 2 * _al(T * 4) + _al(T * cap * 8) + _al(T * cap * 4) + 2 * _al(T * kp * 4)
+    want = _al(T * L * 4) + 2 * _al(T * 4) + _al(T * cap * 8) + _al(T * cap * 4) + _al(T * kp * 4)
     assert ws(10, T, L, 64, 0, 8, k, kp) == want
     assert ws(10, 3, 1001, 64, 0, 8, 10, 20) == (_al(3 * 1004 * 4) + 2 * _al(12) + _al(3 * cap * 8) +
-                                                 _al(3 * cap * 4) + 2 * _al(3 * 20 * 4))
+                                                 _al(3 * cap * 4) + _al(3 * 20 * 4))
     assert ws(10, 0, L, 64, 0, 8, k, kp) == 0
     f = lib.misa_hier_topk_fused
     S = 1000 * 128
