@@ -863,11 +863,7 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
-    fused = args.dagger == "fused" and kp is not None
-    # kernels per step.  Fused: router, sampled scores, list cut, routed scorer keeping the dense
-    # scores of the tokens at or above the cut, the two selections (one CTA per row).  Unfused: router,
-    # routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank, top-k of the candidates.
-    launches_per_step = 5 if fused else 7
+    mode = args.dagger if kp is not None else "unfused"
 
     def route():
         M.misa_route(qd, wd, kd, kbar, nd, B, h, heads=heads, ws=wsp)
@@ -894,11 +890,12 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         route()
         fused_rest()
 
-    step = step_fused if fused else step_unfused
-    other_step = step_unfused if fused else (step_fused if kp is not None else None)
-
+    comps = {"unfused": step_unfused}
+    if kp is not None:
+        comps["fused"] = step_fused
     for _ in range(max(3, args.warmup)):
-        step()
+        for fn in comps.values():
+            fn()
     torch.cuda.synchronize()
 
     clk = ClockSampler(local)
@@ -907,9 +904,9 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         # no host gaps); the routed scoring call is the roofline's kernel
         nrep = max(3, min(args.steps, 20))
         stages_us = {}
-        stage_fns = [("route", route), ("routed_scores", score)]
-        stage_fns += [("scores_and_selections_fused", fused_rest)] if fused else \
-            [("topk_kprime", select), ("rerank", rerank)]
+        stage_fns = [("route", route), ("routed_scores", score), ("topk_kprime", select), ("rerank", rerank)]
+        if kp is not None:
+            stage_fns.append(("scores_and_selections_fused", fused_rest))
         for nm, fn in stage_fns:
             g = _graphed(torch, fn, not args.no_graph)
             g()
@@ -917,13 +914,21 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             if nm == "routed_scores":
                 score_avg = stages_us[nm] / 1000.0
             del g
-        # the other composition of the same MISA-dagger step, for comparison (not the headline)
-        other_ms = None
-        if other_step is not None:
-            g = _graphed(torch, other_step, not args.no_graph)
+        # both compositions of the MISA-dagger step (the same selection): the four separate calls, or
+        # misa_route + misa_hier_topk_fused; --dagger auto times the step with the faster one here
+        comp_ms = {}
+        for nm, fn in comps.items():
+            g = _graphed(torch, fn, not args.no_graph)
             g()
-            other_ms = _event_ms(torch, stream, g, nrep)
+            comp_ms[nm] = _event_ms(torch, stream, g, nrep)
             del g
+        chosen = min(comp_ms, key=comp_ms.get) if mode == "auto" else mode
+        step = comps[chosen]
+        other_ms = {nm: v for nm, v in comp_ms.items() if nm != chosen}
+        # kernels per step.  Fused: router, sampled scores, list cut, routed scorer keeping the dense
+        # scores of the tokens at or above the cut, the two selections (one CTA per row).  Unfused:
+        # router, routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank, top-k.
+        launches_per_step = 5 if chosen == "fused" else 7
         step()  # the stages above reran on the same inputs; leave one whole step's state behind
         torch.cuda.synchronize()
 
@@ -1013,8 +1018,9 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,
-            "dagger_step": "fused (misa_route + misa_hier_topk_fused)" if fused else
-                           "unfused (misa_route, misa_token_scores, misa_topk_select, misa_hier_rerank)",
+            "dagger_step": ("fused (misa_route + misa_hier_topk_fused)" if chosen == "fused" else
+                            "unfused (misa_route, misa_token_scores, misa_topk_select, misa_hier_rerank)") +
+                           ("; auto: the faster of the two compositions on this run" if mode == "auto" else ""),
             "other_dagger_step_ms": other_ms,
             "clocks": clk.summary("scorer, stage and timed passes"),
             "dense_dsa_same_inputs": None if dsa_ms is None else {
@@ -1102,9 +1108,10 @@ def main():
                     help="decode: skip the prefill and GLM-5-shaped decode legs that follow the main line")
     ap.add_argument("--fused", action="store_true",
                     help="prefill main line: score and select each chunk with misa_score_topk_fused (no score rows)")
-    ap.add_argument("--dagger", choices=["fused", "unfused"], default="fused",
-                    help="MISA-dagger decode step: one call for scores and both selections (fused), or the "
-                         "separate scoring, top-k' and re-rank calls (unfused; the other is timed beside it)")
+    ap.add_argument("--dagger", choices=["auto", "fused", "unfused"], default="auto",
+                    help="MISA-dagger decode step: one call for scores and both selections (fused), the "
+                         "separate scoring, top-k' and re-rank calls (unfused), or the faster of the two as "
+                         "timed in the run (auto); the other is reported beside it")
     ap.add_argument("--no-graph", action="store_true", help="launch every call of a step instead of replaying "
                                                               "the step as a CUDA graph")
     ap.add_argument("--paged", type=int, default=64, metavar="PAGE_SIZE",

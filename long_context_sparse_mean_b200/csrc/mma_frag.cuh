@@ -11,6 +11,8 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace misa {
@@ -105,40 +107,27 @@ __device__ __forceinline__ void score_rows(const uint4 (&A)[4], const uint4 (&Bq
 
 // score_rows for a run-time number of head groups ng_count, weights from shared memory (wsel[8 ng +
 // e] for slot e of group ng): the same operations in the same order, so the result is score_rows<NG>
-// bit for bit.  Four head groups are multiplied at a time (four independent accumulator chains), then
-// added in ascending group order.
+// bit for bit.
 __device__ __forceinline__ void score_rows_rt(const uint4 (&A)[4], const uint4 (&Bq)[4], const uint2 (*frag)[8][32],
                                               const float* wsel, int ng_count, int lane, float& s_lo, float& s_hi) {
   const int c = lane & 3;
   float slo = 0.f, shi = 0.f;
-  for (int ng0 = 0; ng0 < ng_count; ng0 += 4) {
-    float acc[4][4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) acc[u][0] = acc[u][1] = acc[u][2] = acc[u][3] = 0.f;
+  for (int ng = 0; ng < ng_count; ++ng) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
       const uint4 xa = A[kk >> 1], xb = Bq[kk >> 1];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        if (ng0 + u < ng_count) {
-          const uint2 bf = frag[ng0 + u][kk][lane];
-          if (kk & 1)
-            mma_bf16_16816(acc[u], xa.z, xb.z, xa.w, xb.w, bf.x, bf.y);
-          else
-            mma_bf16_16816(acc[u], xa.x, xb.x, xa.y, xb.y, bf.x, bf.y);
-        }
-      }
+      const uint2 bf = frag[ng][kk][lane];
+      if (kk & 1)
+        mma_bf16_16816(acc, xa.z, xb.z, xa.w, xb.w, bf.x, bf.y);
+      else
+        mma_bf16_16816(acc, xa.x, xb.x, xa.y, xb.y, bf.x, bf.y);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (ng0 + u < ng_count) {
-        const float wa = wsel[(ng0 + u) * 8 + 2 * c], wb = wsel[(ng0 + u) * 8 + 2 * c + 1];
-        slo = fmaf(wa, relu(acc[u][0]), slo);
-        slo = fmaf(wb, relu(acc[u][1]), slo);
-        shi = fmaf(wa, relu(acc[u][2]), shi);
-        shi = fmaf(wb, relu(acc[u][3]), shi);
-      }
-    }
+    const float wa = wsel[ng * 8 + 2 * c], wb = wsel[ng * 8 + 2 * c + 1];
+    slo = fmaf(wa, relu(acc[0]), slo);
+    slo = fmaf(wb, relu(acc[1]), slo);
+    shi = fmaf(wa, relu(acc[2]), shi);
+    shi = fmaf(wb, relu(acc[3]), shi);
   }
   slo += __shfl_xor_sync(0xffffffffu, slo, 1);
   shi += __shfl_xor_sync(0xffffffffu, shi, 1);
@@ -146,6 +135,31 @@ __device__ __forceinline__ void score_rows_rt(const uint4 (&A)[4], const uint4 (
   shi += __shfl_xor_sync(0xffffffffu, shi, 2);
   s_lo = __fadd_rn(slo, 0.0f);
   s_hi = __fadd_rn(shi, 0.0f);
+}
+
+// score_rows_rt with the group count known at compile time for the common head pools (H_I = 32, 64,
+// 128): the groups' accumulator chains are unrolled and independent, so their MMAs overlap.
+__device__ __forceinline__ void score_rows_any(const uint4 (&A)[4], const uint4 (&Bq)[4], const uint2 (*frag)[8][32],
+                                               const float* wsel, int ng_count, int lane, float& s_lo, float& s_hi) {
+  const int c = lane & 3;
+  auto fixed = [&](auto ngc) {
+    constexpr int NGC = decltype(ngc)::value;
+    float wa[NGC], wb[NGC];
+#pragma unroll
+    for (int ng = 0; ng < NGC; ++ng) {
+      wa[ng] = wsel[ng * 8 + 2 * c];
+      wb[ng] = wsel[ng * 8 + 2 * c + 1];
+    }
+    score_rows<NGC>(A, Bq, frag, wa, wb, lane, s_lo, s_hi);
+  };
+  if (ng_count == 8)
+    fixed(std::integral_constant<int, 8>{});
+  else if (ng_count == 4)
+    fixed(std::integral_constant<int, 4>{});
+  else if (ng_count == 16)
+    fixed(std::integral_constant<int, 16>{});
+  else
+    score_rows_rt(A, Bq, frag, wsel, ng_count, lane, s_lo, s_hi);
 }
 
 }  // namespace misa

@@ -123,7 +123,7 @@ __device__ __noinline__ void flush_ring(const uint8_t* ring, const uint2* meta, 
     B[i] = g + 8 < m ? *reinterpret_cast<const uint4*>(ring + sb * kD * 2 + (4 * i + c) * 16) : make_uint4(0, 0, 0, 0);
   }
   float flo, fhi;
-  score_rows_rt(A, B, frag, wall, ngf, lane, flo, fhi);
+  score_rows_any(A, B, frag, wall, ngf, lane, flo, fhi);
   uint32_t base = 0;
   if (lane == 0) base = atomicAdd(dl.cnt + t, (uint32_t)m);
   base = __shfl_sync(0xffffffffu, base, 0);
