@@ -55,8 +55,8 @@ UNIT = "query-tokens/s"
 # dram__bytes_write.sum), per scored key, with the hash of the source it was taken on; the
 # bench reports null once the kernel source has changed since.
 TRAFFIC = {"file": "long_context_sparse_mean_b200/csrc/score.cu",
-           "sha256": "563bd1e63154ff27fd27781231e980992b784b507515b6f567ad79c3cbb1fc8d",
-           "bytes_per_key": (1.073898e9 + 19.067648e6) / 4194304}
+           "sha256": "2a95e40e8e18e3539ab5c2cf9f6f0e1967940c2ba9bb48f2df57609ca3e91cbc",
+           "bytes_per_key": (1.073908352e9 + 16.844928e6) / 4194304}
 # The same for the tensor-core prefill scorer, per scored (query, key) pair, from a capture of one
 # chunk's launch; the step's traffic is that rate times the pairs the step scores.
 TRAFFIC_PREFILL = {"file": "long_context_sparse_mean_b200/csrc/score_tc.cu",
@@ -952,6 +952,10 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         ms = max_over_ranks(ms, dist, dev)
     units_per_step = T * L * ws
     value = units_per_step * args.steps / (ms / 1000.0)
+    # the paged leg's reference: the same separate calls on the contiguous caches (the fused call's
+    # dense scores round differently, so near-ties at the k-th may be ordered otherwise)
+    step_unfused()
+    torch.cuda.synchronize()
     ref_idx = idx.clone()
 
     # end to end through the public API with host buffers: per step the new queries q, their head
@@ -1008,7 +1012,9 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": _config(wl, {"parallelism": f"{ws} GPU(s), independent sequences per GPU",
                                    "cuda_graph": not args.no_graph}),
-            "roofline": {"bound": "hbm", "kernel": "routed token scoring (score_persist_kernel)",
+            "roofline": {"bound": "hbm",
+                         "kernel": "routed token scoring (score_persist_kernel<1, 0>, the misa_token_scores call; "
+                                   "the fused step runs its list-keeping variant <1, 3> over the same key bytes)",
                          "achieved": achieved, "peak": hbm, "peak_kind": kind, "unit": "GB/s",
                          "frac": achieved / hbm,
                          "traffic": _traffic(TRAFFIC, "bytes_per_key", T * L),
