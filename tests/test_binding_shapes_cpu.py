@@ -48,6 +48,8 @@ def test_well_shaped_calls_reach_the_device_check(per_query):
     _device_check_only(lambda: M.misa_block_filter_topk(q, w, k, kbar, n, heads, B, 4, 10,
                                                         blocks=_t(T, 4, dtype=torch.int32),
                                                         block_scores=_t(T, MB)))
+    if per_query:
+        _device_check_only(lambda: M.misa_hier_topk_fused(q, w, k, n, heads, 50, 10, vals=_t(T, 10)))
 
 
 def test_wrong_shapes_are_rejected_first():
@@ -78,6 +80,10 @@ def test_wrong_shapes_are_rejected_first():
     _shape_error(lambda: M.misa_block_filter_topk(q, w, k, kbar, n, heads, B, 4, 10,
                                                   block_scores=_t(T, MB - 1)), "block_scores must be")
     _shape_error(lambda: M.misa_block_filter_topk(q, w, k, kbar, n, heads, 4, 4, 10), "kbar must be")  # B mismatch
+    kq = _t(T, L, D, dtype=torch.bfloat16)
+    _shape_error(lambda: M.misa_hier_topk_fused(q, w, k, n, heads, 50, 10), "per-query caches")  # a shared cache
+    _shape_error(lambda: M.misa_hier_topk_fused(q, w, kq, n, heads[:2], 50, 10), "heads must be")
+    _shape_error(lambda: M.misa_hier_topk_fused(q, w, kq, n, heads, 50, 10, idx=_t(T, 9, dtype=i32)), "idx must be")
 
 
 def test_device_check_rejects_a_tensor_on_another_gpu(monkeypatch):
