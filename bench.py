@@ -369,7 +369,7 @@ def paged_leg(args, torch, M, qd, wd, kd, nd, wl, stream, dev, ref_idx=None):
     table = perm.reshape(T, lp).to(torch.int32).contiguous()
     kbar = M.misa_pool_keys_paged(pool, table, B, L=L)
     heads = torch.empty((T, h), dtype=torch.int32, device=dev)
-    cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
+    cand = torch.empty((T, kp), dtype=torch.int32, device=dev) if kp is not None else None
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     wsp = M.Workspace(dev)
@@ -860,7 +860,7 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
     kbar = M.misa_pool_keys(kd, B)
     heads = torch.empty((T, h), dtype=torch.int32, device=dev)
     scores = torch.empty((T, L), dtype=torch.float32, device=dev)
-    cand = torch.empty((T, kp), dtype=torch.int32, device=dev)
+    cand = torch.empty((T, kp), dtype=torch.int32, device=dev) if kp is not None else None
     idx = torch.empty((T, kk), dtype=torch.int32, device=dev)
     vals = torch.empty((T, kk), dtype=torch.float32, device=dev)
     mode = args.dagger if kp is not None else "unfused"
@@ -872,10 +872,14 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         M.misa_token_scores(qd, wd, kd, nd, heads, out=scores)
 
     def select():
-        M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws)
+        if kp is not None:  # the k' candidates
+            M.misa_topk_select(scores, nd, kp, idx=cand, want_vals=False, ws=sel_ws)
+        else:  # MISA: the top-k itself
+            M.misa_topk_select(scores, nd, kk, idx=idx, vals=vals, ws=sel_ws)
 
     def rerank():
-        M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
+        if kp is not None:
+            M.misa_hier_rerank(qd, wd, kd, nd, cand, kk, idx=idx, vals=vals, ws=wsp)
 
     def fused_rest():
         M.misa_hier_topk_fused(qd, wd, kd, nd, heads, kp, kk, idx=idx, vals=vals, ws=sel_ws)
@@ -904,9 +908,11 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         # no host gaps); the routed scoring call is the roofline's kernel
         nrep = max(3, min(args.steps, 20))
         stages_us = {}
-        stage_fns = [("route", route), ("routed_scores", score), ("topk_kprime", select), ("rerank", rerank)]
+        stage_fns = [("route", route), ("routed_scores", score)]
         if kp is not None:
-            stage_fns.append(("scores_and_selections_fused", fused_rest))
+            stage_fns += [("topk_kprime", select), ("rerank", rerank), ("scores_and_selections_fused", fused_rest)]
+        else:
+            stage_fns += [("topk", select)]
         for nm, fn in stage_fns:
             g = _graphed(torch, fn, not args.no_graph)
             g()
@@ -928,7 +934,7 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
         # kernels per step.  Fused: router, sampled scores, list cut, routed scorer keeping the dense
         # scores of the tokens at or above the cut, the two selections (one CTA per row).  Unfused:
         # router, routed scorer, list cut, list sweep, top-k' (one CTA per row), re-rank, top-k.
-        launches_per_step = 5 if chosen == "fused" else 7
+        launches_per_step = 5 if chosen == "fused" else (7 if kp is not None else 5)
         step()  # the stages above reran on the same inputs; leave one whole step's state behind
         torch.cuda.synchronize()
 
@@ -1024,7 +1030,8 @@ def _run_ours(args, ws, rank, local, wl, gen_pool):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": launches_per_step * args.steps,
             "stages_us": stages_us,
-            "dagger_step": ("fused (misa_route + misa_hier_topk_fused)" if chosen == "fused" else
+            "dagger_step": None if kp is None else
+                           ("fused (misa_route + misa_hier_topk_fused)" if chosen == "fused" else
                             "unfused (misa_route, misa_token_scores, misa_topk_select, misa_hier_rerank)") +
                            ("; auto: the faster of the two compositions on this run" if mode == "auto" else ""),
             "other_dagger_step_ms": other_ms,
